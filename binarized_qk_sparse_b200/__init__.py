@@ -1,0 +1,280 @@
+"""Python binding of the binarized-QK top-N attention library (include/had.h).
+
+Thin ctypes marshalling over ``libhad_b200.so``: every step of the method runs
+in the library's sm_100a kernels.  PyTorch supplies device memory and the
+current CUDA stream.  There is no fallback: if the shared library or a CUDA
+device is missing, calls raise.
+
+Method ("Hamming Attention Distillation" top-N over binarized keys and
+queries; "BinaryAttention" §2.2-§2.4 scaled binarization, bias, uint8 A x
+int8 V): see include/had.h for the exact formulas and layouts.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libhad_b200.so")
+
+HAD_OK, HAD_ERR_INVALID, HAD_ERR_UNSUPPORTED, HAD_ERR_CUDA, HAD_ERR_DEVICE, HAD_ERR_TIMEOUT = range(6)
+HAD_F32, HAD_BF16 = 0, 1
+HAD_MODE_FLOAT, HAD_MODE_U8I8 = 0, 1
+_MODES = {"float": HAD_MODE_FLOAT, "u8i8": HAD_MODE_U8I8, HAD_MODE_FLOAT: HAD_MODE_FLOAT,
+          HAD_MODE_U8I8: HAD_MODE_U8I8}
+
+
+class HadError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        msg = lib().had_status_string(status).decode()
+        if status == HAD_ERR_CUDA:
+            msg += f" ({lib().had_last_cuda_error().decode()})"
+        super().__init__(f"{what}: {msg}")
+
+
+class had_shape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("H", ctypes.c_int), ("n", ctypes.c_int), ("d", ctypes.c_int),
+                ("in_dtype", ctypes.c_int), ("seqlens", ctypes.c_void_p)]
+
+
+class had_relpos_bias(ctypes.Structure):
+    _fields_ = [("table", ctypes.c_void_p), ("gh", ctypes.c_int), ("gw", ctypes.c_int), ("prefix", ctypes.c_int)]
+
+
+@dataclass
+class RelPosBias:
+    """Per-head relative-position table [H, 2gh-1, 2gw-1] (fp32, on the device)."""
+    table: torch.Tensor
+    gh: int
+    gw: int
+    prefix: int = 0
+
+
+_lib = None
+
+
+def lib():
+    """Load the in-tree CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"CUDA library not built: {LIB_PATH} is missing (run binarized_qk_sparse_b200._build)")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        SP, BP = ctypes.POINTER(had_shape), ctypes.POINTER(had_relpos_bias)
+        L.had_binarize_pack_workspace_size.argtypes = [SP]
+        L.had_binarize_pack_workspace_size.restype = SZ
+        L.had_binarize_pack.argtypes = [P, SP, P, P, P, P, SZ, P]
+        L.had_attention_workspace_size.argtypes = [SP, I, I, BP]
+        L.had_attention_workspace_size.restype = SZ
+        L.had_attention.argtypes = [P, P, P, SP, BP, P, P, I, I, P, I, P, SZ, P]
+        L.had_dense_reference_workspace_size.argtypes = [SP]
+        L.had_dense_reference_workspace_size.restype = SZ
+        L.had_dense_reference_mode.argtypes = [P, P, P, SP, BP, I, P, I, P, SZ, P]
+        L.had_scores_int.argtypes = [P, P, SP, P, P]
+        L.had_topn_indices.argtypes = [P, P, SP, BP, P, P, I, P, P, SZ, P]
+        L.had_attention_codes_u8.argtypes = [P, P, P, SP, BP, P, P, I, I, I, P, P, SZ, P]
+        L.had_quantize_v.argtypes = [P, SP, P, P, P, SZ, P]
+        for f in ("had_binarize_pack", "had_attention", "had_dense_reference_mode", "had_scores_int",
+                  "had_topn_indices", "had_attention_codes_u8", "had_quantize_v", "had_get_device_status"):
+            getattr(L, f).restype = I
+        L.had_get_device_status.argtypes = []
+        L.had_status_string.argtypes = [I]
+        L.had_status_string.restype = ctypes.c_char_p
+        L.had_last_cuda_error.argtypes = []
+        L.had_last_cuda_error.restype = ctypes.c_char_p
+        L.had_version.restype = I
+        _lib = L
+    return _lib
+
+
+# ----------------------------------------------------------------------------- marshalling helpers
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return HAD_BF16
+    if t.dtype == torch.float32:
+        return HAD_F32
+    raise TypeError(f"unsupported dtype {t.dtype}; Q/K/V must be bfloat16 or float32")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_dev(*ts):
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("tensors must live on a CUDA device")
+            if not t.is_contiguous():
+                raise ValueError("tensors must be contiguous")
+
+
+def make_shape(X: torch.Tensor, seqlens: torch.Tensor | None = None) -> had_shape:
+    B, H, n, d = X.shape
+    if seqlens is not None and seqlens.dtype != torch.int32:
+        raise TypeError("seqlens must be int32")
+    return had_shape(B, H, n, d, _dtype_code(X), None if seqlens is None else seqlens.data_ptr())
+
+
+def _bias_struct(bias: RelPosBias | None):
+    if bias is None:
+        return None
+    if bias.table.dtype != torch.float32:
+        raise TypeError("bias table must be float32")
+    _check_dev(bias.table)
+    return ctypes.byref(had_relpos_bias(bias.table.data_ptr(), bias.gh, bias.gw, bias.prefix))
+
+
+def _alpha(a, H):
+    if a is None:
+        return None, None
+    arr = (ctypes.c_float * H)(*[float(x) for x in a])
+    return arr, ctypes.cast(arr, ctypes.c_void_p)
+
+
+def _raise(st, what):
+    if st != HAD_OK:
+        raise HadError(st, what)
+
+
+def _workspace(nbytes: int, device, workspace):
+    if workspace is not None:
+        if workspace.numel() * workspace.element_size() < nbytes:
+            raise ValueError("workspace too small")
+        return workspace
+    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+
+
+# ----------------------------------------------------------------------------- entry points
+
+def had_binarize_pack(X, seqlens=None, mu_in=None, want_mu=True, workspace=None, stream=None):
+    """Sign bits of X - mu packed to uint32 [B,H,n,d/32] (bit 1 = negative), and mu [B,H,d] fp32."""
+    _check_dev(X, seqlens, mu_in)
+    B, H, n, d = X.shape
+    shp = make_shape(X, seqlens)
+    bits = torch.empty((B, H, n, d // 32), dtype=torch.int32, device=X.device)
+    mu = torch.empty((B, H, d), dtype=torch.float32, device=X.device) if want_mu else None
+    ws = None
+    if mu_in is None:
+        ws = _workspace(lib().had_binarize_pack_workspace_size(ctypes.byref(shp)), X.device, workspace)
+    st = lib().had_binarize_pack(_ptr(X), ctypes.byref(shp), _ptr(mu_in), _ptr(mu), _ptr(bits), _ptr(ws),
+                                 0 if ws is None else ws.numel(), _stream(stream))
+    _raise(st, "had_binarize_pack")
+    return bits, (mu if mu_in is None else mu_in)
+
+
+def had_attention_workspace_size(X, N=0, mode="float", seqlens=None, bias=None) -> int:
+    shp = make_shape(X, seqlens)
+    return int(lib().had_attention_workspace_size(ctypes.byref(shp), int(N), _MODES[mode], _bias_struct(bias)))
+
+
+def had_attention(Q, K, V, N=0, mode="float", seqlens=None, bias=None, alpha_q=None, alpha_k=None, out=None,
+                  out_dtype=None, workspace=None, stream=None):
+    """Binarized-QK top-N attention; returns O [B,H,n,d] (dtype of V unless out/out_dtype say otherwise)."""
+    _check_dev(Q, K, V, seqlens, out, workspace)
+    B, H, n, d = Q.shape
+    shp = make_shape(Q, seqlens)
+    m = _MODES[mode]
+    if out is None:
+        out = torch.empty((B, H, n, d), dtype=out_dtype or V.dtype, device=Q.device)
+    bs = _bias_struct(bias)
+    ws = _workspace(lib().had_attention_workspace_size(ctypes.byref(shp), int(N), m, bs), Q.device, workspace)
+    aq_keep, aq = _alpha(alpha_q, H)
+    ak_keep, ak = _alpha(alpha_k, H)
+    st = lib().had_attention(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shp), bs, aq, ak, int(N), m, _ptr(out),
+                             _dtype_code(out), _ptr(ws), ws.numel(), _stream(stream))
+    _raise(st, "had_attention")
+    return out
+
+
+def had_dense_reference_mode(Q, K, V, N=0, seqlens=None, bias=None, out=None, out_dtype=None, stream=None):
+    """Standard dense attention on the unbinarized bf16 inputs (the library's comparison mode)."""
+    _check_dev(Q, K, V, seqlens, out)
+    B, H, n, d = Q.shape
+    shp = make_shape(Q, seqlens)
+    if out is None:
+        out = torch.empty((B, H, n, d), dtype=out_dtype or V.dtype, device=Q.device)
+    st = lib().had_dense_reference_mode(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shp), _bias_struct(bias), int(N),
+                                        _ptr(out), _dtype_code(out), None, 0, _stream(stream))
+    _raise(st, "had_dense_reference_mode")
+    return out
+
+
+def had_scores_int(qbits, kbits, seqlens=None, d=64, stream=None):
+    """Integer scores d - 2*popcount(q XOR k) [B,H,n,n] int32 through the library's tensor-core fragments."""
+    _check_dev(qbits, kbits, seqlens)
+    B, H, n, _ = qbits.shape
+    shp = had_shape(B, H, n, d, HAD_BF16, None if seqlens is None else seqlens.data_ptr())
+    S = torch.empty((B, H, n, n), dtype=torch.int32, device=qbits.device)
+    st = lib().had_scores_int(_ptr(qbits), _ptr(kbits), ctypes.byref(shp), _ptr(S), _stream(stream))
+    _raise(st, "had_scores_int")
+    return S
+
+
+def had_topn_indices(Q, K, N, seqlens=None, bias=None, alpha_q=None, alpha_k=None, workspace=None, stream=None):
+    """Kept key indices per query, ascending, -1 padded: [B,H,n,N] int32."""
+    _check_dev(Q, K, seqlens)
+    B, H, n, d = Q.shape
+    shp = make_shape(Q, seqlens)
+    bs = _bias_struct(bias)
+    ws = _workspace(lib().had_attention_workspace_size(ctypes.byref(shp), int(N), HAD_MODE_FLOAT, bs), Q.device,
+                    workspace)
+    idx = torch.empty((B, H, n, N), dtype=torch.int32, device=Q.device)
+    aq_keep, aq = _alpha(alpha_q, H)
+    ak_keep, ak = _alpha(alpha_k, H)
+    st = lib().had_topn_indices(_ptr(Q), _ptr(K), ctypes.byref(shp), bs, aq, ak, int(N), _ptr(idx), _ptr(ws),
+                                ws.numel(), _stream(stream))
+    _raise(st, "had_topn_indices")
+    return idx
+
+
+def had_attention_codes_u8(Q, K, V, row_begin, row_end, N=0, seqlens=None, bias=None, alpha_q=None, alpha_k=None,
+                           workspace=None, stream=None):
+    """uint8 attention codes floor(255 p + 0.5) of rows [row_begin, row_end): [B,H,rows,n] uint8."""
+    _check_dev(Q, K, V, seqlens)
+    B, H, n, d = Q.shape
+    shp = make_shape(Q, seqlens)
+    bs = _bias_struct(bias)
+    ws = _workspace(lib().had_attention_workspace_size(ctypes.byref(shp), int(N), HAD_MODE_U8I8, bs), Q.device,
+                    workspace)
+    A = torch.empty((B, H, row_end - row_begin, n), dtype=torch.uint8, device=Q.device)
+    aq_keep, aq = _alpha(alpha_q, H)
+    ak_keep, ak = _alpha(alpha_k, H)
+    st = lib().had_attention_codes_u8(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shp), bs, aq, ak, int(N),
+                                      int(row_begin), int(row_end), _ptr(A), _ptr(ws), ws.numel(), _stream(stream))
+    _raise(st, "had_attention_codes_u8")
+    return A
+
+
+def had_quantize_v(V, seqlens=None, workspace=None, stream=None):
+    """Per-channel int8 V [B,H,n,d] and its fp32 scales [B,H,d]."""
+    _check_dev(V, seqlens)
+    B, H, n, d = V.shape
+    shp = make_shape(V, seqlens)
+    ws = _workspace(lib().had_attention_workspace_size(ctypes.byref(shp), 0, HAD_MODE_U8I8, None), V.device, workspace)
+    Vq = torch.empty((B, H, n, d), dtype=torch.int8, device=V.device)
+    sc = torch.empty((B, H, d), dtype=torch.float32, device=V.device)
+    st = lib().had_quantize_v(_ptr(V), ctypes.byref(shp), _ptr(Vq), _ptr(sc), _ptr(ws), ws.numel(), _stream(stream))
+    _raise(st, "had_quantize_v")
+    return Vq, sc
+
+
+def had_get_device_status() -> int:
+    """Synchronize, read and clear the device status word (HAD_OK, HAD_ERR_DEVICE or HAD_ERR_TIMEOUT)."""
+    return int(lib().had_get_device_status())
+
+
+def had_version() -> int:
+    return int(lib().had_version())

@@ -1,0 +1,556 @@
+// had_lib.cu -- C ABI of the binarized-QK top-N attention library (include/had.h).
+//
+// Host side of every entry point: validate on the host (nothing is enqueued
+// on an error), carve the caller's workspace, and enqueue the kernels on the
+// caller's stream.  No allocation, no synchronization on the hot path.
+//
+// had_attention pipeline (method: "Hamming Attention Distillation" top-N over
+// binarized keys/queries; "BinaryAttention" §2.2-§2.4):
+//   k_stats  : fp64 channel partial sums of Q and K (+ fp32 absmax of V in uint8 mode)
+//   k_pack   : mu -> sign bits of Q (packed uint32) and K (+-1 int8 rows);
+//              V scale -> int8 V^T (uint8 mode)
+//   k_bias_minmax (top-N with a bias): per-head bias range for the select band
+//   k_attn   : scores, logits, top-N select, softmax, A.V, output
+#include <climits>
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/had.h"
+#include "common.cuh"
+#include "prep.cuh"
+#include "attn.cuh"
+#include "dense_ref.cuh"
+
+namespace had {
+
+__device__ unsigned g_device_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+thread_local char t_last_error[256] = "";
+
+unsigned* status_ptr(int dev) {
+  static std::mutex mu;
+  static unsigned* ptrs[kMaxDevices] = {nullptr};
+  if (dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_device_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<unsigned*>(p);
+  }
+  return ptrs[dev];
+}
+
+had_status cuda_fail(cudaError_t e, const char* what) {
+  snprintf(t_last_error, sizeof(t_last_error), "%s: %s", what, cudaGetErrorString(e));
+  return HAD_ERR_CUDA;
+}
+
+had_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? HAD_OK : cuda_fail(e, what);
+}
+
+inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Dims {
+  int B, H, n, BH, nchunks, n_pad;
+};
+
+Dims dims_of(const had_shape* s) {
+  Dims d;
+  d.B = s->B; d.H = s->H; d.n = s->n; d.BH = s->B * s->H;
+  d.nchunks = (s->n + kChunk - 1) / kChunk;
+  d.n_pad = d.nchunks * kChunk;
+  return d;
+}
+
+had_status check_shape(const had_shape* s) {
+  if (!s) return HAD_ERR_INVALID;
+  if (s->B <= 0 || s->H <= 0 || s->n <= 0 || s->d <= 0) return HAD_ERR_INVALID;
+  if (s->in_dtype != HAD_F32 && s->in_dtype != HAD_BF16) return HAD_ERR_INVALID;
+  if (s->d != kD || s->n > kMaxN || s->H > kMaxHeads || (long long)s->B * s->H > 65535) return HAD_ERR_UNSUPPORTED;
+  if (s->seqlens && (reinterpret_cast<uintptr_t>(s->seqlens) & 3u)) return HAD_ERR_INVALID;
+  return HAD_OK;
+}
+
+had_status check_bias(const had_shape* s, const had_relpos_bias* bias) {
+  if (!bias || !bias->table) return HAD_OK;
+  if (bias->gh <= 0 || bias->gw <= 0 || bias->prefix < 0) return HAD_ERR_INVALID;
+  if ((long long)bias->gh * bias->gw + bias->prefix != s->n) return HAD_ERR_INVALID;
+  if (reinterpret_cast<uintptr_t>(bias->table) & 3u) return HAD_ERR_INVALID;
+  return HAD_OK;
+}
+
+struct Ws {
+  size_t qbits, kpm, sums, amax, vqT, vscale, bminmax, total;
+};
+
+Ws ws_layout(const had_shape* s, bool quant, bool bias) {
+  Dims d = dims_of(s);
+  Ws w{};
+  size_t off = 0;
+  w.qbits = off; off += align_up((size_t)d.BH * d.n * kW * 4);
+  w.kpm = off; off += align_up((size_t)d.BH * d.n_pad * kD);
+  w.sums = off; off += align_up((size_t)2 * d.BH * d.nchunks * kD * 8);
+  w.amax = w.vqT = w.vscale = w.bminmax = 0;
+  if (quant) {
+    w.amax = off; off += align_up((size_t)d.BH * d.nchunks * kD * 4);
+    w.vqT = off; off += align_up((size_t)d.BH * kD * d.n_pad);
+    w.vscale = off; off += align_up((size_t)d.BH * kD * 4);
+  }
+  if (bias) { w.bminmax = off; off += align_up((size_t)s->H * 2 * 4); }
+  w.total = off;
+  return w;
+}
+
+__global__ void k_bias_minmax(const float* table, int th, int tw, int prefix, float* out) {
+  const int h = blockIdx.x;
+  const float* t = table + (size_t)h * th * tw;
+  float mn = INFINITY, mx = -INFINITY;
+  for (int e = threadIdx.x; e < th * tw; e += blockDim.x) { mn = fminf(mn, t[e]); mx = fmaxf(mx, t[e]); }
+  __shared__ float smn[32], smx[32];
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if ((threadIdx.x & 31) == 0) { smn[threadIdx.x >> 5] = mn; smx[threadIdx.x >> 5] = mx; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) { mn = fminf(mn, smn[w]); mx = fmaxf(mx, smx[w]); }
+    if (prefix > 0) { mn = fminf(mn, 0.0f); mx = fmaxf(mx, 0.0f); }  // class-token pairs have bias 0
+    out[2 * h] = mn;
+    out[2 * h + 1] = mx;
+  }
+}
+
+__global__ void k_untranspose_vq(const int8_t* vqT, int BH, int n, int n_pad, const int32_t* seqlens, int H,
+                                 int8_t* Vq) {
+  const size_t total = (size_t)BH * n * kD;
+  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
+    const int c = (int)(e % kD);
+    const size_t ti = e / kD;
+    const int i = (int)(ti % n);
+    const int bh = (int)(ti / n);
+    Vq[e] = vqT[((size_t)bh * kD + c) * n_pad + i];
+  }
+}
+
+// ---------------------------------------------------------------------------- prep launches
+
+had_status launch_prep(const had_shape* s, const void* X0, const void* X1, const void* X2, int first, int ntens,
+                       double* sums, float* amax, const float* mu_in0, float* mu_out0, uint32_t* bits0,
+                       int8_t* pm0, uint32_t* bits1, int8_t* pm1, int8_t* vqT, float* vscale, cudaStream_t st,
+                       unsigned* status) {
+  Dims d = dims_of(s);
+  PrepArgs pa{};
+  pa.X[0] = X0; pa.X[1] = X1; pa.X[2] = X2;
+  pa.ntens = ntens; pa.first_tensor = first;
+  pa.B = d.B; pa.H = d.H; pa.n = d.n; pa.nchunks = d.nchunks;
+  pa.seqlens = s->seqlens; pa.sums = sums; pa.amax = amax; pa.status = status;
+  dim3 grid(d.nchunks, d.BH, ntens);
+  const bool need_stats = !(mu_in0 && first == 0 && ntens == 1);
+  if (need_stats) {
+    if (s->in_dtype == HAD_BF16) k_stats<__nv_bfloat16><<<grid, kPrepThreads, 0, st>>>(pa);
+    else k_stats<float><<<grid, kPrepThreads, 0, st>>>(pa);
+    had_status r = check_launch("k_stats");
+    if (r != HAD_OK) return r;
+  }
+  PackArgs ka{};
+  ka.X[0] = X0; ka.X[1] = X1; ka.X[2] = X2;
+  ka.ntens = ntens; ka.first_tensor = first;
+  ka.B = d.B; ka.H = d.H; ka.n = d.n; ka.nchunks = d.nchunks; ka.n_pad = d.n_pad;
+  ka.seqlens = s->seqlens; ka.sums = sums; ka.amax = amax;
+  ka.mu_in[0] = mu_in0; ka.mu_in[1] = nullptr;
+  ka.mu_out[0] = mu_out0; ka.mu_out[1] = nullptr;
+  ka.bits[0] = bits0; ka.bits[1] = bits1;
+  ka.pm[0] = pm0; ka.pm[1] = pm1;
+  ka.vqT = vqT; ka.vscale = vscale; ka.status = status;
+  if (s->in_dtype == HAD_BF16) k_pack<__nv_bfloat16><<<grid, kPrepThreads, 0, st>>>(ka);
+  else k_pack<float><<<grid, kPrepThreads, 0, st>>>(ka);
+  return check_launch("k_pack");
+}
+
+// ---------------------------------------------------------------------------- attention launches
+
+template <int SEL, int MODE, bool BIAS, bool VF32, int EXP>
+had_status launch_attn_t(const AttnArgs& a, dim3 grid, cudaStream_t st) {
+  using SL = SmemLayout<MODE, VF32>;
+  const int smem = (SEL == SEL_DENSE) ? SL::kTotalDense : SL::kTotalTopN;
+  auto fn = k_attn<SEL, MODE, BIAS, VF32, EXP>;
+  static std::mutex mu;
+  static bool configured[kMaxDevices] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 0 && dev < kMaxDevices && !configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_attn)");
+      configured[dev] = true;
+    }
+  }
+  fn<<<grid, kAttnThreads, smem, st>>>(a);
+  return check_launch("k_attn");
+}
+
+template <int EXP>
+had_status dispatch_attn(int sel, int mode, bool bias, bool vf32, const AttnArgs& a, dim3 grid, cudaStream_t st) {
+  if (EXP == EXP_NONE) {
+    if (mode == MODE_Q) {
+      if (sel == SEL_DENSE) return bias ? launch_attn_t<SEL_DENSE, MODE_Q, true, false, EXP>(a, grid, st)
+                                        : launch_attn_t<SEL_DENSE, MODE_Q, false, false, EXP>(a, grid, st);
+      if (sel == SEL_TOPN_INT) return launch_attn_t<SEL_TOPN_INT, MODE_Q, false, false, EXP>(a, grid, st);
+      return launch_attn_t<SEL_TOPN_FLOAT, MODE_Q, true, false, EXP>(a, grid, st);
+    }
+    if (vf32) {
+      if (sel == SEL_DENSE) return bias ? launch_attn_t<SEL_DENSE, MODE_F, true, true, EXP>(a, grid, st)
+                                        : launch_attn_t<SEL_DENSE, MODE_F, false, true, EXP>(a, grid, st);
+      if (sel == SEL_TOPN_INT) return launch_attn_t<SEL_TOPN_INT, MODE_F, false, true, EXP>(a, grid, st);
+      return launch_attn_t<SEL_TOPN_FLOAT, MODE_F, true, true, EXP>(a, grid, st);
+    }
+    if (sel == SEL_DENSE) return bias ? launch_attn_t<SEL_DENSE, MODE_F, true, false, EXP>(a, grid, st)
+                                      : launch_attn_t<SEL_DENSE, MODE_F, false, false, EXP>(a, grid, st);
+    if (sel == SEL_TOPN_INT) return launch_attn_t<SEL_TOPN_INT, MODE_F, false, false, EXP>(a, grid, st);
+    return launch_attn_t<SEL_TOPN_FLOAT, MODE_F, true, false, EXP>(a, grid, st);
+  } else if (EXP == EXP_IDX) {
+    if (sel == SEL_DENSE) return bias ? launch_attn_t<SEL_DENSE, MODE_F, true, false, EXP>(a, grid, st)
+                                      : launch_attn_t<SEL_DENSE, MODE_F, false, false, EXP>(a, grid, st);
+    if (sel == SEL_TOPN_INT) return launch_attn_t<SEL_TOPN_INT, MODE_F, false, false, EXP>(a, grid, st);
+    return launch_attn_t<SEL_TOPN_FLOAT, MODE_F, true, false, EXP>(a, grid, st);
+  } else {
+    if (sel == SEL_DENSE) return bias ? launch_attn_t<SEL_DENSE, MODE_Q, true, false, EXP>(a, grid, st)
+                                      : launch_attn_t<SEL_DENSE, MODE_Q, false, false, EXP>(a, grid, st);
+    if (sel == SEL_TOPN_INT) return launch_attn_t<SEL_TOPN_INT, MODE_Q, false, false, EXP>(a, grid, st);
+    return launch_attn_t<SEL_TOPN_FLOAT, MODE_Q, true, false, EXP>(a, grid, st);
+  }
+}
+
+// Host-side validation shared by the attention entry points.
+template <int EXP>
+had_status validate_attention(const void* Q, const void* K, const void* V, const had_shape* s,
+                              const had_relpos_bias* bias, const float* alpha_q, const float* alpha_k, int N,
+                              had_mode mode, const void* O, had_dtype o_dtype, const int32_t* idx,
+                              const uint8_t* codes, int row_begin, int row_end, const void* workspace,
+                              size_t ws_bytes, bool check_qk, bool check_o) {
+  had_status r = check_shape(s);
+  if (r != HAD_OK) return r;
+  if ((r = check_bias(s, bias)) != HAD_OK) return r;
+  if (N < 0 || (mode != HAD_MODE_FLOAT && mode != HAD_MODE_U8I8)) return HAD_ERR_INVALID;
+  if (check_qk && (!Q || !K || !aligned16(Q) || !aligned16(K))) return HAD_ERR_INVALID;
+  if (EXP == EXP_NONE || EXP == EXP_CODES) {
+    if (!V || !aligned16(V)) return HAD_ERR_INVALID;
+  }
+  if (EXP == EXP_NONE && check_o) {
+    if (!O || !aligned16(O) || (o_dtype != HAD_F32 && o_dtype != HAD_BF16)) return HAD_ERR_INVALID;
+  }
+  if (EXP == EXP_IDX && (!idx || N < 1 || (reinterpret_cast<uintptr_t>(idx) & 3u))) return HAD_ERR_INVALID;
+  if (EXP == EXP_CODES && (!codes || row_begin < 0 || row_end <= row_begin || row_end > s->n)) return HAD_ERR_INVALID;
+  for (int h = 0; alpha_q && h < s->H; ++h)
+    if (!(alpha_q[h] > 0.0f) || !std::isfinite(alpha_q[h])) return HAD_ERR_INVALID;
+  for (int h = 0; alpha_k && h < s->H; ++h)
+    if (!(alpha_k[h] > 0.0f) || !std::isfinite(alpha_k[h])) return HAD_ERR_INVALID;
+  const Ws w = ws_layout(s, mode == HAD_MODE_U8I8, bias && bias->table);
+  if (!workspace || ws_bytes < w.total || !aligned16(workspace)) return HAD_ERR_INVALID;
+  return HAD_OK;
+}
+
+int select_kind(const had_shape* s, const had_relpos_bias* bias, int N) {
+  if (N > 0 && N < s->n) return (bias && bias->table) ? SEL_TOPN_FLOAT : SEL_TOPN_INT;
+  return SEL_DENSE;
+}
+
+// Stage 1: statistics, sign/pack of Q and K, int8 V (uint8 mode), bias range (top-N with bias).
+had_status prepare_stage(const void* Q, const void* K, const void* V, const had_shape* s,
+                         const had_relpos_bias* bias, int N, had_mode mode, bool need_v, void* workspace,
+                         cudaStream_t st, unsigned* status) {
+  const bool has_bias = bias && bias->table;
+  const bool quant = (mode == HAD_MODE_U8I8);
+  const Ws w = ws_layout(s, quant, has_bias);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  uint32_t* qbits = reinterpret_cast<uint32_t*>(ws + w.qbits);
+  int8_t* kpm = reinterpret_cast<int8_t*>(ws + w.kpm);
+  double* sums = reinterpret_cast<double*>(ws + w.sums);
+  float* amax = quant ? reinterpret_cast<float*>(ws + w.amax) : nullptr;
+  int8_t* vqT = quant ? reinterpret_cast<int8_t*>(ws + w.vqT) : nullptr;
+  float* vscale = quant ? reinterpret_cast<float*>(ws + w.vscale) : nullptr;
+  const bool do_v = quant && need_v;
+  had_status r = launch_prep(s, Q, K, V, 0, do_v ? 3 : 2, sums, amax, nullptr, nullptr, qbits, nullptr, nullptr,
+                             kpm, vqT, vscale, st, status);
+  if (r != HAD_OK) return r;
+  if (select_kind(s, bias, N) == SEL_TOPN_FLOAT) {
+    float* bmm = reinterpret_cast<float*>(ws + w.bminmax);
+    k_bias_minmax<<<s->H, 256, 0, st>>>(bias->table, 2 * bias->gh - 1, 2 * bias->gw - 1, bias->prefix, bmm);
+    if ((r = check_launch("k_bias_minmax")) != HAD_OK) return r;
+  }
+  return HAD_OK;
+}
+
+// Stage 2: the fused kernel over a prepared workspace.
+template <int EXP>
+had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias* bias, const float* alpha_q,
+                        const float* alpha_k, int N, had_mode mode, void* O, had_dtype o_dtype, int32_t* idx,
+                        uint8_t* codes, int row_begin, int row_end, void* workspace, cudaStream_t st,
+                        unsigned* status) {
+  const bool has_bias = bias && bias->table;
+  const bool quant = (mode == HAD_MODE_U8I8);
+  const Ws w = ws_layout(s, quant, has_bias);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  Dims d = dims_of(s);
+  AttnArgs a{};
+  a.qbits = reinterpret_cast<uint32_t*>(ws + w.qbits);
+  a.kpm = reinterpret_cast<int8_t*>(ws + w.kpm);
+  a.V = V;
+  a.vqT = quant ? reinterpret_cast<int8_t*>(ws + w.vqT) : nullptr;
+  a.vscale = quant ? reinterpret_cast<float*>(ws + w.vscale) : nullptr;
+  a.table = has_bias ? bias->table : nullptr;
+  if (has_bias) {
+    a.gh = bias->gh; a.gw = bias->gw; a.prefix = bias->prefix;
+    a.th = 2 * bias->gh - 1; a.tw = 2 * bias->gw - 1;
+  }
+  a.bminmax = has_bias ? reinterpret_cast<float*>(ws + w.bminmax) : nullptr;
+  a.seqlens = s->seqlens;
+  a.O = O; a.o_bf16 = (o_dtype == HAD_BF16) ? 1 : 0;
+  a.idx = idx; a.codes = codes; a.row_begin = row_begin; a.row_end = row_end;
+  a.B = d.B; a.H = d.H; a.n = d.n; a.n_pad = d.n_pad; a.N = N;
+  a.status = status;
+  for (int h = 0; h < s->H; ++h) {
+    const double aq = alpha_q ? (double)alpha_q[h] : 1.0, ak = alpha_k ? (double)alpha_k[h] : 1.0;
+    a.c_head[h] = (float)(aq * ak / std::sqrt((double)s->d));
+  }
+  dim3 grid((s->n + kQT - 1) / kQT, d.BH);
+  const bool vf32 = (s->in_dtype == HAD_F32) && !quant;
+  return dispatch_attn<EXP>(select_kind(s, bias, N), quant ? MODE_Q : MODE_F, has_bias, vf32, a, grid, st);
+}
+
+had_status device_status_ptr(unsigned** out) {
+  int dev = 0;
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
+  *out = status_ptr(dev);
+  if (!*out) return cuda_fail(cudaErrorInvalidSymbol, "status word");
+  return HAD_OK;
+}
+
+// Shared body of had_attention and its exports.
+template <int EXP>
+had_status run_attention(const void* Q, const void* K, const void* V, const had_shape* s,
+                         const had_relpos_bias* bias, const float* alpha_q, const float* alpha_k, int N,
+                         had_mode mode, void* O, had_dtype o_dtype, int32_t* idx, uint8_t* codes, int row_begin,
+                         int row_end, void* workspace, size_t ws_bytes, void* stream) {
+  had_status r = validate_attention<EXP>(Q, K, V, s, bias, alpha_q, alpha_k, N, mode, O, o_dtype, idx, codes,
+                                         row_begin, row_end, workspace, ws_bytes, true, true);
+  if (r != HAD_OK) return r;
+  unsigned* status = nullptr;
+  if ((r = device_status_ptr(&status)) != HAD_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  r = prepare_stage(Q, K, V, s, bias, N, mode, EXP != EXP_IDX, workspace, st, status);
+  if (r != HAD_OK) return r;
+  return attend_stage<EXP>(V, s, bias, alpha_q, alpha_k, N, mode, O, o_dtype, idx, codes, row_begin, row_end,
+                           workspace, st, status);
+}
+
+}  // namespace
+}  // namespace had
+
+using namespace had;
+
+extern "C" {
+
+size_t had_binarize_pack_workspace_size(const had_shape* s) {
+  if (check_shape(s) != HAD_OK) return 0;
+  Dims d = dims_of(s);
+  return align_up((size_t)2 * d.BH * d.nchunks * kD * 8);
+}
+
+had_status had_binarize_pack(const void* X, const had_shape* s, const float* mu_in, float* mu_out, uint32_t* bits,
+                             void* workspace, size_t ws_bytes, void* stream) {
+  had_status r = check_shape(s);
+  if (r != HAD_OK) return r;
+  if (!X || !bits || !aligned16(X) || (reinterpret_cast<uintptr_t>(bits) & 7u)) return HAD_ERR_INVALID;
+  if ((mu_in && (reinterpret_cast<uintptr_t>(mu_in) & 3u)) || (mu_out && (reinterpret_cast<uintptr_t>(mu_out) & 3u)))
+    return HAD_ERR_INVALID;
+  if (!mu_in && (!workspace || ws_bytes < had_binarize_pack_workspace_size(s) || !aligned16(workspace)))
+    return HAD_ERR_INVALID;
+  int dev = 0;
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
+  unsigned* status = status_ptr(dev);
+  if (!status) return cuda_fail(cudaErrorInvalidSymbol, "status word");
+  return launch_prep(s, X, nullptr, nullptr, 0, 1, static_cast<double*>(workspace), nullptr, mu_in, mu_out, bits,
+                     nullptr, nullptr, nullptr, nullptr, nullptr, static_cast<cudaStream_t>(stream), status);
+}
+
+size_t had_attention_workspace_size(const had_shape* s, int N, had_mode mode, const had_relpos_bias* bias) {
+  (void)N;
+  if (check_shape(s) != HAD_OK) return 0;
+  return ws_layout(s, mode == HAD_MODE_U8I8, bias && bias->table).total;
+}
+
+had_status had_attention(const void* Q, const void* K, const void* V, const had_shape* s,
+                         const had_relpos_bias* bias, const float* alpha_q, const float* alpha_k, int N,
+                         had_mode mode, void* O, had_dtype o_dtype, void* workspace, size_t ws_bytes, void* stream) {
+  return run_attention<EXP_NONE>(Q, K, V, s, bias, alpha_q, alpha_k, N, mode, O, o_dtype, nullptr, nullptr, 0, 0,
+                                 workspace, ws_bytes, stream);
+}
+
+had_status had_attention_prepare(const void* Q, const void* K, const void* V, const had_shape* s,
+                                 const had_relpos_bias* bias, int N, had_mode mode, void* workspace, size_t ws_bytes,
+                                 void* stream) {
+  had_status r = validate_attention<EXP_NONE>(Q, K, V, s, bias, nullptr, nullptr, N, mode, nullptr, HAD_F32, nullptr,
+                                              nullptr, 0, 0, workspace, ws_bytes, true, false);
+  if (r != HAD_OK) return r;
+  unsigned* status = nullptr;
+  if ((r = device_status_ptr(&status)) != HAD_OK) return r;
+  return prepare_stage(Q, K, V, s, bias, N, mode, true, workspace, static_cast<cudaStream_t>(stream), status);
+}
+
+had_status had_attention_prepared(const void* V, const had_shape* s, const had_relpos_bias* bias,
+                                  const float* alpha_q, const float* alpha_k, int N, had_mode mode, void* O,
+                                  had_dtype o_dtype, void* workspace, size_t ws_bytes, void* stream) {
+  had_status r = validate_attention<EXP_NONE>(nullptr, nullptr, V, s, bias, alpha_q, alpha_k, N, mode, O, o_dtype,
+                                              nullptr, nullptr, 0, 0, workspace, ws_bytes, false, true);
+  if (r != HAD_OK) return r;
+  unsigned* status = nullptr;
+  if ((r = device_status_ptr(&status)) != HAD_OK) return r;
+  return attend_stage<EXP_NONE>(V, s, bias, alpha_q, alpha_k, N, mode, O, o_dtype, nullptr, nullptr, 0, 0, workspace,
+                                static_cast<cudaStream_t>(stream), status);
+}
+
+had_status had_topn_indices(const void* Q, const void* K, const had_shape* s, const had_relpos_bias* bias,
+                            const float* alpha_q, const float* alpha_k, int N, int32_t* idx, void* workspace,
+                            size_t ws_bytes, void* stream) {
+  return run_attention<EXP_IDX>(Q, K, nullptr, s, bias, alpha_q, alpha_k, N, HAD_MODE_FLOAT, nullptr, HAD_F32, idx,
+                                nullptr, 0, 0, workspace, ws_bytes, stream);
+}
+
+had_status had_attention_codes_u8(const void* Q, const void* K, const void* V, const had_shape* s,
+                                  const had_relpos_bias* bias, const float* alpha_q, const float* alpha_k, int N,
+                                  int row_begin, int row_end, uint8_t* A, void* workspace, size_t ws_bytes,
+                                  void* stream) {
+  return run_attention<EXP_CODES>(Q, K, V, s, bias, alpha_q, alpha_k, N, HAD_MODE_U8I8, nullptr, HAD_F32, nullptr, A,
+                                  row_begin, row_end, workspace, ws_bytes, stream);
+}
+
+had_status had_quantize_v(const void* V, const had_shape* s, int8_t* Vq, float* vscale, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  had_status r = check_shape(s);
+  if (r != HAD_OK) return r;
+  if (!V || !Vq || !vscale || !aligned16(V) || (reinterpret_cast<uintptr_t>(vscale) & 3u)) return HAD_ERR_INVALID;
+  const Ws w = ws_layout(s, true, false);
+  if (!workspace || ws_bytes < w.total || !aligned16(workspace)) return HAD_ERR_INVALID;
+  int dev = 0;
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
+  unsigned* status = status_ptr(dev);
+  if (!status) return cuda_fail(cudaErrorInvalidSymbol, "status word");
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Dims d = dims_of(s);
+  int8_t* vqT = reinterpret_cast<int8_t*>(ws + w.vqT);
+  r = launch_prep(s, nullptr, nullptr, V, 2, 1, reinterpret_cast<double*>(ws + w.sums),
+                  reinterpret_cast<float*>(ws + w.amax), nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, vqT,
+                  vscale, st, status);
+  if (r != HAD_OK) return r;
+  k_untranspose_vq<<<1024, 256, 0, st>>>(vqT, d.BH, d.n, d.n_pad, s->seqlens, s->H, Vq);
+  return check_launch("k_untranspose_vq");
+}
+
+size_t had_dense_reference_workspace_size(const had_shape* s) {
+  (void)s;
+  return 0;
+}
+
+had_status had_dense_reference_mode(const void* Q, const void* K, const void* V, const had_shape* s,
+                                    const had_relpos_bias* bias, int N, void* O, had_dtype o_dtype,
+                                    void* workspace, size_t ws_bytes, void* stream) {
+  (void)workspace; (void)ws_bytes;
+  had_status r = check_shape(s);
+  if (r != HAD_OK) return r;
+  if ((r = check_bias(s, bias)) != HAD_OK) return r;
+  if (s->in_dtype != HAD_BF16) return HAD_ERR_UNSUPPORTED;
+  if (N < 0) return HAD_ERR_INVALID;
+  if (N != 0 && N < s->n) return HAD_ERR_UNSUPPORTED;
+  if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return HAD_ERR_INVALID;
+  if (o_dtype != HAD_F32 && o_dtype != HAD_BF16) return HAD_ERR_INVALID;
+  int dev = 0;
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
+  unsigned* status = status_ptr(dev);
+  if (!status) return cuda_fail(cudaErrorInvalidSymbol, "status word");
+  const bool has_bias = bias && bias->table;
+  Dims d = dims_of(s);
+  AttnArgs a{};
+  a.V = V;
+  a.table = has_bias ? bias->table : nullptr;
+  if (has_bias) {
+    a.gh = bias->gh; a.gw = bias->gw; a.prefix = bias->prefix;
+    a.th = 2 * bias->gh - 1; a.tw = 2 * bias->gw - 1;
+  }
+  a.seqlens = s->seqlens;
+  a.O = O; a.o_bf16 = (o_dtype == HAD_BF16) ? 1 : 0;
+  a.B = d.B; a.H = d.H; a.n = d.n; a.n_pad = d.n_pad; a.N = 0;
+  a.status = status;
+  dim3 grid((s->n + kQT - 1) / kQT, d.BH);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
+  const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(K);
+  if (has_bias) k_dense_ref<true><<<grid, kAttnThreads, 0, st>>>(a, q, k);
+  else k_dense_ref<false><<<grid, kAttnThreads, 0, st>>>(a, q, k);
+  return check_launch("k_dense_ref");
+}
+
+had_status had_scores_int(const uint32_t* qbits, const uint32_t* kbits, const had_shape* s, int32_t* S,
+                          void* stream) {
+  had_status r = check_shape(s);
+  if (r != HAD_OK) return r;
+  if (!qbits || !kbits || !S || (reinterpret_cast<uintptr_t>(qbits) & 7u) || (reinterpret_cast<uintptr_t>(kbits) & 7u) ||
+      (reinterpret_cast<uintptr_t>(S) & 3u))
+    return HAD_ERR_INVALID;
+  int dev = 0;
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
+  unsigned* status = status_ptr(dev);
+  if (!status) return cuda_fail(cudaErrorInvalidSymbol, "status word");
+  Dims d = dims_of(s);
+  dim3 grid((s->n + kQT - 1) / kQT, d.BH);
+  k_scores_int<MODE_Q><<<grid, kAttnThreads, 0, static_cast<cudaStream_t>(stream)>>>(qbits, kbits, s->H, s->n,
+                                                                                      s->seqlens, S, status);
+  return check_launch("k_scores_int");
+}
+
+had_status had_get_device_status(void) {
+  int dev = 0;
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
+  if ((ce = cudaDeviceSynchronize()) != cudaSuccess) return cuda_fail(ce, "cudaDeviceSynchronize");
+  unsigned v = 0, zero = 0;
+  if ((ce = cudaMemcpyFromSymbol(&v, g_device_status, sizeof(v))) != cudaSuccess) return cuda_fail(ce, "read status");
+  if ((ce = cudaMemcpyToSymbol(g_device_status, &zero, sizeof(zero))) != cudaSuccess) return cuda_fail(ce, "clear status");
+  if (v & kDevErrTimeout) return HAD_ERR_TIMEOUT;
+  if (v) return HAD_ERR_DEVICE;
+  return HAD_OK;
+}
+
+const char* had_status_string(had_status st) {
+  switch (st) {
+    case HAD_OK: return "HAD_OK";
+    case HAD_ERR_INVALID: return "HAD_ERR_INVALID: invalid argument";
+    case HAD_ERR_UNSUPPORTED: return "HAD_ERR_UNSUPPORTED: shape, dtype or mode not supported";
+    case HAD_ERR_CUDA: return "HAD_ERR_CUDA: CUDA call failed";
+    case HAD_ERR_DEVICE: return "HAD_ERR_DEVICE: device-detected error (bad seqlens or candidate overflow)";
+    case HAD_ERR_TIMEOUT: return "HAD_ERR_TIMEOUT: a bounded device wait expired";
+  }
+  return "unknown had_status";
+}
+
+const char* had_last_cuda_error(void) { return t_last_error; }
+
+int had_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,169 @@
+/*
+ * had.h -- C ABI of the B200 (sm_100a) library for binarized-QK top-N
+ * attention, as defined by "Hamming Attention Distillation: Binarizing Keys
+ * and Queries for Efficient Long-Context Transformers" (HAD) and
+ * "BinaryAttention: One-Bit QK-Attention for Vision and Diffusion
+ * Transformers" (BinaryAttention).
+ *
+ * Operation (per batch b, head h, valid length L = seqlens[b] or n):
+ *   mu_X[c]  = mean_{i<L} X[i,c]                 X in {Q, K}   (BinaryAttention §2.2, scaled binarization)
+ *   X~[i,c]  = sign(X[i,c] - mu_X[c]) in {-1,+1}, packed to bits (bit 1 = -1)   (§2.2; HAD abstract)
+ *   s_ij     = d - 2 * popcount(q~_i XOR k~_j)                 (§2.1 distance view, §2.2 XNOR + popcount)
+ *   l_ij     = fmaf(s_ij, c, b_ij),  c = fp32(alpha_q[h] * alpha_k[h] / sqrt(d))   (§2.3 eq.)
+ *   kept_i   = the min(N, L) keys j < L with the largest l_ij, ties to the lower j;
+ *              N == 0 or N >= L keeps all L keys   (HAD method: top-N per query)
+ *   p_ij     = softmax over kept_i of l_ij   (§2.3 eq.)
+ *   O_i      = sum_j p_ij V_j                                   (HAD_MODE_FLOAT)
+ *   O_i[c]   = (sum_j A_ij Vq_jc) * sv_c / 255,  A_ij = floor(255 p_ij + 0.5) in uint8,
+ *              sv_c = absmax_{j<L} |V_jc| / 127, Vq = clamp(rint(V / sv_c), -127, 127)   (HAD_MODE_U8I8, §2.4)
+ * Rows i >= L of O are written as 0.  Padding tokens never enter a mean, a
+ * scale, a score or a softmax.
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller (for example
+ *     torch tensors' data_ptr()).  Q, K, V, O are contiguous [B][H][n][d].
+ *     Device pointers must be 16-byte aligned.
+ *   - The library never allocates, frees or synchronizes in these calls: work
+ *     is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
+ *     stream) and the call returns.  Scratch memory is the caller's
+ *     `workspace` of at least the size the matching *_workspace_size() returns.
+ *   - Host-side validation happens before any launch: on an error status
+ *     nothing was enqueued and no output was touched.
+ *   - Errors detected on the device (a seqlens entry outside [1, n]) set a
+ *     sticky device status word and zero the affected batch's outputs; read
+ *     it with had_get_device_status().
+ *   - Only d == 64 is supported (HAD_ERR_UNSUPPORTED otherwise), n <= 16384,
+ *     H <= 256, and B*H <= 65535.
+ */
+#ifndef HAD_H_
+#define HAD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  HAD_OK = 0,
+  HAD_ERR_INVALID = 1,      /* null/misaligned pointer, bad size, alpha <= 0, workspace too small */
+  HAD_ERR_UNSUPPORTED = 2,  /* d != 64, n > 16384, H > 256, unsupported dtype/mode combination */
+  HAD_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed; see had_last_cuda_error() */
+  HAD_ERR_DEVICE = 4,       /* device-detected error (bad seqlens); from had_get_device_status() */
+  HAD_ERR_TIMEOUT = 5       /* a bounded device-side wait expired; from had_get_device_status() */
+} had_status;
+
+typedef enum { HAD_F32 = 0, HAD_BF16 = 1 } had_dtype;
+
+typedef enum {
+  HAD_MODE_FLOAT = 0,  /* float softmax and float A.V (bf16 P x bf16 V, fp32 accumulate; fp32 V exact to ~1e-5) */
+  HAD_MODE_U8I8 = 1    /* uint8 A (scale 1/255) x per-channel int8 V, int32 accumulate (BinaryAttention §2.4) */
+} had_mode;
+
+typedef struct {
+  int B, H, n, d;           /* batch, heads, tokens per sequence (padded length), head dim */
+  had_dtype in_dtype;       /* dtype of Q, K, V (and of X in had_binarize_pack) */
+  const int32_t* seqlens;   /* DEVICE [B] valid lengths in [1, n], or NULL for all n */
+} had_shape;
+
+/* Learnable relative-position bias (BinaryAttention §2.3, "position-sensitive
+ * bias", the option its experiments use).  Token t >= prefix is patch
+ * (y, x) = divmod(t - prefix, gw) of a gh x gw grid; then
+ * b_ij = table[h][(y_i - y_j) + gh - 1][(x_i - x_j) + gw - 1], and b_ij = 0
+ * when i < prefix or j < prefix (class tokens).  Requires gh*gw + prefix == n. */
+typedef struct {
+  const float* table;  /* DEVICE fp32 [H][2*gh-1][2*gw-1]; NULL means no bias */
+  int gh, gw;
+  int prefix;
+} had_relpos_bias;
+
+/* ---- binarize and pack (BinaryAttention §2.2; HAD abstract) --------------
+ * X: [B][H][n][d] in s->in_dtype.  bits: DEVICE uint32 [B][H][n][d/32]; bit j
+ * of word w is 1 iff X[b,h,i,32w+j] < mu[b,h,32w+j] (sign -1); tokens i >= L
+ * get all-zero words.  mu_in: DEVICE fp32 [B][H][d] to use as the means, or
+ * NULL to compute them (fp64 sum over the valid tokens, / L, rounded once to
+ * fp32).  mu_out: DEVICE fp32 [B][H][d] receives the means used, or NULL.
+ * workspace: needed only when mu_in is NULL. */
+size_t had_binarize_pack_workspace_size(const had_shape* s);
+had_status had_binarize_pack(const void* X, const had_shape* s, const float* mu_in, float* mu_out, uint32_t* bits,
+                             void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- the hot path (HAD + BinaryAttention, formulas above) ----------------
+ * bias: HOST pointer to a had_relpos_bias (its table is device memory), or
+ * NULL.  alpha_q, alpha_k: HOST fp32 [H] positive per-head scales of the
+ * binarized Q and K (BinaryAttention §2.2), or NULL for 1.  N: top-N per
+ * query; 0 (or >= L) = dense.  O: DEVICE [B][H][n][d] in o_dtype. */
+size_t had_attention_workspace_size(const had_shape* s, int N, had_mode mode, const had_relpos_bias* bias);
+had_status had_attention(const void* Q, const void* K, const void* V, const had_shape* s,
+                         const had_relpos_bias* bias, const float* alpha_q, const float* alpha_k, int N,
+                         had_mode mode, void* O, had_dtype o_dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* The same operation in two stages, for callers that time or reuse them:
+ * had_attention_prepare runs the per-head statistics and the sign/pack of Q
+ * and K (and the int8 V of HAD_MODE_U8I8, and the bias range of top-N with a
+ * bias) into `workspace`; had_attention_prepared then runs the fused
+ * score/top-N/softmax/A.V kernel over that workspace.  Both must get the same
+ * s, bias, N and mode; had_attention_prepared reads V only in HAD_MODE_FLOAT.
+ * had_attention == prepare + prepared on one stream. */
+had_status had_attention_prepare(const void* Q, const void* K, const void* V, const had_shape* s,
+                                 const had_relpos_bias* bias, int N, had_mode mode, void* workspace, size_t ws_bytes,
+                                 void* stream);
+had_status had_attention_prepared(const void* V, const had_shape* s, const had_relpos_bias* bias,
+                                  const float* alpha_q, const float* alpha_k, int N, had_mode mode, void* O,
+                                  had_dtype o_dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- in-library dense comparison mode ------------------------------------
+ * Standard attention on the unbinarized inputs: l = (q . k)/sqrt(d) + b_ij with
+ * bf16 q, k on the tensor cores (fp32 accumulate), fp32 softmax, bf16 P x V.
+ * Requires in_dtype == HAD_BF16 and N == 0 or N >= n (dense); otherwise
+ * HAD_ERR_UNSUPPORTED.  Needs no workspace (ws may be NULL/0). */
+size_t had_dense_reference_workspace_size(const had_shape* s);
+had_status had_dense_reference_mode(const void* Q, const void* K, const void* V, const had_shape* s,
+                                    const had_relpos_bias* bias, int N, void* O, had_dtype o_dtype,
+                                    void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- parity / debug exports (small shapes; not part of the timed path) ---
+ * had_scores_int: S DEVICE int32 [B][H][n][n], S = d - 2*popcount(q XOR k) for
+ * i, j < L and 0 elsewhere, from packed bits as had_binarize_pack writes them. */
+had_status had_scores_int(const uint32_t* qbits, const uint32_t* kbits, const had_shape* s, int32_t* S,
+                          void* stream);
+
+/* had_topn_indices: the kept set of every query row, as DEVICE int32
+ * [B][H][n][N] in ascending key order, padded with -1 (rows i >= L are all
+ * -1).  Same arguments and workspace as had_attention with N >= 1. */
+had_status had_topn_indices(const void* Q, const void* K, const had_shape* s, const had_relpos_bias* bias,
+                            const float* alpha_q, const float* alpha_k, int N, int32_t* idx, void* workspace,
+                            size_t ws_bytes, void* stream);
+
+/* had_attention_codes_u8: the uint8 attention codes A_ij = floor(255 p_ij + 0.5)
+ * (0 off the kept set and for j >= L) of query rows [row_begin, row_end) of
+ * every (b, h), as DEVICE uint8 [B][H][row_end-row_begin][n].  Same
+ * arguments and workspace as had_attention in HAD_MODE_U8I8. */
+had_status had_attention_codes_u8(const void* Q, const void* K, const void* V, const had_shape* s,
+                                  const had_relpos_bias* bias, const float* alpha_q, const float* alpha_k, int N,
+                                  int row_begin, int row_end, uint8_t* A, void* workspace, size_t ws_bytes,
+                                  void* stream);
+
+/* had_quantize_v: the per-channel int8 V of HAD_MODE_U8I8 (BinaryAttention
+ * §2.4): Vq DEVICE int8 [B][H][n][d] (0 for tokens i >= L) and vscale DEVICE
+ * fp32 [B][H][d].  Needs had_attention_workspace_size(s, 0, HAD_MODE_U8I8, NULL). */
+had_status had_quantize_v(const void* V, const had_shape* s, int8_t* Vq, float* vscale, void* workspace,
+                          size_t ws_bytes, void* stream);
+
+/* ---- status ---------------------------------------------------------------
+ * had_get_device_status: synchronizes the current device, reads the sticky
+ * device status word of the current device, clears it, and returns HAD_OK,
+ * HAD_ERR_DEVICE or HAD_ERR_TIMEOUT. */
+had_status had_get_device_status(void);
+const char* had_status_string(had_status st);
+/* The last CUDA error string recorded by a call that returned HAD_ERR_CUDA (thread-local). */
+const char* had_last_cuda_error(void);
+/* Library version as an integer (major*10000 + minor*100 + patch). */
+int had_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HAD_H_ */

@@ -1,0 +1,107 @@
+"""CPU checks of the C ABI: the library loads, exports every function include/had.h
+declares, and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "had.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\**\s*(had_[a-z0-9_]+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def L():
+    import binarized_qk_sparse_b200 as m
+    from binarized_qk_sparse_b200 import _build
+    _build.build()
+    return m.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for must in ("had_binarize_pack", "had_attention", "had_dense_reference_mode", "had_scores_int",
+                 "had_topn_indices", "had_attention_codes_u8", "had_get_device_status", "had_status_string"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared_functions():
+        assert hasattr(L, name), f"missing export {name}"
+
+
+def _shape(m, B=1, H=1, n=64, d=64, dtype=1, seqlens=None):
+    return m.had_shape(B, H, n, d, dtype, seqlens)
+
+
+def test_host_validation_rejects_before_launch(L):
+    import binarized_qk_sparse_b200 as m
+    P = ctypes.c_void_p
+    fake = P(0x10000)          # never dereferenced: every case fails validation first
+    odd = P(0x10008)           # 8-byte aligned, not 16
+    ws = P(0x20000)
+    big = 1 << 30
+
+    def att(shape, q=fake, k=fake, v=fake, o=fake, N=0, mode=0, ws_bytes=big, alpha=None, bias=None, wsp=ws):
+        return L.had_attention(q, k, v, ctypes.byref(shape), bias, alpha, None, N, mode, o, 1, wsp, ws_bytes, None)
+
+    assert att(_shape(m, d=32)) == m.HAD_ERR_UNSUPPORTED
+    assert att(_shape(m, n=16385)) == m.HAD_ERR_UNSUPPORTED
+    assert att(_shape(m, H=257)) == m.HAD_ERR_UNSUPPORTED
+    assert att(_shape(m, B=0)) == m.HAD_ERR_INVALID
+    assert att(_shape(m, n=0)) == m.HAD_ERR_INVALID
+    assert att(_shape(m, dtype=7)) == m.HAD_ERR_INVALID
+    assert att(_shape(m), N=-1) == m.HAD_ERR_INVALID
+    assert att(_shape(m), mode=5) == m.HAD_ERR_INVALID
+    assert att(_shape(m), q=P(0)) == m.HAD_ERR_INVALID
+    assert att(_shape(m), v=odd) == m.HAD_ERR_INVALID
+    assert att(_shape(m), o=P(0)) == m.HAD_ERR_INVALID
+    assert att(_shape(m), ws_bytes=16) == m.HAD_ERR_INVALID
+    assert att(_shape(m), wsp=P(0)) == m.HAD_ERR_INVALID
+    assert att(_shape(m, seqlens=0x10002)) == m.HAD_ERR_INVALID
+    neg = (ctypes.c_float * 1)(-1.0)
+    assert att(_shape(m), alpha=ctypes.cast(neg, P)) == m.HAD_ERR_INVALID
+    zero = (ctypes.c_float * 1)(0.0)
+    assert att(_shape(m), alpha=ctypes.cast(zero, P)) == m.HAD_ERR_INVALID
+    # bias grid must cover the sequence: gh*gw + prefix == n
+    bad = m.had_relpos_bias(0x30000, 7, 7, 1)
+    assert att(_shape(m), bias=ctypes.byref(bad)) == m.HAD_ERR_INVALID
+    # dense comparison mode: bf16 only, dense only
+    shp = _shape(m, dtype=0)
+    assert L.had_dense_reference_mode(fake, fake, fake, ctypes.byref(shp), None, 0, fake, 1, None, 0, None) \
+        == m.HAD_ERR_UNSUPPORTED
+    shp = _shape(m)
+    assert L.had_dense_reference_mode(fake, fake, fake, ctypes.byref(shp), None, 5, fake, 1, None, 0, None) \
+        == m.HAD_ERR_UNSUPPORTED
+    # exports
+    assert L.had_topn_indices(fake, fake, ctypes.byref(shp), None, None, None, 0, fake, ws, big, None) \
+        == m.HAD_ERR_INVALID
+    assert L.had_attention_codes_u8(fake, fake, fake, ctypes.byref(shp), None, None, None, 0, 5, 5, fake, ws, big,
+                                    None) == m.HAD_ERR_INVALID
+    assert L.had_binarize_pack(fake, ctypes.byref(shp), None, None, fake, P(0), 0, None) == m.HAD_ERR_INVALID
+
+
+def test_workspace_size_grows_with_mode_and_bias(L):
+    import binarized_qk_sparse_b200 as m
+    shp = _shape(m, B=2, H=3, n=197)
+    f = L.had_attention_workspace_size(ctypes.byref(shp), 0, 0, None)
+    q = L.had_attention_workspace_size(ctypes.byref(shp), 0, 1, None)
+    bias = m.had_relpos_bias(0x30000, 14, 14, 1)
+    qb = L.had_attention_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(bias))
+    assert 0 < f < q < qb
+    bad = _shape(m, d=128)
+    assert L.had_attention_workspace_size(ctypes.byref(bad), 0, 0, None) == 0
+
+
+def test_status_strings(L):
+    import binarized_qk_sparse_b200 as m
+    for st in range(6):
+        assert L.had_status_string(st).startswith(b"HAD_")
+    assert L.had_version() >= 100

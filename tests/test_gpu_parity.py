@@ -1,0 +1,314 @@
+"""GPU parity: the CUDA library (through its C ABI) against the CPU oracle on the
+same seeded inputs.
+
+Bars: bit-exact packed bits, channel means, integer scores, top-N index sets
+and int8 V; O within max-abs 1e-3*max|V| (fp32 V) or 1e-2*max|V| (bf16 V);
+uint8 attention codes within 1 LSB on at most 0.1% of entries and never more.
+The full-size stress workload (B2 H16 n16384) runs in the launch configuration
+the benchmark times; the oracle checks seeded samples of its rows.
+"""
+import numpy as np
+import pytest
+
+import workloads
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():  # pragma: no cover
+    pytest.skip("needs a CUDA device", allow_module_level=True)
+
+import binarized_qk_sparse_b200 as had  # noqa: E402
+
+
+def _dev(w, x):
+    t = torch.from_numpy(np.ascontiguousarray(x))
+    if w.dtype == "bf16":
+        t = t.to(torch.bfloat16)
+    return t.cuda()
+
+
+def _dev_inputs(w):
+    Q, K, V = _dev(w, w.Q), _dev(w, w.K), _dev(w, w.V)
+    seq = None if w.seqlens is None else torch.from_numpy(w.seqlens).cuda()
+    bias = None
+    if w.bias is not None:
+        bias = had.RelPosBias(torch.from_numpy(w.bias.table).cuda(), w.bias.gh, w.bias.gw, w.bias.prefix)
+    return Q, K, V, seq, bias
+
+
+def _tol(w):
+    return (1e-3 if w.dtype == "f32" else 1e-2) * float(np.max(np.abs(w.V)))
+
+
+_cache = {}
+
+
+def _workload(name):
+    if name not in _cache:
+        _cache[name] = workloads.by_name(name)
+    return _cache[name]
+
+
+def _sample_rows(w, per_head, seed):
+    rng = np.random.default_rng(seed)
+    rows = []
+    for bh in range(w.B * w.H):
+        L = w.n if w.seqlens is None else int(w.seqlens[bh // w.H])
+        ii = rng.choice(L, size=min(per_head, L), replace=False)
+        rows.extend(bh * w.n + int(i) for i in sorted(ii))
+    return np.array(rows, np.int64)
+
+
+def _flat(t):
+    return t.reshape(-1, t.shape[-1])
+
+
+# ----------------------------------------------------------------------------- binarize + pack
+
+@pytest.mark.parametrize("name", ["tiny", "deit", "bert", "t5_256"])
+def test_binarize_pack_bit_exact(oracle_mod, name):
+    w = _workload(name)
+    Q, K, V, seq, _ = _dev_inputs(w)
+    for X, Xn in ((Q, w.Q), (K, w.K)):
+        bits, mu = had.had_binarize_pack(X, seq)
+        mu_o = oracle_mod.channel_mean(Xn, w.seqlens)
+        bits_o = oracle_mod.sign_pack(Xn, mu_o, w.seqlens)
+        np.testing.assert_array_equal(mu.cpu().numpy(), mu_o)
+        np.testing.assert_array_equal(bits.cpu().numpy().view(np.uint32), bits_o)
+        # with the oracle's means passed in, the sign/pack step alone
+        bits2, _ = had.had_binarize_pack(X, seq, mu_in=torch.from_numpy(mu_o).cuda())
+        np.testing.assert_array_equal(bits2.cpu().numpy().view(np.uint32), bits_o)
+
+
+def test_binarize_pack_stress_full_size(oracle_mod):
+    w = _workload("stress")
+    Q, K, V, seq, _ = _dev_inputs(w)
+    bits, mu = had.had_binarize_pack(K, seq)
+    mu_o = oracle_mod.channel_mean(w.K)
+    np.testing.assert_array_equal(mu.cpu().numpy(), mu_o)
+    got = bits.cpu().numpy().view(np.uint32)
+    rng = np.random.default_rng(11)
+    for b in range(w.B):
+        for h in range(w.H):
+            ii = np.sort(rng.choice(w.n, size=512, replace=False))
+            ref = oracle_mod.sign_pack(w.K[b, h, ii][None, None], mu_o[b, h][None, None])
+            np.testing.assert_array_equal(got[b, h, ii], ref[0, 0])
+
+
+# ----------------------------------------------------------------------------- scores
+
+@pytest.mark.parametrize("name", ["tiny", "bert", "t5_256"])
+def test_integer_scores_bit_exact(oracle_mod, name):
+    w = _workload(name)
+    if name == "bert":  # keep the score matrix small: 4 sequences
+        w = workloads.Workload(w.name, 4, w.H, w.n, w.d, w.dtype, w.Q[:4], w.K[:4], w.V[:4], w.seqlens[:4], None,
+                               w.passes, w.seed, w.recipe)
+    if name == "t5_256":
+        w = workloads.Workload(w.name, 2, w.H, w.n, w.d, w.dtype, w.Q[:2], w.K[:2], w.V[:2], None, None, w.passes,
+                               w.seed, w.recipe)
+    Q, K, V, seq, _ = _dev_inputs(w)
+    qb, _ = had.had_binarize_pack(Q, seq)
+    kb, _ = had.had_binarize_pack(K, seq)
+    S = had.had_scores_int(qb, kb, seq).cpu().numpy()
+    S_o = oracle_mod.binary_scores(qb.cpu().numpy().view(np.uint32), kb.cpu().numpy().view(np.uint32), 64, w.seqlens)
+    np.testing.assert_array_equal(S, S_o)
+
+
+# ----------------------------------------------------------------------------- top-N index sets
+
+def _oracle_full(oracle_mod, w, N, mode, rows=None, want_idx=False, want_codes=False):
+    key = (w.name, N, mode, None if rows is None else rows.tobytes(), want_idx, want_codes)
+    if key not in _cache:
+        b = None if w.bias is None else oracle_mod.RelPosBias(w.bias.table, w.bias.gh, w.bias.gw, w.bias.prefix)
+        _cache[key] = oracle_mod.attention(w.Q, w.K, w.V, N=N, mode=mode, seqlens=w.seqlens, bias=b, rows=rows,
+                                           want_idx=want_idx, want_codes=want_codes)
+    return _cache[key]
+
+
+@pytest.mark.parametrize("name,N", [("tiny", 15), ("tiny", 1), ("tiny", 127), ("bert", 30), ("t5_128", 15),
+                                    ("t5_256", 30), ("t5_512", 60), ("t5_1024", 120)])
+def test_topn_sets_bit_exact(oracle_mod, name, N):
+    w = _workload(name)
+    Q, K, V, seq, bias = _dev_inputs(w)
+    idx = had.had_topn_indices(Q, K, N, seq, bias).cpu().numpy().reshape(-1, N)
+    ref = _oracle_full(oracle_mod, w, N, 0, want_idx=True).idx
+    np.testing.assert_array_equal(idx, ref)
+
+
+def test_topn_sets_with_bias_deit_shape(oracle_mod):
+    w = _workload("deit")
+    w = workloads.Workload(w.name + "_b4", 4, w.H, w.n, w.d, w.dtype, w.Q[:4], w.K[:4], w.V[:4], None, w.bias,
+                           w.passes, w.seed, w.recipe)
+    Q, K, V, seq, bias = _dev_inputs(w)
+    for N in (1, 16, 100):
+        idx = had.had_topn_indices(Q, K, N, seq, bias).cpu().numpy().reshape(-1, N)
+        ref = _oracle_full(oracle_mod, w, N, 0, want_idx=True).idx
+        np.testing.assert_array_equal(idx, ref)
+
+
+def test_topn_sets_stress_full_size(oracle_mod):
+    w = _workload("stress")
+    Q, K, V, seq, bias = _dev_inputs(w)
+    N = 1920
+    idx = had.had_topn_indices(Q, K, N, seq, bias)
+    rows = _sample_rows(w, 24, 12)
+    got = _flat(idx)[torch.from_numpy(rows).cuda()].cpu().numpy()
+    del idx
+    ref = _oracle_full(oracle_mod, w, N, 0, rows=rows, want_idx=True).idx
+    np.testing.assert_array_equal(got, ref)
+
+
+# ----------------------------------------------------------------------------- outputs
+
+@pytest.mark.parametrize("name,N", [("tiny", 15), ("tiny", 0), ("bert", 30), ("t5_128", 15), ("t5_1024", 120)])
+def test_float_output_within_tolerance(oracle_mod, name, N):
+    w = _workload(name)
+    Q, K, V, seq, bias = _dev_inputs(w)
+    O = had.had_attention(Q, K, V, N=N, mode="float", seqlens=seq, bias=bias).float().cpu().numpy()
+    ref = _oracle_full(oracle_mod, w, N, 0).O
+    err = np.max(np.abs(O - ref))
+    assert err <= _tol(w), (err, _tol(w))
+
+
+def test_float_output_dense_with_bias(oracle_mod):
+    w = _workload("deit")
+    w = workloads.Workload(w.name + "_b4", 4, w.H, w.n, w.d, w.dtype, w.Q[:4], w.K[:4], w.V[:4], None, w.bias,
+                           w.passes, w.seed, w.recipe)
+    Q, K, V, seq, bias = _dev_inputs(w)
+    for N in (0, 50):
+        O = had.had_attention(Q, K, V, N=N, mode="float", bias=bias).float().cpu().numpy()
+        ref = _oracle_full(oracle_mod, w, N, 0).O
+        assert np.max(np.abs(O - ref)) <= _tol(w)
+
+
+def _codes_ok(got, ref):
+    diff = np.abs(got.astype(np.int32) - ref.astype(np.int32))
+    assert diff.max() <= 1, diff.max()
+    assert (diff > 0).mean() <= 1e-3, (diff > 0).mean()
+
+
+def test_u8i8_deit_full(oracle_mod):
+    w = _workload("deit")
+    Q, K, V, seq, bias = _dev_inputs(w)
+    O = had.had_attention(Q, K, V, N=0, mode="u8i8", seqlens=seq, bias=bias).float().cpu().numpy()
+    ref = _oracle_full(oracle_mod, w, 0, 1, want_codes=True)
+    assert np.max(np.abs(O - ref.O)) <= _tol(w)
+    A = had.had_attention_codes_u8(Q, K, V, 0, w.n, N=0, seqlens=seq, bias=bias).cpu().numpy()
+    _codes_ok(A.reshape(-1, w.n), ref.Aq)
+    Vq, sc = had.had_quantize_v(V, seq)
+    np.testing.assert_array_equal(Vq.cpu().numpy(), ref.Vq)
+    np.testing.assert_array_equal(sc.cpu().numpy(), ref.vscale)
+
+
+def test_u8i8_topn_bert(oracle_mod):
+    w = _workload("bert")
+    Q, K, V, seq, bias = _dev_inputs(w)
+    O = had.had_attention(Q, K, V, N=30, mode="u8i8", seqlens=seq).float().cpu().numpy()
+    ref = _oracle_full(oracle_mod, w, 30, 1, want_codes=True)
+    assert np.max(np.abs(O - ref.O)) <= _tol(w)
+    A = had.had_attention_codes_u8(Q, K, V, 0, w.n, N=30, seqlens=seq).cpu().numpy()
+    _codes_ok(A.reshape(-1, w.n), ref.Aq)
+
+
+def test_stress_full_size_both_passes(oracle_mod):
+    w = _workload("stress")
+    Q, K, V, seq, bias = _dev_inputs(w)
+    rows = _sample_rows(w, 16, 13)
+    rows_t = torch.from_numpy(rows).cuda()
+    Of = _flat(had.had_attention(Q, K, V, N=1920, mode="float", bias=bias))[rows_t].float().cpu().numpy()
+    ref_f = _oracle_full(oracle_mod, w, 1920, 0, rows=rows)
+    assert np.max(np.abs(Of - ref_f.O)) <= _tol(w)
+    Oq = _flat(had.had_attention(Q, K, V, N=0, mode="u8i8", bias=bias))[rows_t].float().cpu().numpy()
+    ref_q = _oracle_full(oracle_mod, w, 0, 1, rows=rows, want_codes=True)
+    assert np.max(np.abs(Oq - ref_q.O)) <= _tol(w)
+    # codes of a contiguous band of rows in every head
+    r0, r1 = 5000, 5008
+    A = had.had_attention_codes_u8(Q, K, V, r0, r1, N=0, bias=bias).cpu().numpy().reshape(-1, w.n)
+    band = np.array([bh * w.n + i for bh in range(w.B * w.H) for i in range(r0, r1)], np.int64)
+    ref_c = _oracle_full(oracle_mod, w, 0, 1, rows=band, want_codes=True)
+    _codes_ok(A, ref_c.Aq)
+
+
+# ----------------------------------------------------------------------------- comparison mode
+
+def test_dense_reference_mode(oracle_mod):
+    w = _workload("deit")
+    B = 4
+    Qn, Kn, Vn = w.Q[:B], w.K[:B], w.V[:B]
+    w4 = workloads.Workload(w.name, B, w.H, w.n, w.d, w.dtype, Qn, Kn, Vn, None, w.bias, w.passes, w.seed, w.recipe)
+    Q, K, V, seq, bias = _dev_inputs(w4)
+    O = had.had_dense_reference_mode(Q, K, V, bias=bias).float().cpu().numpy()
+    b = oracle_mod.RelPosBias(w.bias.table, w.bias.gh, w.bias.gw, w.bias.prefix)
+    ref = oracle_mod.dense_attention(Qn, Kn, Vn, bias=b)
+    assert np.max(np.abs(O - ref)) <= 1e-2 * np.max(np.abs(Vn))
+
+
+# ----------------------------------------------------------------------------- edge cases
+
+def _small(seed, B=3, H=2, n=70, dtype="bf16"):
+    rng = np.random.default_rng(seed)
+    Q = workloads.bf16_round(rng.standard_normal((B, H, n, 64)).astype(np.float32))
+    K = workloads.bf16_round(rng.standard_normal((B, H, n, 64)).astype(np.float32))
+    V = workloads.bf16_round(rng.standard_normal((B, H, n, 64)).astype(np.float32))
+    return workloads.Workload(f"small{seed}", B, H, n, 64, dtype, Q, K, V, None, None, [], seed, "")
+
+
+@pytest.mark.parametrize("n", [1, 5, 63, 64, 65, 130])
+def test_edge_lengths(oracle_mod, n):
+    w = _small(20 + n, n=n)
+    w.seqlens = np.array([n, max(1, n // 2), 1], np.int32)
+    Q, K, V, seq, bias = _dev_inputs(w)
+    for N in (0, 1, 3, n + 2):
+        O = had.had_attention(Q, K, V, N=N, seqlens=seq).float().cpu().numpy()
+        ref = oracle_mod.attention(w.Q, w.K, w.V, N=N, seqlens=w.seqlens).O
+        assert np.max(np.abs(O - ref)) <= _tol(w)
+        Oq = had.had_attention(Q, K, V, N=N, mode="u8i8", seqlens=seq).float().cpu().numpy()
+        refq = oracle_mod.attention(w.Q, w.K, w.V, N=N, mode=1, seqlens=w.seqlens).O
+        assert np.max(np.abs(Oq - refq)) <= _tol(w)
+        if N >= 1:
+            idx = had.had_topn_indices(Q, K, N, seq).cpu().numpy().reshape(-1, N)
+            np.testing.assert_array_equal(idx, oracle_mod.attention(w.Q, w.K, w.V, N=N, seqlens=w.seqlens,
+                                                                    want_idx=True).idx)
+
+
+def test_all_ties_keep_lowest_indices(oracle_mod):
+    # constant Q and K: every score equals d, so the kept set must be keys 0..N-1
+    w = _small(30, B=1, H=1, n=200)
+    w.Q[:] = 1.0
+    w.K[:] = -2.0
+    Q, K, V, seq, bias = _dev_inputs(w)
+    idx = had.had_topn_indices(Q, K, 17).cpu().numpy().reshape(-1, 17)
+    assert (idx == np.arange(17)[None, :]).all()
+    O = had.had_attention(Q, K, V, N=17).float().cpu().numpy()
+    ref = oracle_mod.attention(w.Q, w.K, w.V, N=17).O
+    assert np.max(np.abs(O - ref)) <= _tol(w)
+
+
+def test_alpha_and_bias_ties(oracle_mod):
+    # a bias table of few distinct values makes many exact logit ties
+    w = _small(31, B=2, H=2, n=65)
+    gh, gw, prefix = 8, 8, 1
+    rng = np.random.default_rng(5)
+    table = (rng.integers(-2, 3, size=(2, 15, 15)) * 0.25).astype(np.float32)
+    w.bias = workloads.Bias(table, gh, gw, prefix)
+    Q, K, V, seq, bias = _dev_inputs(w)
+    aq, ak = np.array([1.5, 0.5], np.float32), np.array([2.0, 1.0], np.float32)
+    b = oracle_mod.RelPosBias(table, gh, gw, prefix)
+    for N in (1, 7, 30, 64):
+        idx = had.had_topn_indices(Q, K, N, bias=bias, alpha_q=aq, alpha_k=ak).cpu().numpy().reshape(-1, N)
+        ref = oracle_mod.attention(w.Q, w.K, w.V, N=N, bias=b, alpha_q=aq, alpha_k=ak, want_idx=True)
+        np.testing.assert_array_equal(idx, ref.idx)
+        O = had.had_attention(Q, K, V, N=N, bias=bias, alpha_q=aq, alpha_k=ak).float().cpu().numpy()
+        assert np.max(np.abs(O - ref.O)) <= _tol(w)
+
+
+def test_bad_seqlens_raise_device_status():
+    w = _small(32, B=2, H=1, n=64)
+    Q, K, V, _, _ = _dev_inputs(w)
+    assert had.had_get_device_status() == had.HAD_OK
+    seq = torch.tensor([64, 0], dtype=torch.int32, device="cuda")
+    O = had.had_attention(Q, K, V, N=5, seqlens=seq)
+    assert had.had_get_device_status() == had.HAD_ERR_DEVICE
+    assert had.had_get_device_status() == had.HAD_OK   # cleared on read
+    assert not O[1].float().abs().sum().item()
