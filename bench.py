@@ -1,0 +1,399 @@
+"""Benchmark of binarized-QK top-N attention (HAD + BinaryAttention) on B200.
+
+Default workload: the DeiT-shaped BinaryAttention configuration (B64 H12 n197
+d64 bf16, relative-position bias 27x27 per head with one class token, dense,
+uint8 A x int8 V).  A "step" is one pass of the whole hot path over one batch:
+channel means + sign/pack of Q and K, int8 V, scores, logits, (top-N),
+softmax, A.V, output.  Metric: queries/s = valid (batch, head, query) rows per
+second over all ranks.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+Timing: W untimed warm-up steps; K timed steps, each bracketed by CUDA events
+on the launching stream, with an L2 flush (a 256 MiB write, larger than the
+126 MB L2) between steps outside the events; barrier + synchronize on both
+sides; the reported time is the max over ranks.  The fused kernel's own time
+comes from events recorded between the library's two stages
+(had_attention_prepare / had_attention_prepared) on the same stream.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import workloads  # noqa: E402
+
+METRIC = "binary-QK top-N attention queries/sec on 1 B200; % of roofline (HBM or int pipe)"
+UNIT = "queries/s"
+
+# (workload name, N, mode) per bench workload id
+WORKLOADS = {
+    "deit": ("deit", 0, "u8i8"),
+    "tiny": ("tiny", 15, "float"),
+    "bert": ("bert", 30, "float"),
+    "t5_128": ("t5_128", 15, "float"),
+    "t5_256": ("t5_256", 30, "float"),
+    "t5_512": ("t5_512", 60, "float"),
+    "t5_1024": ("t5_1024", 120, "float"),
+    "stress_topn": ("stress", 1920, "float"),
+    "stress_u8i8": ("stress", 0, "u8i8"),
+}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "sm_max_mhz": 1965.0}, \
+        "fallback"
+
+
+def kernel_bytes_per_token(mode: str, v_bytes: int, o_bytes: int) -> int:
+    """Algorithmic bytes per valid token of the fused kernel (k_attn).
+
+    Reads the packed sign bits of Q and K (8 B each at d = 64), V (float mode,
+    d * v_bytes) or int8 V (uint8 mode, d bytes), and writes O (d * o_bytes).
+    """
+    d = 64
+    v = d if mode == "u8i8" else d * v_bytes
+    return 8 + 8 + v + d * o_bytes
+
+
+def path_bytes_per_token(mode: str, in_bytes: int, o_bytes: int) -> int:
+    """Algorithmic bytes per token of the whole path: read Q, K, V once, write and
+    read back the packed bits (and the int8 V in uint8 mode), write O once."""
+    d = 64
+    b = 3 * d * in_bytes + 2 * 8 * 2 + d * o_bytes
+    if mode == "u8i8":
+        b += 2 * d
+    return b
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(prefix="clk", suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) < 9:
+                    continue
+                try:
+                    sm.append(float(f[1]))
+                    smax = float(f[2])
+                except ValueError:
+                    continue
+                for k, v in zip(names, f[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(k)
+            os.unlink(self.path)
+        except Exception:
+            pass
+        if not sm:
+            return None
+        loaded = [x for x in sm if smax is None or x > 0.5 * smax] or sm
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- reference arm (the oracle)
+
+def _oracle_rows_per_sec(w, N, mode, rows):
+    import oracle
+    b = None if w.bias is None else oracle.RelPosBias(w.bias.table, w.bias.gh, w.bias.gw, w.bias.prefix)
+    t0 = time.perf_counter()
+    oracle.attention(w.Q, w.K, w.V, N=N, mode=1 if mode == "u8i8" else 0, seqlens=w.seqlens, bias=b, rows=rows)
+    return len(rows) / (time.perf_counter() - t0)
+
+
+def _valid_rows(w):
+    rows = []
+    for bh in range(w.B * w.H):
+        L = w.n if w.seqlens is None else int(w.seqlens[bh // w.H])
+        rows.append(np.arange(bh * w.n, bh * w.n + L, dtype=np.int64))
+    return np.concatenate(rows)
+
+
+def cpu_baseline(w, N, mode, budget_s=15.0):
+    """The oracle as it stands, on the host cores, on a bounded seeded sample of the workload's rows."""
+    import oracle
+    allrows = _valid_rows(w)
+    rng = np.random.default_rng(99)
+    probe = np.sort(rng.choice(allrows, size=min(len(allrows), 64), replace=False))
+    rate = _oracle_rows_per_sec(w, N, mode, probe)
+    want = int(min(len(allrows), max(64, rate * budget_s)))
+    rows = np.sort(rng.choice(allrows, size=want, replace=False)) if want < len(allrows) else allrows
+    rate = _oracle_rows_per_sec(w, N, mode, rows)
+    return {"value": rate, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(rows)} of {len(allrows)} query rows of {w.name} (seeded), full per-head means/scales"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    import oracle
+    name, N, mode = WORKLOADS[args.workload]
+    w = workloads.by_name(name)
+    allrows = _valid_rows(w)
+    rng = np.random.default_rng(7)
+    probe = np.sort(rng.choice(allrows, size=min(len(allrows), 64), replace=False))
+    rate = _oracle_rows_per_sec(w, N, mode, probe)
+    budget = 90.0 / max(1, args.steps + args.warmup)
+    per_step = int(max(1, min(len(allrows), rate * budget)))
+    times = []
+    for s in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(allrows, size=per_step, replace=False))
+        t0 = time.perf_counter()
+        _oracle_rows_per_sec(w, N, mode, rows)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = per_step * len(times) / total
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config(w, N, mode),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                             "sample": f"{per_step} seeded query rows of {w.name} per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(w, N, mode):
+    c = {"workload": f"{w.name}_{'dense' if N == 0 else f'top{N}'}_{mode}", "B": w.B, "H": w.H, "n": w.n, "d": w.d,
+         "N": N, "mode": mode, "in_dtype": w.dtype, "seed": w.seed,
+         "bias": None if w.bias is None else f"relpos {w.bias.table.shape[1]}x{w.bias.table.shape[2]}/head, "
+                                              f"prefix {w.bias.prefix}",
+         "seqlens": None if w.seqlens is None else "U{32..256} per sequence",
+         "l2": "flushed between timed steps (256 MiB write)"}
+    return c
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    import binarized_qk_sparse_b200 as had
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    name, N, mode = WORKLOADS[args.workload]
+    w = workloads.by_name(name)
+    bf16 = w.dtype == "bf16"
+    tdt = torch.bfloat16 if bf16 else torch.float32
+
+    def dev_t(x):
+        return torch.from_numpy(x).to(tdt).to(dev)
+
+    Q, K, V = dev_t(w.Q), dev_t(w.K), dev_t(w.V)
+    seq = None if w.seqlens is None else torch.from_numpy(w.seqlens).to(dev)
+    bias = None
+    if w.bias is not None:
+        bias = had.RelPosBias(torch.from_numpy(w.bias.table).to(dev), w.bias.gh, w.bias.gw, w.bias.prefix)
+    O = torch.empty_like(V)
+    ws_bytes = had.had_attention_workspace_size(Q, N, mode, seq, bias)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    L = had.lib()
+    import ctypes
+    shp = had.make_shape(Q, seq)
+    bstruct = None if bias is None else ctypes.byref(had.had_relpos_bias(bias.table.data_ptr(), bias.gh, bias.gw,
+                                                                          bias.prefix))
+    mcode = had._MODES[mode]
+    sp = ctypes.c_void_p(stream.cuda_stream)
+
+    def prepare():
+        st = L.had_attention_prepare(ctypes.c_void_p(Q.data_ptr()), ctypes.c_void_p(K.data_ptr()),
+                                     ctypes.c_void_p(V.data_ptr()), ctypes.byref(shp), bstruct, N, mcode,
+                                     ctypes.c_void_p(ws.data_ptr()), ws_bytes, sp)
+        if st:
+            raise had.HadError(st, "had_attention_prepare")
+
+    def attend():
+        st = L.had_attention_prepared(ctypes.c_void_p(V.data_ptr()), ctypes.byref(shp), bstruct, None, None, N, mcode,
+                                      ctypes.c_void_p(O.data_ptr()), had._dtype_code(O),
+                                      ctypes.c_void_p(ws.data_ptr()), ws_bytes, sp)
+        if st:
+            raise had.HadError(st, "had_attention_prepared")
+
+    kernels_per_step = 3 if (N == 0 or N >= w.n or bias is None) else 4
+    if mode == "float" and not (N == 0 or N >= w.n) and bias is None:
+        kernels_per_step = 3
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            prepare()
+            attend()
+        stream.synchronize()
+        assert had.had_get_device_status() == had.HAD_OK
+
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+               torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+        clocks = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+        clocks.start()
+        wall0 = time.perf_counter()
+        for s in range(args.steps):
+            flush.zero_()
+            ev[s][0].record(stream)
+            prepare()
+            ev[s][1].record(stream)
+            attend()
+            ev[s][2].record(stream)
+        torch.cuda.synchronize()
+        wall = time.perf_counter() - wall0
+        clk = clocks.stop()
+        if dist is not None:
+            dist.barrier()
+    step_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    total_ms = sum(step_ms)
+    if dist is not None:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    queries = w.valid_tokens
+    value = queries * world * args.steps / (total_ms * 1e-3)
+    ms_per_step = total_ms / args.steps
+
+    # e2e: pinned host -> device, the call, device -> host of O, every step
+    hQ, hK, hV = Q.cpu().pin_memory(), K.cpu().pin_memory(), V.cpu().pin_memory()
+    hO = torch.empty_like(O, device="cpu").pin_memory()
+    e2e_steps = min(args.steps, 30)
+    h2d = 3 * Q.numel() * Q.element_size()
+    d2h = O.numel() * O.element_size()
+    with torch.cuda.stream(stream):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        for s in range(e2e_steps + 2):
+            if s == 2:
+                e0.record(stream)
+            Q.copy_(hQ, non_blocking=True)
+            K.copy_(hK, non_blocking=True)
+            V.copy_(hV, non_blocking=True)
+            had.had_attention(Q, K, V, N=N, mode=mode, seqlens=seq, bias=bias, out=O, workspace=ws, stream=stream)
+            hO.copy_(O, non_blocking=True)
+        e1.record(stream)
+        stream.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if dist is not None:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    if rank != 0:
+        return 0
+    peaks, peak_kind = _peaks()
+    attn_avg_ms = statistics.mean(attn_ms)
+    kbytes = kernel_bytes_per_token(mode, 2 if bf16 else 4, O.element_size()) * queries
+    if bias is not None:
+        kbytes += w.bias.table.nbytes
+    achieved = kbytes / (attn_avg_ms * 1e-3) / 1e9
+    pbytes = path_bytes_per_token(mode, 2 if bf16 else 4, O.element_size()) * queries
+    path_achieved = pbytes / (ms_per_step * 1e-3) / 1e9
+    traffic = None
+    tr_path = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(tr_path):
+        with open(tr_path) as f:
+            traffic = json.load(f).get(args.workload)
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8i8" if mode == "u8i8" else ("bf16" if bf16 else "f32"),
+        "data": "synthetic", "config": {**_config(w, N, mode), "parallelism": f"replicas x{world} (no collective)"},
+        "score_ops_per_s": w.valid_scores() * world * args.steps / (total_ms * 1e-3),
+        "roofline": {"bound": "hbm", "kernel": "k_attn (fused score/top-N/softmax/A.V)", "achieved": achieved,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": traffic, "algorithmic_bytes_per_launch": kbytes,
+                     "avg_launch_ms": attn_avg_ms, "peak_kind": peak_kind},
+        "roofline_path": {"bound": "hbm", "achieved": path_achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                          "frac": path_achieved / peaks["hbm_gbs"], "algorithmic_bytes_per_step": pbytes},
+        "e2e": {"value": queries * world / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": kernels_per_step * args.steps,
+        "clocks": clk,
+        "wall_s_timed_loop": wall,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, N, mode)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="deit", choices=sorted(WORKLOADS))
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        try:
+            return run_gpu(args, rank, world, local_rank)
+        finally:
+            dist.destroy_process_group()
+    return run_gpu(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())
