@@ -69,6 +69,7 @@ def lib():
         L.had_binarize_pack_workspace_size.argtypes = [SP]
         L.had_binarize_pack_workspace_size.restype = SZ
         L.had_binarize_pack.argtypes = [P, SP, P, P, P, P, SZ, P]
+        L.had_binarize_pack_noalloc.argtypes = [P, SP, P, P, P]
         L.had_attention_workspace_size.argtypes = [SP, I, I, BP]
         L.had_attention_workspace_size.restype = SZ
         L.had_attention.argtypes = [P, P, P, SP, BP, P, P, I, I, P, I, P, SZ, P]
@@ -79,7 +80,7 @@ def lib():
         L.had_topn_indices.argtypes = [P, P, SP, BP, P, P, I, P, P, SZ, P]
         L.had_attention_codes_u8.argtypes = [P, P, P, SP, BP, P, P, I, I, I, P, P, SZ, P]
         L.had_quantize_v.argtypes = [P, SP, P, P, P, SZ, P]
-        for f in ("had_binarize_pack", "had_attention", "had_dense_reference_mode", "had_scores_int",
+        for f in ("had_binarize_pack", "had_binarize_pack_noalloc", "had_attention", "had_dense_reference_mode", "had_scores_int",
                   "had_topn_indices", "had_attention_codes_u8", "had_quantize_v", "had_get_device_status"):
             getattr(L, f).restype = I
         L.had_get_device_status.argtypes = []
@@ -173,6 +174,26 @@ def had_binarize_pack(X, seqlens=None, mu_in=None, want_mu=True, workspace=None,
                                  0 if ws is None else ws.numel(), _stream(stream))
     _raise(st, "had_binarize_pack")
     return bits, (mu if mu_in is None else mu_in)
+
+
+def had_binarize_pack_noalloc(X, seqlens=None, bits=None, mu=None, stream=None):
+    """had_binarize_pack with the library's own fixed device scratch instead of a workspace.
+
+    For callers that cannot allocate device memory when they call (the library
+    allocates nothing either).  Shapes with B*H*ceil(n/64) > 8192 are rejected;
+    concurrent calls on one device share the scratch and must be serialized.
+    Returns (bits [B,H,n,d/32] int32 view of the uint32 words, mu [B,H,d] fp32).
+    """
+    _check_dev(X, seqlens, bits, mu)
+    B, H, n, d = X.shape
+    shp = make_shape(X, seqlens)
+    if bits is None:
+        bits = torch.empty((B, H, n, d // 32), dtype=torch.int32, device=X.device)
+    if mu is None:
+        mu = torch.empty((B, H, d), dtype=torch.float32, device=X.device)
+    st = lib().had_binarize_pack_noalloc(_ptr(X), ctypes.byref(shp), _ptr(mu), _ptr(bits), _stream(stream))
+    _raise(st, "had_binarize_pack_noalloc")
+    return bits, mu
 
 
 def had_attention_workspace_size(X, N=0, mode="float", seqlens=None, bias=None) -> int:

@@ -524,6 +524,70 @@ had_status had_scores_int(const uint32_t* qbits, const uint32_t* kbits, const ha
   return check_launch("k_scores_int");
 }
 
+}  // extern "C"
+
+// ---------------------------------------------------------------------------- no-allocation variant
+//
+// Scratch for had_binarize_pack_noalloc: the fp64 per-chunk channel sums that
+// had_binarize_pack keeps in the caller's workspace live here instead, in a
+// fixed array that every GPU loading this library holds until the process
+// exits.  In host code `g_pack_scratch` only names a host-side stand-in; the
+// device address comes from cudaGetSymbolAddress, taken once per device.
+namespace had {
+namespace {
+
+constexpr size_t kPackScratchBytes = (size_t)4 << 20;  // 4 MiB: B*H*ceil(n/64) <= 8192
+__device__ __align__(256) unsigned char g_pack_scratch[kPackScratchBytes];
+
+had_status pack_scratch_ptr(double** out) {
+  static std::mutex mu;
+  static double* ptrs[kMaxDevices] = {nullptr};
+  int dev = 0;
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return HAD_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    ce = cudaGetSymbolAddress(&p, g_pack_scratch);  // with `dev` current
+    if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetSymbolAddress(g_pack_scratch)");
+    ptrs[dev] = static_cast<double*>(p);
+  }
+  *out = ptrs[dev];
+  return HAD_OK;
+}
+
+}  // namespace
+}  // namespace had
+
+extern "C" {
+
+had_status had_binarize_pack_noalloc(const void* X, const had_shape* s, float* mu_out, uint32_t* bits,
+                                     void* stream) {
+  had_status r = check_shape(s);
+  if (r != HAD_OK) return r;
+  if (!X || !bits || !aligned16(X) || (reinterpret_cast<uintptr_t>(bits) & 7u)) return HAD_ERR_INVALID;
+  if (mu_out && (reinterpret_cast<uintptr_t>(mu_out) & 3u)) return HAD_ERR_INVALID;
+  const Dims d = dims_of(s);
+  const size_t need = (size_t)d.BH * d.nchunks * kD * sizeof(double);
+  if (need > kPackScratchBytes) {
+    snprintf(t_last_error, sizeof(t_last_error),
+             "had_binarize_pack_noalloc: B*H*ceil(n/64) = %lld exceeds the static scratch limit of %lld",
+             (long long)d.BH * d.nchunks, (long long)(kPackScratchBytes / (kD * sizeof(double))));
+    return HAD_ERR_UNSUPPORTED;
+  }
+  double* scratch = nullptr;
+  if ((r = pack_scratch_ptr(&scratch)) != HAD_OK) return r;
+  int dev = 0;
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
+  unsigned* status = status_ptr(dev);
+  if (!status) return cuda_fail(cudaErrorInvalidSymbol, "status word");
+  // k_stats writes every partial sum k_pack reads, so no part of the scratch needs clearing.
+  return launch_prep(s, X, nullptr, nullptr, 0, 1, scratch, nullptr, nullptr, mu_out, bits, nullptr, nullptr, nullptr,
+                     nullptr, nullptr, static_cast<cudaStream_t>(stream), status);
+}
+
 had_status had_get_device_status(void) {
   int dev = 0;
   cudaError_t ce = cudaGetDevice(&dev);

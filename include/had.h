@@ -89,6 +89,24 @@ size_t had_binarize_pack_workspace_size(const had_shape* s);
 had_status had_binarize_pack(const void* X, const had_shape* s, const float* mu_in, float* mu_out, uint32_t* bits,
                              void* workspace, size_t ws_bytes, void* stream);
 
+/* had_binarize_pack_noalloc: the same computed-means pack as had_binarize_pack
+ * (mu_in == NULL), for callers that cannot allocate device memory at the point
+ * of call -- for example a plugin run inside a host framework that owns every
+ * device allocation, or a latency-critical loop that must not call cudaMalloc
+ * (which can synchronize the device) -- and so cannot supply a workspace.  The
+ * paper has no counterpart: this is a library convenience.
+ * Its scratch is a fixed 4 MiB device array inside the library, which every
+ * GPU that loads the library holds until the process exits; shapes with
+ * B*H*ceil(n/64) > 8192 are rejected with HAD_ERR_UNSUPPORTED (message in
+ * had_last_cuda_error()).  The first call on each device looks up the array's
+ * device address (cudaGetSymbolAddress, with that device current), so make
+ * that first call before any stream capture.  All calls on a device share the
+ * one array: calls that overlap on the GPU (other streams, other host
+ * threads) race and corrupt each other's means; serialize them.  Nothing in
+ * the array needs clearing: each call overwrites every entry it reads.
+ * Allocates and frees nothing. */
+had_status had_binarize_pack_noalloc(const void* X, const had_shape* s, float* mu_out, uint32_t* bits, void* stream);
+
 /* ---- the hot path (HAD + BinaryAttention, formulas above) ----------------
  * bias: HOST pointer to a had_relpos_bias (its table is device memory), or
  * NULL.  alpha_q, alpha_k: HOST fp32 [H] positive per-head scales of the
