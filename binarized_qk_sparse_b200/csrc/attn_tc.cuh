@@ -1,0 +1,712 @@
+// attn_tc.cuh -- the fused binarized-QK top-N attention kernel on the sm_100a
+// tensor cores (tcgen05 + TMA + tensor memory).
+//
+// One CTA = one (batch, head) and 128 query rows; query row r of the tile is
+// tensor-memory lane r and softmax thread r, so every per-row step (histogram,
+// threshold, tie rule, softmax, normalization) is thread-local.
+//   warps 0-3  softmax/select: read a 64-key score tile from TMEM, build per-row
+//              histograms, apply the top-N threshold, write P (or uint8 A) back
+//              to TMEM, normalize and store O.
+//   warp 4     MMA issuer (one thread) + TMEM allocation.
+//   warp 5     TMA producer: +-1 int8 K tiles (64 keys x 64 B, 64-byte swizzle),
+//              V tiles (bf16 [64 keys][64], 128-byte swizzle, MN-major B) or int8
+//              V^T tiles ([64 channels][64 keys], 64-byte swizzle, K-major B).
+// Tensor memory (256 columns): two score buffers S0 [0,64) and S1 [64,128) so the
+// score MMA of tile t+1 runs while the softmax warps work on tile t; P [128,160)
+// bf16 (or [128,144) uint8 codes); residual P [160,192) for fp32 V; O [192,256).
+//
+// Score (BinaryAttention §2.1/§2.2): S = Q~ K~^T with kind::i8 on +-1 operands,
+// so S = d - 2*popcount(q XOR k) exactly.  A.V: kind::f16 (bf16 P from TMEM x
+// bf16 V; fp32 V as bf16 head + residual, three products) or kind::i8 (uint8 A
+// from TMEM x int8 V, BinaryAttention §2.4).
+// Top-N (HAD: the N largest scores per query, ties to the lower key index):
+//   LEVELS  histogram of the 65 score levels per row (thread-private counters);
+//   no bias -> threshold level F and r_F ties to keep;
+//   bias    -> band [fmaf(s_N,c,b_min), fmaf(s_max,c,b_max)]; RADIX passes over
+//              the order-preserving uint32 key of l (128 bins) narrow it until the
+//              threshold bin holds <= 64 keys; COLLECT ranks those exactly.
+//   Keys with l > F are kept; keys with l == F are kept in key order while the
+//   row's tie count is < r_F.
+// Every mbarrier wait is bounded in SM clocks; on expiry the CTA records a
+// device status bit, skips the rest of its work, and still frees its TMEM.
+#pragma once
+
+#include <climits>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace had {
+namespace tc {
+
+using namespace had::sm100;
+
+constexpr int kM = 128;            // query rows per CTA (TMEM lanes)
+constexpr int kN = 64;             // keys per tile (score MMA N)
+constexpr int kThreads = 192;
+constexpr int kKStages = 4;
+constexpr int kVStages = 2;
+constexpr int kLevels = 65;
+constexpr int kRadixBins = 128;
+constexpr int kCandCap = 64;
+constexpr uint32_t kColS = 0, kColP = 128, kColPlo = 160, kColO = 192, kTmemCols = 256;
+constexpr long long kWaitCycles = 2000000000LL;  // about one second
+
+enum { SEL_DENSE = 0, SEL_TOPN_INT = 1, SEL_TOPN_FLOAT = 2 };
+enum { MODE_F = 0, MODE_Q = 1 };
+enum { EXP_NONE = 0, EXP_IDX = 1, EXP_CODES = 2 };
+enum { P_DONE = 0, P_NORM, P_LEVELS, P_RADIX, P_COLLECT, P_KEPT_NORM, P_PV, P_IDX, P_CODES };
+
+struct TcArgs {
+  CUtensorMap tm_k;   // +-1 int8 K [BH*n_pad][64], box {64, 64}, 64B swizzle
+  CUtensorMap tm_v;   // V bf16 [BH*n][64], box {64, 64}, 128B swizzle          (float mode)
+  CUtensorMap tm_vq;  // int8 V^T [BH*64][n_pad], box {64, 64}, 64B swizzle      (uint8 mode)
+  CUtensorMap tm_vlo; // bf16 residual of fp32 V [BH*n][64], box {64, 64}         (fp32 V)
+  const uint32_t* qbits;   // [BH][n][2]
+  const float* vscale;     // [BH][64]
+  const float* table;      // [H][th][tw] or null
+  int gh, gw, prefix, th, tw;
+  const float* bminmax;    // [H][2]
+  const int32_t* seqlens;
+  void* O;
+  int o_bf16;
+  int32_t* idx;
+  uint8_t* codes;
+  int row_begin, row_end;
+  int B, H, n, n_pad, N;
+  unsigned* status;
+  float c_head[kMaxHeads];
+};
+
+// Shared memory carve-up (offsets from a 1024-byte aligned base).
+template <int SEL, bool VF32>
+struct Smem {
+  static constexpr int kVStage = (VF32 ? 2 : 1) * kN * kD * 2;   // bf16 V tile (+ residual tile)
+  static constexpr int kQ = 0;                                   // 128 x 64 B
+  static constexpr int kK = kQ + kM * kD;                        // 4 x 4 KB
+  static constexpr int kV = kK + kKStages * kN * kD;             // 2 V stages
+  static constexpr int kKoff = kV + kVStages * kVStage;          // 2 x 64 int
+  static constexpr int kDq = kKoff + 2 * kN * 4;                 // 64 fp32 dequant scales
+  static constexpr int kBar = kDq + kD * 4;
+  static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 7;
+  static constexpr int kMisc = kBar + kNumBars * 8;              // [0] tmem base [1] abort
+  static constexpr int kHist = (kMisc + 16 + 127) / 128 * 128;
+  static constexpr int kHistBytes = (SEL == SEL_DENSE) ? 0
+                                    : (SEL == SEL_TOPN_INT) ? kLevels * kM * 4
+                                    : kCandCap * kM * 8;
+  static constexpr int kTotal = kHist + kHistBytes + 1024;       // + alignment slack
+  static_assert(kCandCap * kM * 8 >= kRadixBins * kM * 4, "radix histogram fits the candidate area");
+  static_assert(kCandCap * kM * 8 >= kLevels * kM * 4, "level histogram fits the candidate area");
+};
+
+enum {
+  B_KFULL = 0,
+  B_KEMPTY = kKStages,
+  B_VFULL = 2 * kKStages,
+  B_VEMPTY = 2 * kKStages + kVStages,
+  B_SFULL = 2 * kKStages + 2 * kVStages,  // 2 (one per score buffer)
+  B_TDONE = B_SFULL + 2,                  // 2
+  B_PEMPTY = B_TDONE + 2,
+  B_OFULL,
+  B_FINAL
+};
+
+template <int SEL, int MODE, bool HAS_BIAS, bool VF32, int EXPORT>
+__global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__ TcArgs a) {
+  using SM = Smem<SEL, VF32>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  uint8_t* sm = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
+  uint8_t* sQ = sm + SM::kQ;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM::kBar);
+  uint32_t* misc = reinterpret_cast<uint32_t*>(sm + SM::kMisc);
+  volatile uint32_t* abort_flag = misc + 1;
+  int* koff_all = reinterpret_cast<int*>(sm + SM::kKoff);
+  float* dq = reinterpret_cast<float*>(sm + SM::kDq);
+  uint32_t* hist = reinterpret_cast<uint32_t*>(sm + SM::kHist);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
+  const int q0 = blockIdx.x * kM;
+  const int L = valid_len(a.seqlens, b, a.n, a.status);
+  const float c = a.c_head[h];
+  const int keff = (a.N == 0 || a.N >= L) ? L : a.N;
+  const int ntiles = (L + kN - 1) / kN;
+
+  // ---------------------------------------------------------------- tile past L: zeros, no TMEM
+  if (q0 >= L) {
+    if (EXPORT == EXP_NONE) {
+      for (int e = tid; e < kM * kD; e += kThreads) {
+        const int r = q0 + e / kD, ch = e % kD;
+        if (r < a.n) {
+          const size_t o = ((size_t)bh * a.n + r) * kD + ch;
+          if (a.o_bf16) reinterpret_cast<__nv_bfloat16*>(a.O)[o] = __float2bfloat16(0.0f);
+          else reinterpret_cast<float*>(a.O)[o] = 0.0f;
+        }
+      }
+    } else if (EXPORT == EXP_IDX) {
+      for (int e = tid; e < kM * a.N; e += kThreads) {
+        const int r = q0 + e / a.N;
+        if (r < a.n) a.idx[((size_t)bh * a.n + r) * a.N + e % a.N] = -1;
+      }
+    } else {
+      const int rows = a.row_end - a.row_begin;
+      for (int e = tid; e < kM * a.n; e += kThreads) {
+        const int r = q0 + e / a.n;
+        if (r >= a.row_begin && r < a.row_end && r < a.n)
+          a.codes[((size_t)bh * rows + (r - a.row_begin)) * a.n + e % a.n] = 0;
+      }
+    }
+    return;
+  }
+
+  // ---------------------------------------------------------------- setup
+  if (warp == 4) {
+    tmem_alloc(misc, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 5 && lane == 0) {
+    for (int s = 0; s < kKStages; ++s) { mbar_init(&bars[B_KFULL + s], 1); mbar_init(&bars[B_KEMPTY + s], 1); }
+    for (int s = 0; s < kVStages; ++s) { mbar_init(&bars[B_VFULL + s], 1); mbar_init(&bars[B_VEMPTY + s], 1); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&bars[B_SFULL + s], 1); mbar_init(&bars[B_TDONE + s], kM); }
+    mbar_init(&bars[B_PEMPTY], 1);
+    mbar_init(&bars[B_OFULL], 1);
+    mbar_init(&bars[B_FINAL], 1);
+    misc[1] = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&a.tm_k);
+    if (EXPORT == EXP_NONE) prefetch_tensormap(MODE == MODE_Q ? &a.tm_vq : &a.tm_v);
+  }
+  const int row = q0 + tid;  // softmax threads
+  const bool row_ok = tid < kM && row < L;
+  if (tid < kM) {
+    // Q~ row into the 64-byte swizzled K-major A operand (16-byte chunk c -> c ^ ((row >> 1) & 3))
+    uint32_t w0 = 0, w1 = 0;
+    if (row_ok) {
+      const uint2 w = __ldg(reinterpret_cast<const uint2*>(a.qbits + ((size_t)bh * a.n + row) * kW));
+      w0 = w.x; w1 = w.y;
+    }
+#pragma unroll
+    for (int cch = 0; cch < 4; ++cch) {
+      const uint32_t f = (cch < 2 ? w0 : w1) >> ((cch & 1) * 16);
+      uint4 v;
+      v.x = expand_nibble_pm1(f & 15u);
+      v.y = expand_nibble_pm1((f >> 4) & 15u);
+      v.z = expand_nibble_pm1((f >> 8) & 15u);
+      v.w = expand_nibble_pm1((f >> 12) & 15u);
+      *reinterpret_cast<uint4*>(sQ + tid * kD + ((cch ^ ((tid >> 1) & 3)) * 16)) = v;
+    }
+    if (SEL != SEL_DENSE)
+      for (int lev = 0; lev < kLevels; ++lev) hist[lev * kM + tid] = 0u;
+    if (MODE == MODE_Q && EXPORT == EXP_NONE && tid < kD) dq[tid] = __fdiv_rn(a.vscale[(size_t)bh * kD + tid], 255.0f);
+    fence_proxy_async();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc[0];
+
+  // ---------------------------------------------------------------- per-row state (softmax threads)
+  float F = -INFINITY, m = -INFINITY, scale = 1.0f, lsum = 0.0f;
+  int rF = 0, cut = 0, tie_seen = 0, kept_seen = 0;
+  uint32_t r_uhi = 0, r_span = 0;
+  int r_shift = 0, r_rank = 0, r_state = 0, r_bin = 0, r_cnt = 0;
+  int rb = -1;
+  if (HAS_BIAS && tid < kM && row >= a.prefix && row < a.n) {
+    const int t = row - a.prefix;
+    rb = (t / a.gw + a.gh - 1) * a.tw + (t % a.gw + a.gw - 1);
+  }
+  const float* tab = HAS_BIAS ? a.table + (size_t)h * a.th * a.tw : nullptr;
+  const float kLog2e = 1.4426950408889634f;
+
+  uint32_t g_k = 0, g_v = 0, g_s = 0, g_p = 0;  // tiles issued so far (all passes), per role
+  int k_par[kKStages], v_par[kVStages];          // producer: parity of the last load per stage (-1 none)
+#pragma unroll
+  for (int s2 = 0; s2 < kKStages; ++s2) k_par[s2] = -1;
+#pragma unroll
+  for (int s2 = 0; s2 < kVStages; ++s2) v_par[s2] = -1;
+
+  int pass = (SEL == SEL_DENSE) ? (EXPORT == EXP_IDX ? P_IDX : P_NORM) : P_LEVELS;
+
+  auto bounded_wait = [&](int bar, uint32_t parity) -> bool {
+    if (*abort_flag) return false;
+    if (mbar_wait(&bars[bar], parity, kWaitCycles)) return true;
+    *abort_flag = 1u;
+    raise_status(a.status, kDevErrTimeout);
+    return false;
+  };
+
+  while (pass != P_DONE) {
+    const bool pv = (pass == P_PV);
+    // ============================================================== producer (warp 5)
+    if (warp == 5) {
+      for (int t = 0; t < ntiles; ++t) {
+        const uint32_t st = g_k % kKStages;
+        if (g_k >= (uint32_t)kKStages) bounded_wait(B_KEMPTY + st, ((g_k / kKStages) - 1) & 1);
+        if (lane == 0 && !*abort_flag) {
+          mbar_arrive_expect_tx(&bars[B_KFULL + st], kN * kD);
+          tma_load_2d(sm + SM::kK + st * kN * kD, &a.tm_k, 0, bh * a.n_pad + t * kN, &bars[B_KFULL + st]);
+          k_par[st] = (int)((g_k / kKStages) & 1);
+        }
+        ++g_k;
+        if (pv) {
+          const uint32_t vs = g_v % kVStages;
+          if (g_v >= (uint32_t)kVStages) bounded_wait(B_VEMPTY + vs, ((g_v / kVStages) - 1) & 1);
+          if (lane == 0 && !*abort_flag) {
+            uint8_t* dst = sm + SM::kV + vs * SM::kVStage;
+            if (MODE == MODE_Q) {
+              mbar_arrive_expect_tx(&bars[B_VFULL + vs], kD * kN);
+              tma_load_2d(dst, &a.tm_vq, t * kN, bh * kD, &bars[B_VFULL + vs]);
+            } else {
+              mbar_arrive_expect_tx(&bars[B_VFULL + vs], SM::kVStage);
+              tma_load_2d(dst, &a.tm_v, 0, bh * a.n + t * kN, &bars[B_VFULL + vs]);
+              if (VF32) tma_load_2d(dst + kN * kD * 2, &a.tm_vlo, 0, bh * a.n + t * kN, &bars[B_VFULL + vs]);
+            }
+            v_par[vs] = (int)((g_v / kVStages) & 1);
+          }
+          ++g_v;
+        }
+      }
+    }
+    // ============================================================== MMA issuer (warp 4, lane 0)
+    else if (warp == 4) {
+      if (lane == 0) {
+        const uint32_t id_s = idesc_i8(kM, kN, true, true, false);
+        const uint32_t id_pv = (MODE == MODE_Q) ? idesc_i8(kM, kD, false, true, false) : idesc_bf16(kM, kD, true);
+        auto issue_scores = [&](int t) {
+          const uint32_t gk = g_k + (uint32_t)t, st = gk % kKStages, buf = (g_s + (uint32_t)t) & 1u;
+          if (!bounded_wait(B_KFULL + st, (gk / kKStages) & 1)) return;
+          tc_fence_after();
+          const uint32_t kq = smem_u32(sQ), kk = smem_u32(sm + SM::kK + st * kN * kD);
+#pragma unroll
+          for (int ks = 0; ks < 2; ++ks)
+            mma_i8_ss(tmem + kColS + buf * kN, sdesc(kq + 32 * ks, 16, 512, kSwizzle64B),
+                      sdesc(kk + 32 * ks, 16, 512, kSwizzle64B), id_s, ks > 0 ? 1u : 0u);
+          mma_commit(&bars[B_SFULL + buf]);
+          mma_commit(&bars[B_KEMPTY + st]);
+        };
+        issue_scores(0);
+        if (ntiles > 1) issue_scores(1);
+        for (int t = 0; t < ntiles; ++t) {
+          const uint32_t gs = g_s + (uint32_t)t, buf = gs & 1u;
+          bounded_wait(B_TDONE + buf, (gs >> 1) & 1);
+          tc_fence_after();
+          if (pv && !*abort_flag) {
+            const uint32_t gv = g_v + (uint32_t)t, vs = gv % kVStages;
+            if (bounded_wait(B_VFULL + vs, (gv / kVStages) & 1)) {
+              tc_fence_after();
+              const uint32_t vbase = smem_u32(sm + SM::kV + vs * SM::kVStage);
+              if (MODE == MODE_Q) {
+#pragma unroll
+                for (int k = 0; k < kN / 32; ++k)
+                  mma_i8_ts(tmem + kColO, tmem + kColP + 8 * k, sdesc(vbase + 32 * k, 16, 512, kSwizzle64B), id_pv,
+                            (t > 0 || k > 0) ? 1u : 0u);
+              } else {
+#pragma unroll
+                for (int k = 0; k < kN / 16; ++k)
+                  mma_f16_ts(tmem + kColO, tmem + kColP + 8 * k, sdesc(vbase + 2048 * k, 0, 1024, kSwizzle128B), id_pv,
+                             (t > 0 || k > 0) ? 1u : 0u);
+                if (VF32) {
+                  // residual products: P_hi x V_lo and P_lo x V_hi
+                  const uint32_t vlo = vbase + kN * kD * 2;
+#pragma unroll
+                  for (int k = 0; k < kN / 16; ++k)
+                    mma_f16_ts(tmem + kColO, tmem + kColP + 8 * k, sdesc(vlo + 2048 * k, 0, 1024, kSwizzle128B), id_pv,
+                               1u);
+#pragma unroll
+                  for (int k = 0; k < kN / 16; ++k)
+                    mma_f16_ts(tmem + kColO, tmem + kColPlo + 8 * k, sdesc(vbase + 2048 * k, 0, 1024, kSwizzle128B),
+                               id_pv, 1u);
+                }
+              }
+              mma_commit(&bars[B_PEMPTY]);
+              mma_commit(&bars[B_VEMPTY + vs]);
+              if (t + 1 == ntiles) mma_commit(&bars[B_OFULL]);
+            }
+          }
+          if (t + 2 < ntiles) issue_scores(t + 2);
+        }
+      }
+      g_k += ntiles;
+      g_s += ntiles;
+      if (pv) { g_v += ntiles; g_p += ntiles; }
+    }
+    // ============================================================== softmax / select (warps 0-3)
+    else {
+      const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+      const uint32_t hist_row = smem_u32(hist) + (uint32_t)tid * 4u;
+      const float mo = -m * kLog2e;
+      for (int t = 0; t < ntiles; ++t) {
+        const uint32_t gs = g_s + (uint32_t)t, buf = gs & 1u;
+        const int j0 = t * kN;
+        const int* ko = koff_all + (t & 1) * kN;
+        if (HAS_BIAS && pass != P_LEVELS) {
+          // bias offsets of this tile's keys, double-buffered by tile parity
+          if (tid < kN) {
+            const int j = j0 + tid;
+            int off = INT_MIN;
+            if (j >= a.prefix && j < a.n) { const int tt = j - a.prefix; off = (tt / a.gw) * a.tw + tt % a.gw; }
+            koff_all[(t & 1) * kN + tid] = off;
+          }
+          asm volatile("bar.sync 1, 128;" ::: "memory");
+        }
+        const bool ok_wait = __all_sync(0xffffffffu, bounded_wait(B_SFULL + buf, (gs >> 1) & 1));
+        tc_fence_after();
+        uint32_t r[64];
+        tmem_ld32(tl + kColS + buf * kN, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(tl + kColS + buf * kN + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        tmem_wait_ld();
+        const int nvalid = row_ok ? max(0, min(kN, L - j0)) : 0;
+        if (ok_wait) {
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            const int jb = j0 + 32 * ch;
+            // logits of the chunk; invalid keys get -inf
+            float lg[32];
+            if (pass != P_LEVELS) {
+#pragma unroll
+              for (int u = 0; u < 32; u += 4) {
+                int kk[4] = {0, 0, 0, 0};
+                if (HAS_BIAS) {
+                  const int4 k4 = *reinterpret_cast<const int4*>(ko + 32 * ch + u);
+                  kk[0] = k4.x; kk[1] = k4.y; kk[2] = k4.z; kk[3] = k4.w;
+                }
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                  const int s = (int)r[32 * ch + u + v];
+                  float l;
+                  if (HAS_BIAS) {
+                    const float bv = (rb >= 0 && kk[v] != INT_MIN) ? __ldg(tab + (rb - kk[v])) : 0.0f;
+                    l = __fmaf_rn((float)s, c, bv);
+                  } else {
+                    l = (float)s * c;
+                  }
+                  lg[u + v] = (32 * ch + u + v < nvalid) ? l : -INFINITY;
+                }
+              }
+            }
+            if (pass == P_LEVELS) {
+              const uint32_t base = hist_row + 32u * kM * 4u;  // level (64 - s)/2 -> + (64 - s) * 256 bytes
+#pragma unroll
+              for (int u = 0; u < 32; ++u) {
+                if (32 * ch + u < nvalid) {
+                  const uint32_t ad = base - (uint32_t)((int)r[32 * ch + u] * (kM * 2));
+                  asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(ad) : "memory");
+                }
+              }
+            } else if (pass == P_NORM) {
+              float tm = -INFINITY;
+#pragma unroll
+              for (int u = 0; u < 32; ++u) tm = fmaxf(tm, lg[u]);
+              if (tm > m) {
+                lsum *= fast_exp2((m - tm) * kLog2e);
+                m = tm;
+              }
+              const float mo2 = -m * kLog2e;
+#pragma unroll
+              for (int u = 0; u < 32; ++u) lsum += fast_exp2(__fmaf_rn(lg[u], kLog2e, mo2));
+            } else if (pass == P_RADIX) {
+              if (r_state == 1) {
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                  const uint32_t dd = r_uhi - float_order_key(lg[u]);
+                  if (32 * ch + u < nvalid && dd <= r_span) atomicAdd(&hist[(dd >> r_shift) * kM + tid], 1u);
+                }
+              }
+            } else if (pass == P_COLLECT) {
+              if (r_state == 2) {
+                uint2* cand = reinterpret_cast<uint2*>(hist);  // [64][128 rows]
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                  const uint32_t key = float_order_key(lg[u]);
+                  const uint32_t dd = r_uhi - key;
+                  if (32 * ch + u < nvalid && dd <= r_span && (int)(dd >> r_shift) == r_bin) {
+                    if (r_cnt < kCandCap) cand[r_cnt * kM + tid] = make_uint2(key, (uint32_t)(jb + u));
+                    ++r_cnt;
+                  }
+                }
+              }
+            } else {
+              // keep mask in key order; ties at F counted per row
+              uint32_t keepm = 0;
+#pragma unroll
+              for (int u = 0; u < 32; ++u) {
+                const bool valid = 32 * ch + u < nvalid;
+                bool k;
+                if (SEL == SEL_DENSE) {
+                  k = valid;
+                } else {
+                  const bool gt = valid && lg[u] > F, eq = valid && lg[u] == F;
+                  k = gt || (eq && (!cut || tie_seen < rF));
+                  tie_seen += eq ? 1 : 0;
+                }
+                keepm |= (k ? 1u : 0u) << u;
+              }
+              if (pass == P_KEPT_NORM) {
+#pragma unroll
+                for (int u = 0; u < 32; ++u)
+                  lsum += ((keepm >> u) & 1u) ? fast_exp2(__fmaf_rn(lg[u], kLog2e, mo)) : 0.0f;
+              } else if (pass == P_IDX) {
+                int32_t* dst = a.idx + ((size_t)bh * a.n + row) * a.N;
+#pragma unroll
+                for (int u = 0; u < 32; ++u)
+                  if ((keepm >> u) & 1u) { if (kept_seen < a.N) dst[kept_seen] = jb + u; ++kept_seen; }
+              } else {
+                float e[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                  const float x = fast_exp2(__fmaf_rn(lg[u], kLog2e, mo));
+                  e[u] = ((keepm >> u) & 1u) ? x : 0.0f;
+                }
+                if (pass == P_CODES || MODE == MODE_Q) {
+                  uint32_t wq[8];
+#pragma unroll
+                  for (int u = 0; u < 8; ++u) {
+                    uint32_t w = 0;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                      const uint32_t code = (uint32_t)min(255, (int)floorf(__fmaf_rn(e[4 * u + v], scale, 0.5f)));
+                      w |= code << (8 * v);
+                    }
+                    wq[u] = w;
+                  }
+                  if (pass == P_CODES) {
+                    if (row >= a.row_begin && row < a.row_end && row < a.n) {
+                      const int rows = a.row_end - a.row_begin;
+                      uint8_t* dst = a.codes + ((size_t)bh * rows + (row - a.row_begin)) * a.n;
+#pragma unroll
+                      for (int u = 0; u < 32; ++u)
+                        if (jb + u < a.n) dst[jb + u] = (uint8_t)((wq[u >> 2] >> (8 * (u & 3))) & 0xFFu);
+                    }
+                  } else {
+                    if (ch == 0 && t > 0) bounded_wait(B_PEMPTY, (g_p + (uint32_t)t - 1) & 1);
+                    tmem_st8(tl + kColP + 8 * ch, wq);
+                  }
+                } else {
+                  uint32_t wp[16];
+#pragma unroll
+                  for (int u = 0; u < 16; ++u) {
+                    wp[u] = pack_bf16x2(e[2 * u], e[2 * u + 1]);
+                    if (SEL == SEL_TOPN_FLOAT) lsum += e[2 * u] + e[2 * u + 1];
+                  }
+                  if (ch == 0 && t > 0) bounded_wait(B_PEMPTY, (g_p + (uint32_t)t - 1) & 1);
+                  tmem_st16(tl + kColP + 16 * ch, wp);
+                  if (VF32) {
+                    uint32_t wl[16];
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                      const float h0 = __uint_as_float(wp[u] << 16), h1 = __uint_as_float(wp[u] & 0xFFFF0000u);
+                      wl[u] = pack_bf16x2(e[2 * u] - h0, e[2 * u + 1] - h1);
+                    }
+                    tmem_st16(tl + kColPlo + 16 * ch, wl);
+                  }
+                }
+              }
+            }
+          }
+        }
+        if (pv) tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&bars[B_TDONE + buf]);
+      }
+      g_k += ntiles;
+      g_s += ntiles;
+      if (pv) { g_v += ntiles; g_p += ntiles; }
+    }
+
+    // ============================================================== per-row decisions after the pass
+    if (tid < kM && row_ok && !*abort_flag) {
+      if (pass == P_LEVELS) {
+        int cnt[kLevels];
+#pragma unroll
+        for (int lev = 0; lev < kLevels; ++lev) cnt[lev] = (int)hist[lev * kM + tid];
+        int hmin = 64, hN = 64, cum = 0;
+        bool found = false;
+#pragma unroll
+        for (int lev = kLevels - 1; lev >= 0; --lev) hmin = cnt[lev] > 0 ? lev : hmin;
+#pragma unroll
+        for (int lev = 0; lev < kLevels; ++lev) {
+          cum += cnt[lev];
+          if (!found && cum >= keff) { hN = lev; found = true; }
+        }
+        const int smax = 64 - 2 * hmin, sN = 64 - 2 * hN;
+        if (SEL == SEL_TOPN_INT) {
+          F = (float)sN * c;
+          m = (float)smax * c;
+          int gt = 0, eq = 0;
+          float ls = 0.0f;
+#pragma unroll
+          for (int lev = 0; lev < kLevels; ++lev) {
+            const float lv = (float)(64 - 2 * lev) * c;
+            gt += (lv > F) ? cnt[lev] : 0;
+            eq += (lv == F) ? cnt[lev] : 0;
+            ls += (lv > F) ? (float)cnt[lev] * fast_exp2((lv - m) * kLog2e) : 0.0f;
+          }
+          rF = keff - gt;
+          cut = rF < eq ? 1 : 0;
+          ls += (float)rF * fast_exp2((F - m) * kLog2e);
+          scale = (MODE == MODE_Q || EXPORT == EXP_CODES) ? 255.0f / ls : 1.0f / ls;
+        } else {
+          const float bmin = a.bminmax[2 * h], bmax = a.bminmax[2 * h + 1];
+          const float lo = __fmaf_rn((float)sN, c, bmin);
+          const float hi = __fmaf_rn((float)smax, c, bmax);
+          r_uhi = float_order_key(hi);
+          r_span = r_uhi - float_order_key(lo);
+          r_shift = 0;
+          while ((r_span >> r_shift) >= (uint32_t)kRadixBins) ++r_shift;
+          r_rank = keff;
+          r_state = 1;
+          m = hi;
+        }
+      } else if (pass == P_RADIX && r_state == 1) {
+        int cum = 0, bsel = kRadixBins - 1, kbin = 0;
+        for (int bb = 0; bb < kRadixBins; ++bb) {
+          const int k = (int)hist[bb * kM + tid];
+          if (cum + k >= r_rank) { bsel = bb; kbin = k; break; }
+          cum += k;
+        }
+        const int rank = r_rank - cum;
+        const uint32_t uhi = r_uhi - ((uint32_t)bsel << r_shift);
+        if (r_shift == 0) {
+          const uint32_t bits = (uhi & 0x80000000u) ? (uhi & 0x7FFFFFFFu) : ~uhi;
+          F = __uint_as_float(bits);
+          rF = rank;
+          cut = rank < kbin ? 1 : 0;
+          r_state = 0;
+        } else if (kbin <= kCandCap) {
+          r_bin = bsel;
+          r_rank = rank;
+          r_state = 2;
+          r_cnt = 0;
+        } else {
+          const uint32_t span_left = r_span - ((uint32_t)bsel << r_shift);
+          r_uhi = uhi;
+          r_span = min(((uint32_t)1 << r_shift) - 1u, span_left);
+          r_shift = r_shift > 7 ? r_shift - 7 : 0;
+          r_rank = rank;
+        }
+      } else if (pass == P_COLLECT && r_state == 2) {
+        const uint2* cand = reinterpret_cast<const uint2*>(hist);
+        const int nc = min(r_cnt, kCandCap);
+        if (r_cnt > kCandCap) raise_status(a.status, kDevErrCapacity);
+        uint32_t uF = 0u;
+        for (int x = 0; x < nc; ++x) {
+          const uint2 cx = cand[x * kM + tid];
+          int before = 0;
+          for (int y = 0; y < nc; ++y) {
+            const uint2 cy = cand[y * kM + tid];
+            before += (cy.x > cx.x || (cy.x == cx.x && cy.y < cx.y)) ? 1 : 0;
+          }
+          if (before == r_rank - 1) uF = cx.x;
+        }
+        int gt = 0, eq = 0;
+        for (int x = 0; x < nc; ++x) {
+          const uint32_t ux = cand[x * kM + tid].x;
+          gt += ux > uF ? 1 : 0;
+          eq += ux == uF ? 1 : 0;
+        }
+        const uint32_t bits = (uF & 0x80000000u) ? (uF & 0x7FFFFFFFu) : ~uF;
+        F = __uint_as_float(bits);
+        rF = r_rank - gt;
+        cut = rF < eq ? 1 : 0;
+        r_state = 0;
+      } else if (pass == P_KEPT_NORM) {
+        scale = 255.0f / lsum;
+      } else if (pass == P_NORM) {
+        scale = (MODE == MODE_Q || EXPORT == EXP_CODES) ? 255.0f / lsum : 1.0f / lsum;
+      }
+    }
+    tie_seen = 0;
+    // ---- the CTA chooses the next pass
+    const int any_refine = __syncthreads_or(tid < kM && r_state == 1);
+    const int any_collect = __syncthreads_or(tid < kM && r_state == 2);
+    int next;
+    if (*abort_flag) next = P_DONE;
+    else if (pass == P_IDX || pass == P_CODES || pass == P_PV) next = P_DONE;
+    else if (pass == P_NORM) next = (EXPORT == EXP_CODES) ? P_CODES : P_PV;
+    else if (any_refine) next = P_RADIX;
+    else if (any_collect) next = P_COLLECT;
+    else if (EXPORT == EXP_IDX) next = P_IDX;
+    else if ((EXPORT == EXP_CODES || MODE == MODE_Q) && SEL == SEL_TOPN_FLOAT && pass != P_KEPT_NORM) next = P_KEPT_NORM;
+    else if (EXPORT == EXP_CODES) next = P_CODES;
+    else next = P_PV;
+    if (next == P_RADIX && tid < kM)
+      for (int bb = 0; bb < kRadixBins; ++bb) hist[bb * kM + tid] = 0u;
+    if (next == P_KEPT_NORM && tid < kM) lsum = 0.0f;
+    __syncthreads();
+    pass = next;
+  }
+
+  // ---------------------------------------------------------------- epilogue
+  if (EXPORT == EXP_NONE) {
+    if (tid < kM) {
+      const bool ok = __all_sync(0xffffffffu, bounded_wait(B_OFULL, 0));
+      tc_fence_after();
+      const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
+      uint32_t o[64];
+      tmem_ld32(tl + kColO, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+      tmem_ld32(tl + kColO + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+      tmem_wait_ld();
+      if (row < a.n) {
+        float out[64];
+        if (!ok || !row_ok) {
+#pragma unroll
+          for (int k = 0; k < 64; ++k) out[k] = 0.0f;
+        } else if (MODE == MODE_Q) {
+#pragma unroll
+          for (int k = 0; k < 64; ++k) out[k] = (float)(int)o[k] * dq[k];
+        } else {
+          const float inv = (SEL == SEL_TOPN_FLOAT) ? 1.0f / lsum : scale;
+#pragma unroll
+          for (int k = 0; k < 64; ++k) out[k] = __uint_as_float(o[k]) * inv;
+        }
+        const size_t ob = ((size_t)bh * a.n + row) * kD;
+        if (a.o_bf16) {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.O) + ob);
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            dst[k] = make_uint4(pack_bf16x2(out[8 * k], out[8 * k + 1]), pack_bf16x2(out[8 * k + 2], out[8 * k + 3]),
+                                pack_bf16x2(out[8 * k + 4], out[8 * k + 5]), pack_bf16x2(out[8 * k + 6], out[8 * k + 7]));
+        } else {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.O) + ob);
+#pragma unroll
+          for (int k = 0; k < 16; ++k) dst[k] = make_float4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
+        }
+      }
+    }
+  } else if (EXPORT == EXP_IDX) {
+    if (tid < kM && row < a.n) {
+      int32_t* dst = a.idx + ((size_t)bh * a.n + row) * a.N;
+      for (int p = row_ok ? min(kept_seen, a.N) : 0; p < a.N; ++p) dst[p] = -1;
+    }
+  } else {
+    if (tid < kM && row >= a.row_begin && row < a.row_end && row < a.n) {
+      const int rows = a.row_end - a.row_begin;
+      uint8_t* dst = a.codes + ((size_t)bh * rows + (row - a.row_begin)) * a.n;
+      for (int j = row_ok ? ntiles * kN : 0; j < a.n; ++j) dst[j] = 0;
+    }
+  }
+
+  // ---------------------------------------------------------------- teardown
+  if (warp == 5 && lane == 0 && *abort_flag) {
+    // let TMA loads still in flight land before the CTA's shared memory goes away
+    for (int s2 = 0; s2 < kKStages; ++s2)
+      if (k_par[s2] >= 0) mbar_wait(&bars[B_KFULL + s2], (uint32_t)k_par[s2], 200000000LL);
+    for (int s2 = 0; s2 < kVStages; ++s2)
+      if (v_par[s2] >= 0) mbar_wait(&bars[B_VFULL + s2], (uint32_t)v_par[s2], 200000000LL);
+  }
+  if (warp == 4 && lane == 0) {
+    // every tcgen05 operation this thread issued is complete before TMEM is freed
+    mma_commit(&bars[B_FINAL]);
+    mbar_wait(&bars[B_FINAL], 0, 200000000LL);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace tc
+}  // namespace had

@@ -22,12 +22,20 @@
 #include "prep.cuh"
 #include "attn.cuh"
 #include "dense_ref.cuh"
+#include "attn_tc.cuh"
 
 namespace had {
 
 __device__ unsigned g_device_status;
 
 namespace {
+
+using tc::SEL_DENSE;
+using tc::SEL_TOPN_INT;
+using tc::SEL_TOPN_FLOAT;
+using tc::EXP_NONE;
+using tc::EXP_IDX;
+using tc::EXP_CODES;
 
 constexpr int kMaxDevices = 64;
 thread_local char t_last_error[256] = "";
@@ -88,7 +96,7 @@ had_status check_bias(const had_shape* s, const had_relpos_bias* bias) {
 }
 
 struct Ws {
-  size_t qbits, kpm, sums, amax, vqT, vscale, bminmax, total;
+  size_t qbits, kpm, sums, amax, vqT, vscale, bminmax, vhi, vlo, total;
 };
 
 Ws ws_layout(const had_shape* s, bool quant, bool bias) {
@@ -105,8 +113,61 @@ Ws ws_layout(const had_shape* s, bool quant, bool bias) {
     w.vscale = off; off += align_up((size_t)d.BH * kD * 4);
   }
   if (bias) { w.bminmax = off; off += align_up((size_t)s->H * 2 * 4); }
+  w.vhi = w.vlo = 0;
+  if (!quant && s->in_dtype == HAD_F32) {
+    // fp32 V in float mode: bf16 head and residual copies for the tensor cores
+    w.vhi = off; off += align_up((size_t)d.BH * d.n * kD * 2);
+    w.vlo = off; off += align_up((size_t)d.BH * d.n * kD * 2);
+  }
   w.total = off;
   return w;
+}
+
+__global__ void k_split_v(const float* __restrict__ V, size_t count, __nv_bfloat16* __restrict__ hi,
+                          __nv_bfloat16* __restrict__ lo) {
+  for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < count; e += (size_t)gridDim.x * blockDim.x) {
+    const float v = V[e];
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    hi[e] = h;
+    lo[e] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+// ---------------------------------------------------------------------------- TMA descriptors
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [outer][inner] of `dt`, tile box {box_in, box_out}.
+had_status encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
+                     uint64_t row_bytes, uint32_t box_in, uint32_t box_out, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cuda_fail(cudaErrorNotSupported, "cuTensorMapEncodeTiled unavailable");
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_in, box_out};
+  const cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    snprintf(t_last_error, sizeof(t_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    return HAD_ERR_CUDA;
+  }
+  return HAD_OK;
 }
 
 __global__ void k_bias_minmax(const float* table, int th, int tw, int prefix, float* out) {
@@ -178,59 +239,6 @@ had_status launch_prep(const had_shape* s, const void* X0, const void* X1, const
 
 // ---------------------------------------------------------------------------- attention launches
 
-template <int SEL, int MODE, bool BIAS, bool VF32, int EXP>
-had_status launch_attn_t(const AttnArgs& a, dim3 grid, cudaStream_t st) {
-  using SL = SmemLayout<MODE, VF32>;
-  const int smem = (SEL == SEL_DENSE) ? SL::kTotalDense : SL::kTotalTopN;
-  auto fn = k_attn<SEL, MODE, BIAS, VF32, EXP>;
-  static std::mutex mu;
-  static bool configured[kMaxDevices] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    if (dev >= 0 && dev < kMaxDevices && !configured[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_attn)");
-      configured[dev] = true;
-    }
-  }
-  fn<<<grid, kAttnThreads, smem, st>>>(a);
-  return check_launch("k_attn");
-}
-
-template <int EXP>
-had_status dispatch_attn(int sel, int mode, bool bias, bool vf32, const AttnArgs& a, dim3 grid, cudaStream_t st) {
-  if (EXP == EXP_NONE) {
-    if (mode == MODE_Q) {
-      if (sel == SEL_DENSE) return bias ? launch_attn_t<SEL_DENSE, MODE_Q, true, false, EXP>(a, grid, st)
-                                        : launch_attn_t<SEL_DENSE, MODE_Q, false, false, EXP>(a, grid, st);
-      if (sel == SEL_TOPN_INT) return launch_attn_t<SEL_TOPN_INT, MODE_Q, false, false, EXP>(a, grid, st);
-      return launch_attn_t<SEL_TOPN_FLOAT, MODE_Q, true, false, EXP>(a, grid, st);
-    }
-    if (vf32) {
-      if (sel == SEL_DENSE) return bias ? launch_attn_t<SEL_DENSE, MODE_F, true, true, EXP>(a, grid, st)
-                                        : launch_attn_t<SEL_DENSE, MODE_F, false, true, EXP>(a, grid, st);
-      if (sel == SEL_TOPN_INT) return launch_attn_t<SEL_TOPN_INT, MODE_F, false, true, EXP>(a, grid, st);
-      return launch_attn_t<SEL_TOPN_FLOAT, MODE_F, true, true, EXP>(a, grid, st);
-    }
-    if (sel == SEL_DENSE) return bias ? launch_attn_t<SEL_DENSE, MODE_F, true, false, EXP>(a, grid, st)
-                                      : launch_attn_t<SEL_DENSE, MODE_F, false, false, EXP>(a, grid, st);
-    if (sel == SEL_TOPN_INT) return launch_attn_t<SEL_TOPN_INT, MODE_F, false, false, EXP>(a, grid, st);
-    return launch_attn_t<SEL_TOPN_FLOAT, MODE_F, true, false, EXP>(a, grid, st);
-  } else if (EXP == EXP_IDX) {
-    if (sel == SEL_DENSE) return bias ? launch_attn_t<SEL_DENSE, MODE_F, true, false, EXP>(a, grid, st)
-                                      : launch_attn_t<SEL_DENSE, MODE_F, false, false, EXP>(a, grid, st);
-    if (sel == SEL_TOPN_INT) return launch_attn_t<SEL_TOPN_INT, MODE_F, false, false, EXP>(a, grid, st);
-    return launch_attn_t<SEL_TOPN_FLOAT, MODE_F, true, false, EXP>(a, grid, st);
-  } else {
-    if (sel == SEL_DENSE) return bias ? launch_attn_t<SEL_DENSE, MODE_Q, true, false, EXP>(a, grid, st)
-                                      : launch_attn_t<SEL_DENSE, MODE_Q, false, false, EXP>(a, grid, st);
-    if (sel == SEL_TOPN_INT) return launch_attn_t<SEL_TOPN_INT, MODE_Q, false, false, EXP>(a, grid, st);
-    return launch_attn_t<SEL_TOPN_FLOAT, MODE_Q, true, false, EXP>(a, grid, st);
-  }
-}
-
 // Host-side validation shared by the attention entry points.
 template <int EXP>
 had_status validate_attention(const void* Q, const void* K, const void* V, const had_shape* s,
@@ -283,12 +291,68 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
   had_status r = launch_prep(s, Q, K, V, 0, do_v ? 3 : 2, sums, amax, nullptr, nullptr, qbits, nullptr, nullptr,
                              kpm, vqT, vscale, st, status);
   if (r != HAD_OK) return r;
+  if (!quant && s->in_dtype == HAD_F32 && need_v) {
+    const size_t count = (size_t)dims_of(s).BH * s->n * kD;
+    k_split_v<<<1024, 256, 0, st>>>(static_cast<const float*>(V), count,
+                                     reinterpret_cast<__nv_bfloat16*>(ws + w.vhi),
+                                     reinterpret_cast<__nv_bfloat16*>(ws + w.vlo));
+    if ((r = check_launch("k_split_v")) != HAD_OK) return r;
+  }
   if (select_kind(s, bias, N) == SEL_TOPN_FLOAT) {
     float* bmm = reinterpret_cast<float*>(ws + w.bminmax);
     k_bias_minmax<<<s->H, 256, 0, st>>>(bias->table, 2 * bias->gh - 1, 2 * bias->gw - 1, bias->prefix, bmm);
     if ((r = check_launch("k_bias_minmax")) != HAD_OK) return r;
   }
   return HAD_OK;
+}
+
+template <int SEL, int MODE, bool BIAS, bool VF32, int EXP>
+had_status launch_tc_t(const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
+  const int smem = tc::Smem<SEL, VF32>::kTotal;
+  auto fn = tc::k_attn_tc<SEL, MODE, BIAS, VF32, EXP>;
+  static std::mutex mu;
+  static bool configured[kMaxDevices] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  {
+    std::lock_guard<std::mutex> lk(mu);
+    if (dev >= 0 && dev < kMaxDevices && !configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_attn_tc)");
+      configured[dev] = true;
+    }
+  }
+  fn<<<grid, tc::kThreads, smem, st>>>(a);
+  return check_launch("k_attn_tc");
+}
+
+template <int SEL, int MODE, bool VF32, int EXP>
+had_status launch_tc_b(bool bias, const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
+  return bias ? launch_tc_t<SEL, MODE, true, VF32, EXP>(a, grid, st) : launch_tc_t<SEL, MODE, false, VF32, EXP>(a, grid, st);
+}
+
+template <int EXP>
+had_status dispatch_tc(int sel, int mode, bool bias, bool vf32, const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
+  using namespace tc;
+  if (EXP == EXP_CODES || (EXP == EXP_NONE && mode == MODE_Q)) {
+    constexpr int E = EXP;
+    if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_Q, false, E>(bias, a, grid, st);
+    if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_Q, false, false, E>(a, grid, st);
+    return launch_tc_t<SEL_TOPN_FLOAT, MODE_Q, true, false, E>(a, grid, st);
+  }
+  if (EXP == EXP_IDX) {
+    if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, false, EXP>(bias, a, grid, st);
+    if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, false, false, EXP>(a, grid, st);
+    return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, true, false, EXP>(a, grid, st);
+  }
+  if (vf32) {
+    if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, true, EXP>(bias, a, grid, st);
+    if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, false, true, EXP>(a, grid, st);
+    return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, true, true, EXP>(a, grid, st);
+  }
+  if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, false, EXP>(bias, a, grid, st);
+  if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, false, false, EXP>(a, grid, st);
+  return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, true, false, EXP>(a, grid, st);
 }
 
 // Stage 2: the fused kernel over a prepared workspace.
@@ -302,11 +366,29 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
   const Ws w = ws_layout(s, quant, has_bias);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   Dims d = dims_of(s);
-  AttnArgs a{};
+  const bool vf32 = (s->in_dtype == HAD_F32) && !quant;
+  tc::TcArgs a;
+  memset(&a, 0, sizeof(a));
+  had_status r = encode_2d(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.kpm, kD, (uint64_t)d.BH * d.n_pad, kD, kD,
+                           tc::kN, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (r != HAD_OK) return r;
+  const bool needs_v = (EXP == EXP_NONE);
+  if (needs_v && quant) {
+    r = encode_2d(&a.tm_vq, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.vqT, d.n_pad, (uint64_t)d.BH * kD, d.n_pad, tc::kN,
+                  kD, CU_TENSOR_MAP_SWIZZLE_64B);
+    if (r != HAD_OK) return r;
+  } else if (needs_v) {
+    const void* vb = vf32 ? static_cast<const void*>(ws + w.vhi) : V;
+    r = encode_2d(&a.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, vb, kD, (uint64_t)d.BH * d.n, kD * 2, kD, tc::kN,
+                  CU_TENSOR_MAP_SWIZZLE_128B);
+    if (r != HAD_OK) return r;
+    if (vf32) {
+      r = encode_2d(&a.tm_vlo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + w.vlo, kD, (uint64_t)d.BH * d.n, kD * 2, kD,
+                    tc::kN, CU_TENSOR_MAP_SWIZZLE_128B);
+      if (r != HAD_OK) return r;
+    }
+  }
   a.qbits = reinterpret_cast<uint32_t*>(ws + w.qbits);
-  a.kpm = reinterpret_cast<int8_t*>(ws + w.kpm);
-  a.V = V;
-  a.vqT = quant ? reinterpret_cast<int8_t*>(ws + w.vqT) : nullptr;
   a.vscale = quant ? reinterpret_cast<float*>(ws + w.vscale) : nullptr;
   a.table = has_bias ? bias->table : nullptr;
   if (has_bias) {
@@ -323,9 +405,8 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
     const double aq = alpha_q ? (double)alpha_q[h] : 1.0, ak = alpha_k ? (double)alpha_k[h] : 1.0;
     a.c_head[h] = (float)(aq * ak / std::sqrt((double)s->d));
   }
-  dim3 grid((s->n + kQT - 1) / kQT, d.BH);
-  const bool vf32 = (s->in_dtype == HAD_F32) && !quant;
-  return dispatch_attn<EXP>(select_kind(s, bias, N), quant ? MODE_Q : MODE_F, has_bias, vf32, a, grid, st);
+  dim3 grid((s->n + tc::kM - 1) / tc::kM, d.BH);
+  return dispatch_tc<EXP>(select_kind(s, bias, N), quant ? tc::MODE_Q : tc::MODE_F, has_bias, vf32, a, grid, st);
 }
 
 had_status device_status_ptr(unsigned** out) {
@@ -519,7 +600,7 @@ had_status had_scores_int(const uint32_t* qbits, const uint32_t* kbits, const ha
   if (!status) return cuda_fail(cudaErrorInvalidSymbol, "status word");
   Dims d = dims_of(s);
   dim3 grid((s->n + kQT - 1) / kQT, d.BH);
-  k_scores_int<MODE_Q><<<grid, kAttnThreads, 0, static_cast<cudaStream_t>(stream)>>>(qbits, kbits, s->H, s->n,
+  k_scores_int<KMAP_U8><<<grid, kAttnThreads, 0, static_cast<cudaStream_t>(stream)>>>(qbits, kbits, s->H, s->n,
                                                                                       s->seqlens, S, status);
   return check_launch("k_scores_int");
 }
