@@ -60,6 +60,21 @@ def _peaks():
         "fallback"
 
 
+HEAD_STAGE_BYTES = 128 * 1024  # heads up to this size are prepared by one kernel from shared memory
+
+
+def launches_per_step(n: int, elem: int, mode: str, has_bias: bool) -> int:
+    """Kernels one prepare + attend step launches: the sign/pack stage (one
+    kernel for short heads, statistics + pack otherwise), the hi/lo split of an
+    fp32 V (float mode), the two bias-table kernels, and the fused attention."""
+    k = 1 if n * 64 * elem <= HEAD_STAGE_BYTES else 2
+    if mode == "float" and elem == 4:
+        k += 1
+    if has_bias:
+        k += 2
+    return k + 1
+
+
 def kernel_bytes_per_token(mode: str, v_bytes: int, o_bytes: int) -> int:
     """Algorithmic bytes per valid token of the fused kernel (k_attn).
 
@@ -264,9 +279,7 @@ def run_gpu(args, rank, world, local_rank):
         if st:
             raise had.HadError(st, "had_attention_prepared")
 
-    kernels_per_step = 3 if (N == 0 or N >= w.n or bias is None) else 4
-    if mode == "float" and not (N == 0 or N >= w.n) and bias is None:
-        kernels_per_step = 3
+    kernels_per_step = launches_per_step(w.n, Q.element_size(), mode, bias is not None)
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
             prepare()

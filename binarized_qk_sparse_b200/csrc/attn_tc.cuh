@@ -32,6 +32,7 @@
 #pragma once
 
 #include <climits>
+#include <type_traits>
 
 #include "common.cuh"
 #include "sm100.cuh"
@@ -51,6 +52,11 @@ constexpr int kRadixBins = 128;
 constexpr int kCandCap = 64;
 constexpr uint32_t kColS = 0, kColP = 128, kColPlo = 160, kColO = 192, kTmemCols = 256;
 constexpr long long kWaitCycles = 2000000000LL;  // about one second
+// How the softmax threads find the bias offset koff(j) = y_j * tw + x_j of a key:
+constexpr int kKoffTable = 0;    // per-head table in shared memory (n_pad <= kKoffTableMax)
+constexpr int kKoffLinear = 1;   // prefix 0 and gw a multiple of 64: koff(j0 + u) = koff(j0) + u within a tile
+constexpr int kKoffTile = 2;     // computed per tile (double-buffered, one named barrier per tile)
+constexpr int kKoffTableMax = 1024;
 
 enum { SEL_DENSE = 0, SEL_TOPN_INT = 1, SEL_TOPN_FLOAT = 2 };
 enum { MODE_F = 0, MODE_Q = 1 };
@@ -66,7 +72,10 @@ struct TcArgs {
   const float* vscale;     // [BH][64]
   const float* table;      // [H][th][tw] or null
   int gh, gw, prefix, th, tw;
-  const float* bminmax;    // [H][2]
+  const float* bminmax;    // [H][2] min/max of each head's table (0 included with class tokens)
+  const float* expb;       // [H][th][tw] exp(b - b_max(h)), or null
+  int int_levels;          // 1 if fp32(c*s) is strictly increasing in s for every head
+  int koff_mode;           // kKoffTable / kKoffLinear / kKoffTile
   const int32_t* seqlens;
   void* O;
   int o_bf16;
@@ -79,19 +88,19 @@ struct TcArgs {
 };
 
 // Shared memory carve-up (offsets from a 1024-byte aligned base).
-template <int SEL, bool VF32>
+template <int SEL, bool VF32, bool HAS_BIAS>
 struct Smem {
   static constexpr int kVStage = (VF32 ? 2 : 1) * kN * kD * 2;   // bf16 V tile (+ residual tile)
   static constexpr int kQ = 0;                                   // 128 x 64 B
   static constexpr int kK = kQ + kM * kD;                        // 4 x 4 KB
   static constexpr int kV = kK + kKStages * kN * kD;             // 2 V stages
-  static constexpr int kKoff = kV + kVStages * kVStage;          // 2 x 64 int
-  static constexpr int kDq = kKoff + 2 * kN * 4;                 // 64 fp32 dequant scales
+  static constexpr int kKoff = kV + kVStages * kVStage;          // bias key offsets (table or 2 x 64)
+  static constexpr int kDq = kKoff + (HAS_BIAS ? kKoffTableMax * 4 : 0);  // 64 fp32 dequant scales
   static constexpr int kBar = kDq + kD * 4;
   static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 7;
   static constexpr int kMisc = kBar + kNumBars * 8;              // [0] tmem base [1] abort
   static constexpr int kHist = (kMisc + 16 + 127) / 128 * 128;
-  static constexpr int kHistBytes = (SEL == SEL_DENSE) ? 0
+  static constexpr int kHistBytes = (SEL == SEL_DENSE) ? kLevels * 32 * 4
                                     : (SEL == SEL_TOPN_INT) ? kLevels * kM * 4
                                     : kCandCap * kM * 8;
   static constexpr int kTotal = kHist + kHistBytes + 1024;       // + alignment slack
@@ -111,9 +120,23 @@ enum {
   B_FINAL
 };
 
+// Ties at the threshold are kept in key order while fewer than r_F have been
+// kept: of this chunk's tie bits `eqm` (bit u = key jb + u), keep the first
+// r_F - tie_seen (all of them when the row needs no cut).
+__device__ __forceinline__ uint32_t tie_keep(uint32_t eqm, int cut, int rF, int& tie_seen) {
+  uint32_t keep = eqm;
+  if (cut && eqm != 0u) {
+    const int allow = rF - tie_seen, cnt = __popc(eqm);
+    if (allow <= 0) keep = 0u;
+    else if (allow < cnt) keep = eqm & ((2u << __fns(eqm, 0u, allow)) - 1u);
+  }
+  tie_seen += __popc(eqm);
+  return keep;
+}
+
 template <int SEL, int MODE, bool HAS_BIAS, bool VF32, int EXPORT>
 __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__ TcArgs a) {
-  using SM = Smem<SEL, VF32>;
+  using SM = Smem<SEL, VF32, HAS_BIAS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -121,7 +144,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + SM::kBar);
   uint32_t* misc = reinterpret_cast<uint32_t*>(sm + SM::kMisc);
   volatile uint32_t* abort_flag = misc + 1;
-  int* koff_all = reinterpret_cast<int*>(sm + SM::kKoff);
+  int* koff_tab = reinterpret_cast<int*>(sm + SM::kKoff);
   float* dq = reinterpret_cast<float*>(sm + SM::kDq);
   uint32_t* hist = reinterpret_cast<uint32_t*>(sm + SM::kHist);
 
@@ -198,7 +221,20 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
     }
     if (SEL != SEL_DENSE)
       for (int lev = 0; lev < kLevels; ++lev) hist[lev * kM + tid] = 0u;
+    if (SEL == SEL_DENSE && tid < 32) {
+      // per-lane copy of the level table exp(c * (s - 64)), level k = (64 - s) / 2
+      const float ck = -2.0f * a.c_head[h] * 1.4426950408889634f;
+      float* lt = reinterpret_cast<float*>(hist);
+      for (int lev = 0; lev < kLevels; ++lev) lt[lev * 32 + tid] = exp2f(ck * (float)lev);
+    }
     if (MODE == MODE_Q && EXPORT == EXP_NONE && tid < kD) dq[tid] = __fdiv_rn(a.vscale[(size_t)bh * kD + tid], 255.0f);
+    if (HAS_BIAS && a.koff_mode == kKoffTable) {
+      for (int j = tid; j < a.n_pad; j += kM) {
+        int off = INT_MIN;
+        if (j >= a.prefix && j < a.n) { const int tt = j - a.prefix; off = (tt / a.gw) * a.tw + tt % a.gw; }
+        koff_tab[j] = off;
+      }
+    }
     fence_proxy_async();
   }
   tc_fence_before();
@@ -218,6 +254,17 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
   }
   const float* tab = HAS_BIAS ? a.table + (size_t)h * a.th * a.tw : nullptr;
   const float kLog2e = 1.4426950408889634f;
+  // Dense weights as (level table) x exp(b - b_max): both factors <= 1, so no row
+  // maximum is needed as long as the smallest product stays far from fp32 underflow.
+  float fb0 = 1.0f;  // factor of a class-token pair (bias 0)
+  bool use_lut = false;
+  if (SEL == SEL_DENSE) {
+    const float range = HAS_BIAS ? a.bminmax[2 * h + 1] - a.bminmax[2 * h] : 0.0f;
+    use_lut = c > 0.0f && (128.0f * c + range) * kLog2e <= 100.0f;
+    if (HAS_BIAS) fb0 = exp2f(-a.bminmax[2 * h + 1] * kLog2e);
+  }
+  const bool sum_in_pv = (MODE == MODE_F) && (SEL == SEL_TOPN_FLOAT || (SEL == SEL_DENSE && use_lut));
+  int sF = 0;  // integer threshold score (top-N without bias)
 
   uint32_t g_k = 0, g_v = 0, g_s = 0, g_p = 0;  // tiles issued so far (all passes), per role
   int k_par[kKStages], v_par[kVStages];          // producer: parity of the last load per stage (-1 none)
@@ -227,6 +274,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
   for (int s2 = 0; s2 < kVStages; ++s2) v_par[s2] = -1;
 
   int pass = (SEL == SEL_DENSE) ? (EXPORT == EXP_IDX ? P_IDX : P_NORM) : P_LEVELS;
+  if (SEL == SEL_DENSE && EXPORT == EXP_NONE && MODE == MODE_F && use_lut) pass = P_PV;
 
   auto bounded_wait = [&](int bar, uint32_t parity) -> bool {
     if (*abort_flag) return false;
@@ -242,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
     if (warp == 5) {
       for (int t = 0; t < ntiles; ++t) {
         const uint32_t st = g_k % kKStages;
-        if (g_k >= (uint32_t)kKStages) bounded_wait(B_KEMPTY + st, ((g_k / kKStages) - 1) & 1);
+        if (lane == 0 && g_k >= (uint32_t)kKStages) bounded_wait(B_KEMPTY + st, ((g_k / kKStages) - 1) & 1);
         if (lane == 0 && !*abort_flag) {
           mbar_arrive_expect_tx(&bars[B_KFULL + st], kN * kD);
           tma_load_2d(sm + SM::kK + st * kN * kD, &a.tm_k, 0, bh * a.n_pad + t * kN, &bars[B_KFULL + st]);
@@ -251,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
         ++g_k;
         if (pv) {
           const uint32_t vs = g_v % kVStages;
-          if (g_v >= (uint32_t)kVStages) bounded_wait(B_VEMPTY + vs, ((g_v / kVStages) - 1) & 1);
+          if (lane == 0 && g_v >= (uint32_t)kVStages) bounded_wait(B_VEMPTY + vs, ((g_v / kVStages) - 1) & 1);
           if (lane == 0 && !*abort_flag) {
             uint8_t* dst = sm + SM::kV + vs * SM::kVStage;
             if (MODE == MODE_Q) {
@@ -336,65 +384,118 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
       const uint32_t hist_row = smem_u32(hist) + (uint32_t)tid * 4u;
       const float mo = -m * kLog2e;
+      const float* lut = reinterpret_cast<const float*>(hist);
+      // lut_e: dense weights from the level table x exp(bias - b_max) (no row max needed)
+      // lut_w: top-N (no bias) weights from the row's level table, zero below the threshold
+      const bool lut_e = (SEL == SEL_DENSE) && use_lut && (pass == P_NORM || pass == P_PV || pass == P_CODES);
+      const bool lut_w = (SEL == SEL_TOPN_INT) && a.int_levels && pass == P_PV;
+      const bool wants_bias = HAS_BIAS && pass != P_LEVELS;
+      const float* expb_h = HAS_BIAS ? a.expb + (size_t)h * a.th * a.tw : nullptr;
       for (int t = 0; t < ntiles; ++t) {
         const uint32_t gs = g_s + (uint32_t)t, buf = gs & 1u;
         const int j0 = t * kN;
-        const int* ko = koff_all + (t & 1) * kN;
-        if (HAS_BIAS && pass != P_LEVELS) {
-          // bias offsets of this tile's keys, double-buffered by tile parity
-          if (tid < kN) {
-            const int j = j0 + tid;
-            int off = INT_MIN;
-            if (j >= a.prefix && j < a.n) { const int tt = j - a.prefix; off = (tt / a.gw) * a.tw + tt % a.gw; }
-            koff_all[(t & 1) * kN + tid] = off;
+        // bias offsets of this tile's keys: per-head table, closed form, or computed per tile
+        const int* ko = koff_tab + j0;
+        int lin_base = 0;
+        if (wants_bias) {
+          if (a.koff_mode == kKoffLinear) {
+            lin_base = (j0 / a.gw) * a.tw + j0 % a.gw;
+          } else if (a.koff_mode == kKoffTile) {
+            ko = koff_tab + buf * kN;  // alternates across passes too
+            if (tid < kN) {
+              const int j = j0 + tid;
+              int off = INT_MIN;
+              if (j >= a.prefix && j < a.n) { const int tt = j - a.prefix; off = (tt / a.gw) * a.tw + tt % a.gw; }
+              koff_tab[buf * kN + tid] = off;
+            }
+            asm volatile("bar.sync 1, 128;" ::: "memory");
           }
-          asm volatile("bar.sync 1, 128;" ::: "memory");
         }
         const bool ok_wait = __all_sync(0xffffffffu, bounded_wait(B_SFULL + buf, (gs >> 1) & 1));
         tc_fence_after();
-        uint32_t r[64];
-        tmem_ld32(tl + kColS + buf * kN, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(tl + kColS + buf * kN + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
-        tmem_wait_ld();
         const int nvalid = row_ok ? max(0, min(kN, L - j0)) : 0;
-        if (ok_wait) {
+        // both 32-column halves of the tile are loaded at once; the loop body
+        // (one copy of the code per pass) then runs on r and moves rn into r
+        uint32_t r[32], rn[32];
+        tmem_ld32(tl + kColS + buf * kN, r);
+        tmem_ld32(tl + kColS + buf * kN + 32, rn);
+        tmem_wait_ld();
+#pragma unroll 1
+        for (int ch = 0; ch < 2; ++ch) {
+          if (ch == 1) {
 #pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
-            const int jb = j0 + 32 * ch;
-            // logits of the chunk; invalid keys get -inf
-            float lg[32];
-            if (pass != P_LEVELS) {
+            for (int u = 0; u < 32; ++u) r[u] = rn[u];
+          }
+          if (!ok_wait) continue;
+          const int jb = j0 + 32 * ch;
+          const int nv = min(32, max(0, nvalid - 32 * ch));
+          const uint32_t vmask = nv >= 32 ? 0xFFFFFFFFu : ((1u << nv) - 1u);
+          auto bias_index = [&](int u, bool& has) -> int {
+            int kk = (a.koff_mode == kKoffLinear) ? lin_base + 32 * ch + u : ko[32 * ch + u];
+            has = rb >= 0 && kk != INT_MIN;
+            return rb - kk;
+          };
+          float e[32];
+          bool have_e = false;
+          if (SEL != SEL_DENSE && pass == P_LEVELS) {
+            const uint32_t base = hist_row + 32u * kM * 4u;  // level (64 - s)/2 -> + (64 - s) * 256 bytes
 #pragma unroll
-              for (int u = 0; u < 32; u += 4) {
-                int kk[4] = {0, 0, 0, 0};
-                if (HAS_BIAS) {
-                  const int4 k4 = *reinterpret_cast<const int4*>(ko + 32 * ch + u);
-                  kk[0] = k4.x; kk[1] = k4.y; kk[2] = k4.z; kk[3] = k4.w;
-                }
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                  const int s = (int)r[32 * ch + u + v];
-                  float l;
-                  if (HAS_BIAS) {
-                    const float bv = (rb >= 0 && kk[v] != INT_MIN) ? __ldg(tab + (rb - kk[v])) : 0.0f;
-                    l = __fmaf_rn((float)s, c, bv);
-                  } else {
-                    l = (float)s * c;
-                  }
-                  lg[u + v] = (32 * ch + u + v < nvalid) ? l : -INFINITY;
-                }
-              }
+            for (int u = 0; u < 32; ++u) {
+              // predicated inside the asm, so a ragged tile costs no branches
+              const uint32_t ad = base - (uint32_t)((int)r[u] * (kM * 2));
+              asm volatile(
+                  "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t@p red.shared.add.u32 [%0], 1;\n\t}" ::"r"(ad),
+                  "r"((vmask >> u) & 1u)
+                  : "memory");
             }
-            if (pass == P_LEVELS) {
-              const uint32_t base = hist_row + 32u * kM * 4u;  // level (64 - s)/2 -> + (64 - s) * 256 bytes
+          } else if (SEL == SEL_DENSE && lut_e) {
 #pragma unroll
-              for (int u = 0; u < 32; ++u) {
-                if (32 * ch + u < nvalid) {
-                  const uint32_t ad = base - (uint32_t)((int)r[32 * ch + u] * (kM * 2));
-                  asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(ad) : "memory");
-                }
+            for (int u = 0; u < 32; ++u) {
+              const int sc = (int)r[u];
+              float x = lut[(32 - (sc >> 1)) * 32 + lane];
+              if (HAS_BIAS) {
+                bool has;
+                const int bi = bias_index(u, has);
+                x *= has ? __ldg(expb_h + bi) : fb0;
               }
-            } else if (pass == P_NORM) {
+              e[u] = ((vmask >> u) & 1u) ? x : 0.0f;
+            }
+            if (pass == P_NORM) {
+#pragma unroll
+              for (int u = 0; u < 32; ++u) lsum += e[u];
+            } else {
+              have_e = true;
+            }
+          } else if (SEL == SEL_TOPN_INT && lut_w) {
+            uint32_t eqm = 0;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+              const int sc = (int)r[u];
+              e[u] = lut[(32 - (sc >> 1)) * kM + tid];
+              eqm |= (sc == sF ? 1u : 0u) << u;
+            }
+            eqm &= vmask;
+            const uint32_t keepm = vmask & ~(eqm & ~tie_keep(eqm, cut, rF, tie_seen));
+#pragma unroll
+            for (int u = 0; u < 32; ++u) e[u] = ((keepm >> u) & 1u) ? e[u] : 0.0f;
+            have_e = true;
+          } else {
+            // generic path: exact logits (invalid keys -inf)
+            float lg[32];
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+              const int sc = (int)r[u];
+              float l;
+              if (HAS_BIAS) {
+                bool has;
+                const int bi = bias_index(u, has);
+                l = __fmaf_rn((float)sc, c, has ? __ldg(tab + bi) : 0.0f);
+              } else {
+                l = (float)sc * c;
+              }
+              lg[u] = ((vmask >> u) & 1u) ? l : -INFINITY;
+            }
+            if (SEL == SEL_DENSE && pass == P_NORM) {
               float tm = -INFINITY;
 #pragma unroll
               for (int u = 0; u < 32; ++u) tm = fmaxf(tm, lg[u]);
@@ -405,22 +506,22 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
               const float mo2 = -m * kLog2e;
 #pragma unroll
               for (int u = 0; u < 32; ++u) lsum += fast_exp2(__fmaf_rn(lg[u], kLog2e, mo2));
-            } else if (pass == P_RADIX) {
+            } else if (SEL == SEL_TOPN_FLOAT && pass == P_RADIX) {
               if (r_state == 1) {
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
                   const uint32_t dd = r_uhi - float_order_key(lg[u]);
-                  if (32 * ch + u < nvalid && dd <= r_span) atomicAdd(&hist[(dd >> r_shift) * kM + tid], 1u);
+                  if (((vmask >> u) & 1u) && dd <= r_span) atomicAdd(&hist[(dd >> r_shift) * kM + tid], 1u);
                 }
               }
-            } else if (pass == P_COLLECT) {
+            } else if (SEL == SEL_TOPN_FLOAT && pass == P_COLLECT) {
               if (r_state == 2) {
                 uint2* cand = reinterpret_cast<uint2*>(hist);  // [64][128 rows]
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
                   const uint32_t key = float_order_key(lg[u]);
                   const uint32_t dd = r_uhi - key;
-                  if (32 * ch + u < nvalid && dd <= r_span && (int)(dd >> r_shift) == r_bin) {
+                  if (((vmask >> u) & 1u) && dd <= r_span && (int)(dd >> r_shift) == r_bin) {
                     if (r_cnt < kCandCap) cand[r_cnt * kM + tid] = make_uint2(key, (uint32_t)(jb + u));
                     ++r_cnt;
                   }
@@ -428,79 +529,80 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
               }
             } else {
               // keep mask in key order; ties at F counted per row
-              uint32_t keepm = 0;
+              uint32_t keepm = vmask;
+              if (SEL != SEL_DENSE) {
+                uint32_t gtm = 0, eqm = 0;
 #pragma unroll
-              for (int u = 0; u < 32; ++u) {
-                const bool valid = 32 * ch + u < nvalid;
-                bool k;
-                if (SEL == SEL_DENSE) {
-                  k = valid;
-                } else {
-                  const bool gt = valid && lg[u] > F, eq = valid && lg[u] == F;
-                  k = gt || (eq && (!cut || tie_seen < rF));
-                  tie_seen += eq ? 1 : 0;
+                for (int u = 0; u < 32; ++u) {
+                  gtm |= (lg[u] > F ? 1u : 0u) << u;
+                  eqm |= (lg[u] == F ? 1u : 0u) << u;
                 }
-                keepm |= (k ? 1u : 0u) << u;
+                keepm = (gtm & vmask) | tie_keep(eqm & vmask, cut, rF, tie_seen);
               }
-              if (pass == P_KEPT_NORM) {
+              if (SEL == SEL_TOPN_FLOAT && (MODE == MODE_Q || EXPORT == EXP_CODES) && pass == P_KEPT_NORM) {
 #pragma unroll
                 for (int u = 0; u < 32; ++u)
                   lsum += ((keepm >> u) & 1u) ? fast_exp2(__fmaf_rn(lg[u], kLog2e, mo)) : 0.0f;
-              } else if (pass == P_IDX) {
-                int32_t* dst = a.idx + ((size_t)bh * a.n + row) * a.N;
+              } else if (EXPORT == EXP_IDX && pass == P_IDX) {
+                if (row_ok) {
+                  int32_t* dst = a.idx + ((size_t)bh * a.n + row) * a.N;
 #pragma unroll
-                for (int u = 0; u < 32; ++u)
-                  if ((keepm >> u) & 1u) { if (kept_seen < a.N) dst[kept_seen] = jb + u; ++kept_seen; }
+                  for (int u = 0; u < 32; ++u)
+                    if ((keepm >> u) & 1u) { if (kept_seen < a.N) dst[kept_seen] = jb + u; ++kept_seen; }
+                }
               } else {
-                float e[32];
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
                   const float x = fast_exp2(__fmaf_rn(lg[u], kLog2e, mo));
                   e[u] = ((keepm >> u) & 1u) ? x : 0.0f;
                 }
-                if (pass == P_CODES || MODE == MODE_Q) {
-                  uint32_t wq[8];
+                have_e = true;
+              }
+            }
+          }
+          // ---- P (or uint8 A) of the chunk into TMEM, or codes to global (export)
+          if (have_e) {
+            if ((EXPORT == EXP_CODES && pass == P_CODES) || (EXPORT == EXP_NONE && MODE == MODE_Q)) {
+              uint32_t wq[8];
 #pragma unroll
-                  for (int u = 0; u < 8; ++u) {
-                    uint32_t w = 0;
+              for (int u = 0; u < 8; ++u) {
+                uint32_t w = 0;
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                      const uint32_t code = (uint32_t)min(255, (int)floorf(__fmaf_rn(e[4 * u + v], scale, 0.5f)));
-                      w |= code << (8 * v);
-                    }
-                    wq[u] = w;
-                  }
-                  if (pass == P_CODES) {
-                    if (row >= a.row_begin && row < a.row_end && row < a.n) {
-                      const int rows = a.row_end - a.row_begin;
-                      uint8_t* dst = a.codes + ((size_t)bh * rows + (row - a.row_begin)) * a.n;
-#pragma unroll
-                      for (int u = 0; u < 32; ++u)
-                        if (jb + u < a.n) dst[jb + u] = (uint8_t)((wq[u >> 2] >> (8 * (u & 3))) & 0xFFu);
-                    }
-                  } else {
-                    if (ch == 0 && t > 0) bounded_wait(B_PEMPTY, (g_p + (uint32_t)t - 1) & 1);
-                    tmem_st8(tl + kColP + 8 * ch, wq);
-                  }
-                } else {
-                  uint32_t wp[16];
-#pragma unroll
-                  for (int u = 0; u < 16; ++u) {
-                    wp[u] = pack_bf16x2(e[2 * u], e[2 * u + 1]);
-                    if (SEL == SEL_TOPN_FLOAT) lsum += e[2 * u] + e[2 * u + 1];
-                  }
-                  if (ch == 0 && t > 0) bounded_wait(B_PEMPTY, (g_p + (uint32_t)t - 1) & 1);
-                  tmem_st16(tl + kColP + 16 * ch, wp);
-                  if (VF32) {
-                    uint32_t wl[16];
-#pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                      const float h0 = __uint_as_float(wp[u] << 16), h1 = __uint_as_float(wp[u] & 0xFFFF0000u);
-                      wl[u] = pack_bf16x2(e[2 * u] - h0, e[2 * u + 1] - h1);
-                    }
-                    tmem_st16(tl + kColPlo + 16 * ch, wl);
-                  }
+                for (int v = 0; v < 4; ++v) {
+                  const uint32_t code = (uint32_t)min(255, (int)floorf(__fmaf_rn(e[4 * u + v], scale, 0.5f)));
+                  w |= code << (8 * v);
                 }
+                wq[u] = w;
+              }
+              if (EXPORT == EXP_CODES) {
+                if (row >= a.row_begin && row < a.row_end && row < a.n) {
+                  const int rows = a.row_end - a.row_begin;
+                  uint8_t* dst = a.codes + ((size_t)bh * rows + (row - a.row_begin)) * a.n;
+#pragma unroll
+                  for (int u = 0; u < 32; ++u)
+                    if (jb + u < a.n) dst[jb + u] = (uint8_t)((wq[u >> 2] >> (8 * (u & 3))) & 0xFFu);
+                }
+              } else {
+                if (ch == 0 && t > 0) bounded_wait(B_PEMPTY, (g_p + (uint32_t)t - 1) & 1);
+                tmem_st8(tl + kColP + 8 * ch, wq);
+              }
+            } else if (EXPORT == EXP_NONE) {
+              uint32_t wp[16];
+#pragma unroll
+              for (int u = 0; u < 16; ++u) {
+                wp[u] = pack_bf16x2(e[2 * u], e[2 * u + 1]);
+                if (sum_in_pv) lsum += e[2 * u] + e[2 * u + 1];
+              }
+              if (ch == 0 && t > 0) bounded_wait(B_PEMPTY, (g_p + (uint32_t)t - 1) & 1);
+              tmem_st16(tl + kColP + 16 * ch, wp);
+              if (VF32) {
+                uint32_t wl[16];
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                  const float h0 = __uint_as_float(wp[u] << 16), h1 = __uint_as_float(wp[u] & 0xFFFF0000u);
+                  wl[u] = pack_bf16x2(e[2 * u] - h0, e[2 * u + 1] - h1);
+                }
+                tmem_st16(tl + kColPlo + 16 * ch, wl);
               }
             }
           }
@@ -546,6 +648,14 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
           cut = rF < eq ? 1 : 0;
           ls += (float)rF * fast_exp2((F - m) * kLog2e);
           scale = (MODE == MODE_Q || EXPORT == EXP_CODES) ? 255.0f / ls : 1.0f / ls;
+          sF = sN;
+          // this row's weight per level: exp(l - m) above the threshold, the tie weight at it, 0 below
+          float* wt = reinterpret_cast<float*>(hist);
+#pragma unroll
+          for (int lev = 0; lev < kLevels; ++lev) {
+            const float lv = (float)(64 - 2 * lev) * c;
+            wt[lev * kM + tid] = (lv >= F) ? fast_exp2((lv - m) * kLog2e) : 0.0f;
+          }
         } else {
           const float bmin = a.bminmax[2 * h], bmax = a.bminmax[2 * h + 1];
           const float lo = __fmaf_rn((float)sN, c, bmin);
@@ -656,7 +766,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
 #pragma unroll
           for (int k = 0; k < 64; ++k) out[k] = (float)(int)o[k] * dq[k];
         } else {
-          const float inv = (SEL == SEL_TOPN_FLOAT) ? 1.0f / lsum : scale;
+          const float inv = sum_in_pv ? 1.0f / lsum : scale;
 #pragma unroll
           for (int k = 0; k < 64; ++k) out[k] = __uint_as_float(o[k]) * inv;
         }

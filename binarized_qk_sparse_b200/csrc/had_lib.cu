@@ -96,10 +96,11 @@ had_status check_bias(const had_shape* s, const had_relpos_bias* bias) {
 }
 
 struct Ws {
-  size_t qbits, kpm, sums, amax, vqT, vscale, bminmax, vhi, vlo, total;
+  size_t qbits, kpm, sums, amax, vqT, vscale, bminmax, expb, vhi, vlo, total;
 };
 
-Ws ws_layout(const had_shape* s, bool quant, bool bias) {
+Ws ws_layout(const had_shape* s, bool quant, const had_relpos_bias* bias_desc) {
+  const bool bias = bias_desc && bias_desc->table;
   Dims d = dims_of(s);
   Ws w{};
   size_t off = 0;
@@ -112,7 +113,12 @@ Ws ws_layout(const had_shape* s, bool quant, bool bias) {
     w.vqT = off; off += align_up((size_t)d.BH * kD * d.n_pad);
     w.vscale = off; off += align_up((size_t)d.BH * kD * 4);
   }
-  if (bias) { w.bminmax = off; off += align_up((size_t)s->H * 2 * 4); }
+  w.expb = 0;
+  if (bias) {
+    w.bminmax = off; off += align_up((size_t)s->H * 2 * 4);
+    const size_t cells = (size_t)(2 * bias_desc->gh - 1) * (size_t)(2 * bias_desc->gw - 1);
+    w.expb = off; off += align_up((size_t)s->H * cells * 4);
+  }
   w.vhi = w.vlo = 0;
   if (!quant && s->in_dtype == HAD_F32) {
     // fp32 V in float mode: bf16 head and residual copies for the tensor cores
@@ -190,6 +196,14 @@ __global__ void k_bias_minmax(const float* table, int th, int tw, int prefix, fl
   }
 }
 
+// exp(b - b_max(h)) of every table cell, the bias factor of the dense weights.
+__global__ void k_bias_exp(const float* table, int cells, const float* bminmax, float* out) {
+  const int h = blockIdx.y;
+  const float bmax = bminmax[2 * h + 1];
+  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < cells; e += gridDim.x * blockDim.x)
+    out[(size_t)h * cells + e] = exp2f((table[(size_t)h * cells + e] - bmax) * 1.4426950408889634f);
+}
+
 __global__ void k_untranspose_vq(const int8_t* vqT, int BH, int n, int n_pad, const int32_t* seqlens, int H,
                                  int8_t* Vq) {
   const size_t total = (size_t)BH * n * kD;
@@ -263,7 +277,7 @@ had_status validate_attention(const void* Q, const void* K, const void* V, const
     if (!(alpha_q[h] > 0.0f) || !std::isfinite(alpha_q[h])) return HAD_ERR_INVALID;
   for (int h = 0; alpha_k && h < s->H; ++h)
     if (!(alpha_k[h] > 0.0f) || !std::isfinite(alpha_k[h])) return HAD_ERR_INVALID;
-  const Ws w = ws_layout(s, mode == HAD_MODE_U8I8, bias && bias->table);
+  const Ws w = ws_layout(s, mode == HAD_MODE_U8I8, bias);
   if (!workspace || ws_bytes < w.total || !aligned16(workspace)) return HAD_ERR_INVALID;
   return HAD_OK;
 }
@@ -279,7 +293,7 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
                          cudaStream_t st, unsigned* status) {
   const bool has_bias = bias && bias->table;
   const bool quant = (mode == HAD_MODE_U8I8);
-  const Ws w = ws_layout(s, quant, has_bias);
+  const Ws w = ws_layout(s, quant, bias);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* qbits = reinterpret_cast<uint32_t*>(ws + w.qbits);
   int8_t* kpm = reinterpret_cast<int8_t*>(ws + w.kpm);
@@ -288,9 +302,43 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
   int8_t* vqT = quant ? reinterpret_cast<int8_t*>(ws + w.vqT) : nullptr;
   float* vscale = quant ? reinterpret_cast<float*>(ws + w.vscale) : nullptr;
   const bool do_v = quant && need_v;
-  had_status r = launch_prep(s, Q, K, V, 0, do_v ? 3 : 2, sums, amax, nullptr, nullptr, qbits, nullptr, nullptr,
-                             kpm, vqT, vscale, st, status);
-  if (r != HAD_OK) return r;
+  had_status r = HAD_OK;
+  const size_t elem = (s->in_dtype == HAD_BF16) ? 2 : 4;
+  const size_t head_bytes = (size_t)s->n * kD * elem;
+  if (head_bytes <= (size_t)kHeadMaxBytes) {
+    // short heads: one read of each head, statistics and packing from shared memory
+    HeadArgs ha{};
+    ha.X[0] = Q; ha.X[1] = K; ha.X[2] = V;
+    ha.first_tensor = 0;
+    ha.B = s->B; ha.H = s->H; ha.n = s->n; ha.n_pad = dims_of(s).n_pad;
+    ha.seqlens = s->seqlens;
+    ha.qbits = qbits; ha.kpm = kpm; ha.vqT = vqT; ha.vscale = vscale; ha.status = status;
+    dim3 grid(dims_of(s).BH, do_v ? 3 : 2);
+    const int smem = (int)head_bytes;
+    int dev = 0;
+    cudaGetDevice(&dev);
+    static std::mutex mu;
+    static bool attr_set[2][kMaxDevices] = {{false}};
+    const int which = (s->in_dtype == HAD_BF16) ? 0 : 1;
+    {
+      std::lock_guard<std::mutex> lk(mu);
+      if (dev >= 0 && dev < kMaxDevices && !attr_set[which][dev]) {
+        cudaError_t e = which == 0 ? cudaFuncSetAttribute(k_prep_head<__nv_bfloat16>,
+                                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kHeadMaxBytes)
+                                   : cudaFuncSetAttribute(k_prep_head<float>,
+                                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kHeadMaxBytes);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_prep_head)");
+        attr_set[which][dev] = true;
+      }
+    }
+    if (which == 0) k_prep_head<__nv_bfloat16><<<grid, kHeadThreads, smem, st>>>(ha);
+    else k_prep_head<float><<<grid, kHeadThreads, smem, st>>>(ha);
+    if ((r = check_launch("k_prep_head")) != HAD_OK) return r;
+  } else {
+    r = launch_prep(s, Q, K, V, 0, do_v ? 3 : 2, sums, amax, nullptr, nullptr, qbits, nullptr, nullptr, kpm, vqT,
+                    vscale, st, status);
+    if (r != HAD_OK) return r;
+  }
   if (!quant && s->in_dtype == HAD_F32 && need_v) {
     const size_t count = (size_t)dims_of(s).BH * s->n * kD;
     k_split_v<<<1024, 256, 0, st>>>(static_cast<const float*>(V), count,
@@ -298,17 +346,21 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
                                      reinterpret_cast<__nv_bfloat16*>(ws + w.vlo));
     if ((r = check_launch("k_split_v")) != HAD_OK) return r;
   }
-  if (select_kind(s, bias, N) == SEL_TOPN_FLOAT) {
+  if (has_bias) {
     float* bmm = reinterpret_cast<float*>(ws + w.bminmax);
-    k_bias_minmax<<<s->H, 256, 0, st>>>(bias->table, 2 * bias->gh - 1, 2 * bias->gw - 1, bias->prefix, bmm);
+    const int th = 2 * bias->gh - 1, tw = 2 * bias->gw - 1;
+    k_bias_minmax<<<s->H, 256, 0, st>>>(bias->table, th, tw, bias->prefix, bmm);
     if ((r = check_launch("k_bias_minmax")) != HAD_OK) return r;
+    k_bias_exp<<<dim3((th * tw + 255) / 256, s->H), 256, 0, st>>>(bias->table, th * tw, bmm,
+                                                                 reinterpret_cast<float*>(ws + w.expb));
+    if ((r = check_launch("k_bias_exp")) != HAD_OK) return r;
   }
   return HAD_OK;
 }
 
 template <int SEL, int MODE, bool BIAS, bool VF32, int EXP>
 had_status launch_tc_t(const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
-  const int smem = tc::Smem<SEL, VF32>::kTotal;
+  const int smem = tc::Smem<SEL, VF32, BIAS>::kTotal;
   auto fn = tc::k_attn_tc<SEL, MODE, BIAS, VF32, EXP>;
   static std::mutex mu;
   static bool configured[kMaxDevices] = {false};
@@ -363,7 +415,7 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
                         unsigned* status) {
   const bool has_bias = bias && bias->table;
   const bool quant = (mode == HAD_MODE_U8I8);
-  const Ws w = ws_layout(s, quant, has_bias);
+  const Ws w = ws_layout(s, quant, bias);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   Dims d = dims_of(s);
   const bool vf32 = (s->in_dtype == HAD_F32) && !quant;
@@ -396,14 +448,29 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
     a.th = 2 * bias->gh - 1; a.tw = 2 * bias->gw - 1;
   }
   a.bminmax = has_bias ? reinterpret_cast<float*>(ws + w.bminmax) : nullptr;
+  a.expb = has_bias ? reinterpret_cast<float*>(ws + w.expb) : nullptr;
   a.seqlens = s->seqlens;
   a.O = O; a.o_bf16 = (o_dtype == HAD_BF16) ? 1 : 0;
   a.idx = idx; a.codes = codes; a.row_begin = row_begin; a.row_end = row_end;
   a.B = d.B; a.H = d.H; a.n = d.n; a.n_pad = d.n_pad; a.N = N;
   a.status = status;
+  a.koff_mode = tc::kKoffTile;
+  if (has_bias) {
+    if (d.n_pad <= tc::kKoffTableMax) a.koff_mode = tc::kKoffTable;
+    else if (bias->prefix == 0 && bias->gw % tc::kN == 0) a.koff_mode = tc::kKoffLinear;
+  }
+  a.int_levels = 1;
   for (int h = 0; h < s->H; ++h) {
     const double aq = alpha_q ? (double)alpha_q[h] : 1.0, ak = alpha_k ? (double)alpha_k[h] : 1.0;
-    a.c_head[h] = (float)(aq * ak / std::sqrt((double)s->d));
+    const float c = (float)(aq * ak / std::sqrt((double)s->d));
+    a.c_head[h] = c;
+    // the 65 score levels must map to 65 distinct fp32 logits for the integer tie test
+    volatile float prev = -INFINITY;
+    for (int sc = -64; sc <= 64; sc += 2) {
+      volatile float lv = (float)sc * c;
+      if (!(lv > prev) || !std::isfinite(lv)) a.int_levels = 0;
+      prev = lv;
+    }
   }
   dim3 grid((s->n + tc::kM - 1) / tc::kM, d.BH);
   return dispatch_tc<EXP>(select_kind(s, bias, N), quant ? tc::MODE_Q : tc::MODE_F, has_bias, vf32, a, grid, st);
@@ -469,8 +536,8 @@ had_status had_binarize_pack(const void* X, const had_shape* s, const float* mu_
 
 size_t had_attention_workspace_size(const had_shape* s, int N, had_mode mode, const had_relpos_bias* bias) {
   (void)N;
-  if (check_shape(s) != HAD_OK) return 0;
-  return ws_layout(s, mode == HAD_MODE_U8I8, bias && bias->table).total;
+  if (check_shape(s) != HAD_OK || check_bias(s, bias) != HAD_OK) return 0;
+  return ws_layout(s, mode == HAD_MODE_U8I8, bias).total;
 }
 
 had_status had_attention(const void* Q, const void* K, const void* V, const had_shape* s,
@@ -523,7 +590,7 @@ had_status had_quantize_v(const void* V, const had_shape* s, int8_t* Vq, float* 
   had_status r = check_shape(s);
   if (r != HAD_OK) return r;
   if (!V || !Vq || !vscale || !aligned16(V) || (reinterpret_cast<uintptr_t>(vscale) & 3u)) return HAD_ERR_INVALID;
-  const Ws w = ws_layout(s, true, false);
+  const Ws w = ws_layout(s, true, nullptr);
   if (!workspace || ws_bytes < w.total || !aligned16(workspace)) return HAD_ERR_INVALID;
   int dev = 0;
   cudaError_t ce = cudaGetDevice(&dev);

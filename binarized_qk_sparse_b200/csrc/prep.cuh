@@ -215,3 +215,121 @@ __global__ void __launch_bounds__(kPrepThreads) k_pack(const PackArgs a) {
 }
 
 }  // namespace had
+
+namespace had {
+
+// ---------------------------------------------------------------------------- one-pass prep for short heads
+//
+// k_prep_head: one CTA per (batch*head, tensor) when the head's valid tokens fit
+// in shared memory.  The head is read from HBM once (16-byte cp.async chunks),
+// then from shared memory: channel sums in fp64 (Q, K) or channel absmax (V),
+// the mean (or scale), and the packed outputs -- Q sign bits, K as +-1 int8
+// rows, V as int8 V^T.  Same definitions as k_stats + k_pack.
+
+constexpr int kHeadThreads = 256;
+constexpr int kHeadMaxBytes = 128 * 1024;   // staged head: n * 64 * sizeof(T)
+
+struct HeadArgs {
+  const void* X[3];
+  int first_tensor;
+  int B, H, n, n_pad;
+  const int32_t* seqlens;
+  uint32_t* qbits;     // tensor 0 -> [BH][n][2]
+  int8_t* kpm;         // tensor 1 -> [BH][n_pad][64]
+  int8_t* vqT;         // tensor 2 -> [BH][64][n_pad]
+  float* vscale;       // [BH][64]
+  unsigned* status;
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kHeadThreads) k_prep_head(const HeadArgs a) {
+  extern __shared__ __align__(16) uint8_t xs[];      // [L][64] of T
+  __shared__ double part[4][kD];
+  __shared__ float stat[kD];
+  const int bh = blockIdx.x, tz = a.first_tensor + blockIdx.y, b = bh / a.H;
+  const int L = valid_len(a.seqlens, b, a.n, a.status);
+  const int tid = threadIdx.x;
+  constexpr int kRow = kD * (int)sizeof(T);          // bytes per token
+  const uint8_t* src = static_cast<const uint8_t*>(a.X[tz]) + (size_t)bh * a.n * kRow;
+  for (int e = tid; e < L * (kRow / 16); e += kHeadThreads) {
+    uint32_t d = (uint32_t)__cvta_generic_to_shared(xs + e * 16);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src + (size_t)e * 16));
+  }
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+  __syncthreads();
+  auto x_at = [&](int i, int ch) -> float {
+    if (sizeof(T) == 2) return __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(xs)[i * kD + ch] << 16);
+    return reinterpret_cast<const float*>(xs)[i * kD + ch];
+  };
+  // ---- channel statistic: thread (g, c) covers tokens i = g, g+4, ...
+  {
+    const int ch = tid & (kD - 1), g = tid >> 6;
+    if (tz < 2) {
+      double acc = 0.0;
+      for (int i = g; i < L; i += 4) acc += (double)x_at(i, ch);
+      part[g][ch] = acc;
+    } else {
+      float mx = 0.0f;
+      for (int i = g; i < L; i += 4) mx = fmaxf(mx, fabsf(x_at(i, ch)));
+      part[g][ch] = (double)mx;
+    }
+  }
+  __syncthreads();
+  if (tid < kD) {
+    if (tz < 2) {
+      const double s = ((part[0][tid] + part[1][tid]) + part[2][tid]) + part[3][tid];
+      stat[tid] = (L > 0) ? __double2float_rn(s / (double)L) : 0.0f;
+    } else {
+      const float mx = fmaxf(fmaxf((float)part[0][tid], (float)part[1][tid]), fmaxf((float)part[2][tid], (float)part[3][tid]));
+      const float sc = (mx > 0.0f) ? __fdiv_rn(mx, 127.0f) : 1.0f;
+      stat[tid] = sc;
+      a.vscale[(size_t)bh * kD + tid] = sc;
+    }
+  }
+  __syncthreads();
+  if (tz < 2) {
+    // one thread per token: sign bits against the means
+    for (int i = tid; i < (tz == 0 ? a.n : a.n_pad); i += kHeadThreads) {
+      uint32_t w0 = 0, w1 = 0;
+      if (i < L) {
+#pragma unroll 8
+        for (int ch = 0; ch < 32; ++ch) {
+          w0 |= (x_at(i, ch) < stat[ch] ? 1u : 0u) << ch;
+          w1 |= (x_at(i, ch + 32) < stat[ch + 32] ? 1u : 0u) << ch;
+        }
+      }
+      if (tz == 0) {
+        *reinterpret_cast<uint2*>(a.qbits + ((size_t)bh * a.n + i) * kW) = make_uint2(w0, w1);
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(a.kpm + ((size_t)bh * a.n_pad + i) * kD);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t f = (q < 2 ? w0 : w1) >> ((q & 1) * 16);
+          dst[q] = make_uint4(expand_nibble_pm1(f & 15u), expand_nibble_pm1((f >> 4) & 15u),
+                              expand_nibble_pm1((f >> 8) & 15u), expand_nibble_pm1((f >> 12) & 15u));
+        }
+      }
+    }
+  } else {
+    // thread (channel, block of 16 tokens): int8 V^T row segments of 16 bytes
+    const int ch = tid & (kD - 1);
+    const float sc = stat[ch];
+    for (int blk = tid >> 6; blk * 16 < a.n_pad; blk += kHeadThreads / kD) {
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        const int i = blk * 16 + u;
+        int q = 0;
+        if (i < L) {
+          float r = rintf(__fdiv_rn(x_at(i, ch), sc));
+          r = fminf(fmaxf(r, -127.0f), 127.0f);
+          q = (int)r;
+        }
+        w[u >> 2] |= ((uint32_t)q & 0xFFu) << (8 * (u & 3));
+      }
+      *reinterpret_cast<uint4*>(a.vqT + ((size_t)bh * kD + ch) * a.n_pad + blk * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+}  // namespace had
