@@ -11,9 +11,12 @@
 //   warp 5     TMA producer: +-1 int8 K tiles (64 keys x 64 B, 64-byte swizzle),
 //              V tiles (bf16 [64 keys][64], 128-byte swizzle, MN-major B) or int8
 //              V^T tiles ([64 channels][64 keys], 64-byte swizzle, K-major B).
-// Tensor memory (256 columns): two score buffers S0 [0,64) and S1 [64,128) so the
-// score MMA of tile t+1 runs while the softmax warps work on tile t; P [128,160)
-// bf16 (or [128,144) uint8 codes); residual P [160,192) for fp32 V; O [192,256).
+// Tensor memory (256 columns): a ring of three score buffers S0..S2 [0,192), so
+// the score MMAs of tiles t+1 and t+2 run while the softmax warps work on tile t,
+// and O [192,256).  P of tile t is written over its own score buffer (bf16 in
+// columns [0,32) of the buffer, the residual for fp32 V in [32,64); uint8 codes
+// in [0,16)): the P.V MMA of tile t is issued before the score MMA that next
+// writes that buffer, and MMAs from one thread run in issue order.
 //
 // Score (BinaryAttention §2.1/§2.2): S = Q~ K~^T with kind::i8 on +-1 operands,
 // so S = d - 2*popcount(q XOR k) exactly.  A.V: kind::f16 (bf16 P from TMEM x
@@ -50,13 +53,17 @@ constexpr int kVStages = 2;
 constexpr int kLevels = 65;
 constexpr int kRadixBins = 128;
 constexpr int kCandCap = 64;
-constexpr uint32_t kColS = 0, kColP = 128, kColPlo = 160, kColO = 192, kTmemCols = 256;
+constexpr int kSBufs = 3;
+constexpr uint32_t kColS = 0, kColO = 192, kTmemCols = 256;
 constexpr long long kWaitCycles = 2000000000LL;  // about one second
 // How the softmax threads find the bias offset koff(j) = y_j * tw + x_j of a key:
 constexpr int kKoffTable = 0;    // per-head table in shared memory (n_pad <= kKoffTableMax)
 constexpr int kKoffLinear = 1;   // prefix 0 and gw a multiple of 64: koff(j0 + u) = koff(j0) + u within a tile
 constexpr int kKoffTile = 2;     // computed per tile (double-buffered, one named barrier per tile)
 constexpr int kKoffTableMax = 1024;
+constexpr int kKoffClass = INT_MIN;        // key is a class token: bias 0
+constexpr int kKoffInvalid = INT_MIN + 1;  // key at or past the valid length: never kept
+constexpr int kBiasSmemMax = 4096;         // exp(bias) tables up to this many entries are staged in shared memory
 
 enum { SEL_DENSE = 0, SEL_TOPN_INT = 1, SEL_TOPN_FLOAT = 2 };
 enum { MODE_F = 0, MODE_Q = 1 };
@@ -76,6 +83,7 @@ struct TcArgs {
   const float* expb;       // [H][th][tw] exp(b - b_max(h)), or null
   int int_levels;          // 1 if fp32(c*s) is strictly increasing in s for every head
   int koff_mode;           // kKoffTable / kKoffLinear / kKoffTile
+  int bias_smem;           // 1: stage this head's exp(bias) table in shared memory
   const int32_t* seqlens;
   void* O;
   int o_bf16;
@@ -95,9 +103,10 @@ struct Smem {
   static constexpr int kK = kQ + kM * kD;                        // 4 x 4 KB
   static constexpr int kV = kK + kKStages * kN * kD;             // 2 V stages
   static constexpr int kKoff = kV + kVStages * kVStage;          // bias key offsets (table or 2 x 64)
-  static constexpr int kDq = kKoff + (HAS_BIAS ? kKoffTableMax * 4 : 0);  // 64 fp32 dequant scales
+  static constexpr int kBiasTab = kKoff + (HAS_BIAS ? kKoffTableMax * 4 : 0);  // exp(bias) table (dense)
+  static constexpr int kDq = kBiasTab + ((HAS_BIAS && SEL == SEL_DENSE) ? kBiasSmemMax * 4 : 0);  // 64 dequant scales
   static constexpr int kBar = kDq + kD * 4;
-  static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 7;
+  static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 2 * kSBufs + 2;
   static constexpr int kMisc = kBar + kNumBars * 8;              // [0] tmem base [1] abort
   static constexpr int kHist = (kMisc + 16 + 127) / 128 * 128;
   static constexpr int kHistBytes = (SEL == SEL_DENSE) ? kLevels * 32 * 4
@@ -113,25 +122,19 @@ enum {
   B_KEMPTY = kKStages,
   B_VFULL = 2 * kKStages,
   B_VEMPTY = 2 * kKStages + kVStages,
-  B_SFULL = 2 * kKStages + 2 * kVStages,  // 2 (one per score buffer)
-  B_TDONE = B_SFULL + 2,                  // 2
-  B_PEMPTY = B_TDONE + 2,
-  B_OFULL,
+  B_SFULL = 2 * kKStages + 2 * kVStages,  // one per score buffer
+  B_TDONE = B_SFULL + kSBufs,             // one per score buffer
+  B_OFULL = B_TDONE + kSBufs,
   B_FINAL
 };
 
-// Ties at the threshold are kept in key order while fewer than r_F have been
-// kept: of this chunk's tie bits `eqm` (bit u = key jb + u), keep the first
-// r_F - tie_seen (all of them when the row needs no cut).
-__device__ __forceinline__ uint32_t tie_keep(uint32_t eqm, int cut, int rF, int& tie_seen) {
-  uint32_t keep = eqm;
-  if (cut && eqm != 0u) {
-    const int allow = rF - tie_seen, cnt = __popc(eqm);
-    if (allow <= 0) keep = 0u;
-    else if (allow < cnt) keep = eqm & ((2u << __fns(eqm, 0u, allow)) - 1u);
-  }
-  tie_seen += __popc(eqm);
-  return keep;
+// Bias offset of key j: koff = y_j * tw + x_j for patch tokens, so that
+// b_ij = table[row_base(i) - koff]; class tokens and keys past L get a sentinel.
+__device__ __forceinline__ int key_offset(int j, int L, int prefix, int gw, int tw) {
+  if (j >= L) return kKoffInvalid;
+  if (j < prefix) return kKoffClass;
+  const int t = j - prefix;
+  return (t / gw) * tw + t % gw;
 }
 
 template <int SEL, int MODE, bool HAS_BIAS, bool VF32, int EXPORT>
@@ -191,8 +194,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
   if (warp == 5 && lane == 0) {
     for (int s = 0; s < kKStages; ++s) { mbar_init(&bars[B_KFULL + s], 1); mbar_init(&bars[B_KEMPTY + s], 1); }
     for (int s = 0; s < kVStages; ++s) { mbar_init(&bars[B_VFULL + s], 1); mbar_init(&bars[B_VEMPTY + s], 1); }
-    for (int s = 0; s < 2; ++s) { mbar_init(&bars[B_SFULL + s], 1); mbar_init(&bars[B_TDONE + s], kM); }
-    mbar_init(&bars[B_PEMPTY], 1);
+    for (int s = 0; s < kSBufs; ++s) { mbar_init(&bars[B_SFULL + s], 1); mbar_init(&bars[B_TDONE + s], kM); }
     mbar_init(&bars[B_OFULL], 1);
     mbar_init(&bars[B_FINAL], 1);
     misc[1] = 0;
@@ -228,12 +230,12 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       for (int lev = 0; lev < kLevels; ++lev) lt[lev * 32 + tid] = exp2f(ck * (float)lev);
     }
     if (MODE == MODE_Q && EXPORT == EXP_NONE && tid < kD) dq[tid] = __fdiv_rn(a.vscale[(size_t)bh * kD + tid], 255.0f);
-    if (HAS_BIAS && a.koff_mode == kKoffTable) {
-      for (int j = tid; j < a.n_pad; j += kM) {
-        int off = INT_MIN;
-        if (j >= a.prefix && j < a.n) { const int tt = j - a.prefix; off = (tt / a.gw) * a.tw + tt % a.gw; }
-        koff_tab[j] = off;
-      }
+    if (HAS_BIAS && a.koff_mode == kKoffTable)
+      for (int j = tid; j < a.n_pad; j += kM) koff_tab[j] = key_offset(j, L, a.prefix, a.gw, a.tw);
+    if (HAS_BIAS && SEL == SEL_DENSE && a.bias_smem) {
+      const float* src = a.expb + (size_t)h * a.th * a.tw;
+      float* dst = reinterpret_cast<float*>(sm + SM::kBiasTab);
+      for (int i = tid; i < a.th * a.tw; i += kM) dst[i] = __ldg(src + i);
     }
     fence_proxy_async();
   }
@@ -266,7 +268,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
   const bool sum_in_pv = (MODE == MODE_F) && (SEL == SEL_TOPN_FLOAT || (SEL == SEL_DENSE && use_lut));
   int sF = 0;  // integer threshold score (top-N without bias)
 
-  uint32_t g_k = 0, g_v = 0, g_s = 0, g_p = 0;  // tiles issued so far (all passes), per role
+  uint32_t g_k = 0, g_v = 0, g_s = 0;  // tiles issued so far (all passes), per role
   int k_par[kKStages], v_par[kVStages];          // producer: parity of the last load per stage (-1 none)
 #pragma unroll
   for (int s2 = 0; s2 < kKStages; ++s2) k_par[s2] = -1;
@@ -322,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
         const uint32_t id_s = idesc_i8(kM, kN, true, true, false);
         const uint32_t id_pv = (MODE == MODE_Q) ? idesc_i8(kM, kD, false, true, false) : idesc_bf16(kM, kD, true);
         auto issue_scores = [&](int t) {
-          const uint32_t gk = g_k + (uint32_t)t, st = gk % kKStages, buf = (g_s + (uint32_t)t) & 1u;
+          const uint32_t gk = g_k + (uint32_t)t, st = gk % kKStages, buf = (g_s + (uint32_t)t) % kSBufs;
           if (!bounded_wait(B_KFULL + st, (gk / kKStages) & 1)) return;
           tc_fence_after();
           const uint32_t kq = smem_u32(sQ), kk = smem_u32(sm + SM::kK + st * kN * kD);
@@ -333,11 +335,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
           mma_commit(&bars[B_SFULL + buf]);
           mma_commit(&bars[B_KEMPTY + st]);
         };
-        issue_scores(0);
-        if (ntiles > 1) issue_scores(1);
+        for (int t = 0; t < kSBufs && t < ntiles; ++t) issue_scores(t);
         for (int t = 0; t < ntiles; ++t) {
-          const uint32_t gs = g_s + (uint32_t)t, buf = gs & 1u;
-          bounded_wait(B_TDONE + buf, (gs >> 1) & 1);
+          const uint32_t gs = g_s + (uint32_t)t, buf = gs % kSBufs;
+          const uint32_t colP = kColS + buf * kN;  // P of this tile sits over its score buffer
+          bounded_wait(B_TDONE + buf, (gs / kSBufs) & 1);
           tc_fence_after();
           if (pv && !*abort_flag) {
             const uint32_t gv = g_v + (uint32_t)t, vs = gv % kVStages;
@@ -347,37 +349,36 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
               if (MODE == MODE_Q) {
 #pragma unroll
                 for (int k = 0; k < kN / 32; ++k)
-                  mma_i8_ts(tmem + kColO, tmem + kColP + 8 * k, sdesc(vbase + 32 * k, 16, 512, kSwizzle64B), id_pv,
+                  mma_i8_ts(tmem + kColO, tmem + colP + 8 * k, sdesc(vbase + 32 * k, 16, 512, kSwizzle64B), id_pv,
                             (t > 0 || k > 0) ? 1u : 0u);
               } else {
 #pragma unroll
                 for (int k = 0; k < kN / 16; ++k)
-                  mma_f16_ts(tmem + kColO, tmem + kColP + 8 * k, sdesc(vbase + 2048 * k, 0, 1024, kSwizzle128B), id_pv,
+                  mma_f16_ts(tmem + kColO, tmem + colP + 8 * k, sdesc(vbase + 2048 * k, 0, 1024, kSwizzle128B), id_pv,
                              (t > 0 || k > 0) ? 1u : 0u);
                 if (VF32) {
                   // residual products: P_hi x V_lo and P_lo x V_hi
                   const uint32_t vlo = vbase + kN * kD * 2;
 #pragma unroll
                   for (int k = 0; k < kN / 16; ++k)
-                    mma_f16_ts(tmem + kColO, tmem + kColP + 8 * k, sdesc(vlo + 2048 * k, 0, 1024, kSwizzle128B), id_pv,
+                    mma_f16_ts(tmem + kColO, tmem + colP + 8 * k, sdesc(vlo + 2048 * k, 0, 1024, kSwizzle128B), id_pv,
                                1u);
 #pragma unroll
                   for (int k = 0; k < kN / 16; ++k)
-                    mma_f16_ts(tmem + kColO, tmem + kColPlo + 8 * k, sdesc(vbase + 2048 * k, 0, 1024, kSwizzle128B),
+                    mma_f16_ts(tmem + kColO, tmem + colP + 32 + 8 * k, sdesc(vbase + 2048 * k, 0, 1024, kSwizzle128B),
                                id_pv, 1u);
                 }
               }
-              mma_commit(&bars[B_PEMPTY]);
               mma_commit(&bars[B_VEMPTY + vs]);
               if (t + 1 == ntiles) mma_commit(&bars[B_OFULL]);
             }
           }
-          if (t + 2 < ntiles) issue_scores(t + 2);
+          if (t + kSBufs < ntiles) issue_scores(t + kSBufs);
         }
       }
       g_k += ntiles;
       g_s += ntiles;
-      if (pv) { g_v += ntiles; g_p += ntiles; }
+      if (pv) g_v += ntiles;
     }
     // ============================================================== softmax / select (warps 0-3)
     else {
@@ -385,14 +386,26 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       const uint32_t hist_row = smem_u32(hist) + (uint32_t)tid * 4u;
       const float mo = -m * kLog2e;
       const float* lut = reinterpret_cast<const float*>(hist);
+      // Passes compiled into this instantiation (the rest are pruned at compile time).
+      constexpr bool kHasLevels = SEL != SEL_DENSE;
+      constexpr bool kHasNorm = SEL == SEL_DENSE;
+      constexpr bool kHasRadix = SEL == SEL_TOPN_FLOAT;
+      constexpr bool kHasKeptNorm = SEL == SEL_TOPN_FLOAT && (MODE == MODE_Q || EXPORT == EXP_CODES);
+      constexpr bool kHasIdx = EXPORT == EXP_IDX;
+      constexpr bool kHasCodes = EXPORT == EXP_CODES;
+      constexpr bool kHasPv = EXPORT == EXP_NONE;
       // lut_e: dense weights from the level table x exp(bias - b_max) (no row max needed)
       // lut_w: top-N (no bias) weights from the row's level table, zero below the threshold
       const bool lut_e = (SEL == SEL_DENSE) && use_lut && (pass == P_NORM || pass == P_PV || pass == P_CODES);
       const bool lut_w = (SEL == SEL_TOPN_INT) && a.int_levels && pass == P_PV;
       const bool wants_bias = HAS_BIAS && pass != P_LEVELS;
-      const float* expb_h = HAS_BIAS ? a.expb + (size_t)h * a.th * a.tw : nullptr;
+      // exp(b - b_max) of this head: staged in shared memory when it fits (dense only)
+      const float* expb_h = nullptr;
+      if (HAS_BIAS && SEL == SEL_DENSE)
+        expb_h = a.bias_smem ? reinterpret_cast<const float*>(sm + SM::kBiasTab) : a.expb + (size_t)h * a.th * a.tw;
       for (int t = 0; t < ntiles; ++t) {
-        const uint32_t gs = g_s + (uint32_t)t, buf = gs & 1u;
+        const uint32_t gs = g_s + (uint32_t)t, buf = gs % kSBufs;
+        const uint32_t colP = kColS + buf * kN;  // P of this tile is written over its score buffer
         const int j0 = t * kN;
         // bias offsets of this tile's keys: per-head table, closed form, or computed per tile
         const int* ko = koff_tab + j0;
@@ -401,211 +414,231 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
           if (a.koff_mode == kKoffLinear) {
             lin_base = (j0 / a.gw) * a.tw + j0 % a.gw;
           } else if (a.koff_mode == kKoffTile) {
-            ko = koff_tab + buf * kN;  // alternates across passes too
-            if (tid < kN) {
-              const int j = j0 + tid;
-              int off = INT_MIN;
-              if (j >= a.prefix && j < a.n) { const int tt = j - a.prefix; off = (tt / a.gw) * a.tw + tt % a.gw; }
-              koff_tab[buf * kN + tid] = off;
-            }
+            const uint32_t kb = gs & 1u;  // alternates across passes too
+            ko = koff_tab + kb * kN;
+            if (tid < kN) koff_tab[kb * kN + tid] = key_offset(j0 + tid, L, a.prefix, a.gw, a.tw);
             asm volatile("bar.sync 1, 128;" ::: "memory");
           }
         }
-        const bool ok_wait = __all_sync(0xffffffffu, bounded_wait(B_SFULL + buf, (gs >> 1) & 1));
+        const bool ok_wait = __all_sync(0xffffffffu, bounded_wait(B_SFULL + buf, (gs / kSBufs) & 1));
         tc_fence_after();
-        const int nvalid = row_ok ? max(0, min(kN, L - j0)) : 0;
-        // both 32-column halves of the tile are loaded at once; the loop body
-        // (one copy of the code per pass) then runs on r and moves rn into r
-        uint32_t r[32], rn[32];
-        tmem_ld32(tl + kColS + buf * kN, r);
-        tmem_ld32(tl + kColS + buf * kN + 32, rn);
+        uint32_t r[64];
+        tmem_ld32(tl + kColS + buf * kN, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        tmem_ld32(tl + kColS + buf * kN + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         tmem_wait_ld();
-#pragma unroll 1
-        for (int ch = 0; ch < 2; ++ch) {
-          if (ch == 1) {
-#pragma unroll
-            for (int u = 0; u < 32; ++u) r[u] = rn[u];
-          }
-          if (!ok_wait) continue;
+        const int nvalid = row_ok ? max(0, min(kN, L - j0)) : 0;
+        // Dense with bias: keys past L carry the kKoffInvalid sentinel (weight 0), and
+        // rows past L are never stored, so every tile takes the unmasked path.
+        constexpr bool kMaskInKoff = SEL == SEL_DENSE && HAS_BIAS;
+        const bool full_tile = kMaskInKoff || __all_sync(0xffffffffu, nvalid == kN);
+
+        // bias offsets of keys 32*ch+u .. +3 of this tile
+        auto koff4 = [&](int idx) -> int4 {
+          if (a.koff_mode == kKoffLinear) return make_int4(lin_base + idx, lin_base + idx + 1, lin_base + idx + 2, lin_base + idx + 3);
+          return *reinterpret_cast<const int4*>(ko + idx);
+        };
+
+        // ---- P (or uint8 A) of one 32-key chunk into TMEM, or codes to global (export)
+        auto emit = [&](const float (&e)[32], int ch) {
           const int jb = j0 + 32 * ch;
-          const int nv = min(32, max(0, nvalid - 32 * ch));
-          const uint32_t vmask = nv >= 32 ? 0xFFFFFFFFu : ((1u << nv) - 1u);
-          auto bias_index = [&](int u, bool& has) -> int {
-            int kk = (a.koff_mode == kKoffLinear) ? lin_base + 32 * ch + u : ko[32 * ch + u];
-            has = rb >= 0 && kk != INT_MIN;
-            return rb - kk;
-          };
-          float e[32];
-          bool have_e = false;
-          if (SEL != SEL_DENSE && pass == P_LEVELS) {
-            const uint32_t base = hist_row + 32u * kM * 4u;  // level (64 - s)/2 -> + (64 - s) * 256 bytes
+          if (kHasCodes || MODE == MODE_Q) {
+            uint32_t wq[8];
 #pragma unroll
-            for (int u = 0; u < 32; ++u) {
-              // predicated inside the asm, so a ragged tile costs no branches
-              const uint32_t ad = base - (uint32_t)((int)r[u] * (kM * 2));
-              asm volatile(
-                  "{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t@p red.shared.add.u32 [%0], 1;\n\t}" ::"r"(ad),
-                  "r"((vmask >> u) & 1u)
-                  : "memory");
+            for (int u = 0; u < 8; ++u) {
+              uint32_t w = 0;
+#pragma unroll
+              for (int v = 0; v < 4; ++v) {
+                const uint32_t code = (uint32_t)min(255, (int)floorf(__fmaf_rn(e[4 * u + v], scale, 0.5f)));
+                w |= code << (8 * v);
+              }
+              wq[u] = w;
             }
-          } else if (SEL == SEL_DENSE && lut_e) {
-#pragma unroll
-            for (int u = 0; u < 32; ++u) {
-              const int sc = (int)r[u];
-              float x = lut[(32 - (sc >> 1)) * 32 + lane];
-              if (HAS_BIAS) {
-                bool has;
-                const int bi = bias_index(u, has);
-                x *= has ? __ldg(expb_h + bi) : fb0;
-              }
-              e[u] = ((vmask >> u) & 1u) ? x : 0.0f;
-            }
-            if (pass == P_NORM) {
-#pragma unroll
-              for (int u = 0; u < 32; ++u) lsum += e[u];
-            } else {
-              have_e = true;
-            }
-          } else if (SEL == SEL_TOPN_INT && lut_w) {
-            uint32_t eqm = 0;
-#pragma unroll
-            for (int u = 0; u < 32; ++u) {
-              const int sc = (int)r[u];
-              e[u] = lut[(32 - (sc >> 1)) * kM + tid];
-              eqm |= (sc == sF ? 1u : 0u) << u;
-            }
-            eqm &= vmask;
-            const uint32_t keepm = vmask & ~(eqm & ~tie_keep(eqm, cut, rF, tie_seen));
-#pragma unroll
-            for (int u = 0; u < 32; ++u) e[u] = ((keepm >> u) & 1u) ? e[u] : 0.0f;
-            have_e = true;
-          } else {
-            // generic path: exact logits (invalid keys -inf)
-            float lg[32];
-#pragma unroll
-            for (int u = 0; u < 32; ++u) {
-              const int sc = (int)r[u];
-              float l;
-              if (HAS_BIAS) {
-                bool has;
-                const int bi = bias_index(u, has);
-                l = __fmaf_rn((float)sc, c, has ? __ldg(tab + bi) : 0.0f);
-              } else {
-                l = (float)sc * c;
-              }
-              lg[u] = ((vmask >> u) & 1u) ? l : -INFINITY;
-            }
-            if (SEL == SEL_DENSE && pass == P_NORM) {
-              float tm = -INFINITY;
-#pragma unroll
-              for (int u = 0; u < 32; ++u) tm = fmaxf(tm, lg[u]);
-              if (tm > m) {
-                lsum *= fast_exp2((m - tm) * kLog2e);
-                m = tm;
-              }
-              const float mo2 = -m * kLog2e;
-#pragma unroll
-              for (int u = 0; u < 32; ++u) lsum += fast_exp2(__fmaf_rn(lg[u], kLog2e, mo2));
-            } else if (SEL == SEL_TOPN_FLOAT && pass == P_RADIX) {
-              if (r_state == 1) {
-#pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                  const uint32_t dd = r_uhi - float_order_key(lg[u]);
-                  if (((vmask >> u) & 1u) && dd <= r_span) atomicAdd(&hist[(dd >> r_shift) * kM + tid], 1u);
-                }
-              }
-            } else if (SEL == SEL_TOPN_FLOAT && pass == P_COLLECT) {
-              if (r_state == 2) {
-                uint2* cand = reinterpret_cast<uint2*>(hist);  // [64][128 rows]
-#pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                  const uint32_t key = float_order_key(lg[u]);
-                  const uint32_t dd = r_uhi - key;
-                  if (((vmask >> u) & 1u) && dd <= r_span && (int)(dd >> r_shift) == r_bin) {
-                    if (r_cnt < kCandCap) cand[r_cnt * kM + tid] = make_uint2(key, (uint32_t)(jb + u));
-                    ++r_cnt;
-                  }
-                }
-              }
-            } else {
-              // keep mask in key order; ties at F counted per row
-              uint32_t keepm = vmask;
-              if (SEL != SEL_DENSE) {
-                uint32_t gtm = 0, eqm = 0;
-#pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                  gtm |= (lg[u] > F ? 1u : 0u) << u;
-                  eqm |= (lg[u] == F ? 1u : 0u) << u;
-                }
-                keepm = (gtm & vmask) | tie_keep(eqm & vmask, cut, rF, tie_seen);
-              }
-              if (SEL == SEL_TOPN_FLOAT && (MODE == MODE_Q || EXPORT == EXP_CODES) && pass == P_KEPT_NORM) {
+            if (kHasCodes) {
+              if (row >= a.row_begin && row < a.row_end && row < a.n) {
+                const int rows = a.row_end - a.row_begin;
+                uint8_t* dst = a.codes + ((size_t)bh * rows + (row - a.row_begin)) * a.n;
 #pragma unroll
                 for (int u = 0; u < 32; ++u)
-                  lsum += ((keepm >> u) & 1u) ? fast_exp2(__fmaf_rn(lg[u], kLog2e, mo)) : 0.0f;
-              } else if (EXPORT == EXP_IDX && pass == P_IDX) {
-                if (row_ok) {
-                  int32_t* dst = a.idx + ((size_t)bh * a.n + row) * a.N;
-#pragma unroll
-                  for (int u = 0; u < 32; ++u)
-                    if ((keepm >> u) & 1u) { if (kept_seen < a.N) dst[kept_seen] = jb + u; ++kept_seen; }
-                }
-              } else {
-#pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                  const float x = fast_exp2(__fmaf_rn(lg[u], kLog2e, mo));
-                  e[u] = ((keepm >> u) & 1u) ? x : 0.0f;
-                }
-                have_e = true;
+                  if (jb + u < a.n) dst[jb + u] = (uint8_t)((wq[u >> 2] >> (8 * (u & 3))) & 0xFFu);
               }
+            } else {
+              tmem_st8(tl + colP + 8 * ch, wq);
             }
-          }
-          // ---- P (or uint8 A) of the chunk into TMEM, or codes to global (export)
-          if (have_e) {
-            if ((EXPORT == EXP_CODES && pass == P_CODES) || (EXPORT == EXP_NONE && MODE == MODE_Q)) {
-              uint32_t wq[8];
+          } else {
+            uint32_t wp[16];
 #pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                uint32_t w = 0;
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                  const uint32_t code = (uint32_t)min(255, (int)floorf(__fmaf_rn(e[4 * u + v], scale, 0.5f)));
-                  w |= code << (8 * v);
-                }
-                wq[u] = w;
-              }
-              if (EXPORT == EXP_CODES) {
-                if (row >= a.row_begin && row < a.row_end && row < a.n) {
-                  const int rows = a.row_end - a.row_begin;
-                  uint8_t* dst = a.codes + ((size_t)bh * rows + (row - a.row_begin)) * a.n;
-#pragma unroll
-                  for (int u = 0; u < 32; ++u)
-                    if (jb + u < a.n) dst[jb + u] = (uint8_t)((wq[u >> 2] >> (8 * (u & 3))) & 0xFFu);
-                }
-              } else {
-                if (ch == 0 && t > 0) bounded_wait(B_PEMPTY, (g_p + (uint32_t)t - 1) & 1);
-                tmem_st8(tl + kColP + 8 * ch, wq);
-              }
-            } else if (EXPORT == EXP_NONE) {
-              uint32_t wp[16];
+            for (int u = 0; u < 16; ++u) {
+              wp[u] = pack_bf16x2(e[2 * u], e[2 * u + 1]);
+              if (sum_in_pv) lsum += e[2 * u] + e[2 * u + 1];
+            }
+            tmem_st16(tl + colP + 16 * ch, wp);
+            if (VF32) {
+              uint32_t wl[16];
 #pragma unroll
               for (int u = 0; u < 16; ++u) {
-                wp[u] = pack_bf16x2(e[2 * u], e[2 * u + 1]);
-                if (sum_in_pv) lsum += e[2 * u] + e[2 * u + 1];
+                const float h0 = __uint_as_float(wp[u] << 16), h1 = __uint_as_float(wp[u] & 0xFFFF0000u);
+                wl[u] = pack_bf16x2(e[2 * u] - h0, e[2 * u + 1] - h1);
               }
-              if (ch == 0 && t > 0) bounded_wait(B_PEMPTY, (g_p + (uint32_t)t - 1) & 1);
-              tmem_st16(tl + kColP + 16 * ch, wp);
-              if (VF32) {
-                uint32_t wl[16];
+              tmem_st16(tl + colP + 32 + 16 * ch, wl);
+            }
+          }
+        };
+
+        auto tile_body = [&](auto full_tag) {
+          constexpr bool FULL = decltype(full_tag)::value;
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                  const float h0 = __uint_as_float(wp[u] << 16), h1 = __uint_as_float(wp[u] & 0xFFFF0000u);
-                  wl[u] = pack_bf16x2(e[2 * u] - h0, e[2 * u + 1] - h1);
+          for (int ch = 0; ch < 2; ++ch) {
+            const int jb = j0 + 32 * ch;
+            if (kHasLevels && pass == P_LEVELS) {
+              const uint32_t base = hist_row + 32u * kM * 4u;  // level (64 - s)/2 -> + (64 - s) * 256 bytes
+#pragma unroll
+              for (int u = 0; u < 32; ++u) {
+                const uint32_t ad = base - (uint32_t)((int)r[32 * ch + u] * (kM * 2));
+                if (FULL) {
+                  asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(ad) : "memory");
+                } else {
+                  asm volatile(
+                      "{\n\t.reg .pred p;\n\tsetp.lt.s32 p, %1, %2;\n\t@p red.shared.add.u32 [%0], 1;\n\t}" ::"r"(ad),
+                      "r"(32 * ch + u), "r"(nvalid)
+                      : "memory");
                 }
-                tmem_st16(tl + kColPlo + 16 * ch, wl);
+              }
+            } else if (SEL == SEL_DENSE && lut_e) {
+              float e[32];
+#pragma unroll
+              for (int u = 0; u < 32; u += 4) {
+                int4 k4 = make_int4(0, 0, 0, 0);
+                if (HAS_BIAS) k4 = koff4(32 * ch + u);
+                const int kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                  const int sc = (int)r[32 * ch + u + v];
+                  float x = lut[(32 - (sc >> 1)) * 32 + lane];
+                  if (HAS_BIAS) {
+                    const float special = (kk[v] == kKoffInvalid) ? 0.0f : fb0;
+                    x *= (rb >= 0 && kk[v] >= 0) ? expb_h[rb - kk[v]] : special;
+                  }
+                  e[u + v] = (FULL || 32 * ch + u + v < nvalid) ? x : 0.0f;
+                }
+              }
+              if (pass == P_NORM) {
+#pragma unroll
+                for (int u = 0; u < 32; ++u) lsum += e[u];
+              } else {
+                emit(e, ch);
+              }
+            } else if (SEL == SEL_TOPN_INT && lut_w) {
+              float e[32];
+#pragma unroll
+              for (int u = 0; u < 32; ++u) {
+                const int sc = (int)r[32 * ch + u];
+                const float w = lut[(32 - (sc >> 1)) * kM + tid];
+                const bool valid = FULL || 32 * ch + u < nvalid;
+                const bool eq = valid && sc == sF;
+                const bool drop_tie = eq && cut && tie_seen >= rF;
+                tie_seen += eq ? 1 : 0;
+                e[u] = (valid && !drop_tie) ? w : 0.0f;
+              }
+              emit(e, ch);
+            } else {
+              // generic path: exact logits (invalid keys -inf)
+              float lg[32];
+              uint32_t kinv = 0;  // keys past L (dense with bias: the sentinel, not the tile mask)
+#pragma unroll
+              for (int u = 0; u < 32; u += 4) {
+                int4 k4 = make_int4(0, 0, 0, 0);
+                if (HAS_BIAS) k4 = koff4(32 * ch + u);
+                const int kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                  const int sc = (int)r[32 * ch + u + v];
+                  float l;
+                  if (HAS_BIAS) {
+                    if (kMaskInKoff) kinv |= (kk[v] == kKoffInvalid ? 1u : 0u) << (u + v);
+                    const float special = (kk[v] == kKoffInvalid) ? -INFINITY : 0.0f;
+                    const float bv = (rb >= 0 && kk[v] >= 0) ? __ldg(tab + (rb - kk[v])) : special;
+                    l = __fmaf_rn((float)sc, c, bv);
+                  } else {
+                    l = (float)sc * c;
+                  }
+                  lg[u + v] = (FULL || 32 * ch + u + v < nvalid) ? l : -INFINITY;
+                }
+              }
+              if (kHasNorm && pass == P_NORM) {
+                float tm = -INFINITY;
+#pragma unroll
+                for (int u = 0; u < 32; ++u) tm = fmaxf(tm, lg[u]);
+                if (tm > m) {
+                  lsum *= fast_exp2((m - tm) * kLog2e);
+                  m = tm;
+                }
+                const float mo2 = -m * kLog2e;
+#pragma unroll
+                for (int u = 0; u < 32; ++u) lsum += fast_exp2(__fmaf_rn(lg[u], kLog2e, mo2));
+              } else if (kHasRadix && pass == P_RADIX) {
+                if (r_state == 1) {
+#pragma unroll
+                  for (int u = 0; u < 32; ++u) {
+                    const uint32_t dd = r_uhi - float_order_key(lg[u]);
+                    if ((FULL || 32 * ch + u < nvalid) && dd <= r_span) atomicAdd(&hist[(dd >> r_shift) * kM + tid], 1u);
+                  }
+                }
+              } else if (kHasRadix && pass == P_COLLECT) {
+                if (r_state == 2) {
+                  uint2* cand = reinterpret_cast<uint2*>(hist);  // [64][128 rows]
+#pragma unroll
+                  for (int u = 0; u < 32; ++u) {
+                    const uint32_t key = float_order_key(lg[u]);
+                    const uint32_t dd = r_uhi - key;
+                    if ((FULL || 32 * ch + u < nvalid) && dd <= r_span && (int)(dd >> r_shift) == r_bin) {
+                      if (r_cnt < kCandCap) cand[r_cnt * kM + tid] = make_uint2(key, (uint32_t)(jb + u));
+                      ++r_cnt;
+                    }
+                  }
+                }
+              } else {
+                // keep mask in key order; ties at F counted per row
+                uint32_t keepm = 0;
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                  const bool valid = FULL || 32 * ch + u < nvalid;
+                  bool k;
+                  if (SEL == SEL_DENSE) {
+                    k = valid && !((kinv >> u) & 1u);
+                  } else {
+                    const bool gt = valid && lg[u] > F, eq = valid && lg[u] == F;
+                    k = gt || (eq && (!cut || tie_seen < rF));
+                    tie_seen += eq ? 1 : 0;
+                  }
+                  keepm |= (k ? 1u : 0u) << u;
+                }
+                if (kHasKeptNorm && pass == P_KEPT_NORM) {
+#pragma unroll
+                  for (int u = 0; u < 32; ++u)
+                    lsum += ((keepm >> u) & 1u) ? fast_exp2(__fmaf_rn(lg[u], kLog2e, mo)) : 0.0f;
+                } else if (kHasIdx && pass == P_IDX) {
+                  if (row_ok) {
+                    int32_t* dst = a.idx + ((size_t)bh * a.n + row) * a.N;
+#pragma unroll
+                    for (int u = 0; u < 32; ++u)
+                      if ((keepm >> u) & 1u) { if (kept_seen < a.N) dst[kept_seen] = jb + u; ++kept_seen; }
+                  }
+                } else if (kHasPv || kHasCodes) {
+                  float e[32];
+#pragma unroll
+                  for (int u = 0; u < 32; ++u) {
+                    const float x = fast_exp2(__fmaf_rn(lg[u], kLog2e, mo));
+                    e[u] = ((keepm >> u) & 1u) ? x : 0.0f;
+                  }
+                  emit(e, ch);
+                }
               }
             }
           }
+        };
+        if (ok_wait) {
+          if (full_tile) tile_body(std::true_type{});
+          else tile_body(std::false_type{});
         }
         if (pv) tmem_wait_st();
         tc_fence_before();
@@ -613,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       }
       g_k += ntiles;
       g_s += ntiles;
-      if (pv) { g_v += ntiles; g_p += ntiles; }
+      if (pv) g_v += ntiles;
     }
 
     // ============================================================== per-row decisions after the pass

@@ -457,8 +457,9 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
   a.koff_mode = tc::kKoffTile;
   if (has_bias) {
     if (d.n_pad <= tc::kKoffTableMax) a.koff_mode = tc::kKoffTable;
-    else if (bias->prefix == 0 && bias->gw % tc::kN == 0) a.koff_mode = tc::kKoffLinear;
+    else if (bias->prefix == 0 && bias->gw % tc::kN == 0 && s->seqlens == nullptr) a.koff_mode = tc::kKoffLinear;
   }
+  a.bias_smem = (has_bias && a.th * a.tw <= tc::kBiasSmemMax) ? 1 : 0;
   a.int_levels = 1;
   for (int h = 0; h < s->H; ++h) {
     const double aq = alpha_q ? (double)alpha_q[h] : 1.0, ak = alpha_k ? (double)alpha_k[h] : 1.0;

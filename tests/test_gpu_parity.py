@@ -230,6 +230,46 @@ def test_stress_full_size_both_passes(oracle_mod):
     _codes_ok(A, ref_c.Aq)
 
 
+# ----------------------------------------------------------------------------- bias layouts and lengths
+
+def _check_grid(oracle_mod, w, per_head, seed):
+    """Dense uint8 (O and codes), top-N float O and index sets, and dense index
+    sets (N = n) of a relative-position-bias workload, on sampled rows."""
+    Q, K, V, seq, bias = _dev_inputs(w)
+    rows = _sample_rows(w, per_head, seed)
+    rows_t = torch.from_numpy(rows).cuda()
+    N = max(1, w.n // 8)
+    Oq = _flat(had.had_attention(Q, K, V, N=0, mode="u8i8", seqlens=seq, bias=bias))[rows_t].float().cpu().numpy()
+    ref_q = _oracle_full(oracle_mod, w, 0, 1, rows=rows)
+    assert np.max(np.abs(Oq - ref_q.O)) <= _tol(w)
+    Of = _flat(had.had_attention(Q, K, V, N=N, mode="float", seqlens=seq, bias=bias))[rows_t].float().cpu().numpy()
+    ref_f = _oracle_full(oracle_mod, w, N, 0, rows=rows)
+    assert np.max(np.abs(Of - ref_f.O)) <= _tol(w)
+    for n_keep in (N, w.n):
+        idx = _flat(had.had_topn_indices(Q, K, n_keep, seq, bias))[rows_t].cpu().numpy()
+        ref_i = _oracle_full(oracle_mod, w, n_keep, 0, rows=rows, want_idx=True).idx
+        np.testing.assert_array_equal(idx, ref_i)
+    # codes of every row of the first head of each batch (keys past L must be 0)
+    A = had.had_attention_codes_u8(Q, K, V, 0, w.n, N=0, seqlens=seq, bias=bias).cpu().numpy()
+    A = A.reshape(w.B, w.H, w.n, w.n)[:, 0].reshape(-1, w.n)
+    band = np.array([b * w.H * w.n + i for b in range(w.B) for i in range(w.n)], np.int64)
+    ref_c = _oracle_full(oracle_mod, w, 0, 1, rows=band, want_codes=True)
+    _codes_ok(A, ref_c.Aq)
+
+
+@pytest.mark.parametrize("gh,gw,prefix,seqlens", [
+    (14, 14, 1, [197, 150, 65, 1]),      # per-head offset table, class token, ragged lengths
+    (16, 128, 0, None),                  # 64-key tiles inside one image row: closed-form offsets
+    (16, 128, 0, [2048, 1000]),          # same grid with lengths: offsets computed per tile
+    (8, 160, 0, None),                   # tiles crossing image rows, n > 1024: offsets per tile
+    (6, 30, 2, [182, 97]),               # two class tokens, ragged lengths, table offsets
+])
+def test_relpos_bias_layouts(oracle_mod, gh, gw, prefix, seqlens):
+    B = 1 if seqlens is None else len(seqlens)
+    w = workloads.grid(B, 2, gh, gw, prefix, seqlens)
+    _check_grid(oracle_mod, w, 24, 21)
+
+
 # ----------------------------------------------------------------------------- comparison mode
 
 def test_dense_reference_mode(oracle_mod):

@@ -171,6 +171,24 @@ def stress() -> Workload:
                     "Q,K,V iid N(0,1); relpos bias 255x255/head ~N(0,0.1), prefix 0")
 
 
+def grid(B: int, H: int, gh: int, gw: int, prefix: int, seqlens=None, seed: int = 11) -> Workload:
+    """Image-grid attention of any size: B x H heads over `prefix` class tokens
+    plus a gh x gw patch grid, d64 bf16 Q,K,V iid N(0,1), a relative-position
+    bias (2gh-1) x (2gw-1) per head ~N(0, 0.1), optional per-batch lengths.
+    Used to cover the grid shapes the fixed workloads do not reach."""
+    rng = np.random.default_rng(seed)
+    n, d = prefix + gh * gw, 64
+    Q = rng.standard_normal((B, H, n, d), dtype=np.float32)
+    K = rng.standard_normal((B, H, n, d), dtype=np.float32)
+    V = rng.standard_normal((B, H, n, d), dtype=np.float32)
+    table = rng.standard_normal((H, 2 * gh - 1, 2 * gw - 1), dtype=np.float32) * np.float32(0.1)
+    sl = None if seqlens is None else np.asarray(seqlens, np.int32)
+    return Workload(f"grid_b{B}_h{H}_{gh}x{gw}_p{prefix}" + ("" if sl is None else "_sl"), B, H, n, d, "bf16",
+                    _finish(Q, "bf16"), _finish(K, "bf16"), _finish(V, "bf16"), sl, Bias(table, gh, gw, prefix),
+                    [(max(1, n // 8), MODE_FLOAT), (0, MODE_U8I8)], seed,
+                    "Q,K,V iid N(0,1); relpos bias ~N(0,0.1)")
+
+
 def by_name(name: str) -> Workload:
     if name == "tiny":
         return tiny()
