@@ -65,13 +65,12 @@ HEAD_STAGE_BYTES = 128 * 1024  # heads up to this size are prepared by one kerne
 
 def launches_per_step(n: int, elem: int, mode: str, has_bias: bool) -> int:
     """Kernels one prepare + attend step launches: the sign/pack stage (one
-    kernel for short heads, statistics + pack otherwise), the hi/lo split of an
-    fp32 V (float mode), the two bias-table kernels, and the fused attention."""
-    k = 1 if n * 64 * elem <= HEAD_STAGE_BYTES else 2
+    kernel for short heads, which also builds the bias tables; statistics +
+    pack + bias tables otherwise), the hi/lo split of an fp32 V (float mode),
+    and the fused attention."""
+    k = 1 if n * 64 * elem <= HEAD_STAGE_BYTES else 2 + (1 if has_bias else 0)
     if mode == "float" and elem == 4:
         k += 1
-    if has_bias:
-        k += 2
     return k + 1
 
 

@@ -9,7 +9,7 @@
 //   k_stats  : fp64 channel partial sums of Q and K (+ fp32 absmax of V in uint8 mode)
 //   k_pack   : mu -> sign bits of Q (packed uint32) and K (+-1 int8 rows);
 //              V scale -> int8 V^T (uint8 mode)
-//   k_bias_minmax (top-N with a bias): per-head bias range for the select band
+//   k_bias_tables (with a bias): per-head bias range and exp(b - b_max) table
 //   k_attn   : scores, logits, top-N select, softmax, A.V, output
 #include <climits>
 #include <cmath>
@@ -176,34 +176,6 @@ had_status encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, u
   return HAD_OK;
 }
 
-__global__ void k_bias_minmax(const float* table, int th, int tw, int prefix, float* out) {
-  const int h = blockIdx.x;
-  const float* t = table + (size_t)h * th * tw;
-  float mn = INFINITY, mx = -INFINITY;
-  for (int e = threadIdx.x; e < th * tw; e += blockDim.x) { mn = fminf(mn, t[e]); mx = fmaxf(mx, t[e]); }
-  __shared__ float smn[32], smx[32];
-  for (int o = 16; o > 0; o >>= 1) {
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  }
-  if ((threadIdx.x & 31) == 0) { smn[threadIdx.x >> 5] = mn; smx[threadIdx.x >> 5] = mx; }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) { mn = fminf(mn, smn[w]); mx = fmaxf(mx, smx[w]); }
-    if (prefix > 0) { mn = fminf(mn, 0.0f); mx = fmaxf(mx, 0.0f); }  // class-token pairs have bias 0
-    out[2 * h] = mn;
-    out[2 * h + 1] = mx;
-  }
-}
-
-// exp(b - b_max(h)) of every table cell, the bias factor of the dense weights.
-__global__ void k_bias_exp(const float* table, int cells, const float* bminmax, float* out) {
-  const int h = blockIdx.y;
-  const float bmax = bminmax[2 * h + 1];
-  for (int e = blockIdx.x * blockDim.x + threadIdx.x; e < cells; e += gridDim.x * blockDim.x)
-    out[(size_t)h * cells + e] = exp2f((table[(size_t)h * cells + e] - bmax) * 1.4426950408889634f);
-}
-
 __global__ void k_untranspose_vq(const int8_t* vqT, int BH, int n, int n_pad, const int32_t* seqlens, int H,
                                  int8_t* Vq) {
   const size_t total = (size_t)BH * n * kD;
@@ -305,6 +277,13 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
   had_status r = HAD_OK;
   const size_t elem = (s->in_dtype == HAD_BF16) ? 2 : 4;
   const size_t head_bytes = (size_t)s->n * kD * elem;
+  BiasArgs ba{};
+  if (has_bias) {
+    ba.table = bias->table;
+    ba.th = 2 * bias->gh - 1; ba.tw = 2 * bias->gw - 1; ba.prefix = bias->prefix;
+    ba.bminmax = reinterpret_cast<float*>(ws + w.bminmax);
+    ba.expb = reinterpret_cast<float*>(ws + w.expb);
+  }
   if (head_bytes <= (size_t)kHeadMaxBytes) {
     // short heads: one read of each head, statistics and packing from shared memory
     HeadArgs ha{};
@@ -313,7 +292,8 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
     ha.B = s->B; ha.H = s->H; ha.n = s->n; ha.n_pad = dims_of(s).n_pad;
     ha.seqlens = s->seqlens;
     ha.qbits = qbits; ha.kpm = kpm; ha.vqT = vqT; ha.vscale = vscale; ha.status = status;
-    dim3 grid(dims_of(s).BH, do_v ? 3 : 2);
+    ha.bias_slice = do_v ? 3 : 2;  // the bias tables ride along as one more grid slice
+    dim3 grid(dims_of(s).BH, ha.bias_slice + (has_bias ? 1 : 0));
     const int smem = (int)head_bytes;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -331,13 +311,17 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
         attr_set[which][dev] = true;
       }
     }
-    if (which == 0) k_prep_head<__nv_bfloat16><<<grid, kHeadThreads, smem, st>>>(ha);
-    else k_prep_head<float><<<grid, kHeadThreads, smem, st>>>(ha);
+    if (which == 0) k_prep_head<__nv_bfloat16><<<grid, kHeadThreads, smem, st>>>(ha, ba);
+    else k_prep_head<float><<<grid, kHeadThreads, smem, st>>>(ha, ba);
     if ((r = check_launch("k_prep_head")) != HAD_OK) return r;
   } else {
     r = launch_prep(s, Q, K, V, 0, do_v ? 3 : 2, sums, amax, nullptr, nullptr, qbits, nullptr, nullptr, kpm, vqT,
                     vscale, st, status);
     if (r != HAD_OK) return r;
+    if (has_bias) {
+      k_bias_tables<<<s->H, 256, 0, st>>>(ba);
+      if ((r = check_launch("k_bias_tables")) != HAD_OK) return r;
+    }
   }
   if (!quant && s->in_dtype == HAD_F32 && need_v) {
     const size_t count = (size_t)dims_of(s).BH * s->n * kD;
@@ -345,15 +329,6 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
                                      reinterpret_cast<__nv_bfloat16*>(ws + w.vhi),
                                      reinterpret_cast<__nv_bfloat16*>(ws + w.vlo));
     if ((r = check_launch("k_split_v")) != HAD_OK) return r;
-  }
-  if (has_bias) {
-    float* bmm = reinterpret_cast<float*>(ws + w.bminmax);
-    const int th = 2 * bias->gh - 1, tw = 2 * bias->gw - 1;
-    k_bias_minmax<<<s->H, 256, 0, st>>>(bias->table, th, tw, bias->prefix, bmm);
-    if ((r = check_launch("k_bias_minmax")) != HAD_OK) return r;
-    k_bias_exp<<<dim3((th * tw + 255) / 256, s->H), 256, 0, st>>>(bias->table, th * tw, bmm,
-                                                                 reinterpret_cast<float*>(ws + w.expb));
-    if ((r = check_launch("k_bias_exp")) != HAD_OK) return r;
   }
   return HAD_OK;
 }

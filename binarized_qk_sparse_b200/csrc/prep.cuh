@@ -239,48 +239,124 @@ struct HeadArgs {
   int8_t* vqT;         // tensor 2 -> [BH][64][n_pad]
   float* vscale;       // [BH][64]
   unsigned* status;
+  int bias_slice;      // grid slice y == bias_slice computes the bias tables (if launched)
 };
 
+// Per-head bias range (0 included when class tokens exist: their pairs have bias
+// 0) and the table exp(b - b_max) the dense weights use; one CTA per head.
+struct BiasArgs {
+  const float* table;  // [H][th][tw] or null
+  int th, tw, prefix;
+  float* bminmax;      // [H][2]
+  float* expb;         // [H][th][tw]
+};
+
+__device__ __forceinline__ void bias_tables_block(const BiasArgs& a, int h) {
+  __shared__ float smn[32], smx[32];
+  const int cells = a.th * a.tw;
+  const float* t = a.table + (size_t)h * cells;
+  float mn = INFINITY, mx = -INFINITY;
+  for (int e = threadIdx.x; e < cells; e += blockDim.x) { mn = fminf(mn, t[e]); mx = fmaxf(mx, t[e]); }
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if ((threadIdx.x & 31) == 0) { smn[threadIdx.x >> 5] = mn; smx[threadIdx.x >> 5] = mx; }
+  __syncthreads();
+  mn = smn[0]; mx = smx[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) { mn = fminf(mn, smn[w]); mx = fmaxf(mx, smx[w]); }
+  if (a.prefix > 0) { mn = fminf(mn, 0.0f); mx = fmaxf(mx, 0.0f); }
+  if (threadIdx.x == 0) { a.bminmax[2 * h] = mn; a.bminmax[2 * h + 1] = mx; }
+  for (int e = threadIdx.x; e < cells; e += blockDim.x)
+    a.expb[(size_t)h * cells + e] = exp2f((t[e] - mx) * 1.4426950408889634f);
+}
+
+__global__ void __launch_bounds__(256) k_bias_tables(const BiasArgs a) { bias_tables_block(a, blockIdx.x); }
+
+// rint(x / sc) clamped to +-127, with x / sc the correctly rounded fp32 quotient.
+// x * (1/sc) is within 2^-15 of that quotient for |x / sc| <= 128, so it rounds
+// to the same integer unless it lies within 2^-12 of a half-integer; only then
+// is the quotient itself computed.
+__device__ __forceinline__ int quant_i8(float x, float sc, float rsc) {
+  const float y = x * rsc;
+  const float f = y - floorf(y);
+  float r;
+  if (fabsf(f - 0.5f) > 0x1p-12f) r = rintf(y);
+  else r = rintf(__fdiv_rn(x, sc));
+  r = fminf(fmaxf(r, -127.0f), 127.0f);
+  return (int)r;
+}
+
 template <typename T>
-__global__ void __launch_bounds__(kHeadThreads) k_prep_head(const HeadArgs a) {
-  extern __shared__ __align__(16) uint8_t xs[];      // [L][64] of T
-  __shared__ double part[4][kD];
-  __shared__ float stat[kD];
+__global__ void __launch_bounds__(kHeadThreads) k_prep_head(const HeadArgs a, const BiasArgs ba) {
+  if ((int)blockIdx.y == a.bias_slice) {  // the bias slice: one CTA per head
+    if ((int)blockIdx.x < a.H) bias_tables_block(ba, blockIdx.x);
+    return;
+  }
+  // The head's valid tokens, 16-byte chunk c of token i stored at chunk c ^ (i & 7)
+  // of its row, so that one thread per token (and one warp per token row) reads
+  // shared memory without bank conflicts.
+  extern __shared__ __align__(16) uint8_t xs[];
+  constexpr int kGroups = kHeadThreads / 32;
+  __shared__ double part[kGroups][kD];
+  __shared__ __align__(16) float stat[kD];
   const int bh = blockIdx.x, tz = a.first_tensor + blockIdx.y, b = bh / a.H;
   const int L = valid_len(a.seqlens, b, a.n, a.status);
   const int tid = threadIdx.x;
-  constexpr int kRow = kD * (int)sizeof(T);          // bytes per token
+  constexpr int kRow = kD * (int)sizeof(T);  // bytes per token
+  constexpr int kChunks = kRow / 16;
   const uint8_t* src = static_cast<const uint8_t*>(a.X[tz]) + (size_t)bh * a.n * kRow;
-  for (int e = tid; e < L * (kRow / 16); e += kHeadThreads) {
-    uint32_t d = (uint32_t)__cvta_generic_to_shared(xs + e * 16);
+  for (int e = tid; e < L * kChunks; e += kHeadThreads) {
+    const int i = e / kChunks, c = e % kChunks;
+    uint32_t d = (uint32_t)__cvta_generic_to_shared(xs + i * kRow + ((c ^ (i & 7)) * 16));
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(src + (size_t)e * 16));
   }
   asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
   __syncthreads();
-  auto x_at = [&](int i, int ch) -> float {
-    if (sizeof(T) == 2) return __uint_as_float((uint32_t)reinterpret_cast<const uint16_t*>(xs)[i * kD + ch] << 16);
-    return reinterpret_cast<const float*>(xs)[i * kD + ch];
+  // channels 2p and 2p+1 of token i
+  auto pair_at = [&](int i, int p) -> float2 {
+    const int byte = 2 * p * (int)sizeof(T);
+    const uint8_t* q = xs + i * kRow + (((byte >> 4) ^ (i & 7)) << 4) + (byte & 15);
+    if (sizeof(T) == 2) {
+      const uint32_t u = *reinterpret_cast<const uint32_t*>(q);
+      return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+    }
+    return *reinterpret_cast<const float2*>(q);
   };
-  // ---- channel statistic: thread (g, c) covers tokens i = g, g+4, ...
+  // ---- channel statistic: warp g covers tokens g, g + 8, ...; lane p channels 2p, 2p+1
   {
-    const int ch = tid & (kD - 1), g = tid >> 6;
+    const int p = tid & 31, g = tid >> 5;
     if (tz < 2) {
-      double acc = 0.0;
-      for (int i = g; i < L; i += 4) acc += (double)x_at(i, ch);
-      part[g][ch] = acc;
+      double s0 = 0.0, s1 = 0.0;
+      for (int i = g; i < L; i += kGroups) {
+        const float2 x = pair_at(i, p);
+        s0 += (double)x.x;
+        s1 += (double)x.y;
+      }
+      part[g][2 * p] = s0;
+      part[g][2 * p + 1] = s1;
     } else {
-      float mx = 0.0f;
-      for (int i = g; i < L; i += 4) mx = fmaxf(mx, fabsf(x_at(i, ch)));
-      part[g][ch] = (double)mx;
+      float m0 = 0.0f, m1 = 0.0f;
+      for (int i = g; i < L; i += kGroups) {
+        const float2 x = pair_at(i, p);
+        m0 = fmaxf(m0, fabsf(x.x));
+        m1 = fmaxf(m1, fabsf(x.y));
+      }
+      part[g][2 * p] = (double)m0;
+      part[g][2 * p + 1] = (double)m1;
     }
   }
   __syncthreads();
   if (tid < kD) {
     if (tz < 2) {
-      const double s = ((part[0][tid] + part[1][tid]) + part[2][tid]) + part[3][tid];
+      double s = 0.0;
+#pragma unroll
+      for (int g = 0; g < kGroups; ++g) s += part[g][tid];
       stat[tid] = (L > 0) ? __double2float_rn(s / (double)L) : 0.0f;
     } else {
-      const float mx = fmaxf(fmaxf((float)part[0][tid], (float)part[1][tid]), fmaxf((float)part[2][tid], (float)part[3][tid]));
+      float mx = 0.0f;
+#pragma unroll
+      for (int g = 0; g < kGroups; ++g) mx = fmaxf(mx, (float)part[g][tid]);
       const float sc = (mx > 0.0f) ? __fdiv_rn(mx, 127.0f) : 1.0f;
       stat[tid] = sc;
       a.vscale[(size_t)bh * kD + tid] = sc;
@@ -288,46 +364,68 @@ __global__ void __launch_bounds__(kHeadThreads) k_prep_head(const HeadArgs a) {
   }
   __syncthreads();
   if (tz < 2) {
-    // one thread per token: sign bits against the means
-    for (int i = tid; i < (tz == 0 ? a.n : a.n_pad); i += kHeadThreads) {
-      uint32_t w0 = 0, w1 = 0;
+    // one thread per token: 64 sign bits against the means (bit 1: x < mu)
+    const int ntok = (tz == 0) ? a.n : a.n_pad;
+    for (int i = tid; i < ntok; i += kHeadThreads) {
+      uint32_t w[2] = {0u, 0u};
       if (i < L) {
-#pragma unroll 8
-        for (int ch = 0; ch < 32; ++ch) {
-          w0 |= (x_at(i, ch) < stat[ch] ? 1u : 0u) << ch;
-          w1 |= (x_at(i, ch + 32) < stat[ch + 32] ? 1u : 0u) << ch;
+#pragma unroll
+        for (int c = 0; c < kChunks; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(xs + i * kRow + ((c ^ (i & 7)) << 4));
+          const uint32_t u[4] = {v.x, v.y, v.z, v.w};
+          if (sizeof(T) == 2) {
+            const float4 m0 = *reinterpret_cast<const float4*>(stat + 8 * c);
+            const float4 m1 = *reinterpret_cast<const float4*>(stat + 8 * c + 4);
+            const float mu[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float x = (e & 1) ? __uint_as_float(u[e >> 1] & 0xFFFF0000u) : __uint_as_float(u[e >> 1] << 16);
+              const int ch = 8 * c + e;
+              w[ch >> 5] |= (x < mu[e] ? 1u : 0u) << (ch & 31);
+            }
+          } else {
+            const float4 m0 = *reinterpret_cast<const float4*>(stat + 4 * c);
+            const float mu[4] = {m0.x, m0.y, m0.z, m0.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int ch = 4 * c + e;
+              w[ch >> 5] |= (__uint_as_float(u[e]) < mu[e] ? 1u : 0u) << (ch & 31);
+            }
+          }
         }
       }
       if (tz == 0) {
-        *reinterpret_cast<uint2*>(a.qbits + ((size_t)bh * a.n + i) * kW) = make_uint2(w0, w1);
+        *reinterpret_cast<uint2*>(a.qbits + ((size_t)bh * a.n + i) * kW) = make_uint2(w[0], w[1]);
       } else {
+        // +-1 int8 row of K (bit 1 -> -1); rows past L are +1
         uint4* dst = reinterpret_cast<uint4*>(a.kpm + ((size_t)bh * a.n_pad + i) * kD);
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const uint32_t f = (q < 2 ? w0 : w1) >> ((q & 1) * 16);
+          const uint32_t f = w[q >> 1] >> ((q & 1) * 16);
           dst[q] = make_uint4(expand_nibble_pm1(f & 15u), expand_nibble_pm1((f >> 4) & 15u),
                               expand_nibble_pm1((f >> 8) & 15u), expand_nibble_pm1((f >> 12) & 15u));
         }
       }
     }
   } else {
-    // thread (channel, block of 16 tokens): int8 V^T row segments of 16 bytes
-    const int ch = tid & (kD - 1);
-    const float sc = stat[ch];
-    for (int blk = tid >> 6; blk * 16 < a.n_pad; blk += kHeadThreads / kD) {
-      uint32_t w[4] = {0u, 0u, 0u, 0u};
+    // thread (channel pair, block of 16 tokens): two int8 V^T row segments of 16 bytes
+    const int p = tid & 31;
+    const float sc0 = stat[2 * p], sc1 = stat[2 * p + 1];
+    const float r0 = 1.0f / sc0, r1 = 1.0f / sc1;
+    for (int blk = tid >> 5; blk * 16 < a.n_pad; blk += kGroups) {
+      uint32_t w0[4] = {0u, 0u, 0u, 0u}, w1[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const int i = blk * 16 + u;
-        int q = 0;
         if (i < L) {
-          float r = rintf(__fdiv_rn(x_at(i, ch), sc));
-          r = fminf(fmaxf(r, -127.0f), 127.0f);
-          q = (int)r;
+          const float2 x = pair_at(i, p);
+          w0[u >> 2] |= ((uint32_t)quant_i8(x.x, sc0, r0) & 0xFFu) << (8 * (u & 3));
+          w1[u >> 2] |= ((uint32_t)quant_i8(x.y, sc1, r1) & 0xFFu) << (8 * (u & 3));
         }
-        w[u >> 2] |= ((uint32_t)q & 0xFFu) << (8 * (u & 3));
       }
-      *reinterpret_cast<uint4*>(a.vqT + ((size_t)bh * kD + ch) * a.n_pad + blk * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      int8_t* base = a.vqT + ((size_t)bh * kD + 2 * p) * a.n_pad + blk * 16;
+      *reinterpret_cast<uint4*>(base) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+      *reinterpret_cast<uint4*>(base + a.n_pad) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
     }
   }
 }
