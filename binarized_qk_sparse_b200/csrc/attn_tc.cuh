@@ -61,9 +61,7 @@ constexpr int kKoffTable = 0;    // per-head table in shared memory (n_pad <= kK
 constexpr int kKoffLinear = 1;   // prefix 0 and gw a multiple of 64: koff(j0 + u) = koff(j0) + u within a tile
 constexpr int kKoffTile = 2;     // computed per tile (double-buffered, one named barrier per tile)
 constexpr int kKoffTableMax = 1024;
-constexpr int kKoffClass = INT_MIN;        // key is a class token: bias 0
-constexpr int kKoffInvalid = INT_MIN + 1;  // key at or past the valid length: never kept
-constexpr int kBiasSmemMax = 4096;         // exp(bias) tables up to this many entries are staged in shared memory
+constexpr int kBiasSmemMax = 4096;  // extended exp(bias) tables up to this many entries are staged in shared memory
 
 enum { SEL_DENSE = 0, SEL_TOPN_INT = 1, SEL_TOPN_FLOAT = 2 };
 enum { MODE_F = 0, MODE_Q = 1 };
@@ -80,7 +78,9 @@ struct TcArgs {
   const float* table;      // [H][th][tw] or null
   int gh, gw, prefix, th, tw;
   const float* bminmax;    // [H][2] min/max of each head's table (0 included with class tokens)
-  const float* expb;       // [H][th][tw] exp(b - b_max(h)), or null
+  const float* expb;       // [H][E] extended exp(b - b_max(h)) table, or null
+  const float* bext;       // [H][E] extended bias table, or null
+  int ext_E, rb_class, k_class, k_invalid;  // extended-table geometry (RelposExt)
   int int_levels;          // 1 if fp32(c*s) is strictly increasing in s for every head
   int koff_mode;           // kKoffTable / kKoffLinear / kKoffTile
   int bias_smem;           // 1: stage this head's exp(bias) table in shared memory
@@ -129,12 +129,24 @@ enum {
 };
 
 // Bias offset of key j: koff = y_j * tw + x_j for patch tokens, so that
-// b_ij = table[row_base(i) - koff]; class tokens and keys past L get a sentinel.
-__device__ __forceinline__ int key_offset(int j, int L, int prefix, int gw, int tw) {
-  if (j >= L) return kKoffInvalid;
-  if (j < prefix) return kKoffClass;
-  const int t = j - prefix;
-  return (t / gw) * tw + t % gw;
+// b_ij = ext[rb(i) - koff(j)]; class tokens and keys past L index the extension.
+__device__ __forceinline__ int key_offset(const TcArgs& a, int j, int L) {
+  if (j >= L) return a.k_invalid;
+  if (j < a.prefix) return a.k_class;
+  const int t = j - a.prefix;
+  return (t / a.gw) * a.tw + t % a.gw;
+}
+
+// Pairwise sum of 32 values (a depth-5 tree instead of a 32-long dependent chain).
+__device__ __forceinline__ float sum32(const float (&e)[32]) {
+  float t[16];
+#pragma unroll
+  for (int u = 0; u < 16; ++u) t[u] = e[2 * u] + e[2 * u + 1];
+#pragma unroll
+  for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+    for (int u = 0; u < w; ++u) t[u] = t[2 * u] + t[2 * u + 1];
+  return t[0];
 }
 
 template <int SEL, int MODE, bool HAS_BIAS, bool VF32, int EXPORT>
@@ -231,11 +243,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
     }
     if (MODE == MODE_Q && EXPORT == EXP_NONE && tid < kD) dq[tid] = __fdiv_rn(a.vscale[(size_t)bh * kD + tid], 255.0f);
     if (HAS_BIAS && a.koff_mode == kKoffTable)
-      for (int j = tid; j < a.n_pad; j += kM) koff_tab[j] = key_offset(j, L, a.prefix, a.gw, a.tw);
+      for (int j = tid; j < a.n_pad; j += kM) koff_tab[j] = key_offset(a, j, L);
     if (HAS_BIAS && SEL == SEL_DENSE && a.bias_smem) {
-      const float* src = a.expb + (size_t)h * a.th * a.tw;
+      const float* src = a.expb + (size_t)h * a.ext_E;
       float* dst = reinterpret_cast<float*>(sm + SM::kBiasTab);
-      for (int i = tid; i < a.th * a.tw; i += kM) dst[i] = __ldg(src + i);
+      for (int i = tid; i < a.ext_E; i += kM) dst[i] = __ldg(src + i);
     }
     fence_proxy_async();
   }
@@ -249,21 +261,24 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
   int rF = 0, cut = 0, tie_seen = 0, kept_seen = 0;
   uint32_t r_uhi = 0, r_span = 0;
   int r_shift = 0, r_rank = 0, r_state = 0, r_bin = 0, r_cnt = 0;
-  int rb = -1;
-  if (HAS_BIAS && tid < kM && row >= a.prefix && row < a.n) {
-    const int t = row - a.prefix;
-    rb = (t / a.gw + a.gh - 1) * a.tw + (t % a.gw + a.gw - 1);
+  // row base of the extended bias tables: rb(i) - koff(j) indexes the pair (i, j);
+  // class-token rows and rows past the tensor use the class-row base
+  int rb = 0;
+  if (HAS_BIAS) {
+    rb = a.rb_class;
+    if (row >= a.prefix && row < a.n) {
+      const int t = row - a.prefix;
+      rb = (t / a.gw + a.gh - 1) * a.tw + (t % a.gw + a.gw - 1);
+    }
   }
-  const float* tab = HAS_BIAS ? a.table + (size_t)h * a.th * a.tw : nullptr;
+  const float* tab = HAS_BIAS ? a.bext + (size_t)h * a.ext_E : nullptr;
   const float kLog2e = 1.4426950408889634f;
   // Dense weights as (level table) x exp(b - b_max): both factors <= 1, so no row
   // maximum is needed as long as the smallest product stays far from fp32 underflow.
-  float fb0 = 1.0f;  // factor of a class-token pair (bias 0)
   bool use_lut = false;
   if (SEL == SEL_DENSE) {
     const float range = HAS_BIAS ? a.bminmax[2 * h + 1] - a.bminmax[2 * h] : 0.0f;
     use_lut = c > 0.0f && (128.0f * c + range) * kLog2e <= 100.0f;
-    if (HAS_BIAS) fb0 = exp2f(-a.bminmax[2 * h + 1] * kLog2e);
   }
   const bool sum_in_pv = (MODE == MODE_F) && (SEL == SEL_TOPN_FLOAT || (SEL == SEL_DENSE && use_lut));
   int sF = 0;  // integer threshold score (top-N without bias)
@@ -386,6 +401,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       const uint32_t hist_row = smem_u32(hist) + (uint32_t)tid * 4u;
       const float mo = -m * kLog2e;
       const float* lut = reinterpret_cast<const float*>(hist);
+      const float* lut_lane = lut + 32 * 32 + lane;  // dense level table: entry for score s at lut_lane[-16 s]
       // Passes compiled into this instantiation (the rest are pruned at compile time).
       constexpr bool kHasLevels = SEL != SEL_DENSE;
       constexpr bool kHasNorm = SEL == SEL_DENSE;
@@ -402,7 +418,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       // exp(b - b_max) of this head: staged in shared memory when it fits (dense only)
       const float* expb_h = nullptr;
       if (HAS_BIAS && SEL == SEL_DENSE)
-        expb_h = a.bias_smem ? reinterpret_cast<const float*>(sm + SM::kBiasTab) : a.expb + (size_t)h * a.th * a.tw;
+        expb_h = a.bias_smem ? reinterpret_cast<const float*>(sm + SM::kBiasTab) : a.expb + (size_t)h * a.ext_E;
       for (int t = 0; t < ntiles; ++t) {
         const uint32_t gs = g_s + (uint32_t)t, buf = gs % kSBufs;
         const uint32_t colP = kColS + buf * kN;  // P of this tile is written over its score buffer
@@ -416,7 +432,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
           } else if (a.koff_mode == kKoffTile) {
             const uint32_t kb = gs & 1u;  // alternates across passes too
             ko = koff_tab + kb * kN;
-            if (tid < kN) koff_tab[kb * kN + tid] = key_offset(j0 + tid, L, a.prefix, a.gw, a.tw);
+            if (tid < kN) koff_tab[kb * kN + tid] = key_offset(a, j0 + tid, L);
             asm volatile("bar.sync 1, 128;" ::: "memory");
           }
         }
@@ -427,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
         tmem_ld32(tl + kColS + buf * kN + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
         tmem_wait_ld();
         const int nvalid = row_ok ? max(0, min(kN, L - j0)) : 0;
-        // Dense with bias: keys past L carry the kKoffInvalid sentinel (weight 0), and
+        // Dense with bias: keys past L carry the k_invalid offset (weight 0), and
         // rows past L are never stored, so every tile takes the unmasked path.
         constexpr bool kMaskInKoff = SEL == SEL_DENSE && HAS_BIAS;
         const bool full_tile = kMaskInKoff || __all_sync(0xffffffffu, nvalid == kN);
@@ -445,13 +461,10 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
             uint32_t wq[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-              uint32_t w = 0;
+              uint32_t q[4];
 #pragma unroll
-              for (int v = 0; v < 4; ++v) {
-                const uint32_t code = (uint32_t)min(255, (int)floorf(__fmaf_rn(e[4 * u + v], scale, 0.5f)));
-                w |= code << (8 * v);
-              }
-              wq[u] = w;
+              for (int v = 0; v < 4; ++v) q[v] = min(__float2uint_rd(__fmaf_rn(e[4 * u + v], scale, 0.5f)), 255u);
+              wq[u] = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
             }
             if (kHasCodes) {
               if (row >= a.row_begin && row < a.row_end && row < a.n) {
@@ -467,10 +480,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
           } else {
             uint32_t wp[16];
 #pragma unroll
-            for (int u = 0; u < 16; ++u) {
-              wp[u] = pack_bf16x2(e[2 * u], e[2 * u + 1]);
-              if (sum_in_pv) lsum += e[2 * u] + e[2 * u + 1];
-            }
+            for (int u = 0; u < 16; ++u) wp[u] = pack_bf16x2(e[2 * u], e[2 * u + 1]);
+            if (sum_in_pv) lsum += sum32(e);
             tmem_st16(tl + colP + 16 * ch, wp);
             if (VF32) {
               uint32_t wl[16];
@@ -513,17 +524,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
                   const int sc = (int)r[32 * ch + u + v];
-                  float x = lut[(32 - (sc >> 1)) * 32 + lane];
-                  if (HAS_BIAS) {
-                    const float special = (kk[v] == kKoffInvalid) ? 0.0f : fb0;
-                    x *= (rb >= 0 && kk[v] >= 0) ? expb_h[rb - kk[v]] : special;
-                  }
+                  float x = lut_lane[-16 * sc];  // level (64 - s) / 2 of this lane's table
+                  if (HAS_BIAS) x *= expb_h[rb - kk[v]];
                   e[u + v] = (FULL || 32 * ch + u + v < nvalid) ? x : 0.0f;
                 }
               }
               if (pass == P_NORM) {
-#pragma unroll
-                for (int u = 0; u < 32; ++u) lsum += e[u];
+                lsum += sum32(e);
               } else {
                 emit(e, ch);
               }
@@ -554,10 +561,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
                   const int sc = (int)r[32 * ch + u + v];
                   float l;
                   if (HAS_BIAS) {
-                    if (kMaskInKoff) kinv |= (kk[v] == kKoffInvalid ? 1u : 0u) << (u + v);
-                    const float special = (kk[v] == kKoffInvalid) ? -INFINITY : 0.0f;
-                    const float bv = (rb >= 0 && kk[v] >= 0) ? __ldg(tab + (rb - kk[v])) : special;
-                    l = __fmaf_rn((float)sc, c, bv);
+                    if (kMaskInKoff) kinv |= (kk[v] == a.k_invalid ? 1u : 0u) << (u + v);
+                    l = __fmaf_rn((float)sc, c, __ldg(tab + (rb - kk[v])));
                   } else {
                     l = (float)sc * c;
                   }
@@ -573,8 +578,10 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
                   m = tm;
                 }
                 const float mo2 = -m * kLog2e;
+                float ex[32];
 #pragma unroll
-                for (int u = 0; u < 32; ++u) lsum += fast_exp2(__fmaf_rn(lg[u], kLog2e, mo2));
+                for (int u = 0; u < 32; ++u) ex[u] = fast_exp2(__fmaf_rn(lg[u], kLog2e, mo2));
+                lsum += sum32(ex);
               } else if (kHasRadix && pass == P_RADIX) {
                 if (r_state == 1) {
 #pragma unroll
@@ -613,9 +620,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
                   keepm |= (k ? 1u : 0u) << u;
                 }
                 if (kHasKeptNorm && pass == P_KEPT_NORM) {
+                  float ex[32];
 #pragma unroll
                   for (int u = 0; u < 32; ++u)
-                    lsum += ((keepm >> u) & 1u) ? fast_exp2(__fmaf_rn(lg[u], kLog2e, mo)) : 0.0f;
+                    ex[u] = ((keepm >> u) & 1u) ? fast_exp2(__fmaf_rn(lg[u], kLog2e, mo)) : 0.0f;
+                  lsum += sum32(ex);
                 } else if (kHasIdx && pass == P_IDX) {
                   if (row_ok) {
                     int32_t* dst = a.idx + ((size_t)bh * a.n + row) * a.N;

@@ -24,6 +24,31 @@ __device__ __forceinline__ void raise_status(unsigned* status, unsigned bits) {
 
 // Valid length of sequence b; an out-of-range entry raises the device status
 // and returns 0, which makes every kernel treat that batch as empty (zero output).
+// Extended relative-position tables.  Entry rb(i) - koff(j) of the raw
+// (2gh-1) x (2gw-1) table is the bias of patch query i and patch key j.  The
+// extension appends regions that the same subtraction reaches for class-token
+// queries (rb = rb_class), class-token keys (koff = k_class) and keys at or past
+// the valid length (koff = k_invalid), so a kernel reads one table entry per
+// (query, key) pair with no case analysis:
+//   [0, T)              the table, T = (2gh-1)(2gw-1)
+//   [T, 2T + 2Kx)       class-token pairs (bias 0)
+//   [2T + 2Kx, 3T + 3Kx) keys past L (weight 0 / logit -inf)
+// with Kx = (gh-1)(2gw-1) + gw the number of distinct patch key offsets.
+struct RelposExt {
+  int T, Kx, E, rb_class, k_class, k_invalid;
+};
+__host__ __device__ inline RelposExt relpos_ext(int gh, int gw) {
+  RelposExt r;
+  const int tw = 2 * gw - 1;
+  r.T = (2 * gh - 1) * tw;
+  r.Kx = (gh - 1) * tw + gw;
+  r.E = 3 * r.T + 3 * r.Kx;
+  r.rb_class = r.T - 1 + r.Kx;
+  r.k_class = -(r.T + r.Kx);
+  r.k_invalid = -(2 * r.T + 2 * r.Kx);
+  return r;
+}
+
 __device__ __forceinline__ int valid_len(const int32_t* seqlens, int b, int n, unsigned* status) {
   if (!seqlens) return n;
   int L = seqlens[b];

@@ -96,7 +96,7 @@ had_status check_bias(const had_shape* s, const had_relpos_bias* bias) {
 }
 
 struct Ws {
-  size_t qbits, kpm, sums, amax, vqT, vscale, bminmax, expb, vhi, vlo, total;
+  size_t qbits, kpm, sums, amax, vqT, vscale, bminmax, bext, expb, vhi, vlo, total;
 };
 
 Ws ws_layout(const had_shape* s, bool quant, const had_relpos_bias* bias_desc) {
@@ -113,10 +113,11 @@ Ws ws_layout(const had_shape* s, bool quant, const had_relpos_bias* bias_desc) {
     w.vqT = off; off += align_up((size_t)d.BH * kD * d.n_pad);
     w.vscale = off; off += align_up((size_t)d.BH * kD * 4);
   }
-  w.expb = 0;
+  w.bext = w.expb = 0;
   if (bias) {
     w.bminmax = off; off += align_up((size_t)s->H * 2 * 4);
-    const size_t cells = (size_t)(2 * bias_desc->gh - 1) * (size_t)(2 * bias_desc->gw - 1);
+    const size_t cells = (size_t)relpos_ext(bias_desc->gh, bias_desc->gw).E;
+    w.bext = off; off += align_up((size_t)s->H * cells * 4);
     w.expb = off; off += align_up((size_t)s->H * cells * 4);
   }
   w.vhi = w.vlo = 0;
@@ -280,8 +281,9 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
   BiasArgs ba{};
   if (has_bias) {
     ba.table = bias->table;
-    ba.th = 2 * bias->gh - 1; ba.tw = 2 * bias->gw - 1; ba.prefix = bias->prefix;
+    ba.gh = bias->gh; ba.gw = bias->gw; ba.prefix = bias->prefix;
     ba.bminmax = reinterpret_cast<float*>(ws + w.bminmax);
+    ba.bext = reinterpret_cast<float*>(ws + w.bext);
     ba.expb = reinterpret_cast<float*>(ws + w.expb);
   }
   if (head_bytes <= (size_t)kHeadMaxBytes) {
@@ -424,6 +426,11 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
   }
   a.bminmax = has_bias ? reinterpret_cast<float*>(ws + w.bminmax) : nullptr;
   a.expb = has_bias ? reinterpret_cast<float*>(ws + w.expb) : nullptr;
+  a.bext = has_bias ? reinterpret_cast<float*>(ws + w.bext) : nullptr;
+  if (has_bias) {
+    const RelposExt x = relpos_ext(bias->gh, bias->gw);
+    a.ext_E = x.E; a.rb_class = x.rb_class; a.k_class = x.k_class; a.k_invalid = x.k_invalid;
+  }
   a.seqlens = s->seqlens;
   a.O = O; a.o_bf16 = (o_dtype == HAD_BF16) ? 1 : 0;
   a.idx = idx; a.codes = codes; a.row_begin = row_begin; a.row_end = row_end;
@@ -434,7 +441,7 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
     if (d.n_pad <= tc::kKoffTableMax) a.koff_mode = tc::kKoffTable;
     else if (bias->prefix == 0 && bias->gw % tc::kN == 0 && s->seqlens == nullptr) a.koff_mode = tc::kKoffLinear;
   }
-  a.bias_smem = (has_bias && a.th * a.tw <= tc::kBiasSmemMax) ? 1 : 0;
+  a.bias_smem = (has_bias && a.ext_E <= tc::kBiasSmemMax) ? 1 : 0;
   a.int_levels = 1;
   for (int h = 0; h < s->H; ++h) {
     const double aq = alpha_q ? (double)alpha_q[h] : 1.0, ak = alpha_k ? (double)alpha_k[h] : 1.0;

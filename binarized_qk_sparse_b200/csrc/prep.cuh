@@ -243,20 +243,23 @@ struct HeadArgs {
 };
 
 // Per-head bias range (0 included when class tokens exist: their pairs have bias
-// 0) and the table exp(b - b_max) the dense weights use; one CTA per head.
+// 0) and the two extended tables (see RelposExt) the attention kernel reads:
+// the bias itself (class pairs 0, keys past L -inf) and exp(b - b_max) (class
+// pairs exp(-b_max), keys past L 0).  One CTA per head.
 struct BiasArgs {
-  const float* table;  // [H][th][tw] or null
-  int th, tw, prefix;
+  const float* table;  // [H][2gh-1][2gw-1] or null
+  int gh, gw, prefix;
   float* bminmax;      // [H][2]
-  float* expb;         // [H][th][tw]
+  float* bext;         // [H][E]
+  float* expb;         // [H][E]
 };
 
 __device__ __forceinline__ void bias_tables_block(const BiasArgs& a, int h) {
   __shared__ float smn[32], smx[32];
-  const int cells = a.th * a.tw;
-  const float* t = a.table + (size_t)h * cells;
+  const RelposExt x = relpos_ext(a.gh, a.gw);
+  const float* t = a.table + (size_t)h * x.T;
   float mn = INFINITY, mx = -INFINITY;
-  for (int e = threadIdx.x; e < cells; e += blockDim.x) { mn = fminf(mn, t[e]); mx = fmaxf(mx, t[e]); }
+  for (int e = threadIdx.x; e < x.T; e += blockDim.x) { mn = fminf(mn, t[e]); mx = fmaxf(mx, t[e]); }
   for (int o = 16; o > 0; o >>= 1) {
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -267,8 +270,19 @@ __device__ __forceinline__ void bias_tables_block(const BiasArgs& a, int h) {
   for (int w = 1; w < (int)(blockDim.x >> 5); ++w) { mn = fminf(mn, smn[w]); mx = fmaxf(mx, smx[w]); }
   if (a.prefix > 0) { mn = fminf(mn, 0.0f); mx = fmaxf(mx, 0.0f); }
   if (threadIdx.x == 0) { a.bminmax[2 * h] = mn; a.bminmax[2 * h + 1] = mx; }
-  for (int e = threadIdx.x; e < cells; e += blockDim.x)
-    a.expb[(size_t)h * cells + e] = exp2f((t[e] - mx) * 1.4426950408889634f);
+  const float kLog2e = 1.4426950408889634f;
+  const float e_class = exp2f((0.0f - mx) * kLog2e);
+  float* be = a.bext + (size_t)h * x.E;
+  float* ee = a.expb + (size_t)h * x.E;
+  const int z0 = 2 * x.T + 2 * x.Kx;
+  for (int e = threadIdx.x; e < x.E; e += blockDim.x) {
+    float b, w;
+    if (e < x.T) { b = t[e]; w = exp2f((b - mx) * kLog2e); }
+    else if (e < z0) { b = 0.0f; w = e_class; }
+    else { b = -INFINITY; w = 0.0f; }
+    be[e] = b;
+    ee[e] = w;
+  }
 }
 
 __global__ void __launch_bounds__(256) k_bias_tables(const BiasArgs a) { bias_tables_block(a, blockIdx.x); }
