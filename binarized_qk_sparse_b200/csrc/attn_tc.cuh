@@ -57,10 +57,12 @@ constexpr int kSBufs = 3;
 constexpr uint32_t kColS = 0, kColO = 192, kTmemCols = 256;
 constexpr long long kWaitCycles = 2000000000LL;  // about one second
 // How the softmax threads find the bias offset koff(j) = y_j * tw + x_j of a key:
-constexpr int kKoffTable = 0;    // per-head table in shared memory (n_pad <= kKoffTableMax)
-constexpr int kKoffLinear = 1;   // prefix 0 and gw a multiple of 64: koff(j0 + u) = koff(j0) + u within a tile
-constexpr int kKoffTile = 2;     // computed per tile (double-buffered, one named barrier per tile)
+constexpr int kKoffTable = 0;  // per-head table in shared memory (n_pad <= kKoffTableMax)
+constexpr int kKoffWarp = 1;   // each softmax warp computes the tile's 64 offsets (double-buffered)
 constexpr int kKoffTableMax = 1024;
+// Bias variants of the kernel: none, extended tables read from global memory,
+// or (dense) the exp(bias) table staged in shared memory.
+enum { BIAS_NONE = 0, BIAS_GLOBAL = 1, BIAS_SMEM = 2 };
 constexpr int kBiasSmemMax = 4096;  // extended exp(bias) tables up to this many entries are staged in shared memory
 
 enum { SEL_DENSE = 0, SEL_TOPN_INT = 1, SEL_TOPN_FLOAT = 2 };
@@ -82,8 +84,7 @@ struct TcArgs {
   const float* bext;       // [H][E] extended bias table, or null
   int ext_E, rb_class, k_class, k_invalid;  // extended-table geometry (RelposExt)
   int int_levels;          // 1 if fp32(c*s) is strictly increasing in s for every head
-  int koff_mode;           // kKoffTable / kKoffLinear / kKoffTile
-  int bias_smem;           // 1: stage this head's exp(bias) table in shared memory
+  int koff_mode;           // kKoffTable / kKoffWarp
   const int32_t* seqlens;
   void* O;
   int o_bf16;
@@ -96,15 +97,16 @@ struct TcArgs {
 };
 
 // Shared memory carve-up (offsets from a 1024-byte aligned base).
-template <int SEL, bool VF32, bool HAS_BIAS>
+template <int SEL, bool VF32, int BIAS>
 struct Smem {
+  static constexpr bool HAS_BIAS = BIAS != BIAS_NONE;
   static constexpr int kVStage = (VF32 ? 2 : 1) * kN * kD * 2;   // bf16 V tile (+ residual tile)
   static constexpr int kQ = 0;                                   // 128 x 64 B
   static constexpr int kK = kQ + kM * kD;                        // 4 x 4 KB
   static constexpr int kV = kK + kKStages * kN * kD;             // 2 V stages
-  static constexpr int kKoff = kV + kVStages * kVStage;          // bias key offsets (table or 2 x 64)
+  static constexpr int kKoff = kV + kVStages * kVStage;          // bias key offsets (table, or 4 warps x 2 x 64)
   static constexpr int kBiasTab = kKoff + (HAS_BIAS ? kKoffTableMax * 4 : 0);  // exp(bias) table (dense)
-  static constexpr int kDq = kBiasTab + ((HAS_BIAS && SEL == SEL_DENSE) ? kBiasSmemMax * 4 : 0);  // 64 dequant scales
+  static constexpr int kDq = kBiasTab + (BIAS == BIAS_SMEM ? kBiasSmemMax * 4 : 0);  // 64 dequant scales
   static constexpr int kBar = kDq + kD * 4;
   static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 2 * kSBufs + 2;
   static constexpr int kMisc = kBar + kNumBars * 8;              // [0] tmem base [1] abort
@@ -149,9 +151,11 @@ __device__ __forceinline__ float sum32(const float (&e)[32]) {
   return t[0];
 }
 
-template <int SEL, int MODE, bool HAS_BIAS, bool VF32, int EXPORT>
+template <int SEL, int MODE, int BIAS, bool VF32, int EXPORT>
 __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__ TcArgs a) {
-  using SM = Smem<SEL, VF32, HAS_BIAS>;
+  static_assert(BIAS != BIAS_SMEM || SEL == SEL_DENSE, "staged exp(bias) tables serve the dense weights only");
+  constexpr bool HAS_BIAS = BIAS != BIAS_NONE;
+  using SM = Smem<SEL, VF32, BIAS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
     if (MODE == MODE_Q && EXPORT == EXP_NONE && tid < kD) dq[tid] = __fdiv_rn(a.vscale[(size_t)bh * kD + tid], 255.0f);
     if (HAS_BIAS && a.koff_mode == kKoffTable)
       for (int j = tid; j < a.n_pad; j += kM) koff_tab[j] = key_offset(a, j, L);
-    if (HAS_BIAS && SEL == SEL_DENSE && a.bias_smem) {
+    if (BIAS == BIAS_SMEM) {
       const float* src = a.expb + (size_t)h * a.ext_E;
       float* dst = reinterpret_cast<float*>(sm + SM::kBiasTab);
       for (int i = tid; i < a.ext_E; i += kM) dst[i] = __ldg(src + i);
@@ -415,29 +419,56 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       const bool lut_e = (SEL == SEL_DENSE) && use_lut && (pass == P_NORM || pass == P_PV || pass == P_CODES);
       const bool lut_w = (SEL == SEL_TOPN_INT) && a.int_levels && pass == P_PV;
       const bool wants_bias = HAS_BIAS && pass != P_LEVELS;
-      // exp(b - b_max) of this head: staged in shared memory when it fits (dense only)
-      const float* expb_h = nullptr;
-      if (HAS_BIAS && SEL == SEL_DENSE)
-        expb_h = a.bias_smem ? reinterpret_cast<const float*>(sm + SM::kBiasTab) : a.expb + (size_t)h * a.ext_E;
+      // exp(b - b_max) of this row (dense): row base rb(i) into the staged or global table
+      const float* eb_row = nullptr;
+      if (BIAS == BIAS_SMEM) eb_row = reinterpret_cast<const float*>(sm + SM::kBiasTab) + rb;
+      else if (HAS_BIAS && SEL == SEL_DENSE) eb_row = a.expb + (size_t)h * a.ext_E + rb;
+      // a warp whose 32 rows all lie past L only keeps the barrier phases going
+      const bool warp_live = __any_sync(0xffffffffu, row < L);
+      // per-warp offsets: patch (y, x) of keys j0 + lane and j0 + 32 + lane, advanced
+      // by 64 keys per tile without a division
+      int ya = 0, xa = 0, yb = 0, xb = 0;
+      const int q64 = HAS_BIAS ? kN / a.gw : 0, r64 = HAS_BIAS ? kN % a.gw : 0;
+      auto patch_of = [&](int j, int& y, int& x) {
+        const int tt = max(j - a.prefix, 0);
+        y = tt / a.gw;
+        x = tt - y * a.gw;
+      };
+      auto advance = [&](int& y, int& x) {
+        y += q64;
+        x += r64;
+        if (x >= a.gw) { x -= a.gw; ++y; }
+      };
+      auto offset_of = [&](int j, int y, int x) -> int {
+        return j >= L ? a.k_invalid : (j < a.prefix ? a.k_class : y * a.tw + x);
+      };
       for (int t = 0; t < ntiles; ++t) {
         const uint32_t gs = g_s + (uint32_t)t, buf = gs % kSBufs;
         const uint32_t colP = kColS + buf * kN;  // P of this tile is written over its score buffer
         const int j0 = t * kN;
-        // bias offsets of this tile's keys: per-head table, closed form, or computed per tile
+        // bias offsets of this tile's keys: per-head table, or computed by this warp
         const int* ko = koff_tab + j0;
-        int lin_base = 0;
-        if (wants_bias) {
-          if (a.koff_mode == kKoffLinear) {
-            lin_base = (j0 / a.gw) * a.tw + j0 % a.gw;
-          } else if (a.koff_mode == kKoffTile) {
-            const uint32_t kb = gs & 1u;  // alternates across passes too
-            ko = koff_tab + kb * kN;
-            if (tid < kN) koff_tab[kb * kN + tid] = key_offset(a, j0 + tid, L);
-            asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (wants_bias && warp_live && a.koff_mode == kKoffWarp) {
+          int* wk = koff_tab + (warp * 2 + (int)(gs & 1u)) * kN;  // alternates across passes too
+          if (j0 < a.prefix + kN) {
+            patch_of(j0 + lane, ya, xa);
+            patch_of(j0 + 32 + lane, yb, xb);
+          } else {
+            advance(ya, xa);
+            advance(yb, xb);
           }
+          wk[lane] = offset_of(j0 + lane, ya, xa);
+          wk[lane + 32] = offset_of(j0 + 32 + lane, yb, xb);
+          __syncwarp();
+          ko = wk;
         }
         const bool ok_wait = __all_sync(0xffffffffu, bounded_wait(B_SFULL + buf, (gs / kSBufs) & 1));
         tc_fence_after();
+        if (!warp_live) {
+          tc_fence_before();
+          mbar_arrive(&bars[B_TDONE + buf]);
+          continue;
+        }
         uint32_t r[64];
         tmem_ld32(tl + kColS + buf * kN, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
         tmem_ld32(tl + kColS + buf * kN + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
@@ -449,10 +480,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
         const bool full_tile = kMaskInKoff || __all_sync(0xffffffffu, nvalid == kN);
 
         // bias offsets of keys 32*ch+u .. +3 of this tile
-        auto koff4 = [&](int idx) -> int4 {
-          if (a.koff_mode == kKoffLinear) return make_int4(lin_base + idx, lin_base + idx + 1, lin_base + idx + 2, lin_base + idx + 3);
-          return *reinterpret_cast<const int4*>(ko + idx);
-        };
+        auto koff4 = [&](int idx) -> int4 { return *reinterpret_cast<const int4*>(ko + idx); };
 
         // ---- P (or uint8 A) of one 32-key chunk into TMEM, or codes to global (export)
         auto emit = [&](const float (&e)[32], int ch) {
@@ -500,6 +528,20 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
 #pragma unroll
           for (int ch = 0; ch < 2; ++ch) {
             const int jb = j0 + 32 * ch;
+            if (jb >= L && pass != P_CODES) {
+              // every key of the chunk lies past L: nothing to count or sum; P is 0
+              if (pv) {
+                if (MODE == MODE_Q) {
+                  const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                  tmem_st8(tl + colP + 8 * ch, z);
+                } else {
+                  const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                  tmem_st16(tl + colP + 16 * ch, z);
+                  if (VF32) tmem_st16(tl + colP + 32 + 16 * ch, z);
+                }
+              }
+              continue;
+            }
             if (kHasLevels && pass == P_LEVELS) {
               const uint32_t base = hist_row + 32u * kM * 4u;  // level (64 - s)/2 -> + (64 - s) * 256 bytes
 #pragma unroll
@@ -525,7 +567,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
                 for (int v = 0; v < 4; ++v) {
                   const int sc = (int)r[32 * ch + u + v];
                   float x = lut_lane[-16 * sc];  // level (64 - s) / 2 of this lane's table
-                  if (HAS_BIAS) x *= expb_h[rb - kk[v]];
+                  if (BIAS == BIAS_SMEM) x *= eb_row[-kk[v]];
+                  else if (HAS_BIAS) x *= __ldg(eb_row - kk[v]);
                   e[u + v] = (FULL || 32 * ch + u + v < nvalid) ? x : 0.0f;
                 }
               }

@@ -335,7 +335,7 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
   return HAD_OK;
 }
 
-template <int SEL, int MODE, bool BIAS, bool VF32, int EXP>
+template <int SEL, int MODE, int BIAS, bool VF32, int EXP>
 had_status launch_tc_t(const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
   const int smem = tc::Smem<SEL, VF32, BIAS>::kTotal;
   auto fn = tc::k_attn_tc<SEL, MODE, BIAS, VF32, EXP>;
@@ -355,33 +355,37 @@ had_status launch_tc_t(const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
   return check_launch("k_attn_tc");
 }
 
+// Dense: no bias, extended tables in global memory, or the exp(bias) table staged in shared memory.
 template <int SEL, int MODE, bool VF32, int EXP>
-had_status launch_tc_b(bool bias, const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
-  return bias ? launch_tc_t<SEL, MODE, true, VF32, EXP>(a, grid, st) : launch_tc_t<SEL, MODE, false, VF32, EXP>(a, grid, st);
+had_status launch_tc_b(int bias, const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
+  using namespace tc;
+  if (bias == BIAS_SMEM) return launch_tc_t<SEL, MODE, BIAS_SMEM, VF32, EXP>(a, grid, st);
+  if (bias == BIAS_GLOBAL) return launch_tc_t<SEL, MODE, BIAS_GLOBAL, VF32, EXP>(a, grid, st);
+  return launch_tc_t<SEL, MODE, BIAS_NONE, VF32, EXP>(a, grid, st);
 }
 
 template <int EXP>
-had_status dispatch_tc(int sel, int mode, bool bias, bool vf32, const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
+had_status dispatch_tc(int sel, int mode, int bias, bool vf32, const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
   using namespace tc;
   if (EXP == EXP_CODES || (EXP == EXP_NONE && mode == MODE_Q)) {
     constexpr int E = EXP;
     if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_Q, false, E>(bias, a, grid, st);
-    if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_Q, false, false, E>(a, grid, st);
-    return launch_tc_t<SEL_TOPN_FLOAT, MODE_Q, true, false, E>(a, grid, st);
+    if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_Q, BIAS_NONE, false, E>(a, grid, st);
+    return launch_tc_t<SEL_TOPN_FLOAT, MODE_Q, BIAS_GLOBAL, false, E>(a, grid, st);
   }
   if (EXP == EXP_IDX) {
     if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, false, EXP>(bias, a, grid, st);
-    if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, false, false, EXP>(a, grid, st);
-    return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, true, false, EXP>(a, grid, st);
+    if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, BIAS_NONE, false, EXP>(a, grid, st);
+    return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, BIAS_GLOBAL, false, EXP>(a, grid, st);
   }
   if (vf32) {
     if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, true, EXP>(bias, a, grid, st);
-    if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, false, true, EXP>(a, grid, st);
-    return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, true, true, EXP>(a, grid, st);
+    if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, BIAS_NONE, true, EXP>(a, grid, st);
+    return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, BIAS_GLOBAL, true, EXP>(a, grid, st);
   }
   if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, false, EXP>(bias, a, grid, st);
-  if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, false, false, EXP>(a, grid, st);
-  return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, true, false, EXP>(a, grid, st);
+  if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, BIAS_NONE, false, EXP>(a, grid, st);
+  return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, BIAS_GLOBAL, false, EXP>(a, grid, st);
 }
 
 // Stage 2: the fused kernel over a prepared workspace.
@@ -436,12 +440,8 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
   a.idx = idx; a.codes = codes; a.row_begin = row_begin; a.row_end = row_end;
   a.B = d.B; a.H = d.H; a.n = d.n; a.n_pad = d.n_pad; a.N = N;
   a.status = status;
-  a.koff_mode = tc::kKoffTile;
-  if (has_bias) {
-    if (d.n_pad <= tc::kKoffTableMax) a.koff_mode = tc::kKoffTable;
-    else if (bias->prefix == 0 && bias->gw % tc::kN == 0 && s->seqlens == nullptr) a.koff_mode = tc::kKoffLinear;
-  }
-  a.bias_smem = (has_bias && a.ext_E <= tc::kBiasSmemMax) ? 1 : 0;
+  a.koff_mode = (d.n_pad <= tc::kKoffTableMax) ? tc::kKoffTable : tc::kKoffWarp;
+  const int bias_kind = !has_bias ? tc::BIAS_NONE : (a.ext_E <= tc::kBiasSmemMax ? tc::BIAS_SMEM : tc::BIAS_GLOBAL);
   a.int_levels = 1;
   for (int h = 0; h < s->H; ++h) {
     const double aq = alpha_q ? (double)alpha_q[h] : 1.0, ak = alpha_k ? (double)alpha_k[h] : 1.0;
@@ -456,7 +456,7 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
     }
   }
   dim3 grid((s->n + tc::kM - 1) / tc::kM, d.BH);
-  return dispatch_tc<EXP>(select_kind(s, bias, N), quant ? tc::MODE_Q : tc::MODE_F, has_bias, vf32, a, grid, st);
+  return dispatch_tc<EXP>(select_kind(s, bias, N), quant ? tc::MODE_Q : tc::MODE_F, bias_kind, vf32, a, grid, st);
 }
 
 had_status device_status_ptr(unsigned** out) {
