@@ -287,18 +287,15 @@ __device__ __forceinline__ void bias_tables_block(const BiasArgs& a, int h) {
 
 __global__ void __launch_bounds__(256) k_bias_tables(const BiasArgs a) { bias_tables_block(a, blockIdx.x); }
 
-// rint(x / sc) clamped to +-127, with x / sc the correctly rounded fp32 quotient.
-// x * (1/sc) is within 2^-15 of that quotient for |x / sc| <= 128, so it rounds
-// to the same integer unless it lies within 2^-12 of a half-integer; only then
-// is the quotient itself computed.
+// int8 code of x at scale sc: rint(x / sc) clamped to +-127, with x / sc the
+// correctly rounded fp32 quotient.  For |x / sc| <= 128 the product x * (1/sc)
+// is within 2^-15 of that quotient, so both round to the same integer unless the
+// product lies within 2^-12 of a half-integer; only then is the quotient computed.
 __device__ __forceinline__ int quant_i8(float x, float sc, float rsc) {
   const float y = x * rsc;
-  const float f = y - floorf(y);
-  float r;
-  if (fabsf(f - 0.5f) > 0x1p-12f) r = rintf(y);
-  else r = rintf(__fdiv_rn(x, sc));
-  r = fminf(fmaxf(r, -127.0f), 127.0f);
-  return (int)r;
+  float q = rintf(y);
+  if (fabsf(y - q) > 0.5f - 0x1p-12f) q = rintf(__fdiv_rn(x, sc));
+  return (int)fminf(fmaxf(q, -127.0f), 127.0f);
 }
 
 template <typename T>
@@ -327,23 +324,26 @@ __global__ void __launch_bounds__(kHeadThreads) k_prep_head(const HeadArgs a, co
   }
   asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
   __syncthreads();
-  // channels 2p and 2p+1 of token i
-  auto pair_at = [&](int i, int p) -> float2 {
+  // byte offset of channels 2p, 2p+1 inside a row whose token index is = k (mod 8)
+  auto pair_off = [&](int p, int k) -> int {
     const int byte = 2 * p * (int)sizeof(T);
-    const uint8_t* q = xs + i * kRow + (((byte >> 4) ^ (i & 7)) << 4) + (byte & 15);
+    return (((byte >> 4) ^ k) << 4) + (byte & 15);
+  };
+  auto pair_load = [&](const uint8_t* q) -> float2 {
     if (sizeof(T) == 2) {
       const uint32_t u = *reinterpret_cast<const uint32_t*>(q);
       return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
     }
     return *reinterpret_cast<const float2*>(q);
   };
-  // ---- channel statistic: warp g covers tokens g, g + 8, ...; lane p channels 2p, 2p+1
+  // ---- channel statistic: warp g covers tokens g, g + 8, ... (all = g mod 8); lane p channels 2p, 2p+1
   {
     const int p = tid & 31, g = tid >> 5;
+    const uint8_t* col = xs + pair_off(p, g);
     if (tz < 2) {
       double s0 = 0.0, s1 = 0.0;
       for (int i = g; i < L; i += kGroups) {
-        const float2 x = pair_at(i, p);
+        const float2 x = pair_load(col + i * kRow);
         s0 += (double)x.x;
         s1 += (double)x.y;
       }
@@ -352,7 +352,7 @@ __global__ void __launch_bounds__(kHeadThreads) k_prep_head(const HeadArgs a, co
     } else {
       float m0 = 0.0f, m1 = 0.0f;
       for (int i = g; i < L; i += kGroups) {
-        const float2 x = pair_at(i, p);
+        const float2 x = pair_load(col + i * kRow);
         m0 = fmaxf(m0, fabsf(x.x));
         m1 = fmaxf(m1, fabsf(x.y));
       }
@@ -426,13 +426,16 @@ __global__ void __launch_bounds__(kHeadThreads) k_prep_head(const HeadArgs a, co
     const int p = tid & 31;
     const float sc0 = stat[2 * p], sc1 = stat[2 * p + 1];
     const float r0 = 1.0f / sc0, r1 = 1.0f / sc1;
+    int off[8];  // token u of a block is = u (mod 8)
+#pragma unroll
+    for (int k = 0; k < 8; ++k) off[k] = pair_off(p, k);
     for (int blk = tid >> 5; blk * 16 < a.n_pad; blk += kGroups) {
       uint32_t w0[4] = {0u, 0u, 0u, 0u}, w1[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
         const int i = blk * 16 + u;
         if (i < L) {
-          const float2 x = pair_at(i, p);
+          const float2 x = pair_load(xs + i * kRow + off[u & 7]);
           w0[u >> 2] |= ((uint32_t)quant_i8(x.x, sc0, r0) & 0xFFu) << (8 * (u & 3));
           w1[u >> 2] |= ((uint32_t)quant_i8(x.y, sc1, r1) & 0xFFu) << (8 * (u & 3));
         }
