@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
     }
     if (MODE == MODE_Q && EXPORT == EXP_NONE && tid < kD) dq[tid] = __fdiv_rn(a.vscale[(size_t)bh * kD + tid], 255.0f);
     if (HAS_BIAS && a.koff_mode == kKoffTable)
-      for (int j = tid; j < a.n_pad; j += kM) koff_tab[j] = key_offset(a, j, L);
+      for (int j = tid; j < a.n_pad; j += kM) koff_tab[j] = 4 * key_offset(a, j, L);  // in bytes
     if (BIAS == BIAS_SMEM) {
       const float* src = a.expb + (size_t)h * a.ext_E;
       float* dst = reinterpret_cast<float*>(sm + SM::kBiasTab);
@@ -420,9 +420,11 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       const bool lut_w = (SEL == SEL_TOPN_INT) && a.int_levels && pass == P_PV;
       const bool wants_bias = HAS_BIAS && pass != P_LEVELS;
       // exp(b - b_max) of this row (dense): row base rb(i) into the staged or global table
-      const float* eb_row = nullptr;
-      if (BIAS == BIAS_SMEM) eb_row = reinterpret_cast<const float*>(sm + SM::kBiasTab) + rb;
-      else if (HAS_BIAS && SEL == SEL_DENSE) eb_row = a.expb + (size_t)h * a.ext_E + rb;
+      // (key offsets are kept in bytes: entry (i, j) sits at row base - koff_bytes(j))
+      const char* eb_bytes = nullptr;
+      if (BIAS == BIAS_SMEM) eb_bytes = reinterpret_cast<const char*>(reinterpret_cast<const float*>(sm + SM::kBiasTab) + rb);
+      else if (HAS_BIAS && SEL == SEL_DENSE) eb_bytes = reinterpret_cast<const char*>(a.expb + (size_t)h * a.ext_E + rb);
+      const char* tab_bytes = HAS_BIAS ? reinterpret_cast<const char*>(tab + rb) : nullptr;
       // a warp whose 32 rows all lie past L only keeps the barrier phases going
       const bool warp_live = __any_sync(0xffffffffu, row < L);
       // per-warp offsets: patch (y, x) of keys j0 + lane and j0 + 32 + lane, advanced
@@ -440,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
         if (x >= a.gw) { x -= a.gw; ++y; }
       };
       auto offset_of = [&](int j, int y, int x) -> int {
-        return j >= L ? a.k_invalid : (j < a.prefix ? a.k_class : y * a.tw + x);
+        return 4 * (j >= L ? a.k_invalid : (j < a.prefix ? a.k_class : y * a.tw + x));  // in bytes
       };
       for (int t = 0; t < ntiles; ++t) {
         const uint32_t gs = g_s + (uint32_t)t, buf = gs % kSBufs;
@@ -486,12 +488,14 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
         auto emit = [&](const float (&e)[32], int ch) {
           const int jb = j0 + 32 * ch;
           if (kHasCodes || MODE == MODE_Q) {
+            // uint8 codes floor(255 p + 0.5): every kept weight is at most the row's
+            // normalizer, so e * (255 / normalizer) + 0.5 < 256 and no clamp is needed
             uint32_t wq[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
               uint32_t q[4];
 #pragma unroll
-              for (int v = 0; v < 4; ++v) q[v] = min(__float2uint_rd(__fmaf_rn(e[4 * u + v], scale, 0.5f)), 255u);
+              for (int v = 0; v < 4; ++v) q[v] = __float2uint_rd(__fmaf_rn(e[4 * u + v], scale, 0.5f));
               wq[u] = __byte_perm(__byte_perm(q[0], q[1], 0x0040), __byte_perm(q[2], q[3], 0x0040), 0x5410);
             }
             if (kHasCodes) {
@@ -567,8 +571,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
                 for (int v = 0; v < 4; ++v) {
                   const int sc = (int)r[32 * ch + u + v];
                   float x = lut_lane[-16 * sc];  // level (64 - s) / 2 of this lane's table
-                  if (BIAS == BIAS_SMEM) x *= eb_row[-kk[v]];
-                  else if (HAS_BIAS) x *= __ldg(eb_row - kk[v]);
+                  if (BIAS == BIAS_SMEM) x *= *reinterpret_cast<const float*>(eb_bytes - kk[v]);
+                  else if (HAS_BIAS) x *= __ldg(reinterpret_cast<const float*>(eb_bytes - kk[v]));
                   e[u + v] = (FULL || 32 * ch + u + v < nvalid) ? x : 0.0f;
                 }
               }
@@ -604,8 +608,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
                   const int sc = (int)r[32 * ch + u + v];
                   float l;
                   if (HAS_BIAS) {
-                    if (kMaskInKoff) kinv |= (kk[v] == a.k_invalid ? 1u : 0u) << (u + v);
-                    l = __fmaf_rn((float)sc, c, __ldg(tab + (rb - kk[v])));
+                    if (kMaskInKoff) kinv |= (kk[v] == 4 * a.k_invalid ? 1u : 0u) << (u + v);
+                    l = __fmaf_rn((float)sc, c, __ldg(reinterpret_cast<const float*>(tab_bytes - kk[v])));
                   } else {
                     l = (float)sc * c;
                   }
