@@ -74,6 +74,34 @@ def launches_per_step(n: int, elem: int, mode: str, has_bias: bool) -> int:
     return k + 1
 
 
+# Issue-limited CUDA-core rate of one B200: 148 SMs x 4 schedulers x 32 lanes x
+# 1965 MHz (clocks.max.sm), one lane-operation per lane per clock.
+ALU_PEAK_TOPS = 148 * 4 * 32 * 1.965e9 / 1e12
+
+
+def alu_ops_per_score(mode: str, N: int, n: int, has_bias: bool) -> float:
+    """CUDA-core operations per valid (query, key) pair that the fused kernel's
+    formulation cannot avoid (address arithmetic, loop control and the tensor-core
+    work not counted).  Dense (N = 0 or N >= n): the weight of a score is a
+    level-table lookup, times an exp(bias) lookup when there is a bias; uint8
+    mode needs the normalizer first, so it computes the weight twice (sum, then
+    scale-round-convert and a quarter of a byte pack); float mode sums in the
+    same pass and packs half a bf16 pair.  Top-N without a bias: one histogram
+    increment, then lookup, tie test, select and the pack.  Top-N with a bias:
+    one histogram increment, one radix pass (bias gather, logit FMA, order key,
+    range test, increment) and the output pass (gather, FMA, two compares,
+    exp as FFMA + ex2, select, pack)."""
+    dense = N == 0 or N >= n
+    if dense:
+        if mode == "u8i8":
+            w = 3.0 if has_bias else 1.0
+            return (w + 1.0) + (w + 2.25)
+        return (3.0 if has_bias else 1.0) + 1.0 + 0.5
+    if not has_bias:
+        return 1.0 + (3.0 + (2.25 if mode == "u8i8" else 0.5))
+    return 1.0 + 6.0 + 7.5
+
+
 def kernel_bytes_per_token(mode: str, v_bytes: int, o_bytes: int) -> int:
     """Algorithmic bytes per valid token of the fused kernel (k_attn).
 
@@ -349,6 +377,9 @@ def run_gpu(args, rank, world, local_rank):
     if bias is not None:
         kbytes += w.bias.table.nbytes
     achieved = kbytes / (attn_avg_ms * 1e-3) / 1e9
+    ops_per_score = alu_ops_per_score(mode, N, w.n, bias is not None)
+    alu_ops = ops_per_score * w.valid_scores()
+    alu_achieved = alu_ops / (attn_avg_ms * 1e-3) / 1e12
     pbytes = path_bytes_per_token(mode, 2 if bf16 else 4, O.element_size()) * queries
     path_achieved = pbytes / (ms_per_step * 1e-3) / 1e9
     traffic = None
@@ -362,10 +393,15 @@ def run_gpu(args, rank, world, local_rank):
         "vs_baseline": None, "dtype": "u8i8" if mode == "u8i8" else ("bf16" if bf16 else "f32"),
         "data": "synthetic", "config": {**_config(w, N, mode), "parallelism": f"replicas x{world} (no collective)"},
         "score_ops_per_s": w.valid_scores() * world * args.steps / (total_ms * 1e-3),
-        "roofline": {"bound": "hbm", "kernel": "k_attn (fused score/top-N/softmax/A.V)", "achieved": achieved,
-                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": traffic, "algorithmic_bytes_per_launch": kbytes,
-                     "avg_launch_ms": attn_avg_ms, "peak_kind": peak_kind},
+        "roofline": {"bound": "alu", "kernel": "k_attn_tc (fused score/top-N/softmax/A.V)",
+                     "achieved": alu_achieved, "peak": ALU_PEAK_TOPS, "unit": "Tlane-op/s",
+                     "frac": alu_achieved / ALU_PEAK_TOPS, "traffic": traffic,
+                     "algorithmic_ops_per_launch": alu_ops, "ops_per_valid_score": ops_per_score,
+                     "avg_launch_ms": attn_avg_ms,
+                     "peak_kind": "derived: 148 SMs x 4 schedulers x 32 lanes x 1965 MHz"},
+        "roofline_hbm": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": kbytes,
+                         "peak_kind": peak_kind},
         "roofline_path": {"bound": "hbm", "achieved": path_achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                           "frac": path_achieved / peaks["hbm_gbs"], "algorithmic_bytes_per_step": pbytes},
         "e2e": {"value": queries * world / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
