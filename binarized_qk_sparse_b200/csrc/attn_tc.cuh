@@ -108,7 +108,7 @@ struct Smem {
   static constexpr int kBiasTab = kKoff + (HAS_BIAS ? kKoffTableMax * 4 : 0);  // exp(bias) table (dense)
   static constexpr int kDq = kBiasTab + (BIAS == BIAS_SMEM ? kBiasSmemMax * 4 : 0);  // 64 dequant scales
   static constexpr int kBar = kDq + kD * 4;
-  static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 2 * kSBufs + 2;
+  static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 2 * kSBufs + 3;
   static constexpr int kMisc = kBar + kNumBars * 8;              // [0] tmem base [1] abort
   static constexpr int kHist = (kMisc + 16 + 127) / 128 * 128;
   static constexpr int kHistBytes = (SEL == SEL_DENSE) ? kLevels * 32 * 4
@@ -127,7 +127,8 @@ enum {
   B_SFULL = 2 * kKStages + 2 * kVStages,  // one per score buffer
   B_TDONE = B_SFULL + kSBufs,             // one per score buffer
   B_OFULL = B_TDONE + kSBufs,
-  B_FINAL
+  B_FINAL,
+  B_BIAS  // staged exp(bias) table landed
 };
 
 // Bias offset of key j: koff = y_j * tw + x_j for patch tokens, so that
@@ -213,8 +214,14 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
     for (int s = 0; s < kSBufs; ++s) { mbar_init(&bars[B_SFULL + s], 1); mbar_init(&bars[B_TDONE + s], kM); }
     mbar_init(&bars[B_OFULL], 1);
     mbar_init(&bars[B_FINAL], 1);
+    mbar_init(&bars[B_BIAS], 1);
     misc[1] = 0;
     fence_barrier_init();
+    if (BIAS == BIAS_SMEM) {
+      // the head's exp(bias) table, one bulk copy that overlaps the rest of the setup
+      mbar_arrive_expect_tx(&bars[B_BIAS], (uint32_t)a.ext_E * 4u);
+      bulk_load(sm + SM::kBiasTab, a.expb + (size_t)h * a.ext_E, (uint32_t)a.ext_E * 4u, &bars[B_BIAS]);
+    }
     prefetch_tensormap(&a.tm_k);
     if (EXPORT == EXP_NONE) prefetch_tensormap(MODE == MODE_Q ? &a.tm_vq : &a.tm_v);
   }
@@ -239,20 +246,15 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
     }
     if (SEL != SEL_DENSE)
       for (int lev = 0; lev < kLevels; ++lev) hist[lev * kM + tid] = 0u;
-    if (SEL == SEL_DENSE && tid < 32) {
-      // per-lane copy of the level table exp(c * (s - 64)), level k = (64 - s) / 2
+    if (SEL == SEL_DENSE) {
+      // per-lane copies of the level table exp(c * (s - 64)), level k = (64 - s) / 2, at [k][lane]
       const float ck = -2.0f * a.c_head[h] * 1.4426950408889634f;
       float* lt = reinterpret_cast<float*>(hist);
-      for (int lev = 0; lev < kLevels; ++lev) lt[lev * 32 + tid] = exp2f(ck * (float)lev);
+      for (int e = tid; e < kLevels * 32; e += kM) lt[e] = exp2f(ck * (float)(e >> 5));
     }
     if (MODE == MODE_Q && EXPORT == EXP_NONE && tid < kD) dq[tid] = __fdiv_rn(a.vscale[(size_t)bh * kD + tid], 255.0f);
     if (HAS_BIAS && a.koff_mode == kKoffTable)
       for (int j = tid; j < a.n_pad; j += kM) koff_tab[j] = 4 * key_offset(a, j, L);  // in bytes
-    if (BIAS == BIAS_SMEM) {
-      const float* src = a.expb + (size_t)h * a.ext_E;
-      float* dst = reinterpret_cast<float*>(sm + SM::kBiasTab);
-      for (int i = tid; i < a.ext_E; i += kM) dst[i] = __ldg(src + i);
-    }
     fence_proxy_async();
   }
   tc_fence_before();
@@ -305,37 +307,48 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
     return false;
   };
 
+  // K tiles of a short key range stay in the K stages for every pass (loaded once)
+  const bool k_res = ntiles <= kKStages;
+  bool first_pass = true;
+  int v_pref = 0;  // producer: V tiles of the P.V pass already issued
   while (pass != P_DONE) {
     const bool pv = (pass == P_PV);
     // ============================================================== producer (warp 5)
     if (warp == 5) {
-      for (int t = 0; t < ntiles; ++t) {
-        const uint32_t st = g_k % kKStages;
-        if (lane == 0 && g_k >= (uint32_t)kKStages) bounded_wait(B_KEMPTY + st, ((g_k / kKStages) - 1) & 1);
+      auto load_v = [&](int t) {
+        const uint32_t vs = g_v % kVStages;
+        if (lane == 0 && g_v >= (uint32_t)kVStages) bounded_wait(B_VEMPTY + vs, ((g_v / kVStages) - 1) & 1);
         if (lane == 0 && !*abort_flag) {
-          mbar_arrive_expect_tx(&bars[B_KFULL + st], kN * kD);
-          tma_load_2d(sm + SM::kK + st * kN * kD, &a.tm_k, 0, bh * a.n_pad + t * kN, &bars[B_KFULL + st]);
-          k_par[st] = (int)((g_k / kKStages) & 1);
-        }
-        ++g_k;
-        if (pv) {
-          const uint32_t vs = g_v % kVStages;
-          if (lane == 0 && g_v >= (uint32_t)kVStages) bounded_wait(B_VEMPTY + vs, ((g_v / kVStages) - 1) & 1);
-          if (lane == 0 && !*abort_flag) {
-            uint8_t* dst = sm + SM::kV + vs * SM::kVStage;
-            if (MODE == MODE_Q) {
-              mbar_arrive_expect_tx(&bars[B_VFULL + vs], kD * kN);
-              tma_load_2d(dst, &a.tm_vq, t * kN, bh * kD, &bars[B_VFULL + vs]);
-            } else {
-              mbar_arrive_expect_tx(&bars[B_VFULL + vs], SM::kVStage);
-              tma_load_2d(dst, &a.tm_v, 0, bh * a.n + t * kN, &bars[B_VFULL + vs]);
-              if (VF32) tma_load_2d(dst + kN * kD * 2, &a.tm_vlo, 0, bh * a.n + t * kN, &bars[B_VFULL + vs]);
-            }
-            v_par[vs] = (int)((g_v / kVStages) & 1);
+          uint8_t* dst = sm + SM::kV + vs * SM::kVStage;
+          if (MODE == MODE_Q) {
+            mbar_arrive_expect_tx(&bars[B_VFULL + vs], kD * kN);
+            tma_load_2d(dst, &a.tm_vq, t * kN, bh * kD, &bars[B_VFULL + vs]);
+          } else {
+            mbar_arrive_expect_tx(&bars[B_VFULL + vs], SM::kVStage);
+            tma_load_2d(dst, &a.tm_v, 0, bh * a.n + t * kN, &bars[B_VFULL + vs]);
+            if (VF32) tma_load_2d(dst + kN * kD * 2, &a.tm_vlo, 0, bh * a.n + t * kN, &bars[B_VFULL + vs]);
           }
-          ++g_v;
+          v_par[vs] = (int)((g_v / kVStages) & 1);
         }
+        ++g_v;
+      };
+      for (int t = 0; t < ntiles; ++t) {
+        if (!k_res || first_pass) {
+          const uint32_t st = k_res ? (uint32_t)t : g_k % kKStages;
+          if (!k_res && lane == 0 && g_k >= (uint32_t)kKStages)
+            bounded_wait(B_KEMPTY + st, ((g_k / kKStages) - 1) & 1);
+          if (lane == 0 && !*abort_flag) {
+            mbar_arrive_expect_tx(&bars[B_KFULL + st], kN * kD);
+            tma_load_2d(sm + SM::kK + st * kN * kD, &a.tm_k, 0, bh * a.n_pad + t * kN, &bars[B_KFULL + st]);
+            k_par[st] = k_res ? 0 : (int)((g_k / kKStages) & 1);
+          }
+          ++g_k;
+        }
+        if (pv && t >= v_pref) load_v(t);
       }
+      // the P.V pass comes last: its first V tiles can load while this pass runs
+      if (EXPORT == EXP_NONE && !pv && v_pref == 0)
+        for (; v_pref < kVStages && v_pref < ntiles; ++v_pref) load_v(v_pref);
     }
     // ============================================================== MMA issuer (warp 4, lane 0)
     else if (warp == 4) {
@@ -343,8 +356,9 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
         const uint32_t id_s = idesc_i8(kM, kN, true, true, false);
         const uint32_t id_pv = (MODE == MODE_Q) ? idesc_i8(kM, kD, false, true, false) : idesc_bf16(kM, kD, true);
         auto issue_scores = [&](int t) {
-          const uint32_t gk = g_k + (uint32_t)t, st = gk % kKStages, buf = (g_s + (uint32_t)t) % kSBufs;
-          if (!bounded_wait(B_KFULL + st, (gk / kKStages) & 1)) return;
+          const uint32_t gk = g_k + (uint32_t)t, buf = (g_s + (uint32_t)t) % kSBufs;
+          const uint32_t st = k_res ? (uint32_t)t : gk % kKStages;
+          if (!bounded_wait(B_KFULL + st, k_res ? 0u : (gk / kKStages) & 1)) return;
           tc_fence_after();
           const uint32_t kq = smem_u32(sQ), kk = smem_u32(sm + SM::kK + st * kN * kD);
 #pragma unroll
@@ -352,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
             mma_i8_ss(tmem + kColS + buf * kN, sdesc(kq + 32 * ks, 16, 512, kSwizzle64B),
                       sdesc(kk + 32 * ks, 16, 512, kSwizzle64B), id_s, ks > 0 ? 1u : 0u);
           mma_commit(&bars[B_SFULL + buf]);
-          mma_commit(&bars[B_KEMPTY + st]);
+          if (!k_res) mma_commit(&bars[B_KEMPTY + st]);
         };
         for (int t = 0; t < kSBufs && t < ntiles; ++t) issue_scores(t);
         for (int t = 0; t < ntiles; ++t) {
@@ -444,6 +458,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       auto offset_of = [&](int j, int y, int x) -> int {
         return 4 * (j >= L ? a.k_invalid : (j < a.prefix ? a.k_class : y * a.tw + x));  // in bytes
       };
+      if (BIAS == BIAS_SMEM && first_pass) bounded_wait(B_BIAS, 0);
       for (int t = 0; t < ntiles; ++t) {
         const uint32_t gs = g_s + (uint32_t)t, buf = gs % kSBufs;
         const uint32_t colP = kColS + buf * kN;  // P of this tile is written over its score buffer
@@ -833,6 +848,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       for (int bb = 0; bb < kRadixBins; ++bb) hist[bb * kM + tid] = 0u;
     if (next == P_KEPT_NORM && tid < kM) lsum = 0.0f;
     __syncthreads();
+    first_pass = false;
     pass = next;
   }
 
@@ -893,6 +909,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       if (k_par[s2] >= 0) mbar_wait(&bars[B_KFULL + s2], (uint32_t)k_par[s2], 200000000LL);
     for (int s2 = 0; s2 < kVStages; ++s2)
       if (v_par[s2] >= 0) mbar_wait(&bars[B_VFULL + s2], (uint32_t)v_par[s2], 200000000LL);
+    if (BIAS == BIAS_SMEM) mbar_wait(&bars[B_BIAS], 0, 200000000LL);
   }
   if (warp == 4 && lane == 0) {
     // every tcgen05 operation this thread issued is complete before TMEM is freed

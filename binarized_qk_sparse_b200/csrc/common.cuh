@@ -32,7 +32,7 @@ __device__ __forceinline__ void raise_status(unsigned* status, unsigned bits) {
 // (query, key) pair with no case analysis:
 //   [0, T)              the table, T = (2gh-1)(2gw-1)
 //   [T, 2T + 2Kx)       class-token pairs (bias 0)
-//   [2T + 2Kx, 3T + 3Kx) keys past L (weight 0 / logit -inf)
+//   [2T + 2Kx, E)       keys past L (weight 0 / logit -inf), E = 3T + 3Kx rounded up to 4
 // with Kx = (gh-1)(2gw-1) + gw the number of distinct patch key offsets.
 struct RelposExt {
   int T, Kx, E, rb_class, k_class, k_invalid;
@@ -42,7 +42,7 @@ __host__ __device__ inline RelposExt relpos_ext(int gh, int gw) {
   const int tw = 2 * gw - 1;
   r.T = (2 * gh - 1) * tw;
   r.Kx = (gh - 1) * tw + gw;
-  r.E = 3 * r.T + 3 * r.Kx;
+  r.E = (3 * r.T + 3 * r.Kx + 3) / 4 * 4;  // padded to 16 bytes per head (bulk copies)
   r.rb_class = r.T - 1 + r.Kx;
   r.k_class = -(r.T + r.Kx);
   r.k_invalid = -(2 * r.T + 2 * r.Kx);
