@@ -13,10 +13,12 @@
 //              V^T tiles ([64 channels][64 keys], 64-byte swizzle, K-major B).
 // Tensor memory (256 columns): a ring of three score buffers S0..S2 [0,192), so
 // the score MMAs of tiles t+1 and t+2 run while the softmax warps work on tile t,
-// and O [192,256).  P of tile t is written over its own score buffer (bf16 in
-// columns [0,32) of the buffer, the residual for fp32 V in [32,64); uint8 codes
-// in [0,16)): the P.V MMA of tile t is issued before the score MMA that next
-// writes that buffer, and MMAs from one thread run in issue order.
+// and O [192,256).  P of tile t is written over its own score buffer, each 32-key
+// chunk inside that chunk's own 32 score columns (bf16 in [32c, 32c+16), the
+// residual for fp32 V in [32c+16, 32c+32); uint8 codes in [32c, 32c+8)), so a
+// thread never overwrites scores another thread has still to read.  The P.V MMA
+// of tile t is issued before the score MMA that next writes that buffer, and
+// MMAs from one thread run in issue order.
 //
 // Score (BinaryAttention §2.1/§2.2): S = Q~ K~^T with kind::i8 on +-1 operands,
 // so S = d - 2*popcount(q XOR k) exactly.  A.V: kind::f16 (bf16 P from TMEM x
@@ -47,7 +49,12 @@ using namespace had::sm100;
 
 constexpr int kM = 128;            // query rows per CTA (TMEM lanes)
 constexpr int kN = 64;             // keys per tile (score MMA N)
-constexpr int kThreads = 192;
+// Softmax threads per query row: dense attention splits each 64-key tile between
+// two threads (warps w and w + 4 share the TMEM lanes of quadrant w), which
+// doubles the warps that hide latency; top-N keeps one thread per row (its tie
+// and kept-index bookkeeping runs in key order).
+__host__ __device__ constexpr int row_split(int sel) { return sel == 0 ? 2 : 1; }
+__host__ __device__ constexpr int cta_threads(int sel) { return 32 * (4 * row_split(sel) + 2); }
 constexpr int kKStages = 4;
 constexpr int kVStages = 2;
 constexpr int kLevels = 65;
@@ -106,7 +113,8 @@ struct Smem {
   static constexpr int kV = kK + kKStages * kN * kD;             // 2 V stages
   static constexpr int kKoff = kV + kVStages * kVStage;          // bias key offsets (table, or 4 warps x 2 x 64)
   static constexpr int kBiasTab = kKoff + (HAS_BIAS ? kKoffTableMax * 4 : 0);  // exp(bias) table (dense)
-  static constexpr int kDq = kBiasTab + (BIAS == BIAS_SMEM ? kBiasSmemMax * 4 : 0);  // 64 dequant scales
+  static constexpr int kXchg = kBiasTab + (BIAS == BIAS_SMEM ? kBiasSmemMax * 4 : 0);  // 2 x 128 fp32 (row partials)
+  static constexpr int kDq = kXchg + 2 * kM * 4;                                        // 64 dequant scales
   static constexpr int kBar = kDq + kD * 4;
   static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 2 * kSBufs + 3;
   static constexpr int kMisc = kBar + kNumBars * 8;              // [0] tmem base [1] abort
@@ -140,6 +148,10 @@ __device__ __forceinline__ int key_offset(const TcArgs& a, int j, int L) {
   return (t / a.gw) * a.tw + t % a.gw;
 }
 
+// TMEM column (within a tile's P) of bf16 K-step k (16 keys): chunk k/2 sits in
+// its own 32 columns, 8 columns per 16 keys.
+__host__ __device__ constexpr uint32_t pcol(int k) { return 32u * (uint32_t)(k >> 1) + 8u * (uint32_t)(k & 1); }
+
 // Pairwise sum of 32 values (a depth-5 tree instead of a 32-long dependent chain).
 __device__ __forceinline__ float sum32(const float (&e)[32]) {
   float t[16];
@@ -153,8 +165,13 @@ __device__ __forceinline__ float sum32(const float (&e)[32]) {
 }
 
 template <int SEL, int MODE, int BIAS, bool VF32, int EXPORT>
-__global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__ TcArgs a) {
+__global__ void __launch_bounds__(cta_threads(SEL), 2) k_attn_tc(const __grid_constant__ TcArgs a) {
   static_assert(BIAS != BIAS_SMEM || SEL == SEL_DENSE, "staged exp(bias) tables serve the dense weights only");
+  constexpr int kSplit = row_split(SEL);
+  constexpr int kSoftWarps = 4 * kSplit;
+  constexpr int kThreads = cta_threads(SEL);
+  constexpr int kMmaWarp = kSoftWarps, kProdWarp = kSoftWarps + 1;
+  constexpr int kChunks = 2 / kSplit;  // 32-key chunks of a tile per softmax thread
   constexpr bool HAS_BIAS = BIAS != BIAS_NONE;
   using SM = Smem<SEL, VF32, BIAS>;
   extern __shared__ uint8_t smem_raw[];
@@ -167,8 +184,12 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
   int* koff_tab = reinterpret_cast<int*>(sm + SM::kKoff);
   float* dq = reinterpret_cast<float*>(sm + SM::kDq);
   uint32_t* hist = reinterpret_cast<uint32_t*>(sm + SM::kHist);
+  float* xchg = reinterpret_cast<float*>(sm + SM::kXchg);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const bool is_soft = warp < kSoftWarps;
+  const int srow = tid & (kM - 1);          // softmax thread: query row within the tile (TMEM lane)
+  const int half = (warp >> 2) & 1;         // softmax thread: which 32-key chunk of a tile (split rows)
   const int bh = blockIdx.y, b = bh / a.H, h = bh % a.H;
   const int q0 = blockIdx.x * kM;
   const int L = valid_len(a.seqlens, b, a.n, a.status);
@@ -204,14 +225,14 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
   }
 
   // ---------------------------------------------------------------- setup
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tmem_alloc(misc, kTmemCols);
     tmem_relinquish();
   }
-  if (warp == 5 && lane == 0) {
+  if (warp == kProdWarp && lane == 0) {
     for (int s = 0; s < kKStages; ++s) { mbar_init(&bars[B_KFULL + s], 1); mbar_init(&bars[B_KEMPTY + s], 1); }
     for (int s = 0; s < kVStages; ++s) { mbar_init(&bars[B_VFULL + s], 1); mbar_init(&bars[B_VEMPTY + s], 1); }
-    for (int s = 0; s < kSBufs; ++s) { mbar_init(&bars[B_SFULL + s], 1); mbar_init(&bars[B_TDONE + s], kM); }
+    for (int s = 0; s < kSBufs; ++s) { mbar_init(&bars[B_SFULL + s], 1); mbar_init(&bars[B_TDONE + s], 32 * kSoftWarps); }
     mbar_init(&bars[B_OFULL], 1);
     mbar_init(&bars[B_FINAL], 1);
     mbar_init(&bars[B_BIAS], 1);
@@ -225,8 +246,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
     prefetch_tensormap(&a.tm_k);
     if (EXPORT == EXP_NONE) prefetch_tensormap(MODE == MODE_Q ? &a.tm_vq : &a.tm_v);
   }
-  const int row = q0 + tid;  // softmax threads
-  const bool row_ok = tid < kM && row < L;
+  const int row = q0 + srow;  // softmax threads
+  const bool row_ok = is_soft && row < L;
   if (tid < kM) {
     // Q~ row into the 64-byte swizzled K-major A operand (16-byte chunk c -> c ^ ((row >> 1) & 3))
     uint32_t w0 = 0, w1 = 0;
@@ -245,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       *reinterpret_cast<uint4*>(sQ + tid * kD + ((cch ^ ((tid >> 1) & 3)) * 16)) = v;
     }
     if (SEL != SEL_DENSE)
-      for (int lev = 0; lev < kLevels; ++lev) hist[lev * kM + tid] = 0u;
+      for (int lev = 0; lev < kLevels; ++lev) hist[lev * kM + srow] = 0u;
     if (SEL == SEL_DENSE) {
       // per-lane copies of the level table exp(c * (s - 64)), level k = (64 - s) / 2, at [k][lane]
       const float ck = -2.0f * a.c_head[h] * 1.4426950408889634f;
@@ -313,8 +334,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
   int v_pref = 0;  // producer: V tiles of the P.V pass already issued
   while (pass != P_DONE) {
     const bool pv = (pass == P_PV);
-    // ============================================================== producer (warp 5)
-    if (warp == 5) {
+    // ============================================================== producer warp
+    if (warp == kProdWarp) {
       auto load_v = [&](int t) {
         const uint32_t vs = g_v % kVStages;
         if (lane == 0 && g_v >= (uint32_t)kVStages) bounded_wait(B_VEMPTY + vs, ((g_v / kVStages) - 1) & 1);
@@ -350,8 +371,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       if (EXPORT == EXP_NONE && !pv && v_pref == 0)
         for (; v_pref < kVStages && v_pref < ntiles; ++v_pref) load_v(v_pref);
     }
-    // ============================================================== MMA issuer (warp 4, lane 0)
-    else if (warp == 4) {
+    // ============================================================== MMA issuer warp (one thread)
+    else if (warp == kMmaWarp) {
       if (lane == 0) {
         const uint32_t id_s = idesc_i8(kM, kN, true, true, false);
         const uint32_t id_pv = (MODE == MODE_Q) ? idesc_i8(kM, kD, false, true, false) : idesc_bf16(kM, kD, true);
@@ -381,24 +402,24 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
               const uint32_t vbase = smem_u32(sm + SM::kV + vs * SM::kVStage);
               if (MODE == MODE_Q) {
 #pragma unroll
-                for (int k = 0; k < kN / 32; ++k)
-                  mma_i8_ts(tmem + kColO, tmem + colP + 8 * k, sdesc(vbase + 32 * k, 16, 512, kSwizzle64B), id_pv,
+                for (int k = 0; k < kN / 32; ++k)  // K-step k = key chunk k: codes at columns 32k
+                  mma_i8_ts(tmem + kColO, tmem + colP + 32 * k, sdesc(vbase + 32 * k, 16, 512, kSwizzle64B), id_pv,
                             (t > 0 || k > 0) ? 1u : 0u);
               } else {
 #pragma unroll
-                for (int k = 0; k < kN / 16; ++k)
-                  mma_f16_ts(tmem + kColO, tmem + colP + 8 * k, sdesc(vbase + 2048 * k, 0, 1024, kSwizzle128B), id_pv,
+                for (int k = 0; k < kN / 16; ++k)  // 16 keys per K-step: chunk k/2, columns 32(k/2) + 8(k%2)
+                  mma_f16_ts(tmem + kColO, tmem + colP + pcol(k), sdesc(vbase + 2048 * k, 0, 1024, kSwizzle128B), id_pv,
                              (t > 0 || k > 0) ? 1u : 0u);
                 if (VF32) {
                   // residual products: P_hi x V_lo and P_lo x V_hi
                   const uint32_t vlo = vbase + kN * kD * 2;
 #pragma unroll
                   for (int k = 0; k < kN / 16; ++k)
-                    mma_f16_ts(tmem + kColO, tmem + colP + 8 * k, sdesc(vlo + 2048 * k, 0, 1024, kSwizzle128B), id_pv,
+                    mma_f16_ts(tmem + kColO, tmem + colP + pcol(k), sdesc(vlo + 2048 * k, 0, 1024, kSwizzle128B), id_pv,
                                1u);
 #pragma unroll
                   for (int k = 0; k < kN / 16; ++k)
-                    mma_f16_ts(tmem + kColO, tmem + colP + 32 + 8 * k, sdesc(vbase + 2048 * k, 0, 1024, kSwizzle128B),
+                    mma_f16_ts(tmem + kColO, tmem + colP + pcol(k) + 16, sdesc(vbase + 2048 * k, 0, 1024, kSwizzle128B),
                                id_pv, 1u);
                 }
               }
@@ -413,10 +434,10 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       g_s += ntiles;
       if (pv) g_v += ntiles;
     }
-    // ============================================================== softmax / select (warps 0-3)
+    // ============================================================== softmax / select warps
     else {
-      const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-      const uint32_t hist_row = smem_u32(hist) + (uint32_t)tid * 4u;
+      const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+      const uint32_t hist_row = smem_u32(hist) + (uint32_t)srow * 4u;
       const float mo = -m * kLog2e;
       const float* lut = reinterpret_cast<const float*>(hist);
       const float* lut_lane = lut + 32 * 32 + lane;  // dense level table: entry for score s at lut_lane[-16 s]
@@ -486,9 +507,13 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
           mbar_arrive(&bars[B_TDONE + buf]);
           continue;
         }
-        uint32_t r[64];
-        tmem_ld32(tl + kColS + buf * kN, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-        tmem_ld32(tl + kColS + buf * kN + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+        uint32_t r[32 * kChunks];
+        if (kSplit == 2) {
+          tmem_ld32(tl + kColS + buf * kN + 32 * half, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+        } else {
+          tmem_ld32(tl + kColS + buf * kN, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          tmem_ld32(tl + kColS + buf * kN + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32 * (kChunks - 1)]));
+        }
         tmem_wait_ld();
         const int nvalid = row_ok ? max(0, min(kN, L - j0)) : 0;
         // Dense with bias: keys past L carry the k_invalid offset (weight 0), and
@@ -522,14 +547,14 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
                   if (jb + u < a.n) dst[jb + u] = (uint8_t)((wq[u >> 2] >> (8 * (u & 3))) & 0xFFu);
               }
             } else {
-              tmem_st8(tl + colP + 8 * ch, wq);
+              tmem_st8(tl + colP + 32 * ch, wq);
             }
           } else {
             uint32_t wp[16];
 #pragma unroll
             for (int u = 0; u < 16; ++u) wp[u] = pack_bf16x2(e[2 * u], e[2 * u + 1]);
             if (sum_in_pv) lsum += sum32(e);
-            tmem_st16(tl + colP + 16 * ch, wp);
+            tmem_st16(tl + colP + 32 * ch, wp);
             if (VF32) {
               uint32_t wl[16];
 #pragma unroll
@@ -537,7 +562,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
                 const float h0 = __uint_as_float(wp[u] << 16), h1 = __uint_as_float(wp[u] & 0xFFFF0000u);
                 wl[u] = pack_bf16x2(e[2 * u] - h0, e[2 * u + 1] - h1);
               }
-              tmem_st16(tl + colP + 32 + 16 * ch, wl);
+              tmem_st16(tl + colP + 32 * ch + 16, wl);
             }
           }
         };
@@ -545,18 +570,19 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
         auto tile_body = [&](auto full_tag) {
           constexpr bool FULL = decltype(full_tag)::value;
 #pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
+          for (int cc = 0; cc < kChunks; ++cc) {
+            const int ch = (kSplit == 2) ? half : cc;  // chunk of the tile; registers r[32 cc ...]
             const int jb = j0 + 32 * ch;
             if (jb >= L && pass != P_CODES) {
               // every key of the chunk lies past L: nothing to count or sum; P is 0
               if (pv) {
                 if (MODE == MODE_Q) {
                   const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-                  tmem_st8(tl + colP + 8 * ch, z);
+                  tmem_st8(tl + colP + 32 * ch, z);
                 } else {
                   const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
-                  tmem_st16(tl + colP + 16 * ch, z);
-                  if (VF32) tmem_st16(tl + colP + 32 + 16 * ch, z);
+                  tmem_st16(tl + colP + 32 * ch, z);
+                  if (VF32) tmem_st16(tl + colP + 32 * ch + 16, z);
                 }
               }
               continue;
@@ -565,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
               const uint32_t base = hist_row + 32u * kM * 4u;  // level (64 - s)/2 -> + (64 - s) * 256 bytes
 #pragma unroll
               for (int u = 0; u < 32; ++u) {
-                const uint32_t ad = base - (uint32_t)((int)r[32 * ch + u] * (kM * 2));
+                const uint32_t ad = base - (uint32_t)((int)r[32 * cc + u] * (kM * 2));
                 if (FULL) {
                   asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(ad) : "memory");
                 } else {
@@ -584,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
                 const int kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
-                  const int sc = (int)r[32 * ch + u + v];
+                  const int sc = (int)r[32 * cc + u + v];
                   float x = lut_lane[-16 * sc];  // level (64 - s) / 2 of this lane's table
                   if (BIAS == BIAS_SMEM) x *= *reinterpret_cast<const float*>(eb_bytes - kk[v]);
                   else if (HAS_BIAS) x *= __ldg(reinterpret_cast<const float*>(eb_bytes - kk[v]));
@@ -600,8 +626,8 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
               float e[32];
 #pragma unroll
               for (int u = 0; u < 32; ++u) {
-                const int sc = (int)r[32 * ch + u];
-                const float w = lut[(32 - (sc >> 1)) * kM + tid];
+                const int sc = (int)r[32 * cc + u];
+                const float w = lut[(32 - (sc >> 1)) * kM + srow];
                 const bool valid = FULL || 32 * ch + u < nvalid;
                 const bool eq = valid && sc == sF;
                 const bool drop_tie = eq && cut && tie_seen >= rF;
@@ -620,7 +646,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
                 const int kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
-                  const int sc = (int)r[32 * ch + u + v];
+                  const int sc = (int)r[32 * cc + u + v];
                   float l;
                   if (HAS_BIAS) {
                     if (kMaskInKoff) kinv |= (kk[v] == 4 * a.k_invalid ? 1u : 0u) << (u + v);
@@ -649,7 +675,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
 #pragma unroll
                   for (int u = 0; u < 32; ++u) {
                     const uint32_t dd = r_uhi - float_order_key(lg[u]);
-                    if ((FULL || 32 * ch + u < nvalid) && dd <= r_span) atomicAdd(&hist[(dd >> r_shift) * kM + tid], 1u);
+                    if ((FULL || 32 * ch + u < nvalid) && dd <= r_span) atomicAdd(&hist[(dd >> r_shift) * kM + srow], 1u);
                   }
                 }
               } else if (kHasRadix && pass == P_COLLECT) {
@@ -660,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
                     const uint32_t key = float_order_key(lg[u]);
                     const uint32_t dd = r_uhi - key;
                     if ((FULL || 32 * ch + u < nvalid) && dd <= r_span && (int)(dd >> r_shift) == r_bin) {
-                      if (r_cnt < kCandCap) cand[r_cnt * kM + tid] = make_uint2(key, (uint32_t)(jb + u));
+                      if (r_cnt < kCandCap) cand[r_cnt * kM + srow] = make_uint2(key, (uint32_t)(jb + u));
                       ++r_cnt;
                     }
                   }
@@ -690,9 +716,16 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
                 } else if (kHasIdx && pass == P_IDX) {
                   if (row_ok) {
                     int32_t* dst = a.idx + ((size_t)bh * a.n + row) * a.N;
+                    if (SEL == SEL_DENSE) {
+                      // dense: every key below L is kept, so key j is the j-th kept index
 #pragma unroll
-                    for (int u = 0; u < 32; ++u)
-                      if ((keepm >> u) & 1u) { if (kept_seen < a.N) dst[kept_seen] = jb + u; ++kept_seen; }
+                      for (int u = 0; u < 32; ++u)
+                        if ((keepm >> u) & 1u) dst[jb + u] = jb + u;
+                    } else {
+#pragma unroll
+                      for (int u = 0; u < 32; ++u)
+                        if ((keepm >> u) & 1u) { if (kept_seen < a.N) dst[kept_seen] = jb + u; ++kept_seen; }
+                    }
                   }
                 } else if (kHasPv || kHasCodes) {
                   float e[32];
@@ -721,11 +754,27 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
     }
 
     // ============================================================== per-row decisions after the pass
+    if (kSplit == 2 && pass == P_NORM) {
+      // the row's two threads combine their partial normalizers (and running maxima)
+      if (is_soft && half == 1) { xchg[srow] = lsum; xchg[kM + srow] = m; }
+      __syncthreads();
+      if (is_soft && half == 0) {
+        const float l1 = xchg[srow], m1 = xchg[kM + srow];
+        if (use_lut) {
+          lsum += l1;
+        } else {
+          const float mm = fmaxf(m, m1);
+          if (mm != -INFINITY)
+            lsum = lsum * fast_exp2((m - mm) * kLog2e) + l1 * fast_exp2((m1 - mm) * kLog2e);
+          m = mm;
+        }
+      }
+    }
     if (tid < kM && row_ok && !*abort_flag) {
       if (pass == P_LEVELS) {
         int cnt[kLevels];
 #pragma unroll
-        for (int lev = 0; lev < kLevels; ++lev) cnt[lev] = (int)hist[lev * kM + tid];
+        for (int lev = 0; lev < kLevels; ++lev) cnt[lev] = (int)hist[lev * kM + srow];
         int hmin = 64, hN = 64, cum = 0;
         bool found = false;
 #pragma unroll
@@ -758,7 +807,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
 #pragma unroll
           for (int lev = 0; lev < kLevels; ++lev) {
             const float lv = (float)(64 - 2 * lev) * c;
-            wt[lev * kM + tid] = (lv >= F) ? fast_exp2((lv - m) * kLog2e) : 0.0f;
+            wt[lev * kM + srow] = (lv >= F) ? fast_exp2((lv - m) * kLog2e) : 0.0f;
           }
         } else {
           const float bmin = a.bminmax[2 * h], bmax = a.bminmax[2 * h + 1];
@@ -775,7 +824,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       } else if (pass == P_RADIX && r_state == 1) {
         int cum = 0, bsel = kRadixBins - 1, kbin = 0;
         for (int bb = 0; bb < kRadixBins; ++bb) {
-          const int k = (int)hist[bb * kM + tid];
+          const int k = (int)hist[bb * kM + srow];
           if (cum + k >= r_rank) { bsel = bb; kbin = k; break; }
           cum += k;
         }
@@ -805,17 +854,17 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
         if (r_cnt > kCandCap) raise_status(a.status, kDevErrCapacity);
         uint32_t uF = 0u;
         for (int x = 0; x < nc; ++x) {
-          const uint2 cx = cand[x * kM + tid];
+          const uint2 cx = cand[x * kM + srow];
           int before = 0;
           for (int y = 0; y < nc; ++y) {
-            const uint2 cy = cand[y * kM + tid];
+            const uint2 cy = cand[y * kM + srow];
             before += (cy.x > cx.x || (cy.x == cx.x && cy.y < cx.y)) ? 1 : 0;
           }
           if (before == r_rank - 1) uF = cx.x;
         }
         int gt = 0, eq = 0;
         for (int x = 0; x < nc; ++x) {
-          const uint32_t ux = cand[x * kM + tid].x;
+          const uint32_t ux = cand[x * kM + srow].x;
           gt += ux > uF ? 1 : 0;
           eq += ux == uF ? 1 : 0;
         }
@@ -829,6 +878,12 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       } else if (pass == P_NORM) {
         scale = (MODE == MODE_Q || EXPORT == EXP_CODES) ? 255.0f / lsum : 1.0f / lsum;
       }
+    }
+    if (kSplit == 2 && pass == P_NORM) {
+      __syncthreads();
+      if (is_soft && half == 0) { xchg[srow] = scale; xchg[kM + srow] = m; }
+      __syncthreads();
+      if (is_soft && half == 1) { scale = xchg[srow]; m = xchg[kM + srow]; }
     }
     tie_seen = 0;
     // ---- the CTA chooses the next pass
@@ -845,7 +900,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
     else if (EXPORT == EXP_CODES) next = P_CODES;
     else next = P_PV;
     if (next == P_RADIX && tid < kM)
-      for (int bb = 0; bb < kRadixBins; ++bb) hist[bb * kM + tid] = 0u;
+      for (int bb = 0; bb < kRadixBins; ++bb) hist[bb * kM + srow] = 0u;
     if (next == P_KEPT_NORM && tid < kM) lsum = 0.0f;
     __syncthreads();
     first_pass = false;
@@ -853,46 +908,54 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
   }
 
   // ---------------------------------------------------------------- epilogue
+  if (kSplit == 2 && sum_in_pv) {
+    // the row's two threads add their partial normalizers
+    if (is_soft) xchg[half * kM + srow] = lsum;
+    __syncthreads();
+    if (is_soft) lsum = xchg[srow] + xchg[kM + srow];
+  }
   if (EXPORT == EXP_NONE) {
-    if (tid < kM) {
+    if (is_soft) {
+      constexpr int kOc = kD / kSplit;               // output channels per softmax thread
+      const int c0 = (kSplit == 2) ? kOc * half : 0;  // first channel
       const bool ok = __all_sync(0xffffffffu, bounded_wait(B_OFULL, 0));
       tc_fence_after();
-      const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-      uint32_t o[64];
-      tmem_ld32(tl + kColO, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
-      tmem_ld32(tl + kColO + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+      const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+      uint32_t o[kOc];
+      tmem_ld32(tl + kColO + c0, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+      if (kOc == 64) tmem_ld32(tl + kColO + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[kOc - 32]));
       tmem_wait_ld();
       if (row < a.n) {
-        float out[64];
+        float out[kOc];
         if (!ok || !row_ok) {
 #pragma unroll
-          for (int k = 0; k < 64; ++k) out[k] = 0.0f;
+          for (int k = 0; k < kOc; ++k) out[k] = 0.0f;
         } else if (MODE == MODE_Q) {
 #pragma unroll
-          for (int k = 0; k < 64; ++k) out[k] = (float)(int)o[k] * dq[k];
+          for (int k = 0; k < kOc; ++k) out[k] = (float)(int)o[k] * dq[c0 + k];
         } else {
           const float inv = sum_in_pv ? 1.0f / lsum : scale;
 #pragma unroll
-          for (int k = 0; k < 64; ++k) out[k] = __uint_as_float(o[k]) * inv;
+          for (int k = 0; k < kOc; ++k) out[k] = __uint_as_float(o[k]) * inv;
         }
-        const size_t ob = ((size_t)bh * a.n + row) * kD;
+        const size_t ob = ((size_t)bh * a.n + row) * kD + c0;
         if (a.o_bf16) {
           uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.O) + ob);
 #pragma unroll
-          for (int k = 0; k < 8; ++k)
+          for (int k = 0; k < kOc / 8; ++k)
             dst[k] = make_uint4(pack_bf16x2(out[8 * k], out[8 * k + 1]), pack_bf16x2(out[8 * k + 2], out[8 * k + 3]),
                                 pack_bf16x2(out[8 * k + 4], out[8 * k + 5]), pack_bf16x2(out[8 * k + 6], out[8 * k + 7]));
         } else {
           float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.O) + ob);
 #pragma unroll
-          for (int k = 0; k < 16; ++k) dst[k] = make_float4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
+          for (int k = 0; k < kOc / 4; ++k) dst[k] = make_float4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
         }
       }
     }
   } else if (EXPORT == EXP_IDX) {
     if (tid < kM && row < a.n) {
       int32_t* dst = a.idx + ((size_t)bh * a.n + row) * a.N;
-      for (int p = row_ok ? min(kept_seen, a.N) : 0; p < a.N; ++p) dst[p] = -1;
+      for (int p = row_ok ? min(SEL == SEL_DENSE ? L : kept_seen, a.N) : 0; p < a.N; ++p) dst[p] = -1;
     }
   } else {
     if (tid < kM && row >= a.row_begin && row < a.row_end && row < a.n) {
@@ -903,7 +966,7 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
   }
 
   // ---------------------------------------------------------------- teardown
-  if (warp == 5 && lane == 0 && *abort_flag) {
+  if (warp == kProdWarp && lane == 0 && *abort_flag) {
     // let TMA loads still in flight land before the CTA's shared memory goes away
     for (int s2 = 0; s2 < kKStages; ++s2)
       if (k_par[s2] >= 0) mbar_wait(&bars[B_KFULL + s2], (uint32_t)k_par[s2], 200000000LL);
@@ -911,14 +974,14 @@ __global__ void __launch_bounds__(kThreads, 2) k_attn_tc(const __grid_constant__
       if (v_par[s2] >= 0) mbar_wait(&bars[B_VFULL + s2], (uint32_t)v_par[s2], 200000000LL);
     if (BIAS == BIAS_SMEM) mbar_wait(&bars[B_BIAS], 0, 200000000LL);
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == kMmaWarp && lane == 0) {
     // every tcgen05 operation this thread issued is complete before TMEM is freed
     mma_commit(&bars[B_FINAL]);
     mbar_wait(&bars[B_FINAL], 0, 200000000LL);
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }

@@ -351,7 +351,7 @@ had_status launch_tc_t(const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
       configured[dev] = true;
     }
   }
-  fn<<<grid, tc::kThreads, smem, st>>>(a);
+  fn<<<grid, tc::cta_threads(SEL), smem, st>>>(a);
   return check_launch("k_attn_tc");
 }
 
