@@ -123,6 +123,25 @@ def path_bytes_per_token(mode: str, in_bytes: int, o_bytes: int) -> int:
     return b
 
 
+# ----------------------------------------------------------------------------- ranks
+
+def max_over_ranks(x: float, dist=None, device="cpu") -> float:
+    """The max of a per-rank scalar over all ranks of the process group (the
+    value itself without one).  Every multi-GPU time is reported this way."""
+    if dist is None:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, world: int, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: every rank processes `units_per_rank` per step (weak
+    scaling), and the job takes the slowest rank's time."""
+    return units_per_rank * world * steps / (total_ms * 1e-3)
+
+
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
@@ -336,13 +355,9 @@ def run_gpu(args, rank, world, local_rank):
             dist.barrier()
     step_ms = [e[0].elapsed_time(e[2]) for e in ev]
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
-    total_ms = sum(step_ms)
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, dev)
     queries = w.valid_tokens
-    value = queries * world * args.steps / (total_ms * 1e-3)
+    value = whole_job_rate(queries, world, args.steps, total_ms)
     ms_per_step = total_ms / args.steps
 
     # e2e: pinned host -> device, the call, device -> host of O, every step
@@ -363,11 +378,7 @@ def run_gpu(args, rank, world, local_rank):
             hO.copy_(O, non_blocking=True)
         e1.record(stream)
         stream.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, dev)
 
     if rank != 0:
         return 0
@@ -392,7 +403,7 @@ def run_gpu(args, rank, world, local_rank):
         "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u8i8" if mode == "u8i8" else ("bf16" if bf16 else "f32"),
         "data": "synthetic", "config": {**_config(w, N, mode), "parallelism": f"replicas x{world} (no collective)"},
-        "score_ops_per_s": w.valid_scores() * world * args.steps / (total_ms * 1e-3),
+        "score_ops_per_s": whole_job_rate(w.valid_scores(), world, args.steps, total_ms),
         "roofline": {"bound": "alu", "kernel": "k_attn_tc (fused score/top-N/softmax/A.V)",
                      "achieved": alu_achieved, "peak": ALU_PEAK_TOPS, "unit": "Tlane-op/s",
                      "frac": alu_achieved / ALU_PEAK_TOPS, "traffic": traffic,
@@ -404,7 +415,7 @@ def run_gpu(args, rank, world, local_rank):
                          "peak_kind": peak_kind},
         "roofline_path": {"bound": "hbm", "achieved": path_achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                           "frac": path_achieved / peaks["hbm_gbs"], "algorithmic_bytes_per_step": pbytes},
-        "e2e": {"value": queries * world / (e2e_ms * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": whole_job_rate(queries, world, 1, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": kernels_per_step * args.steps,
         "clocks": clk,
