@@ -225,6 +225,14 @@ __global__ void __launch_bounds__(cta_threads(SEL), 2) k_attn_tc(const __grid_co
   }
 
   // ---------------------------------------------------------------- setup
+  int k_par[kKStages], v_par[kVStages];  // producer: parity of the last load per stage (-1 none)
+#pragma unroll
+  for (int s2 = 0; s2 < kKStages; ++s2) k_par[s2] = -1;
+#pragma unroll
+  for (int s2 = 0; s2 < kVStages; ++s2) v_par[s2] = -1;
+  // the producer issues the first K tiles before the CTA-wide setup barrier, so
+  // their load latency overlaps the staging of Q
+  const int k_pre = min((L + kN - 1) / kN, kKStages);
   if (warp == kMmaWarp) {
     tmem_alloc(misc, kTmemCols);
     tmem_relinquish();
@@ -245,6 +253,11 @@ __global__ void __launch_bounds__(cta_threads(SEL), 2) k_attn_tc(const __grid_co
     }
     prefetch_tensormap(&a.tm_k);
     if (EXPORT == EXP_NONE) prefetch_tensormap(MODE == MODE_Q ? &a.tm_vq : &a.tm_v);
+    for (int t = 0; t < k_pre; ++t) {  // stage t = tile t, first use of every stage
+      mbar_arrive_expect_tx(&bars[B_KFULL + t], kN * kD);
+      tma_load_2d(sm + SM::kK + t * kN * kD, &a.tm_k, 0, bh * a.n_pad + t * kN, &bars[B_KFULL + t]);
+      k_par[t] = 0;
+    }
   }
   const int row = q0 + srow;  // softmax threads
   const bool row_ok = is_soft && row < L;
@@ -311,16 +324,12 @@ __global__ void __launch_bounds__(cta_threads(SEL), 2) k_attn_tc(const __grid_co
   int sF = 0;  // integer threshold score (top-N without bias)
 
   uint32_t g_k = 0, g_v = 0, g_s = 0;  // tiles issued so far (all passes), per role
-  int k_par[kKStages], v_par[kVStages];          // producer: parity of the last load per stage (-1 none)
-#pragma unroll
-  for (int s2 = 0; s2 < kKStages; ++s2) k_par[s2] = -1;
-#pragma unroll
-  for (int s2 = 0; s2 < kVStages; ++s2) v_par[s2] = -1;
 
   int pass = (SEL == SEL_DENSE) ? (EXPORT == EXP_IDX ? P_IDX : P_NORM) : P_LEVELS;
   if (SEL == SEL_DENSE && EXPORT == EXP_NONE && MODE == MODE_F && use_lut) pass = P_PV;
 
   auto bounded_wait = [&](int bar, uint32_t parity) -> bool {
+    if (mbar_test_wait(smem_u32(&bars[bar]), parity)) return true;  // phase already complete
     if (*abort_flag) return false;
     if (mbar_wait(&bars[bar], parity, kWaitCycles)) return true;
     *abort_flag = 1u;
@@ -354,7 +363,9 @@ __global__ void __launch_bounds__(cta_threads(SEL), 2) k_attn_tc(const __grid_co
         ++g_v;
       };
       for (int t = 0; t < ntiles; ++t) {
-        if (!k_res || first_pass) {
+        if (first_pass && t < k_pre) {
+          ++g_k;  // issued during setup
+        } else if (!k_res || first_pass) {
           const uint32_t st = k_res ? (uint32_t)t : g_k % kKStages;
           if (!k_res && lane == 0 && g_k >= (uint32_t)kKStages)
             bounded_wait(B_KEMPTY + st, ((g_k / kKStages) - 1) & 1);
