@@ -63,14 +63,14 @@ constexpr int kCandCap = 64;
 constexpr int kSBufs = 3;
 constexpr uint32_t kColS = 0, kColO = 192, kTmemCols = 256;
 constexpr long long kWaitCycles = 2000000000LL;  // about one second
-// How the softmax threads find the bias offset koff(j) = y_j * tw + x_j of a key:
+// How the softmax threads find the bias offset koff(j) = y_j * S + x_j of a key (S: table row stride):
 constexpr int kKoffTable = 0;  // per-head table in shared memory (n_pad <= kKoffTableMax)
 constexpr int kKoffWarp = 1;   // each softmax warp computes the tile's 64 offsets (double-buffered)
 constexpr int kKoffTableMax = 1024;
 // Bias variants of the kernel: none, extended tables read from global memory,
 // or (dense) the exp(bias) table staged in shared memory.
 enum { BIAS_NONE = 0, BIAS_GLOBAL = 1, BIAS_SMEM = 2 };
-constexpr int kBiasSmemMax = 4096;  // extended exp(bias) tables up to this many entries are staged in shared memory
+constexpr int kBiasSmemMax = 6144;  // extended exp(bias) tables up to this many entries are staged in shared memory
 
 enum { SEL_DENSE = 0, SEL_TOPN_INT = 1, SEL_TOPN_FLOAT = 2 };
 enum { MODE_F = 0, MODE_Q = 1 };
@@ -89,7 +89,7 @@ struct TcArgs {
   const float* bminmax;    // [H][2] min/max of each head's table (0 included with class tokens)
   const float* expb;       // [H][E] extended exp(b - b_max(h)) table, or null
   const float* bext;       // [H][E] extended bias table, or null
-  int ext_E, rb_class, k_class, k_invalid;  // extended-table geometry (RelposExt)
+  int ext_E, ext_S, rb_class, k_class, k_invalid;  // extended-table geometry (RelposExt)
   int int_levels;          // 1 if fp32(c*s) is strictly increasing in s for every head
   int koff_mode;           // kKoffTable / kKoffWarp
   const int32_t* seqlens;
@@ -139,13 +139,13 @@ enum {
   B_BIAS  // staged exp(bias) table landed
 };
 
-// Bias offset of key j: koff = y_j * tw + x_j for patch tokens, so that
+// Bias offset of key j: koff = y_j * S + x_j for patch tokens, so that
 // b_ij = ext[rb(i) - koff(j)]; class tokens and keys past L index the extension.
 __device__ __forceinline__ int key_offset(const TcArgs& a, int j, int L) {
   if (j >= L) return a.k_invalid;
   if (j < a.prefix) return a.k_class;
   const int t = j - a.prefix;
-  return (t / a.gw) * a.tw + t % a.gw;
+  return (t / a.gw) * a.ext_S + t % a.gw;
 }
 
 // TMEM column (within a tile's P) of bf16 K-step k (16 keys): chunk k/2 sits in
@@ -308,7 +308,7 @@ __global__ void __launch_bounds__(cta_threads(SEL), 2) k_attn_tc(const __grid_co
     rb = a.rb_class;
     if (row >= a.prefix && row < a.n) {
       const int t = row - a.prefix;
-      rb = (t / a.gw + a.gh - 1) * a.tw + (t % a.gw + a.gw - 1);
+      rb = (t / a.gw + a.gh - 1) * a.ext_S + (t % a.gw + a.gw - 1);
     }
   }
   const float* tab = HAS_BIAS ? a.bext + (size_t)h * a.ext_E : nullptr;
@@ -488,7 +488,7 @@ __global__ void __launch_bounds__(cta_threads(SEL), 2) k_attn_tc(const __grid_co
         if (x >= a.gw) { x -= a.gw; ++y; }
       };
       auto offset_of = [&](int j, int y, int x) -> int {
-        return 4 * (j >= L ? a.k_invalid : (j < a.prefix ? a.k_class : y * a.tw + x));  // in bytes
+        return 4 * (j >= L ? a.k_invalid : (j < a.prefix ? a.k_class : y * a.ext_S + x));  // in bytes
       };
       if (BIAS == BIAS_SMEM && first_pass) bounded_wait(B_BIAS, 0);
       for (int t = 0; t < ntiles; ++t) {

@@ -22,26 +22,27 @@ __device__ __forceinline__ void raise_status(unsigned* status, unsigned bits) {
   if (status) atomicOr(status, bits);
 }
 
-// Valid length of sequence b; an out-of-range entry raises the device status
-// and returns 0, which makes every kernel treat that batch as empty (zero output).
-// Extended relative-position tables.  Entry rb(i) - koff(j) of the raw
-// (2gh-1) x (2gw-1) table is the bias of patch query i and patch key j.  The
-// extension appends regions that the same subtraction reaches for class-token
-// queries (rb = rb_class), class-token keys (koff = k_class) and keys at or past
-// the valid length (koff = k_invalid), so a kernel reads one table entry per
-// (query, key) pair with no case analysis:
-//   [0, T)              the table, T = (2gh-1)(2gw-1)
+// Extended relative-position tables.  Entry rb(i) - koff(j) of the table is the
+// bias of patch query i and patch key j, the (2gh-1) x (2gw-1) table being
+// stored with a padded row stride S (the smallest S >= 2gw-1 with S = gw mod 32:
+// the 32 consecutive query tokens of a warp then read 32 different shared-memory
+// banks).  The extension appends regions that the same subtraction reaches for
+// class-token queries (rb = rb_class), class-token keys (koff = k_class) and keys
+// at or past the valid length (koff = k_invalid), so a kernel reads one table
+// entry per (query, key) pair with no case analysis:
+//   [0, T)              the table, T = (2gh-1) S (columns >= 2gw-1 unused)
 //   [T, 2T + 2Kx)       class-token pairs (bias 0)
 //   [2T + 2Kx, E)       keys past L (weight 0 / logit -inf), E = 3T + 3Kx rounded up to 4
-// with Kx = (gh-1)(2gw-1) + gw the number of distinct patch key offsets.
+// with Kx = (gh-1) S + gw the number of distinct patch key offsets y S + x.
 struct RelposExt {
-  int T, Kx, E, rb_class, k_class, k_invalid;
+  int S, T, Kx, E, rb_class, k_class, k_invalid;
 };
 __host__ __device__ inline RelposExt relpos_ext(int gh, int gw) {
   RelposExt r;
   const int tw = 2 * gw - 1;
-  r.T = (2 * gh - 1) * tw;
-  r.Kx = (gh - 1) * tw + gw;
+  r.S = tw + (((gw - tw) % 32) + 32) % 32;
+  r.T = (2 * gh - 1) * r.S;
+  r.Kx = (gh - 1) * r.S + gw;
   r.E = (3 * r.T + 3 * r.Kx + 3) / 4 * 4;  // padded to 16 bytes per head (bulk copies)
   r.rb_class = r.T - 1 + r.Kx;
   r.k_class = -(r.T + r.Kx);
@@ -49,6 +50,8 @@ __host__ __device__ inline RelposExt relpos_ext(int gh, int gw) {
   return r;
 }
 
+// Valid length of sequence b; an out-of-range entry raises the device status
+// and returns 0, which makes every kernel treat that batch as empty (zero output).
 __device__ __forceinline__ int valid_len(const int32_t* seqlens, int b, int n, unsigned* status) {
   if (!seqlens) return n;
   int L = seqlens[b];

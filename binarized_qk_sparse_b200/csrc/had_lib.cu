@@ -433,7 +433,7 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
   a.bext = has_bias ? reinterpret_cast<float*>(ws + w.bext) : nullptr;
   if (has_bias) {
     const RelposExt x = relpos_ext(bias->gh, bias->gw);
-    a.ext_E = x.E; a.rb_class = x.rb_class; a.k_class = x.k_class; a.k_invalid = x.k_invalid;
+    a.ext_E = x.E; a.ext_S = x.S; a.rb_class = x.rb_class; a.k_class = x.k_class; a.k_invalid = x.k_invalid;
   }
   a.seqlens = s->seqlens;
   a.O = O; a.o_bf16 = (o_dtype == HAD_BF16) ? 1 : 0;

@@ -257,9 +257,10 @@ struct BiasArgs {
 __device__ __forceinline__ void bias_tables_block(const BiasArgs& a, int h) {
   __shared__ float smn[32], smx[32];
   const RelposExt x = relpos_ext(a.gh, a.gw);
-  const float* t = a.table + (size_t)h * x.T;
+  const int tw = 2 * a.gw - 1, cells = (2 * a.gh - 1) * tw;
+  const float* t = a.table + (size_t)h * cells;
   float mn = INFINITY, mx = -INFINITY;
-  for (int e = threadIdx.x; e < x.T; e += blockDim.x) { mn = fminf(mn, t[e]); mx = fmaxf(mx, t[e]); }
+  for (int e = threadIdx.x; e < cells; e += blockDim.x) { mn = fminf(mn, t[e]); mx = fmaxf(mx, t[e]); }
   for (int o = 16; o > 0; o >>= 1) {
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -277,7 +278,11 @@ __device__ __forceinline__ void bias_tables_block(const BiasArgs& a, int h) {
   const int z0 = 2 * x.T + 2 * x.Kx;
   for (int e = threadIdx.x; e < x.E; e += blockDim.x) {
     float b, w;
-    if (e < x.T) { b = t[e]; w = exp2f((b - mx) * kLog2e); }
+    if (e < x.T) {  // table row e / S, column e % S (columns past 2gw-2 are padding)
+      const int dy = e / x.S, dx = e - dy * x.S;
+      b = dx < tw ? t[dy * tw + dx] : 0.0f;
+      w = exp2f((b - mx) * kLog2e);
+    }
     else if (e < z0) { b = 0.0f; w = e_class; }
     else { b = -INFINITY; w = 0.0f; }
     be[e] = b;
