@@ -49,12 +49,14 @@ using namespace had::sm100;
 
 constexpr int kM = 128;            // query rows per CTA (TMEM lanes)
 constexpr int kN = 64;             // keys per tile (score MMA N)
-// Softmax threads per query row: dense attention splits each 64-key tile between
-// two threads (warps w and w + 4 share the TMEM lanes of quadrant w), which
-// doubles the warps that hide latency; top-N keeps one thread per row (its tie
-// and kept-index bookkeeping runs in key order).
-__host__ __device__ constexpr int row_split(int sel) { return sel == 0 ? 2 : 1; }
-__host__ __device__ constexpr int cta_threads(int sel) { return 32 * (4 * row_split(sel) + 2); }
+// Softmax threads per query row (SPLIT): dense attention always, and top-N without
+// a bias on its P.V path for short ragged rows, split each 64-key tile between two threads
+// (warps w and w + 4 share the TMEM lanes of quadrant w), which doubles the warps
+// that hide latency; the two threads of a top-N row exchange their threshold-tie
+// counts every tile so that ties are still kept in key order.  Long top-N rows,
+// top-N with a bias and the top-N exports keep one thread per row.
+__host__ __device__ constexpr int cta_threads(int split) { return 32 * (4 * split + 2); }
+constexpr int kSplitMaxKeys = 256;  // top-N without a bias, ragged rows: two threads per row up to this n_pad
 constexpr int kKStages = 4;
 constexpr int kVStages = 2;
 constexpr int kLevels = 65;
@@ -113,8 +115,9 @@ struct Smem {
   static constexpr int kV = kK + kKStages * kN * kD;             // 2 V stages
   static constexpr int kKoff = kV + kVStages * kVStage;          // bias key offsets (table, or 4 warps x 2 x 64)
   static constexpr int kBiasTab = kKoff + (HAS_BIAS ? kKoffTableMax * 4 : 0);  // exp(bias) table (dense)
-  static constexpr int kXchg = kBiasTab + (BIAS == BIAS_SMEM ? kBiasSmemMax * 4 : 0);  // 2 x 128 fp32 (row partials)
-  static constexpr int kDq = kXchg + 2 * kM * 4;                                        // 64 dequant scales
+  // row-pair exchange: dense 2 x 128 fp32 (partials); top-N 6 x 128 (threshold state) + 2 x 2 x 128 tie counts
+  static constexpr int kXchg = kBiasTab + (BIAS == BIAS_SMEM ? kBiasSmemMax * 4 : 0);
+  static constexpr int kDq = kXchg + (SEL == SEL_DENSE ? 2 : SEL == SEL_TOPN_INT ? 10 : 0) * kM * 4;  // 64 dequant scales
   static constexpr int kBar = kDq + kD * 4;
   static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 2 * kSBufs + 3;
   static constexpr int kMisc = kBar + kNumBars * 8;              // [0] tmem base [1] abort
@@ -152,6 +155,18 @@ __device__ __forceinline__ int key_offset(const TcArgs& a, int j, int L) {
 // its own 32 columns, 8 columns per 16 keys.
 __host__ __device__ constexpr uint32_t pcol(int k) { return 32u * (uint32_t)(k >> 1) + 8u * (uint32_t)(k & 1); }
 
+// Of this chunk's threshold ties `eqm` (bit u = key jb + u, in key order), the
+// ones the row keeps: ties are kept while fewer than r_F have been seen.
+__device__ __forceinline__ uint32_t tie_keep(uint32_t eqm, int cut, int rF, int tie_seen) {
+  uint32_t keep = eqm;
+  if (cut && eqm != 0u) {
+    const int allow = rF - tie_seen, cnt = __popc(eqm);
+    if (allow <= 0) keep = 0u;
+    else if (allow < cnt) keep = eqm & ((2u << __fns(eqm, 0u, allow)) - 1u);
+  }
+  return keep;
+}
+
 // Pairwise sum of 32 values (a depth-5 tree instead of a 32-long dependent chain).
 __device__ __forceinline__ float sum32(const float (&e)[32]) {
   float t[16];
@@ -164,12 +179,14 @@ __device__ __forceinline__ float sum32(const float (&e)[32]) {
   return t[0];
 }
 
-template <int SEL, int MODE, int BIAS, bool VF32, int EXPORT>
-__global__ void __launch_bounds__(cta_threads(SEL), 2) k_attn_tc(const __grid_constant__ TcArgs a) {
+template <int SEL, int MODE, int BIAS, bool VF32, int EXPORT, int SPLIT>
+__global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_constant__ TcArgs a) {
+  static_assert(SPLIT == 1 || SEL == SEL_DENSE || (SEL == SEL_TOPN_INT && EXPORT == EXP_NONE),
+                "two threads per row: dense, or top-N without a bias on its P.V path");
   static_assert(BIAS != BIAS_SMEM || SEL == SEL_DENSE, "staged exp(bias) tables serve the dense weights only");
-  constexpr int kSplit = row_split(SEL);
+  constexpr int kSplit = SPLIT;
   constexpr int kSoftWarps = 4 * kSplit;
-  constexpr int kThreads = cta_threads(SEL);
+  constexpr int kThreads = cta_threads(SPLIT);
   constexpr int kMmaWarp = kSoftWarps, kProdWarp = kSoftWarps + 1;
   constexpr int kChunks = 2 / kSplit;  // 32-key chunks of a tile per softmax thread
   constexpr bool HAS_BIAS = BIAS != BIAS_NONE;
@@ -282,9 +299,14 @@ __global__ void __launch_bounds__(cta_threads(SEL), 2) k_attn_tc(const __grid_co
       for (int lev = 0; lev < kLevels; ++lev) hist[lev * kM + srow] = 0u;
     if (SEL == SEL_DENSE) {
       // per-lane copies of the level table exp(c * (s - 64)), level k = (64 - s) / 2, at [k][lane]
+      // (each lane computes three levels; warp w writes levels w, w + 4, ... via shuffles)
       const float ck = -2.0f * a.c_head[h] * 1.4426950408889634f;
       float* lt = reinterpret_cast<float*>(hist);
-      for (int e = tid; e < kLevels * 32; e += kM) lt[e] = exp2f(ck * (float)(e >> 5));
+      const float lv0 = exp2f(ck * (float)lane), lv1 = exp2f(ck * (float)(lane + 32)), lv2 = exp2f(ck * 64.0f);
+      for (int lev = warp; lev < kLevels; lev += 4) {
+        const float v = __shfl_sync(0xffffffffu, lev < 32 ? lv0 : lv1, lev & 31);
+        lt[lev * 32 + lane] = lev == 64 ? lv2 : v;
+      }
     }
     if (MODE == MODE_Q && EXPORT == EXP_NONE && tid < kD) dq[tid] = __fdiv_rn(a.vscale[(size_t)bh * kD + tid], 255.0f);
     if (HAS_BIAS && a.koff_mode == kKoffTable)
@@ -751,7 +773,61 @@ __global__ void __launch_bounds__(cta_threads(SEL), 2) k_attn_tc(const __grid_co
             }
           }
         };
-        if (ok_wait) {
+        if (kSplit == 2 && SEL == SEL_TOPN_INT && pv) {
+          // top-N P.V with two threads per row: weights of this thread's chunk, then
+          // the row's two threshold-tie counts of this tile are exchanged (every live
+          // warp pair reaches the barrier, whatever happened to its waits)
+          const int jb = j0 + 32 * half;
+          const int nv = nvalid - 32 * half;  // valid keys of this chunk (<= 0: none)
+          float e[32];
+          uint32_t eqm = 0u;
+          if (ok_wait && jb < L) {
+            if (lut_w) {
+#pragma unroll
+              for (int u = 0; u < 32; ++u) {
+                const int sc = (int)r[u];
+                const bool valid = u < nv;
+                e[u] = valid ? lut[(32 - (sc >> 1)) * kM + srow] : 0.0f;
+                eqm |= (valid && sc == sF) ? (1u << u) : 0u;
+              }
+            } else {
+#pragma unroll
+              for (int u = 0; u < 32; ++u) {
+                const float l = (float)(int)r[u] * c;
+                const bool valid = u < nv;
+                e[u] = (valid && l >= F) ? fast_exp2(__fmaf_rn(l, kLog2e, mo)) : 0.0f;
+                eqm |= (valid && l == F) ? (1u << u) : 0u;
+              }
+            }
+          } else {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) e[u] = 0.0f;
+          }
+          int* tx = reinterpret_cast<int*>(xchg) + 6 * kM + (int)(gs & 1u) * 2 * kM;
+          tx[half * kM + srow] = __popc(eqm);
+          asm volatile("bar.sync %0, 64;" ::"r"(1 + (warp & 3)) : "memory");
+          const int c0 = tx[srow], c1 = tx[kM + srow];
+          const uint32_t dropm = eqm & ~tie_keep(eqm, cut, rF, tie_seen + (half ? c0 : 0));
+          if (dropm) {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) e[u] = ((dropm >> u) & 1u) ? 0.0f : e[u];
+          }
+          tie_seen += c0 + c1;
+          if (ok_wait) {
+            if (jb >= L) {
+              if (MODE == MODE_Q) {
+                const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                tmem_st8(tl + colP + 32 * half, z);
+              } else {
+                const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+                tmem_st16(tl + colP + 32 * half, z);
+                if (VF32) tmem_st16(tl + colP + 32 * half + 16, z);
+              }
+            } else {
+              emit(e, half);
+            }
+          }
+        } else if (ok_wait) {
           if (full_tile) tile_body(std::true_type{});
           else tile_body(std::false_type{});
         }
@@ -765,6 +841,9 @@ __global__ void __launch_bounds__(cta_threads(SEL), 2) k_attn_tc(const __grid_co
     }
 
     // ============================================================== per-row decisions after the pass
+    // two threads per top-N row: both have finished adding to the row's level
+    // histogram before the first reads it (and overwrites it with the weight table)
+    if (kSplit == 2 && SEL == SEL_TOPN_INT && pass == P_LEVELS) __syncthreads();
     if (kSplit == 2 && pass == P_NORM) {
       // the row's two threads combine their partial normalizers (and running maxima)
       if (is_soft && half == 1) { xchg[srow] = lsum; xchg[kM + srow] = m; }
@@ -888,6 +967,21 @@ __global__ void __launch_bounds__(cta_threads(SEL), 2) k_attn_tc(const __grid_co
         scale = 255.0f / lsum;
       } else if (pass == P_NORM) {
         scale = (MODE == MODE_Q || EXPORT == EXP_CODES) ? 255.0f / lsum : 1.0f / lsum;
+      }
+    }
+    if (kSplit == 2 && SEL == SEL_TOPN_INT && pass == P_LEVELS) {
+      // the row's threshold state (and its weight table, written above) to the second thread
+      __syncthreads();
+      if (is_soft && half == 0) {
+        xchg[srow] = F; xchg[kM + srow] = m; xchg[2 * kM + srow] = scale;
+        xchg[3 * kM + srow] = __int_as_float(sF); xchg[4 * kM + srow] = __int_as_float(rF);
+        xchg[5 * kM + srow] = __int_as_float(cut);
+      }
+      __syncthreads();
+      if (is_soft && half == 1) {
+        F = xchg[srow]; m = xchg[kM + srow]; scale = xchg[2 * kM + srow];
+        sF = __float_as_int(xchg[3 * kM + srow]); rF = __float_as_int(xchg[4 * kM + srow]);
+        cut = __float_as_int(xchg[5 * kM + srow]);
       }
     }
     if (kSplit == 2 && pass == P_NORM) {

@@ -335,10 +335,10 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
   return HAD_OK;
 }
 
-template <int SEL, int MODE, int BIAS, bool VF32, int EXP>
+template <int SEL, int MODE, int BIAS, bool VF32, int EXP, int SPLIT>
 had_status launch_tc_t(const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
   const int smem = tc::Smem<SEL, VF32, BIAS>::kTotal;
-  auto fn = tc::k_attn_tc<SEL, MODE, BIAS, VF32, EXP>;
+  auto fn = tc::k_attn_tc<SEL, MODE, BIAS, VF32, EXP, SPLIT>;
   static std::mutex mu;
   static bool configured[kMaxDevices] = {false};
   int dev = 0;
@@ -351,7 +351,7 @@ had_status launch_tc_t(const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
       configured[dev] = true;
     }
   }
-  fn<<<grid, tc::cta_threads(SEL), smem, st>>>(a);
+  fn<<<grid, tc::cta_threads(SPLIT), smem, st>>>(a);
   return check_launch("k_attn_tc");
 }
 
@@ -359,9 +359,19 @@ had_status launch_tc_t(const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
 template <int SEL, int MODE, bool VF32, int EXP>
 had_status launch_tc_b(int bias, const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
   using namespace tc;
-  if (bias == BIAS_SMEM) return launch_tc_t<SEL, MODE, BIAS_SMEM, VF32, EXP>(a, grid, st);
-  if (bias == BIAS_GLOBAL) return launch_tc_t<SEL, MODE, BIAS_GLOBAL, VF32, EXP>(a, grid, st);
-  return launch_tc_t<SEL, MODE, BIAS_NONE, VF32, EXP>(a, grid, st);
+  if (bias == BIAS_SMEM) return launch_tc_t<SEL, MODE, BIAS_SMEM, VF32, EXP, 2>(a, grid, st);
+  if (bias == BIAS_GLOBAL) return launch_tc_t<SEL, MODE, BIAS_GLOBAL, VF32, EXP, 2>(a, grid, st);
+  return launch_tc_t<SEL, MODE, BIAS_NONE, VF32, EXP, 2>(a, grid, st);
+}
+
+// Top-N without a bias: two threads per row on the P.V path of short ragged rows
+// (per-sequence lengths, n <= 256), where a CTA's few tiles make it latency-bound;
+// on full-length rows the per-tile tie exchange costs more than the extra warps gain.
+template <int SEL, int MODE, bool VF32, int EXP>
+had_status launch_tc_n(const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
+  if (EXP == tc::EXP_NONE && a.n_pad <= tc::kSplitMaxKeys && a.seqlens != nullptr)
+    return launch_tc_t<SEL, MODE, tc::BIAS_NONE, VF32, EXP, (EXP == tc::EXP_NONE ? 2 : 1)>(a, grid, st);
+  return launch_tc_t<SEL, MODE, tc::BIAS_NONE, VF32, EXP, 1>(a, grid, st);
 }
 
 template <int EXP>
@@ -370,22 +380,22 @@ had_status dispatch_tc(int sel, int mode, int bias, bool vf32, const tc::TcArgs&
   if (EXP == EXP_CODES || (EXP == EXP_NONE && mode == MODE_Q)) {
     constexpr int E = EXP;
     if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_Q, false, E>(bias, a, grid, st);
-    if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_Q, BIAS_NONE, false, E>(a, grid, st);
-    return launch_tc_t<SEL_TOPN_FLOAT, MODE_Q, BIAS_GLOBAL, false, E>(a, grid, st);
+    if (sel == SEL_TOPN_INT) return launch_tc_n<SEL_TOPN_INT, MODE_Q, false, E>(a, grid, st);
+    return launch_tc_t<SEL_TOPN_FLOAT, MODE_Q, BIAS_GLOBAL, false, E, 1>(a, grid, st);
   }
   if (EXP == EXP_IDX) {
     if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, false, EXP>(bias, a, grid, st);
-    if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, BIAS_NONE, false, EXP>(a, grid, st);
-    return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, BIAS_GLOBAL, false, EXP>(a, grid, st);
+    if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, BIAS_NONE, false, EXP, 1>(a, grid, st);
+    return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, BIAS_GLOBAL, false, EXP, 1>(a, grid, st);
   }
   if (vf32) {
     if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, true, EXP>(bias, a, grid, st);
-    if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, BIAS_NONE, true, EXP>(a, grid, st);
-    return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, BIAS_GLOBAL, true, EXP>(a, grid, st);
+    if (sel == SEL_TOPN_INT) return launch_tc_n<SEL_TOPN_INT, MODE_F, true, EXP>(a, grid, st);
+    return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, BIAS_GLOBAL, true, EXP, 1>(a, grid, st);
   }
   if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, false, EXP>(bias, a, grid, st);
-  if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, BIAS_NONE, false, EXP>(a, grid, st);
-  return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, BIAS_GLOBAL, false, EXP>(a, grid, st);
+  if (sel == SEL_TOPN_INT) return launch_tc_n<SEL_TOPN_INT, MODE_F, false, EXP>(a, grid, st);
+  return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, BIAS_GLOBAL, false, EXP, 1>(a, grid, st);
 }
 
 // Stage 2: the fused kernel over a prepared workspace.

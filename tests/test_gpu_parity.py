@@ -325,6 +325,41 @@ def test_all_ties_keep_lowest_indices(oracle_mod):
     assert np.max(np.abs(O - ref)) <= _tol(w)
 
 
+@pytest.mark.parametrize("mode", ["float", "u8i8"])
+def test_threshold_ties_across_chunks_and_tiles(oracle_mod, mode):
+    # Integer score levels make many exact ties at the threshold; the values of N
+    # put the cut in different 32-key chunks and tiles of a row (the two threads
+    # of a row must keep ties in key order between them).  fp32 inputs make one
+    # wrongly kept key visible against the 1e-3 bar.
+    # Each case runs without and with per-sequence lengths (the library uses two
+    # threads per row for short ragged batches, one otherwise).  In uint8 mode a
+    # code may differ by one LSB from the oracle's fp64 rounding (the codes' own
+    # bar), which moves O by up to max|V|/255, so that is added to the O bar.
+    m = 1 if mode == "u8i8" else 0
+    w = _small(77, B=2, H=2, n=200, dtype="f32")
+    Q, K, V, seq, bias = _dev_inputs(w)
+    bar = _tol(w) + (float(np.max(np.abs(w.V))) / 255.0 if m else 0.0)
+    lens = np.array([200, 161], np.int32)
+    for N in (20, 40, 70, 100, 131, 180):
+        for sl in (None, lens):
+            seqt = None if sl is None else torch.from_numpy(sl).cuda()
+            O = had.had_attention(Q, K, V, N=N, mode=mode, seqlens=seqt).float().cpu().numpy()
+            ref = oracle_mod.attention(w.Q, w.K, w.V, N=N, mode=m, seqlens=sl).O
+            assert np.max(np.abs(O - ref)) <= bar, (N, sl, np.max(np.abs(O - ref)))
+    # every score equal: the kept set is keys 0..N-1 for any N
+    w = _small(78, B=1, H=1, n=200, dtype="f32")
+    w.Q[:] = 1.0
+    w.K[:] = -2.0
+    Q, K, V, seq, bias = _dev_inputs(w)
+    bar = _tol(w) + (float(np.max(np.abs(w.V))) / 255.0 if m else 0.0)
+    for N in (40, 100, 150):
+        for sl in (None, np.array([200], np.int32)):
+            seqt = None if sl is None else torch.from_numpy(sl).cuda()
+            O = had.had_attention(Q, K, V, N=N, mode=mode, seqlens=seqt).float().cpu().numpy()
+            ref = oracle_mod.attention(w.Q, w.K, w.V, N=N, mode=m, seqlens=sl).O
+            assert np.max(np.abs(O - ref)) <= bar, (N, sl, np.max(np.abs(O - ref)))
+
+
 def test_alpha_and_bias_ties(oracle_mod):
     # a bias table of few distinct values makes many exact logit ties
     w = _small(31, B=2, H=2, n=65)
