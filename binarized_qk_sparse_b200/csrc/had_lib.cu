@@ -260,6 +260,22 @@ int select_kind(const had_shape* s, const had_relpos_bias* bias, int N) {
   return SEL_DENSE;
 }
 
+// Opt-in dynamic shared memory of the short-head prep kernel, once per variant and device.
+had_status set_prep_smem(int which, int small, int dev) {
+  static std::mutex mu;
+  static bool done[2][2][kMaxDevices] = {};
+  std::lock_guard<std::mutex> lk(mu);
+  if (dev < 0 || dev >= kMaxDevices || done[which][small][dev]) return HAD_OK;
+  cudaError_t e;
+  if (which == 0 && small) e = cudaFuncSetAttribute(k_prep_head<__nv_bfloat16, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHeadMaxBytes);
+  else if (which == 0) e = cudaFuncSetAttribute(k_prep_head<__nv_bfloat16, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHeadMaxBytes);
+  else if (small) e = cudaFuncSetAttribute(k_prep_head<float, 128>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHeadMaxBytes);
+  else e = cudaFuncSetAttribute(k_prep_head<float, 256>, cudaFuncAttributeMaxDynamicSharedMemorySize, kHeadMaxBytes);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_prep_head)");
+  done[which][small][dev] = true;
+  return HAD_OK;
+}
+
 // Stage 1: statistics, sign/pack of Q and K, int8 V (uint8 mode), bias range (top-N with bias).
 had_status prepare_stage(const void* Q, const void* K, const void* V, const had_shape* s,
                          const had_relpos_bias* bias, int N, had_mode mode, bool need_v, void* workspace,
@@ -299,22 +315,13 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
     const int smem = (int)head_bytes;
     int dev = 0;
     cudaGetDevice(&dev);
-    static std::mutex mu;
-    static bool attr_set[2][kMaxDevices] = {{false}};
     const int which = (s->in_dtype == HAD_BF16) ? 0 : 1;
-    {
-      std::lock_guard<std::mutex> lk(mu);
-      if (dev >= 0 && dev < kMaxDevices && !attr_set[which][dev]) {
-        cudaError_t e = which == 0 ? cudaFuncSetAttribute(k_prep_head<__nv_bfloat16>,
-                                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kHeadMaxBytes)
-                                   : cudaFuncSetAttribute(k_prep_head<float>,
-                                                          cudaFuncAttributeMaxDynamicSharedMemorySize, kHeadMaxBytes);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_prep_head)");
-        attr_set[which][dev] = true;
-      }
-    }
-    if (which == 0) k_prep_head<__nv_bfloat16><<<grid, kHeadThreads, smem, st>>>(ha, ba);
-    else k_prep_head<float><<<grid, kHeadThreads, smem, st>>>(ha, ba);
+    const int small = head_bytes <= (size_t)kHeadSmallBytes ? 1 : 0;
+    if ((r = set_prep_smem(which, small, dev)) != HAD_OK) return r;
+    if (which == 0 && small) k_prep_head<__nv_bfloat16, 128><<<grid, 128, smem, st>>>(ha, ba);
+    else if (which == 0) k_prep_head<__nv_bfloat16, 256><<<grid, 256, smem, st>>>(ha, ba);
+    else if (small) k_prep_head<float, 128><<<grid, 128, smem, st>>>(ha, ba);
+    else k_prep_head<float, 256><<<grid, 256, smem, st>>>(ha, ba);
     if ((r = check_launch("k_prep_head")) != HAD_OK) return r;
   } else {
     r = launch_prep(s, Q, K, V, 0, do_v ? 3 : 2, sums, amax, nullptr, nullptr, qbits, nullptr, nullptr, kpm, vqT,

@@ -226,7 +226,9 @@ namespace had {
 // the mean (or scale), and the packed outputs -- Q sign bits, K as +-1 int8
 // rows, V as int8 V^T.  Same definitions as k_stats + k_pack.
 
-constexpr int kHeadThreads = 256;
+// Threads of a short-head CTA: 128 for heads up to kHeadSmallBytes (more CTAs per
+// SM, so more heads' loads overlap), 256 above.
+constexpr int kHeadSmallBytes = 48 * 1024;
 constexpr int kHeadMaxBytes = 128 * 1024;   // staged head: n * 64 * sizeof(T)
 
 struct HeadArgs {
@@ -303,7 +305,7 @@ __device__ __forceinline__ int quant_i8(float x, float sc, float rsc) {
   return (int)fminf(fmaxf(q, -127.0f), 127.0f);
 }
 
-template <typename T>
+template <typename T, int kHeadThreads>
 __global__ void __launch_bounds__(kHeadThreads) k_prep_head(const HeadArgs a, const BiasArgs ba) {
   if ((int)blockIdx.y == a.bias_slice) {  // the bias slice: one CTA per head
     if ((int)blockIdx.x < a.H) bias_tables_block(ba, blockIdx.x);
@@ -341,14 +343,15 @@ __global__ void __launch_bounds__(kHeadThreads) k_prep_head(const HeadArgs a, co
     }
     return *reinterpret_cast<const float2*>(q);
   };
-  // ---- channel statistic: warp g covers tokens g, g + 8, ... (all = g mod 8); lane p channels 2p, 2p+1
+  // ---- channel statistic: warp g covers tokens g, g + kGroups, ...; lane p channels 2p, 2p+1
+  // (with 8 warps every token of a warp is = g mod 8, so its swizzled column is fixed)
   {
     const int p = tid & 31, g = tid >> 5;
     const uint8_t* col = xs + pair_off(p, g);
     if (tz < 2) {
       double s0 = 0.0, s1 = 0.0;
       for (int i = g; i < L; i += kGroups) {
-        const float2 x = pair_load(col + i * kRow);
+        const float2 x = pair_load((kGroups % 8 == 0 ? col : xs + pair_off(p, i & 7)) + i * kRow);
         s0 += (double)x.x;
         s1 += (double)x.y;
       }
@@ -357,7 +360,7 @@ __global__ void __launch_bounds__(kHeadThreads) k_prep_head(const HeadArgs a, co
     } else {
       float m0 = 0.0f, m1 = 0.0f;
       for (int i = g; i < L; i += kGroups) {
-        const float2 x = pair_load(col + i * kRow);
+        const float2 x = pair_load((kGroups % 8 == 0 ? col : xs + pair_off(p, i & 7)) + i * kRow);
         m0 = fmaxf(m0, fabsf(x.x));
         m1 = fmaxf(m1, fabsf(x.y));
       }
