@@ -61,7 +61,7 @@ constexpr int kKStages = 4;
 constexpr int kVStages = 2;
 constexpr int kLevels = 65;
 constexpr int kRadixBins = 128;
-constexpr int kCandCap = 64;
+constexpr int kCandCap = 128;    // power of two (the collect slot wraps)
 constexpr int kSBufs = 3;
 constexpr uint32_t kColS = 0, kColO = 192, kTmemCols = 256;
 constexpr long long kWaitCycles = 2000000000LL;  // about one second
@@ -124,10 +124,10 @@ struct Smem {
   static constexpr int kHist = (kMisc + 16 + 127) / 128 * 128;
   static constexpr int kHistBytes = (SEL == SEL_DENSE) ? kLevels * 32 * 4
                                     : (SEL == SEL_TOPN_INT) ? kLevels * kM * 4
-                                    : kCandCap * kM * 8;
+                                    : kCandCap * kM * 4;
   static constexpr int kTotal = kHist + kHistBytes + 1024;       // + alignment slack
-  static_assert(kCandCap * kM * 8 >= kRadixBins * kM * 4, "radix histogram fits the candidate area");
-  static_assert(kCandCap * kM * 8 >= kLevels * kM * 4, "level histogram fits the candidate area");
+  static_assert(kCandCap >= kRadixBins && kCandCap >= kLevels, "radix and level histograms fit the candidate area");
+  static_assert((kCandCap & (kCandCap - 1)) == 0, "candidate slots wrap with a mask");
 };
 
 enum {
@@ -322,7 +322,9 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
   float F = -INFINITY, m = -INFINITY, scale = 1.0f, lsum = 0.0f;
   int rF = 0, cut = 0, tie_seen = 0, kept_seen = 0;
   uint32_t r_uhi = 0, r_span = 0;
-  int r_shift = 0, r_rank = 0, r_state = 0, r_bin = 0, r_cnt = 0;
+  int r_shift = 0, r_rank = 0, r_state = 0, r_cnt = 0;
+  int r_above = 0;      // keys above the first radix window (counted in that pass)
+  bool r_first = false;  // the next radix pass is the first of this row
   // row base of the extended bias tables: rb(i) - koff(j) indexes the pair (i, j);
   // class-token rows and rows past the tensor use the class-row base
   int rb = 0;
@@ -704,26 +706,57 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
                 for (int u = 0; u < 32; ++u) ex[u] = fast_exp2(__fmaf_rn(lg[u], kLog2e, mo2));
                 lsum += sum32(ex);
               } else if (kHasRadix && pass == P_RADIX) {
+                // histogram of the keys inside the window [r_uhi - r_span, r_uhi] (order keys;
+                // keys past L are -inf, below every window), and the count above it
                 if (r_state == 1) {
-#pragma unroll
-                  for (int u = 0; u < 32; ++u) {
-                    const uint32_t dd = r_uhi - float_order_key(lg[u]);
-                    if ((FULL || 32 * ch + u < nvalid) && dd <= r_span) atomicAdd(&hist[(dd >> r_shift) * kM + srow], 1u);
-                  }
-                }
-              } else if (kHasRadix && pass == P_COLLECT) {
-                if (r_state == 2) {
-                  uint2* cand = reinterpret_cast<uint2*>(hist);  // [64][128 rows]
+                  const uint32_t ulo = r_uhi - r_span;
 #pragma unroll
                   for (int u = 0; u < 32; ++u) {
                     const uint32_t key = float_order_key(lg[u]);
-                    const uint32_t dd = r_uhi - key;
-                    if ((FULL || 32 * ch + u < nvalid) && dd <= r_span && (int)(dd >> r_shift) == r_bin) {
-                      if (r_cnt < kCandCap) cand[r_cnt * kM + srow] = make_uint2(key, (uint32_t)(jb + u));
-                      ++r_cnt;
-                    }
+                    const uint32_t t = key - ulo;
+                    r_above += key > r_uhi ? 1 : 0;
+                    const uint32_t ad = hist_row + ((r_span - t) >> r_shift) * (uint32_t)(kM * 4);
+                    asm volatile(
+                        "{\n\t.reg .pred p;\n\tsetp.le.u32 p, %1, %2;\n\t@p red.shared.add.u32 [%0], 1;\n\t}" ::"r"(ad),
+                        "r"(t), "r"(r_span)
+                        : "memory");
                   }
                 }
+              } else if (kHasRadix && pass == P_COLLECT) {
+                // the order keys inside the window, one column per row: [kCandCap][128 rows]
+                // (the slot wraps, so a miscount stays in bounds and is reported after the pass)
+                if (r_state == 2) {
+                  const uint32_t ulo = r_uhi - r_span;
+#pragma unroll
+                  for (int u = 0; u < 32; ++u) {
+                    const uint32_t key = float_order_key(lg[u]);
+                    const uint32_t t = key - ulo;
+                    const uint32_t ad = hist_row + (uint32_t)(r_cnt & (kCandCap - 1)) * (uint32_t)(kM * 4);
+                    asm volatile(
+                        "{\n\t.reg .pred p;\n\tsetp.le.u32 p, %1, %2;\n\t@p st.shared.u32 [%0], %3;\n\t}" ::"r"(ad),
+                        "r"(t), "r"(r_span), "r"(key)
+                        : "memory");
+                    r_cnt += t <= r_span ? 1 : 0;
+                  }
+                }
+              } else if (SEL == SEL_TOPN_FLOAT && (pass == P_PV || pass == P_CODES)) {
+                // weights of the keys at or above F (keys past L are -inf, below it), then
+                // the ties at F past the row's remaining allowance rF dropped in key order
+                float e[32];
+                uint32_t eqm = 0u;
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                  const float x = fast_exp2(__fmaf_rn(lg[u], kLog2e, mo));
+                  e[u] = lg[u] >= F ? x : 0.0f;
+                  eqm |= (lg[u] == F ? 1u : 0u) << u;
+                }
+                const uint32_t dropm = eqm & ~tie_keep(eqm, cut, rF, tie_seen);
+                tie_seen += __popc(eqm);
+                if (dropm) {
+#pragma unroll
+                  for (int u = 0; u < 32; ++u) e[u] = ((dropm >> u) & 1u) ? 0.0f : e[u];
+                }
+                emit(e, ch);
               } else {
                 // keep mask in key order; ties at F counted per row
                 uint32_t keepm = 0;
@@ -900,18 +933,24 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
             wt[lev * kM + srow] = (lv >= F) ? fast_exp2((lv - m) * kLog2e) : 0.0f;
           }
         } else {
+          // the threshold lies in [sN c + b_min, sN c + b_max]: at least keff keys have a
+          // score >= sN (so a logit >= the low end), fewer than keff a score > sN (only
+          // those can exceed the high end); logits are monotone in (score, bias)
           const float bmin = a.bminmax[2 * h], bmax = a.bminmax[2 * h + 1];
           const float lo = __fmaf_rn((float)sN, c, bmin);
-          const float hi = __fmaf_rn((float)smax, c, bmax);
-          r_uhi = float_order_key(hi);
+          const float hw = __fmaf_rn((float)sN, c, bmax);
+          r_uhi = float_order_key(hw);
           r_span = r_uhi - float_order_key(lo);
           r_shift = 0;
           while ((r_span >> r_shift) >= (uint32_t)kRadixBins) ++r_shift;
           r_rank = keff;
+          r_first = true;
           r_state = 1;
-          m = hi;
+          m = __fmaf_rn((float)smax, c, bmax);  // no logit exceeds it
         }
       } else if (pass == P_RADIX && r_state == 1) {
+        if (r_first) r_rank -= r_above;  // rank within the first window
+        r_first = false;
         int cum = 0, bsel = kRadixBins - 1, kbin = 0;
         for (int bb = 0; bb < kRadixBins; ++bb) {
           const int k = (int)hist[bb * kM + srow];
@@ -926,37 +965,41 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
           rF = rank;
           cut = rank < kbin ? 1 : 0;
           r_state = 0;
-        } else if (kbin <= kCandCap) {
-          r_bin = bsel;
-          r_rank = rank;
-          r_state = 2;
-          r_cnt = 0;
         } else {
+          // the chosen bin becomes the window: collected if small, else binned again
           const uint32_t span_left = r_span - ((uint32_t)bsel << r_shift);
           r_uhi = uhi;
           r_span = min(((uint32_t)1 << r_shift) - 1u, span_left);
-          r_shift = r_shift > 7 ? r_shift - 7 : 0;
           r_rank = rank;
+          if (kbin <= kCandCap) {
+            r_state = 2;
+            r_cnt = 0;
+          } else {
+            r_shift = r_shift > 7 ? r_shift - 7 : 0;
+          }
         }
       } else if (pass == P_COLLECT && r_state == 2) {
-        const uint2* cand = reinterpret_cast<const uint2*>(hist);
+        // the r_rank-th largest collected key: the one with fewer than r_rank keys
+        // above it and at least r_rank at or above it
+        const uint32_t* cand = hist;
         const int nc = min(r_cnt, kCandCap);
         if (r_cnt > kCandCap) raise_status(a.status, kDevErrCapacity);
         uint32_t uF = 0u;
-        for (int x = 0; x < nc; ++x) {
-          const uint2 cx = cand[x * kM + srow];
-          int before = 0;
-          for (int y = 0; y < nc; ++y) {
-            const uint2 cy = cand[y * kM + srow];
-            before += (cy.x > cx.x || (cy.x == cx.x && cy.y < cx.y)) ? 1 : 0;
-          }
-          if (before == r_rank - 1) uF = cx.x;
-        }
         int gt = 0, eq = 0;
         for (int x = 0; x < nc; ++x) {
-          const uint32_t ux = cand[x * kM + srow].x;
-          gt += ux > uF ? 1 : 0;
-          eq += ux == uF ? 1 : 0;
+          const uint32_t kx = cand[x * kM + srow];
+          int g = 0, e = 0;
+          for (int y = 0; y < nc; ++y) {
+            const uint32_t ky = cand[y * kM + srow];
+            g += ky > kx ? 1 : 0;
+            e += ky == kx ? 1 : 0;
+          }
+          if (g < r_rank && r_rank <= g + e) {
+            uF = kx;
+            gt = g;
+            eq = e;
+            break;
+          }
         }
         const uint32_t bits = (uF & 0x80000000u) ? (uF & 0x7FFFFFFFu) : ~uF;
         F = __uint_as_float(bits);
@@ -1004,8 +1047,10 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
     else if ((EXPORT == EXP_CODES || MODE == MODE_Q) && SEL == SEL_TOPN_FLOAT && pass != P_KEPT_NORM) next = P_KEPT_NORM;
     else if (EXPORT == EXP_CODES) next = P_CODES;
     else next = P_PV;
-    if (next == P_RADIX && tid < kM)
+    if (next == P_RADIX && tid < kM) {
       for (int bb = 0; bb < kRadixBins; ++bb) hist[bb * kM + srow] = 0u;
+      r_above = 0;
+    }
     if (next == P_KEPT_NORM && tid < kM) lsum = 0.0f;
     __syncthreads();
     first_pass = false;
