@@ -73,6 +73,9 @@ def lib():
         L.had_attention_workspace_size.argtypes = [SP, I, I, BP]
         L.had_attention_workspace_size.restype = SZ
         L.had_attention.argtypes = [P, P, P, SP, BP, P, P, I, I, P, I, P, SZ, P]
+        L.had_attention_host_workspace_size.argtypes = [SP, I, I, BP, I]
+        L.had_attention_host_workspace_size.restype = SZ
+        L.had_attention_host.argtypes = [P, P, P, SP, BP, P, P, I, I, P, I, I, P, SZ, P]
         L.had_dense_reference_workspace_size.argtypes = [SP]
         L.had_dense_reference_workspace_size.restype = SZ
         L.had_dense_reference_mode.argtypes = [P, P, P, SP, BP, I, P, I, P, SZ, P]
@@ -80,7 +83,8 @@ def lib():
         L.had_topn_indices.argtypes = [P, P, SP, BP, P, P, I, P, P, SZ, P]
         L.had_attention_codes_u8.argtypes = [P, P, P, SP, BP, P, P, I, I, I, P, P, SZ, P]
         L.had_quantize_v.argtypes = [P, SP, P, P, P, SZ, P]
-        for f in ("had_binarize_pack", "had_binarize_pack_noalloc", "had_attention", "had_dense_reference_mode", "had_scores_int",
+        for f in ("had_binarize_pack", "had_binarize_pack_noalloc", "had_attention", "had_attention_host",
+                  "had_dense_reference_mode", "had_scores_int",
                   "had_topn_indices", "had_attention_codes_u8", "had_quantize_v", "had_get_device_status"):
             getattr(L, f).restype = I
         L.had_get_device_status.argtypes = []
@@ -217,6 +221,63 @@ def had_attention(Q, K, V, N=0, mode="float", seqlens=None, bias=None, alpha_q=N
     st = lib().had_attention(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shp), bs, aq, ak, int(N), m, _ptr(out),
                              _dtype_code(out), _ptr(ws), ws.numel(), _stream(stream))
     _raise(st, "had_attention")
+    return out
+
+
+def _check_host(*ts):
+    for t in ts:
+        if t is not None:
+            if t.device.type != "cpu":
+                raise ValueError("had_attention_host takes host (CPU) tensors")
+            if not t.is_contiguous():
+                raise ValueError("tensors must be contiguous")
+
+
+def _host_bias_struct(bias: RelPosBias | None):
+    if bias is None:
+        return None
+    if bias.table.dtype != torch.float32:
+        raise TypeError("bias table must be float32")
+    _check_host(bias.table)
+    return ctypes.byref(had_relpos_bias(bias.table.data_ptr(), bias.gh, bias.gw, bias.prefix))
+
+
+def had_attention_host_workspace_size(X, N=0, mode="float", seqlens=None, bias=None, chunk_b=0) -> int:
+    shp = make_shape(X, seqlens)
+    return int(lib().had_attention_host_workspace_size(ctypes.byref(shp), int(N), _MODES[mode],
+                                                       _host_bias_struct(bias), int(chunk_b)))
+
+
+def had_attention_host(Q, K, V, N=0, mode="float", seqlens=None, bias=None, alpha_q=None, alpha_k=None, out=None,
+                       out_dtype=None, chunk_b=0, workspace=None, stream=None, synchronize=True):
+    """had_attention on host tensors: the library copies chunks of the batch in,
+    computes them and copies O out, overlapping the three (from pinned memory).
+
+    Q, K, V, seqlens, the bias table and `out` are CPU tensors; `workspace` is a
+    device uint8 tensor (allocated on the current device if None).  With
+    synchronize=False the call returns once everything is enqueued on `stream`,
+    and `out` is valid after that stream has been synchronized.
+    """
+    _check_host(Q, K, V, seqlens, out)
+    B, H, n, d = Q.shape
+    shp = make_shape(Q, seqlens)
+    m = _MODES[mode]
+    if out is None:
+        out = torch.empty((B, H, n, d), dtype=out_dtype or V.dtype, pin_memory=Q.is_pinned())
+    bs = _host_bias_struct(bias)
+    need = lib().had_attention_host_workspace_size(ctypes.byref(shp), int(N), m, bs, int(chunk_b))
+    if need == 0:
+        _raise(HAD_ERR_INVALID, "had_attention_host_workspace_size")
+    if workspace is not None:
+        _check_dev(workspace)
+    ws = _workspace(need, torch.device("cuda", torch.cuda.current_device()), workspace)
+    aq_keep, aq = _alpha(alpha_q, H)
+    ak_keep, ak = _alpha(alpha_k, H)
+    st = lib().had_attention_host(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shp), bs, aq, ak, int(N), m, _ptr(out),
+                                  _dtype_code(out), int(chunk_b), _ptr(ws), ws.numel(), _stream(stream))
+    _raise(st, "had_attention_host")
+    if synchronize:
+        (stream or torch.cuda.current_stream()).synchronize()
     return out
 
 

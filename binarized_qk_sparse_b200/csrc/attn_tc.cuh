@@ -60,7 +60,7 @@ constexpr int kSplitMaxKeys = 256;  // top-N without a bias, ragged rows: two th
 constexpr int kKStages = 4;
 constexpr int kVStages = 2;
 constexpr int kLevels = 65;
-constexpr int kRadixBins = 128;
+constexpr int kRadixBins = 256;   // 16-bit counters, two per word (a row counts at most kMaxN keys)
 constexpr int kCandCap = 128;    // power of two (the collect slot wraps)
 constexpr int kSBufs = 3;
 constexpr uint32_t kColS = 0, kColO = 192, kTmemCols = 256;
@@ -85,6 +85,9 @@ struct TcArgs {
   CUtensorMap tm_vq;  // int8 V^T [BH*64][n_pad], box {64, 64}, 64B swizzle      (uint8 mode)
   CUtensorMap tm_vlo; // bf16 residual of fp32 V [BH*n][64], box {64, 64}         (fp32 V)
   const uint32_t* qbits;   // [BH][n][2]
+  const int8_t* kpm;       // [BH][n_pad][64] +-1 codes of K (the score MMA's B operand)
+  const void* v_raw;       // V as given, [BH][n][64] bf16 or fp32 (float mode)
+  int v_f32;               // 1 if v_raw is fp32
   const float* vscale;     // [BH][64]
   const float* table;      // [H][th][tw] or null
   int gh, gw, prefix, th, tw;
@@ -126,7 +129,8 @@ struct Smem {
                                     : (SEL == SEL_TOPN_INT) ? kLevels * kM * 4
                                     : kCandCap * kM * 4;
   static constexpr int kTotal = kHist + kHistBytes + 1024;       // + alignment slack
-  static_assert(kCandCap >= kRadixBins && kCandCap >= kLevels, "radix and level histograms fit the candidate area");
+  static_assert(kCandCap >= kRadixBins / 2 && kCandCap >= kLevels, "radix and level histograms fit the candidate area");
+  static_assert(kMaxN < 65536, "a 16-bit radix counter holds every key of a row");
   static_assert((kCandCap & (kCandCap - 1)) == 0, "candidate slots wrap with a mask");
 };
 
@@ -190,6 +194,12 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
   constexpr int kMmaWarp = kSoftWarps, kProdWarp = kSoftWarps + 1;
   constexpr int kChunks = 2 / kSplit;  // 32-key chunks of a tile per softmax thread
   constexpr bool HAS_BIAS = BIAS != BIAS_NONE;
+  // top-N with a bias, float A.V: the final radix bin's keys are recorded (key
+  // index) during the P.V pass and ranked, weighted and added to O afterwards,
+  // instead of in a collect pass of their own; indices in slots [0, 64), their
+  // logits in [64, 128) of the candidate area
+  constexpr bool kMerge = SEL == SEL_TOPN_FLOAT && MODE == MODE_F && EXPORT == EXP_NONE;
+  constexpr int kCap = kCandCap / 2;
   using SM = Smem<SEL, VF32, BIAS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -322,8 +332,14 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
   float F = -INFINITY, m = -INFINITY, scale = 1.0f, lsum = 0.0f;
   int rF = 0, cut = 0, tie_seen = 0, kept_seen = 0;
   uint32_t r_uhi = 0, r_span = 0;
+  // r_state: 0 threshold known, 1 radix pass next, 2 collect pass next, 3 the
+  // window's keys are recorded during the P.V pass (kMerge)
   int r_shift = 0, r_rank = 0, r_state = 0, r_cnt = 0;
   int r_above = 0;      // keys above the first radix window (counted in that pass)
+  // float window of the P.V pass: weight for l >= w_cut; keys in [w_lo, w_hi] are
+  // the ties at F (w_lo = w_hi = w_cut = F), or, with the collect folded into
+  // the P.V pass, the final radix bin (w_cut just above w_hi), ranked after it
+  float w_lo = INFINITY, w_hi = INFINITY, w_cut = INFINITY;
   bool r_first = false;  // the next radix pass is the first of this row
   // row base of the extended bias tables: rb(i) - koff(j) indexes the pair (i, j);
   // class-token rows and rows past the tensor use the class-row base
@@ -708,17 +724,19 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
               } else if (kHasRadix && pass == P_RADIX) {
                 // histogram of the keys inside the window [r_uhi - r_span, r_uhi] (order keys;
                 // keys past L are -inf, below every window), and the count above it
+                // (bin b: the low (b < 128) or high half of word b mod 128)
                 if (r_state == 1) {
                   const uint32_t ulo = r_uhi - r_span;
 #pragma unroll
                   for (int u = 0; u < 32; ++u) {
                     const uint32_t key = float_order_key(lg[u]);
-                    const uint32_t t = key - ulo;
+                    const uint32_t t = key - ulo, bin = (r_span - t) >> r_shift;
                     r_above += key > r_uhi ? 1 : 0;
-                    const uint32_t ad = hist_row + ((r_span - t) >> r_shift) * (uint32_t)(kM * 4);
+                    const uint32_t ad = hist_row + (bin & 127u) * (uint32_t)(kM * 4);
+                    const uint32_t inc = 1u + (bin >> 7) * 0xFFFFu;
                     asm volatile(
-                        "{\n\t.reg .pred p;\n\tsetp.le.u32 p, %1, %2;\n\t@p red.shared.add.u32 [%0], 1;\n\t}" ::"r"(ad),
-                        "r"(t), "r"(r_span)
+                        "{\n\t.reg .pred p;\n\tsetp.le.u32 p, %1, %2;\n\t@p red.shared.add.u32 [%0], %3;\n\t}" ::"r"(ad),
+                        "r"(t), "r"(r_span), "r"(inc)
                         : "memory");
                   }
                 }
@@ -740,21 +758,32 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
                   }
                 }
               } else if (SEL == SEL_TOPN_FLOAT && (pass == P_PV || pass == P_CODES)) {
-                // weights of the keys at or above F (keys past L are -inf, below it), then
-                // the ties at F past the row's remaining allowance rF dropped in key order
+                // weights of the keys at or above w_cut (keys past L are -inf, below it);
+                // the keys in [w_lo, w_hi] are the ties at F, of which those past the
+                // row's remaining allowance rF are dropped in key order, or (folded
+                // collect) the final radix bin, whose key indices are recorded
                 float e[32];
-                uint32_t eqm = 0u;
+                uint32_t inm = 0u;
 #pragma unroll
                 for (int u = 0; u < 32; ++u) {
                   const float x = fast_exp2(__fmaf_rn(lg[u], kLog2e, mo));
-                  e[u] = lg[u] >= F ? x : 0.0f;
-                  eqm |= (lg[u] == F ? 1u : 0u) << u;
+                  e[u] = lg[u] >= w_cut ? x : 0.0f;
+                  inm |= (lg[u] >= w_lo && lg[u] <= w_hi ? 1u : 0u) << u;
                 }
-                const uint32_t dropm = eqm & ~tie_keep(eqm, cut, rF, tie_seen);
-                tie_seen += __popc(eqm);
-                if (dropm) {
+                if (kMerge && r_state == 3) {
+                  while (inm) {
+                    const int u = __ffs(inm) - 1;
+                    inm &= inm - 1u;
+                    hist[(r_cnt & (kCap - 1)) * kM + srow] = (uint32_t)(jb + u);
+                    ++r_cnt;
+                  }
+                } else {
+                  const uint32_t dropm = inm & ~tie_keep(inm, cut, rF, tie_seen);
+                  tie_seen += __popc(inm);
+                  if (dropm) {
 #pragma unroll
-                  for (int u = 0; u < 32; ++u) e[u] = ((dropm >> u) & 1u) ? 0.0f : e[u];
+                    for (int u = 0; u < 32; ++u) e[u] = ((dropm >> u) & 1u) ? 0.0f : e[u];
+                  }
                 }
                 emit(e, ch);
               } else {
@@ -953,29 +982,38 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
         r_first = false;
         int cum = 0, bsel = kRadixBins - 1, kbin = 0;
         for (int bb = 0; bb < kRadixBins; ++bb) {
-          const int k = (int)hist[bb * kM + srow];
+          const int k = (int)((hist[(bb & 127) * kM + srow] >> ((bb >> 7) * 16)) & 0xFFFFu);
           if (cum + k >= r_rank) { bsel = bb; kbin = k; break; }
           cum += k;
         }
         const int rank = r_rank - cum;
         const uint32_t uhi = r_uhi - ((uint32_t)bsel << r_shift);
         if (r_shift == 0) {
-          const uint32_t bits = (uhi & 0x80000000u) ? (uhi & 0x7FFFFFFFu) : ~uhi;
-          F = __uint_as_float(bits);
+          F = order_key_float(uhi);
           rF = rank;
           cut = rank < kbin ? 1 : 0;
           r_state = 0;
+          w_lo = w_hi = w_cut = F;
         } else {
           // the chosen bin becomes the window: collected if small, else binned again
           const uint32_t span_left = r_span - ((uint32_t)bsel << r_shift);
           r_uhi = uhi;
           r_span = min(((uint32_t)1 << r_shift) - 1u, span_left);
           r_rank = rank;
-          if (kbin <= kCandCap) {
+          r_cnt = 0;
+          if (kMerge && kbin <= kCap) {
+            r_state = 3;
+            // no logit has the order key of -0 (keys are taken of l + 0): keep the
+            // window's ends off it so that their float values compare as the keys do
+            if (r_uhi == 0x7FFFFFFFu) { r_uhi -= 1u; r_span -= 1u; }
+            if (r_uhi - r_span == 0x7FFFFFFFu) r_span -= 1u;
+            w_hi = order_key_float(r_uhi);
+            w_lo = order_key_float(r_uhi - r_span);
+            w_cut = order_key_float(r_uhi + 1u);  // the next float above w_hi
+          } else if (kbin <= kCandCap) {
             r_state = 2;
-            r_cnt = 0;
           } else {
-            r_shift = r_shift > 7 ? r_shift - 7 : 0;
+            r_shift = r_shift > 8 ? r_shift - 8 : 0;
           }
         }
       } else if (pass == P_COLLECT && r_state == 2) {
@@ -1001,11 +1039,11 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
             break;
           }
         }
-        const uint32_t bits = (uF & 0x80000000u) ? (uF & 0x7FFFFFFFu) : ~uF;
-        F = __uint_as_float(bits);
+        F = order_key_float(uF);
         rF = r_rank - gt;
         cut = rF < eq ? 1 : 0;
         r_state = 0;
+        w_lo = w_hi = w_cut = F;
       } else if (pass == P_KEPT_NORM) {
         scale = 255.0f / lsum;
       } else if (pass == P_NORM) {
@@ -1042,13 +1080,13 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
     else if (pass == P_IDX || pass == P_CODES || pass == P_PV) next = P_DONE;
     else if (pass == P_NORM) next = (EXPORT == EXP_CODES) ? P_CODES : P_PV;
     else if (any_refine) next = P_RADIX;
-    else if (any_collect) next = P_COLLECT;
+    else if (any_collect) next = kMerge ? P_PV : P_COLLECT;
     else if (EXPORT == EXP_IDX) next = P_IDX;
     else if ((EXPORT == EXP_CODES || MODE == MODE_Q) && SEL == SEL_TOPN_FLOAT && pass != P_KEPT_NORM) next = P_KEPT_NORM;
     else if (EXPORT == EXP_CODES) next = P_CODES;
     else next = P_PV;
     if (next == P_RADIX && tid < kM) {
-      for (int bb = 0; bb < kRadixBins; ++bb) hist[bb * kM + srow] = 0u;
+      for (int bb = 0; bb < kRadixBins / 2; ++bb) hist[bb * kM + srow] = 0u;
       r_above = 0;
     }
     if (next == P_KEPT_NORM && tid < kM) lsum = 0.0f;
@@ -1084,9 +1122,103 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
 #pragma unroll
           for (int k = 0; k < kOc; ++k) out[k] = (float)(int)o[k] * dq[c0 + k];
         } else {
+#pragma unroll
+          for (int k = 0; k < kOc; ++k) out[k] = __uint_as_float(o[k]);
+          if (kMerge && r_state == 3) {
+            // the final radix bin of this row: logits of its recorded keys from the same
+            // integer score (+-1 codes, exact) and bias entry as in the tiles, the
+            // r_rank-th largest as threshold with its ties kept in key order, and the
+            // kept keys' weights and V rows added to the normalizer and to O
+            const int nc = min(r_cnt, kCap);
+            if (r_cnt > kCap) raise_status(a.status, kDevErrCapacity);
+            uint4 qv[4];
+#pragma unroll
+            for (int cch = 0; cch < 4; ++cch)
+              qv[cch] = *reinterpret_cast<const uint4*>(sQ + srow * kD + ((cch ^ ((srow >> 1) & 3)) * 16));
+            const int8_t* kb = a.kpm + (size_t)bh * a.n_pad * kD;
+            for (int x = 0; x < nc; ++x) {
+              const int j = (int)hist[x * kM + srow];
+              const uint4* kr = reinterpret_cast<const uint4*>(kb + (size_t)j * kD);
+              int sc = 0;
+#pragma unroll
+              for (int cch = 0; cch < 4; ++cch) {
+                const uint4 kv = __ldg(kr + cch);
+                sc = __dp4a((int)qv[cch].x, (int)kv.x, sc);
+                sc = __dp4a((int)qv[cch].y, (int)kv.y, sc);
+                sc = __dp4a((int)qv[cch].z, (int)kv.z, sc);
+                sc = __dp4a((int)qv[cch].w, (int)kv.w, sc);
+              }
+              float l;
+              if (HAS_BIAS) {
+                int off;  // entry (i, j) of the extended table sits at rb - off
+                if (j < a.prefix) {
+                  off = a.k_class;
+                } else {
+                  const int t = j - a.prefix, y = t / a.gw;
+                  off = y * a.ext_S + (t - y * a.gw);
+                }
+                l = __fmaf_rn((float)sc, c, __ldg(tab + rb - off));
+              } else {
+                l = (float)sc * c;
+              }
+              hist[(kCap + x) * kM + srow] = __float_as_uint(l);
+            }
+            const float* lc = reinterpret_cast<const float*>(hist) + kCap * kM + srow;  // logit x at lc[x * kM]
+            float vF = INFINITY;
+            int gt = 0;
+            for (int x = 0; x < nc; ++x) {
+              const float vx = lc[x * kM];
+              int g = 0, e = 0;
+              for (int y = 0; y < nc; ++y) {
+                const float vy = lc[y * kM];
+                g += vy > vx ? 1 : 0;
+                e += vy == vx ? 1 : 0;
+              }
+              if (g < r_rank && r_rank <= g + e) {
+                vF = vx;
+                gt = g;
+                break;
+              }
+            }
+            int allow = r_rank - gt;  // keys at the threshold still kept, in key order
+            const float mo_e = -m * kLog2e;
+            for (int x = 0; x < nc; ++x) {
+              const float v = lc[x * kM];
+              const bool at = v == vF;
+              if (!(v > vF || (at && allow > 0))) continue;
+              allow -= at ? 1 : 0;
+              const int j = (int)hist[x * kM + srow];
+              const float p = fast_exp2(__fmaf_rn(v, kLog2e, mo_e));
+              lsum += p;
+              const size_t vrow = (size_t)bh * a.n + j;
+              if (a.v_f32) {
+                const float4* vr = reinterpret_cast<const float4*>(a.v_raw) + vrow * (kD / 4);
+#pragma unroll
+                for (int q = 0; q < kD / 4; ++q) {
+                  const float4 f = __ldg(vr + q);
+                  out[4 * q] = __fmaf_rn(p, f.x, out[4 * q]);
+                  out[4 * q + 1] = __fmaf_rn(p, f.y, out[4 * q + 1]);
+                  out[4 * q + 2] = __fmaf_rn(p, f.z, out[4 * q + 2]);
+                  out[4 * q + 3] = __fmaf_rn(p, f.w, out[4 * q + 3]);
+                }
+              } else {
+                const uint4* vr = reinterpret_cast<const uint4*>(a.v_raw) + vrow * (kD / 8);
+#pragma unroll
+                for (int q = 0; q < kD / 8; ++q) {
+                  const uint4 u4 = __ldg(vr + q);
+                  const uint32_t wv[4] = {u4.x, u4.y, u4.z, u4.w};
+#pragma unroll
+                  for (int t = 0; t < 4; ++t) {
+                    out[8 * q + 2 * t] = __fmaf_rn(p, __uint_as_float(wv[t] << 16), out[8 * q + 2 * t]);
+                    out[8 * q + 2 * t + 1] = __fmaf_rn(p, __uint_as_float(wv[t] & 0xFFFF0000u), out[8 * q + 2 * t + 1]);
+                  }
+                }
+              }
+            }
+          }
           const float inv = sum_in_pv ? 1.0f / lsum : scale;
 #pragma unroll
-          for (int k = 0; k < kOc; ++k) out[k] = __uint_as_float(o[k]) * inv;
+          for (int k = 0; k < kOc; ++k) out[k] *= inv;
         }
         const size_t ob = ((size_t)bh * a.n + row) * kD + c0;
         if (a.o_bf16) {

@@ -125,5 +125,9 @@ __device__ __forceinline__ uint32_t float_order_key(float x) {
   uint32_t u = __float_as_uint(x + 0.0f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+// The float whose order key is k (the inverse of float_order_key on its range).
+__device__ __forceinline__ float order_key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
 
 }  // namespace had

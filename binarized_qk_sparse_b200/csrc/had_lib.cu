@@ -11,6 +11,7 @@
 //              V scale -> int8 V^T (uint8 mode)
 //   k_bias_tables (with a bias): per-head bias range and exp(b - b_max) table
 //   k_attn   : scores, logits, top-N select, softmax, A.V, output
+#include <algorithm>
 #include <climits>
 #include <cmath>
 #include <cstdio>
@@ -439,6 +440,9 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
     }
   }
   a.qbits = reinterpret_cast<uint32_t*>(ws + w.qbits);
+  a.kpm = reinterpret_cast<const int8_t*>(ws + w.kpm);
+  a.v_raw = V;
+  a.v_f32 = (s->in_dtype == HAD_F32) ? 1 : 0;
   a.vscale = quant ? reinterpret_cast<float*>(ws + w.vscale) : nullptr;
   a.table = has_bias ? bias->table : nullptr;
   if (has_bias) {
@@ -503,6 +507,172 @@ had_status run_attention(const void* Q, const void* K, const void* V, const had_
                            workspace, st, status);
 }
 
+// ---------------------------------------------------------------------------- host buffers in and out
+
+// Staging of had_attention_host in its device workspace: the seqlens and bias
+// table copies, then `slots` chunk slots (Q, K, V, O and the kernels'
+// workspace of one chunk of `cb` sequences) that consecutive chunks cycle through.
+struct HostPlan {
+  int cb = 0, chunks = 0, slots = 0;
+  size_t in_b = 0, o_b = 0;                   // bytes of one sequence of Q (= K = V), of O as fp32
+  size_t seq = 0, tab = 0, tab_bytes = 0, slot0 = 0, slot_bytes = 0, total = 0;
+  size_t q = 0, k = 0, v = 0, o = 0, ws = 0;  // offsets inside a slot
+  size_t ws_bytes = 0;
+};
+
+constexpr int kHostSlots = 3;
+constexpr size_t kHostChunkBytes = size_t(8) << 20;  // input bytes per chunk when the caller passes chunk_b = 0
+
+had_status host_plan(const had_shape* s, had_mode mode, const had_relpos_bias* bias, int chunk_b, HostPlan* p) {
+  if (!s) return HAD_ERR_INVALID;
+  had_shape s0 = *s;
+  s0.seqlens = nullptr;  // a host array here: checked by value in had_attention_host
+  had_status r = check_shape(&s0);
+  if (r != HAD_OK) return r;
+  if ((r = check_bias(&s0, bias)) != HAD_OK) return r;
+  if (chunk_b < 0) return HAD_ERR_INVALID;
+  const bool has_bias = bias && bias->table;
+  const size_t esz = s->in_dtype == HAD_BF16 ? 2 : 4;
+  p->in_b = (size_t)s->H * s->n * kD * esz;
+  p->o_b = (size_t)s->H * s->n * kD * 4;
+  size_t cb = chunk_b > 0 ? (size_t)chunk_b : std::max<size_t>(1, kHostChunkBytes / (3 * p->in_b));
+  p->cb = (int)std::min<size_t>(cb, (size_t)s->B);
+  p->chunks = (s->B + p->cb - 1) / p->cb;
+  p->slots = std::min(kHostSlots, p->chunks);
+  had_shape sc = s0;
+  sc.B = p->cb;
+  p->ws_bytes = ws_layout(&sc, mode == HAD_MODE_U8I8, has_bias ? bias : nullptr).total;
+  size_t off = 0;
+  p->seq = off;
+  off += align_up((size_t)s->B * sizeof(int32_t));
+  p->tab = off;
+  p->tab_bytes = has_bias ? (size_t)s->H * (2 * bias->gh - 1) * (2 * bias->gw - 1) * sizeof(float) : 0;
+  off += align_up(p->tab_bytes);
+  p->slot0 = off;
+  size_t so = 0;
+  p->q = so; so += align_up(p->cb * p->in_b);
+  p->k = so; so += align_up(p->cb * p->in_b);
+  p->v = so; so += align_up(p->cb * p->in_b);
+  p->o = so; so += align_up(p->cb * p->o_b);
+  p->ws = so; so += align_up(p->ws_bytes);
+  p->slot_bytes = so;
+  p->total = off + (size_t)p->slots * so;
+  return HAD_OK;
+}
+
+// The side streams and events of one had_attention_host call.  Whatever has
+// been enqueued when it goes out of scope (also after an error), the caller's
+// stream is made to wait for it; the streams and events are then released
+// (CUDA defers that until their pending work is done).
+struct HostStreams {
+  cudaStream_t main = nullptr, in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, join_in = nullptr, join_out = nullptr;
+  cudaEvent_t in_done[kHostSlots] = {}, comp_done[kHostSlots] = {}, out_done[kHostSlots] = {};
+  ~HostStreams() {
+    if (in && join_in && cudaEventRecord(join_in, in) == cudaSuccess) cudaStreamWaitEvent(main, join_in, 0);
+    if (out && join_out && cudaEventRecord(join_out, out) == cudaSuccess) cudaStreamWaitEvent(main, join_out, 0);
+    for (cudaEvent_t e : {start, join_in, join_out})
+      if (e) cudaEventDestroy(e);
+    for (int i = 0; i < kHostSlots; ++i)
+      for (cudaEvent_t e : {in_done[i], comp_done[i], out_done[i]})
+        if (e) cudaEventDestroy(e);
+    if (in) cudaStreamDestroy(in);
+    if (out) cudaStreamDestroy(out);
+  }
+};
+
+// Chunk k: its Q, K, V are copied in on `in` (once the slot's previous chunk has
+// been computed), computed on the caller's stream (once its inputs are in and the
+// slot's previous O has been copied out), and its O copied out on `out`.  Copy
+// in, compute and copy out of consecutive chunks overlap.
+had_status host_attention(const void* Q, const void* K, const void* V, const had_shape* s,
+                          const had_relpos_bias* bias, const float* alpha_q, const float* alpha_k, int N,
+                          had_mode mode, void* O, had_dtype o_dtype, int chunk_b, void* workspace, size_t ws_bytes,
+                          cudaStream_t st) {
+  HostPlan p;
+  had_status r = host_plan(s, mode, bias, chunk_b, &p);
+  if (r != HAD_OK) return r;
+  if (!Q || !K || !V || !O || (o_dtype != HAD_F32 && o_dtype != HAD_BF16)) return HAD_ERR_INVALID;
+  if (N < 0 || (mode != HAD_MODE_FLOAT && mode != HAD_MODE_U8I8)) return HAD_ERR_INVALID;
+  if (!workspace || ws_bytes < p.total || !aligned16(workspace)) return HAD_ERR_INVALID;
+  for (int h = 0; alpha_q && h < s->H; ++h)
+    if (!(alpha_q[h] > 0.0f) || !std::isfinite(alpha_q[h])) return HAD_ERR_INVALID;
+  for (int h = 0; alpha_k && h < s->H; ++h)
+    if (!(alpha_k[h] > 0.0f) || !std::isfinite(alpha_k[h])) return HAD_ERR_INVALID;
+  for (int b = 0; s->seqlens && b < s->B; ++b)
+    if (s->seqlens[b] < 1 || s->seqlens[b] > s->n) return HAD_ERR_INVALID;
+  const bool has_bias = bias && bias->table;
+  char* ws = static_cast<char*>(workspace);
+  const size_t o_b = (size_t)s->H * s->n * kD * (o_dtype == HAD_BF16 ? 2 : 4);
+  auto cu = [](cudaError_t e, const char* what) { return e == cudaSuccess ? HAD_OK : cuda_fail(e, what); };
+
+  HostStreams hs;
+  hs.main = st;
+  if ((r = cu(cudaStreamCreateWithFlags(&hs.in, cudaStreamNonBlocking), "cudaStreamCreateWithFlags")) != HAD_OK ||
+      (r = cu(cudaStreamCreateWithFlags(&hs.out, cudaStreamNonBlocking), "cudaStreamCreateWithFlags")) != HAD_OK)
+    return r;
+  for (cudaEvent_t* e : {&hs.start, &hs.join_in, &hs.join_out})
+    if ((r = cu(cudaEventCreateWithFlags(e, cudaEventDisableTiming), "cudaEventCreateWithFlags")) != HAD_OK) return r;
+  for (int i = 0; i < p.slots; ++i)
+    for (cudaEvent_t* e : {&hs.in_done[i], &hs.comp_done[i], &hs.out_done[i]})
+      if ((r = cu(cudaEventCreateWithFlags(e, cudaEventDisableTiming), "cudaEventCreateWithFlags")) != HAD_OK)
+        return r;
+  // the side streams start behind the work already on the caller's stream
+  if ((r = cu(cudaEventRecord(hs.start, st), "cudaEventRecord")) != HAD_OK ||
+      (r = cu(cudaStreamWaitEvent(hs.in, hs.start, 0), "cudaStreamWaitEvent")) != HAD_OK ||
+      (r = cu(cudaStreamWaitEvent(hs.out, hs.start, 0), "cudaStreamWaitEvent")) != HAD_OK)
+    return r;
+  const int32_t* dseq = nullptr;
+  if (s->seqlens) {
+    int32_t* d = reinterpret_cast<int32_t*>(ws + p.seq);
+    if ((r = cu(cudaMemcpyAsync(d, s->seqlens, (size_t)s->B * sizeof(int32_t), cudaMemcpyHostToDevice, hs.in),
+                "cudaMemcpyAsync(seqlens)")) != HAD_OK)
+      return r;
+    dseq = d;
+  }
+  had_relpos_bias bdev{};
+  if (has_bias) {
+    float* d = reinterpret_cast<float*>(ws + p.tab);
+    if ((r = cu(cudaMemcpyAsync(d, bias->table, p.tab_bytes, cudaMemcpyHostToDevice, hs.in),
+                "cudaMemcpyAsync(bias table)")) != HAD_OK)
+      return r;
+    bdev = *bias;
+    bdev.table = d;
+  }
+  const char* hq = static_cast<const char*>(Q);
+  const char* hk = static_cast<const char*>(K);
+  const char* hv = static_cast<const char*>(V);
+  char* ho = static_cast<char*>(O);
+  for (int k = 0; k < p.chunks; ++k) {
+    const int b0 = k * p.cb, nb = std::min(p.cb, s->B - b0), sl = k % p.slots;
+    char* slot = ws + p.slot0 + (size_t)sl * p.slot_bytes;
+    const size_t in_bytes = (size_t)nb * p.in_b, in_off = (size_t)b0 * p.in_b;
+    if (k >= p.slots && (r = cu(cudaStreamWaitEvent(hs.in, hs.comp_done[sl], 0), "cudaStreamWaitEvent")) != HAD_OK)
+      return r;
+    if ((r = cu(cudaMemcpyAsync(slot + p.q, hq + in_off, in_bytes, cudaMemcpyHostToDevice, hs.in), "cudaMemcpyAsync(Q)")) != HAD_OK ||
+        (r = cu(cudaMemcpyAsync(slot + p.k, hk + in_off, in_bytes, cudaMemcpyHostToDevice, hs.in), "cudaMemcpyAsync(K)")) != HAD_OK ||
+        (r = cu(cudaMemcpyAsync(slot + p.v, hv + in_off, in_bytes, cudaMemcpyHostToDevice, hs.in), "cudaMemcpyAsync(V)")) != HAD_OK ||
+        (r = cu(cudaEventRecord(hs.in_done[sl], hs.in), "cudaEventRecord")) != HAD_OK ||
+        (r = cu(cudaStreamWaitEvent(st, hs.in_done[sl], 0), "cudaStreamWaitEvent")) != HAD_OK)
+      return r;
+    if (k >= p.slots && (r = cu(cudaStreamWaitEvent(st, hs.out_done[sl], 0), "cudaStreamWaitEvent")) != HAD_OK)
+      return r;
+    had_shape cs = *s;
+    cs.B = nb;
+    cs.seqlens = dseq ? dseq + b0 : nullptr;
+    r = run_attention<EXP_NONE>(slot + p.q, slot + p.k, slot + p.v, &cs, has_bias ? &bdev : nullptr, alpha_q, alpha_k,
+                                N, mode, slot + p.o, o_dtype, nullptr, nullptr, 0, 0, slot + p.ws, p.ws_bytes, st);
+    if (r != HAD_OK) return r;
+    if ((r = cu(cudaEventRecord(hs.comp_done[sl], st), "cudaEventRecord")) != HAD_OK ||
+        (r = cu(cudaStreamWaitEvent(hs.out, hs.comp_done[sl], 0), "cudaStreamWaitEvent")) != HAD_OK ||
+        (r = cu(cudaMemcpyAsync(ho + (size_t)b0 * o_b, slot + p.o, (size_t)nb * o_b, cudaMemcpyDeviceToHost, hs.out),
+                "cudaMemcpyAsync(O)")) != HAD_OK ||
+        (r = cu(cudaEventRecord(hs.out_done[sl], hs.out), "cudaEventRecord")) != HAD_OK)
+      return r;
+  }
+  return HAD_OK;
+}
+
 }  // namespace
 }  // namespace had
 
@@ -545,6 +715,21 @@ had_status had_attention(const void* Q, const void* K, const void* V, const had_
                          had_mode mode, void* O, had_dtype o_dtype, void* workspace, size_t ws_bytes, void* stream) {
   return run_attention<EXP_NONE>(Q, K, V, s, bias, alpha_q, alpha_k, N, mode, O, o_dtype, nullptr, nullptr, 0, 0,
                                  workspace, ws_bytes, stream);
+}
+
+size_t had_attention_host_workspace_size(const had_shape* s, int N, had_mode mode, const had_relpos_bias* bias,
+                                         int chunk_b) {
+  (void)N;
+  HostPlan p;
+  return host_plan(s, mode, bias, chunk_b, &p) == HAD_OK ? p.total : 0;
+}
+
+had_status had_attention_host(const void* Q, const void* K, const void* V, const had_shape* s,
+                              const had_relpos_bias* bias, const float* alpha_q, const float* alpha_k, int N,
+                              had_mode mode, void* O, had_dtype o_dtype, int chunk_b, void* workspace,
+                              size_t ws_bytes, void* stream) {
+  return host_attention(Q, K, V, s, bias, alpha_q, alpha_k, N, mode, O, o_dtype, chunk_b, workspace, ws_bytes,
+                        static_cast<cudaStream_t>(stream));
 }
 
 had_status had_attention_prepare(const void* Q, const void* K, const void* V, const had_shape* s,

@@ -21,7 +21,8 @@
  *
  * Conventions for every entry point:
  *   - Tensor pointers are DEVICE pointers owned by the caller (for example
- *     torch tensors' data_ptr()).  Q, K, V, O are contiguous [B][H][n][d].
+ *     torch tensors' data_ptr()), except in had_attention_host, which takes
+ *     host arrays.  Q, K, V, O are contiguous [B][H][n][d].
  *     Device pointers must be 16-byte aligned.
  *   - The library never allocates, frees or synchronizes in these calls: work
  *     is enqueued on `stream` (a cudaStream_t; NULL = the legacy default
@@ -130,6 +131,33 @@ had_status had_attention_prepare(const void* Q, const void* K, const void* V, co
 had_status had_attention_prepared(const void* V, const had_shape* s, const had_relpos_bias* bias,
                                   const float* alpha_q, const float* alpha_k, int N, had_mode mode, void* O,
                                   had_dtype o_dtype, void* workspace, size_t ws_bytes, void* stream);
+
+/* ---- host arrays in, host array out --------------------------------------
+ * had_attention_host: had_attention on HOST memory, with the copies inside the
+ * call.  Q, K, V: HOST [B][H][n][d] in s->in_dtype; O: HOST [B][H][n][d] in
+ * o_dtype; s->seqlens: HOST int32 [B] (each in [1, n], checked on the host) or
+ * NULL; bias->table: HOST fp32 [H][2gh-1][2gw-1] or bias NULL; alpha_q,
+ * alpha_k as in had_attention.  The batch is cut into chunks of chunk_b
+ * sequences (0: the library picks about 8 MiB of inputs per chunk).  Chunk k's
+ * Q, K, V are copied in on one side stream while chunk k-1 is computed on
+ * `stream` and chunk k-2's O is copied out on another.  The chunks cycle
+ * through three device slots in `workspace`, which needs at least
+ * had_attention_host_workspace_size(s, N, mode, bias, chunk_b) bytes.  Every
+ * (b, h) is computed by the same kernels as in had_attention, so O is
+ * bit-identical to it for any chunk_b.
+ * Copies overlap one another and the kernels only from page-locked host memory
+ * (cudaHostAlloc / cudaHostRegister); pageable memory works, serialized.  The
+ * call enqueues all of it behind the work already on `stream` and returns: O
+ * is complete once `stream` has reached that point.  The host arrays must stay
+ * valid and unchanged until then.  Each call creates two streams and some
+ * events and releases them (CUDA frees them once their work is done);
+ * it allocates no memory. */
+size_t had_attention_host_workspace_size(const had_shape* s, int N, had_mode mode, const had_relpos_bias* bias,
+                                         int chunk_b);
+had_status had_attention_host(const void* Q, const void* K, const void* V, const had_shape* s,
+                              const had_relpos_bias* bias, const float* alpha_q, const float* alpha_k, int N,
+                              had_mode mode, void* O, had_dtype o_dtype, int chunk_b, void* workspace,
+                              size_t ws_bytes, void* stream);
 
 /* ---- in-library dense comparison mode ------------------------------------
  * Standard attention on the unbinarized inputs: l = (q . k)/sqrt(d) + b_ij with

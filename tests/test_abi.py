@@ -105,3 +105,52 @@ def test_status_strings(L):
     for st in range(6):
         assert L.had_status_string(st).startswith(b"HAD_")
     assert L.had_version() >= 100
+
+
+def test_host_entry_point_validates_on_the_host(L):
+    # every case fails before a stream or event is created or a byte is copied
+    import binarized_qk_sparse_b200 as m
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    ws = P(0x20000)
+    big = 1 << 34
+
+    def host(shape, q=fake, o=fake, N=0, mode=0, odt=1, chunk=0, ws_bytes=big, wsp=ws, alpha=None):
+        return L.had_attention_host(q, fake, fake, ctypes.byref(shape), None, alpha, None, N, mode, o, odt, chunk,
+                                    wsp, ws_bytes, None)
+
+    shp = _shape(m, B=4, n=64)
+    assert host(_shape(m, d=32)) == m.HAD_ERR_UNSUPPORTED
+    assert host(shp, q=P(0)) == m.HAD_ERR_INVALID
+    assert host(shp, o=P(0)) == m.HAD_ERR_INVALID
+    assert host(shp, odt=9) == m.HAD_ERR_INVALID
+    assert host(shp, N=-2) == m.HAD_ERR_INVALID
+    assert host(shp, mode=3) == m.HAD_ERR_INVALID
+    assert host(shp, chunk=-1) == m.HAD_ERR_INVALID
+    assert host(shp, ws_bytes=1024) == m.HAD_ERR_INVALID
+    assert host(shp, wsp=P(0x20008)) == m.HAD_ERR_INVALID
+    neg = (ctypes.c_float * 1)(-1.0)
+    assert host(shp, alpha=ctypes.cast(neg, P)) == m.HAD_ERR_INVALID
+    # seqlens is a host array here, checked by value
+    for bad in ([64, 0, 5, 5], [64, 65, 5, 5], [-1, 1, 1, 1]):
+        lens = (ctypes.c_int32 * 4)(*bad)
+        s2 = _shape(m, B=4, n=64, seqlens=ctypes.addressof(lens))
+        assert host(s2) == m.HAD_ERR_INVALID
+    bad_bias = m.had_relpos_bias(0x30000, 7, 7, 1)
+    assert L.had_attention_host(fake, fake, fake, ctypes.byref(shp), ctypes.byref(bad_bias), None, None, 0, 0, fake,
+                                1, 0, ws, big, None) == m.HAD_ERR_INVALID
+
+
+def test_host_workspace_grows_with_the_chunk(L):
+    import binarized_qk_sparse_b200 as m
+    shp = _shape(m, B=8, H=3, n=197)
+    bias = m.had_relpos_bias(0x30000, 14, 14, 1)
+    sizes = [L.had_attention_host_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(bias), c) for c in (1, 2, 8)]
+    assert 0 < sizes[0] < sizes[1] < sizes[2]
+    # a chunk larger than the batch is the whole batch; 0 lets the library choose
+    assert L.had_attention_host_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(bias), 100) == sizes[2]
+    assert L.had_attention_host_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(bias), 0) > 0
+    assert L.had_attention_host_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(bias), -1) == 0
+    # three slots of one chunk each hold Q, K, V and O at least
+    one = 3 * 197 * 64 * 2 + 197 * 64 * 4
+    assert sizes[0] >= 3 * one

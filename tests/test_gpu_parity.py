@@ -378,6 +378,63 @@ def test_alpha_and_bias_ties(oracle_mod):
         assert np.max(np.abs(O - ref.O)) <= _tol(w)
 
 
+@pytest.mark.parametrize("mode", ["float", "u8i8"])
+def test_bias_ties_at_the_threshold_fp32(oracle_mod, mode):
+    # A bias table of five values on a 14x14 grid with four class tokens (n = 200,
+    # four 64-key tiles) makes many exact logit ties; the values of N put the
+    # threshold in different tiles, and the radix search ends either on one
+    # logit value or on a bin of keys ranked after the weight pass.  fp32 inputs
+    # make one wrongly kept key visible against the 1e-3 bar (uint8 mode: plus
+    # one code LSB).  Index sets are compared exactly.
+    m = 1 if mode == "u8i8" else 0
+    w = _small(79, B=2, H=2, n=200, dtype="f32")
+    rng = np.random.default_rng(9)
+    table = (rng.integers(-2, 3, size=(2, 27, 27)) * 0.25).astype(np.float32)
+    w.bias = workloads.Bias(table, 14, 14, 4)
+    Q, K, V, seq, bias = _dev_inputs(w)
+    b = oracle_mod.RelPosBias(table, 14, 14, 4)
+    bar = _tol(w) + (float(np.max(np.abs(w.V))) / 255.0 if m else 0.0)
+    for N in (20, 70, 131, 180):
+        for sl in (None, np.array([200, 161], np.int32)):
+            seqt = None if sl is None else torch.from_numpy(sl).cuda()
+            ref = oracle_mod.attention(w.Q, w.K, w.V, N=N, mode=m, seqlens=sl, bias=b, want_idx=True)
+            O = had.had_attention(Q, K, V, N=N, mode=mode, seqlens=seqt, bias=bias).float().cpu().numpy()
+            assert np.max(np.abs(O - ref.O)) <= bar, (N, sl, np.max(np.abs(O - ref.O)))
+            idx = had.had_topn_indices(Q, K, N, seqt, bias).cpu().numpy().reshape(-1, N)
+            np.testing.assert_array_equal(idx, ref.idx)
+
+
+@pytest.mark.parametrize("pinned", [True, False])
+def test_host_entry_point_matches_the_device_call(oracle_mod, pinned):
+    # had_attention_host cuts the batch into chunks that run the same kernels as
+    # had_attention: O is bit-identical for every chunk size, pinned or not
+    w = _workload("deit")
+    B = 6
+    sub = workloads.Workload(w.name + "_b6", B, w.H, w.n, w.d, w.dtype, w.Q[:B], w.K[:B], w.V[:B],
+                             np.array([197, 150, 65, 1, 197, 100], np.int32), w.bias, w.passes, w.seed, w.recipe)
+    Q, K, V, seq, bias = _dev_inputs(sub)
+
+    def host(t):
+        t = t.cpu()
+        return t.pin_memory() if pinned else t
+
+    hQ, hK, hV = host(Q), host(K), host(V)
+    hseq = sub_seq = torch.from_numpy(sub.seqlens)
+    hbias = had.RelPosBias(host(bias.table), bias.gh, bias.gw, bias.prefix)
+    for N, mode in ((0, "u8i8"), (0, "float"), (30, "float"), (30, "u8i8")):
+        ref = had.had_attention(Q, K, V, N=N, mode=mode, seqlens=seq, bias=bias).cpu()
+        for chunk in (0, 1, 4, 6):
+            got = had.had_attention_host(hQ, hK, hV, N=N, mode=mode, seqlens=hseq, bias=hbias, chunk_b=chunk)
+            assert got.device.type == "cpu"
+            assert torch.equal(got, ref), (N, mode, chunk)
+    # and against the oracle once, on fp32 output
+    got = had.had_attention_host(hQ, hK, hV, N=30, mode="float", seqlens=sub_seq, bias=hbias, chunk_b=4,
+                                 out_dtype=torch.float32).numpy()
+    rows = _sample_rows(sub, 24, 5)
+    ref = _oracle_full(oracle_mod, sub, 30, 0, rows=rows).O
+    assert np.max(np.abs(got.reshape(-1, 64)[rows] - ref)) <= _tol(sub)
+
+
 def test_bad_seqlens_raise_device_status():
     w = _small(32, B=2, H=1, n=64)
     Q, K, V, _, _ = _dev_inputs(w)
