@@ -39,6 +39,7 @@ UNIT = "queries/s"
 # (workload name, N, mode) per bench workload id
 WORKLOADS = {
     "deit": ("deit", 0, "u8i8"),
+    "deit_dense_bias": ("deit_dense_bias", 0, "u8i8"),
     "tiny": ("tiny", 15, "float"),
     "bert": ("bert", 30, "float"),
     "t5_128": ("t5_128", 15, "float"),
@@ -63,12 +64,16 @@ def _peaks():
 HEAD_STAGE_BYTES = 128 * 1024  # heads up to this size are prepared by one kernel from shared memory
 
 
-def launches_per_step(n: int, elem: int, mode: str, has_bias: bool) -> int:
+def launches_per_step(n: int, elem: int, mode: str, has_bias: bool, dense_bias: bool = False) -> int:
     """Kernels one prepare + attend step launches: the sign/pack stage (one
-    kernel for short heads, which also builds the bias tables; statistics +
-    pack + bias tables otherwise), the hi/lo split of an fp32 V (float mode),
-    and the fused attention."""
-    k = 1 if n * 64 * elem <= HEAD_STAGE_BYTES else 2 + (1 if has_bias else 0)
+    kernel for short heads, which also builds relative-position bias tables;
+    statistics + pack + bias tables otherwise), the range and tables of a
+    dense bias matrix (two kernels), the hi/lo split of an fp32 V (float
+    mode), and the fused attention."""
+    rel = has_bias and not dense_bias
+    k = 1 if n * 64 * elem <= HEAD_STAGE_BYTES else 2 + (1 if rel else 0)
+    if dense_bias:
+        k += 2
     if mode == "float" and elem == 4:
         k += 1
     return k + 1
@@ -201,9 +206,25 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- reference arm (the oracle)
 
+def _oracle_bias(oracle, w):
+    if w.bias is None:
+        return None
+    if isinstance(w.bias, workloads.DenseBias):
+        return oracle.DenseBias(w.bias.table)
+    return oracle.RelPosBias(w.bias.table, w.bias.gh, w.bias.gw, w.bias.prefix)
+
+
+def _bias_desc(w):
+    if w.bias is None:
+        return None
+    if isinstance(w.bias, workloads.DenseBias):
+        return f"dense {w.bias.table.shape[1]}x{w.bias.table.shape[2]}/head"
+    return f"relpos {w.bias.table.shape[1]}x{w.bias.table.shape[2]}/head, prefix {w.bias.prefix}"
+
+
 def _oracle_rows_per_sec(w, N, mode, rows):
     import oracle
-    b = None if w.bias is None else oracle.RelPosBias(w.bias.table, w.bias.gh, w.bias.gw, w.bias.prefix)
+    b = _oracle_bias(oracle, w)
     t0 = time.perf_counter()
     oracle.attention(w.Q, w.K, w.V, N=N, mode=1 if mode == "u8i8" else 0, seqlens=w.seqlens, bias=b, rows=rows)
     return len(rows) / (time.perf_counter() - t0)
@@ -267,8 +288,7 @@ def run_reference(args, rank, world):
 def _config(w, N, mode):
     c = {"workload": f"{w.name}_{'dense' if N == 0 else f'top{N}'}_{mode}", "B": w.B, "H": w.H, "n": w.n, "d": w.d,
          "N": N, "mode": mode, "in_dtype": w.dtype, "seed": w.seed,
-         "bias": None if w.bias is None else f"relpos {w.bias.table.shape[1]}x{w.bias.table.shape[2]}/head, "
-                                              f"prefix {w.bias.prefix}",
+         "bias": _bias_desc(w),
          "seqlens": None if w.seqlens is None else "U{32..256} per sequence",
          "l2": "flushed between timed steps (256 MiB write)"}
     return c
@@ -296,7 +316,9 @@ def run_gpu(args, rank, world, local_rank):
     Q, K, V = dev_t(w.Q), dev_t(w.K), dev_t(w.V)
     seq = None if w.seqlens is None else torch.from_numpy(w.seqlens).to(dev)
     bias = None
-    if w.bias is not None:
+    if isinstance(w.bias, workloads.DenseBias):
+        bias = had.DenseBias(torch.from_numpy(w.bias.table).to(dev))
+    elif w.bias is not None:
         bias = had.RelPosBias(torch.from_numpy(w.bias.table).to(dev), w.bias.gh, w.bias.gw, w.bias.prefix)
     O = torch.empty_like(V)
     ws_bytes = had.had_attention_workspace_size(Q, N, mode, seq, bias)
@@ -306,8 +328,7 @@ def run_gpu(args, rank, world, local_rank):
     L = had.lib()
     import ctypes
     shp = had.make_shape(Q, seq)
-    bstruct = None if bias is None else ctypes.byref(had.had_relpos_bias(bias.table.data_ptr(), bias.gh, bias.gw,
-                                                                          bias.prefix))
+    bstruct = None if bias is None else ctypes.byref(had._bias_c(bias))
     mcode = had._MODES[mode]
     sp = ctypes.c_void_p(stream.cuda_stream)
 
@@ -325,7 +346,8 @@ def run_gpu(args, rank, world, local_rank):
         if st:
             raise had.HadError(st, "had_attention_prepared")
 
-    kernels_per_step = launches_per_step(w.n, Q.element_size(), mode, bias is not None)
+    kernels_per_step = launches_per_step(w.n, Q.element_size(), mode, bias is not None,
+                                         isinstance(w.bias, workloads.DenseBias))
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
             prepare()
@@ -366,7 +388,11 @@ def run_gpu(args, rank, world, local_rank):
     hQ, hK, hV = Q.cpu().pin_memory(), K.cpu().pin_memory(), V.cpu().pin_memory()
     hO = torch.empty_like(O, device="cpu").pin_memory()
     hseq = None if seq is None else seq.cpu()
-    hbias = None if bias is None else had.RelPosBias(bias.table.cpu().pin_memory(), bias.gh, bias.gw, bias.prefix)
+    hbias = None
+    if isinstance(bias, had.DenseBias):
+        hbias = had.DenseBias(bias.table.cpu().pin_memory())
+    elif bias is not None:
+        hbias = had.RelPosBias(bias.table.cpu().pin_memory(), bias.gh, bias.gw, bias.prefix)
     host_ws = torch.empty(had.had_attention_host_workspace_size(hQ, N, mode, hseq, hbias), dtype=torch.uint8,
                           device=dev)
     e2e_steps = min(args.steps, 30)

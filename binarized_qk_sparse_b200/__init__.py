@@ -42,7 +42,8 @@ class had_shape(ctypes.Structure):
 
 
 class had_relpos_bias(ctypes.Structure):
-    _fields_ = [("table", ctypes.c_void_p), ("gh", ctypes.c_int), ("gw", ctypes.c_int), ("prefix", ctypes.c_int)]
+    _fields_ = [("table", ctypes.c_void_p), ("gh", ctypes.c_int), ("gw", ctypes.c_int), ("prefix", ctypes.c_int),
+                ("dense", ctypes.c_int)]
 
 
 @dataclass
@@ -52,6 +53,18 @@ class RelPosBias:
     gh: int
     gw: int
     prefix: int = 0
+
+
+@dataclass
+class DenseBias:
+    """Per-head dense bias matrix [H, n, n] (fp32): b_ij = table[h, i, j]."""
+    table: torch.Tensor
+
+
+def _bias_c(bias):
+    if isinstance(bias, DenseBias):
+        return had_relpos_bias(bias.table.data_ptr(), 0, 0, 0, 1)
+    return had_relpos_bias(bias.table.data_ptr(), bias.gh, bias.gw, bias.prefix, 0)
 
 
 _lib = None
@@ -139,7 +152,7 @@ def _bias_struct(bias: RelPosBias | None):
     if bias.table.dtype != torch.float32:
         raise TypeError("bias table must be float32")
     _check_dev(bias.table)
-    return ctypes.byref(had_relpos_bias(bias.table.data_ptr(), bias.gh, bias.gw, bias.prefix))
+    return ctypes.byref(_bias_c(bias))
 
 
 def _alpha(a, H):
@@ -239,7 +252,7 @@ def _host_bias_struct(bias: RelPosBias | None):
     if bias.table.dtype != torch.float32:
         raise TypeError("bias table must be float32")
     _check_host(bias.table)
-    return ctypes.byref(had_relpos_bias(bias.table.data_ptr(), bias.gh, bias.gw, bias.prefix))
+    return ctypes.byref(_bias_c(bias))
 
 
 def had_attention_host_workspace_size(X, N=0, mode="float", seqlens=None, bias=None, chunk_b=0) -> int:

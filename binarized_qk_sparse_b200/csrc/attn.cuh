@@ -20,8 +20,9 @@ struct AttnArgs {
   const void* V;           // [BH][n][64] bf16 / fp32   (float mode)
   const int8_t* vqT;       // [BH][64][n_pad]           (uint8 mode)
   const float* vscale;     // [BH][64]
-  const float* table;      // [H][th][tw] or null
+  const float* table;      // [H][th][tw] or null ([H][n][n] when bias_dense)
   int gh, gw, prefix, th, tw;
+  int bias_dense;          // 1: b_ij = table[h][i][j]
   const float* bminmax;    // [H][2]
   const int32_t* seqlens;
   void* O;

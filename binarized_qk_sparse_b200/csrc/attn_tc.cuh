@@ -70,9 +70,10 @@ constexpr int kKoffTable = 0;  // per-head table in shared memory (n_pad <= kKof
 constexpr int kKoffWarp = 1;   // each softmax warp computes the tile's 64 offsets (double-buffered)
 constexpr int kKoffTableMax = 1024;
 // Bias variants of the kernel: none, extended tables read from global memory,
-// or (dense) the exp(bias) table staged in shared memory.
-enum { BIAS_NONE = 0, BIAS_GLOBAL = 1, BIAS_SMEM = 2 };
-constexpr int kBiasSmemMax = 6144;  // extended exp(bias) tables up to this many entries are staged in shared memory
+// (dense weights) the exp(bias) table staged in shared memory, or (dense
+// weights) a dense bias matrix's exp(bias) rows read 4 keys per 16-byte load.
+enum { BIAS_NONE = 0, BIAS_GLOBAL = 1, BIAS_SMEM = 2, BIAS_DGLOBAL = 3 };
+constexpr int kBiasSmemMax = kBiasSmemEntries;
 
 enum { SEL_DENSE = 0, SEL_TOPN_INT = 1, SEL_TOPN_FLOAT = 2 };
 enum { MODE_F = 0, MODE_Q = 1 };
@@ -94,7 +95,8 @@ struct TcArgs {
   const float* bminmax;    // [H][2] min/max of each head's table (0 included with class tokens)
   const float* expb;       // [H][E] extended exp(b - b_max(h)) table, or null
   const float* bext;       // [H][E] extended bias table, or null
-  int ext_E, ext_S, rb_class, k_class, k_invalid;  // extended-table geometry (RelposExt)
+  int ext_E, ext_S, rb_class, k_class, k_invalid;  // extended-table geometry (RelposExt or DenseExt)
+  int bias_dense;          // 1: the bias is a dense [n][n] matrix per head (rb = i S, koff = -j)
   int int_levels;          // 1 if fp32(c*s) is strictly increasing in s for every head
   int koff_mode;           // kKoffTable / kKoffWarp
   const int32_t* seqlens;
@@ -150,6 +152,7 @@ enum {
 // b_ij = ext[rb(i) - koff(j)]; class tokens and keys past L index the extension.
 __device__ __forceinline__ int key_offset(const TcArgs& a, int j, int L) {
   if (j >= L) return a.k_invalid;
+  if (a.bias_dense) return -j;
   if (j < a.prefix) return a.k_class;
   const int t = j - a.prefix;
   return (t / a.gw) * a.ext_S + t % a.gw;
@@ -187,7 +190,8 @@ template <int SEL, int MODE, int BIAS, bool VF32, int EXPORT, int SPLIT>
 __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_constant__ TcArgs a) {
   static_assert(SPLIT == 1 || SEL == SEL_DENSE || (SEL == SEL_TOPN_INT && EXPORT == EXP_NONE),
                 "two threads per row: dense, or top-N without a bias on its P.V path");
-  static_assert(BIAS != BIAS_SMEM || SEL == SEL_DENSE, "staged exp(bias) tables serve the dense weights only");
+  static_assert((BIAS != BIAS_SMEM && BIAS != BIAS_DGLOBAL) || SEL == SEL_DENSE,
+                "staged or vector-read exp(bias) tables serve the dense weights only");
   constexpr int kSplit = SPLIT;
   constexpr int kSoftWarps = 4 * kSplit;
   constexpr int kThreads = cta_threads(SPLIT);
@@ -346,7 +350,9 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
   int rb = 0;
   if (HAS_BIAS) {
     rb = a.rb_class;
-    if (row >= a.prefix && row < a.n) {
+    if (a.bias_dense) {
+      rb = min(row, a.n - 1) * a.ext_S;  // rows past the tensor are never stored
+    } else if (row >= a.prefix && row < a.n) {
       const int t = row - a.prefix;
       rb = (t / a.gw + a.gh - 1) * a.ext_S + (t % a.gw + a.gw - 1);
     }
@@ -527,8 +533,9 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
         x += r64;
         if (x >= a.gw) { x -= a.gw; ++y; }
       };
-      auto offset_of = [&](int j, int y, int x) -> int {
-        return 4 * (j >= L ? a.k_invalid : (j < a.prefix ? a.k_class : y * a.ext_S + x));  // in bytes
+      auto offset_of = [&](int j, int y, int x) -> int {  // in bytes
+        if (a.bias_dense) return 4 * (j >= L ? a.k_invalid : -j);
+        return 4 * (j >= L ? a.k_invalid : (j < a.prefix ? a.k_class : y * a.ext_S + x));
       };
       if (BIAS == BIAS_SMEM && first_pass) bounded_wait(B_BIAS, 0);
       for (int t = 0; t < ntiles; ++t) {
@@ -656,15 +663,24 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
               float e[32];
 #pragma unroll
               for (int u = 0; u < 32; u += 4) {
-                int4 k4 = make_int4(0, 0, 0, 0);
-                if (HAS_BIAS) k4 = koff4(32 * ch + u);
-                const int kk[4] = {k4.x, k4.y, k4.z, k4.w};
+                float bw[4] = {1.0f, 1.0f, 1.0f, 1.0f};
+                if (BIAS == BIAS_DGLOBAL && jb + u + 3 < L) {
+                  // a dense matrix row: keys jb+u .. +3 in one aligned 16-byte load
+                  const float4 w4 = __ldg(reinterpret_cast<const float4*>(eb_bytes) + ((jb + u) >> 2));
+                  bw[0] = w4.x; bw[1] = w4.y; bw[2] = w4.z; bw[3] = w4.w;
+                } else if (HAS_BIAS) {
+                  const int4 k4 = koff4(32 * ch + u);
+                  const int kk[4] = {k4.x, k4.y, k4.z, k4.w};
+#pragma unroll
+                  for (int v = 0; v < 4; ++v)
+                    bw[v] = (BIAS == BIAS_SMEM) ? *reinterpret_cast<const float*>(eb_bytes - kk[v])
+                                                : __ldg(reinterpret_cast<const float*>(eb_bytes - kk[v]));
+                }
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
                   const int sc = (int)r[32 * cc + u + v];
                   float x = lut_lane[-16 * sc];  // level (64 - s) / 2 of this lane's table
-                  if (BIAS == BIAS_SMEM) x *= *reinterpret_cast<const float*>(eb_bytes - kk[v]);
-                  else if (HAS_BIAS) x *= __ldg(reinterpret_cast<const float*>(eb_bytes - kk[v]));
+                  if (HAS_BIAS) x *= bw[v];
                   e[u + v] = (FULL || 32 * ch + u + v < nvalid) ? x : 0.0f;
                 }
               }
@@ -1151,7 +1167,9 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
               float l;
               if (HAS_BIAS) {
                 int off;  // entry (i, j) of the extended table sits at rb - off
-                if (j < a.prefix) {
+                if (a.bias_dense) {
+                  off = -j;
+                } else if (j < a.prefix) {
                   off = a.k_class;
                 } else {
                   const int t = j - a.prefix, y = t / a.gw;

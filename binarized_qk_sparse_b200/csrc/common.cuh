@@ -50,6 +50,31 @@ __host__ __device__ inline RelposExt relpos_ext(int gh, int gw) {
   return r;
 }
 
+// Extended tables of a dense bias matrix [n][n] (BinaryAttention §2.3, the
+// "dense learnable matrix" option: one bias per query-key pair).  Row i sits at
+// i * S with S >= n + 1 -- odd when the tables fit shared memory, so the 32
+// query rows of a warp fall in distinct banks, else a multiple of 4 -- and
+// column n of every row is the masked-key sentinel.  With
+// rb(i) = i * S and koff(j) = -j (k_invalid = -n for keys past L), entry
+// rb(i) - koff(j) is the pair (i, j), as with the relative-position tables.
+// (S is odd only for tables small enough for shared memory; see below.)
+// Tables that do not fit shared memory (more than kBiasSmemEntries entries) are
+// read from global memory, and there a row stride that is a multiple of 4 lets a
+// thread fetch 4 consecutive keys with one 16-byte load instead.
+constexpr int kBiasSmemEntries = 6144;  // extended exp(bias) tables up to this many entries go to shared memory
+struct DenseExt {
+  int S, E, k_invalid;
+};
+__host__ __device__ inline DenseExt dense_ext(int n) {
+  DenseExt r;
+  r.S = (n + 1) | 1;
+  if (n * r.S > kBiasSmemEntries) r.S = (n + 4) & ~3;
+  r.E = (n * r.S + 3) / 4 * 4;  // padded to 16 bytes per head (bulk copies)
+  r.k_invalid = -n;
+  return r;
+}
+constexpr int kDenseBiasMaxN = 4096;  // a dense matrix grows as n^2: 2 tables of H * n * S floats
+
 // Valid length of sequence b; an out-of-range entry raises the device status
 // and returns 0, which makes every kernel treat that batch as empty (zero output).
 __device__ __forceinline__ int valid_len(const int32_t* seqlens, int b, int n, unsigned* status) {

@@ -50,7 +50,10 @@ __global__ void __launch_bounds__(kAttnThreads) k_dense_ref(const __grid_constan
   }
   const float* tab = HAS_BIAS ? a.table + (size_t)h * a.th * a.tw : nullptr;
   int rb0 = -1, rb1 = -1;
-  if (HAS_BIAS) {
+  if (HAS_BIAS && a.bias_dense) {  // entry rb - koff = i n + j
+    if (i0 < a.n) rb0 = i0 * a.n;
+    if (i1 < a.n) rb1 = i1 * a.n;
+  } else if (HAS_BIAS) {
     if (i0 >= a.prefix && i0 < a.n) { int t = i0 - a.prefix; rb0 = (t / a.gw + a.gh - 1) * a.tw + (t % a.gw + a.gw - 1); }
     if (i1 >= a.prefix && i1 < a.n) { int t = i1 - a.prefix; rb1 = (t / a.gw + a.gh - 1) * a.tw + (t % a.gw + a.gw - 1); }
   }
@@ -73,7 +76,8 @@ __global__ void __launch_bounds__(kAttnThreads) k_dense_ref(const __grid_constan
     }
     if (HAS_BIAS && tid < kKT) {
       int j = j0 + tid, off = INT_MIN;
-      if (j >= a.prefix && j < a.n) { int tt = j - a.prefix; off = (tt / a.gw) * a.tw + tt % a.gw; }
+      if (a.bias_dense && j < a.n) off = -j;
+      else if (!a.bias_dense && j >= a.prefix && j < a.n) { int tt = j - a.prefix; off = (tt / a.gw) * a.tw + tt % a.gw; }
       koff[buf][tid] = off;
     }
     cp_async_commit();

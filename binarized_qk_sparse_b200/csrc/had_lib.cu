@@ -90,6 +90,11 @@ had_status check_shape(const had_shape* s) {
 
 had_status check_bias(const had_shape* s, const had_relpos_bias* bias) {
   if (!bias || !bias->table) return HAD_OK;
+  if (reinterpret_cast<uintptr_t>(bias->table) & 3u) return HAD_ERR_INVALID;
+  if (bias->dense != 0) {
+    if (bias->dense != 1) return HAD_ERR_INVALID;
+    return s->n > kDenseBiasMaxN ? HAD_ERR_UNSUPPORTED : HAD_OK;
+  }
   if (bias->gh <= 0 || bias->gw <= 0 || bias->prefix < 0) return HAD_ERR_INVALID;
   if ((long long)bias->gh * bias->gw + bias->prefix != s->n) return HAD_ERR_INVALID;
   if (reinterpret_cast<uintptr_t>(bias->table) & 3u) return HAD_ERR_INVALID;
@@ -117,7 +122,7 @@ Ws ws_layout(const had_shape* s, bool quant, const had_relpos_bias* bias_desc) {
   w.bext = w.expb = 0;
   if (bias) {
     w.bminmax = off; off += align_up((size_t)s->H * 2 * 4);
-    const size_t cells = (size_t)relpos_ext(bias_desc->gh, bias_desc->gw).E;
+    const size_t cells = bias_desc->dense ? (size_t)dense_ext(s->n).E : (size_t)relpos_ext(bias_desc->gh, bias_desc->gw).E;
     w.bext = off; off += align_up((size_t)s->H * cells * 4);
     w.expb = off; off += align_up((size_t)s->H * cells * 4);
   }
@@ -299,9 +304,19 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
   if (has_bias) {
     ba.table = bias->table;
     ba.gh = bias->gh; ba.gw = bias->gw; ba.prefix = bias->prefix;
+    ba.dense = bias->dense; ba.n = s->n;
+    if (ba.dense) { ba.gh = ba.gw = 1; ba.prefix = 0; }
     ba.bminmax = reinterpret_cast<float*>(ws + w.bminmax);
     ba.bext = reinterpret_cast<float*>(ws + w.bext);
     ba.expb = reinterpret_cast<float*>(ws + w.expb);
+  }
+  if (has_bias && ba.dense) {
+    // dense matrix: its range, then its tables over many CTAs per head
+    k_dense_bias_range<<<s->H, kDenseRangeThreads, 0, st>>>(ba);
+    if ((r = check_launch("k_dense_bias_range")) != HAD_OK) return r;
+    dim3 tgrid((dense_ext(s->n).E + kDenseTabPerCta - 1) / kDenseTabPerCta, s->H);
+    k_dense_bias_tables<<<tgrid, 256, 0, st>>>(ba);
+    if ((r = check_launch("k_dense_bias_tables")) != HAD_OK) return r;
   }
   if (head_bytes <= (size_t)kHeadMaxBytes) {
     // short heads: one read of each head, statistics and packing from shared memory
@@ -311,8 +326,8 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
     ha.B = s->B; ha.H = s->H; ha.n = s->n; ha.n_pad = dims_of(s).n_pad;
     ha.seqlens = s->seqlens;
     ha.qbits = qbits; ha.kpm = kpm; ha.vqT = vqT; ha.vscale = vscale; ha.status = status;
-    ha.bias_slice = do_v ? 3 : 2;  // the bias tables ride along as one more grid slice
-    dim3 grid(dims_of(s).BH, ha.bias_slice + (has_bias ? 1 : 0));
+    ha.bias_slice = do_v ? 3 : 2;  // relative-position tables ride along as one more grid slice
+    dim3 grid(dims_of(s).BH, ha.bias_slice + (has_bias && !ba.dense ? 1 : 0));
     const int smem = (int)head_bytes;
     int dev = 0;
     cudaGetDevice(&dev);
@@ -328,7 +343,7 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
     r = launch_prep(s, Q, K, V, 0, do_v ? 3 : 2, sums, amax, nullptr, nullptr, qbits, nullptr, nullptr, kpm, vqT,
                     vscale, st, status);
     if (r != HAD_OK) return r;
-    if (has_bias) {
+    if (has_bias && !ba.dense) {
       k_bias_tables<<<s->H, 256, 0, st>>>(ba);
       if ((r = check_launch("k_bias_tables")) != HAD_OK) return r;
     }
@@ -363,11 +378,13 @@ had_status launch_tc_t(const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
   return check_launch("k_attn_tc");
 }
 
-// Dense: no bias, extended tables in global memory, or the exp(bias) table staged in shared memory.
+// Dense: no bias, extended tables in global memory, the exp(bias) table staged in
+// shared memory, or a dense bias matrix read 4 keys per load.
 template <int SEL, int MODE, bool VF32, int EXP>
 had_status launch_tc_b(int bias, const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
   using namespace tc;
   if (bias == BIAS_SMEM) return launch_tc_t<SEL, MODE, BIAS_SMEM, VF32, EXP, 2>(a, grid, st);
+  if (bias == BIAS_DGLOBAL) return launch_tc_t<SEL, MODE, BIAS_DGLOBAL, VF32, EXP, 2>(a, grid, st);
   if (bias == BIAS_GLOBAL) return launch_tc_t<SEL, MODE, BIAS_GLOBAL, VF32, EXP, 2>(a, grid, st);
   return launch_tc_t<SEL, MODE, BIAS_NONE, VF32, EXP, 2>(a, grid, st);
 }
@@ -445,15 +462,19 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
   a.v_f32 = (s->in_dtype == HAD_F32) ? 1 : 0;
   a.vscale = quant ? reinterpret_cast<float*>(ws + w.vscale) : nullptr;
   a.table = has_bias ? bias->table : nullptr;
-  if (has_bias) {
-    a.gh = bias->gh; a.gw = bias->gw; a.prefix = bias->prefix;
-    a.th = 2 * bias->gh - 1; a.tw = 2 * bias->gw - 1;
-  }
   a.bminmax = has_bias ? reinterpret_cast<float*>(ws + w.bminmax) : nullptr;
   a.expb = has_bias ? reinterpret_cast<float*>(ws + w.expb) : nullptr;
   a.bext = has_bias ? reinterpret_cast<float*>(ws + w.bext) : nullptr;
-  if (has_bias) {
+  if (has_bias && bias->dense) {
+    const DenseExt x = dense_ext(s->n);
+    a.bias_dense = 1;
+    a.gh = 1; a.gw = 1; a.prefix = 0;
+    a.th = s->n; a.tw = s->n;
+    a.ext_E = x.E; a.ext_S = x.S; a.rb_class = 0; a.k_class = 0; a.k_invalid = x.k_invalid;
+  } else if (has_bias) {
     const RelposExt x = relpos_ext(bias->gh, bias->gw);
+    a.gh = bias->gh; a.gw = bias->gw; a.prefix = bias->prefix;
+    a.th = 2 * bias->gh - 1; a.tw = 2 * bias->gw - 1;
     a.ext_E = x.E; a.ext_S = x.S; a.rb_class = x.rb_class; a.k_class = x.k_class; a.k_invalid = x.k_invalid;
   }
   a.seqlens = s->seqlens;
@@ -462,7 +483,10 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
   a.B = d.B; a.H = d.H; a.n = d.n; a.n_pad = d.n_pad; a.N = N;
   a.status = status;
   a.koff_mode = (d.n_pad <= tc::kKoffTableMax) ? tc::kKoffTable : tc::kKoffWarp;
-  const int bias_kind = !has_bias ? tc::BIAS_NONE : (a.ext_E <= tc::kBiasSmemMax ? tc::BIAS_SMEM : tc::BIAS_GLOBAL);
+  const int bias_kind = !has_bias                        ? tc::BIAS_NONE
+                        : a.ext_E <= tc::kBiasSmemMax      ? tc::BIAS_SMEM
+                        : a.bias_dense && a.ext_S % 4 == 0 ? tc::BIAS_DGLOBAL
+                                                           : tc::BIAS_GLOBAL;
   a.int_levels = 1;
   for (int h = 0; h < s->H; ++h) {
     const double aq = alpha_q ? (double)alpha_q[h] : 1.0, ak = alpha_k ? (double)alpha_k[h] : 1.0;
@@ -546,7 +570,9 @@ had_status host_plan(const had_shape* s, had_mode mode, const had_relpos_bias* b
   p->seq = off;
   off += align_up((size_t)s->B * sizeof(int32_t));
   p->tab = off;
-  p->tab_bytes = has_bias ? (size_t)s->H * (2 * bias->gh - 1) * (2 * bias->gw - 1) * sizeof(float) : 0;
+  p->tab_bytes = !has_bias ? 0
+                 : bias->dense ? (size_t)s->H * s->n * s->n * sizeof(float)
+                               : (size_t)s->H * (2 * bias->gh - 1) * (2 * bias->gw - 1) * sizeof(float);
   off += align_up(p->tab_bytes);
   p->slot0 = off;
   size_t so = 0;
@@ -821,7 +847,11 @@ had_status had_dense_reference_mode(const void* Q, const void* K, const void* V,
   AttnArgs a{};
   a.V = V;
   a.table = has_bias ? bias->table : nullptr;
-  if (has_bias) {
+  if (has_bias && bias->dense) {
+    a.bias_dense = 1;
+    a.gh = 1; a.gw = 1; a.prefix = 0;
+    a.th = s->n; a.tw = s->n;
+  } else if (has_bias) {
     a.gh = bias->gh; a.gw = bias->gw; a.prefix = bias->prefix;
     a.th = 2 * bias->gh - 1; a.tw = 2 * bias->gw - 1;
   }

@@ -245,12 +245,14 @@ struct HeadArgs {
 };
 
 // Per-head bias range (0 included when class tokens exist: their pairs have bias
-// 0) and the two extended tables (see RelposExt) the attention kernel reads:
-// the bias itself (class pairs 0, keys past L -inf) and exp(b - b_max) (class
-// pairs exp(-b_max), keys past L 0).  One CTA per head.
+// 0) and the two extended tables (see RelposExt, DenseExt) the attention kernel
+// reads: the bias itself (class pairs 0, keys past L -inf) and exp(b - b_max)
+// (class pairs exp(-b_max), keys past L 0).  One CTA per head (relative-position
+// tables; dense matrices below).
 struct BiasArgs {
-  const float* table;  // [H][2gh-1][2gw-1] or null
+  const float* table;  // [H][2gh-1][2gw-1], or [H][n][n] when dense, or null
   int gh, gw, prefix;
+  int dense, n;        // dense: a bias matrix over the n x n pairs
   float* bminmax;      // [H][2]
   float* bext;         // [H][E]
   float* expb;         // [H][E]
@@ -259,10 +261,11 @@ struct BiasArgs {
 __device__ __forceinline__ void bias_tables_block(const BiasArgs& a, int h) {
   __shared__ float smn[32], smx[32];
   const RelposExt x = relpos_ext(a.gh, a.gw);
-  const int tw = 2 * a.gw - 1, cells = (2 * a.gh - 1) * tw;
+  const int tw = 2 * a.gw - 1;
+  const size_t cells = (size_t)(2 * a.gh - 1) * tw;
   const float* t = a.table + (size_t)h * cells;
   float mn = INFINITY, mx = -INFINITY;
-  for (int e = threadIdx.x; e < cells; e += blockDim.x) { mn = fminf(mn, t[e]); mx = fmaxf(mx, t[e]); }
+  for (size_t e = threadIdx.x; e < cells; e += blockDim.x) { mn = fminf(mn, t[e]); mx = fmaxf(mx, t[e]); }
   for (int o = 16; o > 0; o >>= 1) {
     mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
@@ -293,6 +296,66 @@ __device__ __forceinline__ void bias_tables_block(const BiasArgs& a, int h) {
 }
 
 __global__ void __launch_bounds__(256) k_bias_tables(const BiasArgs a) { bias_tables_block(a, blockIdx.x); }
+
+// A dense bias matrix has n^2 entries per head, too many for one CTA per head to
+// turn into tables quickly: one CTA per head takes the range, then the tables
+// are written by many CTAs per head (grid (entries / kDenseTabPerCta, H)).
+constexpr int kDenseTabPerCta = 4096;
+
+constexpr int kDenseRangeThreads = 1024;
+
+__global__ void __launch_bounds__(kDenseRangeThreads) k_dense_bias_range(const BiasArgs a) {
+  constexpr int kWarps = kDenseRangeThreads / 32, kInFlight = 8;  // loads in flight per thread
+  __shared__ float smn[kWarps], smx[kWarps];
+  const int h = blockIdx.x;
+  const size_t cells = (size_t)a.n * a.n;
+  const float* t = a.table + (size_t)h * cells;
+  float mn = INFINITY, mx = -INFINITY;
+  for (size_t e0 = threadIdx.x; e0 < cells; e0 += (size_t)kInFlight * kDenseRangeThreads) {
+    float v[kInFlight];
+#pragma unroll
+    for (int k = 0; k < kInFlight; ++k) {
+      const size_t e = e0 + (size_t)k * kDenseRangeThreads;
+      v[k] = e < cells ? __ldg(t + e) : t[e0];
+    }
+#pragma unroll
+    for (int k = 0; k < kInFlight; ++k) { mn = fminf(mn, v[k]); mx = fmaxf(mx, v[k]); }
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if ((threadIdx.x & 31) == 0) { smn[threadIdx.x >> 5] = mn; smx[threadIdx.x >> 5] = mx; }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < kWarps; ++w) { mn = fminf(mn, smn[w]); mx = fmaxf(mx, smx[w]); }
+    a.bminmax[2 * h] = mn;
+    a.bminmax[2 * h + 1] = mx;
+  }
+}
+
+__global__ void __launch_bounds__(256) k_dense_bias_tables(const BiasArgs a) {
+  const int h = blockIdx.y;
+  const DenseExt dx = dense_ext(a.n);
+  const float* t = a.table + (size_t)h * a.n * a.n;
+  const float mx = a.bminmax[2 * h + 1];
+  const float kLog2e = 1.4426950408889634f;
+  float* be = a.bext + (size_t)h * dx.E;
+  float* ee = a.expb + (size_t)h * dx.E;
+  const int e1 = min(dx.E, (int)(blockIdx.x + 1) * kDenseTabPerCta);
+  for (int e = blockIdx.x * kDenseTabPerCta + threadIdx.x; e < e1; e += blockDim.x) {
+    const int i = e / dx.S, j = e - i * dx.S;  // row i at i * S, the sentinel in column n, padding 0
+    float b = 0.0f, w = 0.0f;
+    if (i < a.n && j < a.n) {
+      b = t[(size_t)i * a.n + j];
+      w = exp2f((b - mx) * kLog2e);
+    } else if (i < a.n && j == a.n) {
+      b = -INFINITY;
+    }
+    be[e] = b;
+    ee[e] = w;
+  }
+}
 
 // int8 code of x at scale sc: rint(x / sc) clamped to +-127, with x / sc the
 // correctly rounded fp32 quotient.  For |x / sc| <= 128 the product x * (1/sc)

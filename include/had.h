@@ -68,15 +68,24 @@ typedef struct {
   const int32_t* seqlens;   /* DEVICE [B] valid lengths in [1, n], or NULL for all n */
 } had_shape;
 
-/* Learnable relative-position bias (BinaryAttention §2.3, "position-sensitive
- * bias", the option its experiments use).  Token t >= prefix is patch
- * (y, x) = divmod(t - prefix, gw) of a gh x gw grid; then
- * b_ij = table[h][(y_i - y_j) + gh - 1][(x_i - x_j) + gw - 1], and b_ij = 0
- * when i < prefix or j < prefix (class tokens).  Requires gh*gw + prefix == n. */
+/* Learnable attention bias B of BinaryAttention §2.3.
+ * dense == 0: the relative-position bias ("position-sensitive bias", the option
+ *   its experiments use).  Token t >= prefix is patch (y, x) =
+ *   divmod(t - prefix, gw) of a gh x gw grid; then
+ *   b_ij = table[h][(y_i - y_j) + gh - 1][(x_i - x_j) + gw - 1], and b_ij = 0
+ *   when i < prefix or j < prefix (class tokens).  Requires gh*gw + prefix == n.
+ * dense == 1: the dense learnable matrix (one bias per query-key pair):
+ *   b_ij = table[h][i][j], table [H][n][n]; gh, gw and prefix are ignored.  Its
+ *   extended tables take 2 * H * n * (n + 2) floats of workspace, so n is
+ *   limited to 4096 (HAD_ERR_UNSUPPORTED above).
+ * A bias that is a sum of functions of the relative offset (y_i - y_j,
+ * x_i - x_j), such as a spatial plus a directional term, is a
+ * relative-position table: pass its (2gh-1) x (2gw-1) values with dense == 0. */
 typedef struct {
-  const float* table;  /* DEVICE fp32 [H][2*gh-1][2*gw-1]; NULL means no bias */
+  const float* table;  /* DEVICE fp32 (HOST in had_attention_host); NULL means no bias */
   int gh, gw;
   int prefix;
+  int dense;           /* 0: relative-position table; 1: dense [H][n][n] matrix */
 } had_relpos_bias;
 
 /* ---- binarize and pack (BinaryAttention §2.2; HAD abstract) --------------
@@ -136,7 +145,7 @@ had_status had_attention_prepared(const void* V, const had_shape* s, const had_r
  * had_attention_host: had_attention on HOST memory, with the copies inside the
  * call.  Q, K, V: HOST [B][H][n][d] in s->in_dtype; O: HOST [B][H][n][d] in
  * o_dtype; s->seqlens: HOST int32 [B] (each in [1, n], checked on the host) or
- * NULL; bias->table: HOST fp32 [H][2gh-1][2gw-1] or bias NULL; alpha_q,
+ * NULL; bias->table: HOST fp32 (as the bias struct describes) or bias NULL; alpha_q,
  * alpha_k as in had_attention.  The batch is cut into chunks of chunk_b
  * sequences (0: the library picks about 8 MiB of inputs per chunk).  Chunk k's
  * Q, K, V are copied in on one side stream while chunk k-1 is computed on

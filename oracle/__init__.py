@@ -145,9 +145,17 @@ class RelPosBias:
     prefix: int
 
 
+@dataclass
+class DenseBias:
+    """Per-head dense bias matrix [H, n, n]: b_ij = table[h, i, j] (one learnable value per query-key pair)."""
+    table: np.ndarray
+
+
 def _bias_args(bias):
     if bias is None:
         return None, 0, 0, 0
+    if isinstance(bias, DenseBias):
+        return _f32(bias.table), 0, 0, 0  # gh == gw == 0 selects the dense matrix
     return _f32(bias.table), int(bias.gh), int(bias.gw), int(bias.prefix)
 
 

@@ -30,6 +30,9 @@
  *   - relative-position bias: token t >= prefix is patch (y, x) with
  *     t = prefix + y*gw + x; b_ij = table[h][(y_i - y_j) + gh - 1][(x_i - x_j) + gw - 1];
  *     b = 0 when i or j is a prefix (cls) token or when there is no table.
+ *   - dense bias matrix (BinaryAttention §2.3, one learnable bias per query-key
+ *     pair), selected by gh == gw == 0 (prefix 0): b_ij = table[h][i][j] of an
+ *     [H][n][n] table.
  *   - keys j >= L are never kept; output rows i >= L are 0; bits of tokens
  *     i >= L are 0; the V scales use valid tokens only.
  *   - V scale s_c = absmax_c / 127 in fp32 (1 when absmax is 0);
@@ -184,9 +187,11 @@ int hado_v_quant(const float* V, int B, int H, int n, int d, const int32_t* seql
   return HADO_OK;
 }
 
-/* Relative-position bias b_ij for head h (reading stated in the header). */
-static float rel_bias(const float* table, int H, int h, int gh, int gw, int prefix, int i, int j) {
+/* Bias b_ij for head h (readings stated in the header): the relative-position
+ * table, or with gh == gw == 0 the dense matrix [H][n][n]. */
+static float rel_bias(const float* table, int H, int h, int gh, int gw, int prefix, int n, int i, int j) {
   (void)H;
+  if (table && gh == 0 && gw == 0) return table[((size_t)h * n + i) * n + j];
   if (!table || i < prefix || j < prefix) return 0.0f;
   int ti = i - prefix, tj = j - prefix;
   int yi = ti / gw, xi = ti % gw, yj = tj / gw, xj = tj % gw;
@@ -237,7 +242,7 @@ int hado_logits(const uint32_t* qbits, const uint32_t* kbits, int B, int H, int 
           float v = NAN;
           if (i < L && j < L) {
             int s = binary_score(qbits + (bh * n + i) * W, kbits + (bh * n + j) * W, d);
-            v = fmaf((float)s, c, rel_bias(table, H, h, gh, gw, prefix, i, j));
+            v = fmaf((float)s, c, rel_bias(table, H, h, gh, gw, prefix, n, i, j));
           }
           out[(bh * n + i) * (size_t)n + j] = v;
         }
@@ -264,7 +269,9 @@ int hado_attention(const float* Q, const float* K, const float* V, int B, int H,
                    uint32_t* kbits_out, int8_t* Vq_out, float* vscale_out) {
   if (!Q || !K || !V || !O || B <= 0 || H <= 0 || n <= 0 || d <= 0 || d % 32 != 0 || N < 0) return HADO_ERR_ARG;
   if (mode != 0 && mode != 1) return HADO_ERR_ARG;
-  if (table && (gh <= 0 || gw <= 0 || prefix < 0 || (int64_t)gh * gw + prefix != n)) return HADO_ERR_ARG;
+  if (table && !(gh == 0 && gw == 0 && prefix == 0) &&
+      (gh <= 0 || gw <= 0 || prefix < 0 || (int64_t)gh * gw + prefix != n))
+    return HADO_ERR_ARG;
   for (int h = 0; h < H; ++h) {
     if (alpha_q && !(alpha_q[h] > 0.0f)) return HADO_ERR_ARG;
     if (alpha_k && !(alpha_k[h] > 0.0f)) return HADO_ERR_ARG;
@@ -324,7 +331,7 @@ int hado_attention(const float* Q, const float* K, const float* V, int B, int H,
     const uint32_t* q = qb + ((size_t)bh * n + i) * W;
     for (int j = 0; j < L; ++j) {
       int s = binary_score(q, kb + ((size_t)bh * n + j) * W, d);
-      key[j].l = fmaf((float)s, c, rel_bias(table, H, h, gh, gw, prefix, i, j));
+      key[j].l = fmaf((float)s, c, rel_bias(table, H, h, gh, gw, prefix, n, i, j));
       key[j].j = j;
     }
     /* Step 5: the kept set is the first K_eff keys of the full sort. */
@@ -403,7 +410,9 @@ int hado_dense_attention(const float* Q, const float* K, const float* V, int B, 
                          const int32_t* seqlens, const float* table, int gh, int gw, int prefix, int N,
                          const int64_t* rows, int64_t nrows, double* O) {
   if (!Q || !K || !V || !O || B <= 0 || H <= 0 || n <= 0 || d <= 0 || N < 0) return HADO_ERR_ARG;
-  if (table && (gh <= 0 || gw <= 0 || prefix < 0 || (int64_t)gh * gw + prefix != n)) return HADO_ERR_ARG;
+  if (table && !(gh == 0 && gw == 0 && prefix == 0) &&
+      (gh <= 0 || gw <= 0 || prefix < 0 || (int64_t)gh * gw + prefix != n))
+    return HADO_ERR_ARG;
   for (int b = 0; b < B; ++b) {
     int L = valid_len(seqlens, b, n);
     if (L < 1 || L > n) return HADO_ERR_ARG;
@@ -433,7 +442,7 @@ int hado_dense_attention(const float* Q, const float* K, const float* V, int B, 
       const float* k = K + ((size_t)bh * n + j) * d;
       double dot = 0.0;
       for (int c = 0; c < d; ++c) dot += (double)q[c] * (double)k[c];
-      l[j] = dot / sqrt((double)d) + (double)rel_bias(table, H, h, gh, gw, prefix, i, j);
+      l[j] = dot / sqrt((double)d) + (double)rel_bias(table, H, h, gh, gw, prefix, n, i, j);
       order[j] = j;
     }
     int keff = (N == 0 || N >= L) ? L : N;

@@ -154,3 +154,28 @@ def test_host_workspace_grows_with_the_chunk(L):
     # three slots of one chunk each hold Q, K, V and O at least
     one = 3 * 197 * 64 * 2 + 197 * 64 * 4
     assert sizes[0] >= 3 * one
+
+
+def test_dense_bias_matrix_validation(L):
+    import binarized_qk_sparse_b200 as m
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    ws = P(0x20000)
+    big = 1 << 34
+
+    def att(shape, bias):
+        return L.had_attention(fake, fake, fake, ctypes.byref(shape), ctypes.byref(bias), None, None, 0, 0, fake, 1,
+                               ws, big, None)
+
+    shp = _shape(m, n=197)
+    assert att(shp, m.had_relpos_bias(0x30000, 0, 0, 0, 2)) == m.HAD_ERR_INVALID     # unknown kind
+    assert att(shp, m.had_relpos_bias(0x30002, 0, 0, 0, 1)) == m.HAD_ERR_INVALID     # misaligned table
+    assert att(_shape(m, n=4097), m.had_relpos_bias(0x30000, 0, 0, 0, 1)) == m.HAD_ERR_UNSUPPORTED
+    # the grid fields are ignored for a dense matrix; its tables take n * (n + 2) floats per head
+    shp = _shape(m, B=2, H=3, n=197)
+    rel = m.had_relpos_bias(0x30000, 14, 14, 1, 0)
+    dense = m.had_relpos_bias(0x30000, 7, 7, 1, 1)
+    wr = L.had_attention_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(rel))
+    wd = L.had_attention_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(dense))
+    assert wd > wr > 0
+    assert wd - L.had_attention_workspace_size(ctypes.byref(shp), 0, 1, None) >= 2 * 3 * 197 * 198 * 4

@@ -32,9 +32,19 @@ def _dev_inputs(w):
     Q, K, V = _dev(w, w.Q), _dev(w, w.K), _dev(w, w.V)
     seq = None if w.seqlens is None else torch.from_numpy(w.seqlens).cuda()
     bias = None
-    if w.bias is not None:
+    if isinstance(w.bias, workloads.DenseBias):
+        bias = had.DenseBias(torch.from_numpy(w.bias.table).cuda())
+    elif w.bias is not None:
         bias = had.RelPosBias(torch.from_numpy(w.bias.table).cuda(), w.bias.gh, w.bias.gw, w.bias.prefix)
     return Q, K, V, seq, bias
+
+
+def _oracle_bias(oracle_mod, w):
+    if w.bias is None:
+        return None
+    if isinstance(w.bias, workloads.DenseBias):
+        return oracle_mod.DenseBias(w.bias.table)
+    return oracle_mod.RelPosBias(w.bias.table, w.bias.gh, w.bias.gw, w.bias.prefix)
 
 
 def _tol(w):
@@ -120,7 +130,7 @@ def test_integer_scores_bit_exact(oracle_mod, name):
 def _oracle_full(oracle_mod, w, N, mode, rows=None, want_idx=False, want_codes=False):
     key = (w.name, N, mode, None if rows is None else rows.tobytes(), want_idx, want_codes)
     if key not in _cache:
-        b = None if w.bias is None else oracle_mod.RelPosBias(w.bias.table, w.bias.gh, w.bias.gw, w.bias.prefix)
+        b = _oracle_bias(oracle_mod, w)
         _cache[key] = oracle_mod.attention(w.Q, w.K, w.V, N=N, mode=mode, seqlens=w.seqlens, bias=b, rows=rows,
                                            want_idx=want_idx, want_codes=want_codes)
     return _cache[key]
@@ -376,6 +386,56 @@ def test_alpha_and_bias_ties(oracle_mod):
         np.testing.assert_array_equal(idx, ref.idx)
         O = had.had_attention(Q, K, V, N=N, bias=bias, alpha_q=aq, alpha_k=ak).float().cpu().numpy()
         assert np.max(np.abs(O - ref.O)) <= _tol(w)
+
+
+def _dense_bias_workload(B, H, n, seqlens, seed, dtype="bf16"):
+    rng = np.random.default_rng(seed)
+    Q = workloads.bf16_round(rng.standard_normal((B, H, n, 64)).astype(np.float32))
+    K = workloads.bf16_round(rng.standard_normal((B, H, n, 64)).astype(np.float32))
+    V = workloads.bf16_round(rng.standard_normal((B, H, n, 64)).astype(np.float32))
+    table = (rng.standard_normal((H, n, n)) * 0.1).astype(np.float32)
+    sl = None if seqlens is None else np.asarray(seqlens, np.int32)
+    return workloads.Workload(f"dense_bias_b{B}_h{H}_n{n}", B, H, n, 64, dtype, Q, K, V, sl,
+                              workloads.DenseBias(table), [], seed, "")
+
+
+@pytest.mark.parametrize("n,seqlens", [
+    (70, [70, 33]),          # extended tables staged in shared memory, key offsets from a table
+    (197, None),             # DeiT length: tables in global memory
+    (197, [197, 120]),
+    (1100, [1100, 700]),     # n > 1024: key offsets computed per tile by each warp
+])
+def test_dense_bias_matrix(oracle_mod, n, seqlens):
+    # BinaryAttention §2.3's dense learnable matrix, b_ij = table[h][i][j]:
+    # dense uint8 and float O, top-N float O and kept sets, uint8 codes
+    w = _dense_bias_workload(len(seqlens or [0]), 2, n, seqlens, 40 + n)
+    Q, K, V, seq, bias = _dev_inputs(w)
+    rows = _sample_rows(w, 24, 3)
+    rows_t = torch.from_numpy(rows).cuda()
+    N = max(1, n // 8)
+    for Nk, mode in ((0, "u8i8"), (0, "float"), (N, "float")):
+        m = 1 if mode == "u8i8" else 0
+        O = _flat(had.had_attention(Q, K, V, N=Nk, mode=mode, seqlens=seq, bias=bias))[rows_t].float().cpu().numpy()
+        ref = _oracle_full(oracle_mod, w, Nk, m, rows=rows)
+        assert np.max(np.abs(O - ref.O)) <= _tol(w), (Nk, mode)
+    idx = _flat(had.had_topn_indices(Q, K, N, seq, bias))[rows_t].cpu().numpy()
+    np.testing.assert_array_equal(idx, _oracle_full(oracle_mod, w, N, 0, rows=rows, want_idx=True).idx)
+    r0, r1 = 0, min(n, 64)
+    A = had.had_attention_codes_u8(Q, K, V, r0, r1, N=0, seqlens=seq, bias=bias).cpu().numpy().reshape(-1, n)
+    band = np.array([bh * n + i for bh in range(w.B * w.H) for i in range(r0, r1)], np.int64)
+    _codes_ok(A, _oracle_full(oracle_mod, w, 0, 1, rows=band, want_codes=True).Aq)
+
+
+def test_dense_bias_matrix_reference_mode_and_host_entry(oracle_mod):
+    w = _dense_bias_workload(2, 2, 197, [197, 150], 77)
+    Q, K, V, seq, bias = _dev_inputs(w)
+    O = had.had_dense_reference_mode(Q, K, V, seqlens=seq, bias=bias).float().cpu().numpy()
+    ref = oracle_mod.dense_attention(w.Q, w.K, w.V, seqlens=w.seqlens, bias=_oracle_bias(oracle_mod, w))
+    assert np.max(np.abs(O - ref)) <= 1e-2 * np.max(np.abs(w.V))
+    dev = had.had_attention(Q, K, V, N=25, seqlens=seq, bias=bias).cpu()
+    hb = had.DenseBias(bias.table.cpu())
+    got = had.had_attention_host(Q.cpu(), K.cpu(), V.cpu(), N=25, seqlens=seq.cpu(), bias=hb, chunk_b=1)
+    assert torch.equal(got, dev)
 
 
 @pytest.mark.parametrize("mode", ["float", "u8i8"])

@@ -7,7 +7,9 @@ method summary; "BinaryAttention: One-Bit QK-Attention" = BA, §2.1-§2.4):
   - score: the identity dot(sign q, sign k) = d - 2*Hamming (BA §2.1 distance
     view, §2.2 XNOR + popcount; HAD abstract) via numpy +-1 matmuls and an
     exhaustive 8-bit sweep; Theorem 1 (BA §2.1) statistically.
-  - logit: bias indexing with an injective table; alpha scale.
+  - logit: bias indexing with an injective table (relative-position and dense
+    matrix, BA §2.3); a dense matrix built from a relative-position table gives
+    the same result as the table; alpha scale.
   - top-N: numpy lexsort brute force; N >= L reduces to dense; nesting; alpha invariance.
   - softmax / A.V: rows sum to 1; exp(-Hamming) shift form; independent dense
     attention in numpy; padded batch == each sequence alone.
@@ -175,6 +177,35 @@ def test_relpos_bias_indexing(oracle_mod):
                 assert l[0, h, i, j] == np.float32(8.0 + b)
 
 
+def test_dense_bias_matrix_indexing(oracle_mod):
+    # BA §2.3's dense learnable matrix: b_ij = table[h][i][j] for query i, key j
+    n, d, H = 9, 64, 2
+    table = np.zeros((H, n, n), np.float32)
+    for h in range(H):
+        for i in range(n):
+            for j in range(n):
+                table[h, i, j] = 1000 * h + 37 * i + j + 1   # injective, not symmetric
+    bits = np.zeros((1, H, n, 2), np.uint32)                 # all scores = d = 64
+    l = oracle_mod.logits(bits, bits, d, bias=oracle_mod.DenseBias(table))
+    for h in range(H):
+        for i in range(n):
+            for j in range(n):
+                assert l[0, h, i, j] == np.float32(8.0 + 1000 * h + 37 * i + j + 1)
+
+
+def test_dense_bias_matrix_of_a_relpos_table_matches_the_table(oracle_mod):
+    Q, K, V, bias = _small_case(19, with_bias=True)
+    B, H, n, d = Q.shape
+    Bm = _bias_matrix(bias, H, n).astype(np.float32)
+    seq = np.array([40, 23], np.int32)
+    for N, mode in ((0, 0), (7, 0), (0, 1), (12, 1)):
+        a = oracle_mod.attention(Q, K, V, N=N, mode=mode, seqlens=seq, bias=bias, want_idx=N > 0)
+        b = oracle_mod.attention(Q, K, V, N=N, mode=mode, seqlens=seq, bias=oracle_mod.DenseBias(Bm), want_idx=N > 0)
+        np.testing.assert_array_equal(a.O, b.O)
+        if N > 0:
+            np.testing.assert_array_equal(a.idx, b.idx)
+
+
 def test_logit_is_single_rounding_of_scaled_score_plus_bias(oracle_mod):
     rng = _rng(6)
     H, gh, gw = 2, 5, 5
@@ -286,12 +317,16 @@ def _bias_matrix(bias, H, n):
     return Bm
 
 
-@pytest.mark.parametrize("with_bias", [False, True])
+@pytest.mark.parametrize("with_bias", [False, True, "dense"])
 def test_dense_equals_independent_numpy_attention(oracle_mod, with_bias):
-    Q, K, V, bias = _small_case(10 + with_bias, with_bias=with_bias)
+    Q, K, V, bias = _small_case(10 + (with_bias is True), with_bias=with_bias is True)
     B, H, n, d = Q.shape
+    if with_bias == "dense":
+        bias = oracle_mod.DenseBias((_rng(29).standard_normal((H, n, n)) * 0.3).astype(np.float32))
+        Bm = bias.table.astype(np.float64)
+    else:
+        Bm = _bias_matrix(bias, H, n)
     r = oracle_mod.attention(Q, K, V, N=0, bias=bias)
-    Bm = _bias_matrix(bias, H, n)
     for b in range(B):
         for h in range(H):
             mq = np.float32(np.sum(Q[b, h].astype(np.float64), axis=0) / n)

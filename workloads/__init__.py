@@ -46,6 +46,11 @@ class Bias:
 
 
 @dataclass
+class DenseBias:
+    table: np.ndarray      # [H, n, n] fp32: b_ij = table[h, i, j]
+
+
+@dataclass
 class Workload:
     name: str
     B: int
@@ -57,7 +62,7 @@ class Workload:
     K: np.ndarray
     V: np.ndarray
     seqlens: np.ndarray | None
-    bias: Bias | None
+    bias: Bias | DenseBias | None
     passes: list           # list of (N, mode) the workload runs
     seed: int
     recipe: str
@@ -119,6 +124,19 @@ def deit() -> Workload:
                     "Q,K = offset[h,c]~N(0,0.5) + N(0,1); V N(0,1) with 8/768 channels x10; "
                     "relpos bias 27x27/head ~N(0,0.1), prefix 1",
                     extra={"outlier_channels": sorted(int(p) for p in pick)})
+
+
+def deit_dense_bias() -> Workload:
+    """The DeiT workload (same Q, K, V) with a dense bias matrix instead of the
+    relative-position table: one value per query-key pair, [12, 197, 197]
+    ~N(0, 0.1) from seed 101.  Dense, uint8 A x int8 V."""
+    w = deit()
+    rng = np.random.default_rng(101)
+    table = rng.standard_normal((w.H, w.n, w.n), dtype=np.float32) * np.float32(0.1)
+    return Workload("deit_densebias_b64_h12_n197", w.B, w.H, w.n, w.d, w.dtype, w.Q, w.K, w.V, None,
+                    DenseBias(table), [(0, MODE_U8I8)], 101,
+                    w.recipe.replace("relpos bias 27x27/head ~N(0,0.1), prefix 1", "dense bias 197x197/head ~N(0,0.1)"),
+                    extra=w.extra)
 
 
 def bert() -> Workload:
@@ -196,6 +214,8 @@ def by_name(name: str) -> Workload:
         return deit()
     if name == "bert":
         return bert()
+    if name == "deit_dense_bias":
+        return deit_dense_bias()
     if name.startswith("t5_"):
         return t5(int(name[3:]))
     if name == "stress":
