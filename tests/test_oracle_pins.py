@@ -339,6 +339,27 @@ def test_dense_equals_independent_numpy_attention(oracle_mod, with_bias):
             assert np.max(np.abs(r.O[b, h] - ref)) <= 1e-12 * np.max(np.abs(V))
 
 
+@pytest.mark.parametrize("d", [32, 128])
+def test_other_head_dims_equal_independent_numpy_attention(oracle_mod, d):
+    # the oracle's d is any multiple of 32 (the pages' kernel benchmark uses
+    # head dim 128); pinned against the same independent numpy attention
+    rng = _rng(40 + d)
+    B, H, n = 1, 2, 24
+    Q = rng.standard_normal((B, H, n, d)).astype(np.float32)
+    K = rng.standard_normal((B, H, n, d)).astype(np.float32)
+    V = rng.standard_normal((B, H, n, d)).astype(np.float32)
+    r = oracle_mod.attention(Q, K, V, N=0)
+    c = np.float64(np.float32(1.0 / math.sqrt(d)))
+    for h in range(H):
+        mq = np.float32(np.sum(Q[0, h].astype(np.float64), axis=0) / n)
+        mk = np.float32(np.sum(K[0, h].astype(np.float64), axis=0) / n)
+        S = np.where(Q[0, h] < mq, -1.0, 1.0) @ np.where(K[0, h] < mk, -1.0, 1.0).T
+        l = (S * c).astype(np.float32).astype(np.float64)
+        p = np.exp(l - l.max(axis=1, keepdims=True))
+        p /= p.sum(axis=1, keepdims=True)
+        assert np.max(np.abs(r.O[0, h] - p @ V[0, h].astype(np.float64))) <= 1e-12 * np.max(np.abs(V))
+
+
 def test_probabilities_sum_to_one_and_exp_hamming_form(oracle_mod):
     Q, K, V, _ = _small_case(12)
     B, H, n, d = Q.shape
