@@ -167,12 +167,17 @@ def _raise(st, what):
         raise HadError(st, what)
 
 
-def _workspace(nbytes: int, device, workspace):
+def _workspace(nbytes: int, device, workspace, stream=None):
     if workspace is not None:
         if workspace.numel() * workspace.element_size() < nbytes:
             raise ValueError("workspace too small")
         return workspace
-    return torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+    ws = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=device)
+    if stream is not None:
+        # the allocation belongs to the current stream; the kernels run on `stream`,
+        # so the caching allocator must not hand the block out again before they finish
+        ws.record_stream(stream)
+    return ws
 
 
 # ----------------------------------------------------------------------------- entry points
@@ -186,7 +191,7 @@ def had_binarize_pack(X, seqlens=None, mu_in=None, want_mu=True, workspace=None,
     mu = torch.empty((B, H, d), dtype=torch.float32, device=X.device) if want_mu else None
     ws = None
     if mu_in is None:
-        ws = _workspace(lib().had_binarize_pack_workspace_size(ctypes.byref(shp)), X.device, workspace)
+        ws = _workspace(lib().had_binarize_pack_workspace_size(ctypes.byref(shp)), X.device, workspace, stream)
     st = lib().had_binarize_pack(_ptr(X), ctypes.byref(shp), _ptr(mu_in), _ptr(mu), _ptr(bits), _ptr(ws),
                                  0 if ws is None else ws.numel(), _stream(stream))
     _raise(st, "had_binarize_pack")
@@ -228,7 +233,8 @@ def had_attention(Q, K, V, N=0, mode="float", seqlens=None, bias=None, alpha_q=N
     if out is None:
         out = torch.empty((B, H, n, d), dtype=out_dtype or V.dtype, device=Q.device)
     bs = _bias_struct(bias)
-    ws = _workspace(lib().had_attention_workspace_size(ctypes.byref(shp), int(N), m, bs), Q.device, workspace)
+    ws = _workspace(lib().had_attention_workspace_size(ctypes.byref(shp), int(N), m, bs), Q.device, workspace,
+                    stream)
     aq_keep, aq = _alpha(alpha_q, H)
     ak_keep, ak = _alpha(alpha_k, H)
     st = lib().had_attention(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shp), bs, aq, ak, int(N), m, _ptr(out),
@@ -283,7 +289,7 @@ def had_attention_host(Q, K, V, N=0, mode="float", seqlens=None, bias=None, alph
         _raise(HAD_ERR_INVALID, "had_attention_host_workspace_size")
     if workspace is not None:
         _check_dev(workspace)
-    ws = _workspace(need, torch.device("cuda", torch.cuda.current_device()), workspace)
+    ws = _workspace(need, torch.device("cuda", torch.cuda.current_device()), workspace, stream)
     aq_keep, aq = _alpha(alpha_q, H)
     ak_keep, ak = _alpha(alpha_k, H)
     st = lib().had_attention_host(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shp), bs, aq, ak, int(N), m, _ptr(out),
@@ -325,7 +331,7 @@ def had_topn_indices(Q, K, N, seqlens=None, bias=None, alpha_q=None, alpha_k=Non
     shp = make_shape(Q, seqlens)
     bs = _bias_struct(bias)
     ws = _workspace(lib().had_attention_workspace_size(ctypes.byref(shp), int(N), HAD_MODE_FLOAT, bs), Q.device,
-                    workspace)
+                    workspace, stream)
     idx = torch.empty((B, H, n, N), dtype=torch.int32, device=Q.device)
     aq_keep, aq = _alpha(alpha_q, H)
     ak_keep, ak = _alpha(alpha_k, H)
@@ -343,7 +349,7 @@ def had_attention_codes_u8(Q, K, V, row_begin, row_end, N=0, seqlens=None, bias=
     shp = make_shape(Q, seqlens)
     bs = _bias_struct(bias)
     ws = _workspace(lib().had_attention_workspace_size(ctypes.byref(shp), int(N), HAD_MODE_U8I8, bs), Q.device,
-                    workspace)
+                    workspace, stream)
     A = torch.empty((B, H, row_end - row_begin, n), dtype=torch.uint8, device=Q.device)
     aq_keep, aq = _alpha(alpha_q, H)
     ak_keep, ak = _alpha(alpha_k, H)
@@ -358,7 +364,8 @@ def had_quantize_v(V, seqlens=None, workspace=None, stream=None):
     _check_dev(V, seqlens)
     B, H, n, d = V.shape
     shp = make_shape(V, seqlens)
-    ws = _workspace(lib().had_attention_workspace_size(ctypes.byref(shp), 0, HAD_MODE_U8I8, None), V.device, workspace)
+    ws = _workspace(lib().had_attention_workspace_size(ctypes.byref(shp), 0, HAD_MODE_U8I8, None), V.device,
+                    workspace, stream)
     Vq = torch.empty((B, H, n, d), dtype=torch.int8, device=V.device)
     sc = torch.empty((B, H, d), dtype=torch.float32, device=V.device)
     st = lib().had_quantize_v(_ptr(V), ctypes.byref(shp), _ptr(Vq), _ptr(sc), _ptr(ws), ws.numel(), _stream(stream))
