@@ -498,6 +498,9 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
       const float mo = -m * kLog2e;
       const float* lut = reinterpret_cast<const float*>(hist);
       const float* lut_lane = lut + 32 * 32 + lane;  // dense level table: entry for score s at lut_lane[-16 s]
+      // this row's weight table (top-N without a bias): level (64 - s) / 2 at
+      // lut[(32 - s / 2) kM + srow], i.e. byte (32 kM + srow) * 4 - s * 2 kM (s is even)
+      const char* wrow = reinterpret_cast<const char*>(lut + 32 * kM + srow);
       // Passes compiled into this instantiation (the rest are pruned at compile time).
       constexpr bool kHasLevels = SEL != SEL_DENSE;
       constexpr bool kHasNorm = SEL == SEL_DENSE;
@@ -694,7 +697,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
 #pragma unroll
               for (int u = 0; u < 32; ++u) {
                 const int sc = (int)r[32 * cc + u];
-                const float w = lut[(32 - (sc >> 1)) * kM + srow];
+                const float w = *reinterpret_cast<const float*>(wrow - sc * (2 * kM));
                 const bool valid = FULL || 32 * ch + u < nvalid;
                 const bool eq = valid && sc == sF;
                 const bool drop_tie = eq && cut && tie_seen >= rF;
@@ -865,7 +868,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
               for (int u = 0; u < 32; ++u) {
                 const int sc = (int)r[u];
                 const bool valid = u < nv;
-                e[u] = valid ? lut[(32 - (sc >> 1)) * kM + srow] : 0.0f;
+                e[u] = valid ? *reinterpret_cast<const float*>(wrow - sc * (2 * kM)) : 0.0f;
                 eqm |= (valid && sc == sF) ? (1u << u) : 0u;
               }
             } else {
