@@ -179,3 +179,22 @@ def test_dense_bias_matrix_validation(L):
     wd = L.had_attention_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(dense))
     assert wd > wr > 0
     assert wd - L.had_attention_workspace_size(ctypes.byref(shp), 0, 1, None) >= 2 * 3 * 197 * 198 * 4
+
+
+def test_binding_marshals_both_bias_kinds_and_host_arrays(L):
+    import torch
+    import binarized_qk_sparse_b200 as m
+    rel = m.RelPosBias(torch.zeros(3, 27, 27), 14, 14, 1)
+    c = m._bias_c(rel)
+    assert (c.gh, c.gw, c.prefix, c.dense) == (14, 14, 1, 0) and c.table == rel.table.data_ptr()
+    dense = m.DenseBias(torch.zeros(3, 197, 197))
+    c = m._bias_c(dense)
+    assert (c.dense, c.table) == (1, dense.table.data_ptr())
+    Q = torch.zeros(2, 3, 197, 64, dtype=torch.bfloat16)
+    # host workspace sizes come from the host (no device needed); the dense tables are larger
+    wr = m.had_attention_host_workspace_size(Q, 0, "u8i8", None, rel)
+    wd = m.had_attention_host_workspace_size(Q, 0, "u8i8", None, dense)
+    assert 0 < wr < wd
+    # the host entry point takes contiguous CPU tensors only, checked before any call
+    with pytest.raises(ValueError):
+        m.had_attention_host(Q.transpose(2, 3), Q, Q)
