@@ -77,13 +77,17 @@ int hado_channel_mean(const float* X, int B, int H, int n, int d, const int32_t*
   for (int b = 0; b < B; ++b) {
     int L = valid_len(seqlens, b, n);
     if (L < 1 || L > n) return HADO_ERR_ARG;
-    for (int h = 0; h < H; ++h) {
-      const float* Xh = X + ((size_t)b * H + h) * (size_t)n * d;
-      for (int c = 0; c < d; ++c) {
-        double sum = 0.0;
-        for (int i = 0; i < L; ++i) sum += (double)Xh[(size_t)i * d + c];
-        mu[((size_t)b * H + h) * d + c] = (float)(sum / (double)L);
-      }
+  }
+  /* (b, h) pairs are independent; each channel's sum keeps token order. */
+#pragma omp parallel for schedule(static)
+  for (int64_t bh = 0; bh < (int64_t)B * H; ++bh) {
+    int b = (int)(bh / H);
+    int L = valid_len(seqlens, b, n);
+    const float* Xh = X + (size_t)bh * (size_t)n * d;
+    for (int c = 0; c < d; ++c) {
+      double sum = 0.0;
+      for (int i = 0; i < L; ++i) sum += (double)Xh[(size_t)i * d + c];
+      mu[(size_t)bh * d + c] = (float)(sum / (double)L);
     }
   }
   return HADO_OK;
@@ -95,23 +99,22 @@ int hado_sign_pack(const float* X, const float* mu, int B, int H, int n, int d, 
                    uint32_t* bits) {
   if (!X || !mu || !bits || B <= 0 || H <= 0 || n <= 0 || d <= 0 || d % 32 != 0) return HADO_ERR_ARG;
   int W = d / 32;
-  for (int b = 0; b < B; ++b) {
-    int L = valid_len(seqlens, b, n);
-    for (int h = 0; h < H; ++h) {
-      const float* Xh = X + ((size_t)b * H + h) * (size_t)n * d;
-      const float* m = mu + ((size_t)b * H + h) * d;
-      uint32_t* out = bits + ((size_t)b * H + h) * (size_t)n * W;
-      for (int i = 0; i < n; ++i) {
-        for (int w = 0; w < W; ++w) {
-          uint32_t word = 0;
-          if (i < L) {
-            for (int j = 0; j < 32; ++j) {
-              int c = 32 * w + j;
-              if (Xh[(size_t)i * d + c] < m[c]) word |= (uint32_t)1 << j;
-            }
+#pragma omp parallel for schedule(static)
+  for (int64_t bh = 0; bh < (int64_t)B * H; ++bh) {
+    int L = valid_len(seqlens, (int)(bh / H), n);
+    const float* Xh = X + (size_t)bh * (size_t)n * d;
+    const float* m = mu + (size_t)bh * d;
+    uint32_t* out = bits + (size_t)bh * (size_t)n * W;
+    for (int i = 0; i < n; ++i) {
+      for (int w = 0; w < W; ++w) {
+        uint32_t word = 0;
+        if (i < L) {
+          for (int j = 0; j < 32; ++j) {
+            int c = 32 * w + j;
+            if (Xh[(size_t)i * d + c] < m[c]) word |= (uint32_t)1 << j;
           }
-          out[(size_t)i * W + w] = word;
         }
+        out[(size_t)i * W + w] = word;
       }
     }
   }
@@ -158,29 +161,27 @@ int hado_binary_scores(const uint32_t* qbits, const uint32_t* kbits, int B, int 
 /* Per-channel symmetric int8 quantization of V (BinaryAttention §2.4, V bullet). */
 int hado_v_quant(const float* V, int B, int H, int n, int d, const int32_t* seqlens, int8_t* Vq, float* scale) {
   if (!V || !Vq || !scale) return HADO_ERR_ARG;
-  for (int b = 0; b < B; ++b) {
-    int L = valid_len(seqlens, b, n);
-    for (int h = 0; h < H; ++h) {
-      size_t bh = (size_t)b * H + h;
-      const float* Vh = V + bh * (size_t)n * d;
-      for (int c = 0; c < d; ++c) {
-        float amax = 0.0f;
-        for (int i = 0; i < L; ++i) {
-          float a = fabsf(Vh[(size_t)i * d + c]);
-          if (a > amax) amax = a;
+#pragma omp parallel for schedule(static)
+  for (int64_t bh = 0; bh < (int64_t)B * H; ++bh) {
+    int L = valid_len(seqlens, (int)(bh / H), n);
+    const float* Vh = V + (size_t)bh * (size_t)n * d;
+    for (int c = 0; c < d; ++c) {
+      float amax = 0.0f;
+      for (int i = 0; i < L; ++i) {
+        float a = fabsf(Vh[(size_t)i * d + c]);
+        if (a > amax) amax = a;
+      }
+      float s = (amax > 0.0f) ? amax / 127.0f : 1.0f;
+      scale[(size_t)bh * d + c] = s;
+      for (int i = 0; i < n; ++i) {
+        int8_t qv = 0;
+        if (i < L) {
+          float r = rintf(Vh[(size_t)i * d + c] / s);
+          if (r > 127.0f) r = 127.0f;
+          if (r < -127.0f) r = -127.0f;
+          qv = (int8_t)r;
         }
-        float s = (amax > 0.0f) ? amax / 127.0f : 1.0f;
-        scale[bh * d + c] = s;
-        for (int i = 0; i < n; ++i) {
-          int8_t qv = 0;
-          if (i < L) {
-            float r = rintf(Vh[(size_t)i * d + c] / s);
-            if (r > 127.0f) r = 127.0f;
-            if (r < -127.0f) r = -127.0f;
-            qv = (int8_t)r;
-          }
-          Vq[(bh * n + i) * (size_t)d + c] = qv;
-        }
+        Vq[((size_t)bh * n + i) * (size_t)d + c] = qv;
       }
     }
   }

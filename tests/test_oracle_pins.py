@@ -465,3 +465,41 @@ def test_standard_dense_attention(oracle_mod):
             p = np.exp(l - l.max(axis=1, keepdims=True))
             p /= p.sum(axis=1, keepdims=True)
             np.testing.assert_allclose(O[b, h], p @ V[b, h].astype(np.float64), rtol=0, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- rounding ties (constructed)
+
+def test_v_quant_rounds_half_to_even(oracle_mod):
+    """int8 V takes rint (half to even) of V / s: with absmax 127 the scale is
+    exactly 1 (and 0.5 for absmax 63.5), so halves land exactly on ties and a
+    half-away or floor(x + 0.5) rounding would give other codes."""
+    d, n = 64, 12
+    V = np.zeros((1, 1, n, d), np.float32)
+    V[0, 0, :, 0] = [127.0, 0.5, -0.5, 1.5, -1.5, 2.5, -2.5, 3.5, -3.5, 126.5, -126.5, 0.0]
+    V[0, 0, :, 1] = [63.5, 0.25, -0.25, 0.75, -0.75, 1.25, -1.25, 31.75, -31.75, 0.0, 0.0, 0.0]
+    V[0, 0, :, 2:] = 1.0                       # absmax 1: scale 1/127 (no ties asserted there)
+    Vq, sc = oracle_mod.v_quant(V)
+    assert sc[0, 0, 0] == np.float32(1.0) and sc[0, 0, 1] == np.float32(0.5)
+    np.testing.assert_array_equal(Vq[0, 0, :, 0], [127, 0, 0, 2, -2, 2, -2, 4, -4, 126, -126, 0])
+    np.testing.assert_array_equal(Vq[0, 0, :, 1], [127, 0, 0, 2, -2, 2, -2, 64, -64, 0, 0, 0])
+
+
+@pytest.mark.parametrize("L,code", [(6, 43), (30, 9), (102, 3), (510, 1), (2, 128), (10, 26)])
+def test_attention_codes_round_half_up(oracle_mod, L, code):
+    """A_q = floor(255 p + 0.5): a row of L equal logits has p = 1/L, and for
+    L in {6, 30, 102, 510} 255/L is exactly k + 1/2 with k even, where rint
+    (half to even) and floor(255 p) give k, and floor(255 p + 0.5) gives k + 1.
+    Identical Q rows and identical K rows make every score d and every logit equal."""
+    n, d = 512, 64
+    rng = _rng(77)
+    q = rng.standard_normal(d).astype(np.float32)
+    k = rng.standard_normal(d).astype(np.float32)
+    Q = np.broadcast_to(q, (1, 1, n, d)).copy()
+    K = np.broadcast_to(k, (1, 1, n, d)).copy()
+    V = rng.standard_normal((1, 1, n, d)).astype(np.float32)
+    res = oracle_mod.attention(Q, K, V, N=0, mode=1, seqlens=np.array([L], np.int32), want_codes=True,
+                               want_probs=True)
+    A = res.Aq.reshape(n, n)
+    np.testing.assert_array_equal(A[:L, :L], np.full((L, L), code, np.uint8))
+    assert not A[:, L:].any() and not A[L:].any()
+    assert 255.0 / L == code - 0.5
