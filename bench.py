@@ -1,11 +1,13 @@
 """Benchmark of binarized-QK top-N attention (HAD + BinaryAttention) on B200.
 
-Default workload: the DeiT-shaped BinaryAttention configuration (B64 H12 n197
-d64 bf16, relative-position bias 27x27 per head with one class token, dense,
-uint8 A x int8 V).  A "step" is one pass of the whole hot path over one batch:
-channel means + sign/pack of Q and K, int8 V, scores, logits, (top-N),
-softmax, A.V, output.  Metric: queries/s = valid (batch, head, query) rows per
-second over all ranks.
+Default workload: the long-sequence stress configuration with HAD's top-N
+selection (B2 H16 n16384 d64 bf16 -- a 1024x1024 image at 8x8 patches --
+relative-position bias 255x255 per head, top-1920 per query, float softmax and
+A.V), the largest single-GPU configuration of the metric.  Other workloads are
+selected with --workload.  A "step" is one pass of the whole hot path over one
+batch: channel means + sign/pack of Q and K (+ int8 V), bias tables, scores,
+logits, top-N, softmax, A.V, output.  Metric: queries/s = valid (batch, head,
+query) rows per second over all ranks.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
@@ -15,6 +17,11 @@ on the launching stream, with an L2 flush (a 256 MiB write, larger than the
 sides; the reported time is the max over ranks.  The fused kernel's own time
 comes from events recorded between the library's two stages
 (had_attention_prepare / had_attention_prepared) on the same stream.
+
+Roofline of the fused kernel (the method's own definition): the slower of its
+algorithmic HBM bytes at the measured copy bandwidth and its score contraction
+(2 d int8 ops per valid score) at the int8 tensor-pipe peak; the fraction is
+that time over the measured kernel time.
 """
 from __future__ import annotations
 
@@ -80,8 +87,32 @@ def launches_per_step(n: int, elem: int, mode: str, has_bias: bool, dense_bias: 
 
 
 # Issue-limited CUDA-core rate of one B200: 148 SMs x 4 schedulers x 32 lanes x
-# 1965 MHz (clocks.max.sm), one lane-operation per lane per clock.
+# 1965 MHz (clocks.max.sm), one lane-operation per lane per clock.  A derived
+# ceiling for the diagnostic ALU roofline, not a measured peak.
 ALU_PEAK_TOPS = 148 * 4 * 32 * 1.965e9 / 1e12
+
+# tensor-pipe dense rates relative to bf16 (the nominal 4.5 / 2.25 PFLOP/s of int8 / bf16)
+INT8_PER_BF16 = 2.0
+
+
+def score_tensor_ops(valid_scores: int, d: int = 64) -> float:
+    """Operations of the score contraction on the tensor pipe: one d-element
+    +-1 int8 dot product per valid (query, key) pair = 2 d ops."""
+    return 2.0 * d * valid_scores
+
+
+def north_star_roofline(kbytes: float, tensor_ops: float, kernel_ms: float, hbm_gbs: float, i8_tops: float) -> dict:
+    """The fused kernel's roofline as the method defines it: the slower of its
+    algorithmic HBM bytes at the measured bandwidth and its score contraction at
+    the int8 tensor-pipe peak.  frac = that time / the measured kernel time."""
+    t_hbm = kbytes / (hbm_gbs * 1e9)
+    t_tc = tensor_ops / (i8_tops * 1e12)
+    t = kernel_ms * 1e-3
+    if t_tc >= t_hbm:
+        return {"bound": "tensor", "achieved": tensor_ops / t / 1e12, "peak": i8_tops, "unit": "TOPS (int8)",
+                "frac": t_tc / t, "t_roof_ms": t_tc * 1e3, "t_hbm_ms": t_hbm * 1e3, "t_tensor_ms": t_tc * 1e3}
+    return {"bound": "hbm", "achieved": kbytes / t / 1e9, "peak": hbm_gbs, "unit": "GB/s", "frac": t_hbm / t,
+            "t_roof_ms": t_hbm * 1e3, "t_hbm_ms": t_hbm * 1e3, "t_tensor_ms": t_tc * 1e3}
 
 
 def alu_ops_per_score(mode: str, N: int, n: int, has_bias: bool) -> float:
@@ -150,13 +181,16 @@ def whole_job_rate(units_per_rank: float, world: int, steps: int, total_ms: floa
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi sampling of SM clocks and throttle reasons; only the samples
+    whose timestamps fall inside the timed region are summarized."""
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, period_ms: int = 20):
         self.gpu = gpu_index
+        self.period = period_ms
         self.proc = None
         self.path = None
 
@@ -166,12 +200,24 @@ class ClockSampler:
             fd, self.path = tempfile.mkstemp(prefix="clk", suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", str(self.period)],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
-    def stop(self):
+    @staticmethod
+    def _stamp(txt):
+        import datetime
+        for fmt in ("%Y/%m/%d %H:%M:%S.%f", "%Y/%m/%d %H:%M:%S"):
+            try:
+                return datetime.datetime.strptime(txt.strip(), fmt).timestamp()
+            except ValueError:
+                pass
+        return None
+
+    def stop(self, t0=None, t1=None):
+        """Stop sampling; summarize the samples taken in [t0, t1] (wall-clock
+        seconds since the epoch), or all of them without a window."""
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -179,19 +225,22 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        sm, smax, reasons, n_all = [], None, set(), 0
         try:
             for line in open(self.path):
                 f = [x.strip() for x in line.split(",")]
-                if len(f) < 9:
+                if len(f) < 10:
+                    continue
+                n_all += 1
+                ts = self._stamp(f[0])
+                if t0 is not None and (ts is None or ts < t0 or ts > t1):
                     continue
                 try:
-                    sm.append(float(f[1]))
-                    smax = float(f[2])
+                    sm.append(float(f[2]))
+                    smax = float(f[3])
                 except ValueError:
                     continue
-                for k, v in zip(names, f[5:9]):
+                for k, v in zip(self.NAMES, f[6:10]):
                     if v.lower().startswith("active"):
                         reasons.add(k)
             os.unlink(self.path)
@@ -201,10 +250,10 @@ class ClockSampler:
             return None
         loaded = [x for x in sm if smax is None or x > 0.5 * smax] or sm
         return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": smax, "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "period_ms": self.period}
 
 
-# ----------------------------------------------------------------------------- reference arm (the oracle)
+# ----------------------------------------------------------------------------- the oracle on the host cores
 
 def _oracle_bias(oracle, w):
     if w.bias is None:
@@ -222,12 +271,14 @@ def _bias_desc(w):
     return f"relpos {w.bias.table.shape[1]}x{w.bias.table.shape[2]}/head, prefix {w.bias.prefix}"
 
 
-def _oracle_rows_per_sec(w, N, mode, rows):
+def _oracle_call_s(w, N, mode, rows):
+    """Seconds of one oracle call over the given query rows (plus its whole-workload
+    prelude: channel means, sign bits and int8 V of every head)."""
     import oracle
     b = _oracle_bias(oracle, w)
     t0 = time.perf_counter()
     oracle.attention(w.Q, w.K, w.V, N=N, mode=1 if mode == "u8i8" else 0, seqlens=w.seqlens, bias=b, rows=rows)
-    return len(rows) / (time.perf_counter() - t0)
+    return time.perf_counter() - t0
 
 
 def _valid_rows(w):
@@ -238,21 +289,45 @@ def _valid_rows(w):
     return np.concatenate(rows)
 
 
-def cpu_baseline(w, N, mode, budget_s=15.0):
-    """The oracle as it stands, on the host cores, on a bounded seeded sample of the workload's rows."""
-    import oracle
+def oracle_rate(prelude_s: float, row_s: float, total_rows: int) -> float:
+    """Whole-workload oracle rate from its two measured parts: the prelude (run
+    once per workload) and the per-row time (the slope over sampled rows)."""
+    return total_rows / (prelude_s + row_s * total_rows)
+
+
+def _oracle_parts(w, N, mode, budget_s, seed):
+    """Prelude seconds (a call with no rows) and per-row seconds (slope between
+    two seeded samples of m and 2m rows), with m sized to the budget."""
     allrows = _valid_rows(w)
-    rng = np.random.default_rng(99)
-    probe = np.sort(rng.choice(allrows, size=min(len(allrows), 64), replace=False))
-    rate = _oracle_rows_per_sec(w, N, mode, probe)
-    want = int(min(len(allrows), max(64, rate * budget_s)))
-    rows = np.sort(rng.choice(allrows, size=want, replace=False)) if want < len(allrows) else allrows
-    rate = _oracle_rows_per_sec(w, N, mode, rows)
-    return {"value": rate, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{len(rows)} of {len(allrows)} query rows of {w.name} (seeded), full per-head means/scales"}
+    rng = np.random.default_rng(seed)
+    pre = min(_oracle_call_s(w, N, mode, np.zeros(0, np.int64)) for _ in range(2))
+    probe = np.sort(rng.choice(allrows, size=min(len(allrows), 256), replace=False))
+    t = _oracle_call_s(w, N, mode, probe)
+    per_row = max(t - pre, 1e-9) / len(probe)
+    m = int(max(256, min(len(allrows) // 2, (budget_s / 3.0) / per_row)))
+    r1 = np.sort(rng.choice(allrows, size=m, replace=False))
+    r2 = np.sort(rng.choice(allrows, size=min(len(allrows), 2 * m), replace=False))
+    t1, t2 = _oracle_call_s(w, N, mode, r1), _oracle_call_s(w, N, mode, r2)
+    per_row = max((t1 + t2 - 2.0 * pre) / (len(r1) + len(r2)), 1e-12)
+    return pre, per_row, (len(r1), len(r2)), len(allrows)
+
+
+def cpu_baseline(w, N, mode, budget_s=15.0):
+    """The oracle as it stands, on the host cores: whole-workload queries/s from
+    its prelude time and its per-row time over a bounded seeded sample."""
+    import oracle
+    pre, per_row, sampled, total = _oracle_parts(w, N, mode, budget_s, 99)
+    return {"value": oracle_rate(pre, per_row, total), "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"two seeded samples of {sampled[0]} and {sampled[1]} of the {total} query rows of {w.name}; "
+                      f"prelude (means, "
+                      f"sign bits, int8 V of every head) {pre:.3f} s once, {per_row * 1e3:.4f} ms per row; "
+                      f"value extrapolated to all {total} rows"}
 
 
 def run_reference(args, rank, world):
+    """The reference arm: the oracle as it stands on the host cores.  Each step runs
+    the oracle's prelude and a bounded seeded sample of rows; the value is the
+    whole-workload rate from the prelude time and the per-row slope."""
     if rank != 0:
         return 0
     import oracle
@@ -260,38 +335,38 @@ def run_reference(args, rank, world):
     w = workloads.by_name(name)
     allrows = _valid_rows(w)
     rng = np.random.default_rng(7)
-    probe = np.sort(rng.choice(allrows, size=min(len(allrows), 64), replace=False))
-    rate = _oracle_rows_per_sec(w, N, mode, probe)
+    pre = min(_oracle_call_s(w, N, mode, np.zeros(0, np.int64)) for _ in range(2))
+    probe = np.sort(rng.choice(allrows, size=min(len(allrows), 256), replace=False))
+    per_row = max(_oracle_call_s(w, N, mode, probe) - pre, 1e-9) / len(probe)
     budget = 90.0 / max(1, args.steps + args.warmup)
-    per_step = int(max(1, min(len(allrows), rate * budget)))
+    per_step = int(max(64, min(len(allrows), (budget - pre) / per_row)))
     times = []
     for s in range(args.warmup + args.steps):
         rows = np.sort(rng.choice(allrows, size=per_step, replace=False))
-        t0 = time.perf_counter()
-        _oracle_rows_per_sec(w, N, mode, rows)
-        dt = time.perf_counter() - t0
+        dt = _oracle_call_s(w, N, mode, rows)
         if s >= args.warmup:
             times.append(dt)
-    total = sum(times)
-    value = per_step * len(times) / total
+    per_row = max((sum(times) - len(times) * pre) / (len(times) * per_step), 1e-12)
+    value = oracle_rate(pre, per_row, len(allrows))
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / len(times),
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * sum(times) / len(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": _config(w, N, mode),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-                             "sample": f"{per_step} seeded query rows of {w.name} per step"},
+                             "sample": f"{per_step} seeded query rows of {w.name} per step (+ the prelude); "
+                                       f"prelude {pre:.3f} s, {per_row * 1e3:.4f} ms per row; value extrapolated "
+                                       f"to all {len(allrows)} rows"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
 def _config(w, N, mode):
-    c = {"workload": f"{w.name}_{'dense' if N == 0 else f'top{N}'}_{mode}", "B": w.B, "H": w.H, "n": w.n, "d": w.d,
-         "N": N, "mode": mode, "in_dtype": w.dtype, "seed": w.seed,
-         "bias": _bias_desc(w),
-         "seqlens": None if w.seqlens is None else "U{32..256} per sequence",
-         "l2": "flushed between timed steps (256 MiB write)"}
-    return c
+    return {"workload": f"{w.name}_{'dense' if N == 0 else f'top{N}'}_{mode}", "B": w.B, "H": w.H, "n": w.n,
+            "d": w.d, "N": N, "mode": mode, "in_dtype": w.dtype, "seed": w.seed,
+            "bias": _bias_desc(w),
+            "seqlens": None if w.seqlens is None else "U{32..256} per sequence",
+            "l2": "flushed between timed steps (256 MiB write)"}
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -346,8 +421,14 @@ def run_gpu(args, rank, world, local_rank):
         if st:
             raise had.HadError(st, "had_attention_prepared")
 
+    # the tensor pipe's int8 and bf16 MMA rates on this GPU (probe kernel, before the workload)
+    probe_i8, _ = had.had_probe_mma_rate("i8", 200000)
+    probe_bf16, _ = had.had_probe_mma_rate("bf16", 100000)
+
     kernels_per_step = launches_per_step(w.n, Q.element_size(), mode, bias is not None,
                                          isinstance(w.bias, workloads.DenseBias))
+    clocks = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    clocks.start()  # nvidia-smi takes a moment to start: launched before the warm-up
     with torch.cuda.stream(stream):
         for _ in range(max(3, args.warmup)):
             prepare()
@@ -357,12 +438,10 @@ def run_gpu(args, rank, world, local_rank):
 
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
                torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
-        clocks = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
         if dist is not None:
             dist.barrier()
         torch.cuda.synchronize()
-        clocks.start()
-        wall0 = time.perf_counter()
+        wall0 = time.time()
         for s in range(args.steps):
             flush.zero_()
             ev[s][0].record(stream)
@@ -371,10 +450,10 @@ def run_gpu(args, rank, world, local_rank):
             attend()
             ev[s][2].record(stream)
         torch.cuda.synchronize()
-        wall = time.perf_counter() - wall0
-        clk = clocks.stop()
+        wall1 = time.time()
         if dist is not None:
             dist.barrier()
+    clk = clocks.stop(wall0, wall1)
     step_ms = [e[0].elapsed_time(e[2]) for e in ev]
     attn_ms = [e[1].elapsed_time(e[2]) for e in ev]
     total_ms = max_over_ranks(sum(step_ms), dist, dev)
@@ -395,7 +474,7 @@ def run_gpu(args, rank, world, local_rank):
         hbias = had.RelPosBias(bias.table.cpu().pin_memory(), bias.gh, bias.gw, bias.prefix)
     host_ws = torch.empty(had.had_attention_host_workspace_size(hQ, N, mode, hseq, hbias), dtype=torch.uint8,
                           device=dev)
-    e2e_steps = min(args.steps, 30)
+    e2e_steps = max(3, min(args.steps, 30))
     h2d = 3 * Q.numel() * Q.element_size() + (0 if hseq is None else hseq.numel() * 4) + \
         (0 if hbias is None else hbias.table.numel() * 4)
     d2h = O.numel() * O.element_size()
@@ -417,39 +496,46 @@ def run_gpu(args, rank, world, local_rank):
     kbytes = kernel_bytes_per_token(mode, 2 if bf16 else 4, O.element_size()) * queries
     if bias is not None:
         kbytes += w.bias.table.nbytes
-    achieved = kbytes / (attn_avg_ms * 1e-3) / 1e9
-    ops_per_score = alu_ops_per_score(mode, N, w.n, bias is not None)
-    alu_ops = ops_per_score * w.valid_scores()
-    alu_achieved = alu_ops / (attn_avg_ms * 1e-3) / 1e12
-    pbytes = path_bytes_per_token(mode, 2 if bf16 else 4, O.element_size()) * queries
-    path_achieved = pbytes / (ms_per_step * 1e-3) / 1e9
+    tc_ops = score_tensor_ops(w.valid_scores(), w.d)
+    i8_recipe = INT8_PER_BF16 * peaks["bf16_tflops"]
+    i8_peak = max(i8_recipe, probe_i8)
+    roof = north_star_roofline(kbytes, tc_ops, attn_avg_ms, peaks["hbm_gbs"], i8_peak)
     traffic = None
     tr_path = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tr_path):
         with open(tr_path) as f:
             traffic = json.load(f).get(args.workload)
+    roof.update({"traffic": traffic, "kernel": "k_attn_tc (fused score/top-N/softmax/A.V)",
+                 "avg_launch_ms": attn_avg_ms, "algorithmic_bytes_per_launch": kbytes,
+                 "tensor_ops_per_launch": tc_ops,
+                 "peak_kind": (f"int8 = max({INT8_PER_BF16:g} x {peak_kind} bf16 burst {peaks['bf16_tflops']} "
+                               f"TFLOP/s, probe {probe_i8:.0f} TOPS); HBM {peak_kind} {peaks['hbm_gbs']} GB/s")})
+    ops_per_score = alu_ops_per_score(mode, N, w.n, bias is not None)
+    alu_ops = ops_per_score * w.valid_scores()
+    alu_achieved = alu_ops / (attn_avg_ms * 1e-3) / 1e12
+    pbytes = path_bytes_per_token(mode, 2 if bf16 else 4, O.element_size()) * queries
+    path_achieved = pbytes / (ms_per_step * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "u8i8" if mode == "u8i8" else ("bf16" if bf16 else "f32"),
-        "data": "synthetic", "config": {**_config(w, N, mode), "parallelism": f"replicas x{world} (no collective)"},
+        "data": "synthetic", "config": _config(w, N, mode),
+        "parallelism": f"replicas x{world} (no collective)",
         "score_ops_per_s": whole_job_rate(w.valid_scores(), world, args.steps, total_ms),
-        "roofline": {"bound": "alu", "kernel": "k_attn_tc (fused score/top-N/softmax/A.V)",
-                     "achieved": alu_achieved, "peak": ALU_PEAK_TOPS, "unit": "Tlane-op/s",
-                     "frac": alu_achieved / ALU_PEAK_TOPS, "traffic": traffic,
-                     "algorithmic_ops_per_launch": alu_ops, "ops_per_valid_score": ops_per_score,
-                     "avg_launch_ms": attn_avg_ms,
-                     "peak_kind": "derived: 148 SMs x 4 schedulers x 32 lanes x 1965 MHz"},
-        "roofline_hbm": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / peaks["hbm_gbs"], "algorithmic_bytes_per_launch": kbytes,
-                         "peak_kind": peak_kind},
+        "roofline": roof,
+        "tensor_pipe_probe": {"i8_tops": probe_i8, "bf16_tflops": probe_bf16,
+                              "kernel": "k_probe_mma: M128 N256 tcgen05.mma back to back, operands in shared memory"},
+        "roofline_alu": {"bound": "alu", "achieved": alu_achieved, "peak": ALU_PEAK_TOPS, "unit": "Tlane-op/s",
+                         "frac": alu_achieved / ALU_PEAK_TOPS, "ops_per_valid_score": ops_per_score,
+                         "peak_kind": "derived issue ceiling: 148 SMs x 4 schedulers x 32 lanes x 1965 MHz; "
+                                      "ops per score are this library's own count (diagnostic)"},
         "roofline_path": {"bound": "hbm", "achieved": path_achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                           "frac": path_achieved / peaks["hbm_gbs"], "algorithmic_bytes_per_step": pbytes},
         "e2e": {"value": whole_job_rate(queries, world, 1, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
         "gpu_launches": kernels_per_step * args.steps,
         "clocks": clk,
-        "wall_s_timed_loop": wall,
+        "timed_region_s": wall1 - wall0,
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, N, mode)
@@ -460,9 +546,9 @@ def run_gpu(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="deit", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="stress_topn", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

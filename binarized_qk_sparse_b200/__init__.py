@@ -100,6 +100,12 @@ def lib():
                   "had_dense_reference_mode", "had_scores_int",
                   "had_topn_indices", "had_attention_codes_u8", "had_quantize_v", "had_get_device_status"):
             getattr(L, f).restype = I
+        L.had_attention_scores.argtypes = [P, P, SP, P, P, SZ, P]
+        L.had_attention_scores.restype = I
+        L.had_debug_bounded_wait.argtypes = [ctypes.c_longlong, I]
+        L.had_debug_bounded_wait.restype = I
+        L.had_probe_mma_rate.argtypes = [I, I, P, P]
+        L.had_probe_mma_rate.restype = I
         L.had_get_device_status.argtypes = []
         L.had_status_string.argtypes = [I]
         L.had_status_string.restype = ctypes.c_char_p
@@ -211,8 +217,12 @@ def had_binarize_pack_noalloc(X, seqlens=None, bits=None, mu=None, stream=None):
     shp = make_shape(X, seqlens)
     if bits is None:
         bits = torch.empty((B, H, n, d // 32), dtype=torch.int32, device=X.device)
+    elif bits.shape != (B, H, n, d // 32) or bits.dtype not in (torch.int32, torch.uint32) or bits.device != X.device:
+        raise ValueError(f"bits must be int32 [{B}, {H}, {n}, {d // 32}] on {X.device}")
     if mu is None:
         mu = torch.empty((B, H, d), dtype=torch.float32, device=X.device)
+    elif mu.shape != (B, H, d) or mu.dtype != torch.float32 or mu.device != X.device:
+        raise ValueError(f"mu must be float32 [{B}, {H}, {d}] on {X.device}")
     st = lib().had_binarize_pack_noalloc(_ptr(X), ctypes.byref(shp), _ptr(mu), _ptr(bits), _stream(stream))
     _raise(st, "had_binarize_pack_noalloc")
     return bits, mu
@@ -324,6 +334,25 @@ def had_scores_int(qbits, kbits, seqlens=None, d=64, stream=None):
     return S
 
 
+def had_attention_scores(Q, K, seqlens=None, workspace=None, stream=None):
+    """Integer scores [B,H,n,n] int32 as the fused kernel forms them in tensor memory."""
+    _check_dev(Q, K, seqlens)
+    B, H, n, d = Q.shape
+    shp = make_shape(Q, seqlens)
+    ws = _workspace(lib().had_attention_workspace_size(ctypes.byref(shp), 0, HAD_MODE_FLOAT, None), Q.device,
+                    workspace, stream)
+    S = torch.empty((B, H, n, n), dtype=torch.int32, device=Q.device)
+    st = lib().had_attention_scores(_ptr(Q), _ptr(K), ctypes.byref(shp), _ptr(S), _ptr(ws), ws.numel(),
+                                    _stream(stream))
+    _raise(st, "had_attention_scores")
+    return S
+
+
+def had_debug_bounded_wait(max_cycles=0, force_expiry=False):
+    """Test hook of the fused kernel's timeout path (see include/had.h)."""
+    _raise(lib().had_debug_bounded_wait(int(max_cycles), 1 if force_expiry else 0), "had_debug_bounded_wait")
+
+
 def had_topn_indices(Q, K, N, seqlens=None, bias=None, alpha_q=None, alpha_k=None, workspace=None, stream=None):
     """Kept key indices per query, ascending, -1 padded: [B,H,n,N] int32."""
     _check_dev(Q, K, seqlens)
@@ -376,6 +405,17 @@ def had_quantize_v(V, seqlens=None, workspace=None, stream=None):
 def had_get_device_status() -> int:
     """Synchronize, read and clear the device status word (HAD_OK, HAD_ERR_DEVICE or HAD_ERR_TIMEOUT)."""
     return int(lib().had_get_device_status())
+
+
+def had_probe_mma_rate(kind="i8", iters=200000):
+    """Tensor-pipe rate of tcgen05.mma on this GPU: (10^12 ops/s, elapsed ms).
+
+    kind "i8": kind::i8 (the +-1 score contraction); "bf16": kind::f16 with bf16
+    operands.  Synchronizes the device."""
+    k = {"i8": 0, "bf16": 1}[kind]
+    tops, ms = ctypes.c_double(0.0), ctypes.c_double(0.0)
+    _raise(lib().had_probe_mma_rate(k, int(iters), ctypes.byref(tops), ctypes.byref(ms)), "had_probe_mma_rate")
+    return tops.value, ms.value
 
 
 def had_version() -> int:

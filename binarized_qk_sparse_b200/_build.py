@@ -9,7 +9,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhad_b200.so")
 SOURCES = ["had_lib.cu"]
-DEPS = ["common.cuh", "sm100.cuh", "prep.cuh", "attn.cuh", "attn_tc.cuh", "dense_ref.cuh", "had_lib.cu"]
+DEPS = ["common.cuh", "sm100.cuh", "prep.cuh", "attn.cuh", "attn_tc.cuh", "dense_ref.cuh", "probe.cuh", "had_lib.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

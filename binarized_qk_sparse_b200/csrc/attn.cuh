@@ -58,9 +58,11 @@ __device__ __forceinline__ int key_of(int nb, int col) {
 
 namespace had {
 
-// Debug export of the integer scores through the same +-1 int8 tensor-core
-// fragments as k_attn: S[i][j] = q~_i . k~_j = d - 2*popcount(q XOR k) for
-// i, j < L, 0 elsewhere.  The K~ tile is expanded from packed bits in smem.
+// Debug export of the integer scores from packed bits, on legacy mma.sync
+// m16n8k32 s8 fragments (a kernel of its own, independent of k_attn_tc, whose
+// scores the EXP_SCORES export reads from tensor memory):
+// S[i][j] = q~_i . k~_j = d - 2*popcount(q XOR k) for i, j < L, 0 elsewhere.
+// The K~ tile is expanded from packed bits in smem.
 template <int MODE>
 __global__ void __launch_bounds__(kAttnThreads) k_scores_int(const uint32_t* __restrict__ qbits,
                                                              const uint32_t* __restrict__ kbits, int H, int n,

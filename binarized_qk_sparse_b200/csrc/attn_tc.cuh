@@ -64,7 +64,15 @@ constexpr int kRadixBins = 256;   // 16-bit counters, two per word (a row counts
 constexpr int kCandCap = 128;    // power of two (the collect slot wraps)
 constexpr int kSBufs = 3;
 constexpr uint32_t kColS = 0, kColO = 192, kTmemCols = 256;
-constexpr long long kWaitCycles = 2000000000LL;  // about one second
+constexpr long long kWaitCycles = 2000000000LL;  // default bound of a pipeline wait: about one second
+// First select pass of top-N with a bias (FBIN): u = min(fmaf(l, sc, off), kFbTop)
+// is a monotone function of the logit l; with u in [kFbMg, kFbMg + 65536) its
+// float bits carry the integer u - kFbMg in their low 16 bits, and bits 9..15 are
+// the bin (128 bins of 512 units): bin 0 holds everything below the window, bins
+// 1..126 the window, bin 127 (the clamp) only keys above it.
+constexpr float kFbMg = 12582912.0f;             // 1.5 * 2^23: unit spacing, bits 0x4B400000
+constexpr float kFbIn = kFbMg + 512.0f;          // first in-window bin
+constexpr float kFbTop = kFbMg + 127.0f * 512.0f;  // bin 127
 // How the softmax threads find the bias offset koff(j) = y_j * S + x_j of a key (S: table row stride):
 constexpr int kKoffTable = 0;  // per-head table in shared memory (n_pad <= kKoffTableMax)
 constexpr int kKoffWarp = 1;   // each softmax warp computes the tile's 64 offsets (double-buffered)
@@ -72,13 +80,20 @@ constexpr int kKoffTableMax = 1024;
 // Bias variants of the kernel: none, extended tables read from global memory,
 // (dense weights) the exp(bias) table staged in shared memory, or (dense
 // weights) a dense bias matrix's exp(bias) rows read 4 keys per 16-byte load.
-enum { BIAS_NONE = 0, BIAS_GLOBAL = 1, BIAS_SMEM = 2, BIAS_DGLOBAL = 3 };
+enum { BIAS_NONE = 0, BIAS_GLOBAL = 1, BIAS_SMEM = 2, BIAS_DGLOBAL = 3, BIAS_ROWS = 4 };
+// BIAS_ROWS (a relative-position table with no class tokens on a grid whose rows
+// hold a multiple of 64 patches): a warp's 32 query rows lie in one image row and
+// a 64-key tile in another, so the bias of the pair (warp, tile) is 96 consecutive
+// entries of one table row.  Each softmax warp copies that window into its own
+// shared-memory slice (prefetched into registers one tile ahead), and a score's
+// bias is then one shared load at a compile-time offset from a per-thread base.
+constexpr int kRowWin = 96;  // entries of a warp's bias window (32 rows + 64 keys - 1, padded)
 constexpr int kBiasSmemMax = kBiasSmemEntries;
 
 enum { SEL_DENSE = 0, SEL_TOPN_INT = 1, SEL_TOPN_FLOAT = 2 };
 enum { MODE_F = 0, MODE_Q = 1 };
-enum { EXP_NONE = 0, EXP_IDX = 1, EXP_CODES = 2 };
-enum { P_DONE = 0, P_NORM, P_LEVELS, P_RADIX, P_COLLECT, P_KEPT_NORM, P_PV, P_IDX, P_CODES };
+enum { EXP_NONE = 0, EXP_IDX = 1, EXP_CODES = 2, EXP_SCORES = 3 };
+enum { P_DONE = 0, P_NORM, P_LEVELS, P_FBIN, P_RADIX, P_COLLECT, P_KEPT_NORM, P_PV, P_IDX, P_CODES, P_SCORES };
 
 struct TcArgs {
   CUtensorMap tm_k;   // +-1 int8 K [BH*n_pad][64], box {64, 64}, 64B swizzle
@@ -106,7 +121,10 @@ struct TcArgs {
   uint8_t* codes;
   int row_begin, row_end;
   int B, H, n, n_pad, N;
+  int32_t* scores;         // EXP_SCORES: [BH][n][n] int32
   unsigned* status;
+  long long wait_cycles;   // bound of every pipeline wait, in SM clocks
+  int force_expiry;        // test hook: one softmax thread first waits on a barrier nothing completes
   float c_head[kMaxHeads];
 };
 
@@ -124,7 +142,7 @@ struct Smem {
   static constexpr int kXchg = kBiasTab + (BIAS == BIAS_SMEM ? kBiasSmemMax * 4 : 0);
   static constexpr int kDq = kXchg + (SEL == SEL_DENSE ? 2 : SEL == SEL_TOPN_INT ? 10 : 0) * kM * 4;  // 64 dequant scales
   static constexpr int kBar = kDq + kD * 4;
-  static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 2 * kSBufs + 3;
+  static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 2 * kSBufs + 4;
   static constexpr int kMisc = kBar + kNumBars * 8;              // [0] tmem base [1] abort
   static constexpr int kHist = (kMisc + 16 + 127) / 128 * 128;
   static constexpr int kHistBytes = (SEL == SEL_DENSE) ? kLevels * 32 * 4
@@ -145,7 +163,8 @@ enum {
   B_TDONE = B_SFULL + kSBufs,             // one per score buffer
   B_OFULL = B_TDONE + kSBufs,
   B_FINAL,
-  B_BIAS  // staged exp(bias) table landed
+  B_BIAS,  // staged exp(bias) table landed
+  B_STALL  // never completed: the force_expiry test hook waits on it
 };
 
 // Bias offset of key j: koff = y_j * S + x_j for patch tokens, so that
@@ -192,6 +211,8 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
                 "two threads per row: dense, or top-N without a bias on its P.V path");
   static_assert((BIAS != BIAS_SMEM && BIAS != BIAS_DGLOBAL) || SEL == SEL_DENSE,
                 "staged or vector-read exp(bias) tables serve the dense weights only");
+  static_assert(BIAS != BIAS_ROWS || (SEL != SEL_TOPN_INT && 2 * (SPLIT == 2 ? 8 * 64 : 4 * kRowWin) <= kKoffTableMax),
+                "the warps' bias-window slices fit the key-offset area");
   constexpr int kSplit = SPLIT;
   constexpr int kSoftWarps = 4 * kSplit;
   constexpr int kThreads = cta_threads(SPLIT);
@@ -244,6 +265,11 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
         const int r = q0 + e / a.N;
         if (r < a.n) a.idx[((size_t)bh * a.n + r) * a.N + e % a.N] = -1;
       }
+    } else if (EXPORT == EXP_SCORES) {
+      for (int e = tid; e < kM * a.n; e += kThreads) {
+        const int r = q0 + e / a.n;
+        if (r < a.n) a.scores[((size_t)bh * a.n + r) * a.n + e % a.n] = 0;
+      }
     } else {
       const int rows = a.row_end - a.row_begin;
       for (int e = tid; e < kM * a.n; e += kThreads) {
@@ -275,6 +301,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
     mbar_init(&bars[B_OFULL], 1);
     mbar_init(&bars[B_FINAL], 1);
     mbar_init(&bars[B_BIAS], 1);
+    mbar_init(&bars[B_STALL], 1);
     misc[1] = 0;
     fence_barrier_init();
     if (BIAS == BIAS_SMEM) {
@@ -323,7 +350,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
       }
     }
     if (MODE == MODE_Q && EXPORT == EXP_NONE && tid < kD) dq[tid] = __fdiv_rn(a.vscale[(size_t)bh * kD + tid], 255.0f);
-    if (HAS_BIAS && a.koff_mode == kKoffTable)
+    if (HAS_BIAS && BIAS != BIAS_ROWS && a.koff_mode == kKoffTable)
       for (int j = tid; j < a.n_pad; j += kM) koff_tab[j] = 4 * key_offset(a, j, L);  // in bytes
     fence_proxy_async();
   }
@@ -337,9 +364,10 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
   int rF = 0, cut = 0, tie_seen = 0, kept_seen = 0;
   uint32_t r_uhi = 0, r_span = 0;
   // r_state: 0 threshold known, 1 radix pass next, 2 collect pass next, 3 the
-  // window's keys are recorded during the P.V pass (kMerge)
+  // window's keys are recorded during the P.V pass (kMerge), 4 FBIN pass next
   int r_shift = 0, r_rank = 0, r_state = 0, r_cnt = 0;
   int r_above = 0;      // keys above the first radix window (counted in that pass)
+  float fb_sc = 0.0f, fb_off = 0.0f;  // r_state 4: the FBIN pass's map of logits onto bins
   // float window of the P.V pass: weight for l >= w_cut; keys in [w_lo, w_hi] are
   // the ties at F (w_lo = w_hi = w_cut = F), or, with the collect folded into
   // the P.V pass, the final radix bin (w_cut just above w_hi), ranked after it
@@ -371,17 +399,20 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
 
   uint32_t g_k = 0, g_v = 0, g_s = 0;  // tiles issued so far (all passes), per role
 
-  int pass = (SEL == SEL_DENSE) ? (EXPORT == EXP_IDX ? P_IDX : P_NORM) : P_LEVELS;
+  int pass = (SEL == SEL_DENSE) ? (EXPORT == EXP_IDX ? P_IDX : EXPORT == EXP_SCORES ? P_SCORES : P_NORM) : P_LEVELS;
   if (SEL == SEL_DENSE && EXPORT == EXP_NONE && MODE == MODE_F && use_lut) pass = P_PV;
 
   auto bounded_wait = [&](int bar, uint32_t parity) -> bool {
     if (mbar_test_wait(smem_u32(&bars[bar]), parity)) return true;  // phase already complete
     if (*abort_flag) return false;
-    if (mbar_wait(&bars[bar], parity, kWaitCycles)) return true;
+    if (mbar_wait(&bars[bar], parity, a.wait_cycles)) return true;
     *abort_flag = 1u;
     raise_status(a.status, kDevErrTimeout);
     return false;
   };
+  // test hook of the timeout path: one softmax thread first waits on a barrier
+  // that nothing completes, so its bound expires and the CTA winds down
+  if (a.force_expiry && tid == 0) bounded_wait(B_STALL, 0);
 
   // K tiles of a short key range stay in the K stages for every pass (loaded once)
   const bool k_res = ntiles <= kKStages;
@@ -540,6 +571,33 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
         if (a.bias_dense) return 4 * (j >= L ? a.k_invalid : -j);
         return 4 * (j >= L ? a.k_invalid : (j < a.prefix ? a.k_class : y * a.ext_S + x));
       };
+      // BIAS_ROWS: this warp's 32 rows (one image row) and its two window slices.
+      // Entry e of the window of tile t is table[y_w - y_k + gh - 1][x_w - x_k + gw - 64 + e]
+      // (x_k, y_k of the tile's first key): row (lane) and key u of the tile read entry
+      // lane + 63 - u.  One thread per row reads entries 0..94; with two threads per row
+      // each warp takes 32 keys and needs 63 entries starting at 32 (keys 0..31) or 0.
+      constexpr int kRwEnt = kSplit == 2 ? 64 : kRowWin;  // entries per slice (32 per load)
+      const int rw_first = kSplit == 2 ? 32 * (1 - half) : 0;
+      float* rw_slice0 = nullptr;
+      const float* rw_src = nullptr;
+      int rw_yw = 0, rw_xw = 0;
+      float rwb[kRwEnt / 32];
+#pragma unroll
+      for (int i = 0; i < kRwEnt / 32; ++i) rwb[i] = 0.0f;
+      if (BIAS == BIAS_ROWS) {
+        const int r0 = q0 + 32 * (warp & 3);
+        rw_yw = r0 / a.gw;
+        rw_xw = r0 - rw_yw * a.gw;
+        rw_slice0 = reinterpret_cast<float*>(koff_tab) + warp * 2 * kRwEnt;
+        // dense weights read exp(b - b_max) (the level-table path), the rest the bias itself
+        rw_src = ((SEL == SEL_DENSE && use_lut) ? a.expb : a.bext) + (size_t)h * a.ext_E + rw_first;
+      }
+      auto rw_fetch = [&](int tt) {  // tile tt's window into registers (coalesced loads)
+        const int jt = tt * kN, yk = jt / a.gw, xk = jt - yk * a.gw;
+        const float* src = rw_src + (rw_yw - yk + a.gh - 1) * a.ext_S + (rw_xw - xk + a.gw - kN);
+#pragma unroll
+        for (int i = 0; i < kRwEnt / 32; ++i) rwb[i] = __ldg(src + 32 * i + lane);
+      };
       if (BIAS == BIAS_SMEM && first_pass) bounded_wait(B_BIAS, 0);
       for (int t = 0; t < ntiles; ++t) {
         const uint32_t gs = g_s + (uint32_t)t, buf = gs % kSBufs;
@@ -547,7 +605,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
         const int j0 = t * kN;
         // bias offsets of this tile's keys: per-head table, or computed by this warp
         const int* ko = koff_tab + j0;
-        if (wants_bias && warp_live && a.koff_mode == kKoffWarp) {
+        if (BIAS != BIAS_ROWS && wants_bias && warp_live && a.koff_mode == kKoffWarp) {
           int* wk = koff_tab + (warp * 2 + (int)(gs & 1u)) * kN;  // alternates across passes too
           if (j0 < a.prefix + kN) {
             patch_of(j0 + lane, ya, xa);
@@ -560,6 +618,18 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
           wk[lane + 32] = offset_of(j0 + 32 + lane, yb, xb);
           __syncwarp();
           ko = wk;
+        }
+        // BIAS_ROWS: the bias (or exp(bias)) of this thread's row and key 32 cc + u of
+        // its chunk cc is brow[-(32 cc + u)]
+        const float* brow = nullptr;
+        if (BIAS == BIAS_ROWS && wants_bias && warp_live) {
+          float* sl = rw_slice0 + (t & 1) * kRwEnt;  // last read two tiles ago
+          if (t == 0) rw_fetch(0);
+#pragma unroll
+          for (int i = 0; i < kRwEnt / 32; ++i) sl[32 * i + lane] = rwb[i];
+          __syncwarp();
+          if (t + 1 < ntiles) rw_fetch(t + 1);  // lands while this tile is processed
+          brow = sl + lane + (kN - 1) - rw_first - (kSplit == 2 ? 32 * half : 0);
         }
         const bool ok_wait = __all_sync(0xffffffffu, bounded_wait(B_SFULL + buf, (gs / kSBufs) & 1));
         tc_fence_after();
@@ -579,7 +649,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
         const int nvalid = row_ok ? max(0, min(kN, L - j0)) : 0;
         // Dense with bias: keys past L carry the k_invalid offset (weight 0), and
         // rows past L are never stored, so every tile takes the unmasked path.
-        constexpr bool kMaskInKoff = SEL == SEL_DENSE && HAS_BIAS;
+        constexpr bool kMaskInKoff = SEL == SEL_DENSE && HAS_BIAS && BIAS != BIAS_ROWS;
         const bool full_tile = kMaskInKoff || __all_sync(0xffffffffu, nvalid == kN);
 
         // bias offsets of keys 32*ch+u .. +3 of this tile
@@ -671,6 +741,9 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
                   // a dense matrix row: keys jb+u .. +3 in one aligned 16-byte load
                   const float4 w4 = __ldg(reinterpret_cast<const float4*>(eb_bytes) + ((jb + u) >> 2));
                   bw[0] = w4.x; bw[1] = w4.y; bw[2] = w4.z; bw[3] = w4.w;
+                } else if (BIAS == BIAS_ROWS) {
+#pragma unroll
+                  for (int v = 0; v < 4; ++v) bw[v] = brow[-(32 * cc + u + v)];
                 } else if (HAS_BIAS) {
                   const int4 k4 = koff4(32 * ch + u);
                   const int kk[4] = {k4.x, k4.y, k4.z, k4.w};
@@ -712,7 +785,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
 #pragma unroll
               for (int u = 0; u < 32; u += 4) {
                 int4 k4 = make_int4(0, 0, 0, 0);
-                if (HAS_BIAS) k4 = koff4(32 * ch + u);
+                if (HAS_BIAS && BIAS != BIAS_ROWS) k4 = koff4(32 * ch + u);
                 const int kk[4] = {k4.x, k4.y, k4.z, k4.w};
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
@@ -720,7 +793,9 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
                   float l;
                   if (HAS_BIAS) {
                     if (kMaskInKoff) kinv |= (kk[v] == 4 * a.k_invalid ? 1u : 0u) << (u + v);
-                    l = __fmaf_rn((float)sc, c, __ldg(reinterpret_cast<const float*>(tab_bytes - kk[v])));
+                    const float bv = (BIAS == BIAS_ROWS) ? brow[-(32 * cc + u + v)]
+                                                         : __ldg(reinterpret_cast<const float*>(tab_bytes - kk[v]));
+                    l = __fmaf_rn((float)sc, c, bv);
                   } else {
                     l = (float)sc * c;
                   }
@@ -740,6 +815,20 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
 #pragma unroll
                 for (int u = 0; u < 32; ++u) ex[u] = fast_exp2(__fmaf_rn(lg[u], kLog2e, mo2));
                 lsum += sum32(ex);
+              } else if (kHasRadix && pass == P_FBIN) {
+                // bins of the row's logits (min(fmaf(l, sc, off), kFbTop), monotone in l):
+                // bin b at word b of the row's column; bin 0 (below the window) is not counted
+                if (r_state == 4) {
+#pragma unroll
+                  for (int u = 0; u < 32; ++u) {
+                    const float uu = fminf(__fmaf_rn(lg[u], fb_sc, fb_off), kFbTop);
+                    const uint32_t ad = (__float_as_uint(uu) & 0xFE00u) + hist_row;
+                    asm volatile(
+                        "{\n\t.reg .pred p;\n\tsetp.ge.f32 p, %1, %2;\n\t@p red.shared.add.u32 [%0], 1;\n\t}" ::"r"(ad),
+                        "f"(uu), "f"(kFbIn)
+                        : "memory");
+                  }
+                }
               } else if (kHasRadix && pass == P_RADIX) {
                 // histogram of the keys inside the window [r_uhi - r_span, r_uhi] (order keys;
                 // keys past L are -inf, below every window), and the count above it
@@ -854,7 +943,15 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
             }
           }
         };
-        if (kSplit == 2 && SEL == SEL_TOPN_INT && pv) {
+        if (EXPORT == EXP_SCORES) {
+          // the integer scores of this tile as the score MMA left them in TMEM
+          if (ok_wait && row < a.n) {
+            int32_t* dst = a.scores + ((size_t)bh * a.n + row) * a.n;
+#pragma unroll
+            for (int u = 0; u < kN; ++u)
+              if (j0 + u < a.n) dst[j0 + u] = (row_ok && j0 + u < L) ? (int32_t)r[u] : 0;
+          }
+        } else if (kSplit == 2 && SEL == SEL_TOPN_INT && pv) {
           // top-N P.V with two threads per row: weights of this thread's chunk, then
           // the row's two threshold-tie counts of this tile are exchanged (every live
           // warp pair reaches the barrier, whatever happened to its waits)
@@ -987,14 +1084,70 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
           const float bmin = a.bminmax[2 * h], bmax = a.bminmax[2 * h + 1];
           const float lo = __fmaf_rn((float)sN, c, bmin);
           const float hw = __fmaf_rn((float)sN, c, bmax);
-          r_uhi = float_order_key(hw);
-          r_span = r_uhi - float_order_key(lo);
-          r_shift = 0;
-          while ((r_span >> r_shift) >= (uint32_t)kRadixBins) ++r_shift;
           r_rank = keff;
-          r_first = true;
-          r_state = 1;
           m = __fmaf_rn((float)smax, c, bmax);  // no logit exceeds it
+          // FBIN map: lo -> about kFbMg + 768 (bin 1), hw -> about kFbMg + 64768 (bin 126);
+          // the rounding of sc and off moves both by far less than a bin while
+          // |lo * sc| < 2^30, else the order-key radix takes the window
+          const float sc_b = 125.0f * 512.0f / (hw - lo);
+          const float lsc = lo * sc_b;
+          if (hw > lo && isfinite(sc_b) && fabsf(lsc) < 1.0e9f) {
+            fb_sc = sc_b;
+            fb_off = (kFbMg + 768.0f) - lsc;
+            r_state = 4;
+          } else {
+            r_uhi = float_order_key(hw);
+            r_span = r_uhi - float_order_key(lo);
+            r_shift = 0;
+            while ((r_span >> r_shift) >= (uint32_t)kRadixBins) ++r_shift;
+            r_first = true;
+            r_state = 1;
+          }
+        }
+      } else if (pass == P_FBIN && r_state == 4) {
+        // the bin holding rank r_rank, counted from the top (bin 127: keys above the
+        // window, fewer than r_rank of them; bin 0 is never reached: at least r_rank
+        // keys reach the window's low end)
+        int cum = 0, bsel = 1, kbin = 0;
+        for (int bb = 127; bb >= 1; --bb) {
+          const int k = (int)hist[bb * kM + srow];
+          if (cum + k >= r_rank) { bsel = bb; kbin = k; break; }
+          cum += k;
+        }
+        // the bin's keys are the logits in [w_lo, w_cut): the least floats that map to
+        // bins bsel and bsel + 1, found by bisection over the order keys of floats
+        auto fb_bin = [&](float x) -> int {
+          const float uu = fminf(__fmaf_rn(x, fb_sc, fb_off), kFbTop);
+          return uu >= kFbIn ? (int)((__float_as_uint(uu) & 0xFE00u) >> 9) : 0;
+        };
+        auto fb_least = [&](int bin) -> float {
+          uint32_t klo = 0x007FFFFFu, khi = 0xFF800000u;  // -inf (bin 0), +inf (bin 127)
+          while (khi - klo > 1u) {
+            const uint32_t mid = klo + ((khi - klo) >> 1);
+            if (fb_bin(order_key_float(mid)) >= bin) khi = mid;
+            else klo = mid;
+          }
+          return order_key_float(khi);
+        };
+        w_lo = fb_least(bsel);
+        w_cut = bsel >= 127 ? INFINITY : fb_least(bsel + 1);
+        // the largest float below w_cut (no logit is -0, so below +0 means negative)
+        w_hi = (w_cut == 0.0f) ? -1.4e-45f : order_key_float(float_order_key(w_cut) - 1u);
+        r_rank -= cum;
+        r_cnt = 0;
+        if (kMerge && kbin <= kCap) {
+          r_state = 3;
+        } else {
+          r_uhi = float_order_key(w_hi);
+          r_span = r_uhi - float_order_key(w_lo);
+          r_first = false;
+          if (kbin <= kCandCap) {
+            r_state = 2;
+          } else {
+            r_shift = 0;
+            while ((r_span >> r_shift) >= (uint32_t)kRadixBins) ++r_shift;
+            r_state = 1;
+          }
         }
       } else if (pass == P_RADIX && r_state == 1) {
         if (r_first) r_rank -= r_above;  // rank within the first window
@@ -1092,19 +1245,21 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
     }
     tie_seen = 0;
     // ---- the CTA chooses the next pass
+    const int any_fbin = __syncthreads_or(tid < kM && r_state == 4);
     const int any_refine = __syncthreads_or(tid < kM && r_state == 1);
     const int any_collect = __syncthreads_or(tid < kM && r_state == 2);
     int next;
     if (*abort_flag) next = P_DONE;
-    else if (pass == P_IDX || pass == P_CODES || pass == P_PV) next = P_DONE;
+    else if (pass == P_IDX || pass == P_CODES || pass == P_PV || pass == P_SCORES) next = P_DONE;
     else if (pass == P_NORM) next = (EXPORT == EXP_CODES) ? P_CODES : P_PV;
+    else if (any_fbin) next = P_FBIN;
     else if (any_refine) next = P_RADIX;
-    else if (any_collect) next = kMerge ? P_PV : P_COLLECT;
+    else if (any_collect) next = P_COLLECT;
     else if (EXPORT == EXP_IDX) next = P_IDX;
     else if ((EXPORT == EXP_CODES || MODE == MODE_Q) && SEL == SEL_TOPN_FLOAT && pass != P_KEPT_NORM) next = P_KEPT_NORM;
     else if (EXPORT == EXP_CODES) next = P_CODES;
     else next = P_PV;
-    if (next == P_RADIX && tid < kM) {
+    if ((next == P_RADIX || next == P_FBIN) && tid < kM) {
       for (int bb = 0; bb < kRadixBins / 2; ++bb) hist[bb * kM + srow] = 0u;
       r_above = 0;
     }
@@ -1259,6 +1414,11 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
     if (tid < kM && row < a.n) {
       int32_t* dst = a.idx + ((size_t)bh * a.n + row) * a.N;
       for (int p = row_ok ? min(SEL == SEL_DENSE ? L : kept_seen, a.N) : 0; p < a.N; ++p) dst[p] = -1;
+    }
+  } else if (EXPORT == EXP_SCORES) {
+    if (tid < kM && row < a.n) {
+      int32_t* dst = a.scores + ((size_t)bh * a.n + row) * a.n;
+      for (int j = row_ok ? ntiles * kN : 0; j < a.n; ++j) dst[j] = 0;
     }
   } else {
     if (tid < kM && row >= a.row_begin && row < a.row_end && row < a.n) {

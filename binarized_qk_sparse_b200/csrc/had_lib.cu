@@ -16,6 +16,7 @@
 #include <cmath>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "../../include/had.h"
@@ -24,6 +25,7 @@
 #include "attn.cuh"
 #include "dense_ref.cuh"
 #include "attn_tc.cuh"
+#include "probe.cuh"
 
 namespace had {
 
@@ -40,6 +42,10 @@ using tc::EXP_CODES;
 
 constexpr int kMaxDevices = 64;
 thread_local char t_last_error[256] = "";
+// bound of the fused kernel's pipeline waits and the timeout-path test hook
+// (had_debug_bounded_wait); library-wide, read at each launch
+std::atomic<long long> g_wait_cycles{tc::kWaitCycles};
+std::atomic<int> g_force_expiry{0};
 
 unsigned* status_ptr(int dev) {
   static std::mutex mu;
@@ -251,6 +257,7 @@ had_status validate_attention(const void* Q, const void* K, const void* V, const
     if (!O || !aligned16(O) || (o_dtype != HAD_F32 && o_dtype != HAD_BF16)) return HAD_ERR_INVALID;
   }
   if (EXP == EXP_IDX && (!idx || N < 1 || (reinterpret_cast<uintptr_t>(idx) & 3u))) return HAD_ERR_INVALID;
+  if (EXP == tc::EXP_SCORES && (!idx || (reinterpret_cast<uintptr_t>(idx) & 3u))) return HAD_ERR_INVALID;
   if (EXP == EXP_CODES && (!codes || row_begin < 0 || row_end <= row_begin || row_end > s->n)) return HAD_ERR_INVALID;
   for (int h = 0; alpha_q && h < s->H; ++h)
     if (!(alpha_q[h] > 0.0f) || !std::isfinite(alpha_q[h])) return HAD_ERR_INVALID;
@@ -384,6 +391,7 @@ template <int SEL, int MODE, bool VF32, int EXP>
 had_status launch_tc_b(int bias, const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
   using namespace tc;
   if (bias == BIAS_SMEM) return launch_tc_t<SEL, MODE, BIAS_SMEM, VF32, EXP, 2>(a, grid, st);
+  if (bias == BIAS_ROWS) return launch_tc_t<SEL, MODE, BIAS_ROWS, VF32, EXP, 2>(a, grid, st);
   if (bias == BIAS_DGLOBAL) return launch_tc_t<SEL, MODE, BIAS_DGLOBAL, VF32, EXP, 2>(a, grid, st);
   if (bias == BIAS_GLOBAL) return launch_tc_t<SEL, MODE, BIAS_GLOBAL, VF32, EXP, 2>(a, grid, st);
   return launch_tc_t<SEL, MODE, BIAS_NONE, VF32, EXP, 2>(a, grid, st);
@@ -399,28 +407,39 @@ had_status launch_tc_n(const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
   return launch_tc_t<SEL, MODE, tc::BIAS_NONE, VF32, EXP, 1>(a, grid, st);
 }
 
+// Top-N with a bias: per-warp bias windows in shared memory (relative-position
+// tables on grids with rows of a multiple of 64 patches and no class tokens), or
+// gathers from the extended table in global memory.
+template <int MODE, bool VF32, int EXP>
+had_status launch_tc_f(bool rows, const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
+  if (rows) return launch_tc_t<tc::SEL_TOPN_FLOAT, MODE, tc::BIAS_ROWS, VF32, EXP, 1>(a, grid, st);
+  return launch_tc_t<tc::SEL_TOPN_FLOAT, MODE, tc::BIAS_GLOBAL, VF32, EXP, 1>(a, grid, st);
+}
+
 template <int EXP>
-had_status dispatch_tc(int sel, int mode, int bias, bool vf32, const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
+had_status dispatch_tc(int sel, int mode, int bias, bool vf32, bool rows, const tc::TcArgs& a, dim3 grid,
+                       cudaStream_t st) {
   using namespace tc;
+  if (EXP == EXP_SCORES) return launch_tc_t<SEL_DENSE, MODE_F, BIAS_NONE, false, EXP_SCORES, 1>(a, grid, st);
   if (EXP == EXP_CODES || (EXP == EXP_NONE && mode == MODE_Q)) {
     constexpr int E = EXP;
     if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_Q, false, E>(bias, a, grid, st);
     if (sel == SEL_TOPN_INT) return launch_tc_n<SEL_TOPN_INT, MODE_Q, false, E>(a, grid, st);
-    return launch_tc_t<SEL_TOPN_FLOAT, MODE_Q, BIAS_GLOBAL, false, E, 1>(a, grid, st);
+    return launch_tc_f<MODE_Q, false, E>(rows, a, grid, st);
   }
   if (EXP == EXP_IDX) {
     if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, false, EXP>(bias, a, grid, st);
     if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, BIAS_NONE, false, EXP, 1>(a, grid, st);
-    return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, BIAS_GLOBAL, false, EXP, 1>(a, grid, st);
+    return launch_tc_f<MODE_F, false, EXP>(rows, a, grid, st);
   }
   if (vf32) {
     if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, true, EXP>(bias, a, grid, st);
     if (sel == SEL_TOPN_INT) return launch_tc_n<SEL_TOPN_INT, MODE_F, true, EXP>(a, grid, st);
-    return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, BIAS_GLOBAL, true, EXP, 1>(a, grid, st);
+    return launch_tc_f<MODE_F, true, EXP>(rows, a, grid, st);
   }
   if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, false, EXP>(bias, a, grid, st);
   if (sel == SEL_TOPN_INT) return launch_tc_n<SEL_TOPN_INT, MODE_F, false, EXP>(a, grid, st);
-  return launch_tc_t<SEL_TOPN_FLOAT, MODE_F, BIAS_GLOBAL, false, EXP, 1>(a, grid, st);
+  return launch_tc_f<MODE_F, false, EXP>(rows, a, grid, st);
 }
 
 // Stage 2: the fused kernel over a prepared workspace.
@@ -480,11 +499,19 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
   a.seqlens = s->seqlens;
   a.O = O; a.o_bf16 = (o_dtype == HAD_BF16) ? 1 : 0;
   a.idx = idx; a.codes = codes; a.row_begin = row_begin; a.row_end = row_end;
+  if (EXP == tc::EXP_SCORES) a.scores = idx;
+  a.wait_cycles = g_wait_cycles.load();
+  a.force_expiry = g_force_expiry.load();
   a.B = d.B; a.H = d.H; a.n = d.n; a.n_pad = d.n_pad; a.N = N;
   a.status = status;
   a.koff_mode = (d.n_pad <= tc::kKoffTableMax) ? tc::kKoffTable : tc::kKoffWarp;
+  // per-warp bias windows: a relative-position table, no class tokens, grid rows of a
+  // multiple of 64 patches (a warp's 32 rows and a tile's 64 keys each in one image row)
+  const bool rows = has_bias && !bias->dense && bias->prefix == 0 && bias->gw % 64 == 0 &&
+                    a.ext_S == 2 * bias->gw;
   const int bias_kind = !has_bias                        ? tc::BIAS_NONE
                         : a.ext_E <= tc::kBiasSmemMax      ? tc::BIAS_SMEM
+                        : rows                             ? tc::BIAS_ROWS
                         : a.bias_dense && a.ext_S % 4 == 0 ? tc::BIAS_DGLOBAL
                                                            : tc::BIAS_GLOBAL;
   a.int_levels = 1;
@@ -501,7 +528,8 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
     }
   }
   dim3 grid((s->n + tc::kM - 1) / tc::kM, d.BH);
-  return dispatch_tc<EXP>(select_kind(s, bias, N), quant ? tc::MODE_Q : tc::MODE_F, bias_kind, vf32, a, grid, st);
+  return dispatch_tc<EXP>(EXP == tc::EXP_SCORES ? (int)tc::SEL_DENSE : select_kind(s, bias, N),
+                         quant ? tc::MODE_Q : tc::MODE_F, bias_kind, vf32, rows, a, grid, st);
 }
 
 had_status device_status_ptr(unsigned** out) {
@@ -525,7 +553,7 @@ had_status run_attention(const void* Q, const void* K, const void* V, const had_
   unsigned* status = nullptr;
   if ((r = device_status_ptr(&status)) != HAD_OK) return r;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  r = prepare_stage(Q, K, V, s, bias, N, mode, EXP != EXP_IDX, workspace, st, status);
+  r = prepare_stage(Q, K, V, s, bias, N, mode, EXP != EXP_IDX && EXP != tc::EXP_SCORES, workspace, st, status);
   if (r != HAD_OK) return r;
   return attend_stage<EXP>(V, s, bias, alpha_q, alpha_k, N, mode, O, o_dtype, idx, codes, row_begin, row_end,
                            workspace, st, status);
@@ -788,6 +816,19 @@ had_status had_topn_indices(const void* Q, const void* K, const had_shape* s, co
                                 nullptr, 0, 0, workspace, ws_bytes, stream);
 }
 
+had_status had_attention_scores(const void* Q, const void* K, const had_shape* s, int32_t* S, void* workspace,
+                                size_t ws_bytes, void* stream) {
+  return run_attention<tc::EXP_SCORES>(Q, K, nullptr, s, nullptr, nullptr, nullptr, 0, HAD_MODE_FLOAT, nullptr,
+                                       HAD_F32, S, nullptr, 0, 0, workspace, ws_bytes, stream);
+}
+
+had_status had_debug_bounded_wait(long long max_cycles, int force_expiry) {
+  if (max_cycles < 0 || (max_cycles > 0 && max_cycles < 10000)) return HAD_ERR_INVALID;
+  g_wait_cycles.store(max_cycles == 0 ? tc::kWaitCycles : max_cycles);
+  g_force_expiry.store(force_expiry ? 1 : 0);
+  return HAD_OK;
+}
+
 had_status had_attention_codes_u8(const void* Q, const void* K, const void* V, const had_shape* s,
                                   const had_relpos_bias* bias, const float* alpha_q, const float* alpha_k, int N,
                                   int row_begin, int row_end, uint8_t* A, void* workspace, size_t ws_bytes,
@@ -908,7 +949,11 @@ had_status pack_scratch_ptr(double** out) {
   int dev = 0;
   cudaError_t ce = cudaGetDevice(&dev);
   if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return HAD_ERR_UNSUPPORTED;
+  if (dev < 0 || dev >= kMaxDevices) {
+    snprintf(t_last_error, sizeof(t_last_error), "had_binarize_pack_noalloc: device index %d is beyond the %d "
+             "devices the library tracks", dev, kMaxDevices);
+    return HAD_ERR_UNSUPPORTED;
+  }
   std::lock_guard<std::mutex> lk(mu);
   if (!ptrs[dev]) {
     void* p = nullptr;
@@ -949,6 +994,41 @@ had_status had_binarize_pack_noalloc(const void* X, const had_shape* s, float* m
   // k_stats writes every partial sum k_pack reads, so no part of the scratch needs clearing.
   return launch_prep(s, X, nullptr, nullptr, 0, 1, scratch, nullptr, nullptr, mu_out, bits, nullptr, nullptr, nullptr,
                      nullptr, nullptr, static_cast<cudaStream_t>(stream), status);
+}
+
+had_status had_probe_mma_rate(int kind, int iters, double* tops, double* ms) {
+  if ((kind != 0 && kind != 1) || iters < 2 || iters > (1 << 22) || !tops) return HAD_ERR_INVALID;
+  int dev = 0, sms = 0;
+  cudaError_t ce = cudaGetDevice(&dev);
+  if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
+  if ((ce = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+    return cuda_fail(ce, "cudaDeviceGetAttribute");
+  unsigned* status = status_ptr(dev);
+  if (!status) return cuda_fail(cudaErrorInvalidSymbol, "status word");
+  cudaEvent_t e0 = nullptr, e1 = nullptr;
+  if ((ce = cudaEventCreate(&e0)) != cudaSuccess || (ce = cudaEventCreate(&e1)) != cudaSuccess) {
+    if (e0) cudaEventDestroy(e0);
+    return cuda_fail(ce, "cudaEventCreate");
+  }
+  had_status r = HAD_OK;
+  float t = 0.0f;
+  // a short launch first (clocks up, code loaded), then the timed one
+  probe::k_probe_mma<<<sms, probe::kThreads, probe::kSmemTotal, 0>>>(kind, iters / 8 + 2, status);
+  cudaEventRecord(e0, 0);
+  probe::k_probe_mma<<<sms, probe::kThreads, probe::kSmemTotal, 0>>>(kind, iters, status);
+  cudaEventRecord(e1, 0);
+  if ((r = check_launch("k_probe_mma")) == HAD_OK) {
+    if ((ce = cudaEventSynchronize(e1)) != cudaSuccess || (ce = cudaEventElapsedTime(&t, e0, e1)) != cudaSuccess)
+      r = cuda_fail(ce, "probe timing");
+  }
+  cudaEventDestroy(e0);
+  cudaEventDestroy(e1);
+  if (r != HAD_OK) return r;
+  const double k = kind == 0 ? 32.0 : 16.0;  // K elements per MMA
+  const double ops = 2.0 * probe::kM * probe::kN * k * (double)iters * (double)sms;
+  *tops = ops / ((double)t * 1e-3) / 1e12;
+  if (ms) *ms = t;
+  return HAD_OK;
 }
 
 had_status had_get_device_status(void) {

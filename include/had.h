@@ -184,6 +184,15 @@ had_status had_dense_reference_mode(const void* Q, const void* K, const void* V,
 had_status had_scores_int(const uint32_t* qbits, const uint32_t* kbits, const had_shape* s, int32_t* S,
                           void* stream);
 
+/* had_attention_scores: the integer scores s_ij = d - 2*popcount(q~_i XOR k~_j)
+ * (BinaryAttention §2.1-§2.2) exactly as the fused kernel forms them -- the
+ * +-1 int8 tensor-core product of the binarized Q and K in tensor memory --
+ * written out as DEVICE int32 S [B][H][n][n] (0 where i >= L or j >= L).
+ * Q, K as in had_attention; workspace as had_attention_workspace_size(s, 0,
+ * HAD_MODE_FLOAT, NULL).  For parity checks on small shapes. */
+had_status had_attention_scores(const void* Q, const void* K, const had_shape* s, int32_t* S, void* workspace,
+                                size_t ws_bytes, void* stream);
+
 /* had_topn_indices: the kept set of every query row, as DEVICE int32
  * [B][H][n][N] in ascending key order, padded with -1 (rows i >= L are all
  * -1).  Same arguments and workspace as had_attention with N >= 1. */
@@ -205,6 +214,31 @@ had_status had_attention_codes_u8(const void* Q, const void* K, const void* V, c
  * fp32 [B][H][d].  Needs had_attention_workspace_size(s, 0, HAD_MODE_U8I8, NULL). */
 had_status had_quantize_v(const void* V, const had_shape* s, int8_t* Vq, float* vscale, void* workspace,
                           size_t ws_bytes, void* stream);
+
+/* ---- tensor-pipe probe (a measurement aid; the pages have no counterpart) --
+ * had_probe_mma_rate: the rate this GPU's tensor cores sustain on the two MMA
+ * kinds the hot path issues -- kind 0: tcgen05.mma kind::i8 (the +-1 score
+ * contraction of BinaryAttention §2.2, and the uint8 A x int8 V of §2.4);
+ * kind 1: kind::f16 with bf16 operands (the float A.V).  One CTA per SM issues
+ * `iters` (2 .. 2^22) back-to-back M=128 N=256 MMAs (K = 32 int8 or 16 bf16
+ * elements each) from operands resident in shared memory into one tensor-memory
+ * accumulator.  *tops receives 2*M*N*K*iters*SMs / elapsed in 10^12 ops/s, and
+ * *ms (if not NULL) the elapsed milliseconds.  Runs on the legacy default
+ * stream of the current device and waits for it (not for use in a hot loop);
+ * allocates no device memory. */
+had_status had_probe_mma_rate(int kind, int iters, double* tops, double* ms);
+
+/* ---- the timeout path (a test hook; the pages have no counterpart) --------
+ * had_debug_bounded_wait: every pipeline wait of the fused kernel (TMA loads,
+ * tensor-core MMAs, the softmax warps' hand-offs) gives up after max_cycles SM
+ * clocks (0 = the default, about one second; else at least 10000), sets the
+ * HAD_ERR_TIMEOUT bit of the device status word, skips the rest of its work,
+ * writes zero output, waits (with a bound of its own) for its loads and MMAs in
+ * flight, and frees its tensor memory.  force_expiry != 0 makes one thread of
+ * every CTA of the following launches first wait on a barrier that nothing
+ * completes, so that this path runs; force_expiry = 0 restores normal runs.
+ * The setting is library-wide and read at each launch (not thread-safe). */
+had_status had_debug_bounded_wait(long long max_cycles, int force_expiry);
 
 /* ---- status ---------------------------------------------------------------
  * had_get_device_status: synchronizes the current device, reads the sticky

@@ -125,6 +125,23 @@ def test_integer_scores_bit_exact(oracle_mod, name):
     np.testing.assert_array_equal(S, S_o)
 
 
+def _subset(w, B, name_suffix=""):
+    return workloads.Workload(w.name + name_suffix, B, w.H, w.n, w.d, w.dtype, w.Q[:B], w.K[:B], w.V[:B],
+                              None if w.seqlens is None else w.seqlens[:B], None, w.passes, w.seed, w.recipe)
+
+
+@pytest.mark.parametrize("name,B", [("tiny", 1), ("bert", 4), ("t5_256", 2), ("t5_1024", 1)])
+def test_fused_kernel_scores_bit_exact(oracle_mod, name, B):
+    """The scores the fused kernel forms in tensor memory (+-1 int8 tcgen05 MMA),
+    read back from it, against the oracle's d - 2*popcount on its own bits."""
+    w = _subset(_workload(name), B)
+    Q, K, V, seq, _ = _dev_inputs(w)
+    S = had.had_attention_scores(Q, K, seq).cpu().numpy()
+    ref = oracle_mod.attention(w.Q, w.K, w.V, N=0, seqlens=w.seqlens, rows=np.zeros(0, np.int64))
+    S_o = oracle_mod.binary_scores(ref.qbits, ref.kbits, 64, w.seqlens)
+    np.testing.assert_array_equal(S, S_o)
+
+
 # ----------------------------------------------------------------------------- top-N index sets
 
 def _oracle_full(oracle_mod, w, N, mode, rows=None, want_idx=False, want_codes=False):
@@ -171,7 +188,8 @@ def test_topn_sets_stress_full_size(oracle_mod):
 
 # ----------------------------------------------------------------------------- outputs
 
-@pytest.mark.parametrize("name,N", [("tiny", 15), ("tiny", 0), ("bert", 30), ("t5_128", 15), ("t5_1024", 120)])
+@pytest.mark.parametrize("name,N", [("tiny", 15), ("tiny", 0), ("bert", 30), ("t5_128", 15), ("t5_256", 30),
+                                    ("t5_512", 60), ("t5_1024", 120)])
 def test_float_output_within_tolerance(oracle_mod, name, N):
     w = _workload(name)
     Q, K, V, seq, bias = _dev_inputs(w)
@@ -278,6 +296,37 @@ def test_relpos_bias_layouts(oracle_mod, gh, gw, prefix, seqlens):
     B = 1 if seqlens is None else len(seqlens)
     w = workloads.grid(B, 2, gh, gw, prefix, seqlens)
     _check_grid(oracle_mod, w, 24, 21)
+
+
+@pytest.mark.parametrize("gh,gw,seqlens", [
+    (4, 64, None),               # a CTA's 128 rows span two image rows (warps 0-1 and 2-3)
+    (8, 128, [1024, 700]),       # one image row per CTA; ragged lengths (a partial last tile)
+    (3, 192, None),              # image rows of 192 patches: CTAs straddle two rows
+    (2, 256, [512, 333]),        # two CTAs per image row
+])
+def test_topn_bias_row_windows(oracle_mod, gh, gw, seqlens):
+    """Top-N with a relative-position bias on grids whose rows hold a multiple of 64
+    patches (each warp reads its bias from a window staged in shared memory): float
+    and uint8 O, kept sets and the uint8 codes, against the oracle."""
+    B = 1 if seqlens is None else len(seqlens)
+    w = workloads.grid(B, 2, gh, gw, 0, seqlens, seed=31)
+    Q, K, V, seq, bias = _dev_inputs(w)
+    rows = _sample_rows(w, 40, 17)
+    rows_t = torch.from_numpy(rows).cuda()
+    N = max(1, w.n // 8)
+    Of = _flat(had.had_attention(Q, K, V, N=N, mode="float", seqlens=seq, bias=bias))[rows_t].float().cpu().numpy()
+    assert np.max(np.abs(Of - _oracle_full(oracle_mod, w, N, 0, rows=rows).O)) <= _tol(w)
+    Oq = _flat(had.had_attention(Q, K, V, N=N, mode="u8i8", seqlens=seq, bias=bias))[rows_t].float().cpu().numpy()
+    assert np.max(np.abs(Oq - _oracle_full(oracle_mod, w, N, 1, rows=rows).O)) <= _tol(w) + float(np.max(np.abs(w.V))) / 255
+    idx = _flat(had.had_topn_indices(Q, K, N, seq, bias))[rows_t].cpu().numpy()
+    np.testing.assert_array_equal(idx, _oracle_full(oracle_mod, w, N, 0, rows=rows, want_idx=True).idx)
+    A = had.had_attention_codes_u8(Q, K, V, 0, w.n, N=N, seqlens=seq, bias=bias).cpu().numpy()
+    A = A.reshape(w.B, w.H, w.n, w.n)[:, 1].reshape(-1, w.n)
+    band = np.array([(b * w.H + 1) * w.n + i for b in range(w.B) for i in range(w.n)], np.int64)
+    _codes_ok(A, _oracle_full(oracle_mod, w, N, 1, rows=band, want_codes=True).Aq)
+    # dense float: the exp(bias) windows when the table is too large for shared memory
+    Od = _flat(had.had_attention(Q, K, V, N=0, mode="float", seqlens=seq, bias=bias))[rows_t].float().cpu().numpy()
+    assert np.max(np.abs(Od - _oracle_full(oracle_mod, w, 0, 0, rows=rows).O)) <= _tol(w)
 
 
 # ----------------------------------------------------------------------------- comparison mode
@@ -493,6 +542,48 @@ def test_host_entry_point_matches_the_device_call(oracle_mod, pinned):
     rows = _sample_rows(sub, 24, 5)
     ref = _oracle_full(oracle_mod, sub, 30, 0, rows=rows).O
     assert np.max(np.abs(got.reshape(-1, 64)[rows] - ref)) <= _tol(sub)
+
+
+@pytest.mark.parametrize("L,code", [(6, 43), (30, 9), (102, 3), (510, 1)])
+def test_u8_codes_round_half_up_at_exact_ties(oracle_mod, L, code):
+    """Rows of L equal logits (identical Q rows and K rows: every score is d) have
+    p = 1/L, and 255/L = k + 1/2 exactly: the codes must be floor(255 p + 0.5) = k + 1
+    on both sides, bit for bit."""
+    n, d = 512, 64
+    rng = np.random.default_rng(5)
+    q = workloads.bf16_round(rng.standard_normal(d).astype(np.float32))
+    k = workloads.bf16_round(rng.standard_normal(d).astype(np.float32))
+    Qn = np.broadcast_to(q, (1, 1, n, d)).copy()
+    Kn = np.broadcast_to(k, (1, 1, n, d)).copy()
+    Vn = workloads.bf16_round(rng.standard_normal((1, 1, n, d)).astype(np.float32))
+    seq_n = np.array([L], np.int32)
+    Q, K, V = (torch.from_numpy(x).to(torch.bfloat16).cuda() for x in (Qn, Kn, Vn))
+    A = had.had_attention_codes_u8(Q, K, V, 0, n, N=0, seqlens=torch.from_numpy(seq_n).cuda()).cpu().numpy()
+    ref = oracle_mod.attention(Qn, Kn, Vn, N=0, mode=1, seqlens=seq_n, want_codes=True)
+    np.testing.assert_array_equal(A.reshape(n, n), ref.Aq.reshape(n, n))
+    assert (A.reshape(n, n)[:L, :L] == code).all()
+
+
+def test_timeout_path_reports_and_recovers(oracle_mod):
+    """The fused kernel's bounded waits: with the test hook, one thread of every CTA
+    waits on a barrier nothing completes; its bound (2e6 clocks, about 1 ms)
+    expires, the CTAs wind down with zero output, and the status word says
+    HAD_ERR_TIMEOUT.  The next normal call matches the oracle again."""
+    w = _workload("tiny")
+    Q, K, V, seq, bias = _dev_inputs(w)
+    assert had.had_get_device_status() == had.HAD_OK
+    try:
+        had.had_debug_bounded_wait(2_000_000, True)
+        O = had.had_attention(Q, K, V, N=15, mode="float")
+        torch.cuda.synchronize()
+    finally:
+        had.had_debug_bounded_wait(0, False)
+    assert had.had_get_device_status() == had.HAD_ERR_TIMEOUT
+    assert not O.cpu().numpy().any()
+    O2 = had.had_attention(Q, K, V, N=15, mode="float").cpu().numpy()
+    assert had.had_get_device_status() == had.HAD_OK
+    ref = _oracle_full(oracle_mod, w, 15, 0).O
+    assert np.max(np.abs(O2 - ref)) <= _tol(w)
 
 
 def test_bad_seqlens_raise_device_status():
