@@ -55,6 +55,13 @@ WORKLOADS = {
     "t5_1024": ("t5_1024", 120, "float"),
     "stress_topn": ("stress", 1920, "float"),
     "stress_u8i8": ("stress", 0, "u8i8"),
+    # head dim 128 (the BinaryAttention kernel benchmark's head dim)
+    "deit_d128": ("deit_d128", 0, "u8i8"),
+    "t5_1024_d128": ("t5_1024_d128", 120, "float"),
+    # the library's dense comparison mode: standard bf16 attention on the unbinarized inputs
+    "deit_dense_ref": ("deit", 0, "ref"),
+    "t5_1024_dense_ref": ("t5_1024", 0, "ref"),
+    "stress_dense_ref": ("stress", 0, "ref"),
 }
 
 
@@ -71,14 +78,14 @@ def _peaks():
 HEAD_STAGE_BYTES = 128 * 1024  # heads up to this size are prepared by one kernel from shared memory
 
 
-def launches_per_step(n: int, elem: int, mode: str, has_bias: bool, dense_bias: bool = False) -> int:
+def launches_per_step(n: int, elem: int, mode: str, has_bias: bool, dense_bias: bool = False, d: int = 64) -> int:
     """Kernels one prepare + attend step launches: the sign/pack stage (one
     kernel for short heads, which also builds relative-position bias tables;
     statistics + pack + bias tables otherwise), the range and tables of a
     dense bias matrix (two kernels), the hi/lo split of an fp32 V (float
     mode), and the fused attention."""
     rel = has_bias and not dense_bias
-    k = 1 if n * 64 * elem <= HEAD_STAGE_BYTES else 2 + (1 if rel else 0)
+    k = 1 if (d == 64 and n * 64 * elem <= HEAD_STAGE_BYTES) else 2 + (1 if rel else 0)
     if dense_bias:
         k += 2
     if mode == "float" and elem == 4:
@@ -138,22 +145,25 @@ def alu_ops_per_score(mode: str, N: int, n: int, has_bias: bool) -> float:
     return 1.0 + 6.0 + 7.5
 
 
-def kernel_bytes_per_token(mode: str, v_bytes: int, o_bytes: int) -> int:
-    """Algorithmic bytes per valid token of the fused kernel (k_attn).
+def kernel_bytes_per_token(mode: str, v_bytes: int, o_bytes: int, d: int = 64) -> int:
+    """Algorithmic bytes per valid token of the fused kernel.
 
-    Reads the packed sign bits of Q and K (8 B each at d = 64), V (float mode,
+    Reads the packed sign bits of Q and K (d / 8 B each), V (float mode,
     d * v_bytes) or int8 V (uint8 mode, d bytes), and writes O (d * o_bytes).
+    The comparison mode ("ref") reads the bf16 Q, K and V and writes O.
     """
-    d = 64
+    if mode == "ref":
+        return 3 * d * v_bytes + d * o_bytes
     v = d if mode == "u8i8" else d * v_bytes
-    return 8 + 8 + v + d * o_bytes
+    return d // 8 + d // 8 + v + d * o_bytes
 
 
-def path_bytes_per_token(mode: str, in_bytes: int, o_bytes: int) -> int:
+def path_bytes_per_token(mode: str, in_bytes: int, o_bytes: int, d: int = 64) -> int:
     """Algorithmic bytes per token of the whole path: read Q, K, V once, write and
     read back the packed bits (and the int8 V in uint8 mode), write O once."""
-    d = 64
-    b = 3 * d * in_bytes + 2 * 8 * 2 + d * o_bytes
+    if mode == "ref":
+        return 3 * d * in_bytes + d * o_bytes
+    b = 3 * d * in_bytes + 2 * (d // 8) * 2 + d * o_bytes
     if mode == "u8i8":
         b += 2 * d
     return b
@@ -277,7 +287,10 @@ def _oracle_call_s(w, N, mode, rows):
     import oracle
     b = _oracle_bias(oracle, w)
     t0 = time.perf_counter()
-    oracle.attention(w.Q, w.K, w.V, N=N, mode=1 if mode == "u8i8" else 0, seqlens=w.seqlens, bias=b, rows=rows)
+    if mode == "ref":
+        oracle.dense_attention(w.Q, w.K, w.V, seqlens=w.seqlens, bias=b, rows=rows)
+    else:
+        oracle.attention(w.Q, w.K, w.V, N=N, mode=1 if mode == "u8i8" else 0, seqlens=w.seqlens, bias=b, rows=rows)
     return time.perf_counter() - t0
 
 
@@ -362,7 +375,8 @@ def run_reference(args, rank, world):
 
 
 def _config(w, N, mode):
-    return {"workload": f"{w.name}_{'dense' if N == 0 else f'top{N}'}_{mode}", "B": w.B, "H": w.H, "n": w.n,
+    tag = "dense_ref" if mode == "ref" else f"{'dense' if N == 0 else f'top{N}'}_{mode}"
+    return {"workload": f"{w.name}_{tag}", "B": w.B, "H": w.H, "n": w.n,
             "d": w.d, "N": N, "mode": mode, "in_dtype": w.dtype, "seed": w.seed,
             "bias": _bias_desc(w),
             "seqlens": None if w.seqlens is None else "U{32..256} per sequence",
@@ -396,7 +410,11 @@ def run_gpu(args, rank, world, local_rank):
     elif w.bias is not None:
         bias = had.RelPosBias(torch.from_numpy(w.bias.table).to(dev), w.bias.gh, w.bias.gw, w.bias.prefix)
     O = torch.empty_like(V)
-    ws_bytes = had.had_attention_workspace_size(Q, N, mode, seq, bias)
+    ref = mode == "ref"
+    if ref:
+        ws_bytes = max(16, had.had_dense_reference_workspace_size(Q, seq, bias))
+    else:
+        ws_bytes = had.had_attention_workspace_size(Q, N, mode, seq, bias)
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
@@ -404,10 +422,12 @@ def run_gpu(args, rank, world, local_rank):
     import ctypes
     shp = had.make_shape(Q, seq)
     bstruct = None if bias is None else ctypes.byref(had._bias_c(bias))
-    mcode = had._MODES[mode]
+    mcode = had._MODES[mode] if not ref else 0
     sp = ctypes.c_void_p(stream.cuda_stream)
 
     def prepare():
+        if ref:
+            return
         st = L.had_attention_prepare(ctypes.c_void_p(Q.data_ptr()), ctypes.c_void_p(K.data_ptr()),
                                      ctypes.c_void_p(V.data_ptr()), ctypes.byref(shp), bstruct, N, mcode,
                                      ctypes.c_void_p(ws.data_ptr()), ws_bytes, sp)
@@ -415,6 +435,14 @@ def run_gpu(args, rank, world, local_rank):
             raise had.HadError(st, "had_attention_prepare")
 
     def attend():
+        if ref:
+            st = L.had_dense_reference_mode(ctypes.c_void_p(Q.data_ptr()), ctypes.c_void_p(K.data_ptr()),
+                                            ctypes.c_void_p(V.data_ptr()), ctypes.byref(shp), bstruct, 0,
+                                            ctypes.c_void_p(O.data_ptr()), had._dtype_code(O),
+                                            ctypes.c_void_p(ws.data_ptr()), ws_bytes, sp)
+            if st:
+                raise had.HadError(st, "had_dense_reference_mode")
+            return
         st = L.had_attention_prepared(ctypes.c_void_p(V.data_ptr()), ctypes.byref(shp), bstruct, None, None, N, mcode,
                                       ctypes.c_void_p(O.data_ptr()), had._dtype_code(O),
                                       ctypes.c_void_p(ws.data_ptr()), ws_bytes, sp)
@@ -425,8 +453,11 @@ def run_gpu(args, rank, world, local_rank):
     probe_i8, _ = had.had_probe_mma_rate("i8", 200000)
     probe_bf16, _ = had.had_probe_mma_rate("bf16", 100000)
 
-    kernels_per_step = launches_per_step(w.n, Q.element_size(), mode, bias is not None,
-                                         isinstance(w.bias, workloads.DenseBias))
+    if ref:  # the bias tables (range + tables for a dense matrix) and the kernel
+        kernels_per_step = 1 + (0 if bias is None else (2 if isinstance(w.bias, workloads.DenseBias) else 1))
+    else:
+        kernels_per_step = launches_per_step(w.n, Q.element_size(), mode, bias is not None,
+                                             isinstance(w.bias, workloads.DenseBias), w.d)
     clocks = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
     clocks.start()  # nvidia-smi takes a moment to start: launched before the warm-up
     with torch.cuda.stream(stream):
@@ -472,8 +503,9 @@ def run_gpu(args, rank, world, local_rank):
         hbias = had.DenseBias(bias.table.cpu().pin_memory())
     elif bias is not None:
         hbias = had.RelPosBias(bias.table.cpu().pin_memory(), bias.gh, bias.gw, bias.prefix)
-    host_ws = torch.empty(had.had_attention_host_workspace_size(hQ, N, mode, hseq, hbias), dtype=torch.uint8,
-                          device=dev)
+    if not ref:
+        host_ws = torch.empty(had.had_attention_host_workspace_size(hQ, N, mode, hseq, hbias), dtype=torch.uint8,
+                              device=dev)
     e2e_steps = max(3, min(args.steps, 30))
     h2d = 3 * Q.numel() * Q.element_size() + (0 if hseq is None else hseq.numel() * 4) + \
         (0 if hbias is None else hbias.table.numel() * 4)
@@ -483,8 +515,17 @@ def run_gpu(args, rank, world, local_rank):
         for s in range(e2e_steps + 2):
             if s == 2:
                 e0.record(stream)
-            had.had_attention_host(hQ, hK, hV, N=N, mode=mode, seqlens=hseq, bias=hbias, out=hO, workspace=host_ws,
-                                   stream=stream, synchronize=False)
+            if ref:  # no host entry point: copies in, the call, the copy out, on the same stream
+                Q.copy_(hQ, non_blocking=True)
+                K.copy_(hK, non_blocking=True)
+                V.copy_(hV, non_blocking=True)
+                if hbias is not None:
+                    bias.table.copy_(hbias.table, non_blocking=True)
+                attend()
+                hO.copy_(O, non_blocking=True)
+            else:
+                had.had_attention_host(hQ, hK, hV, N=N, mode=mode, seqlens=hseq, bias=hbias, out=hO,
+                                       workspace=host_ws, stream=stream, synchronize=False)
         e1.record(stream)
         stream.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps, dist, dev)
@@ -493,13 +534,21 @@ def run_gpu(args, rank, world, local_rank):
         return 0
     peaks, peak_kind = _peaks()
     attn_avg_ms = statistics.mean(attn_ms)
-    kbytes = kernel_bytes_per_token(mode, 2 if bf16 else 4, O.element_size()) * queries
+    kbytes = kernel_bytes_per_token(mode, 2 if bf16 else 4, O.element_size(), w.d) * queries
     if bias is not None:
         kbytes += w.bias.table.nbytes
-    tc_ops = score_tensor_ops(w.valid_scores(), w.d)
-    i8_recipe = INT8_PER_BF16 * peaks["bf16_tflops"]
-    i8_peak = max(i8_recipe, probe_i8)
-    roof = north_star_roofline(kbytes, tc_ops, attn_avg_ms, peaks["hbm_gbs"], i8_peak)
+    if ref:  # standard attention: the bf16 QK^T and P.V contractions at the bf16 peak
+        tc_ops = 2.0 * score_tensor_ops(w.valid_scores(), w.d)
+        tc_peak = max(peaks["bf16_tflops"], probe_bf16)
+        peak_txt = f"bf16 = max({peak_kind} burst {peaks['bf16_tflops']} TFLOP/s, probe {probe_bf16:.0f})"
+    else:
+        tc_ops = score_tensor_ops(w.valid_scores(), w.d)
+        tc_peak = max(INT8_PER_BF16 * peaks["bf16_tflops"], probe_i8)
+        peak_txt = (f"int8 = max({INT8_PER_BF16:g} x {peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s, "
+                    f"probe {probe_i8:.0f} TOPS)")
+    roof = north_star_roofline(kbytes, tc_ops, attn_avg_ms, peaks["hbm_gbs"], tc_peak)
+    if ref:
+        roof["unit"] = roof["unit"].replace("int8", "bf16")
     traffic = None
     tr_path = os.path.join(ROOT, "profiles", "traffic.json")
     if os.path.exists(tr_path):
@@ -508,12 +557,11 @@ def run_gpu(args, rank, world, local_rank):
     roof.update({"traffic": traffic, "kernel": "k_attn_tc (fused score/top-N/softmax/A.V)",
                  "avg_launch_ms": attn_avg_ms, "algorithmic_bytes_per_launch": kbytes,
                  "tensor_ops_per_launch": tc_ops,
-                 "peak_kind": (f"int8 = max({INT8_PER_BF16:g} x {peak_kind} bf16 burst {peaks['bf16_tflops']} "
-                               f"TFLOP/s, probe {probe_i8:.0f} TOPS); HBM {peak_kind} {peaks['hbm_gbs']} GB/s")})
-    ops_per_score = alu_ops_per_score(mode, N, w.n, bias is not None)
+                 "peak_kind": f"{peak_txt}; HBM {peak_kind} {peaks['hbm_gbs']} GB/s"})
+    ops_per_score = 0.0 if ref else alu_ops_per_score(mode, N, w.n, bias is not None)
     alu_ops = ops_per_score * w.valid_scores()
     alu_achieved = alu_ops / (attn_avg_ms * 1e-3) / 1e12
-    pbytes = path_bytes_per_token(mode, 2 if bf16 else 4, O.element_size()) * queries
+    pbytes = path_bytes_per_token(mode, 2 if bf16 else 4, O.element_size(), w.d) * queries
     path_achieved = pbytes / (ms_per_step * 1e-3) / 1e9
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -89,7 +89,7 @@ def lib():
         L.had_attention_host_workspace_size.argtypes = [SP, I, I, BP, I]
         L.had_attention_host_workspace_size.restype = SZ
         L.had_attention_host.argtypes = [P, P, P, SP, BP, P, P, I, I, P, I, I, P, SZ, P]
-        L.had_dense_reference_workspace_size.argtypes = [SP]
+        L.had_dense_reference_workspace_size.argtypes = [SP, BP]
         L.had_dense_reference_workspace_size.restype = SZ
         L.had_dense_reference_mode.argtypes = [P, P, P, SP, BP, I, P, I, P, SZ, P]
         L.had_scores_int.argtypes = [P, P, SP, P, P]
@@ -310,15 +310,25 @@ def had_attention_host(Q, K, V, N=0, mode="float", seqlens=None, bias=None, alph
     return out
 
 
-def had_dense_reference_mode(Q, K, V, N=0, seqlens=None, bias=None, out=None, out_dtype=None, stream=None):
+def had_dense_reference_workspace_size(X, seqlens=None, bias=None) -> int:
+    shp = make_shape(X, seqlens)
+    return int(lib().had_dense_reference_workspace_size(ctypes.byref(shp), _bias_struct(bias)))
+
+
+def had_dense_reference_mode(Q, K, V, N=0, seqlens=None, bias=None, out=None, out_dtype=None, workspace=None,
+                             stream=None):
     """Standard dense attention on the unbinarized bf16 inputs (the library's comparison mode)."""
-    _check_dev(Q, K, V, seqlens, out)
+    _check_dev(Q, K, V, seqlens, out, workspace)
     B, H, n, d = Q.shape
     shp = make_shape(Q, seqlens)
     if out is None:
         out = torch.empty((B, H, n, d), dtype=out_dtype or V.dtype, device=Q.device)
-    st = lib().had_dense_reference_mode(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shp), _bias_struct(bias), int(N),
-                                        _ptr(out), _dtype_code(out), None, 0, _stream(stream))
+    bs = _bias_struct(bias)
+    need = int(lib().had_dense_reference_workspace_size(ctypes.byref(shp), bs))
+    ws = _workspace(need, Q.device, workspace, stream) if need > 0 else None
+    st = lib().had_dense_reference_mode(_ptr(Q), _ptr(K), _ptr(V), ctypes.byref(shp), bs, int(N),
+                                        _ptr(out), _dtype_code(out), _ptr(ws), 0 if ws is None else ws.numel(),
+                                        _stream(stream))
     _raise(st, "had_dense_reference_mode")
     return out
 

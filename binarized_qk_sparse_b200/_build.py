@@ -1,4 +1,9 @@
-"""Build the CUDA library in-tree: binarized_qk_sparse_b200/libhad_b200.so (sm_100a)."""
+"""Build the CUDA library in-tree: binarized_qk_sparse_b200/libhad_b200.so (sm_100a).
+
+The library is two translation units compiled in parallel -- had_lib.cu (host
+code, the prep kernels and the fused kernel at head dim 64) and attn_d128.cu
+(the fused kernel at head dim 128) -- linked into one shared object.
+"""
 from __future__ import annotations
 
 import os
@@ -8,13 +13,15 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhad_b200.so")
-SOURCES = ["had_lib.cu"]
-DEPS = ["common.cuh", "sm100.cuh", "prep.cuh", "attn.cuh", "attn_tc.cuh", "dense_ref.cuh", "probe.cuh", "had_lib.cu"]
+OBJ_DIR = os.path.join(HERE, "_build")
+SOURCES = ["had_lib.cu", "attn_d128.cu"]
+DEPS = ["common.cuh", "sm100.cuh", "prep.cuh", "attn.cuh", "attn_tc.cuh", "probe.cuh",
+        "launch.cuh", "had_lib.cu", "attn_d128.cu"]
 
-NVCC_FLAGS = [
-    "-gencode", "arch=compute_100a,code=sm_100a",
+ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
+NVCC_FLAGS = ARCH + [
     "-O3", "-lineinfo", "-std=c++17",
-    "-Xcompiler", "-fPIC", "-shared",
+    "-Xcompiler", "-fPIC",
     "--expt-relaxed-constexpr",
 ]
 
@@ -31,11 +38,20 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if not force and not _stale():
         return LIB
     nvcc = os.environ.get("NVCC", "nvcc")
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    objs, procs = [], []
+    for src in SOURCES:
+        obj = os.path.join(OBJ_DIR, os.path.splitext(src)[0] + ".o")
+        cmd = [nvcc, *NVCC_FLAGS, "-c", "-o", obj, os.path.join(CSRC, src)]
+        if verbose:
+            cmd.insert(1, "-Xptxas=-v")
+        procs.append((src, subprocess.Popen(cmd)))
+        objs.append(obj)
+    failed = [src for src, p in procs if p.wait() != 0]
+    if failed:
+        raise RuntimeError(f"nvcc failed on {', '.join(failed)}")
     tmp = LIB + ".tmp"
-    cmd = [nvcc, *NVCC_FLAGS, "-o", tmp] + [os.path.join(CSRC, s) for s in SOURCES]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
+    subprocess.run([nvcc, *ARCH, "-shared", "-o", tmp, *objs], check=True)
     os.replace(tmp, LIB)
     return LIB
 

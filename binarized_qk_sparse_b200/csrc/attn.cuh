@@ -1,7 +1,7 @@
-// attn.cuh -- warp-level (mma.sync) tensor-core pieces shared by the parity
-// export of the integer scores (k_scores_int) and the dense bf16 comparison
-// kernel (dense_ref.cuh): 64-row CTA tiles of 4 warps, cp.async staging.
-// The hot path itself runs on tcgen05 (attn_tc.cuh).
+// attn.cuh -- the parity export of the integer scores from packed bits
+// (k_scores_int) on warp-level mma.sync fragments: 64-row CTA tiles of 4 warps,
+// cp.async staging.  A kernel of its own, independent of the hot path, which
+// runs on tcgen05 (attn_tc.cuh).
 #pragma once
 
 #include "common.cuh"

@@ -59,11 +59,16 @@ __host__ __device__ constexpr int cta_threads(int split) { return 32 * (4 * spli
 constexpr int kSplitMaxKeys = 256;  // top-N without a bias, ragged rows: two threads per row up to this n_pad
 constexpr int kKStages = 4;
 constexpr int kVStages = 2;
-constexpr int kLevels = 65;
+// Score levels of a head dim: s = d - 2h takes d + 1 values.
+__host__ __device__ constexpr int levels_of(int d) { return d + 1; }
 constexpr int kRadixBins = 256;   // 16-bit counters, two per word (a row counts at most kMaxN keys)
 constexpr int kCandCap = 128;    // power of two (the collect slot wraps)
 constexpr int kSBufs = 3;
-constexpr uint32_t kColS = 0, kColO = 192, kTmemCols = 256;
+// TMEM: the score ring in columns [0, 192), O (d columns) from 192; 256 columns at
+// d = 64 (two CTAs per SM), 512 at d = 128 (one CTA per SM).
+constexpr uint32_t kColS = 0, kColO = 192;
+__host__ __device__ constexpr uint32_t tmem_cols(int d) { return d <= 64 ? 256u : 512u; }
+__host__ __device__ constexpr int ctas_per_sm(int d) { return d <= 64 ? 2 : 1; }
 constexpr long long kWaitCycles = 2000000000LL;  // default bound of a pipeline wait: about one second
 // First select pass of top-N with a bias (FBIN): u = min(fmaf(l, sc, off), kFbTop)
 // is a monotone function of the logit l; with u in [kFbMg, kFbMg + 65536) its
@@ -90,7 +95,11 @@ enum { BIAS_NONE = 0, BIAS_GLOBAL = 1, BIAS_SMEM = 2, BIAS_DGLOBAL = 3, BIAS_ROW
 constexpr int kRowWin = 96;  // entries of a warp's bias window (32 rows + 64 keys - 1, padded)
 constexpr int kBiasSmemMax = kBiasSmemEntries;
 
-enum { SEL_DENSE = 0, SEL_TOPN_INT = 1, SEL_TOPN_FLOAT = 2 };
+// SEL_REF: the comparison mode -- standard dense attention on the unbinarized bf16
+// Q and K (scores by a bf16 kind::f16 MMA, fp32 in TMEM), softmax(QK^T / sqrt(d) + B) V;
+// it runs the dense softmax path with an online row maximum.
+enum { SEL_DENSE = 0, SEL_TOPN_INT = 1, SEL_TOPN_FLOAT = 2, SEL_REF = 3 };
+__host__ __device__ constexpr bool sel_dense(int sel) { return sel == SEL_DENSE || sel == SEL_REF; }
 enum { MODE_F = 0, MODE_Q = 1 };
 enum { EXP_NONE = 0, EXP_IDX = 1, EXP_CODES = 2, EXP_SCORES = 3 };
 enum { P_DONE = 0, P_NORM, P_LEVELS, P_FBIN, P_RADIX, P_COLLECT, P_KEPT_NORM, P_PV, P_IDX, P_CODES, P_SCORES };
@@ -100,6 +109,7 @@ struct TcArgs {
   CUtensorMap tm_v;   // V bf16 [BH*n][64], box {64, 64}, 128B swizzle          (float mode)
   CUtensorMap tm_vq;  // int8 V^T [BH*64][n_pad], box {64, 64}, 64B swizzle      (uint8 mode)
   CUtensorMap tm_vlo; // bf16 residual of fp32 V [BH*n][64], box {64, 64}         (fp32 V)
+  CUtensorMap tm_q;   // comparison mode: raw bf16 Q [BH*n][D], box {64, 128}, 128B swizzle (tm_k: raw K, box {64, 64})
   const uint32_t* qbits;   // [BH][n][2]
   const int8_t* kpm;       // [BH][n_pad][64] +-1 codes of K (the score MMA's B operand)
   const void* v_raw;       // V as given, [BH][n][64] bf16 or fp32 (float mode)
@@ -129,27 +139,30 @@ struct TcArgs {
 };
 
 // Shared memory carve-up (offsets from a 1024-byte aligned base).
-template <int SEL, bool VF32, int BIAS>
+// d = 128 tiles are two 64-channel panels, each laid out as a d = 64 tile.
+template <int D, int SEL, bool VF32, int BIAS>
 struct Smem {
   static constexpr bool HAS_BIAS = BIAS != BIAS_NONE;
-  static constexpr int kVStage = (VF32 ? 2 : 1) * kN * kD * 2;   // bf16 V tile (+ residual tile)
-  static constexpr int kQ = 0;                                   // 128 x 64 B
-  static constexpr int kK = kQ + kM * kD;                        // 4 x 4 KB
-  static constexpr int kV = kK + kKStages * kN * kD;             // 2 V stages
+  static constexpr int kLev = levels_of(D);
+  static constexpr int kVStage = (VF32 ? 2 : 1) * kN * D * 2;    // bf16 V tile (+ residual tile)
+  static constexpr int kOpB = SEL == SEL_REF ? 2 : 1;            // bytes per Q, K element (bf16 or +-1 int8)
+  static constexpr int kQ = 0;                                   // 128 x D elements
+  static constexpr int kK = kQ + kM * D * kOpB;                  // 4 x 64 x D elements
+  static constexpr int kV = kK + kKStages * kN * D * kOpB;       // 2 V stages
   static constexpr int kKoff = kV + kVStages * kVStage;          // bias key offsets (table, or 4 warps x 2 x 64)
   static constexpr int kBiasTab = kKoff + (HAS_BIAS ? kKoffTableMax * 4 : 0);  // exp(bias) table (dense)
   // row-pair exchange: dense 2 x 128 fp32 (partials); top-N 6 x 128 (threshold state) + 2 x 2 x 128 tie counts
   static constexpr int kXchg = kBiasTab + (BIAS == BIAS_SMEM ? kBiasSmemMax * 4 : 0);
-  static constexpr int kDq = kXchg + (SEL == SEL_DENSE ? 2 : SEL == SEL_TOPN_INT ? 10 : 0) * kM * 4;  // 64 dequant scales
-  static constexpr int kBar = kDq + kD * 4;
-  static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 2 * kSBufs + 4;
+  static constexpr int kDq = kXchg + (sel_dense(SEL) ? 2 : SEL == SEL_TOPN_INT ? 10 : 0) * kM * 4;  // D dequant scales
+  static constexpr int kBar = kDq + D * 4;
+  static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 2 * kSBufs + 5;
   static constexpr int kMisc = kBar + kNumBars * 8;              // [0] tmem base [1] abort
   static constexpr int kHist = (kMisc + 16 + 127) / 128 * 128;
-  static constexpr int kHistBytes = (SEL == SEL_DENSE) ? kLevels * 32 * 4
-                                    : (SEL == SEL_TOPN_INT) ? kLevels * kM * 4
-                                    : kCandCap * kM * 4;
+  static constexpr int kHistBytes = sel_dense(SEL) ? kLev * 32 * 4
+                                    : (SEL == SEL_TOPN_INT) ? kLev * kM * 4
+                                    : (kCandCap > kLev ? kCandCap : kLev) * kM * 4;
   static constexpr int kTotal = kHist + kHistBytes + 1024;       // + alignment slack
-  static_assert(kCandCap >= kRadixBins / 2 && kCandCap >= kLevels, "radix and level histograms fit the candidate area");
+  static_assert(kCandCap >= kRadixBins / 2, "the radix histogram fits the candidate area");
   static_assert(kMaxN < 65536, "a 16-bit radix counter holds every key of a row");
   static_assert((kCandCap & (kCandCap - 1)) == 0, "candidate slots wrap with a mask");
 };
@@ -164,7 +177,8 @@ enum {
   B_OFULL = B_TDONE + kSBufs,
   B_FINAL,
   B_BIAS,  // staged exp(bias) table landed
-  B_STALL  // never completed: the force_expiry test hook waits on it
+  B_STALL,  // never completed: the force_expiry test hook waits on it
+  B_QFULL   // comparison mode: the raw Q tile landed
 };
 
 // Bias offset of key j: koff = y_j * S + x_j for patch tokens, so that
@@ -205,11 +219,18 @@ __device__ __forceinline__ float sum32(const float (&e)[32]) {
   return t[0];
 }
 
-template <int SEL, int MODE, int BIAS, bool VF32, int EXPORT, int SPLIT>
-__global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_constant__ TcArgs a) {
-  static_assert(SPLIT == 1 || SEL == SEL_DENSE || (SEL == SEL_TOPN_INT && EXPORT == EXP_NONE),
+template <int D, int SEL, int MODE, int BIAS, bool VF32, int EXPORT, int SPLIT>
+__global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(const __grid_constant__ TcArgs a) {
+  static_assert(D == 64 || D == 128, "head dims 64 and 128");
+  constexpr int kLevels = levels_of(D);
+  constexpr int kW = D / 32;        // packed words per token
+  constexpr int kPan = D / 64;      // 64-channel panels of the Q~, K~ and V tiles
+  constexpr uint32_t kTmemCols = tmem_cols(D);
+  constexpr bool kRef = SEL == SEL_REF;        // the unbinarized comparison mode
+  constexpr bool kDense = sel_dense(SEL);
+  static_assert(SPLIT == 1 || kDense || (SEL == SEL_TOPN_INT && EXPORT == EXP_NONE),
                 "two threads per row: dense, or top-N without a bias on its P.V path");
-  static_assert((BIAS != BIAS_SMEM && BIAS != BIAS_DGLOBAL) || SEL == SEL_DENSE,
+  static_assert((BIAS != BIAS_SMEM && BIAS != BIAS_DGLOBAL) || kDense,
                 "staged or vector-read exp(bias) tables serve the dense weights only");
   static_assert(BIAS != BIAS_ROWS || (SEL != SEL_TOPN_INT && 2 * (SPLIT == 2 ? 8 * 64 : 4 * kRowWin) <= kKoffTableMax),
                 "the warps' bias-window slices fit the key-offset area");
@@ -225,7 +246,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
   // logits in [64, 128) of the candidate area
   constexpr bool kMerge = SEL == SEL_TOPN_FLOAT && MODE == MODE_F && EXPORT == EXP_NONE;
   constexpr int kCap = kCandCap / 2;
-  using SM = Smem<SEL, VF32, BIAS>;
+  using SM = Smem<D, SEL, VF32, BIAS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   uint8_t* sm = smem_raw + ((1024u - (raw & 1023u)) & 1023u);
@@ -252,10 +273,10 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
   // ---------------------------------------------------------------- tile past L: zeros, no TMEM
   if (q0 >= L) {
     if (EXPORT == EXP_NONE) {
-      for (int e = tid; e < kM * kD; e += kThreads) {
-        const int r = q0 + e / kD, ch = e % kD;
+      for (int e = tid; e < kM * D; e += kThreads) {
+        const int r = q0 + e / D, ch = e % D;
         if (r < a.n) {
-          const size_t o = ((size_t)bh * a.n + r) * kD + ch;
+          const size_t o = ((size_t)bh * a.n + r) * D + ch;
           if (a.o_bf16) reinterpret_cast<__nv_bfloat16*>(a.O)[o] = __float2bfloat16(0.0f);
           else reinterpret_cast<float*>(a.O)[o] = 0.0f;
         }
@@ -282,6 +303,20 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
   }
 
   // ---------------------------------------------------------------- setup
+  // K~ tile of key tile tt into K stage st: one 64-byte-wide box per 64-channel panel
+  // (comparison mode: raw bf16 K rows, 128-byte panels of 64 channels)
+  auto load_k = [&](uint32_t st, int tt) {
+    mbar_arrive_expect_tx(&bars[B_KFULL + st], kN * D * SM::kOpB);
+#pragma unroll
+    for (int pn = 0; pn < kPan; ++pn) {
+      if (kRef)
+        tma_load_2d(sm + SM::kK + st * kN * D * 2 + pn * kN * 128, &a.tm_k, 64 * pn, bh * a.n + tt * kN,
+                    &bars[B_KFULL + st]);
+      else
+        tma_load_2d(sm + SM::kK + st * kN * D + pn * kN * 64, &a.tm_k, 64 * pn, bh * a.n_pad + tt * kN,
+                    &bars[B_KFULL + st]);
+    }
+  };
   int k_par[kKStages], v_par[kVStages];  // producer: parity of the last load per stage (-1 none)
 #pragma unroll
   for (int s2 = 0; s2 < kKStages; ++s2) k_par[s2] = -1;
@@ -302,6 +337,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
     mbar_init(&bars[B_FINAL], 1);
     mbar_init(&bars[B_BIAS], 1);
     mbar_init(&bars[B_STALL], 1);
+    mbar_init(&bars[B_QFULL], 1);
     misc[1] = 0;
     fence_barrier_init();
     if (BIAS == BIAS_SMEM) {
@@ -311,45 +347,63 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
     }
     prefetch_tensormap(&a.tm_k);
     if (EXPORT == EXP_NONE) prefetch_tensormap(MODE == MODE_Q ? &a.tm_vq : &a.tm_v);
+    if (kRef) {  // the raw Q tile: rows past the tensor read as zeros, other heads' rows are never stored
+      mbar_arrive_expect_tx(&bars[B_QFULL], kM * D * 2);
+#pragma unroll
+      for (int pn = 0; pn < kPan; ++pn)
+        tma_load_2d(sQ + pn * kM * 128, &a.tm_q, 64 * pn, bh * a.n + q0, &bars[B_QFULL]);
+    }
     for (int t = 0; t < k_pre; ++t) {  // stage t = tile t, first use of every stage
-      mbar_arrive_expect_tx(&bars[B_KFULL + t], kN * kD);
-      tma_load_2d(sm + SM::kK + t * kN * kD, &a.tm_k, 0, bh * a.n_pad + t * kN, &bars[B_KFULL + t]);
+      load_k((uint32_t)t, t);
       k_par[t] = 0;
     }
   }
   const int row = q0 + srow;  // softmax threads
   const bool row_ok = is_soft && row < L;
   if (tid < kM) {
-    // Q~ row into the 64-byte swizzled K-major A operand (16-byte chunk c -> c ^ ((row >> 1) & 3))
-    uint32_t w0 = 0, w1 = 0;
-    if (row_ok) {
-      const uint2 w = __ldg(reinterpret_cast<const uint2*>(a.qbits + ((size_t)bh * a.n + row) * kW));
-      w0 = w.x; w1 = w.y;
+    // Q~ row into the 64-byte swizzled K-major A operand, one 128 x 64 B panel per
+    // 64 channels (16-byte chunk c of a panel row -> c ^ ((row >> 1) & 3))
+    uint32_t wq[kW];
+#pragma unroll
+    for (int k = 0; k < kW; ++k) wq[k] = 0u;
+    if (row_ok && !kRef) {
+      const uint2* qw = reinterpret_cast<const uint2*>(a.qbits + ((size_t)bh * a.n + row) * kW);
+#pragma unroll
+      for (int k = 0; k < kW / 2; ++k) {
+        const uint2 w = __ldg(qw + k);
+        wq[2 * k] = w.x;
+        wq[2 * k + 1] = w.y;
+      }
     }
 #pragma unroll
-    for (int cch = 0; cch < 4; ++cch) {
-      const uint32_t f = (cch < 2 ? w0 : w1) >> ((cch & 1) * 16);
+    for (int c16 = 0; c16 < (kRef ? 0 : D / 16); ++c16) {  // 16 channels per chunk
+      const uint32_t f = wq[c16 >> 1] >> ((c16 & 1) * 16);
       uint4 v;
       v.x = expand_nibble_pm1(f & 15u);
       v.y = expand_nibble_pm1((f >> 4) & 15u);
       v.z = expand_nibble_pm1((f >> 8) & 15u);
       v.w = expand_nibble_pm1((f >> 12) & 15u);
-      *reinterpret_cast<uint4*>(sQ + tid * kD + ((cch ^ ((tid >> 1) & 3)) * 16)) = v;
+      const int pn = c16 >> 2, cch = c16 & 3;
+      *reinterpret_cast<uint4*>(sQ + pn * kM * 64 + tid * 64 + ((cch ^ ((tid >> 1) & 3)) * 16)) = v;
     }
-    if (SEL != SEL_DENSE)
+    if (!kDense)
       for (int lev = 0; lev < kLevels; ++lev) hist[lev * kM + srow] = 0u;
-    if (SEL == SEL_DENSE) {
-      // per-lane copies of the level table exp(c * (s - 64)), level k = (64 - s) / 2, at [k][lane]
-      // (each lane computes three levels; warp w writes levels w, w + 4, ... via shuffles)
+    if (kDense) {
+      // per-lane copies of the level table exp(c * (s - d)), level k = (d - s) / 2, at [k][lane]
+      // (lane l computes levels l, l + 32, ...; warp w writes levels w, w + 4, ... via shuffles)
       const float ck = -2.0f * a.c_head[h] * 1.4426950408889634f;
       float* lt = reinterpret_cast<float*>(hist);
-      const float lv0 = exp2f(ck * (float)lane), lv1 = exp2f(ck * (float)(lane + 32)), lv2 = exp2f(ck * 64.0f);
+      float lv[(kLevels + 31) / 32];
+#pragma unroll
+      for (int k = 0; k < (kLevels + 31) / 32; ++k) lv[k] = exp2f(ck * (float)(lane + 32 * k));
       for (int lev = warp; lev < kLevels; lev += 4) {
-        const float v = __shfl_sync(0xffffffffu, lev < 32 ? lv0 : lv1, lev & 31);
-        lt[lev * 32 + lane] = lev == 64 ? lv2 : v;
+        float v = lv[0];
+#pragma unroll
+        for (int k = 1; k < (kLevels + 31) / 32; ++k) v = (lev >> 5) == k ? lv[k] : v;
+        lt[lev * 32 + lane] = __shfl_sync(0xffffffffu, v, lev & 31);
       }
     }
-    if (MODE == MODE_Q && EXPORT == EXP_NONE && tid < kD) dq[tid] = __fdiv_rn(a.vscale[(size_t)bh * kD + tid], 255.0f);
+    if (MODE == MODE_Q && EXPORT == EXP_NONE && tid < D) dq[tid] = __fdiv_rn(a.vscale[(size_t)bh * D + tid], 255.0f);
     if (HAS_BIAS && BIAS != BIAS_ROWS && a.koff_mode == kKoffTable)
       for (int j = tid; j < a.n_pad; j += kM) koff_tab[j] = 4 * key_offset(a, j, L);  // in bytes
     fence_proxy_async();
@@ -390,17 +444,17 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
   // Dense weights as (level table) x exp(b - b_max): both factors <= 1, so no row
   // maximum is needed as long as the smallest product stays far from fp32 underflow.
   bool use_lut = false;
-  if (SEL == SEL_DENSE) {
+  if (kDense && !kRef) {
     const float range = HAS_BIAS ? a.bminmax[2 * h + 1] - a.bminmax[2 * h] : 0.0f;
-    use_lut = c > 0.0f && (128.0f * c + range) * kLog2e <= 100.0f;
+    use_lut = c > 0.0f && (2.0f * D * c + range) * kLog2e <= 100.0f;
   }
-  const bool sum_in_pv = (MODE == MODE_F) && (SEL == SEL_TOPN_FLOAT || (SEL == SEL_DENSE && use_lut));
+  const bool sum_in_pv = (MODE == MODE_F) && (SEL == SEL_TOPN_FLOAT || (kDense && use_lut));
   int sF = 0;  // integer threshold score (top-N without bias)
 
   uint32_t g_k = 0, g_v = 0, g_s = 0;  // tiles issued so far (all passes), per role
 
-  int pass = (SEL == SEL_DENSE) ? (EXPORT == EXP_IDX ? P_IDX : EXPORT == EXP_SCORES ? P_SCORES : P_NORM) : P_LEVELS;
-  if (SEL == SEL_DENSE && EXPORT == EXP_NONE && MODE == MODE_F && use_lut) pass = P_PV;
+  int pass = (kDense) ? (EXPORT == EXP_IDX ? P_IDX : EXPORT == EXP_SCORES ? P_SCORES : P_NORM) : P_LEVELS;
+  if (kDense && EXPORT == EXP_NONE && MODE == MODE_F && use_lut) pass = P_PV;
 
   auto bounded_wait = [&](int bar, uint32_t parity) -> bool {
     if (mbar_test_wait(smem_u32(&bars[bar]), parity)) return true;  // phase already complete
@@ -427,13 +481,18 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
         if (lane == 0 && g_v >= (uint32_t)kVStages) bounded_wait(B_VEMPTY + vs, ((g_v / kVStages) - 1) & 1);
         if (lane == 0 && !*abort_flag) {
           uint8_t* dst = sm + SM::kV + vs * SM::kVStage;
-          if (MODE == MODE_Q) {
-            mbar_arrive_expect_tx(&bars[B_VFULL + vs], kD * kN);
-            tma_load_2d(dst, &a.tm_vq, t * kN, bh * kD, &bars[B_VFULL + vs]);
-          } else {
+          if (MODE == MODE_Q) {  // int8 V^T: D channels x 64 keys in one box
+            mbar_arrive_expect_tx(&bars[B_VFULL + vs], D * kN);
+            tma_load_2d(dst, &a.tm_vq, t * kN, bh * D, &bars[B_VFULL + vs]);
+          } else {  // bf16 V: one [64 keys][64 channels] box per panel (+ the residual panels)
             mbar_arrive_expect_tx(&bars[B_VFULL + vs], SM::kVStage);
-            tma_load_2d(dst, &a.tm_v, 0, bh * a.n + t * kN, &bars[B_VFULL + vs]);
-            if (VF32) tma_load_2d(dst + kN * kD * 2, &a.tm_vlo, 0, bh * a.n + t * kN, &bars[B_VFULL + vs]);
+#pragma unroll
+            for (int pn = 0; pn < kPan; ++pn) {
+              tma_load_2d(dst + pn * kN * 128, &a.tm_v, 64 * pn, bh * a.n + t * kN, &bars[B_VFULL + vs]);
+              if (VF32)
+                tma_load_2d(dst + kN * D * 2 + pn * kN * 128, &a.tm_vlo, 64 * pn, bh * a.n + t * kN,
+                            &bars[B_VFULL + vs]);
+            }
           }
           v_par[vs] = (int)((g_v / kVStages) & 1);
         }
@@ -447,8 +506,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
           if (!k_res && lane == 0 && g_k >= (uint32_t)kKStages)
             bounded_wait(B_KEMPTY + st, ((g_k / kKStages) - 1) & 1);
           if (lane == 0 && !*abort_flag) {
-            mbar_arrive_expect_tx(&bars[B_KFULL + st], kN * kD);
-            tma_load_2d(sm + SM::kK + st * kN * kD, &a.tm_k, 0, bh * a.n_pad + t * kN, &bars[B_KFULL + st]);
+            load_k(st, t);
             k_par[st] = k_res ? 0 : (int)((g_k / kKStages) & 1);
           }
           ++g_k;
@@ -462,18 +520,33 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
     // ============================================================== MMA issuer warp (one thread)
     else if (warp == kMmaWarp) {
       if (lane == 0) {
-        const uint32_t id_s = idesc_i8(kM, kN, true, true, false);
-        const uint32_t id_pv = (MODE == MODE_Q) ? idesc_i8(kM, kD, false, true, false) : idesc_bf16(kM, kD, true);
+        // scores: +-1 int8 (kind::i8), or bf16 Q x bf16 K (kind::f16) in the comparison mode
+        const uint32_t id_s = kRef ? idesc_bf16(kM, kN, false) : idesc_i8(kM, kN, true, true, false);
+        if (kRef && first_pass) bounded_wait(B_QFULL, 0);
+        // P.V: uint8 codes x int8 V^T (N = D, one MMA per K-step), or bf16 P x bf16 V
+        // (N = 64 per 64-channel panel)
+        const uint32_t id_pv = (MODE == MODE_Q) ? idesc_i8(kM, D, false, true, false) : idesc_bf16(kM, 64, true);
         auto issue_scores = [&](int t) {
           const uint32_t gk = g_k + (uint32_t)t, buf = (g_s + (uint32_t)t) % kSBufs;
           const uint32_t st = k_res ? (uint32_t)t : gk % kKStages;
           if (!bounded_wait(B_KFULL + st, k_res ? 0u : (gk / kKStages) & 1)) return;
           tc_fence_after();
-          const uint32_t kq = smem_u32(sQ), kk = smem_u32(sm + SM::kK + st * kN * kD);
+          const uint32_t kq = smem_u32(sQ), kk = smem_u32(sm + SM::kK + st * kN * D * SM::kOpB);
+          if (kRef) {
 #pragma unroll
-          for (int ks = 0; ks < 2; ++ks)
-            mma_i8_ss(tmem + kColS + buf * kN, sdesc(kq + 32 * ks, 16, 512, kSwizzle64B),
-                      sdesc(kk + 32 * ks, 16, 512, kSwizzle64B), id_s, ks > 0 ? 1u : 0u);
+            for (int pn = 0; pn < kPan; ++pn)  // four 16-channel K-steps per 64-channel bf16 panel
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks)
+                mma_f16_ss(tmem + kColS + buf * kN, sdesc(kq + pn * kM * 128 + 32 * ks, 16, 1024, kSwizzle128B),
+                           sdesc(kk + pn * kN * 128 + 32 * ks, 16, 1024, kSwizzle128B), id_s, (pn | ks) > 0 ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int pn = 0; pn < kPan; ++pn)  // two 32-channel K-steps per 64-channel panel
+#pragma unroll
+              for (int ks = 0; ks < 2; ++ks)
+                mma_i8_ss(tmem + kColS + buf * kN, sdesc(kq + pn * kM * 64 + 32 * ks, 16, 512, kSwizzle64B),
+                          sdesc(kk + pn * kN * 64 + 32 * ks, 16, 512, kSwizzle64B), id_s, (pn | ks) > 0 ? 1u : 0u);
+          }
           mma_commit(&bars[B_SFULL + buf]);
           if (!k_res) mma_commit(&bars[B_KEMPTY + st]);
         };
@@ -495,20 +568,23 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
                             (t > 0 || k > 0) ? 1u : 0u);
               } else {
 #pragma unroll
-                for (int k = 0; k < kN / 16; ++k)  // 16 keys per K-step: chunk k/2, columns 32(k/2) + 8(k%2)
-                  mma_f16_ts(tmem + kColO, tmem + colP + pcol(k), sdesc(vbase + 2048 * k, 0, 1024, kSwizzle128B), id_pv,
-                             (t > 0 || k > 0) ? 1u : 0u);
-                if (VF32) {
-                  // residual products: P_hi x V_lo and P_lo x V_hi
-                  const uint32_t vlo = vbase + kN * kD * 2;
+                for (int pn = 0; pn < kPan; ++pn) {  // O columns [64 pn, 64 pn + 64) from V panel pn
+                  const uint32_t vp = vbase + pn * kN * 128, op = tmem + kColO + 64 * pn;
 #pragma unroll
-                  for (int k = 0; k < kN / 16; ++k)
-                    mma_f16_ts(tmem + kColO, tmem + colP + pcol(k), sdesc(vlo + 2048 * k, 0, 1024, kSwizzle128B), id_pv,
-                               1u);
+                  for (int k = 0; k < kN / 16; ++k)  // 16 keys per K-step: chunk k/2, columns 32(k/2) + 8(k%2)
+                    mma_f16_ts(op, tmem + colP + pcol(k), sdesc(vp + 2048 * k, 0, 1024, kSwizzle128B), id_pv,
+                               (t > 0 || k > 0) ? 1u : 0u);
+                  if (VF32) {
+                    // residual products: P_hi x V_lo and P_lo x V_hi
+                    const uint32_t vlo = vbase + kN * D * 2 + pn * kN * 128;
 #pragma unroll
-                  for (int k = 0; k < kN / 16; ++k)
-                    mma_f16_ts(tmem + kColO, tmem + colP + pcol(k) + 16, sdesc(vbase + 2048 * k, 0, 1024, kSwizzle128B),
-                               id_pv, 1u);
+                    for (int k = 0; k < kN / 16; ++k)
+                      mma_f16_ts(op, tmem + colP + pcol(k), sdesc(vlo + 2048 * k, 0, 1024, kSwizzle128B), id_pv, 1u);
+#pragma unroll
+                    for (int k = 0; k < kN / 16; ++k)
+                      mma_f16_ts(op, tmem + colP + pcol(k) + 16, sdesc(vp + 2048 * k, 0, 1024, kSwizzle128B), id_pv,
+                                 1u);
+                  }
                 }
               }
               mma_commit(&bars[B_VEMPTY + vs]);
@@ -528,13 +604,13 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
       const uint32_t hist_row = smem_u32(hist) + (uint32_t)srow * 4u;
       const float mo = -m * kLog2e;
       const float* lut = reinterpret_cast<const float*>(hist);
-      const float* lut_lane = lut + 32 * 32 + lane;  // dense level table: entry for score s at lut_lane[-16 s]
-      // this row's weight table (top-N without a bias): level (64 - s) / 2 at
-      // lut[(32 - s / 2) kM + srow], i.e. byte (32 kM + srow) * 4 - s * 2 kM (s is even)
-      const char* wrow = reinterpret_cast<const char*>(lut + 32 * kM + srow);
+      const float* lut_lane = lut + (D / 2) * 32 + lane;  // dense level table: entry for score s at lut_lane[-16 s]
+      // this row's weight table (top-N without a bias): level (d - s) / 2 at
+      // lut[(d/2 - s / 2) kM + srow], i.e. byte (d/2 kM + srow) * 4 - s * 2 kM (s is even)
+      const char* wrow = reinterpret_cast<const char*>(lut + (D / 2) * kM + srow);
       // Passes compiled into this instantiation (the rest are pruned at compile time).
-      constexpr bool kHasLevels = SEL != SEL_DENSE;
-      constexpr bool kHasNorm = SEL == SEL_DENSE;
+      constexpr bool kHasLevels = !kDense;
+      constexpr bool kHasNorm = kDense;
       constexpr bool kHasRadix = SEL == SEL_TOPN_FLOAT;
       constexpr bool kHasKeptNorm = SEL == SEL_TOPN_FLOAT && (MODE == MODE_Q || EXPORT == EXP_CODES);
       constexpr bool kHasIdx = EXPORT == EXP_IDX;
@@ -542,14 +618,14 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
       constexpr bool kHasPv = EXPORT == EXP_NONE;
       // lut_e: dense weights from the level table x exp(bias - b_max) (no row max needed)
       // lut_w: top-N (no bias) weights from the row's level table, zero below the threshold
-      const bool lut_e = (SEL == SEL_DENSE) && use_lut && (pass == P_NORM || pass == P_PV || pass == P_CODES);
+      const bool lut_e = (kDense) && use_lut && (pass == P_NORM || pass == P_PV || pass == P_CODES);
       const bool lut_w = (SEL == SEL_TOPN_INT) && a.int_levels && pass == P_PV;
       const bool wants_bias = HAS_BIAS && pass != P_LEVELS;
       // exp(b - b_max) of this row (dense): row base rb(i) into the staged or global table
       // (key offsets are kept in bytes: entry (i, j) sits at row base - koff_bytes(j))
       const char* eb_bytes = nullptr;
       if (BIAS == BIAS_SMEM) eb_bytes = reinterpret_cast<const char*>(reinterpret_cast<const float*>(sm + SM::kBiasTab) + rb);
-      else if (HAS_BIAS && SEL == SEL_DENSE) eb_bytes = reinterpret_cast<const char*>(a.expb + (size_t)h * a.ext_E + rb);
+      else if (HAS_BIAS && kDense) eb_bytes = reinterpret_cast<const char*>(a.expb + (size_t)h * a.ext_E + rb);
       const char* tab_bytes = HAS_BIAS ? reinterpret_cast<const char*>(tab + rb) : nullptr;
       // a warp whose 32 rows all lie past L only keeps the barrier phases going
       const bool warp_live = __any_sync(0xffffffffu, row < L);
@@ -590,7 +666,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
         rw_xw = r0 - rw_yw * a.gw;
         rw_slice0 = reinterpret_cast<float*>(koff_tab) + warp * 2 * kRwEnt;
         // dense weights read exp(b - b_max) (the level-table path), the rest the bias itself
-        rw_src = ((SEL == SEL_DENSE && use_lut) ? a.expb : a.bext) + (size_t)h * a.ext_E + rw_first;
+        rw_src = ((kDense && use_lut) ? a.expb : a.bext) + (size_t)h * a.ext_E + rw_first;
       }
       auto rw_fetch = [&](int tt) {  // tile tt's window into registers (coalesced loads)
         const int jt = tt * kN, yk = jt / a.gw, xk = jt - yk * a.gw;
@@ -649,7 +725,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
         const int nvalid = row_ok ? max(0, min(kN, L - j0)) : 0;
         // Dense with bias: keys past L carry the k_invalid offset (weight 0), and
         // rows past L are never stored, so every tile takes the unmasked path.
-        constexpr bool kMaskInKoff = SEL == SEL_DENSE && HAS_BIAS && BIAS != BIAS_ROWS;
+        constexpr bool kMaskInKoff = kDense && HAS_BIAS && BIAS != BIAS_ROWS;
         const bool full_tile = kMaskInKoff || __all_sync(0xffffffffu, nvalid == kN);
 
         // bias offsets of keys 32*ch+u .. +3 of this tile
@@ -719,7 +795,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
               continue;
             }
             if (kHasLevels && pass == P_LEVELS) {
-              const uint32_t base = hist_row + 32u * kM * 4u;  // level (64 - s)/2 -> + (64 - s) * 256 bytes
+              const uint32_t base = hist_row + (uint32_t)(D / 2) * kM * 4u;  // level (d - s)/2: + (d - s) * 256 B
 #pragma unroll
               for (int u = 0; u < 32; ++u) {
                 const uint32_t ad = base - (uint32_t)((int)r[32 * cc + u] * (kM * 2));
@@ -732,7 +808,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
                       : "memory");
                 }
               }
-            } else if (SEL == SEL_DENSE && lut_e) {
+            } else if (kDense && lut_e) {
               float e[32];
 #pragma unroll
               for (int u = 0; u < 32; u += 4) {
@@ -790,14 +866,16 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
 #pragma unroll
                 for (int v = 0; v < 4; ++v) {
                   const int sc = (int)r[32 * cc + u + v];
+                  // the score as a float: the integer count, or the comparison mode's fp32 dot product
+                  const float sf = kRef ? __uint_as_float(r[32 * cc + u + v]) : (float)sc;
                   float l;
                   if (HAS_BIAS) {
                     if (kMaskInKoff) kinv |= (kk[v] == 4 * a.k_invalid ? 1u : 0u) << (u + v);
                     const float bv = (BIAS == BIAS_ROWS) ? brow[-(32 * cc + u + v)]
                                                          : __ldg(reinterpret_cast<const float*>(tab_bytes - kk[v]));
-                    l = __fmaf_rn((float)sc, c, bv);
+                    l = __fmaf_rn(sf, c, bv);
                   } else {
-                    l = (float)sc * c;
+                    l = sf * c;
                   }
                   lg[u + v] = (FULL || 32 * ch + u + v < nvalid) ? l : -INFINITY;
                 }
@@ -901,7 +979,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
                 for (int u = 0; u < 32; ++u) {
                   const bool valid = FULL || 32 * ch + u < nvalid;
                   bool k;
-                  if (SEL == SEL_DENSE) {
+                  if (kDense) {
                     k = valid && !((kinv >> u) & 1u);
                   } else {
                     const bool gt = valid && lg[u] > F, eq = valid && lg[u] == F;
@@ -919,7 +997,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
                 } else if (kHasIdx && pass == P_IDX) {
                   if (row_ok) {
                     int32_t* dst = a.idx + ((size_t)bh * a.n + row) * a.N;
-                    if (SEL == SEL_DENSE) {
+                    if (kDense) {
                       // dense: every key below L is kept, so key j is the j-th kept index
 #pragma unroll
                       for (int u = 0; u < 32; ++u)
@@ -1040,30 +1118,26 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
     }
     if (tid < kM && row_ok && !*abort_flag) {
       if (pass == P_LEVELS) {
-        int cnt[kLevels];
-#pragma unroll
-        for (int lev = 0; lev < kLevels; ++lev) cnt[lev] = (int)hist[lev * kM + srow];
-        int hmin = 64, hN = 64, cum = 0;
+        auto cnt = [&](int lev) -> int { return (int)hist[lev * kM + srow]; };  // level (d - s) / 2
+        int hmin = D, hN = D, cum = 0;
         bool found = false;
-#pragma unroll
-        for (int lev = kLevels - 1; lev >= 0; --lev) hmin = cnt[lev] > 0 ? lev : hmin;
-#pragma unroll
+        for (int lev = kLevels - 1; lev >= 0; --lev) hmin = cnt(lev) > 0 ? lev : hmin;
         for (int lev = 0; lev < kLevels; ++lev) {
-          cum += cnt[lev];
+          cum += cnt(lev);
           if (!found && cum >= keff) { hN = lev; found = true; }
         }
-        const int smax = 64 - 2 * hmin, sN = 64 - 2 * hN;
+        const int smax = D - 2 * hmin, sN = D - 2 * hN;
         if (SEL == SEL_TOPN_INT) {
           F = (float)sN * c;
           m = (float)smax * c;
           int gt = 0, eq = 0;
           float ls = 0.0f;
-#pragma unroll
           for (int lev = 0; lev < kLevels; ++lev) {
-            const float lv = (float)(64 - 2 * lev) * c;
-            gt += (lv > F) ? cnt[lev] : 0;
-            eq += (lv == F) ? cnt[lev] : 0;
-            ls += (lv > F) ? (float)cnt[lev] * fast_exp2((lv - m) * kLog2e) : 0.0f;
+            const float lv = (float)(D - 2 * lev) * c;
+            const int k = cnt(lev);
+            gt += (lv > F) ? k : 0;
+            eq += (lv == F) ? k : 0;
+            ls += (lv > F) ? (float)k * fast_exp2((lv - m) * kLog2e) : 0.0f;
           }
           rF = keff - gt;
           cut = rF < eq ? 1 : 0;
@@ -1072,9 +1146,8 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
           sF = sN;
           // this row's weight per level: exp(l - m) above the threshold, the tie weight at it, 0 below
           float* wt = reinterpret_cast<float*>(hist);
-#pragma unroll
           for (int lev = 0; lev < kLevels; ++lev) {
-            const float lv = (float)(64 - 2 * lev) * c;
+            const float lv = (float)(D - 2 * lev) * c;
             wt[lev * kM + srow] = (lv >= F) ? fast_exp2((lv - m) * kLog2e) : 0.0f;
           }
         } else {
@@ -1278,99 +1351,109 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
   }
   if (EXPORT == EXP_NONE) {
     if (is_soft) {
-      constexpr int kOc = kD / kSplit;               // output channels per softmax thread
+      constexpr int kOc = D / kSplit;                 // output channels per softmax thread
       const int c0 = (kSplit == 2) ? kOc * half : 0;  // first channel
       const bool ok = __all_sync(0xffffffffu, bounded_wait(B_OFULL, 0));
       tc_fence_after();
       const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-      uint32_t o[kOc];
-      tmem_ld32(tl + kColO + c0, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
-      if (kOc == 64) tmem_ld32(tl + kColO + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[kOc - 32]));
-      tmem_wait_ld();
-      if (row < a.n) {
-        float out[kOc];
-        if (!ok || !row_ok) {
+      // the final radix bin of this row (kMerge): logits of its recorded keys from the
+      // same integer score (+-1 codes, exact) and bias entry as in the tiles, the
+      // r_rank-th largest as threshold with its ties kept in key order; each kept key's
+      // weight goes to the normalizer and replaces its logit in slot kCap + x (0 for a
+      // dropped key), and its V row is added to O below, 32 channels at a time
+      int n_merge = 0;
+      const float* pw = reinterpret_cast<const float*>(hist) + kCap * kM + srow;  // weight x at pw[x * kM]
+      if (kMerge && r_state == 3 && ok && row_ok && row < a.n) {
+        n_merge = min(r_cnt, kCap);
+        if (r_cnt > kCap) raise_status(a.status, kDevErrCapacity);
+        const int8_t* kb = a.kpm + (size_t)bh * a.n_pad * D;
+        for (int x = 0; x < n_merge; ++x) {
+          const int j = (int)hist[x * kM + srow];
+          const uint4* kr = reinterpret_cast<const uint4*>(kb + (size_t)j * D);
+          int sc = 0;
 #pragma unroll
-          for (int k = 0; k < kOc; ++k) out[k] = 0.0f;
-        } else if (MODE == MODE_Q) {
-#pragma unroll
-          for (int k = 0; k < kOc; ++k) out[k] = (float)(int)o[k] * dq[c0 + k];
-        } else {
-#pragma unroll
-          for (int k = 0; k < kOc; ++k) out[k] = __uint_as_float(o[k]);
-          if (kMerge && r_state == 3) {
-            // the final radix bin of this row: logits of its recorded keys from the same
-            // integer score (+-1 codes, exact) and bias entry as in the tiles, the
-            // r_rank-th largest as threshold with its ties kept in key order, and the
-            // kept keys' weights and V rows added to the normalizer and to O
-            const int nc = min(r_cnt, kCap);
-            if (r_cnt > kCap) raise_status(a.status, kDevErrCapacity);
-            uint4 qv[4];
-#pragma unroll
-            for (int cch = 0; cch < 4; ++cch)
-              qv[cch] = *reinterpret_cast<const uint4*>(sQ + srow * kD + ((cch ^ ((srow >> 1) & 3)) * 16));
-            const int8_t* kb = a.kpm + (size_t)bh * a.n_pad * kD;
-            for (int x = 0; x < nc; ++x) {
-              const int j = (int)hist[x * kM + srow];
-              const uint4* kr = reinterpret_cast<const uint4*>(kb + (size_t)j * kD);
-              int sc = 0;
-#pragma unroll
-              for (int cch = 0; cch < 4; ++cch) {
-                const uint4 kv = __ldg(kr + cch);
-                sc = __dp4a((int)qv[cch].x, (int)kv.x, sc);
-                sc = __dp4a((int)qv[cch].y, (int)kv.y, sc);
-                sc = __dp4a((int)qv[cch].z, (int)kv.z, sc);
-                sc = __dp4a((int)qv[cch].w, (int)kv.w, sc);
-              }
-              float l;
-              if (HAS_BIAS) {
-                int off;  // entry (i, j) of the extended table sits at rb - off
-                if (a.bias_dense) {
-                  off = -j;
-                } else if (j < a.prefix) {
-                  off = a.k_class;
-                } else {
-                  const int t = j - a.prefix, y = t / a.gw;
-                  off = y * a.ext_S + (t - y * a.gw);
-                }
-                l = __fmaf_rn((float)sc, c, __ldg(tab + rb - off));
-              } else {
-                l = (float)sc * c;
-              }
-              hist[(kCap + x) * kM + srow] = __float_as_uint(l);
+          for (int c16 = 0; c16 < D / 16; ++c16) {
+            const uint4 qv = *reinterpret_cast<const uint4*>(sQ + (c16 >> 2) * kM * 64 + srow * 64 +
+                                                             (((c16 & 3) ^ ((srow >> 1) & 3)) * 16));
+            const uint4 kv = __ldg(kr + c16);
+            sc = __dp4a((int)qv.x, (int)kv.x, sc);
+            sc = __dp4a((int)qv.y, (int)kv.y, sc);
+            sc = __dp4a((int)qv.z, (int)kv.z, sc);
+            sc = __dp4a((int)qv.w, (int)kv.w, sc);
+          }
+          float l;
+          if (HAS_BIAS) {
+            int off;  // entry (i, j) of the extended table sits at rb - off
+            if (a.bias_dense) {
+              off = -j;
+            } else if (j < a.prefix) {
+              off = a.k_class;
+            } else {
+              const int t = j - a.prefix, y = t / a.gw;
+              off = y * a.ext_S + (t - y * a.gw);
             }
-            const float* lc = reinterpret_cast<const float*>(hist) + kCap * kM + srow;  // logit x at lc[x * kM]
-            float vF = INFINITY;
-            int gt = 0;
-            for (int x = 0; x < nc; ++x) {
-              const float vx = lc[x * kM];
-              int g = 0, e = 0;
-              for (int y = 0; y < nc; ++y) {
-                const float vy = lc[y * kM];
-                g += vy > vx ? 1 : 0;
-                e += vy == vx ? 1 : 0;
-              }
-              if (g < r_rank && r_rank <= g + e) {
-                vF = vx;
-                gt = g;
-                break;
-              }
-            }
-            int allow = r_rank - gt;  // keys at the threshold still kept, in key order
-            const float mo_e = -m * kLog2e;
-            for (int x = 0; x < nc; ++x) {
-              const float v = lc[x * kM];
-              const bool at = v == vF;
-              if (!(v > vF || (at && allow > 0))) continue;
-              allow -= at ? 1 : 0;
-              const int j = (int)hist[x * kM + srow];
-              const float p = fast_exp2(__fmaf_rn(v, kLog2e, mo_e));
-              lsum += p;
-              const size_t vrow = (size_t)bh * a.n + j;
+            l = __fmaf_rn((float)sc, c, __ldg(tab + rb - off));
+          } else {
+            l = (float)sc * c;
+          }
+          hist[(kCap + x) * kM + srow] = __float_as_uint(l);
+        }
+        float* lc = reinterpret_cast<float*>(hist) + kCap * kM + srow;  // logit x at lc[x * kM]
+        float vF = INFINITY;
+        int gt = 0;
+        for (int x = 0; x < n_merge; ++x) {
+          const float vx = lc[x * kM];
+          int g = 0, e = 0;
+          for (int y = 0; y < n_merge; ++y) {
+            const float vy = lc[y * kM];
+            g += vy > vx ? 1 : 0;
+            e += vy == vx ? 1 : 0;
+          }
+          if (g < r_rank && r_rank <= g + e) {
+            vF = vx;
+            gt = g;
+            break;
+          }
+        }
+        int allow = r_rank - gt;  // keys at the threshold still kept, in key order
+        const float mo_e = -m * kLog2e;
+        for (int x = 0; x < n_merge; ++x) {
+          const float v = lc[x * kM];
+          const bool at = v == vF;
+          float p = 0.0f;
+          if (v > vF || (at && allow > 0)) {
+            allow -= at ? 1 : 0;
+            p = fast_exp2(__fmaf_rn(v, kLog2e, mo_e));
+            lsum += p;
+          }
+          lc[x * kM] = p;
+        }
+      }
+      const float inv = sum_in_pv ? 1.0f / lsum : scale;
+#pragma unroll
+      for (int cb = 0; cb < kOc; cb += 32) {
+        uint32_t o[32];
+        tmem_ld32(tl + kColO + c0 + cb, o);
+        tmem_wait_ld();
+        if (row < a.n) {
+          float out[32];
+          if (!ok || !row_ok) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) out[k] = 0.0f;
+          } else if (MODE == MODE_Q) {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) out[k] = (float)(int)o[k] * dq[c0 + cb + k];
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) out[k] = __uint_as_float(o[k]);
+            for (int x = 0; x < n_merge; ++x) {  // kept keys of the final bin: p * V[j][channels]
+              const float p = pw[x * kM];
+              if (p == 0.0f) continue;
+              const size_t vrow = (size_t)bh * a.n + (int)hist[x * kM + srow];
               if (a.v_f32) {
-                const float4* vr = reinterpret_cast<const float4*>(a.v_raw) + vrow * (kD / 4);
+                const float4* vr = reinterpret_cast<const float4*>(a.v_raw) + (vrow * D + c0 + cb) / 4;
 #pragma unroll
-                for (int q = 0; q < kD / 4; ++q) {
+                for (int q = 0; q < 8; ++q) {
                   const float4 f = __ldg(vr + q);
                   out[4 * q] = __fmaf_rn(p, f.x, out[4 * q]);
                   out[4 * q + 1] = __fmaf_rn(p, f.y, out[4 * q + 1]);
@@ -1378,9 +1461,9 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
                   out[4 * q + 3] = __fmaf_rn(p, f.w, out[4 * q + 3]);
                 }
               } else {
-                const uint4* vr = reinterpret_cast<const uint4*>(a.v_raw) + vrow * (kD / 8);
+                const uint4* vr = reinterpret_cast<const uint4*>(a.v_raw) + (vrow * D + c0 + cb) / 8;
 #pragma unroll
-                for (int q = 0; q < kD / 8; ++q) {
+                for (int q = 0; q < 4; ++q) {
                   const uint4 u4 = __ldg(vr + q);
                   const uint32_t wv[4] = {u4.x, u4.y, u4.z, u4.w};
 #pragma unroll
@@ -1391,29 +1474,28 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), 2) k_attn_tc(const __grid_
                 }
               }
             }
+#pragma unroll
+            for (int k = 0; k < 32; ++k) out[k] *= inv;
           }
-          const float inv = sum_in_pv ? 1.0f / lsum : scale;
+          const size_t ob = ((size_t)bh * a.n + row) * D + c0 + cb;
+          if (a.o_bf16) {
+            uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.O) + ob);
 #pragma unroll
-          for (int k = 0; k < kOc; ++k) out[k] *= inv;
-        }
-        const size_t ob = ((size_t)bh * a.n + row) * kD + c0;
-        if (a.o_bf16) {
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(a.O) + ob);
+            for (int k = 0; k < 4; ++k)
+              dst[k] = make_uint4(pack_bf16x2(out[8 * k], out[8 * k + 1]), pack_bf16x2(out[8 * k + 2], out[8 * k + 3]),
+                                  pack_bf16x2(out[8 * k + 4], out[8 * k + 5]), pack_bf16x2(out[8 * k + 6], out[8 * k + 7]));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.O) + ob);
 #pragma unroll
-          for (int k = 0; k < kOc / 8; ++k)
-            dst[k] = make_uint4(pack_bf16x2(out[8 * k], out[8 * k + 1]), pack_bf16x2(out[8 * k + 2], out[8 * k + 3]),
-                                pack_bf16x2(out[8 * k + 4], out[8 * k + 5]), pack_bf16x2(out[8 * k + 6], out[8 * k + 7]));
-        } else {
-          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(a.O) + ob);
-#pragma unroll
-          for (int k = 0; k < kOc / 4; ++k) dst[k] = make_float4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
+            for (int k = 0; k < 8; ++k) dst[k] = make_float4(out[4 * k], out[4 * k + 1], out[4 * k + 2], out[4 * k + 3]);
+          }
         }
       }
     }
   } else if (EXPORT == EXP_IDX) {
     if (tid < kM && row < a.n) {
       int32_t* dst = a.idx + ((size_t)bh * a.n + row) * a.N;
-      for (int p = row_ok ? min(SEL == SEL_DENSE ? L : kept_seen, a.N) : 0; p < a.N; ++p) dst[p] = -1;
+      for (int p = row_ok ? min(kDense ? L : kept_seen, a.N) : 0; p < a.N; ++p) dst[p] = -1;
     }
   } else if (EXPORT == EXP_SCORES) {
     if (tid < kM && row < a.n) {

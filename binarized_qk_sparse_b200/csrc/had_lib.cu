@@ -23,13 +23,31 @@
 #include "common.cuh"
 #include "prep.cuh"
 #include "attn.cuh"
-#include "dense_ref.cuh"
 #include "attn_tc.cuh"
+#include "launch.cuh"
 #include "probe.cuh"
 
 namespace had {
 
 __device__ unsigned g_device_status;
+
+namespace {
+thread_local char t_last_error[256] = "";
+}  // namespace
+
+had_status cuda_fail(cudaError_t e, const char* what) {
+  snprintf(t_last_error, sizeof(t_last_error), "%s: %s", what, cudaGetErrorString(e));
+  return HAD_ERR_CUDA;
+}
+
+had_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? HAD_OK : cuda_fail(e, what);
+}
+
+// d = 64 is instantiated here, d = 128 in attn_d128.cu
+HAD_DISPATCH_INST(, 64)
+HAD_DISPATCH_INST(extern, 128)
 
 namespace {
 
@@ -40,8 +58,6 @@ using tc::EXP_NONE;
 using tc::EXP_IDX;
 using tc::EXP_CODES;
 
-constexpr int kMaxDevices = 64;
-thread_local char t_last_error[256] = "";
 // bound of the fused kernel's pipeline waits and the timeout-path test hook
 // (had_debug_bounded_wait); library-wide, read at each launch
 std::atomic<long long> g_wait_cycles{tc::kWaitCycles};
@@ -60,36 +76,29 @@ unsigned* status_ptr(int dev) {
   return ptrs[dev];
 }
 
-had_status cuda_fail(cudaError_t e, const char* what) {
-  snprintf(t_last_error, sizeof(t_last_error), "%s: %s", what, cudaGetErrorString(e));
-  return HAD_ERR_CUDA;
-}
-
-had_status check_launch(const char* what) {
-  cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? HAD_OK : cuda_fail(e, what);
-}
 
 inline size_t align_up(size_t x, size_t a = 256) { return (x + a - 1) / a * a; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 struct Dims {
-  int B, H, n, BH, nchunks, n_pad;
+  int B, H, n, d, BH, nchunks, n_pad;
 };
 
 Dims dims_of(const had_shape* s) {
   Dims d;
-  d.B = s->B; d.H = s->H; d.n = s->n; d.BH = s->B * s->H;
+  d.B = s->B; d.H = s->H; d.n = s->n; d.d = s->d; d.BH = s->B * s->H;
   d.nchunks = (s->n + kChunk - 1) / kChunk;
   d.n_pad = d.nchunks * kChunk;
   return d;
 }
 
-had_status check_shape(const had_shape* s) {
+// Head dims: 64 and 128 everywhere; 32 also in the pack and int8-V entry points.
+had_status check_shape(const had_shape* s, bool allow_d32 = false) {
   if (!s) return HAD_ERR_INVALID;
   if (s->B <= 0 || s->H <= 0 || s->n <= 0 || s->d <= 0) return HAD_ERR_INVALID;
   if (s->in_dtype != HAD_F32 && s->in_dtype != HAD_BF16) return HAD_ERR_INVALID;
-  if (s->d != kD || s->n > kMaxN || s->H > kMaxHeads || (long long)s->B * s->H > 65535) return HAD_ERR_UNSUPPORTED;
+  const bool d_ok = s->d == 64 || s->d == 128 || (allow_d32 && s->d == 32);
+  if (!d_ok || s->n > kMaxN || s->H > kMaxHeads || (long long)s->B * s->H > 65535) return HAD_ERR_UNSUPPORTED;
   if (s->seqlens && (reinterpret_cast<uintptr_t>(s->seqlens) & 3u)) return HAD_ERR_INVALID;
   return HAD_OK;
 }
@@ -116,14 +125,14 @@ Ws ws_layout(const had_shape* s, bool quant, const had_relpos_bias* bias_desc) {
   Dims d = dims_of(s);
   Ws w{};
   size_t off = 0;
-  w.qbits = off; off += align_up((size_t)d.BH * d.n * kW * 4);
-  w.kpm = off; off += align_up((size_t)d.BH * d.n_pad * kD);
-  w.sums = off; off += align_up((size_t)2 * d.BH * d.nchunks * kD * 8);
+  w.qbits = off; off += align_up((size_t)d.BH * d.n * (d.d / 32) * 4);
+  w.kpm = off; off += align_up((size_t)d.BH * d.n_pad * d.d);
+  w.sums = off; off += align_up((size_t)2 * d.BH * d.nchunks * d.d * 8);
   w.amax = w.vqT = w.vscale = w.bminmax = 0;
   if (quant) {
-    w.amax = off; off += align_up((size_t)d.BH * d.nchunks * kD * 4);
-    w.vqT = off; off += align_up((size_t)d.BH * kD * d.n_pad);
-    w.vscale = off; off += align_up((size_t)d.BH * kD * 4);
+    w.amax = off; off += align_up((size_t)d.BH * d.nchunks * d.d * 4);
+    w.vqT = off; off += align_up((size_t)d.BH * d.d * d.n_pad);
+    w.vscale = off; off += align_up((size_t)d.BH * d.d * 4);
   }
   w.bext = w.expb = 0;
   if (bias) {
@@ -135,8 +144,8 @@ Ws ws_layout(const had_shape* s, bool quant, const had_relpos_bias* bias_desc) {
   w.vhi = w.vlo = 0;
   if (!quant && s->in_dtype == HAD_F32) {
     // fp32 V in float mode: bf16 head and residual copies for the tensor cores
-    w.vhi = off; off += align_up((size_t)d.BH * d.n * kD * 2);
-    w.vlo = off; off += align_up((size_t)d.BH * d.n * kD * 2);
+    w.vhi = off; off += align_up((size_t)d.BH * d.n * d.d * 2);
+    w.vlo = off; off += align_up((size_t)d.BH * d.n * d.d * 2);
   }
   w.total = off;
   return w;
@@ -189,15 +198,14 @@ had_status encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, u
   return HAD_OK;
 }
 
-__global__ void k_untranspose_vq(const int8_t* vqT, int BH, int n, int n_pad, const int32_t* seqlens, int H,
-                                 int8_t* Vq) {
-  const size_t total = (size_t)BH * n * kD;
+__global__ void k_untranspose_vq(const int8_t* vqT, int BH, int n, int d, int n_pad, int8_t* Vq) {
+  const size_t total = (size_t)BH * n * d;
   for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
-    const int c = (int)(e % kD);
-    const size_t ti = e / kD;
+    const int c = (int)(e % d);
+    const size_t ti = e / d;
     const int i = (int)(ti % n);
     const int bh = (int)(ti / n);
-    Vq[e] = vqT[((size_t)bh * kD + c) * n_pad + i];
+    Vq[e] = vqT[((size_t)bh * d + c) * n_pad + i];
   }
 }
 
@@ -215,9 +223,11 @@ had_status launch_prep(const had_shape* s, const void* X0, const void* X1, const
   pa.seqlens = s->seqlens; pa.sums = sums; pa.amax = amax; pa.status = status;
   dim3 grid(d.nchunks, d.BH, ntens);
   const bool need_stats = !(mu_in0 && first == 0 && ntens == 1);
+  const bool bf = s->in_dtype == HAD_BF16;
   if (need_stats) {
-    if (s->in_dtype == HAD_BF16) k_stats<__nv_bfloat16><<<grid, kPrepThreads, 0, st>>>(pa);
-    else k_stats<float><<<grid, kPrepThreads, 0, st>>>(pa);
+    if (d.d == 32) bf ? k_stats<__nv_bfloat16, 32><<<grid, kPrepThreads, 0, st>>>(pa) : k_stats<float, 32><<<grid, kPrepThreads, 0, st>>>(pa);
+    else if (d.d == 128) bf ? k_stats<__nv_bfloat16, 128><<<grid, kPrepThreads, 0, st>>>(pa) : k_stats<float, 128><<<grid, kPrepThreads, 0, st>>>(pa);
+    else bf ? k_stats<__nv_bfloat16, 64><<<grid, kPrepThreads, 0, st>>>(pa) : k_stats<float, 64><<<grid, kPrepThreads, 0, st>>>(pa);
     had_status r = check_launch("k_stats");
     if (r != HAD_OK) return r;
   }
@@ -231,8 +241,9 @@ had_status launch_prep(const had_shape* s, const void* X0, const void* X1, const
   ka.bits[0] = bits0; ka.bits[1] = bits1;
   ka.pm[0] = pm0; ka.pm[1] = pm1;
   ka.vqT = vqT; ka.vscale = vscale; ka.status = status;
-  if (s->in_dtype == HAD_BF16) k_pack<__nv_bfloat16><<<grid, kPrepThreads, 0, st>>>(ka);
-  else k_pack<float><<<grid, kPrepThreads, 0, st>>>(ka);
+  if (d.d == 32) bf ? k_pack<__nv_bfloat16, 32><<<grid, kPrepThreads, 0, st>>>(ka) : k_pack<float, 32><<<grid, kPrepThreads, 0, st>>>(ka);
+  else if (d.d == 128) bf ? k_pack<__nv_bfloat16, 128><<<grid, kPrepThreads, 0, st>>>(ka) : k_pack<float, 128><<<grid, kPrepThreads, 0, st>>>(ka);
+  else bf ? k_pack<__nv_bfloat16, 64><<<grid, kPrepThreads, 0, st>>>(ka) : k_pack<float, 64><<<grid, kPrepThreads, 0, st>>>(ka);
   return check_launch("k_pack");
 }
 
@@ -306,7 +317,7 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
   const bool do_v = quant && need_v;
   had_status r = HAD_OK;
   const size_t elem = (s->in_dtype == HAD_BF16) ? 2 : 4;
-  const size_t head_bytes = (size_t)s->n * kD * elem;
+  const size_t head_bytes = (size_t)s->n * s->d * elem;
   BiasArgs ba{};
   if (has_bias) {
     ba.table = bias->table;
@@ -325,7 +336,7 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
     k_dense_bias_tables<<<tgrid, 256, 0, st>>>(ba);
     if ((r = check_launch("k_dense_bias_tables")) != HAD_OK) return r;
   }
-  if (head_bytes <= (size_t)kHeadMaxBytes) {
+  if (s->d == 64 && head_bytes <= (size_t)kHeadMaxBytes) {
     // short heads: one read of each head, statistics and packing from shared memory
     HeadArgs ha{};
     ha.X[0] = Q; ha.X[1] = K; ha.X[2] = V;
@@ -356,7 +367,7 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
     }
   }
   if (!quant && s->in_dtype == HAD_F32 && need_v) {
-    const size_t count = (size_t)dims_of(s).BH * s->n * kD;
+    const size_t count = (size_t)dims_of(s).BH * s->n * s->d;
     k_split_v<<<1024, 256, 0, st>>>(static_cast<const float*>(V), count,
                                      reinterpret_cast<__nv_bfloat16*>(ws + w.vhi),
                                      reinterpret_cast<__nv_bfloat16*>(ws + w.vlo));
@@ -365,81 +376,78 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
   return HAD_OK;
 }
 
-template <int SEL, int MODE, int BIAS, bool VF32, int EXP, int SPLIT>
-had_status launch_tc_t(const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
-  const int smem = tc::Smem<SEL, VF32, BIAS>::kTotal;
-  auto fn = tc::k_attn_tc<SEL, MODE, BIAS, VF32, EXP, SPLIT>;
-  static std::mutex mu;
-  static bool configured[kMaxDevices] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  {
-    std::lock_guard<std::mutex> lk(mu);
-    if (dev >= 0 && dev < kMaxDevices && !configured[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_attn_tc)");
-      configured[dev] = true;
-    }
-  }
-  fn<<<grid, tc::cta_threads(SPLIT), smem, st>>>(a);
-  return check_launch("k_attn_tc");
+// Workspace of the comparison mode: the bias range and extended tables only.
+struct RefWs {
+  size_t bminmax, bext, expb, total;
+};
+
+RefWs ref_ws_layout(const had_shape* s, const had_relpos_bias* bias) {
+  RefWs w{};
+  if (!bias || !bias->table) return w;
+  const size_t cells = bias->dense ? (size_t)dense_ext(s->n).E : (size_t)relpos_ext(bias->gh, bias->gw).E;
+  size_t off = 0;
+  w.bminmax = off; off += align_up((size_t)s->H * 2 * 4);
+  w.bext = off; off += align_up((size_t)s->H * cells * 4);
+  w.expb = off; off += align_up((size_t)s->H * cells * 4);
+  w.total = off;
+  return w;
 }
 
-// Dense: no bias, extended tables in global memory, the exp(bias) table staged in
-// shared memory, or a dense bias matrix read 4 keys per load.
-template <int SEL, int MODE, bool VF32, int EXP>
-had_status launch_tc_b(int bias, const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
-  using namespace tc;
-  if (bias == BIAS_SMEM) return launch_tc_t<SEL, MODE, BIAS_SMEM, VF32, EXP, 2>(a, grid, st);
-  if (bias == BIAS_ROWS) return launch_tc_t<SEL, MODE, BIAS_ROWS, VF32, EXP, 2>(a, grid, st);
-  if (bias == BIAS_DGLOBAL) return launch_tc_t<SEL, MODE, BIAS_DGLOBAL, VF32, EXP, 2>(a, grid, st);
-  if (bias == BIAS_GLOBAL) return launch_tc_t<SEL, MODE, BIAS_GLOBAL, VF32, EXP, 2>(a, grid, st);
-  return launch_tc_t<SEL, MODE, BIAS_NONE, VF32, EXP, 2>(a, grid, st);
+// The bias range and extended tables of a relative-position table or a dense matrix.
+had_status build_bias_tables(const had_shape* s, const had_relpos_bias* bias, uint8_t* bminmax, uint8_t* bext,
+                             uint8_t* expb, cudaStream_t st) {
+  BiasArgs ba{};
+  ba.table = bias->table;
+  ba.gh = bias->gh; ba.gw = bias->gw; ba.prefix = bias->prefix;
+  ba.dense = bias->dense; ba.n = s->n;
+  if (ba.dense) { ba.gh = ba.gw = 1; ba.prefix = 0; }
+  ba.bminmax = reinterpret_cast<float*>(bminmax);
+  ba.bext = reinterpret_cast<float*>(bext);
+  ba.expb = reinterpret_cast<float*>(expb);
+  had_status r;
+  if (ba.dense) {
+    k_dense_bias_range<<<s->H, kDenseRangeThreads, 0, st>>>(ba);
+    if ((r = check_launch("k_dense_bias_range")) != HAD_OK) return r;
+    dim3 tgrid((dense_ext(s->n).E + kDenseTabPerCta - 1) / kDenseTabPerCta, s->H);
+    k_dense_bias_tables<<<tgrid, 256, 0, st>>>(ba);
+    return check_launch("k_dense_bias_tables");
+  }
+  k_bias_tables<<<s->H, 256, 0, st>>>(ba);
+  return check_launch("k_bias_tables");
 }
 
-// Top-N without a bias: two threads per row on the P.V path of short ragged rows
-// (per-sequence lengths, n <= 256), where a CTA's few tiles make it latency-bound;
-// on full-length rows the per-tile tie exchange costs more than the extra warps gain.
-template <int SEL, int MODE, bool VF32, int EXP>
-had_status launch_tc_n(const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
-  if (EXP == tc::EXP_NONE && a.n_pad <= tc::kSplitMaxKeys && a.seqlens != nullptr)
-    return launch_tc_t<SEL, MODE, tc::BIAS_NONE, VF32, EXP, (EXP == tc::EXP_NONE ? 2 : 1)>(a, grid, st);
-  return launch_tc_t<SEL, MODE, tc::BIAS_NONE, VF32, EXP, 1>(a, grid, st);
-}
-
-// Top-N with a bias: per-warp bias windows in shared memory (relative-position
-// tables on grids with rows of a multiple of 64 patches and no class tokens), or
-// gathers from the extended table in global memory.
-template <int MODE, bool VF32, int EXP>
-had_status launch_tc_f(bool rows, const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
-  if (rows) return launch_tc_t<tc::SEL_TOPN_FLOAT, MODE, tc::BIAS_ROWS, VF32, EXP, 1>(a, grid, st);
-  return launch_tc_t<tc::SEL_TOPN_FLOAT, MODE, tc::BIAS_GLOBAL, VF32, EXP, 1>(a, grid, st);
-}
-
-template <int EXP>
-had_status dispatch_tc(int sel, int mode, int bias, bool vf32, bool rows, const tc::TcArgs& a, dim3 grid,
-                       cudaStream_t st) {
-  using namespace tc;
-  if (EXP == EXP_SCORES) return launch_tc_t<SEL_DENSE, MODE_F, BIAS_NONE, false, EXP_SCORES, 1>(a, grid, st);
-  if (EXP == EXP_CODES || (EXP == EXP_NONE && mode == MODE_Q)) {
-    constexpr int E = EXP;
-    if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_Q, false, E>(bias, a, grid, st);
-    if (sel == SEL_TOPN_INT) return launch_tc_n<SEL_TOPN_INT, MODE_Q, false, E>(a, grid, st);
-    return launch_tc_f<MODE_Q, false, E>(rows, a, grid, st);
+// The bias fields of the kernel arguments (extended-table geometry, table
+// pointers) and the bias variant to launch: none, the exp(bias) table staged in
+// shared memory (small tables), per-warp windows (relative-position tables with
+// no class tokens on grid rows of a multiple of 64 patches: a warp's 32 rows and
+// a tile's 64 keys each lie in one image row), 16-byte row loads (a dense matrix
+// with a row stride of 4), or gathers from global memory.
+int fill_bias_args(tc::TcArgs& a, const had_shape* s, const had_relpos_bias* bias, uint8_t* bminmax, uint8_t* bext,
+                   uint8_t* expb, bool* rows) {
+  const bool has_bias = bias && bias->table;
+  *rows = false;
+  if (!has_bias) return tc::BIAS_NONE;
+  a.table = bias->table;
+  a.bminmax = reinterpret_cast<float*>(bminmax);
+  a.bext = reinterpret_cast<float*>(bext);
+  a.expb = reinterpret_cast<float*>(expb);
+  if (bias->dense) {
+    const DenseExt x = dense_ext(s->n);
+    a.bias_dense = 1;
+    a.gh = 1; a.gw = 1; a.prefix = 0;
+    a.th = s->n; a.tw = s->n;
+    a.ext_E = x.E; a.ext_S = x.S; a.rb_class = 0; a.k_class = 0; a.k_invalid = x.k_invalid;
+  } else {
+    const RelposExt x = relpos_ext(bias->gh, bias->gw);
+    a.gh = bias->gh; a.gw = bias->gw; a.prefix = bias->prefix;
+    a.th = 2 * bias->gh - 1; a.tw = 2 * bias->gw - 1;
+    a.ext_E = x.E; a.ext_S = x.S; a.rb_class = x.rb_class; a.k_class = x.k_class; a.k_invalid = x.k_invalid;
   }
-  if (EXP == EXP_IDX) {
-    if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, false, EXP>(bias, a, grid, st);
-    if (sel == SEL_TOPN_INT) return launch_tc_t<SEL_TOPN_INT, MODE_F, BIAS_NONE, false, EXP, 1>(a, grid, st);
-    return launch_tc_f<MODE_F, false, EXP>(rows, a, grid, st);
-  }
-  if (vf32) {
-    if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, true, EXP>(bias, a, grid, st);
-    if (sel == SEL_TOPN_INT) return launch_tc_n<SEL_TOPN_INT, MODE_F, true, EXP>(a, grid, st);
-    return launch_tc_f<MODE_F, true, EXP>(rows, a, grid, st);
-  }
-  if (sel == SEL_DENSE) return launch_tc_b<SEL_DENSE, MODE_F, false, EXP>(bias, a, grid, st);
-  if (sel == SEL_TOPN_INT) return launch_tc_n<SEL_TOPN_INT, MODE_F, false, EXP>(a, grid, st);
-  return launch_tc_f<MODE_F, false, EXP>(rows, a, grid, st);
+  *rows = !bias->dense && bias->prefix == 0 && bias->gw % 64 == 0 && a.ext_S == 2 * bias->gw;
+  return a.ext_E <= tc::kBiasSmemMax           ? tc::BIAS_SMEM
+         : *rows                               ? tc::BIAS_ROWS
+         : a.bias_dense && a.ext_S % 4 == 0    ? tc::BIAS_DGLOBAL
+                                               : tc::BIAS_GLOBAL;
 }
 
 // Stage 2: the fused kernel over a prepared workspace.
@@ -448,7 +456,6 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
                         const float* alpha_k, int N, had_mode mode, void* O, had_dtype o_dtype, int32_t* idx,
                         uint8_t* codes, int row_begin, int row_end, void* workspace, cudaStream_t st,
                         unsigned* status) {
-  const bool has_bias = bias && bias->table;
   const bool quant = (mode == HAD_MODE_U8I8);
   const Ws w = ws_layout(s, quant, bias);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
@@ -456,21 +463,23 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
   const bool vf32 = (s->in_dtype == HAD_F32) && !quant;
   tc::TcArgs a;
   memset(&a, 0, sizeof(a));
-  had_status r = encode_2d(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.kpm, kD, (uint64_t)d.BH * d.n_pad, kD, kD,
+  // tiles are 64-channel panels: K~ boxes of 64 B x 64 keys, V boxes of 64 bf16 x 64 keys,
+  // int8 V^T boxes of 64 keys x d channels
+  had_status r = encode_2d(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.kpm, d.d, (uint64_t)d.BH * d.n_pad, d.d, 64,
                            tc::kN, CU_TENSOR_MAP_SWIZZLE_64B);
   if (r != HAD_OK) return r;
   const bool needs_v = (EXP == EXP_NONE);
   if (needs_v && quant) {
-    r = encode_2d(&a.tm_vq, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.vqT, d.n_pad, (uint64_t)d.BH * kD, d.n_pad, tc::kN,
-                  kD, CU_TENSOR_MAP_SWIZZLE_64B);
+    r = encode_2d(&a.tm_vq, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.vqT, d.n_pad, (uint64_t)d.BH * d.d, d.n_pad, tc::kN,
+                  d.d, CU_TENSOR_MAP_SWIZZLE_64B);
     if (r != HAD_OK) return r;
   } else if (needs_v) {
     const void* vb = vf32 ? static_cast<const void*>(ws + w.vhi) : V;
-    r = encode_2d(&a.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, vb, kD, (uint64_t)d.BH * d.n, kD * 2, kD, tc::kN,
+    r = encode_2d(&a.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, vb, d.d, (uint64_t)d.BH * d.n, d.d * 2, 64, tc::kN,
                   CU_TENSOR_MAP_SWIZZLE_128B);
     if (r != HAD_OK) return r;
     if (vf32) {
-      r = encode_2d(&a.tm_vlo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + w.vlo, kD, (uint64_t)d.BH * d.n, kD * 2, kD,
+      r = encode_2d(&a.tm_vlo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws + w.vlo, d.d, (uint64_t)d.BH * d.n, d.d * 2, 64,
                     tc::kN, CU_TENSOR_MAP_SWIZZLE_128B);
       if (r != HAD_OK) return r;
     }
@@ -480,22 +489,8 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
   a.v_raw = V;
   a.v_f32 = (s->in_dtype == HAD_F32) ? 1 : 0;
   a.vscale = quant ? reinterpret_cast<float*>(ws + w.vscale) : nullptr;
-  a.table = has_bias ? bias->table : nullptr;
-  a.bminmax = has_bias ? reinterpret_cast<float*>(ws + w.bminmax) : nullptr;
-  a.expb = has_bias ? reinterpret_cast<float*>(ws + w.expb) : nullptr;
-  a.bext = has_bias ? reinterpret_cast<float*>(ws + w.bext) : nullptr;
-  if (has_bias && bias->dense) {
-    const DenseExt x = dense_ext(s->n);
-    a.bias_dense = 1;
-    a.gh = 1; a.gw = 1; a.prefix = 0;
-    a.th = s->n; a.tw = s->n;
-    a.ext_E = x.E; a.ext_S = x.S; a.rb_class = 0; a.k_class = 0; a.k_invalid = x.k_invalid;
-  } else if (has_bias) {
-    const RelposExt x = relpos_ext(bias->gh, bias->gw);
-    a.gh = bias->gh; a.gw = bias->gw; a.prefix = bias->prefix;
-    a.th = 2 * bias->gh - 1; a.tw = 2 * bias->gw - 1;
-    a.ext_E = x.E; a.ext_S = x.S; a.rb_class = x.rb_class; a.k_class = x.k_class; a.k_invalid = x.k_invalid;
-  }
+  bool rows = false;
+  const int bias_kind = fill_bias_args(a, s, bias, ws + w.bminmax, ws + w.bext, ws + w.expb, &rows);
   a.seqlens = s->seqlens;
   a.O = O; a.o_bf16 = (o_dtype == HAD_BF16) ? 1 : 0;
   a.idx = idx; a.codes = codes; a.row_begin = row_begin; a.row_end = row_end;
@@ -505,31 +500,24 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
   a.B = d.B; a.H = d.H; a.n = d.n; a.n_pad = d.n_pad; a.N = N;
   a.status = status;
   a.koff_mode = (d.n_pad <= tc::kKoffTableMax) ? tc::kKoffTable : tc::kKoffWarp;
-  // per-warp bias windows: a relative-position table, no class tokens, grid rows of a
-  // multiple of 64 patches (a warp's 32 rows and a tile's 64 keys each in one image row)
-  const bool rows = has_bias && !bias->dense && bias->prefix == 0 && bias->gw % 64 == 0 &&
-                    a.ext_S == 2 * bias->gw;
-  const int bias_kind = !has_bias                        ? tc::BIAS_NONE
-                        : a.ext_E <= tc::kBiasSmemMax      ? tc::BIAS_SMEM
-                        : rows                             ? tc::BIAS_ROWS
-                        : a.bias_dense && a.ext_S % 4 == 0 ? tc::BIAS_DGLOBAL
-                                                           : tc::BIAS_GLOBAL;
   a.int_levels = 1;
   for (int h = 0; h < s->H; ++h) {
     const double aq = alpha_q ? (double)alpha_q[h] : 1.0, ak = alpha_k ? (double)alpha_k[h] : 1.0;
     const float c = (float)(aq * ak / std::sqrt((double)s->d));
     a.c_head[h] = c;
-    // the 65 score levels must map to 65 distinct fp32 logits for the integer tie test
+    // the d + 1 score levels must map to distinct fp32 logits for the integer tie test
     volatile float prev = -INFINITY;
-    for (int sc = -64; sc <= 64; sc += 2) {
+    for (int sc = -s->d; sc <= s->d; sc += 2) {
       volatile float lv = (float)sc * c;
       if (!(lv > prev) || !std::isfinite(lv)) a.int_levels = 0;
       prev = lv;
     }
   }
   dim3 grid((s->n + tc::kM - 1) / tc::kM, d.BH);
-  return dispatch_tc<EXP>(EXP == tc::EXP_SCORES ? (int)tc::SEL_DENSE : select_kind(s, bias, N),
-                         quant ? tc::MODE_Q : tc::MODE_F, bias_kind, vf32, rows, a, grid, st);
+  const int sel = EXP == tc::EXP_SCORES ? (int)tc::SEL_DENSE : select_kind(s, bias, N);
+  const int md = quant ? tc::MODE_Q : tc::MODE_F;
+  if (s->d == 128) return launch::dispatch_tc<128, EXP>(sel, md, bias_kind, vf32, rows, a, grid, st);
+  return launch::dispatch_tc<64, EXP>(sel, md, bias_kind, vf32, rows, a, grid, st);
 }
 
 had_status device_status_ptr(unsigned** out) {
@@ -585,8 +573,8 @@ had_status host_plan(const had_shape* s, had_mode mode, const had_relpos_bias* b
   if (chunk_b < 0) return HAD_ERR_INVALID;
   const bool has_bias = bias && bias->table;
   const size_t esz = s->in_dtype == HAD_BF16 ? 2 : 4;
-  p->in_b = (size_t)s->H * s->n * kD * esz;
-  p->o_b = (size_t)s->H * s->n * kD * 4;
+  p->in_b = (size_t)s->H * s->n * s->d * esz;
+  p->o_b = (size_t)s->H * s->n * s->d * 4;
   size_t cb = chunk_b > 0 ? (size_t)chunk_b : std::max<size_t>(1, kHostChunkBytes / (3 * p->in_b));
   p->cb = (int)std::min<size_t>(cb, (size_t)s->B);
   p->chunks = (s->B + p->cb - 1) / p->cb;
@@ -657,7 +645,7 @@ had_status host_attention(const void* Q, const void* K, const void* V, const had
     if (s->seqlens[b] < 1 || s->seqlens[b] > s->n) return HAD_ERR_INVALID;
   const bool has_bias = bias && bias->table;
   char* ws = static_cast<char*>(workspace);
-  const size_t o_b = (size_t)s->H * s->n * kD * (o_dtype == HAD_BF16 ? 2 : 4);
+  const size_t o_b = (size_t)s->H * s->n * s->d * (o_dtype == HAD_BF16 ? 2 : 4);
   auto cu = [](cudaError_t e, const char* what) { return e == cudaSuccess ? HAD_OK : cuda_fail(e, what); };
 
   HostStreams hs;
@@ -735,16 +723,16 @@ using namespace had;
 extern "C" {
 
 size_t had_binarize_pack_workspace_size(const had_shape* s) {
-  if (check_shape(s) != HAD_OK) return 0;
+  if (check_shape(s, true) != HAD_OK) return 0;
   Dims d = dims_of(s);
-  return align_up((size_t)2 * d.BH * d.nchunks * kD * 8);
+  return align_up((size_t)2 * d.BH * d.nchunks * d.d * 8);
 }
 
 had_status had_binarize_pack(const void* X, const had_shape* s, const float* mu_in, float* mu_out, uint32_t* bits,
                              void* workspace, size_t ws_bytes, void* stream) {
-  had_status r = check_shape(s);
+  had_status r = check_shape(s, true);
   if (r != HAD_OK) return r;
-  if (!X || !bits || !aligned16(X) || (reinterpret_cast<uintptr_t>(bits) & 7u)) return HAD_ERR_INVALID;
+  if (!X || !bits || !aligned16(X) || (reinterpret_cast<uintptr_t>(bits) & 3u)) return HAD_ERR_INVALID;
   if ((mu_in && (reinterpret_cast<uintptr_t>(mu_in) & 3u)) || (mu_out && (reinterpret_cast<uintptr_t>(mu_out) & 3u)))
     return HAD_ERR_INVALID;
   if (!mu_in && (!workspace || ws_bytes < had_binarize_pack_workspace_size(s) || !aligned16(workspace)))
@@ -760,7 +748,7 @@ had_status had_binarize_pack(const void* X, const had_shape* s, const float* mu_
 
 size_t had_attention_workspace_size(const had_shape* s, int N, had_mode mode, const had_relpos_bias* bias) {
   (void)N;
-  if (check_shape(s) != HAD_OK || check_bias(s, bias) != HAD_OK) return 0;
+  if (check_shape(s, true) != HAD_OK || check_bias(s, bias) != HAD_OK) return 0;
   return ws_layout(s, mode == HAD_MODE_U8I8, bias).total;
 }
 
@@ -839,7 +827,7 @@ had_status had_attention_codes_u8(const void* Q, const void* K, const void* V, c
 
 had_status had_quantize_v(const void* V, const had_shape* s, int8_t* Vq, float* vscale, void* workspace,
                           size_t ws_bytes, void* stream) {
-  had_status r = check_shape(s);
+  had_status r = check_shape(s, true);
   if (r != HAD_OK) return r;
   if (!V || !Vq || !vscale || !aligned16(V) || (reinterpret_cast<uintptr_t>(vscale) & 3u)) return HAD_ERR_INVALID;
   const Ws w = ws_layout(s, true, nullptr);
@@ -857,19 +845,18 @@ had_status had_quantize_v(const void* V, const had_shape* s, int8_t* Vq, float* 
                   reinterpret_cast<float*>(ws + w.amax), nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, vqT,
                   vscale, st, status);
   if (r != HAD_OK) return r;
-  k_untranspose_vq<<<1024, 256, 0, st>>>(vqT, d.BH, d.n, d.n_pad, s->seqlens, s->H, Vq);
+  k_untranspose_vq<<<1024, 256, 0, st>>>(vqT, d.BH, d.n, d.d, d.n_pad, Vq);
   return check_launch("k_untranspose_vq");
 }
 
-size_t had_dense_reference_workspace_size(const had_shape* s) {
-  (void)s;
-  return 0;
+size_t had_dense_reference_workspace_size(const had_shape* s, const had_relpos_bias* bias) {
+  if (check_shape(s) != HAD_OK || check_bias(s, bias) != HAD_OK) return 0;
+  return ref_ws_layout(s, bias).total;
 }
 
 had_status had_dense_reference_mode(const void* Q, const void* K, const void* V, const had_shape* s,
                                     const had_relpos_bias* bias, int N, void* O, had_dtype o_dtype,
                                     void* workspace, size_t ws_bytes, void* stream) {
-  (void)workspace; (void)ws_bytes;
   had_status r = check_shape(s);
   if (r != HAD_OK) return r;
   if ((r = check_bias(s, bias)) != HAD_OK) return r;
@@ -878,41 +865,47 @@ had_status had_dense_reference_mode(const void* Q, const void* K, const void* V,
   if (N != 0 && N < s->n) return HAD_ERR_UNSUPPORTED;
   if (!Q || !K || !V || !O || !aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return HAD_ERR_INVALID;
   if (o_dtype != HAD_F32 && o_dtype != HAD_BF16) return HAD_ERR_INVALID;
-  int dev = 0;
-  cudaError_t ce = cudaGetDevice(&dev);
-  if (ce != cudaSuccess) return cuda_fail(ce, "cudaGetDevice");
-  unsigned* status = status_ptr(dev);
-  if (!status) return cuda_fail(cudaErrorInvalidSymbol, "status word");
+  const RefWs w = ref_ws_layout(s, bias);
+  if (w.total > 0 && (!workspace || ws_bytes < w.total || !aligned16(workspace))) return HAD_ERR_INVALID;
+  unsigned* status = nullptr;
+  if ((r = device_status_ptr(&status)) != HAD_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
   const bool has_bias = bias && bias->table;
-  Dims d = dims_of(s);
-  AttnArgs a{};
-  a.V = V;
-  a.table = has_bias ? bias->table : nullptr;
-  if (has_bias && bias->dense) {
-    a.bias_dense = 1;
-    a.gh = 1; a.gw = 1; a.prefix = 0;
-    a.th = s->n; a.tw = s->n;
-  } else if (has_bias) {
-    a.gh = bias->gh; a.gw = bias->gw; a.prefix = bias->prefix;
-    a.th = 2 * bias->gh - 1; a.tw = 2 * bias->gw - 1;
-  }
+  if (has_bias && (r = build_bias_tables(s, bias, ws + w.bminmax, ws + w.bext, ws + w.expb, st)) != HAD_OK) return r;
+  const Dims d = dims_of(s);
+  tc::TcArgs a;
+  memset(&a, 0, sizeof(a));
+  // raw bf16 Q, K, V in 64-channel panels of 128 bytes (128-byte swizzle)
+  if ((r = encode_2d(&a.tm_q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Q, d.d, (uint64_t)d.BH * d.n, d.d * 2, 64, tc::kM,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != HAD_OK ||
+      (r = encode_2d(&a.tm_k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, K, d.d, (uint64_t)d.BH * d.n, d.d * 2, 64, tc::kN,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != HAD_OK ||
+      (r = encode_2d(&a.tm_v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, V, d.d, (uint64_t)d.BH * d.n, d.d * 2, 64, tc::kN,
+                     CU_TENSOR_MAP_SWIZZLE_128B)) != HAD_OK)
+    return r;
+  bool rows = false;
+  const int bias_kind = fill_bias_args(a, s, bias, ws + w.bminmax, ws + w.bext, ws + w.expb, &rows);
+  a.v_raw = V;
   a.seqlens = s->seqlens;
   a.O = O; a.o_bf16 = (o_dtype == HAD_BF16) ? 1 : 0;
+  a.wait_cycles = g_wait_cycles.load();
+  a.force_expiry = g_force_expiry.load();
   a.B = d.B; a.H = d.H; a.n = d.n; a.n_pad = d.n_pad; a.N = 0;
   a.status = status;
-  dim3 grid((s->n + kQT - 1) / kQT, d.BH);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const __nv_bfloat16* q = static_cast<const __nv_bfloat16*>(Q);
-  const __nv_bfloat16* k = static_cast<const __nv_bfloat16*>(K);
-  if (has_bias) k_dense_ref<true><<<grid, kAttnThreads, 0, st>>>(a, q, k);
-  else k_dense_ref<false><<<grid, kAttnThreads, 0, st>>>(a, q, k);
-  return check_launch("k_dense_ref");
+  a.koff_mode = (d.n_pad <= tc::kKoffTableMax) ? tc::kKoffTable : tc::kKoffWarp;
+  const float c = (float)(1.0 / std::sqrt((double)s->d));  // standard attention: l = q.k / sqrt(d) + b
+  for (int h = 0; h < s->H; ++h) a.c_head[h] = c;
+  dim3 grid((s->n + tc::kM - 1) / tc::kM, d.BH);
+  if (s->d == 128) return launch::dispatch_ref<128>(bias_kind, a, grid, st);
+  return launch::dispatch_ref<64>(bias_kind, a, grid, st);
 }
 
 had_status had_scores_int(const uint32_t* qbits, const uint32_t* kbits, const had_shape* s, int32_t* S,
                           void* stream) {
   had_status r = check_shape(s);
   if (r != HAD_OK) return r;
+  if (s->d != 64) return HAD_ERR_UNSUPPORTED;
   if (!qbits || !kbits || !S || (reinterpret_cast<uintptr_t>(qbits) & 7u) || (reinterpret_cast<uintptr_t>(kbits) & 7u) ||
       (reinterpret_cast<uintptr_t>(S) & 3u))
     return HAD_ERR_INVALID;
@@ -972,16 +965,16 @@ extern "C" {
 
 had_status had_binarize_pack_noalloc(const void* X, const had_shape* s, float* mu_out, uint32_t* bits,
                                      void* stream) {
-  had_status r = check_shape(s);
+  had_status r = check_shape(s, true);
   if (r != HAD_OK) return r;
-  if (!X || !bits || !aligned16(X) || (reinterpret_cast<uintptr_t>(bits) & 7u)) return HAD_ERR_INVALID;
+  if (!X || !bits || !aligned16(X) || (reinterpret_cast<uintptr_t>(bits) & 3u)) return HAD_ERR_INVALID;
   if (mu_out && (reinterpret_cast<uintptr_t>(mu_out) & 3u)) return HAD_ERR_INVALID;
   const Dims d = dims_of(s);
-  const size_t need = (size_t)d.BH * d.nchunks * kD * sizeof(double);
+  const size_t need = (size_t)d.BH * d.nchunks * d.d * sizeof(double);
   if (need > kPackScratchBytes) {
     snprintf(t_last_error, sizeof(t_last_error),
-             "had_binarize_pack_noalloc: B*H*ceil(n/64) = %lld exceeds the static scratch limit of %lld",
-             (long long)d.BH * d.nchunks, (long long)(kPackScratchBytes / (kD * sizeof(double))));
+             "had_binarize_pack_noalloc: B*H*ceil(n/64)*d/64 = %lld exceeds the static scratch limit of %lld",
+             (long long)d.BH * d.nchunks * d.d / 64, (long long)(kPackScratchBytes / (64 * sizeof(double))));
     return HAD_ERR_UNSUPPORTED;
   }
   double* scratch = nullptr;

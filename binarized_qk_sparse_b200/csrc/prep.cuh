@@ -46,13 +46,15 @@ struct PrepArgs {
   int first_tensor;     // tensor id of blockIdx.z == 0 (lets a launch do only V, or only one of Q/K)
   int B, H, n, nchunks;
   const int32_t* seqlens;
-  double* sums;         // [2][BH][nchunks][64]
-  float* amax;          // [BH][nchunks][64]
+  double* sums;         // [2][BH][nchunks][D]
+  float* amax;          // [BH][nchunks][D]
   unsigned* status;
 };
 
-template <typename T>
+// Head dims D in {32, 64, 128}: a token row is D / EPT threads of one 16-byte load each.
+template <typename T, int D>
 __global__ void __launch_bounds__(kPrepThreads) k_stats(const PrepArgs a) {
+  constexpr int kD = D;
   constexpr int EPT = LoadTraits<T>::kEPT;
   constexpr int TPT = kD / EPT;                 // threads per token row
   constexpr int TPP = kPrepThreads / TPT;       // tokens per pass
@@ -112,15 +114,17 @@ struct PackArgs {
   const float* amax;
   const float* mu_in[2];  // optional caller means per tensor 0/1
   float* mu_out[2];       // optional mean outputs per tensor 0/1
-  uint32_t* bits[2];      // [BH][n][kW] per tensor 0/1 (or null)
-  int8_t* pm[2];          // [BH][n_pad][64] +-1 int8 rows per tensor 0/1 (or null); +1 past L
-  int8_t* vqT;            // [BH][64][n_pad]
-  float* vscale;          // [BH][64]
+  uint32_t* bits[2];      // [BH][n][D/32] per tensor 0/1 (or null)
+  int8_t* pm[2];          // [BH][n_pad][D] +-1 int8 rows per tensor 0/1 (or null); +1 past L
+  int8_t* vqT;            // [BH][D][n_pad]
+  float* vscale;          // [BH][D]
   unsigned* status;
 };
 
-template <typename T>
+template <typename T, int D>
 __global__ void __launch_bounds__(kPrepThreads) k_pack(const PackArgs a) {
+  constexpr int kD = D;
+  constexpr int kW = D / 32;
   constexpr int EPT = LoadTraits<T>::kEPT;
   constexpr int TPT = kD / EPT;
   constexpr int TPP = kPrepThreads / TPT;
@@ -204,12 +208,13 @@ __global__ void __launch_bounds__(kPrepThreads) k_pack(const PackArgs a) {
       }
     }
     __syncthreads();
-    // write the 64 x 64 int8 block of V^T: row c, tokens [i0, i0+64) -- 16 bytes per thread
+    // write the D x 64 int8 block of V^T: row c, tokens [i0, i0+64) -- 16 bytes per thread and step
     int8_t* dst = a.vqT + (size_t)bh * kD * a.n_pad;
-    const int c = threadIdx.x >> 2, seg = threadIdx.x & 3;
-    if (i0 + seg * 16 < a.n_pad) {
-      *reinterpret_cast<uint4*>(dst + (size_t)c * a.n_pad + i0 + seg * 16) =
-          *reinterpret_cast<const uint4*>(&vt[c][seg * 16]);
+    for (int e = threadIdx.x; e < kD * 4; e += kPrepThreads) {
+      const int c = e >> 2, seg = e & 3;
+      if (i0 + seg * 16 < a.n_pad)
+        *reinterpret_cast<uint4*>(dst + (size_t)c * a.n_pad + i0 + seg * 16) =
+            *reinterpret_cast<const uint4*>(&vt[c][seg * 16]);
     }
   }
 }

@@ -33,8 +33,9 @@
  *   - Errors detected on the device (a seqlens entry outside [1, n]) set a
  *     sticky device status word and zero the affected batch's outputs; read
  *     it with had_get_device_status().
- *   - Only d == 64 is supported (HAD_ERR_UNSUPPORTED otherwise), n <= 16384,
- *     H <= 256, and B*H <= 65535.
+ *   - Head dims d = 64 and 128 (d = 32 too in had_binarize_pack,
+ *     had_binarize_pack_noalloc and had_quantize_v; had_scores_int is d = 64
+ *     only); HAD_ERR_UNSUPPORTED otherwise.  n <= 16384, H <= 256, B*H <= 65535.
  */
 #ifndef HAD_H_
 #define HAD_H_
@@ -49,7 +50,7 @@ extern "C" {
 typedef enum {
   HAD_OK = 0,
   HAD_ERR_INVALID = 1,      /* null/misaligned pointer, bad size, alpha <= 0, workspace too small */
-  HAD_ERR_UNSUPPORTED = 2,  /* d != 64, n > 16384, H > 256, unsupported dtype/mode combination */
+  HAD_ERR_UNSUPPORTED = 2,  /* d not 64 or 128, n > 16384, H > 256, unsupported dtype/mode combination */
   HAD_ERR_CUDA = 3,         /* a CUDA launch or runtime call failed; see had_last_cuda_error() */
   HAD_ERR_DEVICE = 4,       /* device-detected error (bad seqlens); from had_get_device_status() */
   HAD_ERR_TIMEOUT = 5       /* a bounded device-side wait expired; from had_get_device_status() */
@@ -169,11 +170,14 @@ had_status had_attention_host(const void* Q, const void* K, const void* V, const
                               size_t ws_bytes, void* stream);
 
 /* ---- in-library dense comparison mode ------------------------------------
- * Standard attention on the unbinarized inputs: l = (q . k)/sqrt(d) + b_ij with
- * bf16 q, k on the tensor cores (fp32 accumulate), fp32 softmax, bf16 P x V.
- * Requires in_dtype == HAD_BF16 and N == 0 or N >= n (dense); otherwise
- * HAD_ERR_UNSUPPORTED.  Needs no workspace (ws may be NULL/0). */
-size_t had_dense_reference_workspace_size(const had_shape* s);
+ * Standard attention on the unbinarized inputs (the full-precision attention the
+ * pages compare against): l = (q . k)/sqrt(d) + b_ij with bf16 q, k on the
+ * tcgen05 tensor cores (fp32 accumulate in tensor memory), fp32 softmax with an
+ * online row maximum, bf16 P x V.  Requires in_dtype == HAD_BF16 and N == 0 or
+ * N >= n (dense); otherwise HAD_ERR_UNSUPPORTED.  The workspace holds the bias
+ * tables: had_dense_reference_workspace_size(s, bias) bytes (0 without a bias,
+ * when workspace may be NULL). */
+size_t had_dense_reference_workspace_size(const had_shape* s, const had_relpos_bias* bias);
 had_status had_dense_reference_mode(const void* Q, const void* K, const void* V, const had_shape* s,
                                     const had_relpos_bias* bias, int N, void* O, had_dtype o_dtype,
                                     void* workspace, size_t ws_bytes, void* stream);

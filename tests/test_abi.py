@@ -80,6 +80,12 @@ def test_host_validation_rejects_before_launch(L):
     shp = _shape(m)
     assert L.had_dense_reference_mode(fake, fake, fake, ctypes.byref(shp), None, 5, fake, 1, None, 0, None) \
         == m.HAD_ERR_UNSUPPORTED
+    # with a bias it needs the workspace for the bias tables
+    rb = m.had_relpos_bias(0x30000, 8, 8, 0)
+    assert L.had_dense_reference_workspace_size(ctypes.byref(shp), ctypes.byref(rb)) > 0
+    assert L.had_dense_reference_workspace_size(ctypes.byref(shp), None) == 0
+    assert L.had_dense_reference_mode(fake, fake, fake, ctypes.byref(shp), ctypes.byref(rb), 0, fake, 1, None, 0,
+                                      None) == m.HAD_ERR_INVALID
     # exports
     assert L.had_topn_indices(fake, fake, ctypes.byref(shp), None, None, None, 0, fake, ws, big, None) \
         == m.HAD_ERR_INVALID
@@ -96,7 +102,9 @@ def test_workspace_size_grows_with_mode_and_bias(L):
     bias = m.had_relpos_bias(0x30000, 14, 14, 1)
     qb = L.had_attention_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(bias))
     assert 0 < f < q < qb
-    bad = _shape(m, d=128)
+    wide = _shape(m, B=2, H=3, n=197, d=128)   # head dim 128: twice the per-token intermediates
+    assert L.had_attention_workspace_size(ctypes.byref(wide), 0, 1, None) > q
+    bad = _shape(m, d=96)
     assert L.had_attention_workspace_size(ctypes.byref(bad), 0, 0, None) == 0
 
 

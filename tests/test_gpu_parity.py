@@ -331,16 +331,24 @@ def test_topn_bias_row_windows(oracle_mod, gh, gw, seqlens):
 
 # ----------------------------------------------------------------------------- comparison mode
 
-def test_dense_reference_mode(oracle_mod):
-    w = _workload("deit")
-    B = 4
-    Qn, Kn, Vn = w.Q[:B], w.K[:B], w.V[:B]
-    w4 = workloads.Workload(w.name, B, w.H, w.n, w.d, w.dtype, Qn, Kn, Vn, None, w.bias, w.passes, w.seed, w.recipe)
-    Q, K, V, seq, bias = _dev_inputs(w4)
-    O = had.had_dense_reference_mode(Q, K, V, bias=bias).float().cpu().numpy()
-    b = oracle_mod.RelPosBias(w.bias.table, w.bias.gh, w.bias.gw, w.bias.prefix)
-    ref = oracle_mod.dense_attention(Qn, Kn, Vn, bias=b)
-    assert np.max(np.abs(O - ref)) <= 1e-2 * np.max(np.abs(Vn))
+@pytest.mark.parametrize("case", ["deit", "bert", "t5_1024", "grid_rows"])
+def test_dense_reference_mode(oracle_mod, case):
+    """The comparison mode: standard attention on the unbinarized bf16 inputs on the
+    tcgen05 tensor cores, against the oracle's fp64 attention on the same values
+    (relative-position bias in shared memory, ragged lengths, no bias, and per-warp
+    bias windows on a 16x128 grid)."""
+    if case == "grid_rows":
+        w = workloads.grid(1, 2, 16, 128, 0, None, seed=13)
+    else:
+        w = _subset(_workload(case), 4 if case != "t5_1024" else 2)
+        if case == "deit":
+            w = workloads.Workload(w.name, w.B, w.H, w.n, w.d, w.dtype, w.Q, w.K, w.V, None, _workload("deit").bias,
+                                   w.passes, w.seed, w.recipe)
+    Q, K, V, seq, bias = _dev_inputs(w)
+    rows = _sample_rows(w, 48, 3)
+    O = _flat(had.had_dense_reference_mode(Q, K, V, seqlens=seq, bias=bias)).float().cpu().numpy()[rows]
+    ref = oracle_mod.dense_attention(w.Q, w.K, w.V, seqlens=w.seqlens, bias=_oracle_bias(oracle_mod, w), rows=rows)
+    assert np.max(np.abs(O - ref)) <= _tol(w)
 
 
 # ----------------------------------------------------------------------------- edge cases

@@ -86,19 +86,30 @@ def _finish(x, dtype):
     return bf16_round(x) if dtype == "bf16" else np.ascontiguousarray(x, np.float32)
 
 
-def tiny() -> Workload:
+# Head dim 128 (the BinaryAttention kernel benchmark's head dim): the same recipes
+# with d = 128 and seed + 100, named with a "_d128" suffix.
+def _dsuf(d: int) -> str:
+    return "" if d == 64 else f"_d{d}"
+
+
+def _dseed(seed: int, d: int) -> int:
+    return seed if d == 64 else seed + 100
+
+
+def tiny(d: int = 64) -> Workload:
     """HAD-sized toy: B1 H1 n128 d64, fp32 Q,K,V iid N(0,1), seed 0; top-15 and dense, float A.V."""
-    rng = np.random.default_rng(0)
-    shp = (1, 1, 128, 64)
+    seed = _dseed(0, d)
+    rng = np.random.default_rng(seed)
+    shp = (1, 1, 128, d)
     Q = rng.standard_normal(shp, dtype=np.float32)
     K = rng.standard_normal(shp, dtype=np.float32)
     V = rng.standard_normal(shp, dtype=np.float32)
-    return Workload("tiny_b1_h1_n128", 1, 1, 128, 64, "f32", Q, K, V, None, None,
-                    [(15, MODE_FLOAT), (0, MODE_FLOAT)], 0,
+    return Workload("tiny_b1_h1_n128" + _dsuf(d), 1, 1, 128, d, "f32", Q, K, V, None, None,
+                    [(15, MODE_FLOAT), (0, MODE_FLOAT)], seed,
                     "Q,K,V iid N(0,1) fp32; no bias; alpha=1")
 
 
-def deit() -> Workload:
+def deit(d: int = 64, B: int = 64) -> Workload:
     """DeiT-shaped BinaryAttention: B64 H12 n197 (1 cls + 14x14) d64 bf16, seed 1.
 
     Q and K: a per-(head, channel) offset ~N(0, 0.5), shared over batch and
@@ -107,8 +118,9 @@ def deit() -> Workload:
     without replacement, scaled x10.  Relative-position bias 27x27 per head
     ~N(0, 0.1), prefix 1 (the cls token).  Dense, uint8 A x int8 V.
     """
-    rng = np.random.default_rng(1)
-    B, H, n, d = 64, 12, 197, 64
+    seed = _dseed(1, d)
+    rng = np.random.default_rng(seed)
+    H, n = 12, 197
     offq = rng.standard_normal((H, d), dtype=np.float32) * np.float32(0.5)
     offk = rng.standard_normal((H, d), dtype=np.float32) * np.float32(0.5)
     Q = rng.standard_normal((B, H, n, d), dtype=np.float32) + offq[None, :, None, :]
@@ -119,9 +131,9 @@ def deit() -> Workload:
     for p in pick:
         V[:, p // d, :, p % d] *= np.float32(10.0)
     table = rng.standard_normal((H, 27, 27), dtype=np.float32) * np.float32(0.1)
-    return Workload("deit_b64_h12_n197", B, H, n, d, "bf16", _finish(Q, "bf16"), _finish(K, "bf16"),
-                    _finish(V, "bf16"), None, Bias(table, 14, 14, 1), [(0, MODE_U8I8)], 1,
-                    "Q,K = offset[h,c]~N(0,0.5) + N(0,1); V N(0,1) with 8/768 channels x10; "
+    return Workload(f"deit_b{B}_h12_n197" + _dsuf(d), B, H, n, d, "bf16", _finish(Q, "bf16"), _finish(K, "bf16"),
+                    _finish(V, "bf16"), None, Bias(table, 14, 14, 1), [(0, MODE_U8I8)], seed,
+                    f"Q,K = offset[h,c]~N(0,0.5) + N(0,1); V N(0,1) with {n_out}/{H * d} channels x10; "
                     "relpos bias 27x27/head ~N(0,0.1), prefix 1",
                     extra={"outlier_channels": sorted(int(p) for p in pick)})
 
@@ -152,22 +164,22 @@ def bert() -> Workload:
                     "Q,K,V iid N(0,1); L_b ~ U{32..256} per sequence; tokens past L_b are padding")
 
 
-def t5(n: int) -> Workload:
+def t5(n: int, d: int = 64, B: int = 16) -> Workload:
     """T5-Base-shaped long-context sweep: B16 H12 d64 bf16, n in {128..1024}, N = 15n/128, float.
 
     Q ~N(0,1); K_j = 0.6 * Q_{pi(j)} + 0.8 * eps with pi(j) iid uniform over
     the n tokens of the same (b, h) and eps ~N(0,1); V ~N(0,1).  Seed 3 + log2(n/128).
     """
     assert n in (128, 256, 512, 1024)
-    seed = 3 + int(np.log2(n // 128))
+    seed = _dseed(3 + int(np.log2(n // 128)), d)
     rng = np.random.default_rng(seed)
-    B, H, d = 16, 12, 64
+    H = 12
     Q = rng.standard_normal((B, H, n, d), dtype=np.float32)
     pi = rng.integers(0, n, size=(B, H, n))
     eps = rng.standard_normal((B, H, n, d), dtype=np.float32)
     K = np.float32(0.6) * np.take_along_axis(Q, pi[..., None], axis=2) + np.float32(0.8) * eps
     V = rng.standard_normal((B, H, n, d), dtype=np.float32)
-    return Workload(f"t5_b16_h12_n{n}", B, H, n, d, "bf16", _finish(Q, "bf16"), _finish(K, "bf16"),
+    return Workload(f"t5_b{B}_h12_n{n}" + _dsuf(d), B, H, n, d, "bf16", _finish(Q, "bf16"), _finish(K, "bf16"),
                     _finish(V, "bf16"), None, None, [(15 * n // 128, MODE_FLOAT)], seed,
                     "Q N(0,1); K_j = 0.6 Q_pi(j) + 0.8 eps; V N(0,1)", extra={"pi": pi})
 
@@ -189,25 +201,34 @@ def stress() -> Workload:
                     "Q,K,V iid N(0,1); relpos bias 255x255/head ~N(0,0.1), prefix 0")
 
 
-def grid(B: int, H: int, gh: int, gw: int, prefix: int, seqlens=None, seed: int = 11) -> Workload:
+def grid(B: int, H: int, gh: int, gw: int, prefix: int, seqlens=None, seed: int = 11, d: int = 64) -> Workload:
     """Image-grid attention of any size: B x H heads over `prefix` class tokens
     plus a gh x gw patch grid, d64 bf16 Q,K,V iid N(0,1), a relative-position
     bias (2gh-1) x (2gw-1) per head ~N(0, 0.1), optional per-batch lengths.
     Used to cover the grid shapes the fixed workloads do not reach."""
     rng = np.random.default_rng(seed)
-    n, d = prefix + gh * gw, 64
+    n = prefix + gh * gw
     Q = rng.standard_normal((B, H, n, d), dtype=np.float32)
     K = rng.standard_normal((B, H, n, d), dtype=np.float32)
     V = rng.standard_normal((B, H, n, d), dtype=np.float32)
     table = rng.standard_normal((H, 2 * gh - 1, 2 * gw - 1), dtype=np.float32) * np.float32(0.1)
     sl = None if seqlens is None else np.asarray(seqlens, np.int32)
-    return Workload(f"grid_b{B}_h{H}_{gh}x{gw}_p{prefix}" + ("" if sl is None else "_sl"), B, H, n, d, "bf16",
+    return Workload(f"grid_b{B}_h{H}_{gh}x{gw}_p{prefix}" + ("" if sl is None else "_sl") + _dsuf(d), B, H, n, d, "bf16",
                     _finish(Q, "bf16"), _finish(K, "bf16"), _finish(V, "bf16"), sl, Bias(table, gh, gw, prefix),
                     [(max(1, n // 8), MODE_FLOAT), (0, MODE_U8I8)], seed,
                     "Q,K,V iid N(0,1); relpos bias ~N(0,0.1)")
 
 
 def by_name(name: str) -> Workload:
+    if name.endswith("_d128"):
+        base = name[: -len("_d128")]
+        if base == "tiny":
+            return tiny(128)
+        if base == "deit":
+            return deit(128)
+        if base.startswith("t5_"):
+            return t5(int(base[3:]), 128)
+        raise KeyError(name)
     if name == "tiny":
         return tiny()
     if name == "deit":
