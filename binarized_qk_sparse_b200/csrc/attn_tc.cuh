@@ -1518,6 +1518,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
     for (int s2 = 0; s2 < kVStages; ++s2)
       if (v_par[s2] >= 0) mbar_wait(&bars[B_VFULL + s2], (uint32_t)v_par[s2], 200000000LL);
     if (BIAS == BIAS_SMEM) mbar_wait(&bars[B_BIAS], 0, 200000000LL);
+    if (kRef) mbar_wait(&bars[B_QFULL], 0, 200000000LL);
   }
   if (warp == kMmaWarp && lane == 0) {
     // every tcgen05 operation this thread issued is complete before TMEM is freed
