@@ -374,6 +374,21 @@ def run_reference(args, rank, world):
     return 0
 
 
+def _sliced(w, args):
+    """The first --batch sequences and --heads heads of a workload (a smaller case of
+    the same kernel variant, for profiler captures); the whole workload by default."""
+    B = args.batch or w.B
+    H = args.heads or w.H
+    if B == w.B and H == w.H:
+        return w
+    bias = w.bias
+    if bias is not None:
+        bias = type(bias)(bias.table[:H], *[getattr(bias, f) for f in ("gh", "gw", "prefix") if hasattr(bias, f)])
+    cut = lambda x: np.ascontiguousarray(x[:B, :H])  # noqa: E731
+    return workloads.Workload(f"{w.name}_slice_b{B}_h{H}", B, H, w.n, w.d, w.dtype, cut(w.Q), cut(w.K), cut(w.V),
+                              None if w.seqlens is None else w.seqlens[:B], bias, w.passes, w.seed, w.recipe)
+
+
 def _config(w, N, mode):
     tag = "dense_ref" if mode == "ref" else f"{'dense' if N == 0 else f'top{N}'}_{mode}"
     return {"workload": f"{w.name}_{tag}", "B": w.B, "H": w.H, "n": w.n,
@@ -395,7 +410,7 @@ def run_gpu(args, rank, world, local_rank):
     if world > 1:
         import torch.distributed as dist
     name, N, mode = WORKLOADS[args.workload]
-    w = workloads.by_name(name)
+    w = _sliced(workloads.by_name(name), args)
     bf16 = w.dtype == "bf16"
     tdt = torch.bfloat16 if bf16 else torch.float32
 
@@ -599,6 +614,8 @@ def main():
     ap.add_argument("--workload", default="stress_topn", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=0, help="run the first B sequences only (profiler captures)")
+    ap.add_argument("--heads", type=int, default=0, help="run the first H heads only (profiler captures)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -1118,10 +1118,18 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
     }
     if (tid < kM && row_ok && !*abort_flag) {
       if (pass == P_LEVELS) {
-        auto cnt = [&](int lev) -> int { return (int)hist[lev * kM + srow]; };  // level (d - s) / 2
+        // the row's level counts, level (d - s) / 2: in registers at d = 64, read from
+        // shared memory at d = 128 (129 of them)
+        constexpr int kCached = kLevels <= 65 ? kLevels : 1;
+        int cached[kCached];
+#pragma unroll
+        for (int lev = 0; lev < kCached; ++lev) cached[lev] = kCached == kLevels ? (int)hist[lev * kM + srow] : 0;
+        auto cnt = [&](int lev) -> int { return kCached == kLevels ? cached[lev] : (int)hist[lev * kM + srow]; };
         int hmin = D, hN = D, cum = 0;
         bool found = false;
+#pragma unroll
         for (int lev = kLevels - 1; lev >= 0; --lev) hmin = cnt(lev) > 0 ? lev : hmin;
+#pragma unroll
         for (int lev = 0; lev < kLevels; ++lev) {
           cum += cnt(lev);
           if (!found && cum >= keff) { hN = lev; found = true; }
@@ -1132,6 +1140,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
           m = (float)smax * c;
           int gt = 0, eq = 0;
           float ls = 0.0f;
+#pragma unroll
           for (int lev = 0; lev < kLevels; ++lev) {
             const float lv = (float)(D - 2 * lev) * c;
             const int k = cnt(lev);
@@ -1146,6 +1155,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
           sF = sN;
           // this row's weight per level: exp(l - m) above the threshold, the tie weight at it, 0 below
           float* wt = reinterpret_cast<float*>(hist);
+#pragma unroll
           for (int lev = 0; lev < kLevels; ++lev) {
             const float lv = (float)(D - 2 * lev) * c;
             wt[lev * kM + srow] = (lv >= F) ? fast_exp2((lv - m) * kLog2e) : 0.0f;
