@@ -465,8 +465,8 @@ def run_gpu(args, rank, world, local_rank):
             raise had.HadError(st, "had_attention_prepared")
 
     # the tensor pipe's int8 and bf16 MMA rates on this GPU (probe kernel, before the workload)
-    probe_i8, _ = had.had_probe_mma_rate("i8", 200000)
-    probe_bf16, _ = had.had_probe_mma_rate("bf16", 100000)
+    probe_i8, _ = had.had_probe_mma_rate("i8", 40000)      # ~2.6 ms per launch
+    probe_bf16, _ = had.had_probe_mma_rate("bf16", 20000)
 
     if ref:  # the bias tables (range + tables for a dense matrix) and the kernel
         kernels_per_step = 1 + (0 if bias is None else (2 if isinstance(w.bias, workloads.DenseBias) else 1))
