@@ -58,7 +58,7 @@ constexpr int kN = 64;             // keys per tile (score MMA N)
 __host__ __device__ constexpr int cta_threads(int split) { return 32 * (4 * split + 2); }
 constexpr int kSplitMaxKeys = 256;  // top-N without a bias, ragged rows: two threads per row up to this n_pad
 constexpr int kKStages = 4;
-constexpr int kVStages = 2;
+constexpr int kVStagesMax = 3;  // see v_stages()
 // Score levels of a head dim: s = d - 2h takes d + 1 values.
 __host__ __device__ constexpr int levels_of(int d) { return d + 1; }
 constexpr int kRadixBins = 256;   // 16-bit counters, two per word (a row counts at most kMaxN keys)
@@ -100,6 +100,9 @@ constexpr int kBiasSmemMax = kBiasSmemEntries;
 // it runs the dense softmax path with an online row maximum.
 enum { SEL_DENSE = 0, SEL_TOPN_INT = 1, SEL_TOPN_FLOAT = 2, SEL_REF = 3 };
 __host__ __device__ constexpr bool sel_dense(int sel) { return sel == SEL_DENSE || sel == SEL_REF; }
+// V stages: three (the P.V tiles of dense and no-bias top-N kinds load further
+// ahead), two for top-N with a bias and for fp32 V (their shared memory is fuller)
+__host__ __device__ constexpr int v_stages(int sel, bool vf32) { return (sel == SEL_TOPN_FLOAT || vf32) ? 2 : 3; }
 enum { MODE_F = 0, MODE_Q = 1 };
 enum { EXP_NONE = 0, EXP_IDX = 1, EXP_CODES = 2, EXP_SCORES = 3 };
 enum { P_DONE = 0, P_NORM, P_LEVELS, P_FBIN, P_RADIX, P_COLLECT, P_KEPT_NORM, P_PV, P_IDX, P_CODES, P_SCORES };
@@ -148,14 +151,17 @@ struct Smem {
   static constexpr int kOpB = SEL == SEL_REF ? 2 : 1;            // bytes per Q, K element (bf16 or +-1 int8)
   static constexpr int kQ = 0;                                   // 128 x D elements
   static constexpr int kK = kQ + kM * D * kOpB;                  // 4 x 64 x D elements
-  static constexpr int kV = kK + kKStages * kN * D * kOpB;       // 2 V stages
-  static constexpr int kKoff = kV + kVStages * kVStage;          // bias key offsets (table, or 4 warps x 2 x 64)
+  static constexpr int kVS = v_stages(SEL, VF32);
+  static constexpr int kV = kK + kKStages * kN * D * kOpB;       // kVS V stages
+  static constexpr int kKoff = kV + kVS * kVStage;               // bias key offsets (table, or 4 warps x 2 x 64)
   static constexpr int kBiasTab = kKoff + (HAS_BIAS ? kKoffTableMax * 4 : 0);  // exp(bias) table (dense)
   // row-pair exchange: dense 2 x 128 fp32 (partials); top-N 6 x 128 (threshold state) + 2 x 2 x 128 tie counts
   static constexpr int kXchg = kBiasTab + (BIAS == BIAS_SMEM ? kBiasSmemMax * 4 : 0);
-  static constexpr int kDq = kXchg + (sel_dense(SEL) ? 2 : SEL == SEL_TOPN_INT ? 10 : 0) * kM * 4;  // D dequant scales
+  // top-N with a bias: a per-row candidate counter shared by the row's two threads, and a
+  // second row of 128 for exchanging their radix counts
+  static constexpr int kDq = kXchg + (sel_dense(SEL) ? 2 : SEL == SEL_TOPN_INT ? 10 : 2) * kM * 4;  // D dequant scales
   static constexpr int kBar = kDq + D * 4;
-  static constexpr int kNumBars = 2 * kKStages + 2 * kVStages + 2 * kSBufs + 5;
+  static constexpr int kNumBars = 2 * kKStages + 2 * kVStagesMax + 2 * kSBufs + 5;
   static constexpr int kMisc = kBar + kNumBars * 8;              // [0] tmem base [1] abort
   static constexpr int kHist = (kMisc + 16 + 127) / 128 * 128;
   static constexpr int kHistBytes = sel_dense(SEL) ? kLev * 32 * 4
@@ -171,8 +177,8 @@ enum {
   B_KFULL = 0,
   B_KEMPTY = kKStages,
   B_VFULL = 2 * kKStages,
-  B_VEMPTY = 2 * kKStages + kVStages,
-  B_SFULL = 2 * kKStages + 2 * kVStages,  // one per score buffer
+  B_VEMPTY = 2 * kKStages + kVStagesMax,
+  B_SFULL = 2 * kKStages + 2 * kVStagesMax,  // one per score buffer
   B_TDONE = B_SFULL + kSBufs,             // one per score buffer
   B_OFULL = B_TDONE + kSBufs,
   B_FINAL,
@@ -227,9 +233,12 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
   constexpr int kPan = D / 64;      // 64-channel panels of the Q~, K~ and V tiles
   constexpr uint32_t kTmemCols = tmem_cols(D);
   constexpr bool kRef = SEL == SEL_REF;        // the unbinarized comparison mode
+  constexpr int kVStages = v_stages(SEL, VF32);
   constexpr bool kDense = sel_dense(SEL);
-  static_assert(SPLIT == 1 || kDense || (SEL == SEL_TOPN_INT && EXPORT == EXP_NONE),
-                "two threads per row: dense, or top-N without a bias on its P.V path");
+  static_assert(SPLIT == 1 || kDense || (SEL == SEL_TOPN_INT && EXPORT == EXP_NONE) ||
+                    (SEL == SEL_TOPN_FLOAT && EXPORT == EXP_NONE && MODE == MODE_F),
+                "two threads per row: dense, top-N without a bias on its P.V path, or top-N with a bias "
+                "and float A.V");
   static_assert((BIAS != BIAS_SMEM && BIAS != BIAS_DGLOBAL) || kDense,
                 "staged or vector-read exp(bias) tables serve the dense weights only");
   static_assert(BIAS != BIAS_ROWS || (SEL != SEL_TOPN_INT && 2 * (SPLIT == 2 ? 8 * 64 : 4 * kRowWin) <= kKoffTableMax),
@@ -246,6 +255,10 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
   // logits in [64, 128) of the candidate area
   constexpr bool kMerge = SEL == SEL_TOPN_FLOAT && MODE == MODE_F && EXPORT == EXP_NONE;
   constexpr int kCap = kCandCap / 2;
+  // top-N with a bias, two threads per row: both threads take every per-row decision
+  // (from the shared histograms, so identically); candidates and recorded keys get
+  // their slots from a per-row counter in shared memory
+  constexpr bool kSplitF = kSplit == 2 && SEL == SEL_TOPN_FLOAT;
   using SM = Smem<D, SEL, VF32, BIAS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -929,7 +942,18 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
               } else if (kHasRadix && pass == P_COLLECT) {
                 // the order keys inside the window, one column per row: [kCandCap][128 rows]
                 // (the slot wraps, so a miscount stays in bounds and is reported after the pass)
-                if (r_state == 2) {
+                if (r_state == 2 && kSplitF) {
+                  // two threads per row: slots from the row's shared counter
+                  const uint32_t ulo = r_uhi - r_span;
+#pragma unroll
+                  for (int u = 0; u < 32; ++u) {
+                    const uint32_t key = float_order_key(lg[u]);
+                    if (key - ulo <= r_span) {
+                      const int slot = atomicAdd(reinterpret_cast<int*>(xchg) + srow, 1);
+                      hist[(slot & (kCandCap - 1)) * kM + srow] = key;
+                    }
+                  }
+                } else if (r_state == 2) {
                   const uint32_t ulo = r_uhi - r_span;
 #pragma unroll
                   for (int u = 0; u < 32; ++u) {
@@ -1029,6 +1053,74 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
             for (int u = 0; u < kN; ++u)
               if (j0 + u < a.n) dst[j0 + u] = (row_ok && j0 + u < L) ? (int32_t)r[u] : 0;
           }
+        } else if (kSplitF && pv) {
+          // top-N with a bias, P.V with two threads per row: this thread's 32 keys.  Keys at
+          // or above w_cut are weighted; keys in [w_lo, w_hi] are the final bin (recorded
+          // in shared slots, ranked after the pass) or, for a row resolved by a collect
+          // pass, the ties at F, kept in key order: the two threads exchange their tie
+          // counts every tile (both warps of the pair reach the barrier, whatever
+          // happened to their waits)
+          const int jb = j0 + 32 * half;
+          const int nv = nvalid - 32 * half;  // valid keys of this chunk (<= 0: none)
+          float e[32];
+          uint32_t inm = 0u;
+          // weights and final-bin mask of this thread's 32 keys (FULL: no key past L)
+          auto pv_chunk = [&](auto full_tag) {
+            constexpr bool FULL = decltype(full_tag)::value;
+            const float mo_p = -m * kLog2e;
+#pragma unroll
+            for (int u = 0; u < 32; ++u) {
+              const float sf = (float)(int)r[u];
+              float bv = 0.0f;
+              if (BIAS == BIAS_ROWS) {
+                bv = brow[-u];
+              } else {
+                const int kk = ko[32 * half + u];
+                bv = __ldg(reinterpret_cast<const float*>(tab_bytes - kk));
+              }
+              const float l = (FULL || u < nv) ? __fmaf_rn(sf, c, bv) : -INFINITY;
+              const float x = fast_exp2(__fmaf_rn(l, kLog2e, mo_p));
+              e[u] = l >= w_cut ? x : 0.0f;
+              inm |= (l >= w_lo && l <= w_hi ? 1u : 0u) << u;
+            }
+          };
+          if (ok_wait && jb < L) {
+            if (full_tile) pv_chunk(std::true_type{});
+            else pv_chunk(std::false_type{});
+          } else {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) e[u] = 0.0f;
+          }
+          uint32_t eqm = 0u;
+          if (r_state == 3) {
+            while (inm) {
+              const int u = __ffs(inm) - 1;
+              inm &= inm - 1u;
+              const int slot = atomicAdd(reinterpret_cast<int*>(xchg) + srow, 1);
+              hist[(slot & (kCap - 1)) * kM + srow] = (uint32_t)(jb + u);
+            }
+          } else {
+            eqm = inm;
+          }
+          int* tx = reinterpret_cast<int*>(hist) + (kCandCap - 8) * kM + (int)(gs & 1u) * 2 * kM;
+          tx[half * kM + srow] = __popc(eqm);
+          asm volatile("bar.sync %0, 64;" ::"r"(1 + (warp & 3)) : "memory");
+          const int c0 = tx[srow], c1 = tx[kM + srow];
+          const uint32_t dropm = eqm & ~tie_keep(eqm, cut, rF, tie_seen + (half ? c0 : 0));
+          if (dropm) {
+#pragma unroll
+            for (int u = 0; u < 32; ++u) e[u] = ((dropm >> u) & 1u) ? 0.0f : e[u];
+          }
+          tie_seen += c0 + c1;
+          if (ok_wait) {
+            if (jb >= L) {
+              const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+              tmem_st16(tl + colP + 32 * half, z);
+              if (VF32) tmem_st16(tl + colP + 32 * half + 16, z);
+            } else {
+              emit(e, half);
+            }
+          }
         } else if (kSplit == 2 && SEL == SEL_TOPN_INT && pv) {
           // top-N P.V with two threads per row: weights of this thread's chunk, then
           // the row's two threshold-tie counts of this tile are exchanged (every live
@@ -1100,6 +1192,22 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
     // two threads per top-N row: both have finished adding to the row's level
     // histogram before the first reads it (and overwrites it with the weight table)
     if (kSplit == 2 && SEL == SEL_TOPN_INT && pass == P_LEVELS) __syncthreads();
+    if (kSplitF && pass == P_RADIX) {
+      // the row's two threads sum their counts of keys above the first radix window
+      int* ra = reinterpret_cast<int*>(xchg) + kM;
+      if (is_soft && half == 1) ra[srow] = r_above;
+      __syncthreads();
+      const int other = (is_soft && half == 0) ? ra[srow] : 0;
+      __syncthreads();
+      if (is_soft && half == 0) {
+        r_above += other;
+        ra[srow] = r_above;
+      }
+      __syncthreads();
+      if (is_soft && half == 1) r_above = ra[srow];
+    }
+    // both threads of a row have finished adding to its histogram (or candidate list)
+    if (kSplitF) __syncthreads();
     if (kSplit == 2 && pass == P_NORM) {
       // the row's two threads combine their partial normalizers (and running maxima)
       if (is_soft && half == 1) { xchg[srow] = lsum; xchg[kM + srow] = m; }
@@ -1116,7 +1224,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         }
       }
     }
-    if (tid < kM && row_ok && !*abort_flag) {
+    if ((tid < kM || (kSplitF && is_soft)) && row_ok && !*abort_flag) {
       if (pass == P_LEVELS) {
         // the row's level counts, level (d - s) / 2: in registers at d = 64, read from
         // shared memory at d = 128 (129 of them)
@@ -1275,6 +1383,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         // the r_rank-th largest collected key: the one with fewer than r_rank keys
         // above it and at least r_rank at or above it
         const uint32_t* cand = hist;
+        if (kSplitF) r_cnt = reinterpret_cast<const int*>(xchg)[srow];  // the row's shared counter
         const int nc = min(r_cnt, kCandCap);
         if (r_cnt > kCandCap) raise_status(a.status, kDevErrCapacity);
         uint32_t uF = 0u;
@@ -1342,17 +1451,24 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
     else if ((EXPORT == EXP_CODES || MODE == MODE_Q) && SEL == SEL_TOPN_FLOAT && pass != P_KEPT_NORM) next = P_KEPT_NORM;
     else if (EXPORT == EXP_CODES) next = P_CODES;
     else next = P_PV;
-    if ((next == P_RADIX || next == P_FBIN) && tid < kM) {
+    if ((next == P_RADIX || next == P_FBIN) && tid < kM)
       for (int bb = 0; bb < kRadixBins / 2; ++bb) hist[bb * kM + srow] = 0u;
-      r_above = 0;
-    }
-    if (next == P_KEPT_NORM && tid < kM) lsum = 0.0f;
+    if ((next == P_RADIX || next == P_FBIN) && is_soft) r_above = 0;
+    if (kSplitF && (next == P_COLLECT || next == P_PV) && tid < kM) reinterpret_cast<int*>(xchg)[srow] = 0;
+    if (next == P_KEPT_NORM && is_soft) lsum = 0.0f;
     __syncthreads();
     first_pass = false;
     pass = next;
   }
 
   // ---------------------------------------------------------------- epilogue
+  // two threads per top-N row with a bias: the row's count of recorded keys, read
+  // before the normalizer exchange below reuses its shared slot
+  int rc_split = 0;
+  if (kSplitF) {
+    if (is_soft) rc_split = reinterpret_cast<const int*>(xchg)[srow];
+    __syncthreads();
+  }
   if (kSplit == 2 && sum_in_pv) {
     // the row's two threads add their partial normalizers
     if (is_soft) xchg[half * kM + srow] = lsum;
@@ -1373,9 +1489,13 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
       // dropped key), and its V row is added to O below, 32 channels at a time
       int n_merge = 0;
       const float* pw = reinterpret_cast<const float*>(hist) + kCap * kM + srow;  // weight x at pw[x * kM]
-      if (kMerge && r_state == 3 && ok && row_ok && row < a.n) {
-        n_merge = min(r_cnt, kCap);
-        if (r_cnt > kCap) raise_status(a.status, kDevErrCapacity);
+      const bool merge_row = kMerge && r_state == 3 && ok && row_ok && row < a.n;
+      float merged = 0.0f;  // the kept recorded keys' weights
+      // (two threads per row: the first takes the row's decisions, the second reads them)
+      if (merge_row && (!kSplitF || half == 0)) {
+        const int rc = kSplitF ? rc_split : r_cnt;
+        n_merge = min(rc, kCap);
+        if (rc > kCap) raise_status(a.status, kDevErrCapacity);
         const int8_t* kb = a.kpm + (size_t)bh * a.n_pad * D;
         for (int x = 0; x < n_merge; ++x) {
           const int j = (int)hist[x * kM + srow];
@@ -1425,20 +1545,45 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
             break;
           }
         }
-        int allow = r_rank - gt;  // keys at the threshold still kept, in key order
-        const float mo_e = -m * kLog2e;
+        // keys above vF are kept; of the keys at vF, the r_rank - gt with the lowest
+        // key indices (the slots need not be in key order)
+        const int allow = r_rank - gt;
+        uint64_t keep = 0;
         for (int x = 0; x < n_merge; ++x) {
           const float v = lc[x * kM];
-          const bool at = v == vF;
+          bool k = v > vF;
+          if (v == vF) {
+            const int jx = (int)hist[x * kM + srow];
+            int before = 0;
+            for (int y = 0; y < n_merge; ++y)
+              before += (lc[y * kM] == vF && (int)hist[y * kM + srow] < jx) ? 1 : 0;
+            k = before < allow;
+          }
+          keep |= (k ? 1ull : 0ull) << x;
+        }
+        const float mo_e = -m * kLog2e;
+        for (int x = 0; x < n_merge; ++x) {
           float p = 0.0f;
-          if (v > vF || (at && allow > 0)) {
-            allow -= at ? 1 : 0;
-            p = fast_exp2(__fmaf_rn(v, kLog2e, mo_e));
-            lsum += p;
+          if ((keep >> x) & 1ull) {
+            p = fast_exp2(__fmaf_rn(lc[x * kM], kLog2e, mo_e));
+            merged += p;
           }
           lc[x * kM] = p;
         }
       }
+      bool ok_out = ok;
+      if (kSplitF) {
+        // the second thread of the row takes the count and the merged weight sum
+        float* mx = reinterpret_cast<float*>(koff_tab);  // the key-offset area is free after the passes
+        if (half == 0) mx[srow] = merged;
+        asm volatile("bar.sync %0, 64;" ::"r"(1 + (warp & 3)) : "memory");
+        ok_out = ok && !*abort_flag;  // both warps of the pair see the same abort state here
+        if (half == 1) {
+          merged = mx[srow];
+          n_merge = (merge_row && ok_out) ? min(rc_split, kCap) : 0;
+        }
+      }
+      lsum += merged;
       const float inv = sum_in_pv ? 1.0f / lsum : scale;
 #pragma unroll
       for (int cb = 0; cb < kOc; cb += 32) {
@@ -1447,7 +1592,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         tmem_wait_ld();
         if (row < a.n) {
           float out[32];
-          if (!ok || !row_ok) {
+          if (!ok_out || !row_ok) {
 #pragma unroll
             for (int k = 0; k < 32; ++k) out[k] = 0.0f;
           } else if (MODE == MODE_Q) {

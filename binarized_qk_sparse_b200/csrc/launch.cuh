@@ -69,8 +69,10 @@ had_status launch_tc_n(const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
 // gathers from the extended table in global memory.
 template <int D, int MODE, bool VF32, int EXP>
 had_status launch_tc_f(bool rows, const tc::TcArgs& a, dim3 grid, cudaStream_t st) {
-  if (rows) return launch_tc_t<D, tc::SEL_TOPN_FLOAT, MODE, tc::BIAS_ROWS, VF32, EXP, 1>(a, grid, st);
-  return launch_tc_t<D, tc::SEL_TOPN_FLOAT, MODE, tc::BIAS_GLOBAL, VF32, EXP, 1>(a, grid, st);
+  // float A.V: two threads per row (twice the softmax warps to hide latency)
+  constexpr int SP = (MODE == tc::MODE_F && EXP == tc::EXP_NONE) ? 2 : 1;
+  if (rows) return launch_tc_t<D, tc::SEL_TOPN_FLOAT, MODE, tc::BIAS_ROWS, VF32, EXP, SP>(a, grid, st);
+  return launch_tc_t<D, tc::SEL_TOPN_FLOAT, MODE, tc::BIAS_GLOBAL, VF32, EXP, SP>(a, grid, st);
 }
 
 template <int D, int EXP>

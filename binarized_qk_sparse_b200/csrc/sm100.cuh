@@ -58,14 +58,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 }
 // Wait for the phase with the given parity to complete, for at most
 // `max_cycles` SM clocks.  Returns false on timeout (the caller records it and
-// winds down instead of waiting on).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long max_cycles) {
+// winds down instead of waiting on).  Between tries the thread sleeps, 32 ns at
+// first and doubling up to `max_sleep_ns`, so that waiting warps leave the issue
+// slots to the working ones.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long max_cycles,
+                                          uint32_t max_sleep_ns = 128) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const long long t0 = clock64();
+  uint32_t ns = 32;
   while (true) {
+    __nanosleep(ns);
     if (mbar_try_wait(a, parity)) return true;
     if (clock64() - t0 > max_cycles) return false;
+    ns = ns < max_sleep_ns ? 2 * ns : max_sleep_ns;
   }
 }
 
