@@ -871,6 +871,18 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
               // generic path: exact logits (invalid keys -inf)
               float lg[32];
               uint32_t kinv = 0;  // keys past L (dense with bias: the sentinel, not the tile mask)
+              if (BIAS == BIAS_ROWS && !kRef) {
+                // staged bias: two logits per packed fp32x2 FMA (each element rounded once,
+                // as fmaf)
+#pragma unroll
+                for (int u = 0; u < 32; u += 2) {
+                  const float2 sf2 = make_float2((float)(int)r[32 * cc + u], (float)(int)r[32 * cc + u + 1]);
+                  const float2 b2 = make_float2(brow[-(32 * cc + u)], brow[-(32 * cc + u + 1)]);
+                  const float2 l2 = __ffma2_rn(sf2, make_float2(c, c), b2);
+                  lg[u] = (FULL || 32 * ch + u < nvalid) ? l2.x : -INFINITY;
+                  lg[u + 1] = (FULL || 32 * ch + u + 1 < nvalid) ? l2.y : -INFINITY;
+                }
+              } else {
 #pragma unroll
               for (int u = 0; u < 32; u += 4) {
                 int4 k4 = make_int4(0, 0, 0, 0);
@@ -893,6 +905,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
                   lg[u + v] = (FULL || 32 * ch + u + v < nvalid) ? l : -INFINITY;
                 }
               }
+              }
               if (kHasNorm && pass == P_NORM) {
                 float tm = -INFINITY;
 #pragma unroll
@@ -907,17 +920,20 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
                 for (int u = 0; u < 32; ++u) ex[u] = fast_exp2(__fmaf_rn(lg[u], kLog2e, mo2));
                 lsum += sum32(ex);
               } else if (kHasRadix && pass == P_FBIN) {
-                // bins of the row's logits (min(fmaf(l, sc, off), kFbTop), monotone in l):
-                // bin b at word b of the row's column; bin 0 (below the window) is not counted
+                // bins of the row's logits: u = min(max(fmaf(l, sc, off), kFbMg), kFbTop) is
+                // monotone in l; bin b at word b of the row's column.  Every key is counted
+                // (no branch): keys below the window land in bin 0, which is never read,
+                // keys past L (l = -inf) too
                 if (r_state == 4) {
 #pragma unroll
-                  for (int u = 0; u < 32; ++u) {
-                    const float uu = fminf(__fmaf_rn(lg[u], fb_sc, fb_off), kFbTop);
-                    const uint32_t ad = (__float_as_uint(uu) & 0xFE00u) + hist_row;
-                    asm volatile(
-                        "{\n\t.reg .pred p;\n\tsetp.ge.f32 p, %1, %2;\n\t@p red.shared.add.u32 [%0], 1;\n\t}" ::"r"(ad),
-                        "f"(uu), "f"(kFbIn)
-                        : "memory");
+                  for (int u = 0; u < 32; u += 2) {
+                    const float2 u2 = __ffma2_rn(make_float2(lg[u], lg[u + 1]), make_float2(fb_sc, fb_sc),
+                                                 make_float2(fb_off, fb_off));
+                    const float ua = fminf(fmaxf(u2.x, kFbMg), kFbTop), ub = fminf(fmaxf(u2.y, kFbMg), kFbTop);
+                    asm volatile("red.shared.add.u32 [%0], 1;" ::"r"((__float_as_uint(ua) & 0xFE00u) + hist_row)
+                                 : "memory");
+                    asm volatile("red.shared.add.u32 [%0], 1;" ::"r"((__float_as_uint(ub) & 0xFE00u) + hist_row)
+                                 : "memory");
                   }
                 }
               } else if (kHasRadix && pass == P_RADIX) {
@@ -1069,19 +1085,23 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
             constexpr bool FULL = decltype(full_tag)::value;
             const float mo_p = -m * kLog2e;
 #pragma unroll
-            for (int u = 0; u < 32; ++u) {
-              const float sf = (float)(int)r[u];
-              float bv = 0.0f;
+            for (int u = 0; u < 32; u += 2) {
+              float2 b2;
               if (BIAS == BIAS_ROWS) {
-                bv = brow[-u];
+                b2 = make_float2(brow[-u], brow[-(u + 1)]);
               } else {
-                const int kk = ko[32 * half + u];
-                bv = __ldg(reinterpret_cast<const float*>(tab_bytes - kk));
+                b2 = make_float2(__ldg(reinterpret_cast<const float*>(tab_bytes - ko[32 * half + u])),
+                                 __ldg(reinterpret_cast<const float*>(tab_bytes - ko[32 * half + u + 1])));
               }
-              const float l = (FULL || u < nv) ? __fmaf_rn(sf, c, bv) : -INFINITY;
-              const float x = fast_exp2(__fmaf_rn(l, kLog2e, mo_p));
-              e[u] = l >= w_cut ? x : 0.0f;
-              inm |= (l >= w_lo && l <= w_hi ? 1u : 0u) << u;
+              // logits and exp arguments two at a time (packed fp32x2 FMAs, each rounded once)
+              const float2 l2 = __ffma2_rn(make_float2((float)(int)r[u], (float)(int)r[u + 1]), make_float2(c, c), b2);
+              const float la = (FULL || u < nv) ? l2.x : -INFINITY, lb = (FULL || u + 1 < nv) ? l2.y : -INFINITY;
+              const float2 x2 = __ffma2_rn(make_float2(la, lb), make_float2(kLog2e, kLog2e), make_float2(mo_p, mo_p));
+              const float xa = fast_exp2(x2.x), xb = fast_exp2(x2.y);
+              e[u] = la >= w_cut ? xa : 0.0f;
+              e[u + 1] = lb >= w_cut ? xb : 0.0f;
+              inm |= (la >= w_lo && la <= w_hi ? 1u : 0u) << u;
+              inm |= (lb >= w_lo && lb <= w_hi ? 1u : 0u) << (u + 1);
             }
           };
           if (ok_wait && jb < L) {
