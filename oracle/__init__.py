@@ -26,6 +26,7 @@ _LIB = os.path.join(_LIB_DIR, "libhad_oracle.so")
 
 MODE_FLOAT = 0
 MODE_U8I8 = 1
+MODE_U8I4 = 2
 
 
 def build(force: bool = False) -> str:
@@ -57,11 +58,13 @@ def lib():
         L.hado_sign_pack.argtypes = [P, P, I, I, I, I, P, P]
         L.hado_binary_scores.argtypes = [P, P, I, I, I, I, P, P]
         L.hado_v_quant.argtypes = [P, I, I, I, I, P, P, P]
+        L.hado_v_quant4.argtypes = [P, I, I, I, I, P, P, P]
         L.hado_logits.argtypes = [P, P, I, I, I, I, P, P, I, I, I, P, P, P]
         L.hado_attention.argtypes = [P, P, P, I, I, I, I, P, P, I, I, I, P, P, I, I, P, I64, P, P, P, P, P, P,
                                      P, P, P, P]
         L.hado_dense_attention.argtypes = [P, P, P, I, I, I, I, P, P, I, I, I, I, P, I64, P]
-        for f in (L.hado_channel_mean, L.hado_sign_pack, L.hado_binary_scores, L.hado_v_quant, L.hado_logits,
+        for f in (L.hado_channel_mean, L.hado_sign_pack, L.hado_binary_scores, L.hado_v_quant, L.hado_v_quant4,
+                  L.hado_logits,
                   L.hado_attention, L.hado_dense_attention):
             f.restype = I
         _lib = L
@@ -125,14 +128,18 @@ def binary_scores(qbits, kbits, d, seqlens=None):
     return S
 
 
-def v_quant(V, seqlens=None):
-    """Per-channel symmetric int8 V: (Vq [B,H,n,d] int8, scale [B,H,d] fp32)."""
+def v_quant(V, seqlens=None, bits=8):
+    """Per-channel symmetric int8 V (bits=8: [-127, 127], scale absmax/127) or 4-bit
+    V (bits=4: [-7, 7], scale absmax/7): (Vq [B,H,n,d] int8, scale [B,H,d] fp32)."""
     V = _f32(V)
     B, H, n, d = V.shape
     s = _seq(seqlens)
     Vq = np.zeros((B, H, n, d), np.int8)
     sc = np.zeros((B, H, d), np.float32)
-    _check(lib().hado_v_quant(_p(V), B, H, n, d, _p(s), _p(Vq), _p(sc)), "v_quant")
+    fn = lib().hado_v_quant if bits == 8 else lib().hado_v_quant4
+    if bits not in (4, 8):
+        raise ValueError("bits must be 8 or 4")
+    _check(fn(_p(V), B, H, n, d, _p(s), _p(Vq), _p(sc)), "v_quant")
     return Vq, sc
 
 

@@ -38,6 +38,9 @@
  *   - V scale s_c = absmax_c / 127 in fp32 (1 when absmax is 0);
  *     V_q = clamp(rint(V / s_c), -127, 127), fp32 division, half-to-even.
  *   - A_q = floor(255 p + 0.5) from the normalized fp64 p.
+ *   - 4-bit V (mode 2; BinaryAttention's conclusion names lower-bit V as future
+ *     work without defining it): the int8 scheme with 4 bits, s_c = absmax_c / 7,
+ *     V_q = clamp(rint(V / s_c), -7, 7); O = sum_j A_q V_q * s_c / 255 as in mode 1.
  */
 #include <math.h>
 #include <stdint.h>
@@ -159,7 +162,11 @@ int hado_binary_scores(const uint32_t* qbits, const uint32_t* kbits, int B, int 
 }
 
 /* Per-channel symmetric int8 quantization of V (BinaryAttention §2.4, V bullet). */
-int hado_v_quant(const float* V, int B, int H, int n, int d, const int32_t* seqlens, int8_t* Vq, float* scale) {
+/* Per-channel symmetric quantization of V to the integers [-qmax, qmax] with
+ * scale absmax / qmax: qmax = 127 is the int8 V of BinaryAttention §2.4 (V
+ * bullet), qmax = 7 the 4-bit V of mode 2. */
+static int v_quant_q(const float* V, int B, int H, int n, int d, const int32_t* seqlens, float qmax, int8_t* Vq,
+                     float* scale) {
   if (!V || !Vq || !scale) return HADO_ERR_ARG;
 #pragma omp parallel for schedule(static)
   for (int64_t bh = 0; bh < (int64_t)B * H; ++bh) {
@@ -171,14 +178,14 @@ int hado_v_quant(const float* V, int B, int H, int n, int d, const int32_t* seql
         float a = fabsf(Vh[(size_t)i * d + c]);
         if (a > amax) amax = a;
       }
-      float s = (amax > 0.0f) ? amax / 127.0f : 1.0f;
+      float s = (amax > 0.0f) ? amax / qmax : 1.0f;
       scale[(size_t)bh * d + c] = s;
       for (int i = 0; i < n; ++i) {
         int8_t qv = 0;
         if (i < L) {
           float r = rintf(Vh[(size_t)i * d + c] / s);
-          if (r > 127.0f) r = 127.0f;
-          if (r < -127.0f) r = -127.0f;
+          if (r > qmax) r = qmax;
+          if (r < -qmax) r = -qmax;
           qv = (int8_t)r;
         }
         Vq[((size_t)bh * n + i) * (size_t)d + c] = qv;
@@ -186,6 +193,15 @@ int hado_v_quant(const float* V, int B, int H, int n, int d, const int32_t* seql
     }
   }
   return HADO_OK;
+}
+
+int hado_v_quant(const float* V, int B, int H, int n, int d, const int32_t* seqlens, int8_t* Vq, float* scale) {
+  return v_quant_q(V, B, H, n, d, seqlens, 127.0f, Vq, scale);
+}
+
+/* 4-bit V (mode 2): integers in [-7, 7], scale absmax / 7. */
+int hado_v_quant4(const float* V, int B, int H, int n, int d, const int32_t* seqlens, int8_t* Vq, float* scale) {
+  return v_quant_q(V, B, H, n, d, seqlens, 7.0f, Vq, scale);
 }
 
 /* Bias b_ij for head h (readings stated in the header): the relative-position
@@ -253,7 +269,7 @@ int hado_logits(const uint32_t* qbits, const uint32_t* kbits, int B, int H, int 
 }
 
 /*
- * The whole forward pass.  mode 0 = float A.V, mode 1 = uint8 A x int8 V.
+ * The whole forward pass.  mode 0 = float A.V, mode 1 = uint8 A x int8 V, mode 2 = uint8 A x 4-bit V.
  * rows: optional list of flat row ids ((b*H + h)*n + i); NULL = all B*H*n rows.
  * Outputs (row-major over the selected rows):
  *   O   [nrows][d]  fp64 (required)
@@ -269,7 +285,7 @@ int hado_attention(const float* Q, const float* K, const float* V, int B, int H,
                    int32_t* idx, uint8_t* Aq, double* P, float* mu_q_out, float* mu_k_out, uint32_t* qbits_out,
                    uint32_t* kbits_out, int8_t* Vq_out, float* vscale_out) {
   if (!Q || !K || !V || !O || B <= 0 || H <= 0 || n <= 0 || d <= 0 || d % 32 != 0 || N < 0) return HADO_ERR_ARG;
-  if (mode != 0 && mode != 1) return HADO_ERR_ARG;
+  if (mode != 0 && mode != 1 && mode != 2) return HADO_ERR_ARG;
   if (table && !(gh == 0 && gw == 0 && prefix == 0) &&
       (gh <= 0 || gw <= 0 || prefix < 0 || (int64_t)gh * gw + prefix != n))
     return HADO_ERR_ARG;
@@ -297,7 +313,8 @@ int hado_attention(const float* Q, const float* K, const float* V, int B, int H,
   hado_channel_mean(K, B, H, n, d, seqlens, mu_k);
   hado_sign_pack(Q, mu_q, B, H, n, d, seqlens, qb);
   hado_sign_pack(K, mu_k, B, H, n, d, seqlens, kb);
-  hado_v_quant(V, B, H, n, d, seqlens, Vq, vs);
+  if (mode == 2) hado_v_quant4(V, B, H, n, d, seqlens, Vq, vs);
+  else hado_v_quant(V, B, H, n, d, seqlens, Vq, vs);
 
   int64_t total = rows ? nrows : (int64_t)nbh * n;
   int failed = 0;

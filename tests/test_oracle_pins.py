@@ -503,3 +503,49 @@ def test_attention_codes_round_half_up(oracle_mod, L, code):
     np.testing.assert_array_equal(A[:L, :L], np.full((L, L), code, np.uint8))
     assert not A[:, L:].any() and not A[L:].any()
     assert 255.0 / L == code - 0.5
+
+
+# ----------------------------------------------------------------------------- 4-bit V (mode 2)
+
+def test_v_quant4_rounds_half_to_even_and_reconstructs(oracle_mod):
+    """4-bit V: absmax 7 gives scale exactly 1, so halves are exact ties: rint
+    (half to even), not half-away or floor(x + 0.5); every value reconstructs
+    within s/2, and the codes stay in [-7, 7]."""
+    n, d = 10, 64
+    V = _rng(41).standard_normal((2, 3, n, d)).astype(np.float32)
+    V[0, 0, :, 0] = [7.0, 0.5, -0.5, 1.5, -1.5, 2.5, -2.5, 6.5, -6.5, 0.0]
+    Vq, sc = oracle_mod.v_quant(V, bits=4)
+    assert sc[0, 0, 0] == np.float32(1.0)
+    np.testing.assert_array_equal(Vq[0, 0, :, 0], [7, 0, 0, 2, -2, 2, -2, 6, -6, 0])
+    assert np.abs(Vq).max() <= 7
+    err = np.abs(Vq.astype(np.float64) * sc[:, :, None, :] - V)
+    assert np.all(err <= sc[:, :, None, :] * (0.5 + 1e-6))
+    # the scale is absmax / 7 per (batch, head, channel)
+    np.testing.assert_array_equal(sc, (np.abs(V).max(axis=2) / np.float32(7.0)).astype(np.float32))
+
+
+def test_u8i4_output_equals_independent_numpy(oracle_mod):
+    """Mode 2 (uint8 A x 4-bit V) against numpy: p from an independent dense
+    attention, A_q = floor(255 p + 0.5), V_q = clip(rint(V / (absmax / 7)), -7, 7),
+    O = (A_q @ V_q) * s / 255."""
+    Q, K, V, bias = _small_case(12, with_bias=False)
+    B, H, n, d = Q.shape
+    r = oracle_mod.attention(Q, K, V, N=0, mode=2)
+    for b in range(B):
+        for h in range(H):
+            mq = np.float32(np.sum(Q[b, h].astype(np.float64), axis=0) / n)
+            mk = np.float32(np.sum(K[b, h].astype(np.float64), axis=0) / n)
+            S = (np.where(Q[b, h] < mq, -1.0, 1.0) @ np.where(K[b, h] < mk, -1.0, 1.0).T)
+            l = (S * np.float64(np.float32(1 / 8.0))).astype(np.float32).astype(np.float64)
+            p = np.exp(l - l.max(axis=1, keepdims=True))
+            p /= p.sum(axis=1, keepdims=True)
+            A = np.floor(255.0 * p + 0.5)
+            s4 = (np.abs(V[b, h]).max(axis=0) / np.float32(7.0)).astype(np.float32)
+            Vq = np.clip(np.rint(V[b, h] / s4), -7, 7)
+            ref = (A @ Vq) * s4.astype(np.float64) / 255.0
+            assert np.max(np.abs(r.O[b, h] - ref)) <= 1e-9 * np.max(np.abs(V))
+    # and it stays within the closed-form bound of the float output
+    rf = oracle_mod.attention(Q, K, V, N=0, mode=0, want_probs=True)
+    s4 = (np.abs(V).max(axis=2) / 7.0)
+    bound = (0.5 / 255) * np.abs(V).sum(axis=2, keepdims=True) + 0.5 * s4[:, :, None, :] * 1.0
+    assert np.all(np.abs(r.O - rf.O) <= bound + 1e-9)
