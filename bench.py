@@ -57,6 +57,10 @@ WORKLOADS = {
     "stress_u8i8": ("stress", 0, "u8i8"),
     # head dim 128 (the BinaryAttention kernel benchmark's head dim)
     "deit_d128": ("deit_d128", 0, "u8i8"),
+    # 4-bit V (uint8 A x per-channel 4-bit V, two codes per byte)
+    "deit_u8i4": ("deit", 0, "u8i4"),
+    "stress_u8i4": ("stress", 0, "u8i4"),
+    "stress_topn_u8i4": ("stress", 1920, "u8i4"),
     "t5_1024_d128": ("t5_1024_d128", 120, "float"),
     # the library's dense comparison mode: standard bf16 attention on the unbinarized inputs
     "deit_dense_ref": ("deit", 0, "ref"),
@@ -135,13 +139,14 @@ def alu_ops_per_score(mode: str, N: int, n: int, has_bias: bool) -> float:
     range test, increment) and the output pass (gather, FMA, two compares,
     exp as FFMA + ex2, select, pack)."""
     dense = N == 0 or N >= n
+    quant = mode in ("u8i8", "u8i4")
     if dense:
-        if mode == "u8i8":
+        if quant:
             w = 3.0 if has_bias else 1.0
             return (w + 1.0) + (w + 2.25)
         return (3.0 if has_bias else 1.0) + 1.0 + 0.5
     if not has_bias:
-        return 1.0 + (3.0 + (2.25 if mode == "u8i8" else 0.5))
+        return 1.0 + (3.0 + (2.25 if quant else 0.5))
     return 1.0 + 6.0 + 7.5
 
 
@@ -149,23 +154,26 @@ def kernel_bytes_per_token(mode: str, v_bytes: int, o_bytes: int, d: int = 64) -
     """Algorithmic bytes per valid token of the fused kernel.
 
     Reads the packed sign bits of Q and K (d / 8 B each), V (float mode,
-    d * v_bytes) or int8 V (uint8 mode, d bytes), and writes O (d * o_bytes).
+    d * v_bytes), int8 V (d bytes) or 4-bit V (d / 2 bytes), and writes O
+    (d * o_bytes).
     The comparison mode ("ref") reads the bf16 Q, K and V and writes O.
     """
     if mode == "ref":
         return 3 * d * v_bytes + d * o_bytes
-    v = d if mode == "u8i8" else d * v_bytes
+    v = d if mode == "u8i8" else d // 2 if mode == "u8i4" else d * v_bytes
     return d // 8 + d // 8 + v + d * o_bytes
 
 
 def path_bytes_per_token(mode: str, in_bytes: int, o_bytes: int, d: int = 64) -> int:
     """Algorithmic bytes per token of the whole path: read Q, K, V once, write and
-    read back the packed bits (and the int8 V in uint8 mode), write O once."""
+    read back the packed bits (and the int8 or 4-bit V in the uint8 modes), write O once."""
     if mode == "ref":
         return 3 * d * in_bytes + d * o_bytes
     b = 3 * d * in_bytes + 2 * (d // 8) * 2 + d * o_bytes
     if mode == "u8i8":
         b += 2 * d
+    elif mode == "u8i4":
+        b += d
     return b
 
 
@@ -290,7 +298,8 @@ def _oracle_call_s(w, N, mode, rows):
     if mode == "ref":
         oracle.dense_attention(w.Q, w.K, w.V, seqlens=w.seqlens, bias=b, rows=rows)
     else:
-        oracle.attention(w.Q, w.K, w.V, N=N, mode=1 if mode == "u8i8" else 0, seqlens=w.seqlens, bias=b, rows=rows)
+        oracle.attention(w.Q, w.K, w.V, N=N, mode={"u8i8": 1, "u8i4": 2}.get(mode, 0), seqlens=w.seqlens, bias=b,
+                         rows=rows)
     return time.perf_counter() - t0
 
 
@@ -581,7 +590,7 @@ def run_gpu(args, rank, world, local_rank):
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": max(3, args.warmup), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "u8i8" if mode == "u8i8" else ("bf16" if bf16 else "f32"),
+        "vs_baseline": None, "dtype": mode if mode in ("u8i8", "u8i4") else ("bf16" if bf16 else "f32"),
         "data": "synthetic", "config": _config(w, N, mode),
         "parallelism": f"replicas x{world} (no collective)",
         "score_ops_per_s": whole_job_rate(w.valid_scores(), world, args.steps, total_ms),
@@ -609,7 +618,7 @@ def run_gpu(args, rank, world, local_rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--steps", type=int, default=70)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="stress_topn", choices=sorted(WORKLOADS))
     ap.add_argument("--impl", default="own", choices=["own", "reference"])

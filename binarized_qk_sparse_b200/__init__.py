@@ -22,9 +22,9 @@ LIB_PATH = os.path.join(_HERE, "libhad_b200.so")
 
 HAD_OK, HAD_ERR_INVALID, HAD_ERR_UNSUPPORTED, HAD_ERR_CUDA, HAD_ERR_DEVICE, HAD_ERR_TIMEOUT = range(6)
 HAD_F32, HAD_BF16 = 0, 1
-HAD_MODE_FLOAT, HAD_MODE_U8I8 = 0, 1
-_MODES = {"float": HAD_MODE_FLOAT, "u8i8": HAD_MODE_U8I8, HAD_MODE_FLOAT: HAD_MODE_FLOAT,
-          HAD_MODE_U8I8: HAD_MODE_U8I8}
+HAD_MODE_FLOAT, HAD_MODE_U8I8, HAD_MODE_U8I4 = 0, 1, 2
+_MODES = {"float": HAD_MODE_FLOAT, "u8i8": HAD_MODE_U8I8, "u8i4": HAD_MODE_U8I4, HAD_MODE_FLOAT: HAD_MODE_FLOAT,
+          HAD_MODE_U8I8: HAD_MODE_U8I8, HAD_MODE_U8I4: HAD_MODE_U8I4}
 
 
 class HadError(RuntimeError):
@@ -96,9 +96,11 @@ def lib():
         L.had_topn_indices.argtypes = [P, P, SP, BP, P, P, I, P, P, SZ, P]
         L.had_attention_codes_u8.argtypes = [P, P, P, SP, BP, P, P, I, I, I, P, P, SZ, P]
         L.had_quantize_v.argtypes = [P, SP, P, P, P, SZ, P]
+        L.had_quantize_v4.argtypes = [P, SP, P, P, P, SZ, P]
         for f in ("had_binarize_pack", "had_binarize_pack_noalloc", "had_attention", "had_attention_host",
                   "had_dense_reference_mode", "had_scores_int",
-                  "had_topn_indices", "had_attention_codes_u8", "had_quantize_v", "had_get_device_status"):
+                  "had_topn_indices", "had_attention_codes_u8", "had_quantize_v", "had_quantize_v4",
+                  "had_get_device_status"):
             getattr(L, f).restype = I
         L.had_attention_scores.argtypes = [P, P, SP, P, P, SZ, P]
         L.had_attention_scores.restype = I
@@ -398,18 +400,27 @@ def had_attention_codes_u8(Q, K, V, row_begin, row_end, N=0, seqlens=None, bias=
     return A
 
 
-def had_quantize_v(V, seqlens=None, workspace=None, stream=None):
-    """Per-channel int8 V [B,H,n,d] and its fp32 scales [B,H,d]."""
+def _quantize(fn, mode, V, seqlens, workspace, stream):
     _check_dev(V, seqlens)
     B, H, n, d = V.shape
     shp = make_shape(V, seqlens)
-    ws = _workspace(lib().had_attention_workspace_size(ctypes.byref(shp), 0, HAD_MODE_U8I8, None), V.device,
+    ws = _workspace(lib().had_attention_workspace_size(ctypes.byref(shp), 0, mode, None), V.device,
                     workspace, stream)
     Vq = torch.empty((B, H, n, d), dtype=torch.int8, device=V.device)
     sc = torch.empty((B, H, d), dtype=torch.float32, device=V.device)
-    st = lib().had_quantize_v(_ptr(V), ctypes.byref(shp), _ptr(Vq), _ptr(sc), _ptr(ws), ws.numel(), _stream(stream))
-    _raise(st, "had_quantize_v")
+    st = getattr(lib(), fn)(_ptr(V), ctypes.byref(shp), _ptr(Vq), _ptr(sc), _ptr(ws), ws.numel(), _stream(stream))
+    _raise(st, fn)
     return Vq, sc
+
+
+def had_quantize_v(V, seqlens=None, workspace=None, stream=None):
+    """Per-channel int8 V [B,H,n,d] and its fp32 scales [B,H,d]."""
+    return _quantize("had_quantize_v", HAD_MODE_U8I8, V, seqlens, workspace, stream)
+
+
+def had_quantize_v4(V, seqlens=None, workspace=None, stream=None):
+    """Per-channel 4-bit V (codes in [-7, 7], one per int8) [B,H,n,d] and its fp32 scales [B,H,d]."""
+    return _quantize("had_quantize_v4", HAD_MODE_U8I4, V, seqlens, workspace, stream)
 
 
 def had_get_device_status() -> int:

@@ -103,7 +103,9 @@ __host__ __device__ constexpr bool sel_dense(int sel) { return sel == SEL_DENSE 
 // V stages: three (the P.V tiles of dense and no-bias top-N kinds load further
 // ahead), two for top-N with a bias and for fp32 V (their shared memory is fuller)
 __host__ __device__ constexpr int v_stages(int sel, bool vf32) { return (sel == SEL_TOPN_FLOAT || vf32) ? 2 : 3; }
-enum { MODE_F = 0, MODE_Q = 1 };
+// MODE_Q4: uint8 A x 4-bit V (two keys per byte of V^T in HBM, expanded to the
+// int8 MMA operand in shared memory by the TMA warp's lanes); otherwise as MODE_Q
+enum { MODE_F = 0, MODE_Q = 1, MODE_Q4 = 2 };
 enum { EXP_NONE = 0, EXP_IDX = 1, EXP_CODES = 2, EXP_SCORES = 3 };
 enum { P_DONE = 0, P_NORM, P_LEVELS, P_FBIN, P_RADIX, P_COLLECT, P_KEPT_NORM, P_PV, P_IDX, P_CODES, P_SCORES };
 
@@ -118,6 +120,7 @@ struct TcArgs {
   const void* v_raw;       // V as given, [BH][n][64] bf16 or fp32 (float mode)
   int v_f32;               // 1 if v_raw is fp32
   const float* vscale;     // [BH][64]
+  const uint8_t* vq4;      // MODE_Q4: packed 4-bit V^T [BH][D][n_pad / 2], key 2k in the low nibble of byte k
   const float* table;      // [H][th][tw] or null
   int gh, gw, prefix, th, tw;
   const float* bminmax;    // [H][2] min/max of each head's table (0 included with class tokens)
@@ -233,6 +236,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
   constexpr int kPan = D / 64;      // 64-channel panels of the Q~, K~ and V tiles
   constexpr uint32_t kTmemCols = tmem_cols(D);
   constexpr bool kRef = SEL == SEL_REF;        // the unbinarized comparison mode
+  constexpr bool kQuant = MODE != MODE_F;       // uint8 A x int8 (or 4-bit) V
   constexpr int kVStages = v_stages(SEL, VF32);
   constexpr bool kDense = sel_dense(SEL);
   static_assert(SPLIT == 1 || kDense || (SEL == SEL_TOPN_INT && EXPORT == EXP_NONE) ||
@@ -359,7 +363,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
       bulk_load(sm + SM::kBiasTab, a.expb + (size_t)h * a.ext_E, (uint32_t)a.ext_E * 4u, &bars[B_BIAS]);
     }
     prefetch_tensormap(&a.tm_k);
-    if (EXPORT == EXP_NONE) prefetch_tensormap(MODE == MODE_Q ? &a.tm_vq : &a.tm_v);
+    if (EXPORT == EXP_NONE && MODE != MODE_Q4) prefetch_tensormap(MODE == MODE_Q ? &a.tm_vq : &a.tm_v);
     if (kRef) {  // the raw Q tile: rows past the tensor read as zeros, other heads' rows are never stored
       mbar_arrive_expect_tx(&bars[B_QFULL], kM * D * 2);
 #pragma unroll
@@ -416,7 +420,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         lt[lev * 32 + lane] = __shfl_sync(0xffffffffu, v, lev & 31);
       }
     }
-    if (MODE == MODE_Q && EXPORT == EXP_NONE && tid < D) dq[tid] = __fdiv_rn(a.vscale[(size_t)bh * D + tid], 255.0f);
+    if (kQuant && EXPORT == EXP_NONE && tid < D) dq[tid] = __fdiv_rn(a.vscale[(size_t)bh * D + tid], 255.0f);
     if (HAS_BIAS && BIAS != BIAS_ROWS && a.koff_mode == kKoffTable)
       for (int j = tid; j < a.n_pad; j += kM) koff_tab[j] = 4 * key_offset(a, j, L);  // in bytes
     fence_proxy_async();
@@ -485,16 +489,75 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
   const bool k_res = ntiles <= kKStages;
   bool first_pass = true;
   int v_pref = 0;  // producer: V tiles of the P.V pass already issued
+  // producer, 4-bit V: the packed V^T rows (32 bytes = 64 keys per channel row, D / 32
+  // rows per lane) of tile q4_tile, loaded ahead of their expansion
+  uint4 q4_next[MODE == MODE_Q4 ? D / 32 : 1][2];
+  int q4_tile = -1;
+  auto q4_fetch = [&](int t) {
+    if (MODE != MODE_Q4) return;
+    const uint8_t* src = a.vq4 + (size_t)bh * D * (a.n_pad / 2) + (size_t)t * (kN / 2);
+#pragma unroll
+    for (int rr = 0; rr < (MODE == MODE_Q4 ? D / 32 : 1); ++rr) {
+      const uint4* sp = reinterpret_cast<const uint4*>(src + (size_t)(lane + 32 * rr) * (a.n_pad / 2));
+      q4_next[rr][0] = __ldg(sp);
+      q4_next[rr][1] = __ldg(sp + 1);
+    }
+    q4_tile = t;
+  };
   while (pass != P_DONE) {
     const bool pv = (pass == P_PV);
     // ============================================================== producer warp
     if (warp == kProdWarp) {
       auto load_v = [&](int t) {
         const uint32_t vs = g_v % kVStages;
+        if (MODE == MODE_Q4) {
+          // 4-bit V: every lane expands D / 32 channel rows of the packed tile (32 bytes:
+          // keys 64t ... 64t + 63) into the int8 V^T operand ([D][64], 64-byte swizzle:
+          // 16-byte chunk q of row c at q ^ ((c >> 1) & 3)), then lane 0 marks it full.
+          // The packed rows come from registers loaded one call earlier (the calls go
+          // t = 0, 1, 2, ... in every P.V pass), so their latency overlaps a tile of work.
+          if (q4_tile != t) q4_fetch(t);
+          uint4 cur[D / 32][2];
+#pragma unroll
+          for (int rr = 0; rr < D / 32; ++rr) { cur[rr][0] = q4_next[rr][0]; cur[rr][1] = q4_next[rr][1]; }
+          if (t + 1 < ntiles) q4_fetch(t + 1);
+          const bool free_ok = __all_sync(0xffffffffu, g_v < (uint32_t)kVStages ||
+                                                           bounded_wait(B_VEMPTY + vs, ((g_v / kVStages) - 1) & 1));
+          if (free_ok && !*abort_flag) {
+            uint8_t* dst = sm + SM::kV + vs * SM::kVStage;
+#pragma unroll
+            for (int rr = 0; rr < D / 32; ++rr) {
+              const int c = lane + 32 * rr;
+              const uint32_t pw[8] = {cur[rr][0].x, cur[rr][0].y, cur[rr][0].z, cur[rr][0].w,
+                                      cur[rr][1].x, cur[rr][1].y, cur[rr][1].z, cur[rr][1].w};  // 8 keys per word
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {  // 16 keys per 16-byte chunk: packed words 2q, 2q + 1
+                uint32_t o[4];
+#pragma unroll
+                for (int hw = 0; hw < 2; ++hw) {
+                  const uint32_t w = pw[2 * q + hw];
+                  // nibbles to signed bytes: x | 0xF0 where bit 3 is set (8 * 0x1E = 0xF0, no
+                  // carry between bytes); even keys in the low nibbles, odd keys in the high
+                  uint32_t lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu;
+                  lo |= (lo & 0x08080808u) * 0x1Eu;
+                  hi |= (hi & 0x08080808u) * 0x1Eu;
+                  o[2 * hw] = __byte_perm(lo, hi, 0x5140);
+                  o[2 * hw + 1] = __byte_perm(lo, hi, 0x7362);
+                }
+                *reinterpret_cast<uint4*>(dst + c * 64 + ((q ^ ((c >> 1) & 3)) * 16)) = make_uint4(o[0], o[1], o[2], o[3]);
+              }
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars[B_VFULL + vs]);
+          }
+          ++g_v;
+          return;
+        }
         if (lane == 0 && g_v >= (uint32_t)kVStages) bounded_wait(B_VEMPTY + vs, ((g_v / kVStages) - 1) & 1);
         if (lane == 0 && !*abort_flag) {
           uint8_t* dst = sm + SM::kV + vs * SM::kVStage;
-          if (MODE == MODE_Q) {  // int8 V^T: D channels x 64 keys in one box
+          if (kQuant) {  // int8 V^T: D channels x 64 keys in one box
             mbar_arrive_expect_tx(&bars[B_VFULL + vs], D * kN);
             tma_load_2d(dst, &a.tm_vq, t * kN, bh * D, &bars[B_VFULL + vs]);
           } else {  // bf16 V: one [64 keys][64 channels] box per panel (+ the residual panels)
@@ -538,7 +601,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         if (kRef && first_pass) bounded_wait(B_QFULL, 0);
         // P.V: uint8 codes x int8 V^T (N = D, one MMA per K-step), or bf16 P x bf16 V
         // (N = 64 per 64-channel panel)
-        const uint32_t id_pv = (MODE == MODE_Q) ? idesc_i8(kM, D, false, true, false) : idesc_bf16(kM, 64, true);
+        const uint32_t id_pv = (kQuant) ? idesc_i8(kM, D, false, true, false) : idesc_bf16(kM, 64, true);
         auto issue_scores = [&](int t) {
           const uint32_t gk = g_k + (uint32_t)t, buf = (g_s + (uint32_t)t) % kSBufs;
           const uint32_t st = k_res ? (uint32_t)t : gk % kKStages;
@@ -574,7 +637,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
             if (bounded_wait(B_VFULL + vs, (gv / kVStages) & 1)) {
               tc_fence_after();
               const uint32_t vbase = smem_u32(sm + SM::kV + vs * SM::kVStage);
-              if (MODE == MODE_Q) {
+              if (kQuant) {
 #pragma unroll
                 for (int k = 0; k < kN / 32; ++k)  // K-step k = key chunk k: codes at columns 32k
                   mma_i8_ts(tmem + kColO, tmem + colP + 32 * k, sdesc(vbase + 32 * k, 16, 512, kSwizzle64B), id_pv,
@@ -625,7 +688,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
       constexpr bool kHasLevels = !kDense;
       constexpr bool kHasNorm = kDense;
       constexpr bool kHasRadix = SEL == SEL_TOPN_FLOAT;
-      constexpr bool kHasKeptNorm = SEL == SEL_TOPN_FLOAT && (MODE == MODE_Q || EXPORT == EXP_CODES);
+      constexpr bool kHasKeptNorm = SEL == SEL_TOPN_FLOAT && (kQuant || EXPORT == EXP_CODES);
       constexpr bool kHasIdx = EXPORT == EXP_IDX;
       constexpr bool kHasCodes = EXPORT == EXP_CODES;
       constexpr bool kHasPv = EXPORT == EXP_NONE;
@@ -747,7 +810,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         // ---- P (or uint8 A) of one 32-key chunk into TMEM, or codes to global (export)
         auto emit = [&](const float (&e)[32], int ch) {
           const int jb = j0 + 32 * ch;
-          if (kHasCodes || MODE == MODE_Q) {
+          if (kHasCodes || kQuant) {
             // uint8 codes floor(255 p + 0.5): every kept weight is at most the row's
             // normalizer, so e * (255 / normalizer) + 0.5 < 256 and no clamp is needed
             uint32_t wq[8];
@@ -796,7 +859,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
             if (jb >= L && pass != P_CODES) {
               // every key of the chunk lies past L: nothing to count or sum; P is 0
               if (pv) {
-                if (MODE == MODE_Q) {
+                if (kQuant) {
                   const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
                   tmem_st8(tl + colP + 32 * ch, z);
                 } else {
@@ -1183,7 +1246,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
           tie_seen += c0 + c1;
           if (ok_wait) {
             if (jb >= L) {
-              if (MODE == MODE_Q) {
+              if (kQuant) {
                 const uint32_t z[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
                 tmem_st8(tl + colP + 32 * half, z);
               } else {
@@ -1279,7 +1342,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
           rF = keff - gt;
           cut = rF < eq ? 1 : 0;
           ls += (float)rF * fast_exp2((F - m) * kLog2e);
-          scale = (MODE == MODE_Q || EXPORT == EXP_CODES) ? 255.0f / ls : 1.0f / ls;
+          scale = (kQuant || EXPORT == EXP_CODES) ? 255.0f / ls : 1.0f / ls;
           sF = sN;
           // this row's weight per level: exp(l - m) above the threshold, the tie weight at it, 0 below
           float* wt = reinterpret_cast<float*>(hist);
@@ -1431,7 +1494,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
       } else if (pass == P_KEPT_NORM) {
         scale = 255.0f / lsum;
       } else if (pass == P_NORM) {
-        scale = (MODE == MODE_Q || EXPORT == EXP_CODES) ? 255.0f / lsum : 1.0f / lsum;
+        scale = (kQuant || EXPORT == EXP_CODES) ? 255.0f / lsum : 1.0f / lsum;
       }
     }
     if (kSplit == 2 && SEL == SEL_TOPN_INT && pass == P_LEVELS) {
@@ -1468,7 +1531,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
     else if (any_refine) next = P_RADIX;
     else if (any_collect) next = P_COLLECT;
     else if (EXPORT == EXP_IDX) next = P_IDX;
-    else if ((EXPORT == EXP_CODES || MODE == MODE_Q) && SEL == SEL_TOPN_FLOAT && pass != P_KEPT_NORM) next = P_KEPT_NORM;
+    else if ((EXPORT == EXP_CODES || kQuant) && SEL == SEL_TOPN_FLOAT && pass != P_KEPT_NORM) next = P_KEPT_NORM;
     else if (EXPORT == EXP_CODES) next = P_CODES;
     else next = P_PV;
     if ((next == P_RADIX || next == P_FBIN) && tid < kM)
@@ -1615,7 +1678,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
           if (!ok_out || !row_ok) {
 #pragma unroll
             for (int k = 0; k < 32; ++k) out[k] = 0.0f;
-          } else if (MODE == MODE_Q) {
+          } else if (kQuant) {
 #pragma unroll
             for (int k = 0; k < 32; ++k) out[k] = (float)(int)o[k] * dq[c0 + cb + k];
           } else {

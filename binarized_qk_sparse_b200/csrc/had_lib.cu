@@ -120,8 +120,13 @@ struct Ws {
   size_t qbits, kpm, sums, amax, vqT, vscale, bminmax, bext, expb, vhi, vlo, total;
 };
 
-Ws ws_layout(const had_shape* s, bool quant, const had_relpos_bias* bias_desc) {
+// Bits of the quantized V of a mode: 0 (float V), 8 (int8), 4 (packed 4-bit).
+int vbits_of(had_mode mode) { return mode == HAD_MODE_U8I8 ? 8 : mode == HAD_MODE_U8I4 ? 4 : 0; }
+bool mode_ok(had_mode mode) { return mode == HAD_MODE_FLOAT || mode == HAD_MODE_U8I8 || mode == HAD_MODE_U8I4; }
+
+Ws ws_layout(const had_shape* s, int vbits, const had_relpos_bias* bias_desc) {
   const bool bias = bias_desc && bias_desc->table;
+  const bool quant = vbits != 0;
   Dims d = dims_of(s);
   Ws w{};
   size_t off = 0;
@@ -131,7 +136,7 @@ Ws ws_layout(const had_shape* s, bool quant, const had_relpos_bias* bias_desc) {
   w.amax = w.vqT = w.vscale = w.bminmax = 0;
   if (quant) {
     w.amax = off; off += align_up((size_t)d.BH * d.nchunks * d.d * 4);
-    w.vqT = off; off += align_up((size_t)d.BH * d.d * d.n_pad);
+    w.vqT = off; off += align_up((size_t)d.BH * d.d * (vbits == 4 ? d.n_pad / 2 : d.n_pad));
     w.vscale = off; off += align_up((size_t)d.BH * d.d * 4);
   }
   w.bext = w.expb = 0;
@@ -198,14 +203,21 @@ had_status encode_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, u
   return HAD_OK;
 }
 
-__global__ void k_untranspose_vq(const int8_t* vqT, int BH, int n, int d, int n_pad, int8_t* Vq) {
+// V^T codes back to [BH][n][d] int8 (a 4-bit code sign-extended from its nibble).
+__global__ void k_untranspose_vq(const int8_t* vqT, int BH, int n, int d, int n_pad, int vbits, int8_t* Vq) {
   const size_t total = (size_t)BH * n * d;
   for (size_t e = blockIdx.x * (size_t)blockDim.x + threadIdx.x; e < total; e += (size_t)gridDim.x * blockDim.x) {
     const int c = (int)(e % d);
     const size_t ti = e / d;
     const int i = (int)(ti % n);
     const int bh = (int)(ti / n);
-    Vq[e] = vqT[((size_t)bh * d + c) * n_pad + i];
+    if (vbits == 4) {
+      const uint8_t byte = reinterpret_cast<const uint8_t*>(vqT)[((size_t)bh * d + c) * (n_pad / 2) + i / 2];
+      const int nib = (i & 1) ? (byte >> 4) : (byte & 15);
+      Vq[e] = (int8_t)(nib >= 8 ? nib - 16 : nib);
+    } else {
+      Vq[e] = vqT[((size_t)bh * d + c) * n_pad + i];
+    }
   }
 }
 
@@ -214,7 +226,7 @@ __global__ void k_untranspose_vq(const int8_t* vqT, int BH, int n, int d, int n_
 had_status launch_prep(const had_shape* s, const void* X0, const void* X1, const void* X2, int first, int ntens,
                        double* sums, float* amax, const float* mu_in0, float* mu_out0, uint32_t* bits0,
                        int8_t* pm0, uint32_t* bits1, int8_t* pm1, int8_t* vqT, float* vscale, cudaStream_t st,
-                       unsigned* status) {
+                       unsigned* status, int vbits = 8) {
   Dims d = dims_of(s);
   PrepArgs pa{};
   pa.X[0] = X0; pa.X[1] = X1; pa.X[2] = X2;
@@ -240,7 +252,7 @@ had_status launch_prep(const had_shape* s, const void* X0, const void* X1, const
   ka.mu_out[0] = mu_out0; ka.mu_out[1] = nullptr;
   ka.bits[0] = bits0; ka.bits[1] = bits1;
   ka.pm[0] = pm0; ka.pm[1] = pm1;
-  ka.vqT = vqT; ka.vscale = vscale; ka.status = status;
+  ka.vqT = vqT; ka.vscale = vscale; ka.v_bits = vbits; ka.status = status;
   if (d.d == 32) bf ? k_pack<__nv_bfloat16, 32><<<grid, kPrepThreads, 0, st>>>(ka) : k_pack<float, 32><<<grid, kPrepThreads, 0, st>>>(ka);
   else if (d.d == 128) bf ? k_pack<__nv_bfloat16, 128><<<grid, kPrepThreads, 0, st>>>(ka) : k_pack<float, 128><<<grid, kPrepThreads, 0, st>>>(ka);
   else bf ? k_pack<__nv_bfloat16, 64><<<grid, kPrepThreads, 0, st>>>(ka) : k_pack<float, 64><<<grid, kPrepThreads, 0, st>>>(ka);
@@ -259,7 +271,8 @@ had_status validate_attention(const void* Q, const void* K, const void* V, const
   had_status r = check_shape(s);
   if (r != HAD_OK) return r;
   if ((r = check_bias(s, bias)) != HAD_OK) return r;
-  if (N < 0 || (mode != HAD_MODE_FLOAT && mode != HAD_MODE_U8I8)) return HAD_ERR_INVALID;
+  if (N < 0 || !mode_ok(mode)) return HAD_ERR_INVALID;
+  if (mode == HAD_MODE_U8I4 && EXP != EXP_NONE) return HAD_ERR_INVALID;
   if (check_qk && (!Q || !K || !aligned16(Q) || !aligned16(K))) return HAD_ERR_INVALID;
   if (EXP == EXP_NONE || EXP == EXP_CODES) {
     if (!V || !aligned16(V)) return HAD_ERR_INVALID;
@@ -274,7 +287,7 @@ had_status validate_attention(const void* Q, const void* K, const void* V, const
     if (!(alpha_q[h] > 0.0f) || !std::isfinite(alpha_q[h])) return HAD_ERR_INVALID;
   for (int h = 0; alpha_k && h < s->H; ++h)
     if (!(alpha_k[h] > 0.0f) || !std::isfinite(alpha_k[h])) return HAD_ERR_INVALID;
-  const Ws w = ws_layout(s, mode == HAD_MODE_U8I8, bias);
+  const Ws w = ws_layout(s, vbits_of(mode), bias);
   if (!workspace || ws_bytes < w.total || !aligned16(workspace)) return HAD_ERR_INVALID;
   return HAD_OK;
 }
@@ -300,13 +313,14 @@ had_status set_prep_smem(int which, int small, int dev) {
   return HAD_OK;
 }
 
-// Stage 1: statistics, sign/pack of Q and K, int8 V (uint8 mode), bias range (top-N with bias).
+// Stage 1: statistics, sign/pack of Q and K, int8 or 4-bit V (uint8 modes), bias range (top-N with bias).
 had_status prepare_stage(const void* Q, const void* K, const void* V, const had_shape* s,
                          const had_relpos_bias* bias, int N, had_mode mode, bool need_v, void* workspace,
                          cudaStream_t st, unsigned* status) {
   const bool has_bias = bias && bias->table;
-  const bool quant = (mode == HAD_MODE_U8I8);
-  const Ws w = ws_layout(s, quant, bias);
+  const int vbits = vbits_of(mode);
+  const bool quant = vbits != 0;
+  const Ws w = ws_layout(s, vbits, bias);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   uint32_t* qbits = reinterpret_cast<uint32_t*>(ws + w.qbits);
   int8_t* kpm = reinterpret_cast<int8_t*>(ws + w.kpm);
@@ -343,7 +357,7 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
     ha.first_tensor = 0;
     ha.B = s->B; ha.H = s->H; ha.n = s->n; ha.n_pad = dims_of(s).n_pad;
     ha.seqlens = s->seqlens;
-    ha.qbits = qbits; ha.kpm = kpm; ha.vqT = vqT; ha.vscale = vscale; ha.status = status;
+    ha.qbits = qbits; ha.kpm = kpm; ha.vqT = vqT; ha.vscale = vscale; ha.v_bits = vbits; ha.status = status;
     ha.bias_slice = do_v ? 3 : 2;  // relative-position tables ride along as one more grid slice
     dim3 grid(dims_of(s).BH, ha.bias_slice + (has_bias && !ba.dense ? 1 : 0));
     const int smem = (int)head_bytes;
@@ -359,7 +373,7 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
     if ((r = check_launch("k_prep_head")) != HAD_OK) return r;
   } else {
     r = launch_prep(s, Q, K, V, 0, do_v ? 3 : 2, sums, amax, nullptr, nullptr, qbits, nullptr, nullptr, kpm, vqT,
-                    vscale, st, status);
+                    vscale, st, status, vbits);
     if (r != HAD_OK) return r;
     if (has_bias && !ba.dense) {
       k_bias_tables<<<s->H, 256, 0, st>>>(ba);
@@ -456,8 +470,9 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
                         const float* alpha_k, int N, had_mode mode, void* O, had_dtype o_dtype, int32_t* idx,
                         uint8_t* codes, int row_begin, int row_end, void* workspace, cudaStream_t st,
                         unsigned* status) {
-  const bool quant = (mode == HAD_MODE_U8I8);
-  const Ws w = ws_layout(s, quant, bias);
+  const int vbits = vbits_of(mode);
+  const bool quant = vbits != 0;
+  const Ws w = ws_layout(s, vbits, bias);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   Dims d = dims_of(s);
   const bool vf32 = (s->in_dtype == HAD_F32) && !quant;
@@ -469,7 +484,9 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
                            tc::kN, CU_TENSOR_MAP_SWIZZLE_64B);
   if (r != HAD_OK) return r;
   const bool needs_v = (EXP == EXP_NONE);
-  if (needs_v && quant) {
+  if (needs_v && vbits == 4) {
+    a.vq4 = ws + w.vqT;  // packed nibbles, expanded in shared memory by the producer warp
+  } else if (needs_v && quant) {
     r = encode_2d(&a.tm_vq, CU_TENSOR_MAP_DATA_TYPE_UINT8, ws + w.vqT, d.n_pad, (uint64_t)d.BH * d.d, d.n_pad, tc::kN,
                   d.d, CU_TENSOR_MAP_SWIZZLE_64B);
     if (r != HAD_OK) return r;
@@ -515,7 +532,7 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
   }
   dim3 grid((s->n + tc::kM - 1) / tc::kM, d.BH);
   const int sel = EXP == tc::EXP_SCORES ? (int)tc::SEL_DENSE : select_kind(s, bias, N);
-  const int md = quant ? tc::MODE_Q : tc::MODE_F;
+  const int md = vbits == 4 ? tc::MODE_Q4 : quant ? tc::MODE_Q : tc::MODE_F;
   if (s->d == 128) return launch::dispatch_tc<128, EXP>(sel, md, bias_kind, vf32, rows, a, grid, st);
   return launch::dispatch_tc<64, EXP>(sel, md, bias_kind, vf32, rows, a, grid, st);
 }
@@ -581,7 +598,7 @@ had_status host_plan(const had_shape* s, had_mode mode, const had_relpos_bias* b
   p->slots = std::min(kHostSlots, p->chunks);
   had_shape sc = s0;
   sc.B = p->cb;
-  p->ws_bytes = ws_layout(&sc, mode == HAD_MODE_U8I8, has_bias ? bias : nullptr).total;
+  p->ws_bytes = ws_layout(&sc, vbits_of(mode), has_bias ? bias : nullptr).total;
   size_t off = 0;
   p->seq = off;
   off += align_up((size_t)s->B * sizeof(int32_t));
@@ -635,7 +652,7 @@ had_status host_attention(const void* Q, const void* K, const void* V, const had
   had_status r = host_plan(s, mode, bias, chunk_b, &p);
   if (r != HAD_OK) return r;
   if (!Q || !K || !V || !O || (o_dtype != HAD_F32 && o_dtype != HAD_BF16)) return HAD_ERR_INVALID;
-  if (N < 0 || (mode != HAD_MODE_FLOAT && mode != HAD_MODE_U8I8)) return HAD_ERR_INVALID;
+  if (N < 0 || !mode_ok(mode)) return HAD_ERR_INVALID;
   if (!workspace || ws_bytes < p.total || !aligned16(workspace)) return HAD_ERR_INVALID;
   for (int h = 0; alpha_q && h < s->H; ++h)
     if (!(alpha_q[h] > 0.0f) || !std::isfinite(alpha_q[h])) return HAD_ERR_INVALID;
@@ -749,7 +766,7 @@ had_status had_binarize_pack(const void* X, const had_shape* s, const float* mu_
 size_t had_attention_workspace_size(const had_shape* s, int N, had_mode mode, const had_relpos_bias* bias) {
   (void)N;
   if (check_shape(s, true) != HAD_OK || check_bias(s, bias) != HAD_OK) return 0;
-  return ws_layout(s, mode == HAD_MODE_U8I8, bias).total;
+  return ws_layout(s, vbits_of(mode), bias).total;
 }
 
 had_status had_attention(const void* Q, const void* K, const void* V, const had_shape* s,
@@ -825,12 +842,15 @@ had_status had_attention_codes_u8(const void* Q, const void* K, const void* V, c
                                   row_begin, row_end, workspace, ws_bytes, stream);
 }
 
-had_status had_quantize_v(const void* V, const had_shape* s, int8_t* Vq, float* vscale, void* workspace,
-                          size_t ws_bytes, void* stream) {
+namespace {
+
+// Shared body of had_quantize_v (8-bit) and had_quantize_v4 (4-bit).
+had_status quantize_v_bits(const void* V, const had_shape* s, int vbits, int8_t* Vq, float* vscale, void* workspace,
+                           size_t ws_bytes, void* stream) {
   had_status r = check_shape(s, true);
   if (r != HAD_OK) return r;
   if (!V || !Vq || !vscale || !aligned16(V) || (reinterpret_cast<uintptr_t>(vscale) & 3u)) return HAD_ERR_INVALID;
-  const Ws w = ws_layout(s, true, nullptr);
+  const Ws w = ws_layout(s, vbits, nullptr);
   if (!workspace || ws_bytes < w.total || !aligned16(workspace)) return HAD_ERR_INVALID;
   int dev = 0;
   cudaError_t ce = cudaGetDevice(&dev);
@@ -843,10 +863,22 @@ had_status had_quantize_v(const void* V, const had_shape* s, int8_t* Vq, float* 
   int8_t* vqT = reinterpret_cast<int8_t*>(ws + w.vqT);
   r = launch_prep(s, nullptr, nullptr, V, 2, 1, reinterpret_cast<double*>(ws + w.sums),
                   reinterpret_cast<float*>(ws + w.amax), nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, vqT,
-                  vscale, st, status);
+                  vscale, st, status, vbits);
   if (r != HAD_OK) return r;
-  k_untranspose_vq<<<1024, 256, 0, st>>>(vqT, d.BH, d.n, d.d, d.n_pad, Vq);
+  k_untranspose_vq<<<1024, 256, 0, st>>>(vqT, d.BH, d.n, d.d, d.n_pad, vbits, Vq);
   return check_launch("k_untranspose_vq");
+}
+
+}  // namespace
+
+had_status had_quantize_v(const void* V, const had_shape* s, int8_t* Vq, float* vscale, void* workspace,
+                          size_t ws_bytes, void* stream) {
+  return quantize_v_bits(V, s, 8, Vq, vscale, workspace, ws_bytes, stream);
+}
+
+had_status had_quantize_v4(const void* V, const had_shape* s, int8_t* Vq, float* vscale, void* workspace,
+                           size_t ws_bytes, void* stream) {
+  return quantize_v_bits(V, s, 4, Vq, vscale, workspace, ws_bytes, stream);
 }
 
 size_t had_dense_reference_workspace_size(const had_shape* s, const had_relpos_bias* bias) {

@@ -1,7 +1,7 @@
 // launch.cuh -- host-side launch of the fused kernel's instantiations, for one
 // head dim D per translation unit (had_lib.cu builds D = 64, attn_d128.cu D = 128,
 // so the two compile in parallel).  dispatch_tc<D, EXP> picks the instantiation
-// from the select kind, mode, bias layout and V dtype.
+// from the select kind, mode (float, int8 or 4-bit V), bias layout and V dtype.
 #pragma once
 
 #include <mutex>
@@ -80,6 +80,13 @@ had_status dispatch_tc(int sel, int mode, int bias, bool vf32, bool rows, const 
                        cudaStream_t st) {
   using namespace tc;
   if (EXP == EXP_SCORES) return launch_tc_t<D, SEL_DENSE, MODE_F, BIAS_NONE, false, EXP_SCORES, 1>(a, grid, st);
+  if constexpr (EXP == EXP_NONE) {  // 4-bit V: the output path only
+    if (mode == MODE_Q4) {
+      if (sel == SEL_DENSE) return launch_tc_b<D, SEL_DENSE, MODE_Q4, false, EXP>(bias, a, grid, st);
+      if (sel == SEL_TOPN_INT) return launch_tc_n<D, SEL_TOPN_INT, MODE_Q4, false, EXP>(a, grid, st);
+      return launch_tc_f<D, MODE_Q4, false, EXP>(rows, a, grid, st);
+    }
+  }
   if (EXP == EXP_CODES || (EXP == EXP_NONE && mode == MODE_Q)) {
     constexpr int E = EXP;
     if (sel == SEL_DENSE) return launch_tc_b<D, SEL_DENSE, MODE_Q, false, E>(bias, a, grid, st);

@@ -116,8 +116,9 @@ struct PackArgs {
   float* mu_out[2];       // optional mean outputs per tensor 0/1
   uint32_t* bits[2];      // [BH][n][D/32] per tensor 0/1 (or null)
   int8_t* pm[2];          // [BH][n_pad][D] +-1 int8 rows per tensor 0/1 (or null); +1 past L
-  int8_t* vqT;            // [BH][D][n_pad]
+  int8_t* vqT;            // [BH][D][n_pad] int8, or [BH][D][n_pad / 2] packed 4-bit (key 2k in the low nibble of byte k)
   float* vscale;          // [BH][D]
+  int v_bits;             // 8: int8 V, scale absmax/127; 4: 4-bit V, scale absmax/7
   unsigned* status;
 };
 
@@ -155,7 +156,8 @@ __global__ void __launch_bounds__(kPrepThreads) k_pack(const PackArgs a) {
       float m = 0.0f;
       const int nch_valid = (L + kChunk - 1) / kChunk;
       for (int k = 0; k < nch_valid; ++k) m = fmaxf(m, a.amax[((size_t)bh * a.nchunks + k) * kD + c]);
-      float s = (m > 0.0f) ? __fdiv_rn(m, 127.0f) : 1.0f;
+      const float qmax = a.v_bits == 4 ? 7.0f : 127.0f;
+      float s = (m > 0.0f) ? __fdiv_rn(m, qmax) : 1.0f;
       stat[c] = s;
       if (chunk == 0) a.vscale[(size_t)bh * kD + c] = s;
     }
@@ -200,21 +202,42 @@ __global__ void __launch_bounds__(kPrepThreads) k_pack(const PackArgs a) {
 #pragma unroll
         for (int u = 0; u < 8; ++u) x[u] = 0.0f;
       }
+      const float qmax = a.v_bits == 4 ? 7.0f : 127.0f;
 #pragma unroll
       for (int u = 0; u < EPT; ++u) {
         float r = rintf(__fdiv_rn(x[u], stat[cg * EPT + u]));
-        r = fminf(fmaxf(r, -127.0f), 127.0f);
+        r = fminf(fmaxf(r, -qmax), qmax);
         vt[cg * EPT + u][t] = (int8_t)(int)r;
       }
     }
     __syncthreads();
-    // write the D x 64 int8 block of V^T: row c, tokens [i0, i0+64) -- 16 bytes per thread and step
-    int8_t* dst = a.vqT + (size_t)bh * kD * a.n_pad;
-    for (int e = threadIdx.x; e < kD * 4; e += kPrepThreads) {
-      const int c = e >> 2, seg = e & 3;
-      if (i0 + seg * 16 < a.n_pad)
-        *reinterpret_cast<uint4*>(dst + (size_t)c * a.n_pad + i0 + seg * 16) =
-            *reinterpret_cast<const uint4*>(&vt[c][seg * 16]);
+    if (a.v_bits == 4) {
+      // the D x 64 block of packed 4-bit V^T: row c, bytes [i0/2, i0/2 + 32), 16 bytes per thread and step
+      uint8_t* dst = reinterpret_cast<uint8_t*>(a.vqT) + (size_t)bh * kD * (a.n_pad / 2);
+      for (int e = threadIdx.x; e < kD * 2; e += kPrepThreads) {
+        const int c = e >> 1, seg = e & 1;
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint32_t v = 0;
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int t0 = seg * 32 + 8 * k + 2 * b;
+            v |= ((((uint32_t)(uint8_t)vt[c][t0]) & 15u) | ((((uint32_t)(uint8_t)vt[c][t0 + 1]) & 15u) << 4)) << (8 * b);
+          }
+          w[k] = v;
+        }
+        *reinterpret_cast<uint4*>(dst + (size_t)c * (a.n_pad / 2) + i0 / 2 + seg * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+    } else {
+      // write the D x 64 int8 block of V^T: row c, tokens [i0, i0+64) -- 16 bytes per thread and step
+      int8_t* dst = a.vqT + (size_t)bh * kD * a.n_pad;
+      for (int e = threadIdx.x; e < kD * 4; e += kPrepThreads) {
+        const int c = e >> 2, seg = e & 3;
+        if (i0 + seg * 16 < a.n_pad)
+          *reinterpret_cast<uint4*>(dst + (size_t)c * a.n_pad + i0 + seg * 16) =
+              *reinterpret_cast<const uint4*>(&vt[c][seg * 16]);
+      }
     }
   }
 }
@@ -243,8 +266,9 @@ struct HeadArgs {
   const int32_t* seqlens;
   uint32_t* qbits;     // tensor 0 -> [BH][n][2]
   int8_t* kpm;         // tensor 1 -> [BH][n_pad][64]
-  int8_t* vqT;         // tensor 2 -> [BH][64][n_pad]
+  int8_t* vqT;         // tensor 2 -> [BH][64][n_pad] int8, or [BH][64][n_pad / 2] packed 4-bit
   float* vscale;       // [BH][64]
+  int v_bits;          // 8 or 4 (see PackArgs)
   unsigned* status;
   int bias_slice;      // grid slice y == bias_slice computes the bias tables (if launched)
 };
@@ -362,15 +386,16 @@ __global__ void __launch_bounds__(256) k_dense_bias_tables(const BiasArgs a) {
   }
 }
 
-// int8 code of x at scale sc: rint(x / sc) clamped to +-127, with x / sc the
-// correctly rounded fp32 quotient.  For |x / sc| <= 128 the product x * (1/sc)
-// is within 2^-15 of that quotient, so both round to the same integer unless the
-// product lies within 2^-12 of a half-integer; only then is the quotient computed.
-__device__ __forceinline__ int quant_i8(float x, float sc, float rsc) {
+// Integer code of x at scale sc: rint(x / sc) clamped to +-qmax (127 or 7), with
+// x / sc the correctly rounded fp32 quotient.  For |x / sc| <= 128 the product
+// x * (1/sc) is within 2^-15 of that quotient, so both round to the same integer
+// unless the product lies within 2^-12 of a half-integer; only then is the
+// quotient computed.
+__device__ __forceinline__ int quant_v(float x, float sc, float rsc, float qmax) {
   const float y = x * rsc;
   float q = rintf(y);
   if (fabsf(y - q) > 0.5f - 0x1p-12f) q = rintf(__fdiv_rn(x, sc));
-  return (int)fminf(fmaxf(q, -127.0f), 127.0f);
+  return (int)fminf(fmaxf(q, -qmax), qmax);
 }
 
 template <typename T, int kHeadThreads>
@@ -447,7 +472,7 @@ __global__ void __launch_bounds__(kHeadThreads) k_prep_head(const HeadArgs a, co
       float mx = 0.0f;
 #pragma unroll
       for (int g = 0; g < kGroups; ++g) mx = fmaxf(mx, (float)part[g][tid]);
-      const float sc = (mx > 0.0f) ? __fdiv_rn(mx, 127.0f) : 1.0f;
+      const float sc = (mx > 0.0f) ? __fdiv_rn(mx, a.v_bits == 4 ? 7.0f : 127.0f) : 1.0f;
       stat[tid] = sc;
       a.vscale[(size_t)bh * kD + tid] = sc;
     }
@@ -498,10 +523,13 @@ __global__ void __launch_bounds__(kHeadThreads) k_prep_head(const HeadArgs a, co
       }
     }
   } else {
-    // thread (channel pair, block of 16 tokens): two int8 V^T row segments of 16 bytes
+    // thread (channel pair, block of 16 tokens): two V^T row segments of 16 int8
+    // codes (16 bytes) or 16 packed 4-bit codes (8 bytes)
     const int p = tid & 31;
     const float sc0 = stat[2 * p], sc1 = stat[2 * p + 1];
     const float r0 = 1.0f / sc0, r1 = 1.0f / sc1;
+    const bool v4 = a.v_bits == 4;
+    const float qmax = v4 ? 7.0f : 127.0f;
     int off[8];  // token u of a block is = u (mod 8)
 #pragma unroll
     for (int k = 0; k < 8; ++k) off[k] = pair_off(p, k);
@@ -512,13 +540,25 @@ __global__ void __launch_bounds__(kHeadThreads) k_prep_head(const HeadArgs a, co
         const int i = blk * 16 + u;
         if (i < L) {
           const float2 x = pair_load(xs + i * kRow + off[u & 7]);
-          w0[u >> 2] |= ((uint32_t)quant_i8(x.x, sc0, r0) & 0xFFu) << (8 * (u & 3));
-          w1[u >> 2] |= ((uint32_t)quant_i8(x.y, sc1, r1) & 0xFFu) << (8 * (u & 3));
+          const uint32_t q0 = (uint32_t)quant_v(x.x, sc0, r0, qmax), q1 = (uint32_t)quant_v(x.y, sc1, r1, qmax);
+          if (v4) {
+            w0[u >> 3] |= (q0 & 15u) << (4 * (u & 7));
+            w1[u >> 3] |= (q1 & 15u) << (4 * (u & 7));
+          } else {
+            w0[u >> 2] |= (q0 & 0xFFu) << (8 * (u & 3));
+            w1[u >> 2] |= (q1 & 0xFFu) << (8 * (u & 3));
+          }
         }
       }
-      int8_t* base = a.vqT + ((size_t)bh * kD + 2 * p) * a.n_pad + blk * 16;
-      *reinterpret_cast<uint4*>(base) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
-      *reinterpret_cast<uint4*>(base + a.n_pad) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+      if (v4) {
+        uint8_t* base = reinterpret_cast<uint8_t*>(a.vqT) + ((size_t)bh * kD + 2 * p) * (a.n_pad / 2) + blk * 8;
+        *reinterpret_cast<uint2*>(base) = make_uint2(w0[0], w0[1]);
+        *reinterpret_cast<uint2*>(base + a.n_pad / 2) = make_uint2(w1[0], w1[1]);
+      } else {
+        int8_t* base = a.vqT + ((size_t)bh * kD + 2 * p) * a.n_pad + blk * 16;
+        *reinterpret_cast<uint4*>(base) = make_uint4(w0[0], w0[1], w0[2], w0[3]);
+        *reinterpret_cast<uint4*>(base + a.n_pad) = make_uint4(w1[0], w1[1], w1[2], w1[3]);
+      }
     }
   }
 }

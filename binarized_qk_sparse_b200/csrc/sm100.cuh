@@ -58,9 +58,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 }
 // Wait for the phase with the given parity to complete, for at most
 // `max_cycles` SM clocks.  Returns false on timeout (the caller records it and
-// winds down instead of waiting on).  Between tries the thread sleeps, 32 ns at
-// first and doubling up to `max_sleep_ns`, so that waiting warps leave the issue
-// slots to the working ones.
+// winds down instead of waiting on).  A wait that has not ended after
+// kSpinCycles (about a microsecond, longer than a pipeline hand-off) sleeps
+// between tries, 32 ns at first and doubling up to `max_sleep_ns`, so that warps
+// waiting a long time leave the issue slots to the working ones.
+constexpr long long kSpinCycles = 2000;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long max_cycles,
                                           uint32_t max_sleep_ns = 128) {
   const uint32_t a = smem_u32(bar);
@@ -68,10 +70,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long l
   const long long t0 = clock64();
   uint32_t ns = 32;
   while (true) {
-    __nanosleep(ns);
     if (mbar_try_wait(a, parity)) return true;
-    if (clock64() - t0 > max_cycles) return false;
-    ns = ns < max_sleep_ns ? 2 * ns : max_sleep_ns;
+    const long long dt = clock64() - t0;
+    if (dt > max_cycles) return false;
+    if (dt > kSpinCycles) {
+      __nanosleep(ns);
+      ns = ns < max_sleep_ns ? 2 * ns : max_sleep_ns;
+    }
   }
 }
 

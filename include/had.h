@@ -16,6 +16,9 @@
  *   O_i      = sum_j p_ij V_j                                   (HAD_MODE_FLOAT)
  *   O_i[c]   = (sum_j A_ij Vq_jc) * sv_c / 255,  A_ij = floor(255 p_ij + 0.5) in uint8,
  *              sv_c = absmax_{j<L} |V_jc| / 127, Vq = clamp(rint(V / sv_c), -127, 127)   (HAD_MODE_U8I8, §2.4)
+ *   O_i[c]   = the same with sv_c = absmax_{j<L} |V_jc| / 7, Vq = clamp(rint(V / sv_c), -7, 7)   (HAD_MODE_U8I4:
+ *              BinaryAttention's conclusion names lower-bit V without defining it; this is the §2.4
+ *              scheme at 4 bits)
  * Rows i >= L of O are written as 0.  Padding tokens never enter a mean, a
  * scale, a score or a softmax.
  *
@@ -34,7 +37,7 @@
  *     sticky device status word and zero the affected batch's outputs; read
  *     it with had_get_device_status().
  *   - Head dims d = 64 and 128 (d = 32 too in had_binarize_pack,
- *     had_binarize_pack_noalloc and had_quantize_v; had_scores_int is d = 64
+ *     had_binarize_pack_noalloc, had_quantize_v and had_quantize_v4; had_scores_int is d = 64
  *     only); HAD_ERR_UNSUPPORTED otherwise.  n <= 16384, H <= 256, B*H <= 65535.
  */
 #ifndef HAD_H_
@@ -60,7 +63,9 @@ typedef enum { HAD_F32 = 0, HAD_BF16 = 1 } had_dtype;
 
 typedef enum {
   HAD_MODE_FLOAT = 0,  /* float softmax and float A.V (bf16 P x bf16 V, fp32 accumulate; fp32 V exact to ~1e-5) */
-  HAD_MODE_U8I8 = 1    /* uint8 A (scale 1/255) x per-channel int8 V, int32 accumulate (BinaryAttention §2.4) */
+  HAD_MODE_U8I8 = 1,   /* uint8 A (scale 1/255) x per-channel int8 V, int32 accumulate (BinaryAttention §2.4) */
+  HAD_MODE_U8I4 = 2    /* uint8 A x per-channel 4-bit V (codes in [-7, 7], stored two per byte), int32 accumulate;
+                          had_attention, had_attention_prepare/_prepared and had_attention_host only */
 } had_mode;
 
 typedef struct {
@@ -130,7 +135,7 @@ had_status had_attention(const void* Q, const void* K, const void* V, const had_
 
 /* The same operation in two stages, for callers that time or reuse them:
  * had_attention_prepare runs the per-head statistics and the sign/pack of Q
- * and K (and the int8 V of HAD_MODE_U8I8, and the bias range of top-N with a
+ * and K (and the int8 or 4-bit V of the uint8 modes, and the bias range of top-N with a
  * bias) into `workspace`; had_attention_prepared then runs the fused
  * score/top-N/softmax/A.V kernel over that workspace.  Both must get the same
  * s, bias, N and mode; had_attention_prepared reads V only in HAD_MODE_FLOAT.
@@ -218,6 +223,14 @@ had_status had_attention_codes_u8(const void* Q, const void* K, const void* V, c
  * fp32 [B][H][d].  Needs had_attention_workspace_size(s, 0, HAD_MODE_U8I8, NULL). */
 had_status had_quantize_v(const void* V, const had_shape* s, int8_t* Vq, float* vscale, void* workspace,
                           size_t ws_bytes, void* stream);
+
+/* had_quantize_v4: the per-channel 4-bit V of HAD_MODE_U8I4, one code in
+ * [-7, 7] per int8 of Vq DEVICE [B][H][n][d] (0 for tokens i >= L; the attention
+ * kernel stores them two per byte), vscale DEVICE fp32 [B][H][d] = absmax / 7
+ * (1 where the absmax is 0).  Needs had_attention_workspace_size(s, 0,
+ * HAD_MODE_U8I4, NULL); errors as had_quantize_v. */
+had_status had_quantize_v4(const void* V, const had_shape* s, int8_t* Vq, float* vscale, void* workspace,
+                           size_t ws_bytes, void* stream);
 
 /* ---- tensor-pipe probe (a measurement aid; the pages have no counterpart) --
  * had_probe_mma_rate: the rate this GPU's tensor cores sustain on the two MMA

@@ -60,6 +60,7 @@ def test_host_validation_rejects_before_launch(L):
     assert att(_shape(m, dtype=7)) == m.HAD_ERR_INVALID
     assert att(_shape(m), N=-1) == m.HAD_ERR_INVALID
     assert att(_shape(m), mode=5) == m.HAD_ERR_INVALID
+    assert att(_shape(m), mode=3) == m.HAD_ERR_INVALID
     assert att(_shape(m), q=P(0)) == m.HAD_ERR_INVALID
     assert att(_shape(m), v=odd) == m.HAD_ERR_INVALID
     assert att(_shape(m), o=P(0)) == m.HAD_ERR_INVALID
@@ -102,10 +103,28 @@ def test_workspace_size_grows_with_mode_and_bias(L):
     bias = m.had_relpos_bias(0x30000, 14, 14, 1)
     qb = L.had_attention_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(bias))
     assert 0 < f < q < qb
+    # 4-bit V: half the bytes of the int8 V^T (n_pad = 256 keys -> 128 bytes per channel row)
+    q4 = L.had_attention_workspace_size(ctypes.byref(shp), 0, 2, None)
+    assert f < q4 < q and q - q4 >= 2 * 3 * 64 * 128
     wide = _shape(m, B=2, H=3, n=197, d=128)   # head dim 128: twice the per-token intermediates
     assert L.had_attention_workspace_size(ctypes.byref(wide), 0, 1, None) > q
     bad = _shape(m, d=96)
     assert L.had_attention_workspace_size(ctypes.byref(bad), 0, 0, None) == 0
+
+
+def test_four_bit_mode_is_the_output_path_only(L):
+    # the index and code exports and the quantizer keep their own modes; the
+    # 4-bit quantizer validates like the int8 one
+    import binarized_qk_sparse_b200 as m
+    P = ctypes.c_void_p
+    fake = P(0x10000)
+    shp = _shape(m)
+    assert L.had_quantize_v4(P(0), ctypes.byref(shp), fake, fake, fake, 1 << 30, None) == m.HAD_ERR_INVALID
+    assert L.had_quantize_v4(fake, ctypes.byref(shp), fake, P(0x10002), fake, 1 << 30, None) == m.HAD_ERR_INVALID
+    assert L.had_quantize_v4(fake, ctypes.byref(shp), fake, fake, fake, 16, None) == m.HAD_ERR_INVALID
+    bad = _shape(m, d=96)
+    assert L.had_quantize_v4(fake, ctypes.byref(bad), fake, fake, fake, 1 << 30, None) == m.HAD_ERR_UNSUPPORTED
+    assert m._MODES["u8i4"] == m.HAD_MODE_U8I4 == 2
 
 
 def test_status_strings(L):
