@@ -64,20 +64,39 @@ __host__ __device__ constexpr int levels_of(int d) { return d + 1; }
 constexpr int kRadixBins = 256;   // 16-bit counters, two per word (a row counts at most kMaxN keys)
 constexpr int kCandCap = 128;    // power of two (the collect slot wraps)
 constexpr int kSBufs = 3;
+// Top-N with a bias on rows of at least kSampleMinTiles tiles: the first level pass
+// reads one tile in kSampleStride (tile 8u + u % 8, which staggers the sample over
+// every tile position), and each row brackets its threshold level from that sample
+// with a margin of 5 binomial standard deviations.  The float-binned pass counts
+// every key exactly and so verifies the bracket; if it failed for any row, the CTA
+// runs the level pass again over every tile.
+constexpr int kSampleStride = 8;   // power of two
+constexpr int kSampleMinTiles = 64;
+__host__ __device__ constexpr int tile_at(int u, int stride) { return stride == 1 ? u : u * stride + (u & (stride - 1)); }
+// tiles u with tile_at(u, stride) < ntiles
+__host__ __device__ constexpr int tiles_in_pass(int ntiles, int stride) {
+  return stride == 1 ? ntiles : ntiles / stride + (((ntiles / stride) & (stride - 1)) < (ntiles & (stride - 1)) ? 1 : 0);
+}
 // TMEM: the score ring in columns [0, 192), O (d columns) from 192; 256 columns at
 // d = 64 (two CTAs per SM), 512 at d = 128 (one CTA per SM).
 constexpr uint32_t kColS = 0, kColO = 192;
 __host__ __device__ constexpr uint32_t tmem_cols(int d) { return d <= 64 ? 256u : 512u; }
 __host__ __device__ constexpr int ctas_per_sm(int d) { return d <= 64 ? 2 : 1; }
 constexpr long long kWaitCycles = 2000000000LL;  // default bound of a pipeline wait: about one second
-// First select pass of top-N with a bias (FBIN): u = min(fmaf(l, sc, off), kFbTop)
-// is a monotone function of the logit l; with u in [kFbMg, kFbMg + 65536) its
-// float bits carry the integer u - kFbMg in their low 16 bits, and bits 9..15 are
-// the bin (128 bins of 512 units): bin 0 holds everything below the window, bins
-// 1..126 the window, bin 127 (the clamp) only keys above it.
-constexpr float kFbMg = 12582912.0f;             // 1.5 * 2^23: unit spacing, bits 0x4B400000
-constexpr float kFbIn = kFbMg + 512.0f;          // first in-window bin
-constexpr float kFbTop = kFbMg + 127.0f * 512.0f;  // bin 127
+// First select pass of top-N with a bias (FBIN): u = sat(fmaf(l, sc, off)) in [0, 1]
+// (one saturating FMA) and w = fmaf(u, 65535, kFbMg) are monotone functions of the
+// logit l; w is an integer in [kFbMg, kFbMg + 65535] whose float bits carry w - kFbMg
+// in their low 16 bits, and bits 9..15 are the bin (128 bins of 512 units): bin 0
+// holds everything below the window, bins 1..126 the window, bin 127 the keys above
+// it (and the top edge of the window).
+constexpr float kFbMg = 12582912.0f;  // 1.5 * 2^23: unit spacing, bits 0x4B400000
+constexpr float kFbSpan = 65535.0f;
+constexpr int kFbGroup = 16;  // keys whose staged bias is read ahead of their histogram adds
+__device__ __forceinline__ float fma_sat(float x, float y, float z) {
+  float r;
+  asm("fma.rn.sat.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(x), "f"(y), "f"(z));
+  return r;
+}
 // How the softmax threads find the bias offset koff(j) = y_j * S + x_j of a key (S: table row stride):
 constexpr int kKoffTable = 0;  // per-head table in shared memory (n_pad <= kKoffTableMax)
 constexpr int kKoffWarp = 1;   // each softmax warp computes the tile's 64 offsets (double-buffered)
@@ -341,7 +360,15 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
   for (int s2 = 0; s2 < kVStages; ++s2) v_par[s2] = -1;
   // the producer issues the first K tiles before the CTA-wide setup barrier, so
   // their load latency overlaps the staging of Q
-  const int k_pre = min((L + kN - 1) / kN, kKStages);
+  bool sample_levels = false;
+  if (SEL == SEL_TOPN_FLOAT && ntiles >= kSampleMinTiles && keff < L) {
+    // weights exp(l - m) with m from the sample stay inside fp32 while (2 d c + bias range) log2 e <= 100
+    const float range = HAS_BIAS ? a.bminmax[2 * h + 1] - a.bminmax[2 * h] : 0.0f;
+    sample_levels = c > 0.0f && (2.0f * D * c + range) * 1.4426950408889634f <= 100.0f;
+  }
+  const int s_first = sample_levels ? kSampleStride : 1;  // stride of the first pass's tiles
+  const int n_sampled = tiles_in_pass(ntiles, kSampleStride);
+  const int k_pre = min(tiles_in_pass(ntiles, s_first), kKStages);
   if (warp == kMmaWarp) {
     tmem_alloc(misc, kTmemCols);
     tmem_relinquish();
@@ -370,9 +397,9 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
       for (int pn = 0; pn < kPan; ++pn)
         tma_load_2d(sQ + pn * kM * 128, &a.tm_q, 64 * pn, bh * a.n + q0, &bars[B_QFULL]);
     }
-    for (int t = 0; t < k_pre; ++t) {  // stage t = tile t, first use of every stage
-      load_k((uint32_t)t, t);
-      k_par[t] = 0;
+    for (int u = 0; u < k_pre; ++u) {  // stage u = the first pass's u-th tile, first use of every stage
+      load_k((uint32_t)u, tile_at(u, s_first));
+      k_par[u] = 0;
     }
   }
   const int row = q0 + srow;  // softmax threads
@@ -435,9 +462,11 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
   int rF = 0, cut = 0, tie_seen = 0, kept_seen = 0;
   uint32_t r_uhi = 0, r_span = 0;
   // r_state: 0 threshold known, 1 radix pass next, 2 collect pass next, 3 the
-  // window's keys are recorded during the P.V pass (kMerge), 4 FBIN pass next
+  // window's keys are recorded during the P.V pass (kMerge), 4 FBIN pass next,
+  // 5 a bracket from the sampled level pass missed (the level pass runs again)
   int r_shift = 0, r_rank = 0, r_state = 0, r_cnt = 0;
   int r_above = 0;      // keys above the first radix window (counted in that pass)
+  bool r_sampled = false;  // the FBIN bracket came from the sampled level pass
   float fb_sc = 0.0f, fb_off = 0.0f;  // r_state 4: the FBIN pass's map of logits onto bins
   // float window of the P.V pass: weight for l >= w_cut; keys in [w_lo, w_hi] are
   // the ties at F (w_lo = w_hi = w_cut = F), or, with the collect folded into
@@ -506,6 +535,10 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
   };
   while (pass != P_DONE) {
     const bool pv = (pass == P_PV);
+    // this pass's tiles: tile_at(u, p_stride) for u < npass (the sampled first level
+    // pass, or every tile); the ring counters advance by npass
+    const int p_stride = (pass == P_LEVELS && sample_levels) ? kSampleStride : 1;
+    const int npass = p_stride == 1 ? ntiles : n_sampled;
     // ============================================================== producer warp
     if (warp == kProdWarp) {
       auto load_v = [&](int t) {
@@ -574,8 +607,9 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         }
         ++g_v;
       };
-      for (int t = 0; t < ntiles; ++t) {
-        if (first_pass && t < k_pre) {
+      for (int u = 0; u < npass; ++u) {
+        const int t = tile_at(u, p_stride);
+        if (first_pass && u < k_pre) {
           ++g_k;  // issued during setup
         } else if (!k_res || first_pass) {
           const uint32_t st = k_res ? (uint32_t)t : g_k % kKStages;
@@ -626,8 +660,8 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
           mma_commit(&bars[B_SFULL + buf]);
           if (!k_res) mma_commit(&bars[B_KEMPTY + st]);
         };
-        for (int t = 0; t < kSBufs && t < ntiles; ++t) issue_scores(t);
-        for (int t = 0; t < ntiles; ++t) {
+        for (int t = 0; t < kSBufs && t < npass; ++t) issue_scores(t);
+        for (int t = 0; t < npass; ++t) {  // t counts this pass's tiles (all of them in the P.V pass)
           const uint32_t gs = g_s + (uint32_t)t, buf = gs % kSBufs;
           const uint32_t colP = kColS + buf * kN;  // P of this tile sits over its score buffer
           bounded_wait(B_TDONE + buf, (gs / kSBufs) & 1);
@@ -667,11 +701,11 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
               if (t + 1 == ntiles) mma_commit(&bars[B_OFULL]);
             }
           }
-          if (t + kSBufs < ntiles) issue_scores(t + kSBufs);
+          if (t + kSBufs < npass) issue_scores(t + kSBufs);
         }
       }
-      g_k += ntiles;
-      g_s += ntiles;
+      g_k += npass;
+      g_s += npass;
       if (pv) g_v += ntiles;
     }
     // ============================================================== softmax / select warps
@@ -751,8 +785,9 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         for (int i = 0; i < kRwEnt / 32; ++i) rwb[i] = __ldg(src + 32 * i + lane);
       };
       if (BIAS == BIAS_SMEM && first_pass) bounded_wait(B_BIAS, 0);
-      for (int t = 0; t < ntiles; ++t) {
-        const uint32_t gs = g_s + (uint32_t)t, buf = gs % kSBufs;
+      for (int u = 0; u < npass; ++u) {
+        const int t = tile_at(u, p_stride);
+        const uint32_t gs = g_s + (uint32_t)u, buf = gs % kSBufs;
         const uint32_t colP = kColS + buf * kN;  // P of this tile is written over its score buffer
         const int j0 = t * kN;
         // bias offsets of this tile's keys: per-head table, or computed by this warp
@@ -930,6 +965,31 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
                 e[u] = (valid && !drop_tie) ? w : 0.0f;
               }
               emit(e, ch);
+            } else if (kHasRadix && BIAS == BIAS_ROWS && !kRef && pass == P_FBIN) {
+              // FBIN with the staged bias: per pair of keys the logits (a packed fp32x2 FMA,
+              // each element rounded once as fmaf), the saturating bin map and two counts.
+              // The bias is read first, so that the histogram adds wait on no load.
+              if (r_state == 4) {
+#pragma unroll
+                for (int g = 0; g < 32; g += kFbGroup) {
+                float bv[kFbGroup];
+#pragma unroll
+                for (int u = 0; u < kFbGroup; ++u) bv[u] = brow[-(32 * cc + g + u)];
+#pragma unroll
+                for (int u = g; u < g + kFbGroup; u += 2) {
+                  const float2 sf2 = make_float2((float)(int)r[32 * cc + u], (float)(int)r[32 * cc + u + 1]);
+                  const float2 l2 = __ffma2_rn(sf2, make_float2(c, c), make_float2(bv[u - g], bv[u - g + 1]));
+                  const float la = (FULL || 32 * ch + u < nvalid) ? l2.x : -INFINITY;
+                  const float lb = (FULL || 32 * ch + u + 1 < nvalid) ? l2.y : -INFINITY;
+                  const float2 w2 = __ffma2_rn(make_float2(fma_sat(la, fb_sc, fb_off), fma_sat(lb, fb_sc, fb_off)),
+                                               make_float2(kFbSpan, kFbSpan), make_float2(kFbMg, kFbMg));
+                  asm volatile("red.shared.add.u32 [%0], 1;" ::"r"((__float_as_uint(w2.x) & 0xFE00u) + hist_row)
+                               : "memory");
+                  asm volatile("red.shared.add.u32 [%0], 1;" ::"r"((__float_as_uint(w2.y) & 0xFE00u) + hist_row)
+                               : "memory");
+                }
+                }
+              }
             } else {
               // generic path: exact logits (invalid keys -inf)
               float lg[32];
@@ -983,19 +1043,18 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
                 for (int u = 0; u < 32; ++u) ex[u] = fast_exp2(__fmaf_rn(lg[u], kLog2e, mo2));
                 lsum += sum32(ex);
               } else if (kHasRadix && pass == P_FBIN) {
-                // bins of the row's logits: u = min(max(fmaf(l, sc, off), kFbMg), kFbTop) is
+                // bins of the row's logits: w = fmaf(sat(fmaf(l, sc, off)), 65535, kFbMg) is
                 // monotone in l; bin b at word b of the row's column.  Every key is counted
                 // (no branch): keys below the window land in bin 0, which is never read,
                 // keys past L (l = -inf) too
                 if (r_state == 4) {
 #pragma unroll
                   for (int u = 0; u < 32; u += 2) {
-                    const float2 u2 = __ffma2_rn(make_float2(lg[u], lg[u + 1]), make_float2(fb_sc, fb_sc),
-                                                 make_float2(fb_off, fb_off));
-                    const float ua = fminf(fmaxf(u2.x, kFbMg), kFbTop), ub = fminf(fmaxf(u2.y, kFbMg), kFbTop);
-                    asm volatile("red.shared.add.u32 [%0], 1;" ::"r"((__float_as_uint(ua) & 0xFE00u) + hist_row)
+                    const float2 w2 = __ffma2_rn(make_float2(fma_sat(lg[u], fb_sc, fb_off), fma_sat(lg[u + 1], fb_sc, fb_off)),
+                                                 make_float2(kFbSpan, kFbSpan), make_float2(kFbMg, kFbMg));
+                    asm volatile("red.shared.add.u32 [%0], 1;" ::"r"((__float_as_uint(w2.x) & 0xFE00u) + hist_row)
                                  : "memory");
-                    asm volatile("red.shared.add.u32 [%0], 1;" ::"r"((__float_as_uint(ub) & 0xFE00u) + hist_row)
+                    asm volatile("red.shared.add.u32 [%0], 1;" ::"r"((__float_as_uint(w2.y) & 0xFE00u) + hist_row)
                                  : "memory");
                   }
                 }
@@ -1167,12 +1226,54 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
               inm |= (lb >= w_lo && lb <= w_hi ? 1u : 0u) << (u + 1);
             }
           };
+          // bf16 V: P goes straight into packed words with a running sum (no weight array
+          // held across the tie exchange); the rare chunk that drops threshold ties is
+          // recomputed below through pv_chunk
+          uint32_t wp[16];
+          float cs = 0.0f;
+          auto pv_words = [&](auto full_tag, auto drop_tag, uint32_t drop) {
+            constexpr bool FULL = decltype(full_tag)::value;
+            constexpr bool DROP = decltype(drop_tag)::value;  // zero the keys of `drop` (dropped ties)
+            const float mo_p = -m * kLog2e;
+            cs = 0.0f;
+            float cs1 = 0.0f;
+#pragma unroll
+            for (int u = 0; u < 32; u += 2) {
+              float2 b2;
+              if (BIAS == BIAS_ROWS) {
+                b2 = make_float2(brow[-u], brow[-(u + 1)]);
+              } else {
+                b2 = make_float2(__ldg(reinterpret_cast<const float*>(tab_bytes - ko[32 * half + u])),
+                                 __ldg(reinterpret_cast<const float*>(tab_bytes - ko[32 * half + u + 1])));
+              }
+              const float2 l2 = __ffma2_rn(make_float2((float)(int)r[u], (float)(int)r[u + 1]), make_float2(c, c), b2);
+              const float la = (FULL || u < nv) ? l2.x : -INFINITY, lb = (FULL || u + 1 < nv) ? l2.y : -INFINITY;
+              const float2 x2 = __ffma2_rn(make_float2(la, lb), make_float2(kLog2e, kLog2e), make_float2(mo_p, mo_p));
+              const bool ka = la >= w_cut && (!DROP || !((drop >> u) & 1u));
+              const bool kb = lb >= w_cut && (!DROP || !((drop >> (u + 1)) & 1u));
+              const float ea = ka ? fast_exp2(x2.x) : 0.0f, eb = kb ? fast_exp2(x2.y) : 0.0f;
+              wp[u >> 1] = pack_bf16x2(ea, eb);
+              cs += ea;
+              cs1 += eb;
+              inm |= (la >= w_lo && la <= w_hi ? 1u : 0u) << u;
+              inm |= (lb >= w_lo && lb <= w_hi ? 1u : 0u) << (u + 1);
+            }
+            cs += cs1;
+          };
           if (ok_wait && jb < L) {
-            if (full_tile) pv_chunk(std::true_type{});
-            else pv_chunk(std::false_type{});
-          } else {
+            if (VF32) {
+              if (full_tile) pv_chunk(std::true_type{});
+              else pv_chunk(std::false_type{});
+            } else {
+              if (full_tile) pv_words(std::true_type{}, std::false_type{}, 0u);
+              else pv_words(std::false_type{}, std::false_type{}, 0u);
+            }
+          } else if (VF32) {
 #pragma unroll
             for (int u = 0; u < 32; ++u) e[u] = 0.0f;
+          } else {
+#pragma unroll
+            for (int u = 0; u < 16; ++u) wp[u] = 0u;
           }
           uint32_t eqm = 0u;
           if (r_state == 3) {
@@ -1190,7 +1291,11 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
           asm volatile("bar.sync %0, 64;" ::"r"(1 + (warp & 3)) : "memory");
           const int c0 = tx[srow], c1 = tx[kM + srow];
           const uint32_t dropm = eqm & ~tie_keep(eqm, cut, rF, tie_seen + (half ? c0 : 0));
-          if (dropm) {
+          if (!VF32 && dropm && ok_wait && jb < L) {  // the chunk again, without the dropped ties
+            if (full_tile) pv_words(std::true_type{}, std::true_type{}, dropm);
+            else pv_words(std::false_type{}, std::true_type{}, dropm);
+          }
+          if (VF32) {
 #pragma unroll
             for (int u = 0; u < 32; ++u) e[u] = ((dropm >> u) & 1u) ? 0.0f : e[u];
           }
@@ -1200,8 +1305,11 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
               const uint32_t z[16] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
               tmem_st16(tl + colP + 32 * half, z);
               if (VF32) tmem_st16(tl + colP + 32 * half + 16, z);
-            } else {
+            } else if (VF32) {
               emit(e, half);
+            } else {
+              lsum += cs;
+              tmem_st16(tl + colP + 32 * half, wp);
             }
           }
         } else if (kSplit == 2 && SEL == SEL_TOPN_INT && pv) {
@@ -1266,8 +1374,8 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         tc_fence_before();
         mbar_arrive(&bars[B_TDONE + buf]);
       }
-      g_k += ntiles;
-      g_s += ntiles;
+      g_k += npass;
+      g_s += npass;
       if (pv) g_v += ntiles;
     }
 
@@ -1356,19 +1464,46 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
           // score >= sN (so a logit >= the low end), fewer than keff a score > sN (only
           // those can exceed the high end); logits are monotone in (score, bias)
           const float bmin = a.bminmax[2 * h], bmax = a.bminmax[2 * h + 1];
-          const float lo = __fmaf_rn((float)sN, c, bmin);
-          const float hw = __fmaf_rn((float)sN, c, bmax);
+          int s_lo = sN, s_hi = sN;
+          if (p_stride != 1) {
+            // a sample of ns keys: rank keff of the row maps to about rho in the sample.
+            // s_hi: fewer than rho - del sampled keys score above it, so (likely) fewer
+            // than keff keys do; s_lo: at least rho + del sampled keys reach it, so (likely)
+            // keff keys do.  The FBIN pass checks both with exact counts.
+            const int last = tile_at(n_sampled - 1, kSampleStride);
+            const int ns = n_sampled * kN - (last == ntiles - 1 ? ntiles * kN - L : 0);
+            const float rho = (float)keff * (float)ns / (float)L;
+            const float del = 5.0f * sqrtf(rho * (1.0f - (float)keff / (float)L)) + 2.0f;
+            const int k_hi = max(1, (int)floorf(rho - del)), k_lo = (int)ceilf(rho + del);
+            int lhi = kLevels - 1, llo = kLevels - 1, cs = 0;
+            bool fh = false, fl = false;
+#pragma unroll
+            for (int lev = 0; lev < kLevels; ++lev) {
+              cs += cnt(lev);
+              if (!fh && cs >= k_hi) { lhi = lev; fh = true; }
+              if (!fl && cs >= k_lo) { llo = lev; fl = true; }
+            }
+            s_hi = D - 2 * lhi;
+            s_lo = D - 2 * llo;  // the lowest level when the sample never reaches k_lo
+          }
+          const float lo = __fmaf_rn((float)s_lo, c, bmin);
+          const float hw = __fmaf_rn((float)s_hi, c, bmax);
           r_rank = keff;
-          m = __fmaf_rn((float)smax, c, bmax);  // no logit exceeds it
-          // FBIN map: lo -> about kFbMg + 768 (bin 1), hw -> about kFbMg + 64768 (bin 126);
-          // the rounding of sc and off moves both by far less than a bin while
-          // |lo * sc| < 2^30, else the order-key radix takes the window
-          const float sc_b = 125.0f * 512.0f / (hw - lo);
+          r_sampled = p_stride != 1;
+          // no logit exceeds m (with a sample: none by more than 2 d c, which the
+          // sampling condition keeps inside fp32)
+          m = __fmaf_rn((float)smax, c, bmax);
+          // FBIN map: lo -> about u = 768 / 65535 (w in bin 1), hw -> about 64768 / 65535
+          // (bin 126); the rounding of sc and off moves both by far less than a bin
+          // (1 / 128 of u) while |lo * sc| < 2048, else the order-key radix takes the window
+          const float sc_b = (125.0f * 512.0f / kFbSpan) / (hw - lo);
           const float lsc = lo * sc_b;
-          if (hw > lo && isfinite(sc_b) && fabsf(lsc) < 1.0e9f) {
+          if (hw > lo && isfinite(sc_b) && fabsf(lsc) < 2048.0f) {
             fb_sc = sc_b;
-            fb_off = (kFbMg + 768.0f) - lsc;
+            fb_off = 768.0f / kFbSpan - lsc;
             r_state = 4;
+          } else if (p_stride != 1) {
+            r_state = 5;  // the radix window cannot check a sampled bracket: count every tile
           } else {
             r_uhi = float_order_key(hw);
             r_span = r_uhi - float_order_key(lo);
@@ -1382,17 +1517,30 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         // the bin holding rank r_rank, counted from the top (bin 127: keys above the
         // window, fewer than r_rank of them; bin 0 is never reached: at least r_rank
         // keys reach the window's low end)
-        int cum = 0, bsel = 1, kbin = 0;
+        int cum = 0, bsel = 0, kbin = 0;
         for (int bb = 127; bb >= 1; --bb) {
           const int k = (int)hist[bb * kM + srow];
           if (cum + k >= r_rank) { bsel = bb; kbin = k; break; }
           cum += k;
         }
+        // a sampled bracket that missed: rank r_rank above the window (bin 127) or
+        // below it (bin 0).  A bracket from every tile's levels cannot miss; should
+        // rounding ever make it, the radix passes take the whole float range.
+        if ((bsel == 0 || bsel == 127) && r_sampled) {
+          r_state = 5;
+        } else if (bsel == 0 || bsel == 127) {
+          r_uhi = float_order_key(INFINITY);
+          r_span = r_uhi - float_order_key(-INFINITY);
+          r_shift = 0;
+          while ((r_span >> r_shift) >= (uint32_t)kRadixBins) ++r_shift;
+          r_first = true;
+          r_state = 1;
+        } else {
         // the bin's keys are the logits in [w_lo, w_cut): the least floats that map to
         // bins bsel and bsel + 1, found by bisection over the order keys of floats
         auto fb_bin = [&](float x) -> int {
-          const float uu = fminf(__fmaf_rn(x, fb_sc, fb_off), kFbTop);
-          return uu >= kFbIn ? (int)((__float_as_uint(uu) & 0xFE00u) >> 9) : 0;
+          const float w = __fmaf_rn(fma_sat(x, fb_sc, fb_off), kFbSpan, kFbMg);
+          return (int)((__float_as_uint(w) & 0xFE00u) >> 9);
         };
         auto fb_least = [&](int bin) -> float {
           uint32_t klo = 0x007FFFFFu, khi = 0xFF800000u;  // -inf (bin 0), +inf (bin 127)
@@ -1422,6 +1570,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
             while ((r_span >> r_shift) >= (uint32_t)kRadixBins) ++r_shift;
             r_state = 1;
           }
+        }
         }
       } else if (pass == P_RADIX && r_state == 1) {
         if (r_first) r_rank -= r_above;  // rank within the first window
@@ -1520,6 +1669,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
     }
     tie_seen = 0;
     // ---- the CTA chooses the next pass
+    const int any_relevel = __syncthreads_or(tid < kM && r_state == 5);
     const int any_fbin = __syncthreads_or(tid < kM && r_state == 4);
     const int any_refine = __syncthreads_or(tid < kM && r_state == 1);
     const int any_collect = __syncthreads_or(tid < kM && r_state == 2);
@@ -1527,6 +1677,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
     if (*abort_flag) next = P_DONE;
     else if (pass == P_IDX || pass == P_CODES || pass == P_PV || pass == P_SCORES) next = P_DONE;
     else if (pass == P_NORM) next = (EXPORT == EXP_CODES) ? P_CODES : P_PV;
+    else if (any_relevel) next = P_LEVELS;
     else if (any_fbin) next = P_FBIN;
     else if (any_refine) next = P_RADIX;
     else if (any_collect) next = P_COLLECT;
@@ -1536,6 +1687,9 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
     else next = P_PV;
     if ((next == P_RADIX || next == P_FBIN) && tid < kM)
       for (int bb = 0; bb < kRadixBins / 2; ++bb) hist[bb * kM + srow] = 0u;
+    if (next == P_LEVELS && tid < kM)
+      for (int lev = 0; lev < kLevels; ++lev) hist[lev * kM + srow] = 0u;
+    if (pass == P_LEVELS) sample_levels = false;  // a second level pass counts every tile
     if ((next == P_RADIX || next == P_FBIN) && is_soft) r_above = 0;
     if (kSplitF && (next == P_COLLECT || next == P_PV) && tid < kM) reinterpret_cast<int*>(xchg)[srow] = 0;
     if (next == P_KEPT_NORM && is_soft) lsum = 0.0f;
