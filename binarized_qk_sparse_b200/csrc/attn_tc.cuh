@@ -518,6 +518,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
   const bool k_res = ntiles <= kKStages;
   bool first_pass = true;
   int v_pref = 0;  // producer: V tiles of the P.V pass already issued
+  int pv_xchg = 1;  // split P.V: some row of the CTA cuts its ties at F (the halves exchange tie counts)
   // producer, 4-bit V: the packed V^T rows (32 bytes = 64 keys per channel row, D / 32
   // rows per lane) of tile q4_tile, loaded ahead of their expansion
   uint4 q4_next[MODE == MODE_Q4 ? D / 32 : 1][2];
@@ -713,6 +714,9 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
       const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
       const uint32_t hist_row = smem_u32(hist) + (uint32_t)srow * 4u;
       const float mo = -m * kLog2e;
+      // P.V with two threads per row: the weighting cut, the float just above F for a row
+      // whose ties at F are resolved by count (w_lo == w_cut), else w_cut itself
+      const float pv_cut = (w_lo == w_cut && w_cut != INFINITY) ? order_key_float(float_order_key(w_cut) + 1u) : w_cut;
       const float* lut = reinterpret_cast<const float*>(hist);
       const float* lut_lane = lut + (D / 2) * 32 + lane;  // dense level table: entry for score s at lut_lane[-16 s]
       // this row's weight table (top-N without a bias): level (d - s) / 2 at
@@ -778,11 +782,16 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         // dense weights read exp(b - b_max) (the level-table path), the rest the bias itself
         rw_src = ((kDense && use_lut) ? a.expb : a.bext) + (size_t)h * a.ext_E + rw_first;
       }
-      auto rw_fetch = [&](int tt) {  // tile tt's window into registers (coalesced loads)
-        const int jt = tt * kN, yk = jt / a.gw, xk = jt - yk * a.gw;
-        const float* src = rw_src + (rw_yw - yk + a.gh - 1) * a.ext_S + (rw_xw - xk + a.gw - kN);
+      // the next tile's window into registers (coalesced loads); the tiles of a pass are
+      // fetched in order, so the key tile's patch (rw_fy, rw_fx) advances by 64 columns
+      // (grid rows hold a multiple of 64 patches)
+      int rw_fy = 0, rw_fx = 0;
+      auto rw_fetch = [&]() {
+        const float* src = rw_src + (rw_yw - rw_fy + a.gh - 1) * a.ext_S + (rw_xw - rw_fx + a.gw - kN);
 #pragma unroll
         for (int i = 0; i < kRwEnt / 32; ++i) rwb[i] = __ldg(src + 32 * i + lane);
+        rw_fx += kN;
+        if (rw_fx == a.gw) { rw_fx = 0; ++rw_fy; }
       };
       if (BIAS == BIAS_SMEM && first_pass) bounded_wait(B_BIAS, 0);
       for (int u = 0; u < npass; ++u) {
@@ -811,11 +820,11 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         const float* brow = nullptr;
         if (BIAS == BIAS_ROWS && wants_bias && warp_live) {
           float* sl = rw_slice0 + (t & 1) * kRwEnt;  // last read two tiles ago
-          if (t == 0) rw_fetch(0);
+          if (t == 0) { rw_fy = 0; rw_fx = 0; rw_fetch(); }
 #pragma unroll
           for (int i = 0; i < kRwEnt / 32; ++i) sl[32 * i + lane] = rwb[i];
           __syncwarp();
-          if (t + 1 < ntiles) rw_fetch(t + 1);  // lands while this tile is processed
+          if (t + 1 < ntiles) rw_fetch();  // tile t + 1, lands while this tile is processed
           brow = sl + lane + (kN - 1) - rw_first - (kSplit == 2 ? 32 * half : 0);
         }
         const bool ok_wait = __all_sync(0xffffffffu, bounded_wait(B_SFULL + buf, (gs / kSBufs) & 1));
@@ -1227,13 +1236,15 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
             }
           };
           // bf16 V: P goes straight into packed words with a running sum (no weight array
-          // held across the tie exchange); the rare chunk that drops threshold ties is
-          // recomputed below through pv_chunk
+          // held across the tie exchange).  Keys at or above pv_cut are weighted, keys in
+          // [w_lo, pv_cut) go to the mask: the final bin of a merge row, or a row's ties
+          // at F (pv_cut just above F), which are weighted in a second computation of the
+          // chunk if the tie rule keeps them (rare: the chunk that holds the threshold)
           uint32_t wp[16];
           float cs = 0.0f;
-          auto pv_words = [&](auto full_tag, auto drop_tag, uint32_t drop) {
+          auto pv_words = [&](auto full_tag, auto add_tag, uint32_t add) {
             constexpr bool FULL = decltype(full_tag)::value;
-            constexpr bool DROP = decltype(drop_tag)::value;  // zero the keys of `drop` (dropped ties)
+            constexpr bool ADD = decltype(add_tag)::value;  // also weight the keys of `add` (kept ties)
             const float mo_p = -m * kLog2e;
             cs = 0.0f;
             float cs1 = 0.0f;
@@ -1249,14 +1260,16 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
               const float2 l2 = __ffma2_rn(make_float2((float)(int)r[u], (float)(int)r[u + 1]), make_float2(c, c), b2);
               const float la = (FULL || u < nv) ? l2.x : -INFINITY, lb = (FULL || u + 1 < nv) ? l2.y : -INFINITY;
               const float2 x2 = __ffma2_rn(make_float2(la, lb), make_float2(kLog2e, kLog2e), make_float2(mo_p, mo_p));
-              const bool ka = la >= w_cut && (!DROP || !((drop >> u) & 1u));
-              const bool kb = lb >= w_cut && (!DROP || !((drop >> (u + 1)) & 1u));
+              const bool ga = la >= pv_cut, gb = lb >= pv_cut;
+              const bool ka = ga || (ADD && ((add >> u) & 1u)), kb = gb || (ADD && ((add >> (u + 1)) & 1u));
               const float ea = ka ? fast_exp2(x2.x) : 0.0f, eb = kb ? fast_exp2(x2.y) : 0.0f;
               wp[u >> 1] = pack_bf16x2(ea, eb);
               cs += ea;
               cs1 += eb;
-              inm |= (la >= w_lo && la <= w_hi ? 1u : 0u) << u;
-              inm |= (lb >= w_lo && lb <= w_hi ? 1u : 0u) << (u + 1);
+              if (!ADD) {
+                inm |= (la >= w_lo && !ga ? 1u : 0u) << u;
+                inm |= (lb >= w_lo && !gb ? 1u : 0u) << (u + 1);
+              }
             }
             cs += cs1;
           };
@@ -1286,14 +1299,21 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
           } else {
             eqm = inm;
           }
-          int* tx = reinterpret_cast<int*>(hist) + (kCandCap - 8) * kM + (int)(gs & 1u) * 2 * kM;
-          tx[half * kM + srow] = __popc(eqm);
-          asm volatile("bar.sync %0, 64;" ::"r"(1 + (warp & 3)) : "memory");
-          const int c0 = tx[srow], c1 = tx[kM + srow];
-          const uint32_t dropm = eqm & ~tie_keep(eqm, cut, rF, tie_seen + (half ? c0 : 0));
-          if (!VF32 && dropm && ok_wait && jb < L) {  // the chunk again, without the dropped ties
-            if (full_tile) pv_words(std::true_type{}, std::true_type{}, dropm);
-            else pv_words(std::false_type{}, std::true_type{}, dropm);
+          // the row's tie counts of this tile, from both threads (only when some row of
+          // the CTA cuts its ties at F; the flag is the same for every thread)
+          int c0 = 0, c1 = 0;
+          if (pv_xchg) {
+            int* tx = reinterpret_cast<int*>(hist) + (kCandCap - 8) * kM + (int)(gs & 1u) * 2 * kM;
+            tx[half * kM + srow] = __popc(eqm);
+            asm volatile("bar.sync %0, 64;" ::"r"(1 + (warp & 3)) : "memory");
+            c0 = tx[srow];
+            c1 = tx[kM + srow];
+          }
+          const uint32_t keep_t = tie_keep(eqm, cut, rF, tie_seen + (half ? c0 : 0));
+          const uint32_t dropm = eqm & ~keep_t;
+          if (!VF32 && (eqm & keep_t) && ok_wait && jb < L) {  // the chunk again, with its kept ties
+            if (full_tile) pv_words(std::true_type{}, std::true_type{}, eqm & keep_t);
+            else pv_words(std::false_type{}, std::true_type{}, eqm & keep_t);
           }
           if (VF32) {
 #pragma unroll
@@ -1669,12 +1689,19 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
     }
     tie_seen = 0;
     // ---- the CTA chooses the next pass
-    const int any_relevel = __syncthreads_or(tid < kM && r_state == 5);
-    const int any_fbin = __syncthreads_or(tid < kM && r_state == 4);
-    const int any_refine = __syncthreads_or(tid < kM && r_state == 1);
-    const int any_collect = __syncthreads_or(tid < kM && r_state == 2);
+    // Every thread takes the same next pass: the abort flag is voted on (a thread that
+    // gave up a wait in this pass set it before reaching the vote), and the CTA-wide
+    // votes on the row states run only where the select kind has the passes they
+    // choose between.
+    const int aborted = __syncthreads_or(*abort_flag != 0u);
+    constexpr bool kVotes = SEL == SEL_TOPN_FLOAT;
+    const int any_relevel = kVotes && __syncthreads_or(tid < kM && r_state == 5);
+    if (kSplitF) pv_xchg = VF32 || __syncthreads_or(is_soft && row_ok && cut && w_lo == w_cut && w_cut != INFINITY);
+    const int any_fbin = kVotes && __syncthreads_or(tid < kM && r_state == 4);
+    const int any_refine = kVotes && __syncthreads_or(tid < kM && r_state == 1);
+    const int any_collect = kVotes && __syncthreads_or(tid < kM && r_state == 2);
     int next;
-    if (*abort_flag) next = P_DONE;
+    if (aborted) next = P_DONE;
     else if (pass == P_IDX || pass == P_CODES || pass == P_PV || pass == P_SCORES) next = P_DONE;
     else if (pass == P_NORM) next = (EXPORT == EXP_CODES) ? P_CODES : P_PV;
     else if (any_relevel) next = P_LEVELS;
