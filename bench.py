@@ -85,11 +85,12 @@ HEAD_STAGE_BYTES = 128 * 1024  # heads up to this size are prepared by one kerne
 def launches_per_step(n: int, elem: int, mode: str, has_bias: bool, dense_bias: bool = False, d: int = 64) -> int:
     """Kernels one prepare + attend step launches: the sign/pack stage (one
     kernel for short heads, which also builds relative-position bias tables;
-    statistics + pack + bias tables otherwise), the range and tables of a
-    dense bias matrix (two kernels), the hi/lo split of an fp32 V (float
-    mode), and the fused attention."""
+    otherwise statistics, their per-head finalization and the pack, plus the
+    bias range and the table fill), the range and tables of a dense bias
+    matrix (two kernels), the hi/lo split of an fp32 V (float mode), and the
+    fused attention."""
     rel = has_bias and not dense_bias
-    k = 1 if (d == 64 and n * 64 * elem <= HEAD_STAGE_BYTES) else 2 + (1 if rel else 0)
+    k = 1 if (d == 64 and n * 64 * elem <= HEAD_STAGE_BYTES) else 3 + (2 if rel else 0)
     if dense_bias:
         k += 2
     if mode == "float" and elem == 4:

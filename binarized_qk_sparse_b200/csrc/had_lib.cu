@@ -6,11 +6,14 @@
 //
 // had_attention pipeline (method: "Hamming Attention Distillation" top-N over
 // binarized keys/queries; "BinaryAttention" §2.2-§2.4):
-//   k_stats  : fp64 channel partial sums of Q and K (+ fp32 absmax of V in uint8 mode)
-//   k_pack   : mu -> sign bits of Q (packed uint32) and K (+-1 int8 rows);
-//              V scale -> int8 V^T (uint8 mode)
-//   k_bias_tables (with a bias): per-head bias range and exp(b - b_max) table
-//   k_attn   : scores, logits, top-N select, softmax, A.V, output
+//   k_stats       : fp64 channel partial sums of Q and K (+ fp32 absmax of V in uint8 modes)
+//   k_stats_final : per-head means (and V absmax) from the partials
+//   k_pack        : mu -> sign bits of Q (packed uint32) and K (+-1 int8 rows);
+//                   V scale -> int8 or 4-bit V^T (uint8 modes)
+//   k_bias_range + k_bias_fill (with a bias): per-head bias range, extended bias
+//                   and exp(b - b_max) tables
+//   k_attn_tc     : scores, logits, top-N select, softmax, A.V, output
+//   (heads up to 128 KB: k_prep_head does the statistics, packing and tables in one launch)
 #include <algorithm>
 #include <climits>
 #include <cmath>
@@ -242,6 +245,11 @@ had_status launch_prep(const had_shape* s, const void* X0, const void* X1, const
     else bf ? k_stats<__nv_bfloat16, 64><<<grid, kPrepThreads, 0, st>>>(pa) : k_stats<float, 64><<<grid, kPrepThreads, 0, st>>>(pa);
     had_status r = check_launch("k_stats");
     if (r != HAD_OK) return r;
+    dim3 fgrid(d.BH, ntens);
+    if (d.d == 32) k_stats_final<32><<<fgrid, 128, 0, st>>>(pa);
+    else if (d.d == 128) k_stats_final<128><<<fgrid, 128, 0, st>>>(pa);
+    else k_stats_final<64><<<fgrid, 128, 0, st>>>(pa);
+    if ((r = check_launch("k_stats_final")) != HAD_OK) return r;
   }
   PackArgs ka{};
   ka.X[0] = X0; ka.X[1] = X1; ka.X[2] = X2;
@@ -376,8 +384,11 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
                     vscale, st, status, vbits);
     if (r != HAD_OK) return r;
     if (has_bias && !ba.dense) {
-      k_bias_tables<<<s->H, 256, 0, st>>>(ba);
-      if ((r = check_launch("k_bias_tables")) != HAD_OK) return r;
+      k_bias_range<<<s->H, kBiasRangeThreads, 0, st>>>(ba);
+      if ((r = check_launch("k_bias_range")) != HAD_OK) return r;
+      dim3 fgrid((relpos_ext(ba.gh, ba.gw).E + kBiasFillPerCta - 1) / kBiasFillPerCta, s->H);
+      k_bias_fill<<<fgrid, 256, 0, st>>>(ba);
+      if ((r = check_launch("k_bias_fill")) != HAD_OK) return r;
     }
   }
   if (!quant && s->in_dtype == HAD_F32 && need_v) {
@@ -426,8 +437,11 @@ had_status build_bias_tables(const had_shape* s, const had_relpos_bias* bias, ui
     k_dense_bias_tables<<<tgrid, 256, 0, st>>>(ba);
     return check_launch("k_dense_bias_tables");
   }
-  k_bias_tables<<<s->H, 256, 0, st>>>(ba);
-  return check_launch("k_bias_tables");
+  k_bias_range<<<s->H, kBiasRangeThreads, 0, st>>>(ba);
+  if ((r = check_launch("k_bias_range")) != HAD_OK) return r;
+  dim3 fgrid((relpos_ext(ba.gh, ba.gw).E + kBiasFillPerCta - 1) / kBiasFillPerCta, s->H);
+  k_bias_fill<<<fgrid, 256, 0, st>>>(ba);
+  return check_launch("k_bias_fill");
 }
 
 // The bias fields of the kernel arguments (extended-table geometry, table

@@ -105,6 +105,42 @@ __global__ void __launch_bounds__(kPrepThreads) k_stats(const PrepArgs a) {
   }
 }
 
+// The per-head statistic from the chunk partials, once per (b, h, channel): the
+// mean of Q or K (fp64 sum of the partials in chunk order, one rounding to fp32,
+// stored back as a double in chunk 0's slot) or the V absmax (chunk 0's slot).
+// k_pack then reads chunk 0 instead of every CTA reducing all of the head's chunks.
+template <int D>
+__global__ void __launch_bounds__(128) k_stats_final(const PrepArgs a) {
+  const int bh = blockIdx.x, tz = a.first_tensor + blockIdx.y, c = threadIdx.x;
+  if (c >= D) return;
+  const int L = valid_len(a.seqlens, bh / a.H, a.n, nullptr);  // k_stats already reported bad lengths
+  const int nv = (L + kChunk - 1) / kChunk;
+  constexpr int kBatch = 64;  // loads in flight; the adds still run in chunk order
+  if (tz < 2) {
+    double* col = a.sums + ((size_t)tz * gridDim.x + bh) * a.nchunks * D + c;
+    double s = 0.0;
+    for (int k0 = 0; k0 < nv; k0 += kBatch) {
+      double v[kBatch];
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) v[k] = k0 + k < nv ? col[(size_t)(k0 + k) * D] : 0.0;
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) if (k0 + k < nv) s += v[k];
+    }
+    col[0] = (double)((L > 0) ? __double2float_rn(s / (double)L) : 0.0f);
+  } else {
+    float* col = a.amax + (size_t)bh * a.nchunks * D + c;
+    float m = 0.0f;
+    for (int k0 = 0; k0 < nv; k0 += kBatch) {
+      float v[kBatch];
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) v[k] = k0 + k < nv ? col[(size_t)(k0 + k) * D] : 0.0f;
+#pragma unroll
+      for (int k = 0; k < kBatch; ++k) m = fmaxf(m, v[k]);
+    }
+    col[0] = m;
+  }
+}
+
 struct PackArgs {
   const void* X[3];
   int ntens, first_tensor;
@@ -144,18 +180,13 @@ __global__ void __launch_bounds__(kPrepThreads) k_pack(const PackArgs a) {
       float mu;
       if (a.mu_in[tz]) {
         mu = a.mu_in[tz][(size_t)bh * kD + c];
-      } else {
-        double s = 0.0;
-        const int nch_valid = (L + kChunk - 1) / kChunk;
-        for (int k = 0; k < nch_valid; ++k) s += a.sums[(((size_t)tz * gridDim.y + bh) * a.nchunks + k) * kD + c];
-        mu = (L > 0) ? __double2float_rn(s / (double)L) : 0.0f;
+      } else {  // the mean k_stats_final left in chunk 0's slot
+        mu = (float)a.sums[((size_t)tz * gridDim.y + bh) * a.nchunks * kD + c];
       }
       stat[c] = mu;
       if (chunk == 0 && a.mu_out[tz]) a.mu_out[tz][(size_t)bh * kD + c] = mu;
     } else {
-      float m = 0.0f;
-      const int nch_valid = (L + kChunk - 1) / kChunk;
-      for (int k = 0; k < nch_valid; ++k) m = fmaxf(m, a.amax[((size_t)bh * a.nchunks + k) * kD + c]);
+      const float m = a.amax[(size_t)bh * a.nchunks * kD + c];  // the absmax k_stats_final left in chunk 0
       const float qmax = a.v_bits == 4 ? 7.0f : 127.0f;
       float s = (m > 0.0f) ? __fdiv_rn(m, qmax) : 1.0f;
       stat[c] = s;
@@ -287,30 +318,17 @@ struct BiasArgs {
   float* expb;         // [H][E]
 };
 
-__device__ __forceinline__ void bias_tables_block(const BiasArgs& a, int h) {
-  __shared__ float smn[32], smx[32];
+// The extended tables of head h, entries [e0, e1), given the table maximum mx.
+__device__ __forceinline__ void relpos_fill(const BiasArgs& a, int h, float mx, int e0, int e1) {
   const RelposExt x = relpos_ext(a.gh, a.gw);
   const int tw = 2 * a.gw - 1;
-  const size_t cells = (size_t)(2 * a.gh - 1) * tw;
-  const float* t = a.table + (size_t)h * cells;
-  float mn = INFINITY, mx = -INFINITY;
-  for (size_t e = threadIdx.x; e < cells; e += blockDim.x) { mn = fminf(mn, t[e]); mx = fmaxf(mx, t[e]); }
-  for (int o = 16; o > 0; o >>= 1) {
-    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  }
-  if ((threadIdx.x & 31) == 0) { smn[threadIdx.x >> 5] = mn; smx[threadIdx.x >> 5] = mx; }
-  __syncthreads();
-  mn = smn[0]; mx = smx[0];
-  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) { mn = fminf(mn, smn[w]); mx = fmaxf(mx, smx[w]); }
-  if (a.prefix > 0) { mn = fminf(mn, 0.0f); mx = fmaxf(mx, 0.0f); }
-  if (threadIdx.x == 0) { a.bminmax[2 * h] = mn; a.bminmax[2 * h + 1] = mx; }
+  const float* t = a.table + (size_t)h * (2 * a.gh - 1) * tw;
   const float kLog2e = 1.4426950408889634f;
   const float e_class = exp2f((0.0f - mx) * kLog2e);
   float* be = a.bext + (size_t)h * x.E;
   float* ee = a.expb + (size_t)h * x.E;
   const int z0 = 2 * x.T + 2 * x.Kx;
-  for (int e = threadIdx.x; e < x.E; e += blockDim.x) {
+  for (int e = e0 + threadIdx.x; e < e1; e += blockDim.x) {
     float b, w;
     if (e < x.T) {  // table row e / S, column e % S (columns past 2gw-2 are padding)
       const int dy = e / x.S, dx = e - dy * x.S;
@@ -324,7 +342,51 @@ __device__ __forceinline__ void bias_tables_block(const BiasArgs& a, int h) {
   }
 }
 
+// The range of head h's table (0 included when class tokens exist) into bminmax,
+// then, with `fill`, its extended tables.
+__device__ __forceinline__ void bias_tables_block(const BiasArgs& a, int h, bool fill = true) {
+  __shared__ float smn[32], smx[32];
+  const RelposExt x = relpos_ext(a.gh, a.gw);
+  const int tw = 2 * a.gw - 1;
+  const size_t cells = (size_t)(2 * a.gh - 1) * tw;
+  const float* t = a.table + (size_t)h * cells;
+  float mn = INFINITY, mx = -INFINITY;
+  constexpr int kInFlight = 8;
+  for (size_t e0 = threadIdx.x; e0 < cells; e0 += (size_t)kInFlight * blockDim.x) {
+    float v[kInFlight];
+#pragma unroll
+    for (int k = 0; k < kInFlight; ++k) {
+      const size_t e = e0 + (size_t)k * blockDim.x;
+      v[k] = e < cells ? t[e] : t[e0];
+    }
+#pragma unroll
+    for (int k = 0; k < kInFlight; ++k) { mn = fminf(mn, v[k]); mx = fmaxf(mx, v[k]); }
+  }
+  for (int o = 16; o > 0; o >>= 1) {
+    mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  }
+  if ((threadIdx.x & 31) == 0) { smn[threadIdx.x >> 5] = mn; smx[threadIdx.x >> 5] = mx; }
+  __syncthreads();
+  mn = smn[0]; mx = smx[0];
+  for (int w = 1; w < (int)(blockDim.x >> 5); ++w) { mn = fminf(mn, smn[w]); mx = fmaxf(mx, smx[w]); }
+  if (a.prefix > 0) { mn = fminf(mn, 0.0f); mx = fmaxf(mx, 0.0f); }
+  if (threadIdx.x == 0) { a.bminmax[2 * h] = mn; a.bminmax[2 * h + 1] = mx; }
+  if (fill) relpos_fill(a, h, mx, 0, x.E);
+}
+
 __global__ void __launch_bounds__(256) k_bias_tables(const BiasArgs a) { bias_tables_block(a, blockIdx.x); }
+
+// Long sequences: one CTA per head takes the range (k_bias_range), then the tables,
+// up to 2.4 MB per head at 128 x 128 patches, are written by many CTAs per head
+// (k_bias_fill, grid (entries / kBiasFillPerCta, H)).
+constexpr int kBiasFillPerCta = 8192;
+constexpr int kBiasRangeThreads = 1024;
+__global__ void __launch_bounds__(kBiasRangeThreads) k_bias_range(const BiasArgs a) { bias_tables_block(a, blockIdx.x, false); }
+__global__ void __launch_bounds__(256) k_bias_fill(const BiasArgs a) {
+  const int h = blockIdx.y, e0 = blockIdx.x * kBiasFillPerCta;
+  relpos_fill(a, h, a.bminmax[2 * h + 1], e0, min(e0 + kBiasFillPerCta, relpos_ext(a.gh, a.gw).E));
+}
 
 // A dense bias matrix has n^2 entries per head, too many for one CTA per head to
 // turn into tables quickly: one CTA per head takes the range, then the tables

@@ -35,9 +35,9 @@ def test_launch_counts_per_step():
     assert bench.launches_per_step(197, 2, "u8i8", True) == 2
     # a dense bias matrix adds its range and table kernels
     assert bench.launches_per_step(197, 2, "u8i8", True, dense_bias=True) == 4
-    # long heads: statistics + pack (+ bias tables) + the fused kernel
-    assert bench.launches_per_step(16384, 2, "float", True) == 4
-    assert bench.launches_per_step(16384, 2, "float", False) == 3
+    # long heads: statistics + their finalization + pack (+ bias range and table fill) + the fused kernel
+    assert bench.launches_per_step(16384, 2, "float", True) == 6
+    assert bench.launches_per_step(16384, 2, "float", False) == 4
     # fp32 V in float mode adds the hi/lo split
     assert bench.launches_per_step(128, 4, "float", False) == 3
 
