@@ -256,6 +256,10 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
   constexpr uint32_t kTmemCols = tmem_cols(D);
   constexpr bool kRef = SEL == SEL_REF;        // the unbinarized comparison mode
   constexpr bool kQuant = MODE != MODE_F;       // uint8 A x int8 (or 4-bit) V
+  // Top-N with a bias scores on the fp8 path: +-1 as e4m3 (kind::f8f6f4, fp32
+  // accumulate), exact integers that the softmax threads read as floats; the other
+  // kinds index level tables by the integer score and keep kind::i8.
+  constexpr bool kF8 = SEL == SEL_TOPN_FLOAT;
   constexpr int kVStages = v_stages(SEL, VF32);
   constexpr bool kDense = sel_dense(SEL);
   static_assert(SPLIT == 1 || kDense || (SEL == SEL_TOPN_INT && EXPORT == EXP_NONE) ||
@@ -423,10 +427,10 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
     for (int c16 = 0; c16 < (kRef ? 0 : D / 16); ++c16) {  // 16 channels per chunk
       const uint32_t f = wq[c16 >> 1] >> ((c16 & 1) * 16);
       uint4 v;
-      v.x = expand_nibble_pm1(f & 15u);
-      v.y = expand_nibble_pm1((f >> 4) & 15u);
-      v.z = expand_nibble_pm1((f >> 8) & 15u);
-      v.w = expand_nibble_pm1((f >> 12) & 15u);
+      v.x = expand_nibble_pm(f & 15u, kF8);
+      v.y = expand_nibble_pm((f >> 4) & 15u, kF8);
+      v.z = expand_nibble_pm((f >> 8) & 15u, kF8);
+      v.w = expand_nibble_pm((f >> 12) & 15u, kF8);
       const int pn = c16 >> 2, cch = c16 & 3;
       *reinterpret_cast<uint4*>(sQ + pn * kM * 64 + tid * 64 + ((cch ^ ((tid >> 1) & 3)) * 16)) = v;
     }
@@ -632,7 +636,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
     else if (warp == kMmaWarp) {
       if (lane == 0) {
         // scores: +-1 int8 (kind::i8), or bf16 Q x bf16 K (kind::f16) in the comparison mode
-        const uint32_t id_s = kRef ? idesc_bf16(kM, kN, false) : idesc_i8(kM, kN, true, true, false);
+        const uint32_t id_s = kRef ? idesc_bf16(kM, kN, false) : kF8 ? idesc_e4m3(kM, kN) : idesc_i8(kM, kN, true, true, false);
         if (kRef && first_pass) bounded_wait(B_QFULL, 0);
         // P.V: uint8 codes x int8 V^T (N = D, one MMA per K-step), or bf16 P x bf16 V
         // (N = 64 per 64-channel panel)
@@ -655,8 +659,12 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
             for (int pn = 0; pn < kPan; ++pn)  // two 32-channel K-steps per 64-channel panel
 #pragma unroll
               for (int ks = 0; ks < 2; ++ks)
-                mma_i8_ss(tmem + kColS + buf * kN, sdesc(kq + pn * kM * 64 + 32 * ks, 16, 512, kSwizzle64B),
-                          sdesc(kk + pn * kN * 64 + 32 * ks, 16, 512, kSwizzle64B), id_s, (pn | ks) > 0 ? 1u : 0u);
+                if (kF8)
+                  mma_f8_ss(tmem + kColS + buf * kN, sdesc(kq + pn * kM * 64 + 32 * ks, 16, 512, kSwizzle64B),
+                            sdesc(kk + pn * kN * 64 + 32 * ks, 16, 512, kSwizzle64B), id_s, (pn | ks) > 0 ? 1u : 0u);
+                else
+                  mma_i8_ss(tmem + kColS + buf * kN, sdesc(kq + pn * kM * 64 + 32 * ks, 16, 512, kSwizzle64B),
+                            sdesc(kk + pn * kN * 64 + 32 * ks, 16, 512, kSwizzle64B), id_s, (pn | ks) > 0 ? 1u : 0u);
           }
           mma_commit(&bars[B_SFULL + buf]);
           if (!k_res) mma_commit(&bars[B_KEMPTY + st]);
@@ -711,6 +719,8 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
     }
     // ============================================================== softmax / select warps
     else {
+      // a score from its TMEM word: an fp32 integer on the fp8 path, else an int32
+      auto score_f = [&](uint32_t v) -> float { return kF8 ? __uint_as_float(v) : (float)(int)v; };
       const uint32_t tl = tmem + ((uint32_t)((warp & 3) * 32) << 16);
       const uint32_t hist_row = smem_u32(hist) + (uint32_t)srow * 4u;
       const float mo = -m * kLog2e;
@@ -918,7 +928,8 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
               const uint32_t base = hist_row + (uint32_t)(D / 2) * kM * 4u;  // level (d - s)/2: + (d - s) * 256 B
 #pragma unroll
               for (int u = 0; u < 32; ++u) {
-                const uint32_t ad = base - (uint32_t)((int)r[32 * cc + u] * (kM * 2));
+                const int sc = kF8 ? (int)__uint_as_float(r[32 * cc + u]) : (int)r[32 * cc + u];
+                const uint32_t ad = base - (uint32_t)(sc * (kM * 2));
                 if (FULL) {
                   asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(ad) : "memory");
                 } else {
@@ -986,7 +997,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
                 for (int u = 0; u < kFbGroup; ++u) bv[u] = brow[-(32 * cc + g + u)];
 #pragma unroll
                 for (int u = g; u < g + kFbGroup; u += 2) {
-                  const float2 sf2 = make_float2((float)(int)r[32 * cc + u], (float)(int)r[32 * cc + u + 1]);
+                  const float2 sf2 = make_float2(score_f(r[32 * cc + u]), score_f(r[32 * cc + u + 1]));
                   const float2 l2 = __ffma2_rn(sf2, make_float2(c, c), make_float2(bv[u - g], bv[u - g + 1]));
                   const float la = (FULL || 32 * ch + u < nvalid) ? l2.x : -INFINITY;
                   const float lb = (FULL || 32 * ch + u + 1 < nvalid) ? l2.y : -INFINITY;
@@ -1008,7 +1019,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
                 // as fmaf)
 #pragma unroll
                 for (int u = 0; u < 32; u += 2) {
-                  const float2 sf2 = make_float2((float)(int)r[32 * cc + u], (float)(int)r[32 * cc + u + 1]);
+                  const float2 sf2 = make_float2(score_f(r[32 * cc + u]), score_f(r[32 * cc + u + 1]));
                   const float2 b2 = make_float2(brow[-(32 * cc + u)], brow[-(32 * cc + u + 1)]);
                   const float2 l2 = __ffma2_rn(sf2, make_float2(c, c), b2);
                   lg[u] = (FULL || 32 * ch + u < nvalid) ? l2.x : -INFINITY;
@@ -1024,7 +1035,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
                 for (int v = 0; v < 4; ++v) {
                   const int sc = (int)r[32 * cc + u + v];
                   // the score as a float: the integer count, or the comparison mode's fp32 dot product
-                  const float sf = kRef ? __uint_as_float(r[32 * cc + u + v]) : (float)sc;
+                  const float sf = (kRef || kF8) ? __uint_as_float(r[32 * cc + u + v]) : (float)sc;
                   float l;
                   if (HAS_BIAS) {
                     if (kMaskInKoff) kinv |= (kk[v] == 4 * a.k_invalid ? 1u : 0u) << (u + v);
@@ -1225,7 +1236,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
                                  __ldg(reinterpret_cast<const float*>(tab_bytes - ko[32 * half + u + 1])));
               }
               // logits and exp arguments two at a time (packed fp32x2 FMAs, each rounded once)
-              const float2 l2 = __ffma2_rn(make_float2((float)(int)r[u], (float)(int)r[u + 1]), make_float2(c, c), b2);
+              const float2 l2 = __ffma2_rn(make_float2(score_f(r[u]), score_f(r[u + 1])), make_float2(c, c), b2);
               const float la = (FULL || u < nv) ? l2.x : -INFINITY, lb = (FULL || u + 1 < nv) ? l2.y : -INFINITY;
               const float2 x2 = __ffma2_rn(make_float2(la, lb), make_float2(kLog2e, kLog2e), make_float2(mo_p, mo_p));
               const float xa = fast_exp2(x2.x), xb = fast_exp2(x2.y);
@@ -1257,7 +1268,7 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
                 b2 = make_float2(__ldg(reinterpret_cast<const float*>(tab_bytes - ko[32 * half + u])),
                                  __ldg(reinterpret_cast<const float*>(tab_bytes - ko[32 * half + u + 1])));
               }
-              const float2 l2 = __ffma2_rn(make_float2((float)(int)r[u], (float)(int)r[u + 1]), make_float2(c, c), b2);
+              const float2 l2 = __ffma2_rn(make_float2(score_f(r[u]), score_f(r[u + 1])), make_float2(c, c), b2);
               const float la = (FULL || u < nv) ? l2.x : -INFINITY, lb = (FULL || u + 1 < nv) ? l2.y : -INFINITY;
               const float2 x2 = __ffma2_rn(make_float2(la, lb), make_float2(kLog2e, kLog2e), make_float2(mo_p, mo_p));
               const bool ga = la >= pv_cut, gb = lb >= pv_cut;
@@ -1764,17 +1775,18 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         for (int x = 0; x < n_merge; ++x) {
           const int j = (int)hist[x * kM + srow];
           const uint4* kr = reinterpret_cast<const uint4*>(kb + (size_t)j * D);
-          int sc = 0;
+          // s = d - 2 (channels whose signs differ): bit 7 of a +-1 byte is its sign in
+          // both encodings (int8 and e4m3)
+          int diff = 0;
 #pragma unroll
           for (int c16 = 0; c16 < D / 16; ++c16) {
             const uint4 qv = *reinterpret_cast<const uint4*>(sQ + (c16 >> 2) * kM * 64 + srow * 64 +
                                                              (((c16 & 3) ^ ((srow >> 1) & 3)) * 16));
             const uint4 kv = __ldg(kr + c16);
-            sc = __dp4a((int)qv.x, (int)kv.x, sc);
-            sc = __dp4a((int)qv.y, (int)kv.y, sc);
-            sc = __dp4a((int)qv.z, (int)kv.z, sc);
-            sc = __dp4a((int)qv.w, (int)kv.w, sc);
+            diff += __popc((qv.x ^ kv.x) & 0x80808080u) + __popc((qv.y ^ kv.y) & 0x80808080u) +
+                    __popc((qv.z ^ kv.z) & 0x80808080u) + __popc((qv.w ^ kv.w) & 0x80808080u);
           }
+          const int sc = D - 2 * diff;
           float l;
           if (HAS_BIAS) {
             int off;  // entry (i, j) of the extended table sits at rb - off

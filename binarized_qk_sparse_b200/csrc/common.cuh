@@ -95,6 +95,15 @@ __device__ __forceinline__ uint32_t expand_nibble_pm1(uint32_t nib) {
   uint32_t m = (nib * 0x00204081u) & 0x01010101u;  // one bit per byte, no carries
   return 0x01010101u | (m * 0xFEu);                // 0x01 -> +1, 0xFF -> -1
 }
+// The same four signs as e4m3 floats: +1.0 = 0x38, -1.0 = 0xB8 (the sign bit).
+__device__ __forceinline__ uint32_t expand_nibble_pm1_e4m3(uint32_t nib) {
+  uint32_t m = (nib * 0x00204081u) & 0x01010101u;
+  return 0x38383838u | (m * 0x80u);
+}
+// Either encoding (bit 7 of a byte is its sign in both).
+__device__ __forceinline__ uint32_t expand_nibble_pm(uint32_t nib, bool e4m3) {
+  return e4m3 ? expand_nibble_pm1_e4m3(nib) : expand_nibble_pm1(nib);
+}
 
 // ---- legacy warp-level tensor-core MMAs (mma.sync), fp32 / s32 accumulators
 

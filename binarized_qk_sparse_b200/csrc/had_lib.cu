@@ -229,7 +229,7 @@ __global__ void k_untranspose_vq(const int8_t* vqT, int BH, int n, int d, int n_
 had_status launch_prep(const had_shape* s, const void* X0, const void* X1, const void* X2, int first, int ntens,
                        double* sums, float* amax, const float* mu_in0, float* mu_out0, uint32_t* bits0,
                        int8_t* pm0, uint32_t* bits1, int8_t* pm1, int8_t* vqT, float* vscale, cudaStream_t st,
-                       unsigned* status, int vbits = 8) {
+                       unsigned* status, int vbits = 8, bool pm_e4m3 = false) {
   Dims d = dims_of(s);
   PrepArgs pa{};
   pa.X[0] = X0; pa.X[1] = X1; pa.X[2] = X2;
@@ -260,7 +260,7 @@ had_status launch_prep(const had_shape* s, const void* X0, const void* X1, const
   ka.mu_out[0] = mu_out0; ka.mu_out[1] = nullptr;
   ka.bits[0] = bits0; ka.bits[1] = bits1;
   ka.pm[0] = pm0; ka.pm[1] = pm1;
-  ka.vqT = vqT; ka.vscale = vscale; ka.v_bits = vbits; ka.status = status;
+  ka.vqT = vqT; ka.vscale = vscale; ka.v_bits = vbits; ka.pm_e4m3 = pm_e4m3 ? 1 : 0; ka.status = status;
   if (d.d == 32) bf ? k_pack<__nv_bfloat16, 32><<<grid, kPrepThreads, 0, st>>>(ka) : k_pack<float, 32><<<grid, kPrepThreads, 0, st>>>(ka);
   else if (d.d == 128) bf ? k_pack<__nv_bfloat16, 128><<<grid, kPrepThreads, 0, st>>>(ka) : k_pack<float, 128><<<grid, kPrepThreads, 0, st>>>(ka);
   else bf ? k_pack<__nv_bfloat16, 64><<<grid, kPrepThreads, 0, st>>>(ka) : k_pack<float, 64><<<grid, kPrepThreads, 0, st>>>(ka);
@@ -337,6 +337,8 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
   int8_t* vqT = quant ? reinterpret_cast<int8_t*>(ws + w.vqT) : nullptr;
   float* vscale = quant ? reinterpret_cast<float*>(ws + w.vscale) : nullptr;
   const bool do_v = quant && need_v;
+  // top-N with a bias scores on the fp8 tensor path: K~ as e4m3 +-1
+  const bool e4m3 = select_kind(s, bias, N) == SEL_TOPN_FLOAT;
   had_status r = HAD_OK;
   const size_t elem = (s->in_dtype == HAD_BF16) ? 2 : 4;
   const size_t head_bytes = (size_t)s->n * s->d * elem;
@@ -366,6 +368,7 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
     ha.B = s->B; ha.H = s->H; ha.n = s->n; ha.n_pad = dims_of(s).n_pad;
     ha.seqlens = s->seqlens;
     ha.qbits = qbits; ha.kpm = kpm; ha.vqT = vqT; ha.vscale = vscale; ha.v_bits = vbits; ha.status = status;
+    ha.kpm_e4m3 = e4m3 ? 1 : 0;
     ha.bias_slice = do_v ? 3 : 2;  // relative-position tables ride along as one more grid slice
     dim3 grid(dims_of(s).BH, ha.bias_slice + (has_bias && !ba.dense ? 1 : 0));
     const int smem = (int)head_bytes;
@@ -381,7 +384,7 @@ had_status prepare_stage(const void* Q, const void* K, const void* V, const had_
     if ((r = check_launch("k_prep_head")) != HAD_OK) return r;
   } else {
     r = launch_prep(s, Q, K, V, 0, do_v ? 3 : 2, sums, amax, nullptr, nullptr, qbits, nullptr, nullptr, kpm, vqT,
-                    vscale, st, status, vbits);
+                    vscale, st, status, vbits, e4m3);
     if (r != HAD_OK) return r;
     if (has_bias && !ba.dense) {
       k_bias_range<<<s->H, kBiasRangeThreads, 0, st>>>(ba);

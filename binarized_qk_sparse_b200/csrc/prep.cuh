@@ -151,7 +151,8 @@ struct PackArgs {
   const float* mu_in[2];  // optional caller means per tensor 0/1
   float* mu_out[2];       // optional mean outputs per tensor 0/1
   uint32_t* bits[2];      // [BH][n][D/32] per tensor 0/1 (or null)
-  int8_t* pm[2];          // [BH][n_pad][D] +-1 int8 rows per tensor 0/1 (or null); +1 past L
+  int8_t* pm[2];          // [BH][n_pad][D] +-1 rows per tensor 0/1 (or null); +1 past L
+  int pm_e4m3;            // the +-1 rows as e4m3 bytes (0x38 / 0xB8) instead of int8 (0x01 / 0xFF)
   int8_t* vqT;            // [BH][D][n_pad] int8, or [BH][D][n_pad / 2] packed 4-bit (key 2k in the low nibble of byte k)
   float* vscale;          // [BH][D]
   int v_bits;             // 8: int8 V, scale absmax/127; 4: 4-bit V, scale absmax/7
@@ -208,10 +209,10 @@ __global__ void __launch_bounds__(kPrepThreads) k_pack(const PackArgs a) {
         for (int u = 0; u < EPT; ++u) v |= (x[u] < stat[cg * EPT + u] ? 1u : 0u) << u;
       }
       if (pmo && i < a.n_pad) {
-        // +-1 int8 copy of the same signs: bit 1 -> 0xFF (-1), bit 0 -> 0x01 (+1)
-        uint32_t w0 = expand_nibble_pm1(v & 15u);
+        // +-1 copy of the same signs (bit 1 -> -1): int8 0xFF / 0x01, or e4m3 0xB8 / 0x38
+        uint32_t w0 = expand_nibble_pm(v & 15u, a.pm_e4m3);
         if (EPT == 8) {
-          uint32_t w1 = expand_nibble_pm1((v >> 4) & 15u);
+          uint32_t w1 = expand_nibble_pm((v >> 4) & 15u, a.pm_e4m3);
           *reinterpret_cast<uint2*>(pmo + (size_t)i * kD + cg * EPT) = make_uint2(w0, w1);
         } else {
           *reinterpret_cast<uint32_t*>(pmo + (size_t)i * kD + cg * EPT) = w0;
@@ -297,6 +298,7 @@ struct HeadArgs {
   const int32_t* seqlens;
   uint32_t* qbits;     // tensor 0 -> [BH][n][2]
   int8_t* kpm;         // tensor 1 -> [BH][n_pad][64]
+  int kpm_e4m3;        // K~ as e4m3 bytes (see PackArgs::pm_e4m3)
   int8_t* vqT;         // tensor 2 -> [BH][64][n_pad] int8, or [BH][64][n_pad / 2] packed 4-bit
   float* vscale;       // [BH][64]
   int v_bits;          // 8 or 4 (see PackArgs)
@@ -574,13 +576,14 @@ __global__ void __launch_bounds__(kHeadThreads) k_prep_head(const HeadArgs a, co
       if (tz == 0) {
         *reinterpret_cast<uint2*>(a.qbits + ((size_t)bh * a.n + i) * kW) = make_uint2(w[0], w[1]);
       } else {
-        // +-1 int8 row of K (bit 1 -> -1); rows past L are +1
+        // +-1 row of K (bit 1 -> -1), int8 or e4m3; rows past L are +1
         uint4* dst = reinterpret_cast<uint4*>(a.kpm + ((size_t)bh * a.n_pad + i) * kD);
+        const bool e4 = a.kpm_e4m3 != 0;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const uint32_t f = w[q >> 1] >> ((q & 1) * 16);
-          dst[q] = make_uint4(expand_nibble_pm1(f & 15u), expand_nibble_pm1((f >> 4) & 15u),
-                              expand_nibble_pm1((f >> 8) & 15u), expand_nibble_pm1((f >> 12) & 15u));
+          dst[q] = make_uint4(expand_nibble_pm(f & 15u, e4), expand_nibble_pm((f >> 4) & 15u, e4),
+                              expand_nibble_pm((f >> 8) & 15u, e4), expand_nibble_pm((f >> 12) & 15u, e4));
         }
       }
     }

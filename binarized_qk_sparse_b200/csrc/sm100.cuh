@@ -58,22 +58,26 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar_addr, uint32_t parity
 }
 // Wait for the phase with the given parity to complete, for at most
 // `max_cycles` SM clocks.  Returns false on timeout (the caller records it and
-// winds down instead of waiting on).  A wait that has not ended after
-// kSpinCycles (about a microsecond, longer than a pipeline hand-off) sleeps
-// between tries, 32 ns at first and doubling up to `max_sleep_ns`, so that warps
-// waiting a long time leave the issue slots to the working ones.
+// winds down instead of waiting on).  The clock is read once per kTriesPerCheck
+// tries (a try itself suspends the thread for a while in hardware), so a polling
+// warp spends few issue slots on the bookkeeping; a wait that has not ended after
+// `spin_cycles` (about a microsecond, longer than a pipeline hand-off) sleeps
+// between rounds, 32 ns at first and doubling up to `max_sleep_ns`.
 constexpr long long kSpinCycles = 2000;
+constexpr int kTriesPerCheck = 8;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, long long max_cycles,
-                                          uint32_t max_sleep_ns = 128) {
+                                          uint32_t max_sleep_ns = 128, long long spin_cycles = kSpinCycles) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
   const long long t0 = clock64();
   uint32_t ns = 32;
   while (true) {
-    if (mbar_try_wait(a, parity)) return true;
+#pragma unroll 1
+    for (int i = 0; i < kTriesPerCheck; ++i)
+      if (mbar_try_wait(a, parity)) return true;
     const long long dt = clock64() - t0;
     if (dt > max_cycles) return false;
-    if (dt > kSpinCycles) {
+    if (dt > spin_cycles) {
       __nanosleep(ns);
       ns = ns < max_sleep_ns ? 2 * ns : max_sleep_ns;
     }
@@ -176,6 +180,20 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N, bool a_signed, boo
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
+}
+
+// e4m3 x e4m3 -> f32 (kind::f8f6f4, both K-major).
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc], fp8 operands (32 per K-step, as int8)
+__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 // D[tmem] (+)= A[smem desc] * B[smem desc]
