@@ -1549,10 +1549,16 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         // window, fewer than r_rank of them; bin 0 is never reached: at least r_rank
         // keys reach the window's low end)
         int cum = 0, bsel = 0, kbin = 0;
-        for (int bb = 127; bb >= 1; --bb) {
-          const int k = (int)hist[bb * kM + srow];
-          if (cum + k >= r_rank) { bsel = bb; kbin = k; break; }
-          cum += k;
+        for (int b0 = 127; b0 >= 1 && bsel == 0; b0 -= 8) {  // eight counts in flight
+          int kk[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) kk[j] = b0 - j >= 1 ? (int)hist[(b0 - j) * kM + srow] : 0;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            if (bsel != 0 || b0 - j < 1) continue;
+            if (cum + kk[j] >= r_rank) { bsel = b0 - j; kbin = kk[j]; }
+            else cum += kk[j];
+          }
         }
         // a sampled bracket that missed: rank r_rank above the window (bin 127) or
         // below it (bin 0).  A bracket from every tile's levels cannot miss; should
@@ -1568,13 +1574,24 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
           r_state = 1;
         } else {
         // the bin's keys are the logits in [w_lo, w_cut): the least floats that map to
-        // bins bsel and bsel + 1, found by bisection over the order keys of floats
+        // bins bsel and bsel + 1, found by bisection over the order keys of floats,
+        // from 128 keys around the map's inverse when the map confirms that bracket
         auto fb_bin = [&](float x) -> int {
           const float w = __fmaf_rn(fma_sat(x, fb_sc, fb_off), kFbSpan, kFbMg);
           return (int)((__float_as_uint(w) & 0xFE00u) >> 9);
         };
         auto fb_least = [&](int bin) -> float {
           uint32_t klo = 0x007FFFFFu, khi = 0xFF800000u;  // -inf (bin 0), +inf (bin 127)
+          const float est = ((512.0f * (float)bin - 0.5f) / kFbSpan - fb_off) / fb_sc;
+          if (isfinite(est)) {
+            const uint32_t ke = float_order_key(est);
+            const uint32_t ka = ke - 64u, kb = ke + 64u;
+            if (ka > klo && ka < ke && kb < khi && kb > ke && fb_bin(order_key_float(ka)) < bin &&
+                fb_bin(order_key_float(kb)) >= bin) {
+              klo = ka;
+              khi = kb;
+            }
+          }
           while (khi - klo > 1u) {
             const uint32_t mid = klo + ((khi - klo) >> 1);
             if (fb_bin(order_key_float(mid)) >= bin) khi = mid;
