@@ -14,27 +14,6 @@ constexpr int kAttnThreads = 128;   // 4 warps
 
 enum { KMAP_NATURAL = 0, KMAP_U8 = 1 };
 
-struct AttnArgs {
-  const uint32_t* qbits;   // [BH][n][2]
-  const int8_t* kpm;       // [BH][n_pad][64] +-1 int8
-  const void* V;           // [BH][n][64] bf16 / fp32   (float mode)
-  const int8_t* vqT;       // [BH][64][n_pad]           (uint8 mode)
-  const float* vscale;     // [BH][64]
-  const float* table;      // [H][th][tw] or null ([H][n][n] when bias_dense)
-  int gh, gw, prefix, th, tw;
-  int bias_dense;          // 1: b_ij = table[h][i][j]
-  const float* bminmax;    // [H][2]
-  const int32_t* seqlens;
-  void* O;
-  int o_bf16;
-  int32_t* idx;            // EXP_IDX  [BH][n][N]
-  uint8_t* codes;          // EXP_CODES [BH][row_end-row_begin][n]
-  int row_begin, row_end;
-  int B, H, n, n_pad, N;
-  unsigned* status;
-  float c_head[kMaxHeads];
-};
-
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
   uint32_t d = (uint32_t)__cvta_generic_to_shared(smem_dst);
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(d), "l"(gmem_src));
