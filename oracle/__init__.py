@@ -59,12 +59,13 @@ def lib():
         L.hado_binary_scores.argtypes = [P, P, I, I, I, I, P, P]
         L.hado_v_quant.argtypes = [P, I, I, I, I, P, P, P]
         L.hado_v_quant4.argtypes = [P, I, I, I, I, P, P, P]
+        L.hado_qkv_project.argtypes = [P, P, I, I, I, I, I, P, P, P, P, P, P, P, P]
         L.hado_logits.argtypes = [P, P, I, I, I, I, P, P, I, I, I, P, P, P]
         L.hado_attention.argtypes = [P, P, P, I, I, I, I, P, P, I, I, I, P, P, I, I, P, I64, P, P, P, P, P, P,
                                      P, P, P, P]
         L.hado_dense_attention.argtypes = [P, P, P, I, I, I, I, P, P, I, I, I, I, P, I64, P]
         for f in (L.hado_channel_mean, L.hado_sign_pack, L.hado_binary_scores, L.hado_v_quant, L.hado_v_quant4,
-                  L.hado_logits,
+                  L.hado_logits, L.hado_qkv_project,
                   L.hado_attention, L.hado_dense_attention):
             f.restype = I
         _lib = L
@@ -141,6 +142,23 @@ def v_quant(V, seqlens=None, bits=8):
         raise ValueError("bits must be 8 or 4")
     _check(fn(_p(V), B, H, n, d, _p(s), _p(Vq), _p(sc)), "v_quant")
     return Vq, sc
+
+
+def qkv_project(X, W, H, d, seqlens=None):
+    """The projection that precedes the path and its binarization: X [B, n, Dm],
+    W [3*H*d, Dm] -> (Q, K, V) fp64 [B, H, n, d], mu_q, mu_k fp32 [B, H, d],
+    qbits, kbits uint32 [B, H, n, d/32]."""
+    X, W = _f32(X), _f32(W)
+    B, n, Dm = X.shape
+    if W.shape != (3 * H * d, Dm):
+        raise ValueError("W must be [3*H*d, Dm]")
+    s = _seq(seqlens)
+    Q, K, V = (np.zeros((B, H, n, d), np.float64) for _ in range(3))
+    mq, mk = np.zeros((B, H, d), np.float32), np.zeros((B, H, d), np.float32)
+    qb, kb = np.zeros((B, H, n, d // 32), np.uint32), np.zeros((B, H, n, d // 32), np.uint32)
+    _check(lib().hado_qkv_project(_p(X), _p(W), B, n, Dm, H, d, _p(s), _p(Q), _p(K), _p(V), _p(mq), _p(mk),
+                                  _p(qb), _p(kb)), "qkv_project")
+    return Q, K, V, mq, mk, qb, kb
 
 
 @dataclass

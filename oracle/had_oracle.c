@@ -96,6 +96,69 @@ int hado_channel_mean(const float* X, int B, int H, int n, int d, const int32_t*
   return HADO_OK;
 }
 
+/* The projection that precedes the path, with its binarization (the step the
+ * attention's inputs come from; BinaryAttention's Table 8 counts the Q/K/V
+ * quantization of this step against the kernel).  X is [B][n][Dm] tokens,
+ * W is [3*H*d][Dm] (output channel o = t*H*d + h*d + c of tensor t in {Q, K, V},
+ * the row layout of a linear layer's weight).  Per the plain definition:
+ *   P[t][b][h][i][c] = sum_k X[b][i][k] * W[o][k]          (fp64, k in order)
+ *   mu_t[b][h][c]    = mean over the valid tokens of P[t]   (fp64 sum in token
+ *                      order, divided by L, rounded once to fp32; t in {Q, K})
+ *   bits_t           = P[t] < mu_t, packed as in hado_sign_pack (tokens past L: 0)
+ * Q, K, V receive P in fp64 [B][H][n][d] (rows past L included). */
+int hado_qkv_project(const float* X, const float* W, int B, int n, int Dm, int H, int d, const int32_t* seqlens,
+                     double* Q, double* K, double* V, float* mu_q, float* mu_k, uint32_t* qbits, uint32_t* kbits) {
+  if (!X || !W || !Q || !K || !V || !mu_q || !mu_k || !qbits || !kbits || B <= 0 || n <= 0 || Dm <= 0 || H <= 0 ||
+      d <= 0 || d % 32 != 0)
+    return HADO_ERR_ARG;
+  for (int b = 0; b < B; ++b) {
+    int L = valid_len(seqlens, b, n);
+    if (L < 1 || L > n) return HADO_ERR_ARG;
+  }
+  double* outs[3] = {Q, K, V};
+  const int64_t hd = (int64_t)H * d;
+#pragma omp parallel for schedule(static)
+  for (int64_t bi = 0; bi < (int64_t)B * n; ++bi) {
+    int b = (int)(bi / n), i = (int)(bi % n);
+    const float* x = X + (size_t)bi * Dm;
+    for (int t = 0; t < 3; ++t)
+      for (int h = 0; h < H; ++h)
+        for (int c = 0; c < d; ++c) {
+          const float* w = W + (size_t)(t * hd + (int64_t)h * d + c) * Dm;
+          double acc = 0.0;
+          for (int k = 0; k < Dm; ++k) acc += (double)x[k] * (double)w[k];
+          outs[t][(((size_t)b * H + h) * n + i) * d + c] = acc;
+        }
+  }
+  const int Wd = d / 32;
+  for (int t = 0; t < 2; ++t) {
+    const double* P = outs[t];
+    float* mu = t == 0 ? mu_q : mu_k;
+    uint32_t* bits = t == 0 ? qbits : kbits;
+#pragma omp parallel for schedule(static)
+    for (int64_t bh = 0; bh < (int64_t)B * H; ++bh) {
+      int L = valid_len(seqlens, (int)(bh / H), n);
+      const double* Ph = P + (size_t)bh * n * d;
+      for (int c = 0; c < d; ++c) {
+        double sum = 0.0;
+        for (int i = 0; i < L; ++i) sum += Ph[(size_t)i * d + c];
+        mu[(size_t)bh * d + c] = (float)(sum / (double)L);
+      }
+      for (int i = 0; i < n; ++i)
+        for (int w = 0; w < Wd; ++w) {
+          uint32_t word = 0;
+          if (i < L)
+            for (int j = 0; j < 32; ++j) {
+              int c = 32 * w + j;
+              if (Ph[(size_t)i * d + c] < (double)mu[(size_t)bh * d + c]) word |= (uint32_t)1 << j;
+            }
+          bits[((size_t)bh * n + i) * Wd + w] = word;
+        }
+    }
+  }
+  return HADO_OK;
+}
+
 /* Step 2: sign and pack.  bits[b][h][i][w], bit j of word w <=> channel 32w+j is
  * negative after centering (x < mu).  Tokens i >= L get all-zero words. */
 int hado_sign_pack(const float* X, const float* mu, int B, int H, int n, int d, const int32_t* seqlens,

@@ -549,3 +549,54 @@ def test_u8i4_output_equals_independent_numpy(oracle_mod):
     s4 = (np.abs(V).max(axis=2) / 7.0)
     bound = (0.5 / 255) * np.abs(V).sum(axis=2, keepdims=True) + 0.5 * s4[:, :, None, :] * 1.0
     assert np.all(np.abs(r.O - rf.O) <= bound + 1e-9)
+
+
+# ----------------------------------------------------------------------------- the projection before the path
+
+def _np_pack_lsb(mask):
+    """[..., d] bool -> [..., d/32] uint32, channel 32w + j at bit j of word w (numpy, no oracle code)."""
+    d = mask.shape[-1]
+    m = mask.reshape(mask.shape[:-1] + (d // 32, 32)).astype(np.uint64)
+    return (m << np.arange(32, dtype=np.uint64)).sum(axis=-1).astype(np.uint32)
+
+
+@pytest.mark.parametrize("seqlens", [None, [70, 33, 1]])
+def test_qkv_projection_against_independent_numpy(oracle_mod, seqlens):
+    """Projection, means and sign bits of the step before the path, against numpy:
+    P = X W^T in fp64 (einsum), the mean over the valid tokens, and the LSB-first packing
+    of P < mu; tokens past L carry zero words."""
+    rng = np.random.default_rng(41)
+    B, n, Dm, H, d = 3, 70, 192, 2, 64
+    X = workloads.bf16_round(rng.standard_normal((B, n, Dm)).astype(np.float32))
+    W = workloads.bf16_round((rng.standard_normal((3 * H * d, Dm)) * 0.05).astype(np.float32))
+    sl = None if seqlens is None else np.array(seqlens, np.int32)
+    Q, K, V, mq, mk, qb, kb = oracle_mod.qkv_project(X, W, H, d, sl)
+    P = np.einsum("bik,ok->bio", X.astype(np.float64), W.astype(np.float64)).reshape(B, n, 3, H, d)
+    P = P.transpose(2, 0, 3, 1, 4)  # [t][b][h][i][c]
+    for t, got in enumerate((Q, K, V)):
+        np.testing.assert_allclose(got, P[t], rtol=0, atol=1e-12)
+    L = np.full(B, n) if sl is None else sl
+    for t, (mu, bits) in enumerate(((mq, qb), (mk, kb))):
+        ref_mu = np.stack([P[t][b, :, :L[b]].mean(axis=1) for b in range(B)]).astype(np.float32)
+        np.testing.assert_array_equal(mu, ref_mu)
+        mask = P[t] < mu[:, :, None, :].astype(np.float64)
+        for b in range(B):
+            mask[b, :, L[b]:] = False
+        np.testing.assert_array_equal(bits, _np_pack_lsb(mask))
+
+
+def test_qkv_means_are_the_projected_token_mean(oracle_mod):
+    """The mean of a linear map's outputs is the map of the mean input: mu_t = mean_i(X_i) W_t^T.
+    This is the identity the fused projection uses to binarize in its epilogue; in fp64 both
+    sides agree to rounding, so the fp32 means agree to one unit in the last place."""
+    rng = np.random.default_rng(43)
+    B, n, Dm, H, d = 2, 197, 256, 3, 64
+    X = workloads.bf16_round(rng.standard_normal((B, n, Dm)).astype(np.float32))
+    W = workloads.bf16_round((rng.standard_normal((3 * H * d, Dm)) * 0.05).astype(np.float32))
+    sl = np.array([197, 120], np.int32)
+    _, _, _, mq, mk, _, _ = oracle_mod.qkv_project(X, W, H, d, sl)
+    for b in range(B):
+        xbar = X[b, :sl[b]].astype(np.float64).mean(axis=0)
+        lin = (W.astype(np.float64) @ xbar).reshape(3, H, d)
+        for t, mu in enumerate((mq, mk)):
+            np.testing.assert_array_max_ulp(mu[b], lin[t].astype(np.float32), maxulp=1)
