@@ -97,9 +97,15 @@ def lib():
         L.had_attention_codes_u8.argtypes = [P, P, P, SP, BP, P, P, I, I, I, P, P, SZ, P]
         L.had_quantize_v.argtypes = [P, SP, P, P, P, SZ, P]
         L.had_quantize_v4.argtypes = [P, SP, P, P, P, SZ, P]
+        L.had_attention_prepare.argtypes = [P, P, P, SP, BP, I, I, P, SZ, P]
+        L.had_attention_prepared.argtypes = [P, SP, BP, P, P, I, I, P, I, P, SZ, P]
+        L.had_qkv_workspace_size.argtypes = [SP, I, I, I, BP]
+        L.had_qkv_workspace_size.restype = SZ
+        L.had_qkv_prepare.argtypes = [P, P, SP, I, BP, I, I, P, P, SZ, P]
         for f in ("had_binarize_pack", "had_binarize_pack_noalloc", "had_attention", "had_attention_host",
                   "had_dense_reference_mode", "had_scores_int",
                   "had_topn_indices", "had_attention_codes_u8", "had_quantize_v", "had_quantize_v4",
+                  "had_attention_prepare", "had_attention_prepared", "had_qkv_prepare",
                   "had_get_device_status"):
             getattr(L, f).restype = I
         L.had_attention_scores.argtypes = [P, P, SP, P, P, SZ, P]
@@ -421,6 +427,53 @@ def had_quantize_v(V, seqlens=None, workspace=None, stream=None):
 def had_quantize_v4(V, seqlens=None, workspace=None, stream=None):
     """Per-channel 4-bit V (codes in [-7, 7], one per int8) [B,H,n,d] and its fp32 scales [B,H,d]."""
     return _quantize("had_quantize_v4", HAD_MODE_U8I4, V, seqlens, workspace, stream)
+
+
+def had_qkv_attention(X, W, H, N=0, mode="float", seqlens=None, bias=None, alpha_q=None, alpha_k=None, out=None,
+                      out_dtype=None, workspace=None, stream=None, return_v=False):
+    """The projection before the path (Q|K|V = X W^T, W in a linear layer's [3*H*64, Dm]
+    layout), with Q and K binarized in its epilogue, then the fused attention.
+
+    X: bf16 [B, n, Dm]; W: bf16 [3*H*64, Dm].  Returns O [B, H, 64-channel heads] as
+    [B, H, n, 64] (and V, the bf16 projection the attention read, with return_v)."""
+    _check_dev(X, W, seqlens, out, workspace)
+    if X.dtype != torch.bfloat16 or W.dtype != torch.bfloat16:
+        raise TypeError("X and W must be bfloat16")
+    B, n, Dm = X.shape
+    d = 64
+    if seqlens is not None and seqlens.dtype != torch.int32:
+        raise TypeError("seqlens must be int32")
+    shp = had_shape(B, H, n, d, HAD_BF16, None if seqlens is None else seqlens.data_ptr())
+    m = _MODES[mode]
+    bs = _bias_struct(bias)
+    V = torch.empty((B, H, n, d), dtype=torch.bfloat16, device=X.device)
+    if out is None:
+        out = torch.empty((B, H, n, d), dtype=out_dtype or torch.bfloat16, device=X.device)
+    need = lib().had_qkv_workspace_size(ctypes.byref(shp), int(Dm), int(N), m, bs)
+    if need == 0:
+        _raise(HAD_ERR_UNSUPPORTED, "had_qkv_workspace_size")
+    ws = _workspace(need, X.device, workspace, stream)
+    st = lib().had_qkv_prepare(_ptr(X), _ptr(W), ctypes.byref(shp), int(Dm), bs, int(N), m, _ptr(V), _ptr(ws),
+                               ws.numel(), _stream(stream))
+    _raise(st, "had_qkv_prepare")
+    aq_keep, aq = _alpha(alpha_q, H)
+    ak_keep, ak = _alpha(alpha_k, H)
+    st = lib().had_attention_prepared(_ptr(V), ctypes.byref(shp), bs, aq, ak, int(N), m, _ptr(out), _dtype_code(out),
+                                      _ptr(ws), ws.numel(), _stream(stream))
+    _raise(st, "had_attention_prepared")
+    return (out, V) if return_v else out
+
+
+def had_qkv_workspace(X, H, N=0, mode="float", seqlens=None, bias=None):
+    """A workspace of the size had_qkv_attention needs (uint8 tensor on X's device).  It
+    starts with the attention workspace: Q's sign bits as [B, H, n, 2] uint32 words at
+    offset 0, then K's +-1 rows [B, H, n_pad, 64] at the next 256-byte boundary."""
+    B, n, Dm = X.shape
+    shp = had_shape(B, H, n, 64, HAD_BF16, None if seqlens is None else seqlens.data_ptr())
+    need = lib().had_qkv_workspace_size(ctypes.byref(shp), int(Dm), int(N), _MODES[mode], _bias_struct(bias))
+    if need == 0:
+        _raise(HAD_ERR_UNSUPPORTED, "had_qkv_workspace_size")
+    return torch.empty(need, dtype=torch.uint8, device=X.device)
 
 
 def had_get_device_status() -> int:

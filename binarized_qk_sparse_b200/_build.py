@@ -15,7 +15,7 @@ CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libhad_b200.so")
 OBJ_DIR = os.path.join(HERE, "_build")
 SOURCES = ["had_lib.cu", "attn_d128.cu"]
-DEPS = ["common.cuh", "sm100.cuh", "prep.cuh", "attn.cuh", "attn_tc.cuh", "probe.cuh",
+DEPS = ["common.cuh", "sm100.cuh", "prep.cuh", "attn.cuh", "attn_tc.cuh", "probe.cuh", "qkv.cuh",
         "launch.cuh", "had_lib.cu", "attn_d128.cu"]
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

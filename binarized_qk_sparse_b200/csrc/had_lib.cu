@@ -29,6 +29,7 @@
 #include "attn_tc.cuh"
 #include "launch.cuh"
 #include "probe.cuh"
+#include "qkv.cuh"
 
 namespace had {
 
@@ -86,6 +87,8 @@ inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 
 struct Dims {
   int B, H, n, d, BH, nchunks, n_pad;
 };
+
+constexpr int kQkvMaxDm = 16384;  // model width of the fused projection
 
 Dims dims_of(const had_shape* s) {
   Dims d;
@@ -554,6 +557,33 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
   return launch::dispatch_tc<64, EXP>(sel, md, bias_kind, vf32, rows, a, grid, st);
 }
 
+// Workspace of the fused projection: the attention workspace (so that
+// had_attention_prepared can run on it), then X's token partial sums and the
+// means of Q and K.
+struct QkvWs {
+  size_t xpart, mu, total;
+  int nch;
+};
+
+QkvWs qkv_ws_layout(const had_shape* s, int Dm, int vbits, const had_relpos_bias* bias) {
+  QkvWs q{};
+  size_t off = align_up(ws_layout(s, vbits, bias).total);
+  q.nch = (s->n + qkv::kXsumChunk - 1) / qkv::kXsumChunk;
+  q.xpart = off; off += align_up((size_t)s->B * q.nch * Dm * 8);
+  q.mu = off; off += align_up((size_t)2 * s->B * s->H * 64 * 4);
+  q.total = off;
+  return q;
+}
+
+had_status check_qkv_shape(const had_shape* s, int Dm) {
+  had_status r = check_shape(s);
+  if (r != HAD_OK) return r;
+  if (s->d != 64 || s->in_dtype != HAD_BF16) return HAD_ERR_UNSUPPORTED;
+  if (Dm <= 0 || Dm % 64 != 0) return HAD_ERR_INVALID;
+  if (Dm > kQkvMaxDm || 3 * s->H > 65535) return HAD_ERR_UNSUPPORTED;
+  return HAD_OK;
+}
+
 had_status device_status_ptr(unsigned** out) {
   int dev = 0;
   cudaError_t ce = cudaGetDevice(&dev);
@@ -829,6 +859,84 @@ had_status had_attention_prepared(const void* V, const had_shape* s, const had_r
   if ((r = device_status_ptr(&status)) != HAD_OK) return r;
   return attend_stage<EXP_NONE>(V, s, bias, alpha_q, alpha_k, N, mode, O, o_dtype, nullptr, nullptr, 0, 0, workspace,
                                 static_cast<cudaStream_t>(stream), status);
+}
+
+size_t had_qkv_workspace_size(const had_shape* s, int Dm, int N, had_mode mode, const had_relpos_bias* bias) {
+  (void)N;
+  if (check_qkv_shape(s, Dm) != HAD_OK || check_bias(s, bias) != HAD_OK || !mode_ok(mode)) return 0;
+  return qkv_ws_layout(s, Dm, vbits_of(mode), bias).total;
+}
+
+had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, int Dm, const had_relpos_bias* bias,
+                           int N, had_mode mode, void* V_out, void* workspace, size_t ws_bytes, void* stream) {
+  had_status r = check_qkv_shape(s, Dm);
+  if (r != HAD_OK) return r;
+  if ((r = check_bias(s, bias)) != HAD_OK) return r;
+  if (N < 0 || !mode_ok(mode)) return HAD_ERR_INVALID;
+  if (!X || !Wqkv || !V_out || !aligned16(X) || !aligned16(Wqkv) || !aligned16(V_out)) return HAD_ERR_INVALID;
+  const int vbits = vbits_of(mode);
+  const QkvWs q = qkv_ws_layout(s, Dm, vbits, bias);
+  if (!workspace || ws_bytes < q.total || !aligned16(workspace)) return HAD_ERR_INVALID;
+  unsigned* status = nullptr;
+  if ((r = device_status_ptr(&status)) != HAD_OK) return r;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const Ws w = ws_layout(s, vbits, bias);
+  Dims d = dims_of(s);
+  const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
+  const __nv_bfloat16* Wb = static_cast<const __nv_bfloat16*>(Wqkv);
+  double* xpart = reinterpret_cast<double*>(ws + q.xpart);
+  float* mu = reinterpret_cast<float*>(ws + q.mu);
+  // the means of Q and K from X's token means
+  qkv::k_xsum<<<dim3((Dm + qkv::kXsumThreads - 1) / qkv::kXsumThreads, q.nch, d.B), qkv::kXsumThreads, 0, st>>>(
+      Xb, d.n, Dm, s->seqlens, q.nch, xpart);
+  if ((r = check_launch("k_xsum")) != HAD_OK) return r;
+  qkv::k_mu<<<dim3((2 * d.H * 64 + qkv::kMuWarps - 1) / qkv::kMuWarps, d.B), qkv::kMuWarps * 32, 0, st>>>(
+      Wb, xpart, q.nch, d.n, d.B, d.H, Dm, s->seqlens, status, mu);
+  if ((r = check_launch("k_mu")) != HAD_OK) return r;
+  // the projection, binarized in its epilogue, into the attention workspace
+  qkv::QkvArgs qa;
+  memset(&qa, 0, sizeof(qa));
+  if ((r = encode_2d(&qa.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, Dm, (uint64_t)d.B * d.n, (uint64_t)Dm * 2, 64,
+                     qkv::kM, CU_TENSOR_MAP_SWIZZLE_128B)) != HAD_OK)
+    return r;
+  if ((r = encode_2d(&qa.tm_w, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Wqkv, Dm, (uint64_t)3 * d.H * 64, (uint64_t)Dm * 2,
+                     64, qkv::kN, CU_TENSOR_MAP_SWIZZLE_128B)) != HAD_OK)
+    return r;
+  qa.B = d.B; qa.H = d.H; qa.n = d.n; qa.n_pad = d.n_pad; qa.Dm = Dm;
+  qa.seqlens = s->seqlens;
+  qa.mu = mu;
+  qa.qbits = reinterpret_cast<uint32_t*>(ws + w.qbits);
+  qa.kpm = reinterpret_cast<int8_t*>(ws + w.kpm);
+  qa.k_e4m3 = select_kind(s, bias, N) == SEL_TOPN_FLOAT ? 1 : 0;  // the fp8 score path's +-1 encoding
+  qa.V = static_cast<__nv_bfloat16*>(V_out);
+  qa.status = status;
+  {
+    static std::mutex smu;
+    static bool configured[kMaxDevices] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(smu);
+    if (dev >= 0 && dev < kMaxDevices && !configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(qkv::k_qkv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           qkv::QkvSmem::kTotal);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_qkv_tc)");
+      configured[dev] = true;
+    }
+  }
+  qkv::k_qkv_tc<<<dim3((d.n + qkv::kM - 1) / qkv::kM, d.B, 3 * d.H), qkv::kThreads, qkv::QkvSmem::kTotal, st>>>(qa);
+  if ((r = check_launch("k_qkv_tc")) != HAD_OK) return r;
+  // the bias tables and, in the uint8 modes, the quantized V^T, as the attention's prepare stage makes them
+  if (bias && bias->table &&
+      (r = build_bias_tables(s, bias, ws + w.bminmax, ws + w.bext, ws + w.expb, st)) != HAD_OK)
+    return r;
+  if (vbits != 0) {
+    r = launch_prep(s, nullptr, nullptr, V_out, 2, 1, reinterpret_cast<double*>(ws + w.sums),
+                    reinterpret_cast<float*>(ws + w.amax), nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                    reinterpret_cast<int8_t*>(ws + w.vqT), reinterpret_cast<float*>(ws + w.vscale), st, status, vbits);
+    if (r != HAD_OK) return r;
+  }
+  return HAD_OK;
 }
 
 had_status had_topn_indices(const void* Q, const void* K, const had_shape* s, const had_relpos_bias* bias,

@@ -147,6 +147,32 @@ had_status had_attention_prepared(const void* V, const had_shape* s, const had_r
                                   const float* alpha_q, const float* alpha_k, int N, had_mode mode, void* O,
                                   had_dtype o_dtype, void* workspace, size_t ws_bytes, void* stream);
 
+/* ---- the projection before the path, fused with the binarization ---------
+ * had_qkv_prepare takes the step that produces the attention's inputs, the QKV
+ * projection Q|K|V = X Wqkv^T, and binarizes Q and K in its epilogue instead of
+ * in a separate quantization pass (BinaryAttention §2.2 scaled binarization; its
+ * Table 8 counts that pass against the kernel):
+ *   mu_Q[b][h][c] = mean over the valid tokens of X[b] Wq^T, computed as
+ *                   xbar_b . Wq[h*64 + c] with xbar_b the mean of X[b]'s valid tokens
+ *                   (the same value in exact arithmetic; fp64, one rounding to fp32);
+ *   Q bits        = (X Wq^T < mu_Q) per token and channel, from the fp32 tensor-core
+ *                   projection; likewise K (as the +-1 rows the score MMA reads);
+ *   V_out         = X Wv^T, rounded to bf16.
+ * It fills `workspace` as had_attention_prepare does (including the bias tables
+ * and, in the uint8 modes, the quantized V), so that had_attention_prepared(V_out,
+ * s, bias, alpha_q, alpha_k, N, mode, O, ...) on the same stream and workspace
+ * completes the path.
+ *   X:     DEVICE bf16 [B][n][Dm] tokens; Dm > 0, a multiple of 64, <= 16384.
+ *   Wqkv:  DEVICE bf16 [3*H*64][Dm], a linear layer's weight layout: row h*64 + c
+ *          is Q's channel c of head h, row H*64 + h*64 + c K's, row 2*H*64 + h*64 + c V's.
+ *   s:     B, H, n, d = 64, in_dtype HAD_BF16 (HAD_ERR_UNSUPPORTED otherwise), seqlens.
+ *   V_out: DEVICE bf16 [B][H][n][64] (written for every token < n).
+ *   workspace: at least had_qkv_workspace_size(s, Dm, N, mode, bias) bytes.
+ * Errors as had_attention (host validation first; device errors in the status word). */
+size_t had_qkv_workspace_size(const had_shape* s, int Dm, int N, had_mode mode, const had_relpos_bias* bias);
+had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, int Dm, const had_relpos_bias* bias,
+                           int N, had_mode mode, void* V_out, void* workspace, size_t ws_bytes, void* stream);
+
 /* ---- host arrays in, host array out --------------------------------------
  * had_attention_host: had_attention on HOST memory, with the copies inside the
  * call.  Q, K, V: HOST [B][H][n][d] in s->in_dtype; O: HOST [B][H][n][d] in

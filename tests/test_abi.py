@@ -225,3 +225,32 @@ def test_binding_marshals_both_bias_kinds_and_host_arrays(L):
     # the host entry point takes contiguous CPU tensors only, checked before any call
     with pytest.raises(ValueError):
         m.had_attention_host(Q.transpose(2, 3), Q, Q)
+
+
+def test_qkv_prepare_validates_on_the_host(L):
+    # the fused projection takes bf16 at head dim 64 and a model width of a multiple of 64
+    import binarized_qk_sparse_b200 as m
+    P = ctypes.c_void_p
+    fake, ws = P(0x10000), P(0x20000)
+    big = 1 << 34
+
+    def qkv(shape, Dm=256, x=fake, w=fake, v=fake, mode=0, ws_bytes=big, wsp=ws, N=0):
+        return L.had_qkv_prepare(x, w, ctypes.byref(shape), Dm, None, N, mode, v, wsp, ws_bytes, None)
+
+    shp = _shape(m, B=2, H=3, n=197)
+    assert qkv(_shape(m, d=128)) == m.HAD_ERR_UNSUPPORTED
+    assert qkv(_shape(m, dtype=0)) == m.HAD_ERR_UNSUPPORTED      # fp32 X
+    assert qkv(shp, Dm=100) == m.HAD_ERR_INVALID
+    assert qkv(shp, Dm=0) == m.HAD_ERR_INVALID
+    assert qkv(shp, Dm=16384 + 64) == m.HAD_ERR_UNSUPPORTED
+    assert qkv(shp, x=P(0)) == m.HAD_ERR_INVALID
+    assert qkv(shp, w=P(0x10008)) == m.HAD_ERR_INVALID
+    assert qkv(shp, v=P(0)) == m.HAD_ERR_INVALID
+    assert qkv(shp, mode=7) == m.HAD_ERR_INVALID
+    assert qkv(shp, N=-1) == m.HAD_ERR_INVALID
+    assert qkv(shp, ws_bytes=1024) == m.HAD_ERR_INVALID
+    # its workspace holds the attention workspace plus X's token sums and the means
+    att = L.had_attention_workspace_size(ctypes.byref(shp), 0, 1, None)
+    q = L.had_qkv_workspace_size(ctypes.byref(shp), 256, 0, 1, None)
+    assert q >= att + 2 * 256 * 8 + 2 * 2 * 3 * 64 * 4
+    assert L.had_qkv_workspace_size(ctypes.byref(_shape(m, d=128)), 256, 0, 1, None) == 0
