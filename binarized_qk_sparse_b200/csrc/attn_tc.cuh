@@ -1788,6 +1788,14 @@ __global__ void __launch_bounds__(cta_threads(SPLIT), ctas_per_sm(D)) k_attn_tc(
         const int rc = kSplitF ? rc_split : r_cnt;
         n_merge = min(rc, kCap);
         if (rc > kCap) raise_status(a.status, kDevErrCapacity);
+        // the recorded keys in key order (the two threads of a row fill the slots in whatever
+        // order they reach them), so that the sums over the slots below are reproducible
+        for (int x = 1; x < n_merge; ++x) {
+          const uint32_t v = hist[x * kM + srow];
+          int y = x - 1;
+          for (; y >= 0 && hist[y * kM + srow] > v; --y) hist[(y + 1) * kM + srow] = hist[y * kM + srow];
+          hist[(y + 1) * kM + srow] = v;
+        }
         const int8_t* kb = a.kpm + (size_t)bh * a.n_pad * D;
         for (int x = 0; x < n_merge; ++x) {
           const int j = (int)hist[x * kM + srow];
