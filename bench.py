@@ -632,12 +632,166 @@ def run_gpu(args, rank, world, local_rank):
     return 0
 
 
+QKV_WORKLOAD = "deit_qkv"
+
+
+def run_qkv(args, rank, world, local_rank):
+    """DeiT's attention from its inputs' projection (B64 n197, model width 768, 12
+    heads, relative-position bias, dense uint8 A x int8 V): the fused path
+    (had_qkv_prepare: the projection with Q and K binarized in its epilogue, then the
+    fused attention) against the unfused one on the same box (a cuBLAS projection,
+    the copy into [B, H, n, d] heads, the library's prepare stage, the same attention).
+    One JSON line; the fused path is the line's value."""
+    import ctypes
+    import torch
+    import binarized_qk_sparse_b200 as had
+    from binarized_qk_sparse_b200 import _build
+    _build.build()
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    X, W, H, bw, _ = workloads.deit_qkv()
+    B, n, Dm = X.shape
+    d, N, mode = 64, 0, "u8i8"
+    Xd = torch.from_numpy(X).to(torch.bfloat16).to(dev)
+    Wd = torch.from_numpy(W).to(torch.bfloat16).to(dev)
+    bias = had.RelPosBias(torch.from_numpy(bw.table).to(dev), bw.gh, bw.gw, bw.prefix)
+    L = had.lib()
+    shp = had.had_shape(B, H, n, d, had.HAD_BF16, None)
+    bst = had._bias_c(bias)
+    bs = ctypes.byref(bst)
+    mcode = had._MODES[mode]
+    sp_stream = torch.cuda.Stream(device=dev)
+    sp = ctypes.c_void_p(sp_stream.cuda_stream)
+    ptr = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    ws_q = torch.empty(L.had_qkv_workspace_size(ctypes.byref(shp), Dm, N, mcode, bs), dtype=torch.uint8, device=dev)
+    ws_a = torch.empty(L.had_attention_workspace_size(ctypes.byref(shp), N, mcode, bs), dtype=torch.uint8, device=dev)
+    V = torch.empty((B, H, n, d), dtype=torch.bfloat16, device=dev)
+    O = torch.empty_like(V)
+    Pj = torch.empty((B * n, 3 * H * d), dtype=torch.bfloat16, device=dev)
+    Qh, Kh, Vh = (torch.empty((B, H, n, d), dtype=torch.bfloat16, device=dev) for _ in range(3))
+    O2 = torch.empty_like(V)
+
+    def ok(st, what):
+        if st:
+            raise had.HadError(st, what)
+
+    def fused_prep():
+        ok(L.had_qkv_prepare(ptr(Xd), ptr(Wd), ctypes.byref(shp), Dm, bs, N, mcode, ptr(V), ptr(ws_q), ws_q.numel(),
+                             sp), "had_qkv_prepare")
+
+    def fused_attend():
+        ok(L.had_attention_prepared(ptr(V), ctypes.byref(shp), bs, None, None, N, mcode, ptr(O), had._dtype_code(O),
+                                    ptr(ws_q), ws_q.numel(), sp), "had_attention_prepared")
+
+    def unfused_prep():
+        torch.matmul(Xd.view(B * n, Dm), Wd.t(), out=Pj)
+        Pv = Pj.view(B, n, 3, H, d)
+        for tns, k in ((Qh, 0), (Kh, 1), (Vh, 2)):
+            tns.copy_(Pv[:, :, k].permute(0, 2, 1, 3))
+        ok(L.had_attention_prepare(ptr(Qh), ptr(Kh), ptr(Vh), ctypes.byref(shp), bs, N, mcode, ptr(ws_a),
+                                   ws_a.numel(), sp), "had_attention_prepare")
+
+    def unfused_attend():
+        ok(L.had_attention_prepared(ptr(Vh), ctypes.byref(shp), bs, None, None, N, mcode, ptr(O2),
+                                    had._dtype_code(O2), ptr(ws_a), ws_a.numel(), sp), "had_attention_prepared")
+
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    probe_i8, _ = had.had_probe_mma_rate("i8", 40000)
+    clocks = ClockSampler(local_rank if "CUDA_VISIBLE_DEVICES" not in os.environ else 0)
+    clocks.start()
+    graphs = {}
+    with torch.cuda.stream(sp_stream):
+        for _ in range(max(3, args.warmup)):
+            fused_prep(); fused_attend(); unfused_prep(); unfused_attend()
+        sp_stream.synchronize()
+        assert had.had_get_device_status() == had.HAD_OK
+        for name, fn in (("fp", fused_prep), ("fa", fused_attend), ("up", unfused_prep), ("ua", unfused_attend)):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=sp_stream):
+                fn()
+            graphs[name] = g
+        for g in graphs.values():
+            g.replay()
+        sp_stream.synchronize()
+
+        def timed(gp, ga):
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+                   torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+            torch.cuda.synchronize()
+            w0 = time.time()
+            for s_ in range(args.steps):
+                flush.zero_()
+                ev[s_][0].record(sp_stream)
+                gp.replay()
+                ev[s_][1].record(sp_stream)
+                ga.replay()
+                ev[s_][2].record(sp_stream)
+            torch.cuda.synchronize()
+            w1 = time.time()
+            return ([e[0].elapsed_time(e[2]) for e in ev], [e[0].elapsed_time(e[1]) for e in ev],
+                    [e[1].elapsed_time(e[2]) for e in ev], w0, w1)
+
+        f_step, f_prep, f_att, wall0, wall1 = timed(graphs["fp"], graphs["fa"])
+        u_step, u_prep, u_att, _, _ = timed(graphs["up"], graphs["ua"])
+        # e2e: X from pinned host memory, the fused path, O back, every step
+        hX = Xd.cpu().pin_memory()
+        hO = torch.empty_like(O, device="cpu").pin_memory()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e2e_steps = max(3, min(args.steps, 30))
+        for s_ in range(e2e_steps + 2):
+            if s_ == 2:
+                e0.record(sp_stream)
+            Xd.copy_(hX, non_blocking=True)
+            graphs["fp"].replay()
+            graphs["fa"].replay()
+            hO.copy_(O, non_blocking=True)
+        e1.record(sp_stream)
+        sp_stream.synchronize()
+    clk = clocks.stop(wall0, wall1)
+    diff = (O.float() - O2.float()).abs().max().item()  # the two paths, for the record
+    if rank != 0:
+        return 0
+    peaks, peak_kind = _peaks()
+    queries = B * H * n
+    f_ms = max_over_ranks(sum(f_step), None) / args.steps
+    att_ms = sum(f_att) / args.steps
+    flop = 2.0 * B * n * Dm * 3 * H * d
+    i8 = max(probe_i8, INT8_PER_BF16 * peaks["bf16_tflops"])
+    kb = kernel_bytes_per_token(mode, 2, 2, d) * queries + bw.table.nbytes
+    roof = north_star_roofline(kb, score_tensor_ops(B * H * n * n, d), att_ms, peaks["hbm_gbs"], i8)
+    roof.update({"traffic": None, "kernel": "k_attn_tc (fused score/top-N/softmax/A.V)", "avg_launch_ms": att_ms})
+    line = {
+        "metric": METRIC, "value": whole_job_rate(queries, world, args.steps, sum(f_step)), "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": f_ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8i8", "data": "synthetic",
+        "config": {"workload": f"deit_qkv_b{B}_h{H}_n{n}_dm{Dm}_dense_{mode}", "B": B, "H": H, "n": n, "d": d,
+                   "Dm": Dm, "N": N, "mode": mode, "in_dtype": "bf16", "seed": 9,
+                   "bias": "relpos 27x27/head, prefix 1", "seqlens": None,
+                   "l2": "flushed between timed steps (256 MiB write)"},
+        "launch": "each step replays CUDA graphs of the two library calls (projection + prepare, attend)",
+        "qkv": {"fused_prep_ms": sum(f_prep) / args.steps, "attn_ms": att_ms,
+                "unfused_ms_per_step": sum(u_step) / args.steps, "unfused_prep_ms": sum(u_prep) / args.steps,
+                "unfused_attn_ms": sum(u_att) / args.steps,
+                "projection_gflop": flop / 1e9,
+                "fused_prep_tflops": flop / (sum(f_prep) / args.steps * 1e-3) / 1e12,
+                "max_abs_diff_fused_vs_unfused_O": diff,
+                "unfused": "cuBLAS bf16 projection (torch.matmul), copy into [B,H,n,d] heads, had_attention_prepare"},
+        "roofline": roof,
+        "e2e": {"value": queries / (e0.elapsed_time(e1) / e2e_steps * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": X.size * 2, "d2h_bytes_per_step": O.numel() * 2},
+        "gpu_launches": args.steps * 9,  # the fused loop: k_xsum, k_mu, k_qkv_tc, 2 bias-table, 3 V-quantization kernels, k_attn_tc
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=80)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="stress_topn", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="stress_topn", choices=sorted(WORKLOADS) + [QKV_WORKLOAD])
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batch", type=int, default=0, help="run the first B sequences only (profiler captures)")
@@ -648,6 +802,11 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.workload == QKV_WORKLOAD:
+        if world > 1:
+            import torch
+            torch.cuda.set_device(local_rank)
+        return run_qkv(args, rank, 1, local_rank)
     if world > 1:
         import datetime
         import torch

@@ -232,7 +232,8 @@ __global__ void k_untranspose_vq(const int8_t* vqT, int BH, int n, int d, int n_
 had_status launch_prep(const had_shape* s, const void* X0, const void* X1, const void* X2, int first, int ntens,
                        double* sums, float* amax, const float* mu_in0, float* mu_out0, uint32_t* bits0,
                        int8_t* pm0, uint32_t* bits1, int8_t* pm1, int8_t* vqT, float* vscale, cudaStream_t st,
-                       unsigned* status, int vbits = 8, bool pm_e4m3 = false) {
+                       unsigned* status, int vbits = 8, bool pm_e4m3 = false,
+                       const float* v_amax = nullptr) {
   Dims d = dims_of(s);
   PrepArgs pa{};
   pa.X[0] = X0; pa.X[1] = X1; pa.X[2] = X2;
@@ -240,7 +241,8 @@ had_status launch_prep(const had_shape* s, const void* X0, const void* X1, const
   pa.B = d.B; pa.H = d.H; pa.n = d.n; pa.nchunks = d.nchunks;
   pa.seqlens = s->seqlens; pa.sums = sums; pa.amax = amax; pa.status = status;
   dim3 grid(d.nchunks, d.BH, ntens);
-  const bool need_stats = !(mu_in0 && first == 0 && ntens == 1);
+  // no statistics pass when the caller gives Q's mean (bits of Q alone) or V's absmax (V alone)
+  const bool need_stats = !(mu_in0 && first == 0 && ntens == 1) && !(v_amax && first == 2 && ntens == 1);
   const bool bf = s->in_dtype == HAD_BF16;
   if (need_stats) {
     if (d.d == 32) bf ? k_stats<__nv_bfloat16, 32><<<grid, kPrepThreads, 0, st>>>(pa) : k_stats<float, 32><<<grid, kPrepThreads, 0, st>>>(pa);
@@ -258,7 +260,9 @@ had_status launch_prep(const had_shape* s, const void* X0, const void* X1, const
   ka.X[0] = X0; ka.X[1] = X1; ka.X[2] = X2;
   ka.ntens = ntens; ka.first_tensor = first;
   ka.B = d.B; ka.H = d.H; ka.n = d.n; ka.nchunks = d.nchunks; ka.n_pad = d.n_pad;
-  ka.seqlens = s->seqlens; ka.sums = sums; ka.amax = amax;
+  ka.seqlens = s->seqlens; ka.sums = sums;
+  ka.amax = need_stats ? amax : v_amax;
+  ka.amax_ld = need_stats ? d.nchunks * d.d : d.d;
   ka.mu_in[0] = mu_in0; ka.mu_in[1] = nullptr;
   ka.mu_out[0] = mu_out0; ka.mu_out[1] = nullptr;
   ka.bits[0] = bits0; ka.bits[1] = bits1;
@@ -558,10 +562,10 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
 }
 
 // Workspace of the fused projection: the attention workspace (so that
-// had_attention_prepared can run on it), then X's token partial sums and the
-// means of Q and K.
+// had_attention_prepared can run on it), then X's token partial sums, X's token
+// means, the means of Q and K, and V's column absmax per head.
 struct QkvWs {
-  size_t xpart, mu, total;
+  size_t xpart, xbar, mu, vamax, total;
   int nch;
 };
 
@@ -570,7 +574,9 @@ QkvWs qkv_ws_layout(const had_shape* s, int Dm, int vbits, const had_relpos_bias
   size_t off = align_up(ws_layout(s, vbits, bias).total);
   q.nch = (s->n + qkv::kXsumChunk - 1) / qkv::kXsumChunk;
   q.xpart = off; off += align_up((size_t)s->B * q.nch * Dm * 8);
-  q.mu = off; off += align_up((size_t)2 * s->B * s->H * 64 * 4);
+  q.xbar = off; off += align_up((size_t)s->B * Dm * 8);
+  q.mu = off; off += align_up((size_t)qkv::kMuSplit * 2 * s->B * s->H * 64 * 8);
+  q.vamax = off; off += align_up((size_t)s->B * s->H * 64 * 4);
   q.total = off;
   return q;
 }
@@ -886,13 +892,19 @@ had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, 
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
   const __nv_bfloat16* Wb = static_cast<const __nv_bfloat16*>(Wqkv);
   double* xpart = reinterpret_cast<double*>(ws + q.xpart);
-  float* mu = reinterpret_cast<float*>(ws + q.mu);
+  double* mupart = reinterpret_cast<double*>(ws + q.mu);
   // the means of Q and K from X's token means
-  qkv::k_xsum<<<dim3((Dm + qkv::kXsumThreads - 1) / qkv::kXsumThreads, q.nch, d.B), qkv::kXsumThreads, 0, st>>>(
+  qkv::k_xsum<<<dim3((Dm / 8 + qkv::kXsumThreads - 1) / qkv::kXsumThreads, q.nch, d.B),
+                  qkv::kXsumThreads * qkv::kXsumGroups, 0, st>>>(
       Xb, d.n, Dm, s->seqlens, q.nch, xpart);
   if ((r = check_launch("k_xsum")) != HAD_OK) return r;
-  qkv::k_mu<<<dim3((2 * d.H * 64 + qkv::kMuWarps - 1) / qkv::kMuWarps, d.B), qkv::kMuWarps * 32, 0, st>>>(
-      Wb, xpart, q.nch, d.n, d.B, d.H, Dm, s->seqlens, status, mu);
+  double* xbar = reinterpret_cast<double*>(ws + q.xbar);
+  uint32_t* vamax = reinterpret_cast<uint32_t*>(ws + q.vamax);
+  qkv::k_xmean<<<dim3((Dm + qkv::kXsumThreads - 1) / qkv::kXsumThreads, d.B), qkv::kXsumThreads, 0, st>>>(
+      xpart, q.nch, d.n, Dm, d.H, s->seqlens, status, xbar, vamax);
+  if ((r = check_launch("k_xmean")) != HAD_OK) return r;
+  qkv::k_mu<<<dim3((2 * d.H * 64 + qkv::kMuO - 1) / qkv::kMuO, (d.B + qkv::kMuB - 1) / qkv::kMuB, qkv::kMuSplit), qkv::kMuThreads, 0,
+             st>>>(Wb, xbar, d.B, d.H, Dm, mupart);
   if ((r = check_launch("k_mu")) != HAD_OK) return r;
   // the projection, binarized in its epilogue, into the attention workspace
   qkv::QkvArgs qa;
@@ -905,11 +917,12 @@ had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, 
     return r;
   qa.B = d.B; qa.H = d.H; qa.n = d.n; qa.n_pad = d.n_pad; qa.Dm = Dm;
   qa.seqlens = s->seqlens;
-  qa.mu = mu;
+  qa.mupart = mupart;
   qa.qbits = reinterpret_cast<uint32_t*>(ws + w.qbits);
   qa.kpm = reinterpret_cast<int8_t*>(ws + w.kpm);
   qa.k_e4m3 = select_kind(s, bias, N) == SEL_TOPN_FLOAT ? 1 : 0;  // the fp8 score path's +-1 encoding
   qa.V = static_cast<__nv_bfloat16*>(V_out);
+  qa.vamax = vbits != 0 ? vamax : nullptr;
   qa.status = status;
   {
     static std::mutex smu;
@@ -924,16 +937,19 @@ had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, 
       configured[dev] = true;
     }
   }
-  qkv::k_qkv_tc<<<dim3((d.n + qkv::kM - 1) / qkv::kM, d.B, 3 * d.H), qkv::kThreads, qkv::QkvSmem::kTotal, st>>>(qa);
+  qkv::k_qkv_tc<<<dim3((d.n + qkv::kM - 1) / qkv::kM, d.B, (3 * d.H + qkv::kNB - 1) / qkv::kNB), qkv::kThreads,
+                   qkv::QkvSmem::kTotal, st>>>(qa);
   if ((r = check_launch("k_qkv_tc")) != HAD_OK) return r;
-  // the bias tables and, in the uint8 modes, the quantized V^T, as the attention's prepare stage makes them
+  // the bias tables and, in the uint8 modes, the quantized V^T (scales from the epilogue's absmax), as the
+  // attention's prepare stage makes them
   if (bias && bias->table &&
       (r = build_bias_tables(s, bias, ws + w.bminmax, ws + w.bext, ws + w.expb, st)) != HAD_OK)
     return r;
   if (vbits != 0) {
     r = launch_prep(s, nullptr, nullptr, V_out, 2, 1, reinterpret_cast<double*>(ws + w.sums),
                     reinterpret_cast<float*>(ws + w.amax), nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
-                    reinterpret_cast<int8_t*>(ws + w.vqT), reinterpret_cast<float*>(ws + w.vscale), st, status, vbits);
+                    reinterpret_cast<int8_t*>(ws + w.vqT), reinterpret_cast<float*>(ws + w.vscale), st, status, vbits,
+                    false, reinterpret_cast<const float*>(vamax));
     if (r != HAD_OK) return r;
   }
   return HAD_OK;

@@ -147,7 +147,8 @@ struct PackArgs {
   int B, H, n, nchunks, n_pad;
   const int32_t* seqlens;
   const double* sums;     // from k_stats (unused when mu_in != nullptr)
-  const float* amax;
+  const float* amax;      // V's column absmax of head bh at amax[bh * amax_ld + c]
+  int amax_ld;
   const float* mu_in[2];  // optional caller means per tensor 0/1
   float* mu_out[2];       // optional mean outputs per tensor 0/1
   uint32_t* bits[2];      // [BH][n][D/32] per tensor 0/1 (or null)
@@ -187,7 +188,7 @@ __global__ void __launch_bounds__(kPrepThreads) k_pack(const PackArgs a) {
       stat[c] = mu;
       if (chunk == 0 && a.mu_out[tz]) a.mu_out[tz][(size_t)bh * kD + c] = mu;
     } else {
-      const float m = a.amax[(size_t)bh * a.nchunks * kD + c];  // the absmax k_stats_final left in chunk 0
+      const float m = a.amax[(size_t)bh * a.amax_ld + c];  // k_stats_final's (chunk 0 slot) or the caller's
       const float qmax = a.v_bits == 4 ? 7.0f : 127.0f;
       float s = (m > 0.0f) ? __fdiv_rn(m, qmax) : 1.0f;
       stat[c] = s;

@@ -8,14 +8,18 @@
 // map's outputs is the map of the mean input, so
 //   mu_Q[b][h][c] = (1/L_b) sum_{i<L_b} (X_i W_Q^T)[h*d + c] = xbar_b . W_Q[h*d + c],
 // with xbar_b the mean of the valid tokens of X (k_xsum: fp64 token sums per
-// 256-token chunk; k_mu: one warp per output channel, fp64 dot product, one
-// rounding to fp32).  Then k_qkv_tc runs the projection on the tensor cores and
+// 32-token chunk; k_xmean: the means; k_mu: a tiled fp64 product of the means
+// with W in feature slices, added in order and rounded once to fp32 by k_qkv_tc).  Then k_qkv_tc runs the projection on the tensor cores and
 // compares each fp32 result with its mean in the epilogue:
 //   - Q columns: the 64 sign bits of a token (bit 1 = below the mean), in the
 //     attention workspace's packed layout;
 //   - K columns: the +-1 row of a token (int8, or e4m3 for the fp8 score path),
 //     rows past L (and up to n_pad) +1;
-//   - V columns: the bf16 row of V, the attention's V input.
+//   - V columns: the bf16 row of V, the attention's V input, and in the uint8
+//     modes V's column absmax per head (atomic maxima), from which the
+//     quantization of V takes its scales without a statistics pass.
+// A CTA takes 128 tokens and 256 output channels (four heads' column blocks): one
+// M128 N256 K16 MMA per K-step, so that each X tile serves four blocks.
 #pragma once
 
 #include <cuda.h>
@@ -29,81 +33,196 @@ namespace qkv {
 
 using namespace had::sm100;
 
-constexpr int kXsumChunk = 256;    // tokens per partial sum of X
-constexpr int kXsumThreads = 128;  // features per k_xsum CTA
-constexpr int kMuWarps = 8;        // output channels per k_mu CTA
+constexpr int kXsumChunk = 32;     // tokens per partial sum of X
+constexpr int kXsumThreads = 128;  // k_xsum: feature threads (8 features each) per token group; k_xmean: one feature per thread
+constexpr int kMuB = 16, kMuO = 32, kMuK = 32;  // k_mu tile: batches x output channels x features
 
-// Token sums of X over the valid tokens of each 256-token chunk: part[b][ch][k], fp64.
-__global__ void __launch_bounds__(kXsumThreads) k_xsum(const __nv_bfloat16* __restrict__ X, int n, int Dm,
-                                                       const int32_t* seqlens, int nch, double* __restrict__ part) {
-  const int k = blockIdx.x * kXsumThreads + threadIdx.x, ch = blockIdx.y, b = blockIdx.z;
-  if (k >= Dm) return;
+// Token sums of X over the valid tokens of each 32-token chunk: part[b][ch][k], fp64.
+// Thread (g, f) of a CTA adds 8 adjacent features over the g-th 8 tokens of the
+// chunk (eight 16-byte loads issued together); the four groups' sums are then
+// added in group order.
+constexpr int kXsumGroups = kXsumChunk / 8;
+__global__ void __launch_bounds__(kXsumThreads * kXsumGroups) k_xsum(const __nv_bfloat16* __restrict__ X, int n,
+                                                                     int Dm, const int32_t* seqlens, int nch,
+                                                                     double* __restrict__ part) {
+  __shared__ double red[kXsumGroups - 1][8][kXsumThreads];
+  const int ft = threadIdx.x % kXsumThreads, tg = threadIdx.x / kXsumThreads;
+  const int k0 = (blockIdx.x * kXsumThreads + ft) * 8, ch = blockIdx.y, b = blockIdx.z;
+  const bool act = k0 < Dm;
   const int L = valid_len(seqlens, b, n, nullptr);
-  const int i0 = ch * kXsumChunk, i1 = min(i0 + kXsumChunk, L);
-  double s = 0.0;
-  for (int i = i0; i < i1; ++i) s += (double)__bfloat162float(X[((size_t)b * n + i) * Dm + k]);
-  part[((size_t)b * nch + ch) * Dm + k] = s;
+  const int i0 = ch * kXsumChunk + tg * 8, i1 = min(i0 + 8, L);
+  double s[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) s[u] = 0.0;
+  if (act && i0 < i1) {
+    // rows past the group's end re-read its last row and are zeroed after the load
+    uint4 x[8];
+#pragma unroll
+    for (int t = 0; t < 8; ++t)
+      x[t] = __ldg(reinterpret_cast<const uint4*>(X + ((size_t)b * n + min(i0 + t, i1 - 1)) * Dm + k0));
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+      if (i0 + t >= i1) x[t] = make_uint4(0u, 0u, 0u, 0u);
+      const uint32_t w[4] = {x[t].x, x[t].y, x[t].z, x[t].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        s[2 * u] += (double)__uint_as_float(w[u] << 16);
+        s[2 * u + 1] += (double)__uint_as_float(w[u] & 0xFFFF0000u);
+      }
+    }
+  }
+  if (tg > 0) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) red[tg - 1][u][ft] = s[u];
+  }
+  __syncthreads();
+  if (tg == 0 && act) {
+#pragma unroll
+    for (int g = 0; g < kXsumGroups - 1; ++g)
+#pragma unroll
+      for (int u = 0; u < 8; ++u) s[u] += red[g][u][ft];
+    double* dst = part + ((size_t)b * nch + ch) * Dm + k0;
+#pragma unroll
+    for (int u = 0; u < 8; u += 2) *reinterpret_cast<double2*>(dst + u) = make_double2(s[u], s[u + 1]);
+  }
 }
 
-// mu[t][b][h][c] for t in {Q, K}: one warp per output channel o = t*H*64 + h*64 + c,
-// the fp64 dot product of the token sum of X with W's row o, divided by L.
-__global__ void __launch_bounds__(kMuWarps * 32) k_mu(const __nv_bfloat16* __restrict__ W,
-                                                      const double* __restrict__ part, int nch, int n, int B, int H,
-                                                      int Dm, const int32_t* seqlens, unsigned* status,
-                                                      float* __restrict__ mu) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int o = blockIdx.x * kMuWarps + warp, b = blockIdx.y;
-  if (o >= 2 * H * 64) return;
+// The token means of X: xbar[b][k] = (chunk sums added in order) / L_b, fp64.
+// Also clears V's column absmax of batch b (H*64 words), which the projection's
+// epilogue raises with atomic maxima.
+__global__ void __launch_bounds__(kXsumThreads) k_xmean(const double* __restrict__ part, int nch, int n, int Dm,
+                                                        int H, const int32_t* seqlens, unsigned* status,
+                                                        double* __restrict__ xbar, uint32_t* __restrict__ vamax) {
+  const int k = blockIdx.x * kXsumThreads + threadIdx.x, b = blockIdx.y;
+  if (k >= Dm) return;
+  for (int e = k; e < H * 64; e += Dm) vamax[(size_t)b * H * 64 + e] = 0u;
   const int L = valid_len(seqlens, b, n, status);
   const int nv = (L + kXsumChunk - 1) / kXsumChunk;
-  double acc = 0.0;
-  for (int k = lane; k < Dm; k += 32) {
-    double xs = 0.0;
-    for (int c = 0; c < nv; ++c) xs += part[((size_t)b * nch + c) * Dm + k];
-    acc += xs * (double)__bfloat162float(W[(size_t)o * Dm + k]);
+  double v = 0.0;
+  for (int c = 0; c < nv; ++c) v += part[((size_t)b * nch + c) * Dm + k];
+  xbar[(size_t)b * Dm + k] = L > 0 ? v / (double)L : 0.0;
+}
+
+// Partial dot products of the means with W: mupart[z][t][b][h][c] = sum over the
+// z-th of kMuSplit feature slices of xbar[b][k] W[o][k], o = t*H*64 + h*64 + c, in
+// fp64.  k_qkv_tc adds the kMuSplit partials in slice order and rounds once to
+// fp32.  A CTA of 128 threads computes 16 batches x 32 output channels of one
+// slice, two batches x two channels per thread; the mean tile and the W tile
+// (converted to fp64 once, as it is staged) of kMuK features sit in shared memory
+// while the next tile is already in registers.
+constexpr int kMuThreads = 128;
+constexpr int kMuSplit = 8;
+__global__ void __launch_bounds__(kMuThreads) k_mu(const __nv_bfloat16* __restrict__ W,
+                                                   const double* __restrict__ xbar, int B, int H, int Dm,
+                                                   double* __restrict__ mupart) {
+  __shared__ __align__(16) double xs[kMuB][kMuK + 1];
+  __shared__ __align__(16) double ws[kMuO][kMuK + 1];
+  // thread (ty, tx): channels tx and tx + 16, batches ty and ty + 8 (rows 16 apart: no bank conflicts)
+  const int tid = threadIdx.x, tx = tid % (kMuO / 2), ty = tid / (kMuO / 2);
+  const int o0 = blockIdx.x * kMuO, b0 = blockIdx.y * kMuB;
+  const int no = 2 * H * 64;
+  const int slice = Dm / kMuSplit;  // a multiple of 8 (Dm is a multiple of 64)
+  const int kbeg = blockIdx.z * slice, kend = kbeg + slice;
+  constexpr int kWPieces = kMuO * kMuK / 8 / kMuThreads;  // 8-feature pieces of W per thread and tile
+  constexpr int kXPairs = kMuB * kMuK / 2 / kMuThreads;   // feature pairs of the means per thread and tile
+  uint4 wr[kWPieces];
+  double2 xr[kXPairs];
+  auto fetch = [&](int k0) {
+#pragma unroll
+    for (int j = 0; j < kWPieces; ++j) {
+      const int e = tid + kMuThreads * j, row = e / (kMuK / 8), kk = k0 + (e % (kMuK / 8)) * 8;
+      wr[j] = (o0 + row < no && kk < kend) ? __ldg(reinterpret_cast<const uint4*>(W + (size_t)(o0 + row) * Dm + kk))
+                                         : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int j = 0; j < kXPairs; ++j) {
+      const int e = tid + kMuThreads * j, br = e / (kMuK / 2), kx = k0 + (e % (kMuK / 2)) * 2;
+      xr[j] = (b0 + br < B && kx < kend) ? *reinterpret_cast<const double2*>(xbar + (size_t)(b0 + br) * Dm + kx)
+                                       : make_double2(0.0, 0.0);
+    }
+  };
+  double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
+  fetch(kbeg);
+  for (int k0 = kbeg; k0 < kend; k0 += kMuK) {
+#pragma unroll
+    for (int j = 0; j < kWPieces; ++j) {
+      const int e = tid + kMuThreads * j, row = e / (kMuK / 8), c = (e % (kMuK / 8)) * 8;
+      const uint32_t w[4] = {wr[j].x, wr[j].y, wr[j].z, wr[j].w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        ws[row][c + 2 * u] = (double)__uint_as_float(w[u] << 16);
+        ws[row][c + 2 * u + 1] = (double)__uint_as_float(w[u] & 0xFFFF0000u);
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kXPairs; ++j) {
+      const int e = tid + kMuThreads * j, br = e / (kMuK / 2), cx = (e % (kMuK / 2)) * 2;
+      xs[br][cx] = xr[j].x;
+      xs[br][cx + 1] = xr[j].y;
+    }
+    __syncthreads();
+    if (k0 + kMuK < kend) fetch(k0 + kMuK);
+#pragma unroll 8
+    for (int kk = 0; kk < kMuK; ++kk) {
+      const double x0 = xs[ty][kk], x1 = xs[ty + kMuB / 2][kk];
+      const double w0 = ws[tx][kk], w1 = ws[tx + kMuO / 2][kk];
+      acc[0][0] = fma(x0, w0, acc[0][0]);
+      acc[0][1] = fma(x0, w1, acc[0][1]);
+      acc[1][0] = fma(x1, w0, acc[1][0]);
+      acc[1][1] = fma(x1, w1, acc[1][1]);
+    }
+    __syncthreads();
   }
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) {
-    const int t = o / (H * 64), r = o - t * H * 64;  // r = h * 64 + c
-    mu[((size_t)t * B + b) * H * 64 + r] = (L > 0) ? (float)(acc / (double)L) : 0.0f;
-  }
+#pragma unroll
+  for (int ib = 0; ib < 2; ++ib)
+#pragma unroll
+    for (int ic = 0; ic < 2; ++ic) {
+      const int b = b0 + ty + (kMuB / 2) * ib, o = o0 + tx + (kMuO / 2) * ic;
+      if (b < B && o < no) {
+        const int t = o / (H * 64), r = o - t * H * 64;  // r = h * 64 + c
+        mupart[(((size_t)blockIdx.z * 2 + t) * B + b) * H * 64 + r] = acc[ib][ic];
+      }
+    }
 }
 
 // ---------------------------------------------------------------------------- the fused projection
 
 constexpr int kM = 128;        // tokens per CTA (TMEM lanes)
-constexpr int kN = 64;         // output channels per CTA: one head's d = 64 channels of Q, K or V
+constexpr int kHd = 64;        // a head's channels: one column block of Q, K or V
+constexpr int kNB = 4;         // column blocks per CTA
+constexpr int kN = kHd * kNB;  // output channels per CTA (one M128 N256 MMA per K-step)
 constexpr int kK = 64;         // features per panel (128 bytes of bf16: one 128-byte swizzle row)
-constexpr int kStages = 4;
+constexpr int kStages = 2;     // 2 x 48 KB: two CTAs per SM, so one's epilogue overlaps the other's main loop
 constexpr int kThreads = 192;  // warps 0-3: epilogue (TMEM lane quadrants); 4: MMA; 5: TMA
 constexpr int kMmaWarp = 4, kProdWarp = 5;
-constexpr uint32_t kTmemCols = 64;
+constexpr uint32_t kTmemCols = kN;
 constexpr long long kWaitCycles = 2000000000LL;  // bound of a pipeline wait: about one second
 
 struct QkvArgs {
   CUtensorMap tm_x;   // X [B*n][Dm] bf16, box {64, 128}, 128-byte swizzle
-  CUtensorMap tm_w;   // W [3*H*64][Dm] bf16, box {64, 64}, 128-byte swizzle
+  CUtensorMap tm_w;   // W [3*H*64][Dm] bf16, box {64, 256}, 128-byte swizzle
   int B, H, n, n_pad, Dm;
   const int32_t* seqlens;
-  const float* mu;    // [2][B][H][64]: the means of Q, then of K
+  const double* mupart;  // [kMuSplit][2][B][H][64]: partial means of Q, then of K (k_mu)
   uint32_t* qbits;    // [B*H][n][2]
   int8_t* kpm;        // [B*H][n_pad][64] +-1 rows of K
   int k_e4m3;         // the +-1 rows as e4m3 (0x38 / 0xB8) instead of int8 (0x01 / 0xFF)
   __nv_bfloat16* V;   // [B][H][n][64]
+  uint32_t* vamax;    // [B*H][64] float bits: V's column absmax over the valid tokens (or null)
   unsigned* status;
 };
 
 struct QkvSmem {
   static constexpr int kA = 0;                          // kStages x [128 tokens][64 features] bf16
-  static constexpr int kB = kA + kStages * kM * kK * 2;  // kStages x [64 channels][64 features] bf16
+  static constexpr int kB = kA + kStages * kM * kK * 2;  // kStages x [256 channels][64 features] bf16
   static constexpr int kBar = kB + kStages * kN * kK * 2;
   static constexpr int kNumBars = 2 * kStages + 2;       // full, empty, accumulator done, final
-  static constexpr int kMu = kBar + kNumBars * 8;        // 64 means
+  static constexpr int kMu = kBar + kNumBars * 8;        // the 256 columns' means
   static constexpr int kMisc = kMu + kN * 4;             // [0] TMEM base, [1] abort
   static constexpr int kTotal = kMisc + 16 + 1024;       // + alignment slack
 };
 
-__global__ void __launch_bounds__(kThreads, 1) k_qkv_tc(const __grid_constant__ QkvArgs a) {
+__global__ void __launch_bounds__(kThreads, 2) k_qkv_tc(const __grid_constant__ QkvArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   uint64_t* bars = reinterpret_cast<uint64_t*>(sm + QkvSmem::kBar);
@@ -116,8 +235,8 @@ __global__ void __launch_bounds__(kThreads, 1) k_qkv_tc(const __grid_constant__ 
   volatile uint32_t* abort_flag = misc + 1;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int m0 = blockIdx.x * kM, b = blockIdx.y, j = blockIdx.z;
-  const int t = j / a.H, h = j - t * a.H;  // tensor (0 Q, 1 K, 2 V) and head of this CTA's 64 columns
+  const int m0 = blockIdx.x * kM, b = blockIdx.y, j0 = blockIdx.z * kNB;  // first column block
+  const int nblk = 3 * a.H;  // column blocks of Q, K and V: block j is tensor j / H, head j % H
   const int L = valid_len(a.seqlens, b, a.n, a.status);
   const int npanel = a.Dm / kK;
 
@@ -134,7 +253,13 @@ __global__ void __launch_bounds__(kThreads, 1) k_qkv_tc(const __grid_constant__ 
     prefetch_tensormap(&a.tm_x);
     prefetch_tensormap(&a.tm_w);
   }
-  if (tid < kN) smu[tid] = (t < 2) ? a.mu[(((size_t)t * a.B + b) * a.H + h) * kN + tid] : 0.0f;
+  for (int e = tid; e < kN; e += kThreads) {
+    const int j = j0 + e / kHd, t = j / a.H, h = j - t * a.H;
+    double m = 0.0;
+    if (j < nblk && t < 2)
+      for (int z = 0; z < kMuSplit; ++z) m += a.mupart[((((size_t)z * 2 + t) * a.B + b) * a.H + h) * kHd + (e % kHd)];
+    smu[e] = (float)m;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -158,11 +283,11 @@ __global__ void __launch_bounds__(kThreads, 1) k_qkv_tc(const __grid_constant__ 
       if (*abort_flag) break;
       mbar_arrive_expect_tx(&full[st], (uint32_t)(kM + kN) * kK * 2);
       tma_load_2d(sm + QkvSmem::kA + st * kM * kK * 2, &a.tm_x, p * kK, b * a.n + m0, &full[st]);
-      tma_load_2d(sm + QkvSmem::kB + st * kN * kK * 2, &a.tm_w, p * kK, j * kN, &full[st]);
+      tma_load_2d(sm + QkvSmem::kB + st * kN * kK * 2, &a.tm_w, p * kK, j0 * kHd, &full[st]);
       par[st] = (p / kStages) & 1;
     }
   } else if (warp == kMmaWarp && lane == 0) {
-    // D[128 tokens][64 channels] += X panel [128][64] x W panel [64][64]^T: 4 K-steps of 16
+    // D[128 tokens][256 channels] += X panel [128][64] x W panel [256][64]^T: 4 K-steps of 16
     const uint32_t idesc = idesc_bf16(kM, kN, false);
     for (int p = 0; p < npanel; ++p) {
       const int st = p % kStages;
@@ -178,47 +303,78 @@ __global__ void __launch_bounds__(kThreads, 1) k_qkv_tc(const __grid_constant__ 
     }
     mma_commit(acc_bar);
   } else if (warp < 4) {
-    // epilogue: thread (warp w, lane l) owns token m0 + 32 w + l, TMEM lane 32 w + l
+    // epilogue: thread (warp w, lane l) owns token m0 + 32 w + l, TMEM lane 32 w + l, and
+    // takes the CTA's column blocks one after the other
     const bool ok = __all_sync(0xffffffffu, bounded_wait(acc_bar, 0));
     tc_fence_after();
-    uint32_t v0[32], v1[32];
     const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
-    tmem_ld32(tl, v0);
-    tmem_ld32(tl + 32, v1);
-    tmem_wait_ld();
     const int r = m0 + 32 * warp + lane;
-    const size_t bh = (size_t)b * a.H + h;
-    if (ok && t < 2) {
-      uint32_t w0 = 0u, w1 = 0u;
-      if (r < L) {
+    for (int jb = 0; jb < kNB; ++jb) {
+      const int j = j0 + jb;
+      if (j >= nblk) break;  // uniform over the CTA
+      const int t = j / a.H, h = j - t * a.H;
+      uint32_t v0[32], v1[32];
+      tmem_ld32(tl + jb * kHd, v0);
+      tmem_ld32(tl + jb * kHd + 32, v1);
+      tmem_wait_ld();
+      const float* mu = smu + jb * kHd;
+      const size_t bh = (size_t)b * a.H + h;
+      if (ok && t < 2) {
+        uint32_t w0 = 0u, w1 = 0u;
+        if (r < L) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          w0 |= (__uint_as_float(v0[c]) < smu[c] ? 1u : 0u) << c;
-          w1 |= (__uint_as_float(v1[c]) < smu[32 + c] ? 1u : 0u) << c;
+          for (int c = 0; c < 32; ++c) {
+            w0 |= (__uint_as_float(v0[c]) < mu[c] ? 1u : 0u) << c;
+            w1 |= (__uint_as_float(v1[c]) < mu[32 + c] ? 1u : 0u) << c;
+          }
         }
-      }
-      if (t == 0) {
-        if (r < a.n) *reinterpret_cast<uint2*>(a.qbits + (bh * a.n + r) * 2) = make_uint2(w0, w1);
-      } else if (r < a.n_pad) {
-        uint4* dst = reinterpret_cast<uint4*>(a.kpm + (bh * a.n_pad + r) * kN);
-        const bool e4 = a.k_e4m3 != 0;
+        if (t == 0) {
+          if (r < a.n) *reinterpret_cast<uint2*>(a.qbits + (bh * a.n + r) * 2) = make_uint2(w0, w1);
+        } else if (r < a.n_pad) {
+          uint4* dst = reinterpret_cast<uint4*>(a.kpm + (bh * a.n_pad + r) * kHd);
+          const bool e4 = a.k_e4m3 != 0;
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint32_t f = (q < 2 ? w0 : w1) >> ((q & 1) * 16);
-          dst[q] = make_uint4(expand_nibble_pm(f & 15u, e4), expand_nibble_pm((f >> 4) & 15u, e4),
-                              expand_nibble_pm((f >> 8) & 15u, e4), expand_nibble_pm((f >> 12) & 15u, e4));
+          for (int q = 0; q < 4; ++q) {
+            const uint32_t f = (q < 2 ? w0 : w1) >> ((q & 1) * 16);
+            dst[q] = make_uint4(expand_nibble_pm(f & 15u, e4), expand_nibble_pm((f >> 4) & 15u, e4),
+                                expand_nibble_pm((f >> 8) & 15u, e4), expand_nibble_pm((f >> 12) & 15u, e4));
+          }
         }
-      }
-    } else if (ok && r < a.n) {
-      // V: the bf16 row
-      uint4* dst = reinterpret_cast<uint4*>(a.V + (bh * a.n + r) * kN);
+      } else if (ok) {
+        // V: the bf16 row
+        uint32_t pk[32];
 #pragma unroll
-      for (int q = 0; q < 8; ++q) {
-        const uint32_t* src = q < 4 ? &v0[8 * q] : &v1[8 * (q - 4)];
-        uint32_t pk[4];
+        for (int e = 0; e < 32; ++e) {
+          const uint32_t* src = e < 16 ? &v0[2 * e] : &v1[2 * (e - 16)];
+          pk[e] = pack_bf16x2(__uint_as_float(src[0]), __uint_as_float(src[1]));
+        }
+        if (r < a.n) {
+          uint4* dst = reinterpret_cast<uint4*>(a.V + (bh * a.n + r) * kHd);
 #pragma unroll
-        for (int e = 0; e < 4; ++e) pk[e] = pack_bf16x2(__uint_as_float(src[2 * e]), __uint_as_float(src[2 * e + 1]));
-        dst[q] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          for (int q = 0; q < 8; ++q) dst[q] = make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+        }
+        if (a.vamax) {
+          // the column absmax of the bf16 values over this warp's valid tokens: the warp's 32 rows go
+          // through shared memory (the first stage buffer is free once the accumulator is done; 4 KB
+          // per warp, 16-byte chunks swizzled by row), then lane l scans columns 2l and 2l + 1 down
+          // the rows (magnitude bits, whose order is the values' order) and raises their maxima
+          uint32_t* tile = reinterpret_cast<uint32_t*>(sm + QkvSmem::kA) + warp * 32 * 32;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<uint4*>(tile + lane * 32 + ((q ^ (lane & 7)) << 2)) =
+                make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+          __syncwarp();
+          const int nvalid = min(32, L - (m0 + 32 * warp));  // rows of this warp below L
+          uint32_t mlo = 0u, mhi = 0u;
+          for (int rr = 0; rr < nvalid; ++rr) {
+            const uint32_t wv = tile[rr * 32 + ((((lane >> 2) ^ (rr & 7)) << 2) | (lane & 3))];
+            mlo = max(mlo, wv & 0x7FFFu);
+            mhi = max(mhi, (wv >> 16) & 0x7FFFu);
+          }
+          __syncwarp();
+          if (mlo) atomicMax(a.vamax + bh * kHd + 2 * lane, mlo << 16);
+          if (mhi) atomicMax(a.vamax + bh * kHd + 2 * lane + 1, mhi << 16);
+        }
       }
     }
   }

@@ -138,6 +138,20 @@ def deit(d: int = 64, B: int = 64) -> Workload:
                     extra={"outlier_channels": sorted(int(p) for p in pick)})
 
 
+def deit_qkv(B: int = 64):
+    """DeiT's attention inputs from their projection: X [B, 197, 768] bf16 tokens
+    ~N(0,1), a random-init projection weight W [3*12*64, 768] ~N(0, 1/768) in a
+    linear layer's layout (rows: Q's 768 channels, then K's, then V's), seed 9; the
+    DeiT relative-position bias (27x27 per head ~N(0, 0.1), prefix 1).  Returns
+    (X, W, H, bias, seqlens)."""
+    rng = np.random.default_rng(9)
+    H, n, Dm = 12, 197, 768
+    X = _finish(rng.standard_normal((B, n, Dm), dtype=np.float32), "bf16")
+    W = _finish(rng.standard_normal((3 * H * 64, Dm), dtype=np.float32) * np.float32(Dm ** -0.5), "bf16")
+    table = rng.standard_normal((H, 27, 27), dtype=np.float32) * np.float32(0.1)
+    return X, W, H, Bias(table, 14, 14, 1), None
+
+
 def deit_dense_bias() -> Workload:
     """The DeiT workload (same Q, K, V) with a dense bias matrix instead of the
     relative-position table: one value per query-key pair, [12, 197, 197]
