@@ -903,7 +903,7 @@ had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, 
   qkv::k_xmean<<<dim3((Dm + qkv::kXsumThreads - 1) / qkv::kXsumThreads, d.B), qkv::kXsumThreads, 0, st>>>(
       xpart, q.nch, d.n, Dm, d.H, s->seqlens, status, xbar, vamax);
   if ((r = check_launch("k_xmean")) != HAD_OK) return r;
-  qkv::k_mu<<<dim3((2 * d.H * 64 + qkv::kMuO - 1) / qkv::kMuO, (d.B + qkv::kMuB - 1) / qkv::kMuB, qkv::kMuSplit), qkv::kMuThreads, 0,
+  qkv::k_mu<<<dim3((2 * d.H * 64 + qkv::kMuThreads * qkv::kMuC - 1) / (qkv::kMuThreads * qkv::kMuC), (d.B + qkv::kMuB - 1) / qkv::kMuB, qkv::kMuSplit), qkv::kMuThreads, 0,
              st>>>(Wb, xbar, d.B, d.H, Dm, mupart);
   if ((r = check_launch("k_mu")) != HAD_OK) return r;
   // the projection, binarized in its epilogue, into the attention workspace

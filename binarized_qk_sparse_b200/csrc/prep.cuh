@@ -160,6 +160,18 @@ struct PackArgs {
   unsigned* status;
 };
 
+// Integer code of x at scale sc: rint(x / sc) clamped to +-qmax (127 or 7), with
+// x / sc the correctly rounded fp32 quotient.  For |x / sc| <= 128 the product
+// x * (1/sc) is within 2^-15 of that quotient, so both round to the same integer
+// unless the product lies within 2^-12 of a half-integer; only then is the
+// quotient computed.
+__device__ __forceinline__ int quant_v(float x, float sc, float rsc, float qmax) {
+  const float y = x * rsc;
+  float q = rintf(y);
+  if (fabsf(y - q) > 0.5f - 0x1p-12f) q = rintf(__fdiv_rn(x, sc));
+  return (int)fminf(fmaxf(q, -qmax), qmax);
+}
+
 template <typename T, int D>
 __global__ void __launch_bounds__(kPrepThreads) k_pack(const PackArgs a) {
   constexpr int kD = D;
@@ -174,7 +186,7 @@ __global__ void __launch_bounds__(kPrepThreads) k_pack(const PackArgs a) {
   const int cg = threadIdx.x % TPT, tok = threadIdx.x / TPT;
   const int i0 = chunk * kChunk;
   const size_t head = (size_t)bh * a.n * kD;
-  __shared__ float stat[kD];
+  __shared__ float stat[kD], rstat[kD];
   __shared__ __align__(16) int8_t vt[kD][kChunk];
   if (threadIdx.x < kD) {
     const int c = threadIdx.x;
@@ -192,6 +204,7 @@ __global__ void __launch_bounds__(kPrepThreads) k_pack(const PackArgs a) {
       const float qmax = a.v_bits == 4 ? 7.0f : 127.0f;
       float s = (m > 0.0f) ? __fdiv_rn(m, qmax) : 1.0f;
       stat[c] = s;
+      rstat[c] = 1.0f / s;
       if (chunk == 0) a.vscale[(size_t)bh * kD + c] = s;
     }
   }
@@ -237,11 +250,8 @@ __global__ void __launch_bounds__(kPrepThreads) k_pack(const PackArgs a) {
       }
       const float qmax = a.v_bits == 4 ? 7.0f : 127.0f;
 #pragma unroll
-      for (int u = 0; u < EPT; ++u) {
-        float r = rintf(__fdiv_rn(x[u], stat[cg * EPT + u]));
-        r = fminf(fmaxf(r, -qmax), qmax);
-        vt[cg * EPT + u][t] = (int8_t)(int)r;
-      }
+      for (int u = 0; u < EPT; ++u)
+        vt[cg * EPT + u][t] = (int8_t)quant_v(x[u], stat[cg * EPT + u], rstat[cg * EPT + u], qmax);
     }
     __syncthreads();
     if (a.v_bits == 4) {
@@ -449,18 +459,6 @@ __global__ void __launch_bounds__(256) k_dense_bias_tables(const BiasArgs a) {
     be[e] = b;
     ee[e] = w;
   }
-}
-
-// Integer code of x at scale sc: rint(x / sc) clamped to +-qmax (127 or 7), with
-// x / sc the correctly rounded fp32 quotient.  For |x / sc| <= 128 the product
-// x * (1/sc) is within 2^-15 of that quotient, so both round to the same integer
-// unless the product lies within 2^-12 of a half-integer; only then is the
-// quotient computed.
-__device__ __forceinline__ int quant_v(float x, float sc, float rsc, float qmax) {
-  const float y = x * rsc;
-  float q = rintf(y);
-  if (fabsf(y - q) > 0.5f - 0x1p-12f) q = rintf(__fdiv_rn(x, sc));
-  return (int)fminf(fmaxf(q, -qmax), qmax);
 }
 
 template <typename T, int kHeadThreads>

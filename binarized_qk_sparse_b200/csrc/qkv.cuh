@@ -35,7 +35,7 @@ using namespace had::sm100;
 
 constexpr int kXsumChunk = 32;     // tokens per partial sum of X
 constexpr int kXsumThreads = 128;  // k_xsum: feature threads (8 features each) per token group; k_xmean: one feature per thread
-constexpr int kMuB = 16, kMuO = 32, kMuK = 32;  // k_mu tile: batches x output channels x features
+constexpr int kMuB = 8, kMuK = 64;  // k_mu: batches per CTA, features per staged chunk
 
 // Token sums of X over the valid tokens of each 32-token chunk: part[b][ch][k], fp64.
 // Thread (g, f) of a CTA adds 8 adjacent features over the g-th 8 tokens of the
@@ -106,83 +106,75 @@ __global__ void __launch_bounds__(kXsumThreads) k_xmean(const double* __restrict
 // Partial dot products of the means with W: mupart[z][t][b][h][c] = sum over the
 // z-th of kMuSplit feature slices of xbar[b][k] W[o][k], o = t*H*64 + h*64 + c, in
 // fp64.  k_qkv_tc adds the kMuSplit partials in slice order and rounds once to
-// fp32.  A CTA of 128 threads computes 16 batches x 32 output channels of one
-// slice, two batches x two channels per thread; the mean tile and the W tile
-// (converted to fp64 once, as it is staged) of kMuK features sit in shared memory
-// while the next tile is already in registers.
+// fp32.  Thread x of a CTA owns output channels o = 512 * blockIdx.x + x + 128 c
+// (c < 4) and 8 batches: it reads its W rows in 16-byte pieces (eight features,
+// converted to fp64 once) and applies each piece to the 8 batches' means, which the
+// CTA stages in shared memory 64 features at a time; every lane of a warp reads the
+// same means (broadcasts), and each 16-byte read serves the four channels.
 constexpr int kMuThreads = 128;
+constexpr int kMuC = 4;  // channels per thread
 constexpr int kMuSplit = 8;
 __global__ void __launch_bounds__(kMuThreads) k_mu(const __nv_bfloat16* __restrict__ W,
                                                    const double* __restrict__ xbar, int B, int H, int Dm,
                                                    double* __restrict__ mupart) {
-  __shared__ __align__(16) double xs[kMuB][kMuK + 1];
-  __shared__ __align__(16) double ws[kMuO][kMuK + 1];
-  // thread (ty, tx): channels tx and tx + 16, batches ty and ty + 8 (rows 16 apart: no bank conflicts)
-  const int tid = threadIdx.x, tx = tid % (kMuO / 2), ty = tid / (kMuO / 2);
-  const int o0 = blockIdx.x * kMuO, b0 = blockIdx.y * kMuB;
+  __shared__ __align__(16) double xs[kMuB][kMuK];
+  const int o0 = blockIdx.x * kMuThreads * kMuC + threadIdx.x, b0 = blockIdx.y * kMuB;
   const int no = 2 * H * 64;
   const int slice = Dm / kMuSplit;  // a multiple of 8 (Dm is a multiple of 64)
   const int kbeg = blockIdx.z * slice, kend = kbeg + slice;
-  constexpr int kWPieces = kMuO * kMuK / 8 / kMuThreads;  // 8-feature pieces of W per thread and tile
-  constexpr int kXPairs = kMuB * kMuK / 2 / kMuThreads;   // feature pairs of the means per thread and tile
-  uint4 wr[kWPieces];
-  double2 xr[kXPairs];
-  auto fetch = [&](int k0) {
+  double acc[kMuB][kMuC];
 #pragma unroll
-    for (int j = 0; j < kWPieces; ++j) {
-      const int e = tid + kMuThreads * j, row = e / (kMuK / 8), kk = k0 + (e % (kMuK / 8)) * 8;
-      wr[j] = (o0 + row < no && kk < kend) ? __ldg(reinterpret_cast<const uint4*>(W + (size_t)(o0 + row) * Dm + kk))
-                                         : make_uint4(0u, 0u, 0u, 0u);
-    }
+  for (int bb = 0; bb < kMuB; ++bb)
 #pragma unroll
-    for (int j = 0; j < kXPairs; ++j) {
-      const int e = tid + kMuThreads * j, br = e / (kMuK / 2), kx = k0 + (e % (kMuK / 2)) * 2;
-      xr[j] = (b0 + br < B && kx < kend) ? *reinterpret_cast<const double2*>(xbar + (size_t)(b0 + br) * Dm + kx)
-                                       : make_double2(0.0, 0.0);
-    }
-  };
-  double acc[2][2] = {{0.0, 0.0}, {0.0, 0.0}};
-  fetch(kbeg);
+    for (int c = 0; c < kMuC; ++c) acc[bb][c] = 0.0;
   for (int k0 = kbeg; k0 < kend; k0 += kMuK) {
+    const int kn = min(kMuK, kend - k0);  // a multiple of 8
+    __syncthreads();  // the previous chunk's reads are done
+    for (int e = threadIdx.x; e < kMuB * kMuK / 2; e += kMuThreads) {
+      const int br = e / (kMuK / 2), cc = (e % (kMuK / 2)) * 2;
+      *reinterpret_cast<double2*>(&xs[br][cc]) =
+          (b0 + br < B && cc < kn) ? *reinterpret_cast<const double2*>(xbar + (size_t)(b0 + br) * Dm + k0 + cc)
+                                   : make_double2(0.0, 0.0);
+    }
+    __syncthreads();
+    for (int q = 0; q < kn / 8; ++q) {
+      double w[kMuC][8];
 #pragma unroll
-    for (int j = 0; j < kWPieces; ++j) {
-      const int e = tid + kMuThreads * j, row = e / (kMuK / 8), c = (e % (kMuK / 8)) * 8;
-      const uint32_t w[4] = {wr[j].x, wr[j].y, wr[j].z, wr[j].w};
+      for (int c = 0; c < kMuC; ++c) {
+        const int o = o0 + kMuThreads * c;
+        const uint4 wr = o < no ? __ldg(reinterpret_cast<const uint4*>(W + (size_t)o * Dm + k0 + 8 * q))
+                                : make_uint4(0u, 0u, 0u, 0u);
+        const uint32_t u[4] = {wr.x, wr.y, wr.z, wr.w};
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        ws[row][c + 2 * u] = (double)__uint_as_float(w[u] << 16);
-        ws[row][c + 2 * u + 1] = (double)__uint_as_float(w[u] & 0xFFFF0000u);
+        for (int v = 0; v < 4; ++v) {
+          w[c][2 * v] = (double)__uint_as_float(u[v] << 16);
+          w[c][2 * v + 1] = (double)__uint_as_float(u[v] & 0xFFFF0000u);
+        }
+      }
+#pragma unroll
+      for (int bb = 0; bb < kMuB; ++bb) {
+        const double2* xp = reinterpret_cast<const double2*>(&xs[bb][8 * q]);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          const double2 x2 = xp[v];
+#pragma unroll
+          for (int c = 0; c < kMuC; ++c) {
+            acc[bb][c] = fma(x2.x, w[c][2 * v], acc[bb][c]);
+            acc[bb][c] = fma(x2.y, w[c][2 * v + 1], acc[bb][c]);
+          }
+        }
       }
     }
-#pragma unroll
-    for (int j = 0; j < kXPairs; ++j) {
-      const int e = tid + kMuThreads * j, br = e / (kMuK / 2), cx = (e % (kMuK / 2)) * 2;
-      xs[br][cx] = xr[j].x;
-      xs[br][cx + 1] = xr[j].y;
-    }
-    __syncthreads();
-    if (k0 + kMuK < kend) fetch(k0 + kMuK);
-#pragma unroll 8
-    for (int kk = 0; kk < kMuK; ++kk) {
-      const double x0 = xs[ty][kk], x1 = xs[ty + kMuB / 2][kk];
-      const double w0 = ws[tx][kk], w1 = ws[tx + kMuO / 2][kk];
-      acc[0][0] = fma(x0, w0, acc[0][0]);
-      acc[0][1] = fma(x0, w1, acc[0][1]);
-      acc[1][0] = fma(x1, w0, acc[1][0]);
-      acc[1][1] = fma(x1, w1, acc[1][1]);
-    }
-    __syncthreads();
   }
 #pragma unroll
-  for (int ib = 0; ib < 2; ++ib)
+  for (int c = 0; c < kMuC; ++c) {
+    const int o = o0 + kMuThreads * c;
+    if (o >= no) continue;
+    const int t = o / (H * 64), r = o - t * H * 64;  // r = h * 64 + c
 #pragma unroll
-    for (int ic = 0; ic < 2; ++ic) {
-      const int b = b0 + ty + (kMuB / 2) * ib, o = o0 + tx + (kMuO / 2) * ic;
-      if (b < B && o < no) {
-        const int t = o / (H * 64), r = o - t * H * 64;  // r = h * 64 + c
-        mupart[(((size_t)blockIdx.z * 2 + t) * B + b) * H * 64 + r] = acc[ib][ic];
-      }
-    }
+    for (int bb = 0; bb < kMuB; ++bb)
+      if (b0 + bb < B) mupart[(((size_t)blockIdx.z * 2 + t) * B + b0 + bb) * H * 64 + r] = acc[bb][c];
+  }
 }
 
 // ---------------------------------------------------------------------------- the fused projection

@@ -54,7 +54,7 @@ def _read_workspace(ws, B, H, n):
 def _ambiguous(P, mu, X, W, H, t):
     """Entries whose sign an fp32 projection may legitimately take either way."""
     Wt = np.abs(W.astype(np.float64)).reshape(3, H, 64, -1)[t]  # [H, 64, Dm]
-    mag = np.einsum("bik,hck->bhic", np.abs(X.astype(np.float64)), Wt)
+    mag = np.einsum("bik,hck->bhic", np.abs(X.astype(np.float64)), Wt, optimize=True)
     tol = 2.0 ** -20 * mag + 2.0 ** -22 * np.abs(mu.astype(np.float64))[:, :, None, :]
     return np.abs(P - mu.astype(np.float64)[:, :, None, :]) <= tol
 
@@ -75,6 +75,8 @@ def _check_bits(got, ref_bits, P, mu, X, W, H, t, L):
     (2, 197, 256, 2, [197, 120], 0, "u8i8"),     # DeiT-like rows, ragged, dense uint8
     (1, 300, 192, 3, None, 30, "float"),         # 3 heads, top-30 float (n not a multiple of 128)
     (2, 70, 64, 1, [70, 9], 0, "float"),         # one panel, a short second sequence
+    # 720 CTAs of 128 tokens x 4 heads (several waves, two CTAs per SM), ragged lengths
+    (40, 197, 256, 12, list(range(197, 157, -1)), 0, "u8i8"),
 ])
 def test_qkv_bits_rows_and_v(oracle_mod, B, n, Dm, H, seqlens, N, mode):
     X, W = _inputs(B, n, Dm, H, seed=100 + n)
@@ -103,19 +105,20 @@ def test_qkv_bits_rows_and_v(oracle_mod, B, n, Dm, H, seqlens, N, mode):
     # V: bf16 of the fp64 projection, within bf16 rounding and the accumulation bound
     Vg = V.float().cpu().numpy()
     mag = np.einsum("bik,hck->bhic", np.abs(X.astype(np.float64)),
-                    np.abs(W.astype(np.float64)).reshape(3, H, 64, -1)[2])
+                    np.abs(W.astype(np.float64)).reshape(3, H, 64, -1)[2], optimize=True)
     assert np.all(np.abs(Vg - V64) <= np.abs(V64) * 2.0 ** -8 + 2.0 ** -20 * mag + 1e-30)
 
 
-@pytest.mark.parametrize("N,mode,with_bias", [(0, "u8i8", True), (0, "float", False), (40, "float", True),
-                                              (40, "u8i4", False)])
-def test_qkv_attention_end_to_end(oracle_mod, N, mode, with_bias):
+@pytest.mark.parametrize("B,H,N,mode,with_bias", [(2, 2, 0, "u8i8", True), (2, 2, 0, "float", False),
+                                                  (2, 2, 40, "float", True), (2, 2, 40, "u8i4", False),
+                                                  (24, 12, 0, "u8i8", True)])  # 432 CTAs, V absmax over many
+def test_qkv_attention_end_to_end(oracle_mod, B, H, N, mode, with_bias):
     """The attention on the fused workspace against the oracle's attention on +-1
     tensors that carry exactly the GPU's sign bits (their own means keep those signs)
     and the GPU's bf16 V: kept sets bit-exact, O within the usual bars."""
-    B, n, Dm, H = 2, 197, 256, 2
+    n, Dm = 197, 256
     X, W = _inputs(B, n, Dm, H, seed=77)
-    sl = np.array([197, 150], np.int32)
+    sl = np.array([197, 150] + [197 - 3 * i for i in range(B - 2)], np.int32)
     Xd = torch.from_numpy(X).to(torch.bfloat16).cuda()
     Wd = torch.from_numpy(W).to(torch.bfloat16).cuda()
     sd = torch.from_numpy(sl).cuda()
