@@ -891,6 +891,21 @@ had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, 
   Dims d = dims_of(s);
   const __nv_bfloat16* Xb = static_cast<const __nv_bfloat16*>(X);
   const __nv_bfloat16* Wb = static_cast<const __nv_bfloat16*>(Wqkv);
+  {
+    static std::mutex smu;
+    static bool configured[kMaxDevices] = {false};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    std::lock_guard<std::mutex> lk(smu);
+    if (dev >= 0 && dev < kMaxDevices && !configured[dev]) {
+      cudaError_t e = cudaFuncSetAttribute(qkv::k_qkv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           qkv::QkvSmem::kTotal);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_qkv_tc)");
+      e = cudaFuncSetAttribute(qkv::k_mu, cudaFuncAttributeMaxDynamicSharedMemorySize, qkv::MuSmem::kTotal);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_mu)");
+      configured[dev] = true;
+    }
+  }
   double* xpart = reinterpret_cast<double*>(ws + q.xpart);
   double* mupart = reinterpret_cast<double*>(ws + q.mu);
   // the means of Q and K from X's token means
@@ -903,7 +918,7 @@ had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, 
   qkv::k_xmean<<<dim3((Dm + qkv::kXsumThreads - 1) / qkv::kXsumThreads, d.B), qkv::kXsumThreads, 0, st>>>(
       xpart, q.nch, d.n, Dm, d.H, s->seqlens, status, xbar, vamax);
   if ((r = check_launch("k_xmean")) != HAD_OK) return r;
-  qkv::k_mu<<<dim3((2 * d.H * 64 + qkv::kMuThreads * qkv::kMuC - 1) / (qkv::kMuThreads * qkv::kMuC), (d.B + qkv::kMuB - 1) / qkv::kMuB, qkv::kMuSplit), qkv::kMuThreads, 0,
+  qkv::k_mu<<<dim3((2 * d.H * 64 + qkv::kMuThreads * qkv::kMuC - 1) / (qkv::kMuThreads * qkv::kMuC), (d.B + qkv::kMuB - 1) / qkv::kMuB, qkv::kMuSplit), qkv::kMuThreads, qkv::MuSmem::kTotal,
              st>>>(Wb, xbar, d.B, d.H, Dm, mupart);
   if ((r = check_launch("k_mu")) != HAD_OK) return r;
   // the projection, binarized in its epilogue, into the attention workspace
@@ -924,19 +939,6 @@ had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, 
   qa.V = static_cast<__nv_bfloat16*>(V_out);
   qa.vamax = vbits != 0 ? vamax : nullptr;
   qa.status = status;
-  {
-    static std::mutex smu;
-    static bool configured[kMaxDevices] = {false};
-    int dev = 0;
-    cudaGetDevice(&dev);
-    std::lock_guard<std::mutex> lk(smu);
-    if (dev >= 0 && dev < kMaxDevices && !configured[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(qkv::k_qkv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           qkv::QkvSmem::kTotal);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_qkv_tc)");
-      configured[dev] = true;
-    }
-  }
   qkv::k_qkv_tc<<<dim3((d.n + qkv::kM - 1) / qkv::kM, d.B, (3 * d.H + qkv::kNB - 1) / qkv::kNB), qkv::kThreads,
                    qkv::QkvSmem::kTotal, st>>>(qa);
   if ((r = check_launch("k_qkv_tc")) != HAD_OK) return r;
@@ -946,11 +948,10 @@ had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, 
       (r = build_bias_tables(s, bias, ws + w.bminmax, ws + w.bext, ws + w.expb, st)) != HAD_OK)
     return r;
   if (vbits != 0) {
-    r = launch_prep(s, nullptr, nullptr, V_out, 2, 1, reinterpret_cast<double*>(ws + w.sums),
-                    reinterpret_cast<float*>(ws + w.amax), nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
-                    reinterpret_cast<int8_t*>(ws + w.vqT), reinterpret_cast<float*>(ws + w.vscale), st, status, vbits,
-                    false, reinterpret_cast<const float*>(vamax));
-    if (r != HAD_OK) return r;
+    qkv::k_vcodes<<<dim3(d.n_pad / 64, d.BH), qkv::kVcThreads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(V_out), vamax, d.H, d.n, d.n_pad, s->seqlens, vbits,
+        reinterpret_cast<int8_t*>(ws + w.vqT), reinterpret_cast<float*>(ws + w.vscale));
+    if ((r = check_launch("k_vcodes")) != HAD_OK) return r;
   }
   return HAD_OK;
 }

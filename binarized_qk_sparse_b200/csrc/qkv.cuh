@@ -26,6 +26,7 @@
 #include <cuda_bf16.h>
 
 #include "common.cuh"
+#include "prep.cuh"
 #include "sm100.cuh"
 
 namespace had {
@@ -106,19 +107,36 @@ __global__ void __launch_bounds__(kXsumThreads) k_xmean(const double* __restrict
 // Partial dot products of the means with W: mupart[z][t][b][h][c] = sum over the
 // z-th of kMuSplit feature slices of xbar[b][k] W[o][k], o = t*H*64 + h*64 + c, in
 // fp64.  k_qkv_tc adds the kMuSplit partials in slice order and rounds once to
-// fp32.  Thread x of a CTA owns output channels o = 512 * blockIdx.x + x + 128 c
-// (c < 4) and 8 batches: it reads its W rows in 16-byte pieces (eight features,
-// converted to fp64 once) and applies each piece to the 8 batches' means, which the
-// CTA stages in shared memory 64 features at a time; every lane of a warp reads the
-// same means (broadcasts), and each 16-byte read serves the four channels.
+// fp32.  A CTA takes 512 output channels and 8 batches, 64 features at a time: all
+// its threads copy the 512 W rows of the chunk into shared memory at once
+// (cp.async, 16 bytes each, rows padded to 144 bytes so that 16-byte reads of
+// eight rows hit distinct banks), and the 8 batches' means beside them.  Thread x
+// then owns channels x + 128 c (c < 4): it converts a 16-byte piece of each of
+// its rows to fp64 and applies it to the 8 batches' means (every lane of a warp
+// reads the same means: broadcasts).
 constexpr int kMuThreads = 128;
-constexpr int kMuC = 4;  // channels per thread
-constexpr int kMuSplit = 8;
+constexpr int kMuC = 4;                     // channels per thread
+constexpr int kMuSplit = 8;                 // feature slices
+constexpr int kMuRow = kMuK * 2 + 16;       // bytes per staged W row
+struct MuSmem {
+  static constexpr int kW = 0;                                // [512 rows][kMuRow] bf16
+  static constexpr int kX = kW + kMuThreads * kMuC * kMuRow;  // [kMuB][kMuK] fp64
+  static constexpr int kTotal = kX + kMuB * kMuK * 8;
+};
+
+__device__ __forceinline__ void cp_async16_zfill(void* smem_dst, const void* gmem_src, bool valid) {
+  const uint32_t d = smem_u32(smem_dst);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(gmem_src), "r"(valid ? 16 : 0)
+               : "memory");
+}
+
 __global__ void __launch_bounds__(kMuThreads) k_mu(const __nv_bfloat16* __restrict__ W,
                                                    const double* __restrict__ xbar, int B, int H, int Dm,
                                                    double* __restrict__ mupart) {
-  __shared__ __align__(16) double xs[kMuB][kMuK];
-  const int o0 = blockIdx.x * kMuThreads * kMuC + threadIdx.x, b0 = blockIdx.y * kMuB;
+  extern __shared__ __align__(16) uint8_t musm[];
+  uint8_t* wsm = musm + MuSmem::kW;
+  double* xs = reinterpret_cast<double*>(musm + MuSmem::kX);
+  const int ob = blockIdx.x * kMuThreads * kMuC, b0 = blockIdx.y * kMuB;
   const int no = 2 * H * 64;
   const int slice = Dm / kMuSplit;  // a multiple of 8 (Dm is a multiple of 64)
   const int kbeg = blockIdx.z * slice, kend = kbeg + slice;
@@ -130,20 +148,26 @@ __global__ void __launch_bounds__(kMuThreads) k_mu(const __nv_bfloat16* __restri
   for (int k0 = kbeg; k0 < kend; k0 += kMuK) {
     const int kn = min(kMuK, kend - k0);  // a multiple of 8
     __syncthreads();  // the previous chunk's reads are done
+    for (int e = threadIdx.x; e < kMuThreads * kMuC * (kMuK / 8); e += kMuThreads) {
+      const int row = e / (kMuK / 8), q = e % (kMuK / 8), o = ob + row;
+      const bool v = o < no && 8 * q < kn;
+      cp_async16_zfill(wsm + row * kMuRow + 16 * q, v ? static_cast<const void*>(W + (size_t)o * Dm + k0 + 8 * q) : W,
+                       v);
+    }
+    asm volatile("cp.async.commit_group;\n" ::: "memory");
     for (int e = threadIdx.x; e < kMuB * kMuK / 2; e += kMuThreads) {
       const int br = e / (kMuK / 2), cc = (e % (kMuK / 2)) * 2;
-      *reinterpret_cast<double2*>(&xs[br][cc]) =
+      *reinterpret_cast<double2*>(xs + br * kMuK + cc) =
           (b0 + br < B && cc < kn) ? *reinterpret_cast<const double2*>(xbar + (size_t)(b0 + br) * Dm + k0 + cc)
                                    : make_double2(0.0, 0.0);
     }
+    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
     __syncthreads();
     for (int q = 0; q < kn / 8; ++q) {
       double w[kMuC][8];
 #pragma unroll
       for (int c = 0; c < kMuC; ++c) {
-        const int o = o0 + kMuThreads * c;
-        const uint4 wr = o < no ? __ldg(reinterpret_cast<const uint4*>(W + (size_t)o * Dm + k0 + 8 * q))
-                                : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 wr = *reinterpret_cast<const uint4*>(wsm + (threadIdx.x + kMuThreads * c) * kMuRow + 16 * q);
         const uint32_t u[4] = {wr.x, wr.y, wr.z, wr.w};
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
@@ -153,7 +177,7 @@ __global__ void __launch_bounds__(kMuThreads) k_mu(const __nv_bfloat16* __restri
       }
 #pragma unroll
       for (int bb = 0; bb < kMuB; ++bb) {
-        const double2* xp = reinterpret_cast<const double2*>(&xs[bb][8 * q]);
+        const double2* xp = reinterpret_cast<const double2*>(xs + bb * kMuK + 8 * q);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const double2 x2 = xp[v];
@@ -168,12 +192,77 @@ __global__ void __launch_bounds__(kMuThreads) k_mu(const __nv_bfloat16* __restri
   }
 #pragma unroll
   for (int c = 0; c < kMuC; ++c) {
-    const int o = o0 + kMuThreads * c;
+    const int o = ob + threadIdx.x + kMuThreads * c;
     if (o >= no) continue;
     const int t = o / (H * 64), r = o - t * H * 64;  // r = h * 64 + c
 #pragma unroll
     for (int bb = 0; bb < kMuB; ++bb)
       if (b0 + bb < B) mupart[(((size_t)blockIdx.z * 2 + t) * B + b0 + bb) * H * 64 + r] = acc[bb][c];
+  }
+}
+
+// V's codes from the projection's bf16 V and the epilogue's column absmax, as the
+// prepare stage makes them (scale absmax/qmax, 1 if the absmax is 0; codes
+// rint(V/scale) clamped to +-qmax, 0 past L), transposed to V^T: int8
+// [B*H][64][n_pad], or packed 4-bit [B*H][64][n_pad/2] with key 2k in the low
+// nibble of byte k.  A CTA takes 64 tokens of one head: thread (g, t) reads token
+// t's channels 8g..8g+7 and 32+8g..32+8g+7 (16-byte loads), writes their codes
+// into a [64 channels][64 tokens] byte tile, and the tile's rows leave as 16-byte
+// (int8) or 8-byte (4-bit) stores.
+constexpr int kVcThreads = 256;
+__global__ void __launch_bounds__(kVcThreads) k_vcodes(const __nv_bfloat16* __restrict__ V,
+                                                       const uint32_t* __restrict__ vamax, int H, int n,
+                                                       int n_pad, const int32_t* seqlens, int vbits,
+                                                       int8_t* __restrict__ vqT, float* __restrict__ vscale) {
+  __shared__ float sc[64], rsc[64];
+  __shared__ __align__(16) uint8_t tile[64][64 + 16];
+  const int bh = blockIdx.y, i0 = blockIdx.x * 64, tid = threadIdx.x;
+  const int L = valid_len(seqlens, bh / H, n, nullptr);  // the projection reported bad lengths
+  const float qmax = vbits == 4 ? 7.0f : 127.0f;
+  if (tid < 64) {
+    const float m = __uint_as_float(vamax[(size_t)bh * 64 + tid]);
+    const float s = m > 0.0f ? __fdiv_rn(m, qmax) : 1.0f;
+    sc[tid] = s;
+    rsc[tid] = 1.0f / s;
+    if (blockIdx.x == 0) vscale[(size_t)bh * 64 + tid] = s;
+  }
+  __syncthreads();
+  {
+    const int t = tid & 63, g = tid >> 6, i = i0 + t;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int c0 = 32 * half + 8 * g;
+      uint4 x = make_uint4(0u, 0u, 0u, 0u);
+      if (i < L) x = __ldg(reinterpret_cast<const uint4*>(V + ((size_t)bh * n + i) * 64 + c0));
+      const uint32_t u[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+      for (int v = 0; v < 4; ++v) {
+        const int c = c0 + 2 * v;
+        tile[c][t] = (uint8_t)quant_v(__uint_as_float(u[v] << 16), sc[c], rsc[c], qmax);
+        tile[c + 1][t] = (uint8_t)quant_v(__uint_as_float(u[v] & 0xFFFF0000u), sc[c + 1], rsc[c + 1], qmax);
+      }
+    }
+  }
+  __syncthreads();
+  const int c = tid >> 2, seg = tid & 3;  // channel row c, 16 of its 64 tokens
+  const uint4 w = *reinterpret_cast<const uint4*>(&tile[c][16 * seg]);
+  if (vbits == 4) {
+    const uint32_t in[4] = {w.x, w.y, w.z, w.w};
+    uint32_t out[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      uint32_t o = 0u;
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {  // byte b of word k: keys 8k + 2b (low nibble) and 8k + 2b + 1
+        const uint32_t wd = in[2 * k + (b >> 1)], sh = (b & 1) * 16;
+        o |= (((wd >> sh) & 15u) | (((wd >> (sh + 8)) & 15u) << 4)) << (8 * b);
+      }
+      out[k] = o;
+    }
+    uint8_t* dst = reinterpret_cast<uint8_t*>(vqT) + ((size_t)bh * 64 + c) * (n_pad / 2) + i0 / 2 + 8 * seg;
+    *reinterpret_cast<uint2*>(dst) = make_uint2(out[0], out[1]);
+  } else {
+    *reinterpret_cast<uint4*>(vqT + ((size_t)bh * 64 + c) * n_pad + i0 + 16 * seg) = w;
   }
 }
 
