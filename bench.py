@@ -99,6 +99,21 @@ def launches_per_step(n: int, elem: int, mode: str, has_bias: bool, dense_bias: 
     return k + 1
 
 
+def relpos_table_launches(gh: int, gw: int) -> int:
+    """Kernels that build a relative-position table's extended tables outside the
+    prepare stage (the fused projection, the dense comparison mode): one CTA per
+    head for tables of at most 8192 extended entries, else the range and a fill
+    over many CTAs per head.  The extended size is E = 3T + 3K_x rounded up to 4,
+    T = (2gh - 1) S, K_x = (gh - 1) S + gw, S the smallest row stride >= 2gw - 1
+    with S = gw (mod 32)."""
+    S = 2 * gw - 1
+    while S % 32 != gw % 32:
+        S += 1
+    T, Kx = (2 * gh - 1) * S, (gh - 1) * S + gw
+    E = (3 * T + 3 * Kx + 3) // 4 * 4
+    return 1 if E <= 8192 else 2
+
+
 # Issue-limited CUDA-core rate of one B200: 148 SMs x 4 schedulers x 32 lanes x
 # 1965 MHz (clocks.max.sm), one lane-operation per lane per clock.  A derived
 # ceiling for the diagnostic ALU roofline, not a measured peak.
@@ -481,7 +496,8 @@ def run_gpu(args, rank, world, local_rank):
     probe_bf16, _ = had.had_probe_mma_rate("bf16", 20000)
 
     if ref:  # the bias tables (range + tables for a dense matrix) and the kernel
-        kernels_per_step = 1 + (0 if bias is None else (2 if isinstance(w.bias, workloads.DenseBias) else 1))
+        kernels_per_step = 1 + (0 if bias is None else (2 if isinstance(w.bias, workloads.DenseBias)
+                                                        else relpos_table_launches(w.bias.gh, w.bias.gw)))
     else:
         kernels_per_step = launches_per_step(w.n, Q.element_size(), mode, bias is not None,
                                              isinstance(w.bias, workloads.DenseBias), w.d)
@@ -779,7 +795,7 @@ def run_qkv(args, rank, world, local_rank):
         "roofline": roof,
         "e2e": {"value": queries / (e0.elapsed_time(e1) / e2e_steps * 1e-3), "unit": UNIT,
                 "h2d_bytes_per_step": X.size * 2, "d2h_bytes_per_step": O.numel() * 2},
-        "gpu_launches": args.steps * 9,  # the fused loop: k_xsum, k_mu, k_qkv_tc, 2 bias-table, 3 V-quantization kernels, k_attn_tc
+        "gpu_launches": args.steps * (6 + relpos_table_launches(bw.gh, bw.gw)),  # k_xsum, k_xmean, k_mu, k_qkv_tc, the bias tables, k_vcodes, k_attn_tc
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)

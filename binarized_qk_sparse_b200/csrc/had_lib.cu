@@ -447,9 +447,14 @@ had_status build_bias_tables(const had_shape* s, const had_relpos_bias* bias, ui
     k_dense_bias_tables<<<tgrid, 256, 0, st>>>(ba);
     return check_launch("k_dense_bias_tables");
   }
+  const int E = relpos_ext(ba.gh, ba.gw).E;
+  if (E <= kBiasFillPerCta) {  // small tables: one CTA per head takes the range and fills the tables
+    k_bias_tables<<<s->H, 256, 0, st>>>(ba);
+    return check_launch("k_bias_tables");
+  }
   k_bias_range<<<s->H, kBiasRangeThreads, 0, st>>>(ba);
   if ((r = check_launch("k_bias_range")) != HAD_OK) return r;
-  dim3 fgrid((relpos_ext(ba.gh, ba.gw).E + kBiasFillPerCta - 1) / kBiasFillPerCta, s->H);
+  dim3 fgrid((E + kBiasFillPerCta - 1) / kBiasFillPerCta, s->H);
   k_bias_fill<<<fgrid, 256, 0, st>>>(ba);
   return check_launch("k_bias_fill");
 }
@@ -562,10 +567,10 @@ had_status attend_stage(const void* V, const had_shape* s, const had_relpos_bias
 }
 
 // Workspace of the fused projection: the attention workspace (so that
-// had_attention_prepared can run on it), then X's token partial sums, X's token
-// means, the means of Q and K, and V's column absmax per head.
+// had_attention_prepared can run on it), then X's token partial sums, the
+// partial means of Q and K, and V's column absmax per head.
 struct QkvWs {
-  size_t xpart, xbar, mu, vamax, total;
+  size_t xpart, mu, vamax, total;
   int nch;
 };
 
@@ -574,7 +579,6 @@ QkvWs qkv_ws_layout(const had_shape* s, int Dm, int vbits, const had_relpos_bias
   size_t off = align_up(ws_layout(s, vbits, bias).total);
   q.nch = (s->n + qkv::kXsumChunk - 1) / qkv::kXsumChunk;
   q.xpart = off; off += align_up((size_t)s->B * q.nch * Dm * 8);
-  q.xbar = off; off += align_up((size_t)s->B * Dm * 8);
   q.mu = off; off += align_up((size_t)qkv::kMuSplit * 2 * s->B * s->H * 64 * 8);
   q.vamax = off; off += align_up((size_t)s->B * s->H * 64 * 4);
   q.total = off;
@@ -909,17 +913,14 @@ had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, 
   double* xpart = reinterpret_cast<double*>(ws + q.xpart);
   double* mupart = reinterpret_cast<double*>(ws + q.mu);
   // the means of Q and K from X's token means
-  qkv::k_xsum<<<dim3((Dm / 8 + qkv::kXsumThreads - 1) / qkv::kXsumThreads, q.nch, d.B),
-                  qkv::kXsumThreads * qkv::kXsumGroups, 0, st>>>(
-      Xb, d.n, Dm, s->seqlens, q.nch, xpart);
-  if ((r = check_launch("k_xsum")) != HAD_OK) return r;
-  double* xbar = reinterpret_cast<double*>(ws + q.xbar);
   uint32_t* vamax = reinterpret_cast<uint32_t*>(ws + q.vamax);
-  qkv::k_xmean<<<dim3((Dm + qkv::kXsumThreads - 1) / qkv::kXsumThreads, d.B), qkv::kXsumThreads, 0, st>>>(
-      xpart, q.nch, d.n, Dm, d.H, s->seqlens, status, xbar, vamax);
-  if ((r = check_launch("k_xmean")) != HAD_OK) return r;
-  qkv::k_mu<<<dim3((2 * d.H * 64 + qkv::kMuThreads * qkv::kMuC - 1) / (qkv::kMuThreads * qkv::kMuC), (d.B + qkv::kMuB - 1) / qkv::kMuB, qkv::kMuSplit), qkv::kMuThreads, qkv::MuSmem::kTotal,
-             st>>>(Wb, xbar, d.B, d.H, Dm, mupart);
+  qkv::k_xsum<<<dim3((Dm / 8 + qkv::kXsumThreads - 1) / qkv::kXsumThreads, q.nch, d.B),
+                  qkv::kXsumThreads * qkv::kXsumGroups, 0, st>>>(Xb, d.n, Dm, d.H, s->seqlens, q.nch, xpart,
+                                                                  vbits != 0 ? vamax : nullptr);
+  if ((r = check_launch("k_xsum")) != HAD_OK) return r;
+  qkv::k_mu<<<dim3((2 * d.H * 64 + qkv::kMuThreads * qkv::kMuC - 1) / (qkv::kMuThreads * qkv::kMuC),
+                   (d.B + qkv::kMuB - 1) / qkv::kMuB, qkv::kMuSplit),
+              qkv::kMuThreads, qkv::MuSmem::kTotal, st>>>(Wb, xpart, q.nch, d.n, s->seqlens, d.B, d.H, Dm, mupart);
   if ((r = check_launch("k_mu")) != HAD_OK) return r;
   // the projection, binarized in its epilogue, into the attention workspace
   qkv::QkvArgs qa;

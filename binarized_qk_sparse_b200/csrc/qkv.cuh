@@ -8,8 +8,8 @@
 // map's outputs is the map of the mean input, so
 //   mu_Q[b][h][c] = (1/L_b) sum_{i<L_b} (X_i W_Q^T)[h*d + c] = xbar_b . W_Q[h*d + c],
 // with xbar_b the mean of the valid tokens of X (k_xsum: fp64 token sums per
-// 32-token chunk; k_xmean: the means; k_mu: a tiled fp64 product of the means
-// with W in feature slices, added in order and rounded once to fp32 by k_qkv_tc).  Then k_qkv_tc runs the projection on the tensor cores and
+// 32-token chunk; k_mu: the means from those sums, then their fp64 product with
+// W in feature slices, added in order and rounded once to fp32 by k_qkv_tc).  Then k_qkv_tc runs the projection on the tensor cores and
 // compares each fp32 result with its mean in the epilogue:
 //   - Q columns: the 64 sign bits of a token (bit 1 = below the mean), in the
 //     attention workspace's packed layout;
@@ -35,7 +35,7 @@ namespace qkv {
 using namespace had::sm100;
 
 constexpr int kXsumChunk = 32;     // tokens per partial sum of X
-constexpr int kXsumThreads = 128;  // k_xsum: feature threads (8 features each) per token group; k_xmean: one feature per thread
+constexpr int kXsumThreads = 128;  // k_xsum: feature threads (8 features each) per token group
 constexpr int kMuB = 8, kMuK = 64;  // k_mu: batches per CTA, features per staged chunk
 
 // Token sums of X over the valid tokens of each 32-token chunk: part[b][ch][k], fp64.
@@ -44,9 +44,12 @@ constexpr int kMuB = 8, kMuK = 64;  // k_mu: batches per CTA, features per stage
 // added in group order.
 constexpr int kXsumGroups = kXsumChunk / 8;
 __global__ void __launch_bounds__(kXsumThreads * kXsumGroups) k_xsum(const __nv_bfloat16* __restrict__ X, int n,
-                                                                     int Dm, const int32_t* seqlens, int nch,
-                                                                     double* __restrict__ part) {
+                                                                     int Dm, int H, const int32_t* seqlens, int nch,
+                                                                     double* __restrict__ part,
+                                                                     uint32_t* __restrict__ vamax) {
   __shared__ double red[kXsumGroups - 1][8][kXsumThreads];
+  if (vamax && blockIdx.x == 0 && blockIdx.y == 0)  // V's column absmax of batch b, raised later by the projection
+    for (int e = threadIdx.x; e < H * 64; e += blockDim.x) vamax[(size_t)blockIdx.z * H * 64 + e] = 0u;
   const int ft = threadIdx.x % kXsumThreads, tg = threadIdx.x / kXsumThreads;
   const int k0 = (blockIdx.x * kXsumThreads + ft) * 8, ch = blockIdx.y, b = blockIdx.z;
   const bool act = k0 < Dm;
@@ -88,22 +91,6 @@ __global__ void __launch_bounds__(kXsumThreads * kXsumGroups) k_xsum(const __nv_
   }
 }
 
-// The token means of X: xbar[b][k] = (chunk sums added in order) / L_b, fp64.
-// Also clears V's column absmax of batch b (H*64 words), which the projection's
-// epilogue raises with atomic maxima.
-__global__ void __launch_bounds__(kXsumThreads) k_xmean(const double* __restrict__ part, int nch, int n, int Dm,
-                                                        int H, const int32_t* seqlens, unsigned* status,
-                                                        double* __restrict__ xbar, uint32_t* __restrict__ vamax) {
-  const int k = blockIdx.x * kXsumThreads + threadIdx.x, b = blockIdx.y;
-  if (k >= Dm) return;
-  for (int e = k; e < H * 64; e += Dm) vamax[(size_t)b * H * 64 + e] = 0u;
-  const int L = valid_len(seqlens, b, n, status);
-  const int nv = (L + kXsumChunk - 1) / kXsumChunk;
-  double v = 0.0;
-  for (int c = 0; c < nv; ++c) v += part[((size_t)b * nch + c) * Dm + k];
-  xbar[(size_t)b * Dm + k] = L > 0 ? v / (double)L : 0.0;
-}
-
 // Partial dot products of the means with W: mupart[z][t][b][h][c] = sum over the
 // z-th of kMuSplit feature slices of xbar[b][k] W[o][k], o = t*H*64 + h*64 + c, in
 // fp64.  k_qkv_tc adds the kMuSplit partials in slice order and rounds once to
@@ -131,7 +118,8 @@ __device__ __forceinline__ void cp_async16_zfill(void* smem_dst, const void* gme
 }
 
 __global__ void __launch_bounds__(kMuThreads) k_mu(const __nv_bfloat16* __restrict__ W,
-                                                   const double* __restrict__ xbar, int B, int H, int Dm,
+                                                   const double* __restrict__ part, int nch, int n,
+                                                   const int32_t* seqlens, int B, int H, int Dm,
                                                    double* __restrict__ mupart) {
   extern __shared__ __align__(16) uint8_t musm[];
   uint8_t* wsm = musm + MuSmem::kW;
@@ -155,11 +143,21 @@ __global__ void __launch_bounds__(kMuThreads) k_mu(const __nv_bfloat16* __restri
                        v);
     }
     asm volatile("cp.async.commit_group;\n" ::: "memory");
+    // the means: the chunk sums of k_xsum added in chunk order, divided by L
     for (int e = threadIdx.x; e < kMuB * kMuK / 2; e += kMuThreads) {
-      const int br = e / (kMuK / 2), cc = (e % (kMuK / 2)) * 2;
-      *reinterpret_cast<double2*>(xs + br * kMuK + cc) =
-          (b0 + br < B && cc < kn) ? *reinterpret_cast<const double2*>(xbar + (size_t)(b0 + br) * Dm + k0 + cc)
-                                   : make_double2(0.0, 0.0);
+      const int br = e / (kMuK / 2), cc = (e % (kMuK / 2)) * 2, b = b0 + br;
+      double2 m = make_double2(0.0, 0.0);
+      if (b < B && cc < kn) {
+        const int L = valid_len(seqlens, b, n, nullptr);  // the projection reports bad lengths
+        const int nv = (L + kXsumChunk - 1) / kXsumChunk;
+        for (int c = 0; c < nv; ++c) {
+          const double2 p = *reinterpret_cast<const double2*>(part + ((size_t)b * nch + c) * Dm + k0 + cc);
+          m.x += p.x;
+          m.y += p.y;
+        }
+        if (L > 0) m = make_double2(m.x / (double)L, m.y / (double)L);
+      }
+      *reinterpret_cast<double2*>(xs + br * kMuK + cc) = m;
     }
     asm volatile("cp.async.wait_group 0;\n" ::: "memory");
     __syncthreads();
