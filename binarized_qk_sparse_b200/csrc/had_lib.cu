@@ -627,16 +627,24 @@ had_status run_attention(const void* Q, const void* K, const void* V, const had_
 // table copies, then `slots` chunk slots (Q, K, V, O and the kernels'
 // workspace of one chunk of `cb` sequences) that consecutive chunks cycle through.
 struct HostPlan {
-  int cb = 0, chunks = 0, slots = 0;
-  size_t in_b = 0, o_b = 0;                   // bytes of one sequence of Q (= K = V), of O as fp32
+  int cb = 0, hc = 0, hgroups = 0, chunks = 0, slots = 0;  // sequences per chunk, heads per chunk (when a
+                                                            // sequence is split), head groups per sequence
+  size_t in_b = 0, head_b = 0;                // bytes of one sequence, of one head, of Q (= K = V)
   size_t seq = 0, tab = 0, tab_bytes = 0, slot0 = 0, slot_bytes = 0, total = 0;
   size_t q = 0, k = 0, v = 0, o = 0, ws = 0;  // offsets inside a slot
   size_t ws_bytes = 0;
 };
 
-constexpr int kHostSlots = 3;
+constexpr int kHostSlots = 4;    // two chunks computing, one copying in, one copying out
+constexpr int kHostCompute = 2;  // compute streams: the caller's and one side stream, alternating chunks
 constexpr size_t kHostChunkBytes = size_t(8) << 20;  // input bytes per chunk when the caller passes chunk_b = 0
+constexpr size_t kHostSplitBytes = size_t(16) << 20;  // at most this per chunk when a sequence is split by heads
 
+// Chunks: chunk_b > 0 takes chunk_b whole sequences per chunk.  chunk_b = 0 takes
+// about kHostChunkBytes of inputs: whole sequences while one fits, else one
+// sequence's heads in equal groups of at most kHostSplitBytes (so that long
+// sequences also start computing after a short copy, and the copy of the last O
+// is short).
 had_status host_plan(const had_shape* s, had_mode mode, const had_relpos_bias* bias, int chunk_b, HostPlan* p) {
   if (!s) return HAD_ERR_INVALID;
   had_shape s0 = *s;
@@ -647,14 +655,28 @@ had_status host_plan(const had_shape* s, had_mode mode, const had_relpos_bias* b
   if (chunk_b < 0) return HAD_ERR_INVALID;
   const bool has_bias = bias && bias->table;
   const size_t esz = s->in_dtype == HAD_BF16 ? 2 : 4;
-  p->in_b = (size_t)s->H * s->n * s->d * esz;
-  p->o_b = (size_t)s->H * s->n * s->d * 4;
-  size_t cb = chunk_b > 0 ? (size_t)chunk_b : std::max<size_t>(1, kHostChunkBytes / (3 * p->in_b));
-  p->cb = (int)std::min<size_t>(cb, (size_t)s->B);
-  p->chunks = (s->B + p->cb - 1) / p->cb;
+  p->head_b = (size_t)s->n * s->d * esz;
+  p->in_b = (size_t)s->H * p->head_b;
+  const size_t head_ob = (size_t)s->n * s->d * 4;  // O as fp32 (the larger output type)
+  p->hc = s->H;
+  if (chunk_b > 0) {
+    p->cb = std::min(chunk_b, s->B);
+  } else if (3 * p->in_b <= kHostChunkBytes) {
+    p->cb = (int)std::min<size_t>(kHostChunkBytes / (3 * p->in_b), (size_t)s->B);
+  } else {
+    // head groups of at most kHostSplitBytes of inputs, of equal size: enough rows per chunk that two
+    // chunks in flight fill the GPU
+    p->cb = 1;
+    const int hmax = (int)std::max<size_t>(1, std::min<size_t>(kHostSplitBytes / (3 * p->head_b), (size_t)s->H));
+    const int groups = (s->H + hmax - 1) / hmax;
+    p->hc = (s->H + groups - 1) / groups;
+  }
+  p->hgroups = (s->H + p->hc - 1) / p->hc;
+  p->chunks = ((s->B + p->cb - 1) / p->cb) * p->hgroups;
   p->slots = std::min(kHostSlots, p->chunks);
   had_shape sc = s0;
   sc.B = p->cb;
+  sc.H = p->hc;
   p->ws_bytes = ws_layout(&sc, vbits_of(mode), has_bias ? bias : nullptr).total;
   size_t off = 0;
   p->seq = off;
@@ -665,11 +687,12 @@ had_status host_plan(const had_shape* s, had_mode mode, const had_relpos_bias* b
                                : (size_t)s->H * (2 * bias->gh - 1) * (2 * bias->gw - 1) * sizeof(float);
   off += align_up(p->tab_bytes);
   p->slot0 = off;
+  const size_t cin = (size_t)p->cb * p->hc * p->head_b, cout = (size_t)p->cb * p->hc * head_ob;
   size_t so = 0;
-  p->q = so; so += align_up(p->cb * p->in_b);
-  p->k = so; so += align_up(p->cb * p->in_b);
-  p->v = so; so += align_up(p->cb * p->in_b);
-  p->o = so; so += align_up(p->cb * p->o_b);
+  p->q = so; so += align_up(cin);
+  p->k = so; so += align_up(cin);
+  p->v = so; so += align_up(cin);
+  p->o = so; so += align_up(cout);
   p->ws = so; so += align_up(p->ws_bytes);
   p->slot_bytes = so;
   p->total = off + (size_t)p->slots * so;
@@ -681,26 +704,31 @@ had_status host_plan(const had_shape* s, had_mode mode, const had_relpos_bias* b
 // stream is made to wait for it; the streams and events are then released
 // (CUDA defers that until their pending work is done).
 struct HostStreams {
-  cudaStream_t main = nullptr, in = nullptr, out = nullptr;
-  cudaEvent_t start = nullptr, join_in = nullptr, join_out = nullptr;
+  cudaStream_t main = nullptr, in = nullptr, out = nullptr, comp = nullptr;
+  cudaEvent_t start = nullptr, join_in = nullptr, join_out = nullptr, join_comp = nullptr;
   cudaEvent_t in_done[kHostSlots] = {}, comp_done[kHostSlots] = {}, out_done[kHostSlots] = {};
   ~HostStreams() {
     if (in && join_in && cudaEventRecord(join_in, in) == cudaSuccess) cudaStreamWaitEvent(main, join_in, 0);
     if (out && join_out && cudaEventRecord(join_out, out) == cudaSuccess) cudaStreamWaitEvent(main, join_out, 0);
-    for (cudaEvent_t e : {start, join_in, join_out})
+    if (comp && join_comp && cudaEventRecord(join_comp, comp) == cudaSuccess)
+      cudaStreamWaitEvent(main, join_comp, 0);
+    for (cudaEvent_t e : {start, join_in, join_out, join_comp})
       if (e) cudaEventDestroy(e);
     for (int i = 0; i < kHostSlots; ++i)
       for (cudaEvent_t e : {in_done[i], comp_done[i], out_done[i]})
         if (e) cudaEventDestroy(e);
     if (in) cudaStreamDestroy(in);
     if (out) cudaStreamDestroy(out);
+    if (comp) cudaStreamDestroy(comp);
   }
 };
 
 // Chunk k: its Q, K, V are copied in on `in` (once the slot's previous chunk has
-// been computed), computed on the caller's stream (once its inputs are in and the
-// slot's previous O has been copied out), and its O copied out on `out`.  Copy
-// in, compute and copy out of consecutive chunks overlap.
+// been computed), computed on compute stream k % 2 (the caller's stream or the
+// side compute stream; once its inputs are in and the slot's previous O has been
+// copied out), and its O copied out on `out`.  Copy in, compute and copy out of
+// consecutive chunks overlap, and so do the kernels of two consecutive chunks (the
+// next chunk's CTAs fill the SMs that the last wave of the previous one leaves).
 had_status host_attention(const void* Q, const void* K, const void* V, const had_shape* s,
                           const had_relpos_bias* bias, const float* alpha_q, const float* alpha_k, int N,
                           had_mode mode, void* O, had_dtype o_dtype, int chunk_b, void* workspace, size_t ws_bytes,
@@ -719,15 +747,18 @@ had_status host_attention(const void* Q, const void* K, const void* V, const had
     if (s->seqlens[b] < 1 || s->seqlens[b] > s->n) return HAD_ERR_INVALID;
   const bool has_bias = bias && bias->table;
   char* ws = static_cast<char*>(workspace);
-  const size_t o_b = (size_t)s->H * s->n * s->d * (o_dtype == HAD_BF16 ? 2 : 4);
   auto cu = [](cudaError_t e, const char* what) { return e == cudaSuccess ? HAD_OK : cuda_fail(e, what); };
 
   HostStreams hs;
   hs.main = st;
+  const bool two = p.chunks > 1;  // a second compute stream only when there are chunks to overlap
   if ((r = cu(cudaStreamCreateWithFlags(&hs.in, cudaStreamNonBlocking), "cudaStreamCreateWithFlags")) != HAD_OK ||
       (r = cu(cudaStreamCreateWithFlags(&hs.out, cudaStreamNonBlocking), "cudaStreamCreateWithFlags")) != HAD_OK)
     return r;
-  for (cudaEvent_t* e : {&hs.start, &hs.join_in, &hs.join_out})
+  if (two && (r = cu(cudaStreamCreateWithFlags(&hs.comp, cudaStreamNonBlocking), "cudaStreamCreateWithFlags")) !=
+                 HAD_OK)
+    return r;
+  for (cudaEvent_t* e : {&hs.start, &hs.join_in, &hs.join_out, &hs.join_comp})
     if ((r = cu(cudaEventCreateWithFlags(e, cudaEventDisableTiming), "cudaEventCreateWithFlags")) != HAD_OK) return r;
   for (int i = 0; i < p.slots; ++i)
     for (cudaEvent_t* e : {&hs.in_done[i], &hs.comp_done[i], &hs.out_done[i]})
@@ -738,6 +769,8 @@ had_status host_attention(const void* Q, const void* K, const void* V, const had
       (r = cu(cudaStreamWaitEvent(hs.in, hs.start, 0), "cudaStreamWaitEvent")) != HAD_OK ||
       (r = cu(cudaStreamWaitEvent(hs.out, hs.start, 0), "cudaStreamWaitEvent")) != HAD_OK)
     return r;
+  if (two && (r = cu(cudaStreamWaitEvent(hs.comp, hs.start, 0), "cudaStreamWaitEvent")) != HAD_OK) return r;
+  const cudaStream_t comp[kHostCompute] = {st, two ? hs.comp : st};
   const int32_t* dseq = nullptr;
   if (s->seqlens) {
     int32_t* d = reinterpret_cast<int32_t*>(ws + p.seq);
@@ -759,30 +792,41 @@ had_status host_attention(const void* Q, const void* K, const void* V, const had
   const char* hk = static_cast<const char*>(K);
   const char* hv = static_cast<const char*>(V);
   char* ho = static_cast<char*>(O);
+  const size_t head_ob = (size_t)s->n * s->d * (o_dtype == HAD_BF16 ? 2 : 4);
+  const size_t tab_head = !has_bias ? 0
+                          : bias->dense ? (size_t)s->n * s->n
+                                        : (size_t)(2 * bias->gh - 1) * (2 * bias->gw - 1);
   for (int k = 0; k < p.chunks; ++k) {
-    const int b0 = k * p.cb, nb = std::min(p.cb, s->B - b0), sl = k % p.slots;
+    const int g = k % p.hgroups, b0 = (k / p.hgroups) * p.cb, nb = std::min(p.cb, s->B - b0);
+    const int h0 = g * p.hc, nh = std::min(p.hc, s->H - h0), sl = k % p.slots;
+    const cudaStream_t cs = comp[k % kHostCompute];
     char* slot = ws + p.slot0 + (size_t)sl * p.slot_bytes;
-    const size_t in_bytes = (size_t)nb * p.in_b, in_off = (size_t)b0 * p.in_b;
+    // a chunk is whole sequences (h0 = 0, nh = H) or one sequence's heads h0 .. h0 + nh - 1: contiguous either way
+    const size_t in_off = (size_t)b0 * p.in_b + (size_t)h0 * p.head_b, in_bytes = (size_t)nb * nh * p.head_b;
+    const size_t o_off = ((size_t)b0 * s->H + h0) * head_ob, o_bytes = (size_t)nb * nh * head_ob;
     if (k >= p.slots && (r = cu(cudaStreamWaitEvent(hs.in, hs.comp_done[sl], 0), "cudaStreamWaitEvent")) != HAD_OK)
       return r;
     if ((r = cu(cudaMemcpyAsync(slot + p.q, hq + in_off, in_bytes, cudaMemcpyHostToDevice, hs.in), "cudaMemcpyAsync(Q)")) != HAD_OK ||
         (r = cu(cudaMemcpyAsync(slot + p.k, hk + in_off, in_bytes, cudaMemcpyHostToDevice, hs.in), "cudaMemcpyAsync(K)")) != HAD_OK ||
         (r = cu(cudaMemcpyAsync(slot + p.v, hv + in_off, in_bytes, cudaMemcpyHostToDevice, hs.in), "cudaMemcpyAsync(V)")) != HAD_OK ||
         (r = cu(cudaEventRecord(hs.in_done[sl], hs.in), "cudaEventRecord")) != HAD_OK ||
-        (r = cu(cudaStreamWaitEvent(st, hs.in_done[sl], 0), "cudaStreamWaitEvent")) != HAD_OK)
+        (r = cu(cudaStreamWaitEvent(cs, hs.in_done[sl], 0), "cudaStreamWaitEvent")) != HAD_OK)
       return r;
-    if (k >= p.slots && (r = cu(cudaStreamWaitEvent(st, hs.out_done[sl], 0), "cudaStreamWaitEvent")) != HAD_OK)
+    if (k >= p.slots && (r = cu(cudaStreamWaitEvent(cs, hs.out_done[sl], 0), "cudaStreamWaitEvent")) != HAD_OK)
       return r;
-    had_shape cs = *s;
-    cs.B = nb;
-    cs.seqlens = dseq ? dseq + b0 : nullptr;
-    r = run_attention<EXP_NONE>(slot + p.q, slot + p.k, slot + p.v, &cs, has_bias ? &bdev : nullptr, alpha_q, alpha_k,
-                                N, mode, slot + p.o, o_dtype, nullptr, nullptr, 0, 0, slot + p.ws, p.ws_bytes, st);
+    had_shape csh = *s;
+    csh.B = nb;
+    csh.H = nh;
+    csh.seqlens = dseq ? dseq + b0 : nullptr;
+    had_relpos_bias cb = bdev;
+    if (has_bias) cb.table = bdev.table + (size_t)h0 * tab_head;
+    r = run_attention<EXP_NONE>(slot + p.q, slot + p.k, slot + p.v, &csh, has_bias ? &cb : nullptr,
+                                alpha_q ? alpha_q + h0 : nullptr, alpha_k ? alpha_k + h0 : nullptr, N, mode,
+                                slot + p.o, o_dtype, nullptr, nullptr, 0, 0, slot + p.ws, p.ws_bytes, cs);
     if (r != HAD_OK) return r;
-    if ((r = cu(cudaEventRecord(hs.comp_done[sl], st), "cudaEventRecord")) != HAD_OK ||
+    if ((r = cu(cudaEventRecord(hs.comp_done[sl], cs), "cudaEventRecord")) != HAD_OK ||
         (r = cu(cudaStreamWaitEvent(hs.out, hs.comp_done[sl], 0), "cudaStreamWaitEvent")) != HAD_OK ||
-        (r = cu(cudaMemcpyAsync(ho + (size_t)b0 * o_b, slot + p.o, (size_t)nb * o_b, cudaMemcpyDeviceToHost, hs.out),
-                "cudaMemcpyAsync(O)")) != HAD_OK ||
+        (r = cu(cudaMemcpyAsync(ho + o_off, slot + p.o, o_bytes, cudaMemcpyDeviceToHost, hs.out), "cudaMemcpyAsync(O)")) != HAD_OK ||
         (r = cu(cudaEventRecord(hs.out_done[sl], hs.out), "cudaEventRecord")) != HAD_OK)
       return r;
   }

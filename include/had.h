@@ -179,10 +179,12 @@ had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, 
  * o_dtype; s->seqlens: HOST int32 [B] (each in [1, n], checked on the host) or
  * NULL; bias->table: HOST fp32 (as the bias struct describes) or bias NULL; alpha_q,
  * alpha_k as in had_attention.  The batch is cut into chunks of chunk_b
- * sequences (0: the library picks about 8 MiB of inputs per chunk).  Chunk k's
- * Q, K, V are copied in on one side stream while chunk k-1 is computed on
- * `stream` and chunk k-2's O is copied out on another.  The chunks cycle
- * through three device slots in `workspace`, which needs at least
+ * sequences (0: the library picks about 8 MiB of inputs per chunk, and when one
+ * sequence holds more, cuts each sequence into equal groups of heads of at most
+ * 16 MiB).  Chunk k's Q, K, V are copied in on one side stream while chunks k-1
+ * and k-2 are computed, alternately on `stream` and on a side compute stream,
+ * and chunk k-3's O is copied out on another side stream.  The chunks cycle
+ * through four device slots in `workspace`, which needs at least
  * had_attention_host_workspace_size(s, N, mode, bias, chunk_b) bytes.  Every
  * (b, h) is computed by the same kernels as in had_attention, so O is
  * bit-identical to it for any chunk_b.
@@ -190,8 +192,8 @@ had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, 
  * (cudaHostAlloc / cudaHostRegister); pageable memory works, serialized.  The
  * call enqueues all of it behind the work already on `stream` and returns: O
  * is complete once `stream` has reached that point.  The host arrays must stay
- * valid and unchanged until then.  Each call creates two streams and some
- * events and releases them (CUDA frees them once their work is done);
+ * valid and unchanged until then.  Each call creates up to three streams and
+ * some events and releases them (CUDA frees them once their work is done);
  * it allocates no memory. */
 size_t had_attention_host_workspace_size(const had_shape* s, int N, had_mode mode, const had_relpos_bias* bias,
                                          int chunk_b);
