@@ -170,17 +170,32 @@ def test_host_entry_point_validates_on_the_host(L):
 
 def test_host_workspace_grows_with_the_chunk(L):
     import binarized_qk_sparse_b200 as m
-    shp = _shape(m, B=8, H=3, n=197)
+    # B=16: four slots of 1 and of 2 sequences, two slots of 8
+    shp = _shape(m, B=16, H=3, n=197)
     bias = m.had_relpos_bias(0x30000, 14, 14, 1)
     sizes = [L.had_attention_host_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(bias), c) for c in (1, 2, 8)]
     assert 0 < sizes[0] < sizes[1] < sizes[2]
     # a chunk larger than the batch is the whole batch; 0 lets the library choose
-    assert L.had_attention_host_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(bias), 100) == sizes[2]
+    whole = L.had_attention_host_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(bias), 16)
+    assert L.had_attention_host_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(bias), 100) == whole
     assert L.had_attention_host_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(bias), 0) > 0
     assert L.had_attention_host_workspace_size(ctypes.byref(shp), 0, 1, ctypes.byref(bias), -1) == 0
-    # three slots of one chunk each hold Q, K, V and O at least
+    # four slots of one chunk each hold Q, K, V and O at least
     one = 3 * 197 * 64 * 2 + 197 * 64 * 4
-    assert sizes[0] >= 3 * one
+    assert sizes[0] >= 4 * one
+
+
+def test_host_workspace_of_head_groups(L):
+    # B2 H8 n16384 bf16: 100 MB of inputs per sequence, more than one chunk holds, so chunk_b = 0 cuts each
+    # sequence into groups of 2 heads (at most 16 MiB): four slots of 2 heads against two slots of 8
+    import binarized_qk_sparse_b200 as m
+    shp = _shape(m, B=2, H=8, n=16384)
+    bias = m.had_relpos_bias(0x30000, 128, 128, 0)
+    split = L.had_attention_host_workspace_size(ctypes.byref(shp), 0, 0, ctypes.byref(bias), 0)
+    whole = L.had_attention_host_workspace_size(ctypes.byref(shp), 0, 0, ctypes.byref(bias), 1)
+    head_in = 16384 * 64 * 2
+    assert 0 < split < whole
+    assert split >= 4 * 2 * (3 * head_in + 2 * head_in)  # Q, K, V and fp32 O of two heads in each of four slots
 
 
 def test_dense_bias_matrix_validation(L):
