@@ -332,13 +332,6 @@ __global__ void __launch_bounds__(kThreads, 2) k_qkv_tc(const __grid_constant__ 
     prefetch_tensormap(&a.tm_x);
     prefetch_tensormap(&a.tm_w);
   }
-  for (int e = tid; e < kN; e += kThreads) {
-    const int j = j0 + e / kHd, t = j / a.H, h = j - t * a.H;
-    double m = 0.0;
-    if (j < nblk && t < 2)
-      for (int z = 0; z < kMuSplit; ++z) m += a.mupart[((((size_t)z * 2 + t) * a.B + b) * a.H + h) * kHd + (e % kHd)];
-    smu[e] = (float)m;
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -383,7 +376,17 @@ __global__ void __launch_bounds__(kThreads, 2) k_qkv_tc(const __grid_constant__ 
     mma_commit(acc_bar);
   } else if (warp < 4) {
     // epilogue: thread (warp w, lane l) owns token m0 + 32 w + l, TMEM lane 32 w + l, and
-    // takes the CTA's column blocks one after the other
+    // takes the CTA's column blocks one after the other.  First the means of the CTA's Q and K
+    // columns (the partials added in slice order, one rounding), while the main loop runs
+    for (int e = tid; e < kN; e += 128) {
+      const int j = j0 + e / kHd, t = j / a.H, h = j - t * a.H;
+      double m = 0.0;
+      if (j < nblk && t < 2)
+        for (int z = 0; z < kMuSplit; ++z)
+          m += a.mupart[((((size_t)z * 2 + t) * a.B + b) * a.H + h) * kHd + (e % kHd)];
+      smu[e] = (float)m;
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");  // the four epilogue warps
     const bool ok = __all_sync(0xffffffffu, bounded_wait(acc_bar, 0));
     tc_fence_after();
     const uint32_t tl = tmem + ((uint32_t)(32 * warp) << 16);
