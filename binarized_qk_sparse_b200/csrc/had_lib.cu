@@ -949,8 +949,6 @@ had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, 
       cudaError_t e = cudaFuncSetAttribute(qkv::k_qkv_tc, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            qkv::QkvSmem::kTotal);
       if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_qkv_tc)");
-      e = cudaFuncSetAttribute(qkv::k_mu, cudaFuncAttributeMaxDynamicSharedMemorySize, qkv::MuSmem::kTotal);
-      if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(k_mu)");
       configured[dev] = true;
     }
   }
@@ -962,9 +960,8 @@ had_status had_qkv_prepare(const void* X, const void* Wqkv, const had_shape* s, 
                   qkv::kXsumThreads * qkv::kXsumGroups, 0, st>>>(Xb, d.n, Dm, d.H, s->seqlens, q.nch, xpart,
                                                                   vbits != 0 ? vamax : nullptr);
   if ((r = check_launch("k_xsum")) != HAD_OK) return r;
-  qkv::k_mu<<<dim3((2 * d.H * 64 + qkv::kMuThreads * qkv::kMuC - 1) / (qkv::kMuThreads * qkv::kMuC),
-                   (d.B + qkv::kMuB - 1) / qkv::kMuB, qkv::kMuSplit),
-              qkv::kMuThreads, qkv::MuSmem::kTotal, st>>>(Wb, xpart, q.nch, d.n, s->seqlens, d.B, d.H, Dm, mupart);
+  qkv::k_mu<<<dim3((2 * d.H * 64 + qkv::kMuO - 1) / qkv::kMuO, (d.B + qkv::kMuB - 1) / qkv::kMuB, qkv::kMuSplit),
+              qkv::kMuThreads, 0, st>>>(Wb, xpart, q.nch, d.n, s->seqlens, d.B, d.H, Dm, mupart);
   if ((r = check_launch("k_mu")) != HAD_OK) return r;
   // the projection, binarized in its epilogue, into the attention workspace
   qkv::QkvArgs qa;

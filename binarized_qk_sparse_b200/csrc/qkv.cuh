@@ -36,7 +36,7 @@ using namespace had::sm100;
 
 constexpr int kXsumChunk = 32;     // tokens per partial sum of X
 constexpr int kXsumThreads = 128;  // k_xsum: feature threads (8 features each) per token group
-constexpr int kMuB = 8, kMuK = 64;  // k_mu: batches per CTA, features per staged chunk
+constexpr int kMuB = 16, kMuK = 64;  // k_mu: batches per CTA, features per staged chunk
 
 // Token sums of X over the valid tokens of each 32-token chunk: part[b][ch][k], fp64.
 // Thread (g, f) of a CTA adds 8 adjacent features over the g-th 8 tokens of the
@@ -93,56 +93,53 @@ __global__ void __launch_bounds__(kXsumThreads * kXsumGroups) k_xsum(const __nv_
 
 // Partial dot products of the means with W: mupart[z][t][b][h][c] = sum over the
 // z-th of kMuSplit feature slices of xbar[b][k] W[o][k], o = t*H*64 + h*64 + c, in
-// fp64.  k_qkv_tc adds the kMuSplit partials in slice order and rounds once to
-// fp32.  A CTA takes 512 output channels and 8 batches, 64 features at a time: all
-// its threads copy the 512 W rows of the chunk into shared memory at once
-// (cp.async, 16 bytes each, rows padded to 144 bytes so that 16-byte reads of
-// eight rows hit distinct banks), and the 8 batches' means beside them.  Thread x
-// then owns channels x + 128 c (c < 4): it converts a 16-byte piece of each of
-// its rows to fp64 and applies it to the 8 batches' means (every lane of a warp
-// reads the same means: broadcasts).
-constexpr int kMuThreads = 128;
-constexpr int kMuC = 4;                     // channels per thread
-constexpr int kMuSplit = 8;                 // feature slices
-constexpr int kMuRow = kMuK * 2 + 16;       // bytes per staged W row
-struct MuSmem {
-  static constexpr int kW = 0;                                // [512 rows][kMuRow] bf16
-  static constexpr int kX = kW + kMuThreads * kMuC * kMuRow;  // [kMuB][kMuK] fp64
-  static constexpr int kTotal = kX + kMuB * kMuK * 8;
-};
+// fp64 on the tensor cores (mma.sync m8n8k4 f64: an 8 x 4 block of means times a
+// 4 x 8 block of W per instruction).  k_qkv_tc adds the kMuSplit partials in slice
+// order and rounds once to fp32.  A CTA of 8 warps takes 16 batches and 128
+// channels of one slice, 64 features at a time: it stages the 16 batches' means
+// (the chunk sums of k_xsum added in chunk order, divided by L) in shared memory,
+// and warp w takes channels 16w .. 16w + 15 as two 8 x 8 output blocks per batch
+// group.  Inside a 32-feature step, the lane with k-slot q (lane % 4) supplies
+// features 8q .. 8q + 7 to the step's eight MMAs, one per MMA, for the means and
+// for W alike, so that its W piece is one 16-byte load.
+constexpr int kMuThreads = 256;
+constexpr int kMuO = 128;    // channels per CTA
+constexpr int kMuSplit = 8;  // feature slices
 
-__device__ __forceinline__ void cp_async16_zfill(void* smem_dst, const void* gmem_src, bool valid) {
-  const uint32_t d = smem_u32(smem_dst);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;\n" ::"r"(d), "l"(gmem_src), "r"(valid ? 16 : 0)
-               : "memory");
+__device__ __forceinline__ void dmma_8x8x4(double (&c)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(c[0]), "+d"(c[1])
+               : "d"(a), "d"(b));
 }
 
 __global__ void __launch_bounds__(kMuThreads) k_mu(const __nv_bfloat16* __restrict__ W,
                                                    const double* __restrict__ part, int nch, int n,
                                                    const int32_t* seqlens, int B, int H, int Dm,
                                                    double* __restrict__ mupart) {
-  extern __shared__ __align__(16) uint8_t musm[];
-  uint8_t* wsm = musm + MuSmem::kW;
-  double* xs = reinterpret_cast<double*>(musm + MuSmem::kX);
-  const int ob = blockIdx.x * kMuThreads * kMuC, b0 = blockIdx.y * kMuB;
+  __shared__ __align__(16) double xs[kMuB][kMuK + 2];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+  const int o0 = blockIdx.x * kMuO + 16 * warp, b0 = blockIdx.y * kMuB;
   const int no = 2 * H * 64;
   const int slice = Dm / kMuSplit;  // a multiple of 8 (Dm is a multiple of 64)
   const int kbeg = blockIdx.z * slice, kend = kbeg + slice;
-  double acc[kMuB][kMuC];
+  double acc[2][2][2];  // [batch group][channel group][the lane's two outputs]
 #pragma unroll
-  for (int bb = 0; bb < kMuB; ++bb)
+  for (int mg = 0; mg < 2; ++mg)
 #pragma unroll
-    for (int c = 0; c < kMuC; ++c) acc[bb][c] = 0.0;
+    for (int ng = 0; ng < 2; ++ng) acc[mg][ng][0] = acc[mg][ng][1] = 0.0;
   for (int k0 = kbeg; k0 < kend; k0 += kMuK) {
     const int kn = min(kMuK, kend - k0);  // a multiple of 8
-    __syncthreads();  // the previous chunk's reads are done
-    for (int e = threadIdx.x; e < kMuThreads * kMuC * (kMuK / 8); e += kMuThreads) {
-      const int row = e / (kMuK / 8), q = e % (kMuK / 8), o = ob + row;
-      const bool v = o < no && 8 * q < kn;
-      cp_async16_zfill(wsm + row * kMuRow + 16 * q, v ? static_cast<const void*>(W + (size_t)o * Dm + k0 + 8 * q) : W,
-                       v);
-    }
-    asm volatile("cp.async.commit_group;\n" ::: "memory");
+    // this chunk's W pieces: two 32-feature steps x two channel groups, issued before the staging
+    uint4 wv[kMuK / 32][2];
+#pragma unroll
+    for (int st = 0; st < kMuK / 32; ++st)
+#pragma unroll
+      for (int ng = 0; ng < 2; ++ng) {
+        const int o = o0 + 8 * ng + g, kk = 32 * st + 8 * q;
+        wv[st][ng] = (o < no && kk < kn) ? __ldg(reinterpret_cast<const uint4*>(W + (size_t)o * Dm + k0 + kk))
+                                         : make_uint4(0u, 0u, 0u, 0u);
+      }
+    __syncthreads();  // the previous chunk's reads of xs are done
     // the means: the chunk sums of k_xsum added in chunk order, divided by L
     for (int e = threadIdx.x; e < kMuB * kMuK / 2; e += kMuThreads) {
       const int br = e / (kMuK / 2), cc = (e % (kMuK / 2)) * 2, b = b0 + br;
@@ -157,46 +154,51 @@ __global__ void __launch_bounds__(kMuThreads) k_mu(const __nv_bfloat16* __restri
         }
         if (L > 0) m = make_double2(m.x / (double)L, m.y / (double)L);
       }
-      *reinterpret_cast<double2*>(xs + br * kMuK + cc) = m;
+      *reinterpret_cast<double2*>(&xs[br][cc]) = m;
     }
-    asm volatile("cp.async.wait_group 0;\n" ::: "memory");
     __syncthreads();
-    for (int q = 0; q < kn / 8; ++q) {
-      double w[kMuC][8];
 #pragma unroll
-      for (int c = 0; c < kMuC; ++c) {
-        const uint4 wr = *reinterpret_cast<const uint4*>(wsm + (threadIdx.x + kMuThreads * c) * kMuRow + 16 * q);
-        const uint32_t u[4] = {wr.x, wr.y, wr.z, wr.w};
+    for (int st = 0; st < kMuK / 32; ++st) {
+      if (32 * st >= kn) break;  // uniform over the CTA
+      double wb[2][8];
+#pragma unroll
+      for (int ng = 0; ng < 2; ++ng) {
+        const uint32_t u[4] = {wv[st][ng].x, wv[st][ng].y, wv[st][ng].z, wv[st][ng].w};
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-          w[c][2 * v] = (double)__uint_as_float(u[v] << 16);
-          w[c][2 * v + 1] = (double)__uint_as_float(u[v] & 0xFFFF0000u);
+          wb[ng][2 * v] = (double)__uint_as_float(u[v] << 16);
+          wb[ng][2 * v + 1] = (double)__uint_as_float(u[v] & 0xFFFF0000u);
         }
       }
 #pragma unroll
-      for (int bb = 0; bb < kMuB; ++bb) {
-        const double2* xp = reinterpret_cast<const double2*>(xs + bb * kMuK + 8 * q);
+      for (int mg = 0; mg < 2; ++mg) {
+        double xa[8];
+        const double2* xp = reinterpret_cast<const double2*>(&xs[8 * mg + g][32 * st + 8 * q]);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           const double2 x2 = xp[v];
-#pragma unroll
-          for (int c = 0; c < kMuC; ++c) {
-            acc[bb][c] = fma(x2.x, w[c][2 * v], acc[bb][c]);
-            acc[bb][c] = fma(x2.y, w[c][2 * v + 1], acc[bb][c]);
-          }
+          xa[2 * v] = x2.x;
+          xa[2 * v + 1] = x2.y;
         }
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj)
+#pragma unroll
+          for (int ng = 0; ng < 2; ++ng) dmma_8x8x4(acc[mg][ng], xa[jj], wb[ng][jj]);
       }
     }
   }
+  // lane (g, q) holds outputs (batch 8 mg + g, channels 8 ng + 2q, 8 ng + 2q + 1)
 #pragma unroll
-  for (int c = 0; c < kMuC; ++c) {
-    const int o = ob + threadIdx.x + kMuThreads * c;
-    if (o >= no) continue;
-    const int t = o / (H * 64), r = o - t * H * 64;  // r = h * 64 + c
+  for (int mg = 0; mg < 2; ++mg)
 #pragma unroll
-    for (int bb = 0; bb < kMuB; ++bb)
-      if (b0 + bb < B) mupart[(((size_t)blockIdx.z * 2 + t) * B + b0 + bb) * H * 64 + r] = acc[bb][c];
-  }
+    for (int ng = 0; ng < 2; ++ng)
+#pragma unroll
+      for (int v = 0; v < 2; ++v) {
+        const int b = b0 + 8 * mg + g, o = o0 + 8 * ng + 2 * q + v;
+        if (b >= B || o >= no) continue;
+        const int t = o / (H * 64), r = o - t * H * 64;  // r = h * 64 + c
+        mupart[(((size_t)blockIdx.z * 2 + t) * B + b) * H * 64 + r] = acc[mg][ng][v];
+      }
 }
 
 // V's codes from the projection's bf16 V and the epilogue's column absmax, as the
