@@ -129,7 +129,7 @@ def score_tensor_ops(valid_scores: int, d: int = 64) -> float:
     return 2.0 * d * valid_scores
 
 
-def north_star_roofline(kbytes: float, tensor_ops: float, kernel_ms: float, hbm_gbs: float, i8_tops: float) -> dict:
+def method_roofline(kbytes: float, tensor_ops: float, kernel_ms: float, hbm_gbs: float, i8_tops: float) -> dict:
     """The fused kernel's roofline as the method defines it: the slower of its
     algorithmic HBM bytes at the measured bandwidth and its score contraction at
     the int8 tensor-pipe peak.  frac = that time / the measured kernel time."""
@@ -602,7 +602,7 @@ def run_gpu(args, rank, world, local_rank):
         tc_peak = max(INT8_PER_BF16 * peaks["bf16_tflops"], probe_i8)
         peak_txt = (f"int8 = max({INT8_PER_BF16:g} x {peak_kind} bf16 burst {peaks['bf16_tflops']} TFLOP/s, "
                     f"probe {probe_i8:.0f} TOPS)")
-    roof = north_star_roofline(kbytes, tc_ops, attn_avg_ms, peaks["hbm_gbs"], tc_peak)
+    roof = method_roofline(kbytes, tc_ops, attn_avg_ms, peaks["hbm_gbs"], tc_peak)
     if ref:
         roof["unit"] = roof["unit"].replace("int8", "bf16")
     traffic = None
@@ -774,7 +774,7 @@ def run_qkv(args, rank, world, local_rank):
     flop = 2.0 * B * n * Dm * 3 * H * d
     i8 = max(probe_i8, INT8_PER_BF16 * peaks["bf16_tflops"])
     kb = kernel_bytes_per_token(mode, 2, 2, d) * queries + bw.table.nbytes
-    roof = north_star_roofline(kb, score_tensor_ops(B * H * n * n, d), att_ms, peaks["hbm_gbs"], i8)
+    roof = method_roofline(kb, score_tensor_ops(B * H * n * n, d), att_ms, peaks["hbm_gbs"], i8)
     roof.update({"traffic": None, "kernel": "k_attn_tc (fused score/top-N/softmax/A.V)", "avg_launch_ms": att_ms})
     line = {
         "metric": METRIC, "value": whole_job_rate(queries, world, args.steps, sum(f_step)), "unit": UNIT,
