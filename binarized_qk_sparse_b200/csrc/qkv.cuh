@@ -205,10 +205,10 @@ __global__ void __launch_bounds__(kMuThreads) k_mu(const __nv_bfloat16* __restri
 // prepare stage makes them (scale absmax/qmax, 1 if the absmax is 0; codes
 // rint(V/scale) clamped to +-qmax, 0 past L), transposed to V^T: int8
 // [B*H][64][n_pad], or packed 4-bit [B*H][64][n_pad/2] with key 2k in the low
-// nibble of byte k.  A CTA takes 64 tokens of one head: thread (g, t) reads token
-// t's channels 8g..8g+7 and 32+8g..32+8g+7 (16-byte loads), writes their codes
-// into a [64 channels][64 tokens] byte tile, and the tile's rows leave as 16-byte
-// (int8) or 8-byte (4-bit) stores.
+// nibble of byte k.  A CTA takes 64 tokens of one head: each thread reads four
+// channels of four tokens, writes their codes into a [64 channels][64 tokens] byte
+// tile four tokens at a time, and the tile's rows leave as 16-byte (int8) or
+// 8-byte (4-bit) stores.
 constexpr int kVcThreads = 256;
 __global__ void __launch_bounds__(kVcThreads) k_vcodes(const __nv_bfloat16* __restrict__ V,
                                                        const uint32_t* __restrict__ vamax, int H, int n,
@@ -228,24 +228,32 @@ __global__ void __launch_bounds__(kVcThreads) k_vcodes(const __nv_bfloat16* __re
   }
   __syncthreads();
   {
-    const int t = tid & 63, g = tid >> 6, i = i0 + t;
+    // thread (channel quad cq, token quad tq): tokens 4tq .. 4tq + 3, channels 4cq .. 4cq + 3 (8-byte
+    // loads), then one 4-byte store of four tokens' codes per channel
+    const int cq = tid & 15, tq = tid >> 4;
+    uint2 x[4];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int c0 = 32 * half + 8 * g;
-      uint4 x = make_uint4(0u, 0u, 0u, 0u);
-      if (i < L) x = __ldg(reinterpret_cast<const uint4*>(V + ((size_t)bh * n + i) * 64 + c0));
-      const uint32_t u[4] = {x.x, x.y, x.z, x.w};
+    for (int u = 0; u < 4; ++u) {
+      const int i = i0 + 4 * tq + u;
+      x[u] = i < L ? __ldg(reinterpret_cast<const uint2*>(V + ((size_t)bh * n + i) * 64 + 4 * cq)) : make_uint2(0u, 0u);
+    }
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        const int c = c0 + 2 * v;
-        tile[c][t] = (uint8_t)quant_v(__uint_as_float(u[v] << 16), sc[c], rsc[c], qmax);
-        tile[c + 1][t] = (uint8_t)quant_v(__uint_as_float(u[v] & 0xFFFF0000u), sc[c + 1], rsc[c + 1], qmax);
+    for (int v = 0; v < 4; ++v) {
+      const int c = 4 * cq + v;
+      uint32_t w = 0u;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t pr = (v < 2) ? x[u].x : x[u].y;
+        const float xv = __uint_as_float((v & 1) ? (pr & 0xFFFF0000u) : (pr << 16));
+        w |= ((uint32_t)quant_v(xv, sc[c], rsc[c], qmax) & 0xFFu) << (8 * u);
       }
+      // 16-byte chunk k of row c sits at chunk k ^ (c / 4 % 4): the 32 lanes' stores hit 16 banks
+      *reinterpret_cast<uint32_t*>(&tile[c][16 * ((tq >> 2) ^ (cq & 3)) + 4 * (tq & 3)]) = w;
     }
   }
   __syncthreads();
   const int c = tid >> 2, seg = tid & 3;  // channel row c, 16 of its 64 tokens
-  const uint4 w = *reinterpret_cast<const uint4*>(&tile[c][16 * seg]);
+  const uint4 w = *reinterpret_cast<const uint4*>(&tile[c][16 * (seg ^ ((c >> 2) & 3))]);
   if (vbits == 4) {
     const uint32_t in[4] = {w.x, w.y, w.z, w.w};
     uint32_t out[2];
